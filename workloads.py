@@ -1,0 +1,206 @@
+"""Seeded synthetic inputs for the Tensor Cache layer.
+
+This module only draws random numbers in the shapes and distributions of the
+workloads described for "Tensor Cache: Eviction-conditioned Associative Memory
+for Transformers" (arXiv 2605.22884): the associative-recall task (planted
+key/value pairs re-issued as noisy queries), LM-shaped prefill, a long-context
+run at 32x a 1024-token training length, and batched streaming decode.  It
+holds none of the layer's arithmetic, so both the CUDA path and the CPU oracle
+can take their inputs from it.  The pages use OpenWebText, Shakespeare and
+trained weights; none of that is here, and these seeded tensors stand in for
+them with the same shapes.
+
+Prefill inputs (q, k, v, lam, eta, g) are drawn on the CPU with
+``torch.Generator`` so every machine gets identical values.  The batched
+decode workload is 9 GB and is drawn on the GPU with a seeded CUDA generator;
+callers copy sampled heads to the host for checking.
+"""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass, field
+
+import torch
+
+# Name -> shape and parameter recipe.  seed = 1000 + position in this list.
+PREFILL_CONFIGS = {
+    # tiny case the oracle finishes in well under a second
+    "tiny_fp32": dict(B=1, H=1, T=256, dk=16, dv=16, W=32, C=16, dtype="f32", seed=1001),
+    # associative-recall shaped, fp32
+    "recall_fp32": dict(B=8, H=4, T=2048, dk=64, dv=64, W=256, C=64, dtype="f32", seed=1002),
+    # LM-shaped prefill, bf16 inputs, fp32 state
+    "lm_prefill_bf16": dict(B=8, H=12, T=4096, dk=64, dv=64, W=512, C=64, dtype="bf16", seed=1003),
+    # long-context prefill at 32 x 1024 tokens, bf16 inputs, fp32 state
+    "long_prefill_bf16": dict(B=1, H=16, T=32768, dk=64, dv=64, W=1024, C=128, dtype="bf16",
+                              seed=1004),
+}
+DECODE_CONFIG = dict(B=256, H=32, dk=128, dv=128, W=2048, steps=512, history=10240,
+                     prewarm_evictions=8192, dtype="bf16", seed=1005)
+
+_TDTYPE = {"f32": torch.float32, "bf16": torch.bfloat16}
+
+
+def torch_dtype(name: str) -> torch.dtype:
+    return _TDTYPE[name]
+
+
+@dataclass
+class PrefillInputs:
+    q: torch.Tensor
+    k: torch.Tensor
+    v: torch.Tensor
+    lam: torch.Tensor  # [H] float32
+    eta: torch.Tensor  # [H] float32
+    g: torch.Tensor  # [H] float32
+    W: int
+    C: int
+    meta: dict = field(default_factory=dict)
+
+
+def _gen(seed: int) -> torch.Generator:
+    gen = torch.Generator(device="cpu")
+    gen.manual_seed(seed)
+    return gen
+
+
+def _uniform(gen, n, lo, hi):
+    return lo + (hi - lo) * torch.rand(n, generator=gen, dtype=torch.float64)
+
+
+def prefill_config(name: str) -> PrefillInputs:
+    """Inputs of one named prefill workload (CPU tensors)."""
+    cfg = PREFILL_CONFIGS[name]
+    B, H, T, dk, dv = cfg["B"], cfg["H"], cfg["T"], cfg["dk"], cfg["dv"]
+    gen = _gen(cfg["seed"])
+    dt = _TDTYPE[cfg["dtype"]]
+    meta = {"name": name, **cfg}
+    if name == "tiny_fp32":
+        s = 1.0 / math.sqrt(dk)
+        q = torch.randn(B, H, T, dk, generator=gen, dtype=torch.float64) * s
+        k = torch.randn(B, H, T, dk, generator=gen, dtype=torch.float64) * s
+        v = torch.randn(B, H, T, dv, generator=gen, dtype=torch.float64) * s
+        lam = torch.full((H,), 0.95, dtype=torch.float64)
+        eta = torch.full((H,), 0.5, dtype=torch.float64)
+        g = torch.zeros(H, dtype=torch.float64)
+    elif name == "recall_fp32":
+        q, k, v, plant = _recall_qkv(gen, B, H, T, dk, dv)
+        meta["plant"] = plant
+        lam = _uniform(gen, H, 0.97, 0.999)
+        eta = _uniform(gen, H, 0.1, 1.0)
+        g = torch.randn(H, generator=gen, dtype=torch.float64)
+    elif name == "lm_prefill_bf16":
+        def rms_normed(d):
+            x = torch.randn(B, H, T, d, generator=gen, dtype=torch.float64)
+            return x / torch.sqrt(torch.mean(x * x, dim=-1, keepdim=True))
+        q, k, v = rms_normed(dk), rms_normed(dk), rms_normed(dv)
+        lam = torch.sigmoid(_uniform(gen, H, 3.0, 7.0))
+        eta = torch.nn.functional.softplus(torch.randn(H, generator=gen, dtype=torch.float64))
+        g = torch.randn(H, generator=gen, dtype=torch.float64)
+    elif name == "long_prefill_bf16":
+        q = torch.randn(B, H, T, dk, generator=gen, dtype=torch.float64) / 8
+        k = torch.randn(B, H, T, dk, generator=gen, dtype=torch.float64) / 8
+        v = torch.randn(B, H, T, dv, generator=gen, dtype=torch.float64) / 8
+        lam = _uniform(gen, H, 0.99, 0.9999)
+        eta = _uniform(gen, H, 0.05, 0.5)
+        g = torch.randn(H, generator=gen, dtype=torch.float64)
+    else:  # pragma: no cover
+        raise KeyError(name)
+    return PrefillInputs(q.to(dt).contiguous(), k.to(dt).contiguous(), v.to(dt).contiguous(),
+                         lam.float(), eta.float(), g.float(), cfg["W"], cfg["C"], meta)
+
+
+def _recall_qkv(gen, B, H, T, dk, dv, n_pairs=64, spacing=8, query_start=1800, noise=0.05):
+    """Associative-recall layout: pair p sits at position spacing*p with a
+    unit-norm Gaussian key and an N(0,1)/8 value; the queries at positions
+    query_start + j re-issue key (j mod n_pairs) plus N(0, noise^2) noise.
+    Everything else is N(0,1)/8 (norm close to 1 at d = 64)."""
+    q = torch.randn(B, H, T, dk, generator=gen, dtype=torch.float64) / 8
+    k = torch.randn(B, H, T, dk, generator=gen, dtype=torch.float64) / 8
+    v = torch.randn(B, H, T, dv, generator=gen, dtype=torch.float64) / 8
+    pk = torch.randn(B, H, n_pairs, dk, generator=gen, dtype=torch.float64)
+    pk = pk / torch.linalg.vector_norm(pk, dim=-1, keepdim=True)
+    pv = torch.randn(B, H, n_pairs, dv, generator=gen, dtype=torch.float64) / 8
+    pos = torch.arange(n_pairs) * spacing
+    k[:, :, pos] = pk
+    v[:, :, pos] = pv
+    qpos = torch.arange(query_start, T)
+    which = (qpos - query_start) % n_pairs
+    q[:, :, qpos] = pk[:, :, which] + noise * torch.randn(B, H, len(qpos), dk, generator=gen,
+                                                         dtype=torch.float64)
+    return q, k, v, {"positions": pos.tolist(), "query_start": query_start, "n_pairs": n_pairs}
+
+
+def random_prefill(B, H, T, dk, dv, W, C, *, dtype="f32", seed=0, scale=None,
+                   lam_range=(0.9, 0.999), eta_range=(0.1, 1.0)) -> PrefillInputs:
+    """Generic seeded prefill inputs for parity cases at arbitrary shapes."""
+    gen = _gen(seed)
+    s = scale if scale is not None else 1.0 / math.sqrt(dk)
+    q = torch.randn(B, H, T, dk, generator=gen, dtype=torch.float64) * s
+    k = torch.randn(B, H, T, dk, generator=gen, dtype=torch.float64) * s
+    v = torch.randn(B, H, T, dv, generator=gen, dtype=torch.float64) * s
+    lam = _uniform(gen, H, *lam_range)
+    eta = _uniform(gen, H, *eta_range)
+    g = torch.randn(H, generator=gen, dtype=torch.float64)
+    dt = _TDTYPE[dtype]
+    return PrefillInputs(q.to(dt).contiguous(), k.to(dt).contiguous(), v.to(dt).contiguous(),
+                         lam.float(), eta.float(), g.float(), W, C,
+                         {"name": "random", "seed": seed, "dtype": dtype})
+
+
+@dataclass
+class DecodeInputs:
+    ring_k: torch.Tensor  # [B,H,W,dk]
+    ring_v: torch.Tensor  # [B,H,W,dv]
+    A: torch.Tensor  # [B,H,dk,dv] float32
+    q: torch.Tensor  # [steps,B,H,dk]
+    k: torch.Tensor  # [steps,B,H,dk]
+    v: torch.Tensor  # [steps,B,H,dv]
+    lam: torch.Tensor
+    eta: torch.Tensor
+    g: torch.Tensor
+    t0: int
+    W: int
+
+
+def decode_workload(*, B=None, H=None, dk=None, dv=None, W=None, steps=None, history=None,
+                    prewarm_evictions=None, dtype=None, seed=None, device="cuda") -> DecodeInputs:
+    """Batched-decode workload: a full ring (tokens history-W..history-1 at
+    slot t mod W), a pre-warmed A and ``steps`` fresh (q, k, v) per head.
+
+    The pre-warmed A stands for the state left by ``prewarm_evictions``
+    earlier evictions of N(0,1)/sqrt(dk) keys and values; it is drawn as a
+    Gaussian matrix whose entry scale matches such a state,
+    eta * sqrt(sum_{j<n} lam^(2j)) / sqrt(dk*dv).  Defaults are the full
+    256 x 32 head, d = 128, W = 2048, 512-step workload."""
+    c = dict(DECODE_CONFIG)
+    for key, val in dict(B=B, H=H, dk=dk, dv=dv, W=W, steps=steps, history=history,
+                         prewarm_evictions=prewarm_evictions, dtype=dtype, seed=seed).items():
+        if val is not None:
+            c[key] = val
+    B, H, dk, dv, W, n = c["B"], c["H"], c["dk"], c["dv"], c["W"], c["steps"]
+    dt = _TDTYPE[c["dtype"]]
+    dev = torch.device(device)
+    cpu_gen = _gen(c["seed"])
+    lam = _uniform(cpu_gen, H, 0.99, 0.9999)
+    eta = _uniform(cpu_gen, H, 0.1, 1.0)
+    g = torch.randn(H, generator=cpu_gen, dtype=torch.float64)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(c["seed"])
+    sk, sv = 1.0 / math.sqrt(dk), 1.0 / math.sqrt(dv)
+
+    def draw(shape, s):
+        x = torch.randn(shape, generator=gen, device=dev, dtype=torch.float32)
+        return x.mul_(s).to(dt)
+
+    ring_k = draw((B, H, W, dk), sk)
+    ring_v = draw((B, H, W, dv), sv)
+    npre = c["prewarm_evictions"]
+    geo = (1.0 - lam.pow(2 * npre)) / (1.0 - lam.pow(2))
+    a_scale = (eta * geo.sqrt() * sk * sv).float().to(dev)
+    A = torch.randn((B, H, dk, dv), generator=gen, device=dev, dtype=torch.float32)
+    A.mul_(a_scale.view(1, H, 1, 1))
+    q = draw((n, B, H, dk), sk)
+    k = draw((n, B, H, dk), sk)
+    v = draw((n, B, H, dv), sv)
+    return DecodeInputs(ring_k, ring_v, A, q, k, v, lam.float().to(dev), eta.float().to(dev),
+                        g.float().to(dev), int(c["history"]), W)
