@@ -1,0 +1,501 @@
+"""Benchmark of the Tensor Cache layer (libtc) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl tc|reference]
+
+One step = one pass of the whole prefill hot path (L1 window softmax, L2
+eviction chunk scan and memory read, gated fusion) over the LM-shaped prefill
+workload: B=8, H=12, T=4096, d=64, W=512, C=64, bf16 inputs, float32 state.
+The headline metric is prefill tokens/s (B*H*T per second) per GPU summed
+over GPUs.  The same JSON line also carries the streaming-decode workload
+(256 x 32 heads, d=128, W=2048, 512 consecutive decode steps), the
+long-context prefill (1 x 16 x 32768, W=1024, C=128), the L1-only runs that
+give the cost of the L2 path, the roofline of the dominant kernel, the
+end-to-end number through the host-buffer entry point and the CPU oracle
+timed on a bounded sample.
+
+Multi-GPU: heads and batches are independent, so every rank runs its own
+copy of the workload with no collective on the data path (weak scaling);
+the timed region is bracketed by barriers and the max over ranks is taken.
+
+--impl reference runs the CPU oracle (the float64 token-by-token definition)
+on the host cores on a bounded sample of the same workload and prints the
+same JSON line with "impl": "reference".
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads as wl  # noqa: E402
+
+HEADLINE = "lm_prefill_bf16"
+METRIC = "prefill tokens/s & decode tok/s per B200; % of TC/HBM roofline"
+UNIT = "tokens/s"
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ---------------------------------------------------------------------------
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    except (OSError, ValueError):
+        return dict(PEAKS_FALLBACK), "fallback"
+
+
+def prefill_flops(B, H, T, dk, dv, W):
+    """Algorithmic FLOPs of one prefill: L1 = 2*(dk+dv) per (query, key in
+    window); L2 = 2*dk*dv write + 2*dk*dv read per eviction / evicted read."""
+    n_pairs = T * W - W * (W - 1) // 2 if T >= W else T * (T + 1) // 2
+    E = max(0, T - W)
+    l1 = 2 * (dk + dv) * n_pairs * B * H
+    l2 = 4 * dk * dv * E * B * H
+    return l1, l2
+
+
+def decode_bytes(B, H, W, dk, dv, esz=2):
+    ring = B * H * W * (dk + dv) * esz
+    A = 2 * B * H * dk * dv * 4
+    io = B * H * (2 * dk + 2 * dv) * esz + B * H * (dk + dv) * esz  # q,k,v,y + ring write
+    return ring + A + io
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.samples = []
+        self.windows = []
+        self._stop = threading.Event()
+        self._thread = None
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self._thread = threading.Thread(target=self._read, daemon=True)
+        self._thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) >= 9:
+                self.samples.append((time.time(), parts))
+
+    def window(self, t0, t1):
+        self.windows.append((t0, t1))
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        inside = [p for (ts, p) in self.samples if any(a <= ts <= b for a, b in self.windows)]
+        use = inside if inside else [p for _, p in self.samples]
+
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        sm = [num(p[1]) for p in use if num(p[1]) is not None]
+        mx = [num(p[2]) for p in use if num(p[2]) is not None]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for p in use for i in range(4) if p[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(use), "samples_in_timed_regions": len(inside)}
+
+
+# ---------------------------------------------------------------------------
+def _dist():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def _barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def _max_over_ranks(x: float, world: int, dev) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def _prefill_device_inputs(name, dev, copies):
+    x = wl.prefill_config(name)
+    sets = []
+    for _ in range(copies):
+        sets.append(tuple(t.to(dev) for t in (x.q, x.k, x.v)))
+    prm = tuple(t.to(dev) for t in (x.lam, x.eta, x.g))
+    return x, sets, prm
+
+
+def time_prefill(tc, name, dev, steps, warmup, world, l1_only=False, clocks=None):
+    """Device time of `steps` prefill calls on rotating input sets (so no
+    step reads inputs left in L2 by the previous one).  Returns per-step
+    event times (ms), the wall of the bracketed region, and launch count."""
+    x, sets, prm = _prefill_device_inputs(name, dev, copies=3)
+    B, H, T, dk = x.q.shape
+    dv = x.v.shape[-1]
+    y = [torch.empty(B, H, T, dv, dtype=x.q.dtype, device=dev) for _ in range(2)]
+    A = torch.empty(B, H, dk, dv, dtype=torch.float32, device=dev)
+    desc = tc.make_prefill_desc(B, H, T, dk, dv, x.W, x.C, tc.TC_BF16 if x.q.dtype ==
+                                torch.bfloat16 else tc.TC_F32, l1_only)
+    ws_n = tc.prefill_workspace_size(desc)
+    ws = torch.empty(max(ws_n, 1), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(i):
+        q, k, v = sets[i % len(sets)]
+        tc.prefill(q, k, v, *prm, x.W, x.C, l1_only=l1_only, y=y[i % 2],
+                   A_final=None if l1_only else A, workspace=ws if ws_n else None, stream=stream)
+
+    for i in range(warmup):
+        step(i)
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    _barrier(world)
+    torch.cuda.synchronize()
+    t0 = time.time()
+    start.record(stream)
+    for i in range(steps):
+        ev[i][0].record(stream)
+        step(i)
+        ev[i][1].record(stream)
+    end.record(stream)
+    torch.cuda.synchronize()
+    _barrier(world)
+    t1 = time.time()
+    if clocks:
+        clocks.window(t0, t1)
+    per = [a.elapsed_time(b) for a, b in ev]
+    total_ms = start.elapsed_time(end)
+    launches = tc_launches_per_prefill(tc, desc)
+    return {"x": x, "per_step_ms": per, "total_ms": total_ms, "wall_s": t1 - t0,
+            "launches_per_step": launches, "tokens_per_step": B * H * T}
+
+
+def tc_launches_per_prefill(tc, desc):
+    """Kernels one tc_prefill call enqueues (from the library's own report)."""
+    fn = getattr(tc, "prefill_launch_count", None)
+    return fn(desc) if fn else None
+
+
+def time_decode(tc, dev, world, clocks=None, steps=None):
+    x = wl.decode_workload(device=dev)
+    n = x.q.shape[0] if steps is None else steps
+    st = tc.DecodeState(x.ring_k, x.ring_v, x.A, x.lam, x.eta, x.g, x.t0)
+    B, H, W, dk = x.ring_k.shape
+    dv = x.ring_v.shape[-1]
+    y = torch.empty(B, H, dv, dtype=x.v.dtype, device=dev)
+    stream = torch.cuda.current_stream()
+    # warm-up on scratch copies is not possible at 9 GB; warm up with 3 real
+    # steps of a separate clock (the state they leave is still a valid state)
+    for i in range(3):
+        tc.decode_step(st, x.q[i], x.k[i], x.v[i], y=y, stream=stream)
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(n)]
+    _barrier(world)
+    torch.cuda.synchronize()
+    t0 = time.time()
+    for i in range(n):
+        ev[i][0].record(stream)
+        tc.decode_step(st, x.q[i], x.k[i], x.v[i], y=y, stream=stream)
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    _barrier(world)
+    t1 = time.time()
+    if clocks:
+        clocks.window(t0, t1)
+    per = [a.elapsed_time(b) for a, b in ev]
+    out = {"B": B, "H": H, "W": W, "d": dk, "steps": n, "per_step_ms": per,
+           "bytes_per_step": decode_bytes(B, H, W, dk, dv)}
+    # end to end: host q/k/v in, host y out, through tc_decode_step_host
+    pin = [tuple(t[i].cpu().pin_memory() for t in (x.q, x.k, x.v)) for i in range(8)]
+    yh = torch.empty(B, H, dv, dtype=x.v.dtype).pin_memory()
+    ws = torch.empty(tc.decode_step_host_workspace_size(st), dtype=torch.uint8, device=dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ne = 32
+    e0.record(stream)
+    for i in range(ne):
+        q, k, v = pin[i % len(pin)]
+        tc.decode_step_host(st, q, k, v, yh, workspace=ws, stream=stream)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    out["e2e_ms_per_step"] = e0.elapsed_time(e1) / ne
+    out["e2e_h2d_bytes"] = sum(t.numel() * t.element_size() for t in pin[0])
+    out["e2e_d2h_bytes"] = yh.numel() * yh.element_size()
+    del x, st
+    torch.cuda.empty_cache()
+    return out
+
+
+def time_prefill_e2e(tc, name, dev, steps):
+    """Same workload through tc_prefill_host: pinned host q, k, v, lam, eta,
+    g in, y and A_final back to pinned host memory, copies inside the timed
+    region."""
+    x = wl.prefill_config(name)
+    B, H, T, dk = x.q.shape
+    dv = x.v.shape[-1]
+    pin = [t.contiguous().pin_memory() for t in (x.q, x.k, x.v, x.lam, x.eta, x.g)]
+    yh = torch.empty(B, H, T, dv, dtype=x.q.dtype).pin_memory()
+    Ah = torch.empty(B, H, dk, dv, dtype=torch.float32).pin_memory()
+    desc = tc.make_prefill_desc(B, H, T, dk, dv, x.W, x.C, tc.TC_BF16)
+    ws = torch.empty(tc.prefill_host_workspace_size(desc), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    for _ in range(2):
+        tc.prefill_host(*pin, x.W, x.C, yh, Ah, workspace=ws, stream=stream)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        tc.prefill_host(*pin, x.W, x.C, yh, Ah, workspace=ws, stream=stream)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    h2d = sum(t.numel() * t.element_size() for t in pin)
+    d2h = yh.numel() * yh.element_size() + Ah.numel() * 4
+    return {"ms_per_step": ms, "tokens_per_s": B * H * T / (ms * 1e-3), "h2d": h2d, "d2h": d2h}
+
+
+# ---------------------------------------------------------------------------
+def oracle_sample(name, budget_s=12.0):
+    """Time the CPU oracle as it stands on a bounded sample of a prefill
+    workload: whole heads (from t = 0, as the layer requires) until about
+    budget_s seconds are spent.  Returns tokens/s and the sample used."""
+    import oracle
+    x = wl.prefill_config(name)
+    B, H, T = x.q.shape[:3]
+    cores = oracle.threads()
+    n_heads, spent, tokens = 0, 0.0, 0
+    order = [(b, h) for b in range(B) for h in range(H)]
+    batch = max(1, cores)
+    while spent < budget_s and n_heads < len(order):
+        group = order[n_heads:n_heads + batch]
+        hs = sorted({h for _, h in group})
+        t0 = time.perf_counter()
+        for h in hs:
+            bs = [b for b, hh in group if hh == h]
+            oracle.prefill(x.q[bs, h:h + 1], x.k[bs, h:h + 1], x.v[bs, h:h + 1],
+                           x.lam[h:h + 1], x.eta[h:h + 1], x.g[h:h + 1], x.W)
+        spent += time.perf_counter() - t0
+        n_heads += len(group)
+        tokens += len(group) * T
+    return {"value": tokens / spent, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"{n_heads} of {B * H} heads x {T} tokens of {name} "
+                      f"(float64 token loop, OpenMP over heads), {spent:.1f} s"}
+
+
+def run_reference(args):
+    world, rank, _ = _dist()
+    if world > 1 and rank != 0:
+        return 0
+    import oracle
+    oracle.build()
+    x = wl.prefill_config(HEADLINE)
+    B, H, T = x.q.shape[:3]
+    cores = oracle.threads()
+    total_budget = 150.0
+    per_step = total_budget / max(1, args.steps + args.warmup)
+    # calibrate: one head for the whole sequence
+    t0 = time.perf_counter()
+    oracle.prefill(x.q[:1, :1], x.k[:1, :1], x.v[:1, :1], x.lam[:1], x.eta[:1], x.g[:1], x.W,
+                   nthreads=1)
+    one = time.perf_counter() - t0
+    heads = max(1, min(B * H, int(per_step / one * cores)))
+    order = [(b, h) for b in range(B) for h in range(H)][:heads]
+
+    def step():
+        by_h = {}
+        for b, h in order:
+            by_h.setdefault(h, []).append(b)
+        for h, bs in by_h.items():
+            oracle.prefill(x.q[bs, h:h + 1], x.k[bs, h:h + 1], x.v[bs, h:h + 1],
+                           x.lam[h:h + 1], x.eta[h:h + 1], x.g[h:h + 1], x.W)
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    el = time.perf_counter() - t0
+    tokens = heads * T * args.steps
+    value = tokens / el
+    sample = (f"{heads} of {B * H} heads x {T} tokens of {HEADLINE} per step "
+              f"(float64 token loop, OpenMP over heads)")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": el / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": HEADLINE, "B": B, "H": H, "T": T, "d": 64, "W": x.W,
+                       "C": x.C},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="tc", choices=["tc", "reference"])
+    ap.add_argument("--no-extras", action="store_true",
+                    help="headline prefill only (skip decode, long prefill, oracle)")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        return run_reference(args)
+
+    world, rank, local = _dist()
+    if world != args.gpus:
+        print(f"warning: --gpus {args.gpus} but WORLD_SIZE={world}", file=sys.stderr)
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    import sliding_window_attention_tc_b200 as tc
+
+    peaks, peak_src = load_peaks()
+    clocks = ClockSampler(local)
+    clocks.start()
+    try:
+        head = time_prefill(tc, HEADLINE, dev, args.steps, args.warmup, world, clocks=clocks)
+        x = head["x"]
+        B, H, T, dk = x.q.shape
+        dv = x.v.shape[-1]
+        total_ms = _max_over_ranks(head["total_ms"], world, dev)
+        ms_step = total_ms / args.steps
+        tokens = head["tokens_per_step"] * args.steps * world
+        value = tokens / (total_ms * 1e-3)
+        l1f, l2f = prefill_flops(B, H, T, dk, dv, x.W)
+        mean_ms = statistics.mean(head["per_step_ms"])
+        achieved_tflops = (l1f + l2f) / (mean_ms * 1e-3) / 1e12
+        peak_tf = float(peaks["bf16_tflops"])
+        roofline = {"bound": "tensor", "achieved": achieved_tflops, "peak": peak_tf,
+                    "unit": "TFLOP/s", "frac": achieved_tflops / peak_tf, "traffic": None,
+                    "peak_source": f"{peak_src} bf16 burst",
+                    "kernel": "tc_prefill (all launches of one call)",
+                    "algorithmic_flops_per_launch": l1f + l2f}
+        extras = {}
+        if not args.no_extras:
+            l1 = time_prefill(tc, HEADLINE, dev, max(20, args.steps // 4), 3, world,
+                              l1_only=True, clocks=clocks)
+            t_l1 = statistics.mean(l1["per_step_ms"])
+            extras["l2_overhead_lm"] = {"tc_ms": mean_ms, "l1_only_ms": t_l1,
+                                        "ratio": mean_ms / t_l1 - 1.0,
+                                        "algorithmic_floor": l2f / l1f}
+            lp = time_prefill(tc, "long_prefill_bf16", dev, 20, 3, world, clocks=clocks)
+            lp1 = time_prefill(tc, "long_prefill_bf16", dev, 20, 3, world, l1_only=True,
+                               clocks=clocks)
+            xl = lp["x"]
+            Bl, Hl, Tl, dl = xl.q.shape
+            f1, f2 = prefill_flops(Bl, Hl, Tl, dl, dl, xl.W)
+            t_lp = statistics.mean(lp["per_step_ms"])
+            t_lp1 = statistics.mean(lp1["per_step_ms"])
+            extras["long_prefill"] = {
+                "workload": "long_prefill_bf16", "B": Bl, "H": Hl, "T": Tl, "d": dl, "W": xl.W,
+                "C": xl.C, "ms": t_lp, "tokens_per_s": Bl * Hl * Tl / (t_lp * 1e-3),
+                "achieved_tflops": (f1 + f2) / (t_lp * 1e-3) / 1e12,
+                "frac_of_bf16_peak": (f1 + f2) / (t_lp * 1e-3) / 1e12 / peak_tf,
+                "l1_only_ms": t_lp1, "l2_overhead_ratio": t_lp / t_lp1 - 1.0,
+                "algorithmic_floor": f2 / f1}
+            del lp, lp1
+            dec = time_decode(tc, dev, world, clocks=clocks)
+            dms = statistics.mean(dec["per_step_ms"])
+            gbs = dec["bytes_per_step"] / (dms * 1e-3) / 1e9
+            extras["decode"] = {
+                "workload": "batched decode 256x32 heads, d=128, W=2048, bf16 ring, fp32 A",
+                "steps": dec["steps"], "ms_per_step_mean": dms,
+                "ms_per_step_p50": statistics.median(dec["per_step_ms"]),
+                "tokens_per_s": dec["B"] / (dms * 1e-3),
+                "roofline": {"bound": "hbm", "achieved": gbs, "peak": float(peaks["hbm_gbs"]),
+                             "unit": "GB/s", "frac": gbs / float(peaks["hbm_gbs"]),
+                             "traffic": None, "peak_source": f"{peak_src} copy bandwidth",
+                             "algorithmic_bytes_per_launch": dec["bytes_per_step"]},
+                "e2e": {"ms_per_step": dec["e2e_ms_per_step"],
+                        "tokens_per_s": dec["B"] / (dec["e2e_ms_per_step"] * 1e-3),
+                        "h2d_bytes_per_step": dec["e2e_h2d_bytes"],
+                        "d2h_bytes_per_step": dec["e2e_d2h_bytes"]}}
+        e2e = time_prefill_e2e(tc, HEADLINE, dev, max(5, min(20, args.steps // 10)))
+    finally:
+        clocks.stop()
+
+    if rank != 0:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+        return 0
+    launches = head["launches_per_step"]
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": HEADLINE, "B": B, "H": H, "T": T, "d": dk, "W": x.W, "C": x.C,
+                   "parallelism": f"replicas x{world} (heads independent, no collective)",
+                   "l2_cache": "inputs rotate over 3 buffer sets (603 MB > 126 MB L2)"},
+        "roofline": roofline,
+        "e2e": {"value": e2e["tokens_per_s"] * world, "unit": UNIT,
+                "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"]},
+        "gpu_launches": None if launches is None else launches * args.steps,
+        "clocks": clocks.summary(),
+    }
+    line.update(extras)
+    if world == 1 and not args.no_extras:
+        line["cpu_baseline"] = oracle_sample(HEADLINE)
+    print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

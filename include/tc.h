@@ -1,0 +1,200 @@
+/*
+ * libtc -- the Tensor Cache layer on NVIDIA B200 (sm_100a).
+ *
+ * The layer is the one of "Tensor Cache: Eviction-conditioned Associative
+ * Memory for Transformers" (arXiv 2605.22884).  Per batch b and head h it
+ * combines two read paths over the keys/values seen so far:
+ *
+ *   L1 (§3.1, eq. (1))  y_local_t = softmax_j(<q_t,k_j>/sqrt(d_k)) v_j over
+ *                       the window j = t-W+1 .. t (exact causal attention);
+ *   L2 (§3.2)           A in R^{d_k x d_v}, A = 0 at the start, written only
+ *                       when a pair leaves the window (Fig. 2 step (3)):
+ *                       A <- lambda_h A + eta_h k_{t-W} v_{t-W}^T,
+ *                       read as the row vector m_t = q_t A (abstract, read
+ *                       identity q (k (x) v) = <q,k> v);
+ *   fusion (Fig. 2 (5)) y_t = y_local_t + sigmoid(g_h) m_t.
+ *
+ * Read-after-write order: inside step t the eviction of token t-W is written
+ * into A BEFORE q_t reads A, and k_t is inserted into the window before the
+ * softmax.  The query at step t therefore sees token t-W through A and tokens
+ * t-W+1..t through the window: every earlier token reaches it through exactly
+ * one path (§3.2).
+ *
+ * Conventions shared by every call:
+ *  - Layouts are row-major and contiguous.  q, k: [B,H,T,d_k]; v, y:
+ *    [B,H,T,d_v]; A: [B,H,d_k,d_v] (so m = q A is a row-vector product);
+ *    lambda, eta, g: [H] float32.  A is always float32.
+ *  - Every pointer is a device pointer unless the function name ends in
+ *    _host.  Every device pointer must be 16-byte aligned.
+ *  - The caller owns every buffer; libtc never allocates device or pinned
+ *    memory.  Scratch space ("workspace") is caller-provided, sized by the
+ *    matching *_workspace_size query.
+ *  - Work is enqueued asynchronously on the caller's stream (NULL = legacy
+ *    default stream).  A call returns once its kernels are enqueued.
+ *  - Host-side validation failures return an error code and enqueue nothing.
+ *    A kernel launch failure returns TC_ERR_CUDA.
+ *  - The library is stateless apart from one per-device status word that
+ *    kernels set when they detect a device-side error (read and cleared by
+ *    tc_get_device_status).
+ */
+#ifndef TC_H
+#define TC_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define TC_API __attribute__((visibility("default")))
+#else
+#define TC_API
+#endif
+
+/* Same type as cudaStream_t; declared here so this header needs no CUDA
+ * headers. */
+typedef struct CUstream_st *tc_stream_t;
+
+typedef enum tc_status {
+    TC_OK = 0,
+    TC_ERR_INVALID_ARG = 1,    /* null / misaligned / host pointer, bad size */
+    TC_ERR_UNSUPPORTED = 2,    /* valid request outside the supported set    */
+    TC_ERR_NO_DEVICE = 3,      /* no CUDA device, or not an sm_100 device    */
+    TC_ERR_CUDA = 4,           /* a CUDA runtime call or launch failed       */
+    TC_ERR_DEVICE_BOUNDS = 5,  /* a kernel caught an out-of-range index      */
+    TC_ERR_DEVICE_TIMEOUT = 6, /* a bounded device wait ran out              */
+    TC_ERR_WORKSPACE = 7       /* workspace missing or smaller than queried  */
+} tc_status;
+
+typedef enum tc_dtype {
+    TC_F32 = 0, /* float32 q/k/v/y, float32 arithmetic                     */
+    TC_BF16 = 1 /* bfloat16 q/k/v/y (RNE output), float32 accumulation/state */
+} tc_dtype;
+
+/* tc_prefill_desc.flags */
+#define TC_PREFILL_L1_ONLY 1u /* skip L2 entirely: y = y_local (sigmoid(g) = 0
+                                 taken literally, no A work); A_final unused */
+
+/* Shapes of one prefill call.  Supported: B, H >= 1; T >= 0; 1 <= d_k, d_v
+ * <= 128; W >= 1; C >= 1. */
+typedef struct tc_prefill_desc {
+    int64_t B, H, T; /* batch, heads, tokens                                 */
+    int64_t dk, dv;  /* key and value head dimensions                        */
+    int64_t W;       /* window length (ring capacity) of L1                  */
+    int64_t C;       /* eviction chunk length of the state scan; the result
+                        does not depend on C beyond rounding                  */
+    tc_dtype dtype;  /* dtype of q, k, v and y                               */
+    uint32_t flags;  /* TC_PREFILL_* bits                                    */
+} tc_prefill_desc;
+
+/* Bytes of device workspace tc_prefill needs for desc (0 if none).  Returns
+ * (size_t)-1 when desc is NULL or invalid. */
+TC_API size_t tc_prefill_workspace_size(const tc_prefill_desc *desc);
+
+/* Training / prefill form of the layer over T tokens from an empty state
+ * (ring empty, A = 0).
+ *
+ * Computes y [B,H,T,d_v] (dtype of desc) and, unless TC_PREFILL_L1_ONLY is
+ * set, A_final [B,H,d_k,d_v] float32 = A after the last eviction (all zero
+ * when T <= W).  A is obtained by the parallel weighted-sum chunk scan of
+ * the paper (abstract; §1 contributions; §2 training considerations):
+ *   A_{c+1} = lambda^{C_c} A_c + eta sum_{i<C_c} lambda^{C_c-1-i} k_i v_i^T
+ * over chunks of evictions, which equals the per-token writes exactly in
+ * real arithmetic; the chunk-mean shortcut is never used.
+ *
+ * q, k, v: device inputs.  lambda, eta, g: [H] float32 device.
+ * y: device output.  With T = 0, q, k, v and y may be NULL.  A_final: device output, may be NULL only with
+ * TC_PREFILL_L1_ONLY.  workspace: device scratch of at least
+ * tc_prefill_workspace_size(desc) bytes (NULL allowed when that is 0); its
+ * contents on entry are ignored and on exit are undefined.
+ * Inputs must not overlap outputs.
+ *
+ * Errors: TC_ERR_INVALID_ARG, TC_ERR_UNSUPPORTED, TC_ERR_WORKSPACE,
+ * TC_ERR_NO_DEVICE, TC_ERR_CUDA.  On error nothing is enqueued except for
+ * TC_ERR_CUDA, after which the outputs are undefined. */
+TC_API tc_status tc_prefill(const tc_prefill_desc *desc, const void *q, const void *k, const void *v,
+                     const float *lambda, const float *eta, const float *g, void *y,
+                     float *A_final, void *workspace, size_t workspace_bytes, tc_stream_t stream);
+
+/* Number of kernel launches one tc_prefill call enqueues for desc on the
+ * current device (the path depends on shapes and dtype), or -1 when desc is
+ * NULL or invalid.  tc_decode_step always enqueues exactly one. */
+TC_API int tc_prefill_launch_count(const tc_prefill_desc *desc);
+
+/* Device staging bytes tc_prefill_host needs: tc_prefill_workspace_size
+ * plus room for q, k, v, y, A_final and the [H] parameters on the device.
+ * Returns (size_t)-1 when desc is NULL or invalid. */
+TC_API size_t tc_prefill_host_workspace_size(const tc_prefill_desc *desc);
+
+/* tc_prefill with HOST inputs and outputs (use pinned memory for overlap).
+ * Enqueues on stream: host-to-device copies of q, k, v, lambda, eta, g into
+ * the caller's device workspace, the prefill, and device-to-host copies of y
+ * and A_final.  The host buffers must stay valid until the stream reaches
+ * that point; synchronize the stream before reading y or A_final.
+ * A_final may be NULL (it is then not copied back). */
+TC_API tc_status tc_prefill_host(const tc_prefill_desc *desc, const void *q, const void *k,
+                          const void *v, const float *lambda, const float *eta, const float *g,
+                          void *y, float *A_final, void *workspace, size_t workspace_bytes,
+                          tc_stream_t stream);
+
+/* Streaming state of one layer: the L1 ring buffer, the L2 matrix and the
+ * clock.  All arrays are caller-owned device memory, updated in place.
+ *   ring_k [B,H,W,d_k], ring_v [B,H,W,d_v] in kv_dtype: slot s holds the
+ *     token t' < t with t' mod W = s among the last min(t,W) tokens;
+ *   A [B,H,d_k,d_v] float32: the L2 state after the evictions so far;
+ *   t: number of tokens consumed so far (the next step's clock).
+ * A prefill over T tokens continues as a stream with t = T, A = A_final and
+ * token j (for the last min(T,W) tokens) copied to slot j mod W. */
+typedef struct tc_decode_state {
+    int64_t B, H, dk, dv, W;
+    int64_t t;
+    tc_dtype kv_dtype; /* dtype of ring_k/ring_v and of q_t, k_t, v_t, y_t */
+    void *ring_k;
+    void *ring_v;
+    float *A;
+    const float *lambda; /* [H] */
+    const float *eta;    /* [H] */
+    const float *g;      /* [H] */
+} tc_decode_state;
+
+/* One streaming step (§3.2, Fig. 2) for every (b,h), in the paper's order:
+ * (2) if t >= W the pair in slot pos = t mod W is evicted, (3) written
+ * A <- lambda A + eta k_old v_old^T, (4) (k_t, v_t) is stored in slot pos,
+ * (5) y_t = softmax-attention(q_t, filled slots) + sigmoid(g) q_t A.
+ * Before the ring fills (t < W) slots t+1..W-1 are masked out.
+ *
+ * q_t, k_t: [B,H,d_k]; v_t, y_t: [B,H,d_v]; device, kv_dtype.
+ * On TC_OK the kernels are enqueued and state->t is incremented on the host.
+ * Supported: d_k = d_v in {16, 32, 64, 128}, 1 <= W.
+ * Errors: as tc_prefill (state->t is unchanged on error). */
+TC_API tc_status tc_decode_step(tc_decode_state *state, const void *q_t, const void *k_t,
+                         const void *v_t, void *y_t, tc_stream_t stream);
+
+/* Device staging bytes tc_decode_step_host needs (q_t, k_t, v_t, y_t).
+ * Returns (size_t)-1 when state is NULL or invalid. */
+TC_API size_t tc_decode_step_host_workspace_size(const tc_decode_state *state);
+
+/* tc_decode_step with HOST q_t, k_t, v_t and y_t (the state stays on the
+ * device): copies the inputs into the device workspace, runs the step and
+ * copies y_t back, all enqueued on stream. */
+TC_API tc_status tc_decode_step_host(tc_decode_state *state, const void *q_t, const void *k_t,
+                              const void *v_t, void *y_t, void *workspace,
+                              size_t workspace_bytes, tc_stream_t stream);
+
+/* Synchronizes stream, then returns and clears the device status word of the
+ * current device: TC_OK, TC_ERR_DEVICE_BOUNDS or TC_ERR_DEVICE_TIMEOUT. */
+TC_API tc_status tc_get_device_status(tc_stream_t stream);
+
+/* Static description of a status code (never NULL). */
+TC_API const char *tc_status_string(tc_status status);
+
+/* Library version, "major.minor.patch". */
+TC_API const char *tc_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TC_H */

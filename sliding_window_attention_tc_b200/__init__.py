@@ -1,0 +1,281 @@
+"""Python binding of libtc, the Tensor Cache layer for B200 (sm_100a).
+
+This module only marshals arguments: it checks that tensors are contiguous
+and of the right dtype, allocates outputs and workspace with PyTorch when the
+caller does not pass them, and calls the C-ABI entry points declared in
+``include/tc.h`` through ctypes.  Every step of the layer runs in the CUDA
+kernels of ``libtc.so``; there is no CPU or PyTorch fallback.  Importing this
+package fails if ``libtc.so`` has not been built
+(``python sliding_window_attention_tc_b200/build.py``).
+
+The layer ("Tensor Cache: Eviction-conditioned Associative Memory for
+Transformers", §3.1-§3.2): per head, exact softmax attention over the last W
+keys (L1) plus a d_k x d_v matrix A written only by pairs evicted from the
+window, A <- lambda A + eta k v^T, read as m = q A (L2), fused as
+y = y_local + sigmoid(g) m.  Within a step the eviction is written before the
+read.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libtc.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"libtc.so not found at {LIB_PATH}; build it with "
+                      "`python sliding_window_attention_tc_b200/build.py`")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+TC_OK = 0
+STATUS_NAMES = {0: "TC_OK", 1: "TC_ERR_INVALID_ARG", 2: "TC_ERR_UNSUPPORTED",
+                3: "TC_ERR_NO_DEVICE", 4: "TC_ERR_CUDA", 5: "TC_ERR_DEVICE_BOUNDS",
+                6: "TC_ERR_DEVICE_TIMEOUT", 7: "TC_ERR_WORKSPACE"}
+TC_F32, TC_BF16 = 0, 1
+TC_PREFILL_L1_ONLY = 1
+
+# Exported C symbols declared in include/tc.h.
+EXPORTED = ("tc_prefill_workspace_size", "tc_prefill", "tc_prefill_launch_count", "tc_prefill_host_workspace_size",
+            "tc_prefill_host", "tc_decode_step", "tc_decode_step_host_workspace_size",
+            "tc_decode_step_host", "tc_get_device_status", "tc_status_string", "tc_version")
+
+
+class PrefillDesc(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int64), ("H", ctypes.c_int64), ("T", ctypes.c_int64),
+                ("dk", ctypes.c_int64), ("dv", ctypes.c_int64), ("W", ctypes.c_int64),
+                ("C", ctypes.c_int64), ("dtype", ctypes.c_int), ("flags", ctypes.c_uint32)]
+
+
+class DecodeStateC(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int64), ("H", ctypes.c_int64), ("dk", ctypes.c_int64),
+                ("dv", ctypes.c_int64), ("W", ctypes.c_int64), ("t", ctypes.c_int64),
+                ("kv_dtype", ctypes.c_int), ("ring_k", ctypes.c_void_p),
+                ("ring_v", ctypes.c_void_p), ("A", ctypes.c_void_p),
+                ("lam", ctypes.c_void_p), ("eta", ctypes.c_void_p), ("g", ctypes.c_void_p)]
+
+
+_vp, _sz, _int = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int
+_PD = ctypes.POINTER(PrefillDesc)
+_DS = ctypes.POINTER(DecodeStateC)
+_lib.tc_prefill_workspace_size.argtypes = [_PD]
+_lib.tc_prefill_workspace_size.restype = _sz
+_lib.tc_prefill.argtypes = [_PD] + [_vp] * 9 + [_sz, _vp]
+_lib.tc_prefill.restype = _int
+_lib.tc_prefill_launch_count.argtypes = [_PD]
+_lib.tc_prefill_launch_count.restype = _int
+_lib.tc_prefill_host_workspace_size.argtypes = [_PD]
+_lib.tc_prefill_host_workspace_size.restype = _sz
+_lib.tc_prefill_host.argtypes = [_PD] + [_vp] * 9 + [_sz, _vp]
+_lib.tc_prefill_host.restype = _int
+_lib.tc_decode_step.argtypes = [_DS] + [_vp] * 4 + [_vp]
+_lib.tc_decode_step.restype = _int
+_lib.tc_decode_step_host_workspace_size.argtypes = [_DS]
+_lib.tc_decode_step_host_workspace_size.restype = _sz
+_lib.tc_decode_step_host.argtypes = [_DS] + [_vp] * 5 + [_sz, _vp]
+_lib.tc_decode_step_host.restype = _int
+_lib.tc_get_device_status.argtypes = [_vp]
+_lib.tc_get_device_status.restype = _int
+_lib.tc_status_string.argtypes = [_int]
+_lib.tc_status_string.restype = ctypes.c_char_p
+_lib.tc_version.argtypes = []
+_lib.tc_version.restype = ctypes.c_char_p
+
+SIZE_ERROR = ctypes.c_size_t(-1).value
+
+
+class TCError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = int(status)
+        super().__init__(f"{where}: {STATUS_NAMES.get(self.status, self.status)} "
+                         f"({status_string(self.status)})")
+
+
+def status_string(status: int) -> str:
+    return _lib.tc_status_string(int(status)).decode()
+
+
+def version() -> str:
+    return _lib.tc_version().decode()
+
+
+def lib_handle() -> ctypes.CDLL:
+    """The loaded libtc (for tests that call the C-ABI directly)."""
+    return _lib
+
+
+def _check(st: int, where: str):
+    if st != TC_OK:
+        raise TCError(st, where)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return TC_F32
+    if t.dtype == torch.bfloat16:
+        return TC_BF16
+    raise TypeError(f"unsupported dtype {t.dtype}; use float32 or bfloat16")
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _contig(*ts):
+    for t in ts:
+        if t is not None and not t.is_contiguous():
+            raise ValueError("tensors must be contiguous")
+
+
+def make_prefill_desc(B, H, T, dk, dv, W, C, dtype: int, l1_only: bool = False) -> PrefillDesc:
+    return PrefillDesc(int(B), int(H), int(T), int(dk), int(dv), int(W), int(C), int(dtype),
+                       TC_PREFILL_L1_ONLY if l1_only else 0)
+
+
+def prefill_workspace_size(desc: PrefillDesc) -> int:
+    n = _lib.tc_prefill_workspace_size(ctypes.byref(desc))
+    if n == SIZE_ERROR:
+        raise TCError(1, "tc_prefill_workspace_size")
+    return int(n)
+
+
+def _desc_of(q, v, W, C, l1_only):
+    B, H, T, dk = q.shape
+    return make_prefill_desc(B, H, T, dk, v.shape[-1], W, C, _dtype_code(q), l1_only)
+
+
+def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, lam: torch.Tensor,
+            eta: torch.Tensor, g: torch.Tensor, W: int, C: int, *, l1_only: bool = False,
+            y: Optional[torch.Tensor] = None, A_final: Optional[torch.Tensor] = None,
+            workspace: Optional[torch.Tensor] = None, stream=None):
+    """tc_prefill on device tensors q, k [B,H,T,dk], v [B,H,T,dv] (float32 or
+    bfloat16), lam, eta, g [H] float32.  Returns (y, A_final); A_final is
+    None with l1_only."""
+    desc = _desc_of(q, v, W, C, l1_only)
+    B, H, T, dk = q.shape
+    dv = v.shape[-1]
+    if y is None:
+        y = torch.empty((B, H, T, dv), dtype=q.dtype, device=q.device)
+    if A_final is None and not l1_only:
+        A_final = torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device)
+    need = prefill_workspace_size(desc)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    _contig(q, k, v, lam, eta, g, y, A_final, workspace)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = _lib.tc_prefill(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(lam), _ptr(eta),
+                         _ptr(g), _ptr(y), _ptr(A_final), _ptr(workspace), ws_bytes,
+                         _stream(stream))
+    _check(st, "tc_prefill")
+    return y, A_final
+
+
+def prefill_launch_count(desc: PrefillDesc) -> int:
+    """Kernel launches one tc_prefill call enqueues for desc."""
+    n = _lib.tc_prefill_launch_count(ctypes.byref(desc))
+    if n < 0:
+        raise TCError(1, "tc_prefill_launch_count")
+    return int(n)
+
+
+def prefill_host_workspace_size(desc: PrefillDesc) -> int:
+    n = _lib.tc_prefill_host_workspace_size(ctypes.byref(desc))
+    if n == SIZE_ERROR:
+        raise TCError(1, "tc_prefill_host_workspace_size")
+    return int(n)
+
+
+def prefill_host(q, k, v, lam, eta, g, W, C, y, A_final=None, *, workspace, l1_only=False,
+                 stream=None):
+    """tc_prefill_host: q, k, v, lam, eta, g, y (and A_final) are HOST tensors
+    (pinned for asynchronous copies); workspace is a device byte tensor of
+    prefill_host_workspace_size bytes.  Enqueued on stream; synchronize
+    before reading y."""
+    desc = _desc_of(q, v, W, C, l1_only)
+    _contig(q, k, v, lam, eta, g, y, A_final, workspace)
+    st = _lib.tc_prefill_host(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(lam),
+                              _ptr(eta), _ptr(g), _ptr(y), _ptr(A_final), _ptr(workspace),
+                              workspace.numel(), _stream(stream))
+    _check(st, "tc_prefill_host")
+    return y, A_final
+
+
+@dataclass
+class DecodeState:
+    """Streaming state (caller-owned device tensors, updated in place):
+    ring_k [B,H,W,dk], ring_v [B,H,W,dv], A [B,H,dk,dv] float32, lam/eta/g
+    [H] float32 and the clock t (tokens consumed so far)."""
+    ring_k: torch.Tensor
+    ring_v: torch.Tensor
+    A: torch.Tensor
+    lam: torch.Tensor
+    eta: torch.Tensor
+    g: torch.Tensor
+    t: int
+
+    def c_struct(self) -> DecodeStateC:
+        B, H, W, dk = self.ring_k.shape
+        dv = self.ring_v.shape[-1]
+        _contig(self.ring_k, self.ring_v, self.A, self.lam, self.eta, self.g)
+        return DecodeStateC(B, H, dk, dv, W, int(self.t), _dtype_code(self.ring_k),
+                            self.ring_k.data_ptr(), self.ring_v.data_ptr(), self.A.data_ptr(),
+                            self.lam.data_ptr(), self.eta.data_ptr(), self.g.data_ptr())
+
+    @staticmethod
+    def empty(B, H, W, dk, dv, lam, eta, g, dtype=torch.bfloat16, device="cuda"):
+        return DecodeState(torch.zeros((B, H, W, dk), dtype=dtype, device=device),
+                           torch.zeros((B, H, W, dv), dtype=dtype, device=device),
+                           torch.zeros((B, H, dk, dv), dtype=torch.float32, device=device),
+                           lam, eta, g, 0)
+
+
+def decode_step(state: DecodeState, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                y: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """tc_decode_step: q, k [B,H,dk], v [B,H,dv] device tensors in the ring's
+    dtype.  Updates the ring and A in place, advances state.t, returns y."""
+    cs = state.c_struct()
+    if y is None:
+        y = torch.empty(v.shape, dtype=v.dtype, device=v.device)
+    _contig(q, k, v, y)
+    st = _lib.tc_decode_step(ctypes.byref(cs), _ptr(q), _ptr(k), _ptr(v), _ptr(y),
+                             _stream(stream))
+    _check(st, "tc_decode_step")
+    state.t = int(cs.t)
+    return y
+
+
+def decode_step_host_workspace_size(state: DecodeState) -> int:
+    cs = state.c_struct()
+    n = _lib.tc_decode_step_host_workspace_size(ctypes.byref(cs))
+    if n == SIZE_ERROR:
+        raise TCError(1, "tc_decode_step_host_workspace_size")
+    return int(n)
+
+
+def decode_step_host(state: DecodeState, q, k, v, y, *, workspace, stream=None):
+    """tc_decode_step_host: q, k, v, y are HOST tensors (pinned); the state
+    stays on the device.  Enqueued on stream; synchronize before reading y."""
+    cs = state.c_struct()
+    _contig(q, k, v, y, workspace)
+    st = _lib.tc_decode_step_host(ctypes.byref(cs), _ptr(q), _ptr(k), _ptr(v), _ptr(y),
+                                  _ptr(workspace), workspace.numel(), _stream(stream))
+    _check(st, "tc_decode_step_host")
+    state.t = int(cs.t)
+    return y
+
+
+def device_status(stream=None) -> int:
+    """tc_get_device_status: synchronizes stream, returns and clears the
+    device status word."""
+    return int(_lib.tc_get_device_status(_stream(stream)))

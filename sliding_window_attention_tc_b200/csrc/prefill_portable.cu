@@ -1,0 +1,261 @@
+// Portable prefill of the Tensor Cache layer: float32 SIMT arithmetic for any
+// supported shape (1 <= d_k, d_v <= 128, any W and C, float32 or bf16
+// inputs).  It is the float32 path, and the path for shapes the tensor-core
+// kernel does not take.
+//
+// "Tensor Cache: Eviction-conditioned Associative Memory for Transformers":
+//  - L1 (§3.1, eq. (1)): softmax over keys t-W+1..t, scaled by 1/sqrt(d_k);
+//  - L2 (§3.2, Fig. 2 step (3); abstract and §1 for the chunk scan): the
+//    evictions e = 0..E-1 (E = max(0, T-W), token e leaves the window at
+//    step e+W) are cut into chunks of C.  A chunk-state kernel runs the
+//    weighted-sum scan  S_{c+1} = lambda^{C_c} S_c + eta sum_i lambda^{C_c-1-i}
+//    k_i v_i^T  per head and stores every chunk's starting state S_c;
+//  - the read at step t (eviction e = t-W, chunk c = e / C, offset r) is
+//    m_t = lambda^{r+1} q_t S_c + eta sum_{i=cC}^{e} lambda^{e-i} <q_t,k_i> v_i
+//    (inter-chunk read of the stored state plus the decay-weighted
+//    intra-chunk part), which is q_t A_t with A_t including token t-W;
+//  - fusion (Fig. 2 step (5)): y_t = y_local_t + sigmoid(g) m_t.
+
+#include "tc_internal.cuh"
+
+namespace tc {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kMaxD = 128;
+constexpr int kMaxPerThread = kMaxD * kMaxD / kThreads;  // 64
+
+__host__ __device__ inline int64_t evictions(int64_t T, int64_t W) { return T > W ? T - W : 0; }
+__host__ __device__ inline int64_t num_chunks(int64_t E, int64_t C) { return (E + C - 1) / C; }
+
+// Chunk scan over one head's evictions; stores S_c (state at the start of
+// chunk c) for c = 0..nC-1 and A_final = the state after all evictions.
+template <typename T>
+__global__ void __launch_bounds__(kThreads) chunk_state_kernel(PrefillParams p, float *states,
+                                                               int64_t nC) {
+    constexpr int KT = 32;
+    __shared__ float sk[KT][kMaxD + 1], sv[KT][kMaxD + 1];
+    __shared__ float sw[KT];
+    const int tid = threadIdx.x;
+    const int64_t bh = blockIdx.x;
+    const int h = (int)(bh % p.H);
+    const int dk = p.dk, dv = p.dv, nel = dk * dv;
+    const int64_t E = evictions(p.T, p.W), C = p.C;
+    const double lam = p.lam[h], eta = p.eta[h];
+    const T *kb = reinterpret_cast<const T *>(p.k) + bh * p.T * dk;
+    const T *vb = reinterpret_cast<const T *>(p.v) + bh * p.T * dv;
+
+    // thread -> column col, rows row0 + i * rstep
+    const int rstep = kThreads / dv;
+    const int col = tid % dv, row0 = tid / dv;
+    const bool active = tid < rstep * dv;
+    float S[kMaxPerThread], D[kMaxPerThread];
+#pragma unroll
+    for (int i = 0; i < kMaxPerThread; ++i) S[i] = 0.f;
+
+    for (int64_t c = 0; c < nC; ++c) {
+        float *Sc = states + (bh * nC + c) * nel;
+        if (active) {
+#pragma unroll
+            for (int i = 0; i < kMaxPerThread; ++i) {
+                const int r = row0 + i * rstep;
+                if (r < dk) Sc[r * dv + col] = S[i];
+            }
+        }
+        const int64_t c0 = c * C;
+        const int64_t Cc = (E - c0 < C) ? E - c0 : C;
+#pragma unroll
+        for (int i = 0; i < kMaxPerThread; ++i) D[i] = 0.f;
+        for (int64_t i0 = 0; i0 < Cc; i0 += KT) {
+            const int nt = (int)((Cc - i0 < KT) ? Cc - i0 : KT);
+            __syncthreads();
+            for (int x = tid; x < nt * dk; x += kThreads)
+                sk[x / dk][x % dk] = to_f32(kb[(c0 + i0 + x / dk) * dk + x % dk]);
+            for (int x = tid; x < nt * dv; x += kThreads)
+                sv[x / dv][x % dv] = to_f32(vb[(c0 + i0 + x / dv) * dv + x % dv]);
+            if (tid < nt) sw[tid] = (float)(eta * pow(lam, (double)(Cc - 1 - (i0 + tid))));
+            __syncthreads();
+            if (active) {
+                for (int j = 0; j < nt; ++j) {
+                    const float wv = sw[j] * sv[j][col];
+#pragma unroll
+                    for (int i = 0; i < kMaxPerThread; ++i) {
+                        const int r = row0 + i * rstep;
+                        if (r < dk) D[i] = fmaf(sk[j][r], wv, D[i]);
+                    }
+                }
+            }
+        }
+        const float dec = (float)pow(lam, (double)Cc);
+#pragma unroll
+        for (int i = 0; i < kMaxPerThread; ++i) S[i] = fmaf(dec, S[i], D[i]);
+    }
+    if (p.A_final && active) {
+        float *A = p.A_final + bh * nel;
+#pragma unroll
+        for (int i = 0; i < kMaxPerThread; ++i) {
+            const int r = row0 + i * rstep;
+            if (r < dk) A[r * dv + col] = S[i];
+        }
+    }
+}
+
+__device__ __forceinline__ float warp_max(float x) {
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));
+    return x;
+}
+__device__ __forceinline__ float warp_sum(float x) {
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+    return x;
+}
+
+// One warp per query row, ROWS consecutive rows per CTA sharing key tiles.
+template <typename Tin>
+__global__ void __launch_bounds__(kThreads) prefill_rows_kernel(PrefillParams p,
+                                                                const float *states, int64_t nC) {
+    constexpr int ROWS = kThreads / 32, KT = 32, CPL = kMaxD / 32;
+    __shared__ float sk[KT][kMaxD + 1], sv[KT][kMaxD + 1];
+    __shared__ float sq[ROWS][kMaxD];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int64_t bh = blockIdx.y;
+    const int h = (int)(bh % p.H);
+    const int dk = p.dk, dv = p.dv;
+    const int64_t T = p.T, W = p.W, C = p.C;
+    const int64_t t0 = (int64_t)blockIdx.x * ROWS;
+    const int64_t t = t0 + warp;
+    const bool row_ok = t < T;
+    const bool use_l2 = !p.l1_only;
+    const Tin *qb = reinterpret_cast<const Tin *>(p.q) + bh * T * dk;
+    const Tin *kb = reinterpret_cast<const Tin *>(p.k) + bh * T * dk;
+    const Tin *vb = reinterpret_cast<const Tin *>(p.v) + bh * T * dv;
+
+    for (int x = tid; x < ROWS * dk; x += kThreads) {
+        const int64_t tt = t0 + x / dk;
+        sq[x / dk][x % dk] = tt < T ? to_f32(qb[tt * dk + x % dk]) : 0.f;
+    }
+
+    const float lam = p.lam[h], eta = p.eta[h];
+    const float log2lam = (float)log2((double)lam);
+    const float scale = (float)(1.4426950408889634 / sqrt((double)dk));
+    const int64_t win_lo = t - W + 1 > 0 ? t - W + 1 : 0;
+    const int64_t e = t - W;                       // eviction read at step t
+    const bool has_l2 = use_l2 && row_ok && e >= 0;
+    const int64_t ch = has_l2 ? e / C : 0;
+    const int64_t intra_lo = ch * C;
+
+    // key range needed by the CTA's rows
+    const int64_t t_last = (t0 + ROWS - 1 < T - 1) ? t0 + ROWS - 1 : T - 1;
+    int64_t lo = t0 - W + 1 > 0 ? t0 - W + 1 : 0;
+    if (use_l2 && t_last >= W) {
+        const int64_t e_first = t0 - W > 0 ? t0 - W : 0;
+        const int64_t l2lo = (e_first / C) * C;
+        if (l2lo < lo) lo = l2lo;
+    }
+
+    float acc[CPL], macc[CPL];
+#pragma unroll
+    for (int i = 0; i < CPL; ++i) acc[i] = macc[i] = 0.f;
+    float m_run = -INFINITY, l_run = 0.f;
+
+    for (int64_t j0 = lo; j0 <= t_last; j0 += KT) {
+        const int nt = (int)((t_last - j0 + 1 < KT) ? t_last - j0 + 1 : KT);
+        __syncthreads();
+        for (int x = tid; x < nt * dk; x += kThreads)
+            sk[x / dk][x % dk] = to_f32(kb[(j0 + x / dk) * dk + x % dk]);
+        for (int x = tid; x < nt * dv; x += kThreads)
+            sv[x / dv][x % dv] = to_f32(vb[(j0 + x / dv) * dv + x % dv]);
+        __syncthreads();
+        if (!row_ok) continue;
+        const int64_t j = j0 + lane;
+        const bool in_win = lane < nt && j >= win_lo && j <= t;
+        const bool in_intra = has_l2 && lane < nt && j >= intra_lo && j <= e;
+        float dot = 0.f;
+        if (in_win || in_intra)
+            for (int r = 0; r < dk; ++r) dot = fmaf(sq[warp][r], sk[lane][r], dot);
+        const float s = in_win ? dot * scale : -INFINITY;
+        const float w = in_intra ? eta * exp2f((float)(e - j) * log2lam) * dot : 0.f;
+        const float m_new = fmaxf(m_run, warp_max(s));
+        float pj = 0.f;
+        if (m_new != -INFINITY) {
+            const float corr = exp2f(m_run - m_new);
+            pj = exp2f(s - m_new);
+            l_run = l_run * corr + warp_sum(pj);
+#pragma unroll
+            for (int i = 0; i < CPL; ++i) acc[i] *= corr;
+            m_run = m_new;
+        }
+        for (int jj = 0; jj < nt; ++jj) {
+            const float pb = __shfl_sync(0xffffffffu, pj, jj);
+            const float wb = __shfl_sync(0xffffffffu, w, jj);
+#pragma unroll
+            for (int i = 0; i < CPL; ++i) {
+                const int c = lane + 32 * i;
+                if (c < dv) {
+                    const float vv = sv[jj][c];
+                    acc[i] = fmaf(pb, vv, acc[i]);
+                    macc[i] = fmaf(wb, vv, macc[i]);
+                }
+            }
+        }
+    }
+    if (!row_ok) return;
+
+    float gate = 0.f;
+    if (has_l2) {
+        // inter-chunk read: lambda^{r+1} q_t S_c
+        gate = sigmoidf_acc(p.g[h]);
+        const int64_t r = e - intra_lo;
+        const float dec = (float)exp2((double)(r + 1) * (double)log2((double)lam));
+        const float *S = states + (bh * nC + ch) * dk * dv;
+#pragma unroll
+        for (int i = 0; i < CPL; ++i) {
+            const int c = lane + 32 * i;
+            if (c < dv) {
+                float mi = 0.f;
+                for (int rr = 0; rr < dk; ++rr) mi = fmaf(sq[warp][rr], S[rr * dv + c], mi);
+                macc[i] = fmaf(dec, mi, macc[i]);
+            }
+        }
+    }
+    Tin *y = reinterpret_cast<Tin *>(p.y) + (bh * T + t) * dv;
+    const float inv_l = 1.0f / l_run;
+#pragma unroll
+    for (int i = 0; i < CPL; ++i) {
+        const int c = lane + 32 * i;
+        if (c < dv) y[c] = from_f32<Tin>(acc[i] * inv_l + gate * macc[i]);
+    }
+}
+
+template <typename T>
+cudaError_t launch_t(const PrefillParams &p, cudaStream_t s) {
+    const int64_t BH = p.B * p.H;
+    if (BH == 0) return cudaSuccess;
+    const int64_t nC = p.l1_only ? 0 : num_chunks(evictions(p.T, p.W), p.C);
+    float *states = reinterpret_cast<float *>(p.workspace);
+    if (!p.l1_only) {
+        chunk_state_kernel<T><<<(unsigned)BH, kThreads, 0, s>>>(p, states, nC);
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    if (p.T > 0) {
+        const dim3 grid((unsigned)((p.T + 7) / 8), (unsigned)BH);
+        prefill_rows_kernel<T><<<grid, kThreads, 0, s>>>(p, states, nC);
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+size_t portable_workspace_bytes(const tc_prefill_desc &d) {
+    if (d.flags & TC_PREFILL_L1_ONLY) return 0;
+    const int64_t nC = num_chunks(evictions(d.T, d.W), d.C);
+    return (size_t)(d.B * d.H * nC * d.dk * d.dv) * sizeof(float);
+}
+
+cudaError_t launch_prefill_portable(const PrefillParams &p, tc_dtype dtype, cudaStream_t s) {
+    return dtype == TC_BF16 ? launch_t<__nv_bfloat16>(p, s) : launch_t<float>(p, s);
+}
+
+}  // namespace tc

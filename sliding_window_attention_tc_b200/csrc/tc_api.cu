@@ -1,0 +1,340 @@
+// C-ABI entry points of libtc: argument validation, path selection and the
+// host-buffer variants.  Everything numeric happens in the kernels of
+// decode.cu, prefill_portable.cu and prefill_sm100.cu.
+
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstring>
+
+#include "tc.h"
+#include "tc_internal.cuh"
+
+// Per-device status word written by kernels that detect an error on the
+// device (never by a trap).
+__device__ int tc_device_status_word;
+
+namespace {
+
+constexpr int64_t kMaxDim = 128;
+constexpr size_t kAlign = 256;
+
+size_t round_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t elem_size(tc_dtype d) { return d == TC_BF16 ? 2 : 4; }
+
+bool valid_dtype(tc_dtype d) { return d == TC_F32 || d == TC_BF16; }
+
+// Host-side checks of a prefill description (no CUDA calls).
+tc_status check_desc(const tc_prefill_desc *d) {
+    if (!d) return TC_ERR_INVALID_ARG;
+    if (d->B < 1 || d->H < 1 || d->T < 0 || d->dk < 1 || d->dv < 1 || d->W < 1 || d->C < 1)
+        return TC_ERR_INVALID_ARG;
+    if (!valid_dtype(d->dtype)) return TC_ERR_INVALID_ARG;
+    if (d->flags & ~TC_PREFILL_L1_ONLY) return TC_ERR_INVALID_ARG;
+    if (d->dk > kMaxDim || d->dv > kMaxDim) return TC_ERR_UNSUPPORTED;
+    // grid limits of the portable path and 32-bit-safe element counts
+    if (d->B * d->H > 65535) return TC_ERR_UNSUPPORTED;
+    if (d->T > (int64_t(1) << 31) || d->W > (int64_t(1) << 31)) return TC_ERR_UNSUPPORTED;
+    if (d->B * d->H * d->T * (d->dk > d->dv ? d->dk : d->dv) > (int64_t(1) << 40))
+        return TC_ERR_UNSUPPORTED;
+    return TC_OK;
+}
+
+// Current device, required to be sm_100 (B200).
+tc_status current_device(int *dev, int *num_sms) {
+    int count = 0;
+    if (cudaGetDeviceCount(&count) != cudaSuccess || count == 0) {
+        cudaGetLastError();
+        return TC_ERR_NO_DEVICE;
+    }
+    if (cudaGetDevice(dev) != cudaSuccess) return TC_ERR_NO_DEVICE;
+    int major = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, *dev) != cudaSuccess)
+        return TC_ERR_CUDA;
+    if (major != 10) return TC_ERR_NO_DEVICE;
+    if (num_sms &&
+        cudaDeviceGetAttribute(num_sms, cudaDevAttrMultiProcessorCount, *dev) != cudaSuccess)
+        return TC_ERR_CUDA;
+    return TC_OK;
+}
+
+// A pointer the device can dereference (device or managed memory).
+bool is_device_ptr(const void *p) {
+    cudaPointerAttributes a;
+    if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+        cudaGetLastError();
+        return false;
+    }
+    return a.type == cudaMemoryTypeDevice || a.type == cudaMemoryTypeManaged;
+}
+
+int *status_ptr() {
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, tc_device_status_word) != cudaSuccess) {
+        cudaGetLastError();
+        return nullptr;
+    }
+    return static_cast<int *>(p);
+}
+
+bool use_sm100(const tc_prefill_desc &d) { return tc::sm100_supported(d); }
+
+size_t prefill_ws(const tc_prefill_desc &d, int num_sms) {
+    return use_sm100(d) ? tc::sm100_workspace_bytes(d, num_sms) : tc::portable_workspace_bytes(d);
+}
+
+int sm_count_or_default() {
+    int dev = 0, sms = 0;
+    if (current_device(&dev, &sms) != TC_OK) return 148;
+    return sms;
+}
+
+tc_status check_decode_state(const tc_decode_state *s) {
+    if (!s) return TC_ERR_INVALID_ARG;
+    if (s->B < 1 || s->H < 1 || s->dk < 1 || s->dv < 1 || s->W < 1 || s->t < 0)
+        return TC_ERR_INVALID_ARG;
+    if (!valid_dtype(s->kv_dtype)) return TC_ERR_INVALID_ARG;
+    if (!s->ring_k || !s->ring_v || !s->A || !s->lambda || !s->eta || !s->g)
+        return TC_ERR_INVALID_ARG;
+    if (!aligned16(s->ring_k) || !aligned16(s->ring_v) || !aligned16(s->A))
+        return TC_ERR_INVALID_ARG;
+    if (!tc::decode_supported((int)s->dk, (int)s->dv, s->kv_dtype)) return TC_ERR_UNSUPPORTED;
+    if (s->B * s->H > (int64_t(1) << 31)) return TC_ERR_UNSUPPORTED;
+    return TC_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *tc_version(void) { return "0.1.0"; }
+
+const char *tc_status_string(tc_status s) {
+    switch (s) {
+        case TC_OK: return "ok";
+        case TC_ERR_INVALID_ARG: return "invalid argument";
+        case TC_ERR_UNSUPPORTED: return "unsupported shape or dtype";
+        case TC_ERR_NO_DEVICE: return "no sm_100 CUDA device";
+        case TC_ERR_CUDA: return "CUDA runtime or launch error";
+        case TC_ERR_DEVICE_BOUNDS: return "device-side bounds check failed";
+        case TC_ERR_DEVICE_TIMEOUT: return "device-side bounded wait timed out";
+        case TC_ERR_WORKSPACE: return "workspace missing or too small";
+    }
+    return "unknown status";
+}
+
+size_t tc_prefill_workspace_size(const tc_prefill_desc *d) {
+    if (check_desc(d) != TC_OK) return (size_t)-1;
+    return prefill_ws(*d, sm_count_or_default());
+}
+
+tc_status tc_prefill(const tc_prefill_desc *d, const void *q, const void *k, const void *v,
+                     const float *lambda, const float *eta, const float *g, void *y,
+                     float *A_final, void *workspace, size_t workspace_bytes,
+                     tc_stream_t stream) {
+    tc_status st = check_desc(d);
+    if (st != TC_OK) return st;
+    const bool l1_only = (d->flags & TC_PREFILL_L1_ONLY) != 0;
+    // With T = 0 the token tensors are empty and may be NULL.
+    const bool empty = d->T == 0;
+    if ((!empty && (!q || !k || !v || !y)) || !lambda || !eta || !g || (!l1_only && !A_final))
+        return TC_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(y) ||
+        (A_final && !aligned16(A_final)) || (workspace && !aligned16(workspace)))
+        return TC_ERR_INVALID_ARG;
+    int dev = 0, sms = 0;
+    st = current_device(&dev, &sms);
+    if (st != TC_OK) return st;
+    const size_t need = prefill_ws(*d, sms);
+    if (need > 0 && (!workspace || workspace_bytes < need)) return TC_ERR_WORKSPACE;
+    const void *ptrs[] = {q, k, v, y, lambda, eta, g};
+    for (int i = 0; i < 7; ++i)
+        if (!(empty && i < 4 && !ptrs[i]) && !is_device_ptr(ptrs[i])) return TC_ERR_INVALID_ARG;
+    if (A_final && !is_device_ptr(A_final)) return TC_ERR_INVALID_ARG;
+    if (need > 0 && !is_device_ptr(workspace)) return TC_ERR_INVALID_ARG;
+
+    tc::PrefillParams p{};
+    p.q = q;
+    p.k = k;
+    p.v = v;
+    p.y = y;
+    p.A_final = l1_only ? nullptr : A_final;
+    p.lam = lambda;
+    p.eta = eta;
+    p.g = g;
+    p.B = d->B;
+    p.H = d->H;
+    p.T = d->T;
+    p.W = d->W;
+    p.C = d->C;
+    p.dk = (int)d->dk;
+    p.dv = (int)d->dv;
+    p.l1_only = l1_only;
+    p.workspace = workspace;
+    p.workspace_bytes = workspace_bytes;
+    p.status = status_ptr();
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = use_sm100(*d) ? tc::launch_prefill_sm100(p, sms, s)
+                                  : tc::launch_prefill_portable(p, d->dtype, s);
+    return e == cudaSuccess ? TC_OK : TC_ERR_CUDA;
+}
+
+int tc_prefill_launch_count(const tc_prefill_desc *d) {
+    if (check_desc(d) != TC_OK) return -1;
+    if (use_sm100(*d)) return tc::sm100_launch_count(*d);
+    const bool l1_only = (d->flags & TC_PREFILL_L1_ONLY) != 0;
+    return (l1_only ? 0 : 1) + (d->T > 0 ? 1 : 0);
+}
+
+size_t tc_prefill_host_workspace_size(const tc_prefill_desc *d) {
+    if (check_desc(d) != TC_OK) return (size_t)-1;
+    const size_t es = elem_size(d->dtype);
+    const size_t nq = (size_t)(d->B * d->H * d->T * d->dk) * es;
+    const size_t nv = (size_t)(d->B * d->H * d->T * d->dv) * es;
+    const size_t na = (size_t)(d->B * d->H * d->dk * d->dv) * sizeof(float);
+    const size_t np = (size_t)d->H * sizeof(float);
+    return round_up(prefill_ws(*d, sm_count_or_default())) + 2 * round_up(nq) + 2 * round_up(nv) +
+           3 * round_up(np) + round_up(na);
+}
+
+tc_status tc_prefill_host(const tc_prefill_desc *d, const void *q, const void *k, const void *v,
+                          const float *lambda, const float *eta, const float *g, void *y,
+                          float *A_final, void *workspace, size_t workspace_bytes,
+                          tc_stream_t stream) {
+    tc_status st = check_desc(d);
+    if (st != TC_OK) return st;
+    const bool l1_only = (d->flags & TC_PREFILL_L1_ONLY) != 0;
+    if ((d->T > 0 && (!q || !k || !v || !y)) || !lambda || !eta || !g) return TC_ERR_INVALID_ARG;
+    int dev = 0, sms = 0;
+    st = current_device(&dev, &sms);
+    if (st != TC_OK) return st;
+    const size_t need = tc_prefill_host_workspace_size(d);
+    if (!workspace || workspace_bytes < need) return TC_ERR_WORKSPACE;
+    if (!aligned16(workspace) || !is_device_ptr(workspace)) return TC_ERR_INVALID_ARG;
+
+    const size_t es = elem_size(d->dtype);
+    const size_t nq = (size_t)(d->B * d->H * d->T * d->dk) * es;
+    const size_t nv = (size_t)(d->B * d->H * d->T * d->dv) * es;
+    const size_t na = (size_t)(d->B * d->H * d->dk * d->dv) * sizeof(float);
+    const size_t np = (size_t)d->H * sizeof(float);
+    char *base = static_cast<char *>(workspace);
+    const size_t ws = round_up(prefill_ws(*d, sms));
+    char *dq = base + ws;
+    char *dk_ = dq + round_up(nq);
+    char *dv_ = dk_ + round_up(nq);
+    char *dy = dv_ + round_up(nv);
+    char *dl = dy + round_up(nv);
+    char *de = dl + round_up(np);
+    char *dg = de + round_up(np);
+    char *da = dg + round_up(np);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const cudaMemcpyKind h2d = cudaMemcpyHostToDevice, d2h = cudaMemcpyDeviceToHost;
+    if (cudaMemcpyAsync(dq, q, nq, h2d, s) != cudaSuccess ||
+        cudaMemcpyAsync(dk_, k, nq, h2d, s) != cudaSuccess ||
+        cudaMemcpyAsync(dv_, v, nv, h2d, s) != cudaSuccess ||
+        cudaMemcpyAsync(dl, lambda, np, h2d, s) != cudaSuccess ||
+        cudaMemcpyAsync(de, eta, np, h2d, s) != cudaSuccess ||
+        cudaMemcpyAsync(dg, g, np, h2d, s) != cudaSuccess)
+        return TC_ERR_CUDA;
+    st = tc_prefill(d, dq, dk_, dv_, reinterpret_cast<float *>(dl), reinterpret_cast<float *>(de),
+                    reinterpret_cast<float *>(dg), dy, l1_only ? nullptr : reinterpret_cast<float *>(da),
+                    ws ? base : nullptr, ws, stream);
+    if (st != TC_OK) return st;
+    if (cudaMemcpyAsync(y, dy, nv, d2h, s) != cudaSuccess) return TC_ERR_CUDA;
+    if (A_final && !l1_only && cudaMemcpyAsync(A_final, da, na, d2h, s) != cudaSuccess)
+        return TC_ERR_CUDA;
+    return TC_OK;
+}
+
+tc_status tc_decode_step(tc_decode_state *s, const void *q_t, const void *k_t, const void *v_t,
+                         void *y_t, tc_stream_t stream) {
+    tc_status st = check_decode_state(s);
+    if (st != TC_OK) return st;
+    if (!q_t || !k_t || !v_t || !y_t) return TC_ERR_INVALID_ARG;
+    if (!aligned16(q_t) || !aligned16(k_t) || !aligned16(v_t) || !aligned16(y_t))
+        return TC_ERR_INVALID_ARG;
+    int dev = 0;
+    st = current_device(&dev, nullptr);
+    if (st != TC_OK) return st;
+    const void *ptrs[] = {q_t, k_t, v_t, y_t, s->ring_k, s->ring_v, s->A, s->lambda, s->eta, s->g};
+    for (const void *p : ptrs)
+        if (!is_device_ptr(p)) return TC_ERR_INVALID_ARG;
+    tc::DecodeParams p{};
+    p.q = q_t;
+    p.k = k_t;
+    p.v = v_t;
+    p.y = y_t;
+    p.ring_k = s->ring_k;
+    p.ring_v = s->ring_v;
+    p.A = s->A;
+    p.lam = s->lambda;
+    p.eta = s->eta;
+    p.g = s->g;
+    p.H = s->H;
+    p.W = s->W;
+    p.t = s->t;
+    p.dk = (int)s->dk;
+    p.dv = (int)s->dv;
+    p.status = status_ptr();
+    cudaError_t e = tc::launch_decode(p, s->kv_dtype, s->B * s->H,
+                                      reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return TC_ERR_CUDA;
+    s->t += 1;
+    return TC_OK;
+}
+
+size_t tc_decode_step_host_workspace_size(const tc_decode_state *s) {
+    if (check_decode_state(s) != TC_OK) return (size_t)-1;
+    const size_t es = elem_size(s->kv_dtype);
+    return 2 * round_up((size_t)(s->B * s->H * s->dk) * es) +
+           2 * round_up((size_t)(s->B * s->H * s->dv) * es);
+}
+
+tc_status tc_decode_step_host(tc_decode_state *s, const void *q_t, const void *k_t,
+                              const void *v_t, void *y_t, void *workspace,
+                              size_t workspace_bytes, tc_stream_t stream) {
+    tc_status st = check_decode_state(s);
+    if (st != TC_OK) return st;
+    if (!q_t || !k_t || !v_t || !y_t) return TC_ERR_INVALID_ARG;
+    int dev = 0;
+    st = current_device(&dev, nullptr);
+    if (st != TC_OK) return st;
+    const size_t need = tc_decode_step_host_workspace_size(s);
+    if (!workspace || workspace_bytes < need) return TC_ERR_WORKSPACE;
+    if (!aligned16(workspace) || !is_device_ptr(workspace)) return TC_ERR_INVALID_ARG;
+    const size_t es = elem_size(s->kv_dtype);
+    const size_t nk = (size_t)(s->B * s->H * s->dk) * es, nv = (size_t)(s->B * s->H * s->dv) * es;
+    char *dq = static_cast<char *>(workspace);
+    char *dk_ = dq + round_up(nk);
+    char *dv_ = dk_ + round_up(nk);
+    char *dy = dv_ + round_up(nv);
+    cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaMemcpyAsync(dq, q_t, nk, cudaMemcpyHostToDevice, cs) != cudaSuccess ||
+        cudaMemcpyAsync(dk_, k_t, nk, cudaMemcpyHostToDevice, cs) != cudaSuccess ||
+        cudaMemcpyAsync(dv_, v_t, nv, cudaMemcpyHostToDevice, cs) != cudaSuccess)
+        return TC_ERR_CUDA;
+    st = tc_decode_step(s, dq, dk_, dv_, dy, stream);
+    if (st != TC_OK) return st;
+    if (cudaMemcpyAsync(y_t, dy, nv, cudaMemcpyDeviceToHost, cs) != cudaSuccess) return TC_ERR_CUDA;
+    return TC_OK;
+}
+
+tc_status tc_get_device_status(tc_stream_t stream) {
+    int dev = 0;
+    tc_status st = current_device(&dev, nullptr);
+    if (st != TC_OK) return st;
+    if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+        return TC_ERR_CUDA;
+    int v = 0;
+    if (cudaMemcpyFromSymbol(&v, tc_device_status_word, sizeof(int)) != cudaSuccess)
+        return TC_ERR_CUDA;
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(tc_device_status_word, &zero, sizeof(int)) != cudaSuccess)
+        return TC_ERR_CUDA;
+    return v == 0 ? TC_OK : static_cast<tc_status>(v);
+}
+
+}  // extern "C"

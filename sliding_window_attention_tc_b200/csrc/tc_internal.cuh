@@ -1,0 +1,102 @@
+// Internal declarations shared by the libtc translation units.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "tc.h"
+
+namespace tc {
+
+// ---- element access -------------------------------------------------------
+
+__device__ __forceinline__ float to_f32(float x) { return x; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+template <typename T> __device__ __forceinline__ T from_f32(float x);
+template <> __device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
+    return __float2bfloat16_rn(x);
+}
+
+// Unpack 16 bytes holding VEC elements of T into floats.
+template <typename T> struct Vec16;
+template <> struct Vec16<float> {
+    static constexpr int N = 4;
+    __device__ __forceinline__ static void unpack(const uint4 &r, float *f) {
+        f[0] = __uint_as_float(r.x);
+        f[1] = __uint_as_float(r.y);
+        f[2] = __uint_as_float(r.z);
+        f[3] = __uint_as_float(r.w);
+    }
+};
+template <> struct Vec16<__nv_bfloat16> {
+    static constexpr int N = 8;
+    __device__ __forceinline__ static void unpack(const uint4 &r, float *f) {
+        const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            f[2 * i] = __uint_as_float(w[i] << 16);
+            f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+        }
+    }
+};
+
+__device__ __forceinline__ uint4 ldg_nc_v4(const void *p) {
+    uint4 r;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+                 : "l"(p));
+    return r;
+}
+
+__device__ __forceinline__ float sigmoidf_acc(float g) { return 1.0f / (1.0f + expf(-g)); }
+
+// ---- device status word ---------------------------------------------------
+
+__device__ __forceinline__ void report(int *status, int code) {
+    if (status) atomicCAS(status, 0, code);
+}
+
+// ---- launch parameter blocks ---------------------------------------------
+
+struct DecodeParams {
+    const void *q, *k, *v;
+    void *y;
+    void *ring_k, *ring_v;
+    float *A;
+    const float *lam, *eta, *g;
+    int64_t H, W, t;
+    int dk, dv;
+    int *status;
+};
+
+struct PrefillParams {
+    const void *q, *k, *v;
+    void *y;
+    float *A_final;
+    const float *lam, *eta, *g;
+    int64_t B, H, T, W, C;
+    int dk, dv;
+    bool l1_only;
+    void *workspace;
+    size_t workspace_bytes;
+    int *status;
+};
+
+// decode.cu
+cudaError_t launch_decode(const DecodeParams &p, tc_dtype dtype, int64_t BH, cudaStream_t s);
+bool decode_supported(int dk, int dv, tc_dtype dtype);
+
+// prefill_portable.cu: any shape in the supported range, SIMT float32 math.
+size_t portable_workspace_bytes(const tc_prefill_desc &d);
+cudaError_t launch_prefill_portable(const PrefillParams &p, tc_dtype dtype, cudaStream_t s);
+
+// prefill_sm100.cu: tcgen05 / TMA path for bf16, d_k = d_v = 64.
+bool sm100_supported(const tc_prefill_desc &d);
+size_t sm100_workspace_bytes(const tc_prefill_desc &d, int num_sms);
+cudaError_t launch_prefill_sm100(const PrefillParams &p, int num_sms, cudaStream_t s);
+int sm100_launch_count(const tc_prefill_desc &d);
+
+}  // namespace tc
