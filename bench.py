@@ -221,9 +221,9 @@ def tc_launches_per_prefill(tc, desc):
     return fn(desc) if fn else None
 
 
-def time_decode(tc, dev, world, clocks=None, steps=None):
-    x = wl.decode_workload(device=dev)
-    n = x.q.shape[0] if steps is None else steps
+def time_decode(tc, dev, world, clocks=None, steps=None, batch=None, e2e=True):
+    x = wl.decode_workload(device=dev, B=batch, steps=None if steps is None else steps + 3)
+    n = x.q.shape[0] - 3 if steps is not None else x.q.shape[0]
     st = tc.DecodeState(x.ring_k, x.ring_v, x.A, x.lam, x.eta, x.g, x.t0)
     B, H, W, dk = x.ring_k.shape
     dv = x.ring_v.shape[-1]
@@ -239,9 +239,10 @@ def time_decode(tc, dev, world, clocks=None, steps=None):
     _barrier(world)
     torch.cuda.synchronize()
     t0 = time.time()
+    off = 3 if steps is not None else 0
     for i in range(n):
         ev[i][0].record(stream)
-        tc.decode_step(st, x.q[i], x.k[i], x.v[i], y=y, stream=stream)
+        tc.decode_step(st, x.q[i + off], x.k[i + off], x.v[i + off], y=y, stream=stream)
         ev[i][1].record(stream)
     torch.cuda.synchronize()
     _barrier(world)
@@ -251,6 +252,8 @@ def time_decode(tc, dev, world, clocks=None, steps=None):
     per = [a.elapsed_time(b) for a, b in ev]
     out = {"B": B, "H": H, "W": W, "d": dk, "steps": n, "per_step_ms": per,
            "bytes_per_step": decode_bytes(B, H, W, dk, dv)}
+    if not e2e:
+        return out
     # end to end: host q/k/v in, host y out, through tc_decode_step_host
     pin = [tuple(t[i].cpu().pin_memory() for t in (x.q, x.k, x.v)) for i in range(8)]
     yh = torch.empty(B, H, dv, dtype=x.v.dtype).pin_memory()
@@ -377,6 +380,28 @@ def run_reference(args):
     return 0
 
 
+def run_only(args, tc, dev, world, peaks):
+    """One workload, numbers only: used for profiler runs (ncu), never for the
+    benchmark line."""
+    if args.only == "decode":
+        d = time_decode(tc, dev, world, steps=args.decode_steps or 16, batch=args.decode_batch,
+                        e2e=False)
+        ms = statistics.mean(d["per_step_ms"])
+        print(json.dumps({"only": "decode", "B": d["B"], "steps": d["steps"], "ms_per_step": ms,
+                          "GB_per_s": d["bytes_per_step"] / (ms * 1e-3) / 1e9}))
+        return 0
+    name = HEADLINE if args.only == "prefill" else "long_prefill_bf16"
+    r = time_prefill(tc, name, dev, args.steps, args.warmup, world)
+    x = r["x"]
+    B, H, T, dk = x.q.shape
+    l1f, l2f = prefill_flops(B, H, T, dk, dk, x.W)
+    ms = statistics.mean(r["per_step_ms"])
+    print(json.dumps({"only": name, "ms_per_step": ms,
+                      "tflops": (l1f + l2f) / (ms * 1e-3) / 1e12,
+                      "launches_per_step": r["launches_per_step"]}))
+    return 0
+
+
 # ---------------------------------------------------------------------------
 def main():
     ap = argparse.ArgumentParser()
@@ -386,6 +411,12 @@ def main():
     ap.add_argument("--impl", default="tc", choices=["tc", "reference"])
     ap.add_argument("--no-extras", action="store_true",
                     help="headline prefill only (skip decode, long prefill, oracle)")
+    ap.add_argument("--only", choices=["prefill", "long", "decode"], default=None,
+                    help="time one workload only and print its numbers (profiling runs)")
+    ap.add_argument("--decode-batch", type=int, default=None,
+                    help="batch of the decode workload (default 256)")
+    ap.add_argument("--decode-steps", type=int, default=None,
+                    help="decode steps (default 512)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -404,6 +435,8 @@ def main():
     import sliding_window_attention_tc_b200 as tc
 
     peaks, peak_src = load_peaks()
+    if args.only:
+        return run_only(args, tc, dev, world, peaks)
     clocks = ClockSampler(local)
     clocks.start()
     try:

@@ -1,29 +1,947 @@
-// Tensor-core prefill path (tcgen05 + TMA); filled in below the portable path.
+// Tensor-core prefill of the Tensor Cache layer for B200 (tcgen05 + TMA),
+// bf16 inputs with d_k = d_v = 64 and W a multiple of 128.
+//
+// "Tensor Cache: Eviction-conditioned Associative Memory for Transformers":
+// L1 is exact softmax attention over the window (§3.1 eq. (1)); L2 is the
+// matrix A written by evicted pairs A <- lambda A + eta k v^T and read as
+// m = q A (§3.2, Fig. 2 steps (3) and (5)); y = y_local + sigmoid(g) m.  The
+// training form computes A with the parallel weighted-sum chunk scan
+// (abstract; §1; §2), here with chunks of 128 evictions = one query tile.
+//
+// Tiling.  Query tile = 128 rows t0..t0+127 of one (b,h).  Its keys are
+// 128-row key tiles:
+//   LEAD  [t0-W, t0-W+128)  (when t0 >= W): column c <= row r is eviction
+//         e = t0-W+c <= t-W, i.e. already in A -> decay-weighted linear read
+//         eta lam^(r-c) <q,k> v (intra-chunk part of m); c > r is in the
+//         window -> softmax.  One Q K^T product serves both paths.
+//   FULL  tiles fully inside every row's window -> softmax.
+//   DIAG  [t0, t0+128): causal mask c <= r.
+// The inter-chunk read lam^(r+1) q S(n0) uses the state S(n0) = A after the
+// first n0 = t0-W evictions, and the state advances per tile as
+//   S(n0+128) = lam^128 S(n0) + K_lead^T diag(eta lam^(127-c)) V_lead,
+// a tensor-core contraction whose scaled keys are split into bf16 hi + lo
+// parts (stacked as the M = 128 rows of one MMA) so that A keeps float32
+// accuracy.
+//
+// Work split.  Each head's query tiles are cut into n_s contiguous spans; a
+// persistent CTA (one per SM) runs spans.  A span that starts after other
+// evictions of its head needs S at its start: a small pre-pass kernel
+// (span_summary_kernel) computes for every span u the state its own
+// evictions add, dA_u; the main kernel combines the predecessors' dA_u with
+// the decay between them.
+//
+// Roles in the main kernel (384 threads):
+//   warp 0        TMA producer: Q tile, then K/V tiles through an NS-stage ring
+//   warp 1        MMA issuer: S = Q K^T into TMEM (double buffered), O += P V
+//                 with P read from TMEM, the L2 MMAs; owns TMEM
+//   warps 4-7     softmax + epilogue: one thread per query row / TMEM lane
+//   warps 8-11    state: keeps S (float32, registers), stages it as bf16 for
+//                 the inter read, builds the scaled hi/lo keys
+// All waits are bounded (mbar_wait); on timeout every role drains and the
+// kernel returns with TC_ERR_DEVICE_TIMEOUT in the status word.
+
+#include <cuda.h>
+
+#include "sm100_ptx.cuh"
 #include "tc_internal.cuh"
 
 namespace tc {
+namespace {
+
+using namespace sm100;
+
+constexpr int BM = 128;                  // query / key rows per tile, eviction chunk
+constexpr int HD = 64;                   // head dimension handled here
+constexpr int NS = 4;                    // K/V stages (main kernel)
+constexpr uint32_t TILE_B = BM * HD * 2; // 16 KB bf16 tile
+constexpr int kMainThreads = 512;
+
+// main-kernel shared memory (offsets from a 1024-aligned base)
+constexpr uint32_t OFF_Q = 0;                          // 2 Q tiles
+constexpr uint32_t OFF_KV = OFF_Q + 2 * TILE_B;        // NS x (K, V)
+constexpr uint32_t OFF_KT = OFF_KV + NS * 2 * TILE_B;  // scaled keys hi | lo
+constexpr uint32_t OFF_SB = OFF_KT + 2 * TILE_B;       // state bf16 [64 k][64 n]
+constexpr uint32_t OFF_DS = OFF_SB + 8192;             // float32 64x64 scratch
+constexpr uint32_t OFF_EPW = OFF_DS + 16384;           // [256]: eta lam^(i-128), 0 for i < 128
+constexpr uint32_t OFF_XM = OFF_EPW + 1024;            // [2 parity][2 halves][128] row maxima
+constexpr uint32_t OFF_XL = OFF_XM + 2048;             // [2 halves][128] row sums
+constexpr uint32_t OFF_BAR = OFF_XL + 1024;
+constexpr uint32_t SMEM_MAIN = OFF_BAR + 256 + 1024;
+
+// TMEM columns (512 allocated)
+constexpr uint32_t TM_S = 0;    // two 128-column score buffers (P / P' alias them)
+constexpr uint32_t TM_O = 256;  // O accumulator, 64 columns
+constexpr uint32_t TM_MI = 320; // intra-chunk memory read
+constexpr uint32_t TM_MX = 384; // inter-chunk memory read q S(n0)
+constexpr uint32_t TM_DS = 448; // state increment: rows 0-63 hi part, 64-127 lo part
+
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kRescale = 8.0f;  // rescale O only when the running max grows by > 2^8
+
+struct MainParams {
+    void *y;
+    float *A_final;
+    const float *lam, *eta, *g;
+    const float *dA;  // [BH * n_s][64][64] span summaries
+    int T, W, H, BH, nT, n_s, l1_only;
+    int *status;
+};
+
+struct SumParams {
+    float *dA;
+    const float *lam, *eta;
+    int T, W, H, BH, nT, n_s;
+    int *status;
+};
+
+__device__ __forceinline__ void span_range(int j, int nT, int n_s, int &i0, int &i1) {
+    i0 = (int)((long long)j * nT / n_s);
+    i1 = (int)((long long)(j + 1) * nT / n_s);
+}
+
+__device__ __forceinline__ void named_bar(int id, int n) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+
+// Barrier for one 128-thread role group on an mbarrier (count 128): unlike
+// bar.sync it gives up with the bounded wait, so an aborting thread cannot
+// leave the rest of its group blocked.
+__device__ __forceinline__ bool group_sync(uint64_t *bar, uint32_t &phase, volatile int *abort,
+                                           int *status) {
+    mbar_arrive(bar);
+    const bool ok = __all_sync(0xffffffffu, mbar_wait(bar, phase & 1, abort, status));
+    ++phase;
+    return ok;
+}
+
+// mbar_wait with one answer for the whole warp, so that warps which go on to
+// warp-collective tcgen05.ld / st never diverge on a failed wait.
+__device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volatile int *abort,
+                                          int *status) {
+    return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort, status));
+}
+
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// Per-tile schedule shared by every role.
+struct TileInfo {
+    int t0, nk, kt0;
+    bool lead, l2;
+};
+__device__ __forceinline__ TileInfo tile_info(int i, int W, bool l1_only) {
+    TileInfo ti;
+    ti.t0 = i * BM;
+    ti.lead = ti.t0 >= W;
+    ti.l2 = ti.lead && !l1_only;
+    if (ti.lead) {
+        ti.nk = W / BM + 1;
+        ti.kt0 = (ti.t0 - W) / BM;
+    } else {
+        ti.nk = i + 1;
+        ti.kt0 = 0;
+    }
+    return ti;
+}
+
+// Kinds of key tile seen by one query row r (column c of the tile):
+//   FULL     every column is in the window            -> softmax
+//   DIAG     c <= r in the window (causal diagonal)   -> softmax, c > r masked
+//   LEAD     c > r in the window, c <= r evicted      -> softmax on c > r, and
+//   LEAD_L2  ... plus the linear read eta lam^(r-c) <q,k> for c <= r (P')
+enum { KIND_FULL = 0, KIND_DIAG = 1, KIND_LEAD = 2, KIND_LEAD_L2 = 3 };
+
+template <int KIND>
+__device__ __forceinline__ bool in_window(int c, int r) {
+    return KIND == KIND_FULL ? true : (KIND == KIND_DIAG ? c <= r : c > r);
+}
+
+// The 128 columns of a score tile are split between two softmax warpgroups:
+// half h owns columns 64h .. 64h+63 (CB = 64h) of every row.
+
+// Row maximum of the raw scores over this half's window columns (-inf if none).
+template <int KIND, int CB>
+__device__ __forceinline__ float window_max(const float (&s)[64], int r) {
+    float m[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) m[i] = -INFINITY;
+#pragma unroll
+    for (int c = 0; c < 64; ++c)
+        m[c & 7] = fmaxf(m[c & 7], in_window<KIND>(CB + c, r) ? s[c] : -INFINITY);
+#pragma unroll
+    for (int i = 4; i >= 1; i >>= 1)
+#pragma unroll
+        for (int j = 0; j < i; ++j) m[j] = fmaxf(m[j], m[j + i]);
+    return m[0];
+}
+
+// P = exp2(s * sl2 - m) on window columns (0 elsewhere) as bf16 pairs into 32
+// TMEM columns starting at taddr; returns this half's row sum of P.
+template <int KIND, int CB>
+__device__ __forceinline__ float write_p(const float (&s)[64], int r, float sl2, float m,
+                                         uint32_t taddr) {
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int c0 = 0; c0 < 64; c0 += 32) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+            const int c = c0 + 2 * e;
+            const float x0 = in_window<KIND>(CB + c, r) ? fmaf(s[c], sl2, -m) : -INFINITY;
+            const float x1 = in_window<KIND>(CB + c + 1, r) ? fmaf(s[c + 1], sl2, -m) : -INFINITY;
+            const float p0 = ex2(x0), p1 = ex2(x1);
+            acc[e & 3] += p0 + p1;
+            pk[e] = pack_bf16(p0, p1);
+        }
+        tmem_st16(taddr + c0 / 2, pk);
+    }
+    return (acc[0] + acc[1]) + (acc[2] + acc[3]);
+}
+
+// P' = eta lam^(r-c) s for c <= r (the zero-padded table gives 0 for c > r)
+// as bf16 pairs into 32 TMEM columns starting at taddr.
+template <int CB>
+__device__ __forceinline__ void write_plin(const float (&s)[64], int r, const float *epw_pad,
+                                           uint32_t taddr) {
+    const float *w = epw_pad + 128 + r - CB;  // w[-c] = eta lam^(r-CB-c), or 0
+#pragma unroll
+    for (int c0 = 0; c0 < 64; c0 += 32) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+            const int c = c0 + 2 * e;
+            pk[e] = pack_bf16(s[c] * w[-c], s[c + 1] * w[-c - 1]);
+        }
+        tmem_st16(taddr + c0 / 2, pk);
+    }
+}
+
+template <int CB>
+__device__ __forceinline__ float half_max(int kind, const float (&s)[64], int r) {
+    switch (kind) {
+        case KIND_FULL: return window_max<KIND_FULL, CB>(s, r);
+        case KIND_DIAG: return window_max<KIND_DIAG, CB>(s, r);
+        default: return window_max<KIND_LEAD, CB>(s, r);
+    }
+}
+template <int CB>
+__device__ __forceinline__ float half_p(int kind, const float (&s)[64], int r, float sl2, float m,
+                                        uint32_t taddr) {
+    switch (kind) {
+        case KIND_FULL: return write_p<KIND_FULL, CB>(s, r, sl2, m, taddr);
+        case KIND_DIAG: return write_p<KIND_DIAG, CB>(s, r, sl2, m, taddr);
+        default: return write_p<KIND_LEAD, CB>(s, r, sl2, m, taddr);
+    }
+}
+
+// Scaled key row for the state MMA: row u of the key tile times w, split into
+// bf16 hi and lo = bf16(x - hi), written to two SWIZZLE_128B tiles.
+__device__ __forceinline__ void build_scaled_key_row(const uint8_t *ktile, uint8_t *hi_tile,
+                                                     uint8_t *lo_tile, int u, float w) {
+#pragma unroll
+    for (int ch = 0; ch < 8; ++ch) {
+        const uint32_t off = sw128_offset(u, ch * 8);
+        const uint4 raw = *reinterpret_cast<const uint4 *>(ktile + off);
+        float f[8];
+        Vec16<__nv_bfloat16>::unpack(raw, f);
+        uint32_t h[4], l[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const float x0 = f[2 * e] * w, x1 = f[2 * e + 1] * w;
+            const uint32_t hp = pack_bf16(x0, x1);
+            const float h0 = __uint_as_float(hp << 16), h1 = __uint_as_float(hp & 0xffff0000u);
+            h[e] = hp;
+            l[e] = pack_bf16(x0 - h0, x1 - h1);
+        }
+        *reinterpret_cast<uint4 *>(hi_tile + off) = make_uint4(h[0], h[1], h[2], h[3]);
+        *reinterpret_cast<uint4 *>(lo_tile + off) = make_uint4(l[0], l[1], l[2], l[3]);
+    }
+}
+
+// ============================================================================
+// Pre-pass: dA_u = sum over the evictions e of span u of
+//           eta lam^(e_end - 1 - e) k_e v_e^T     (e_end = end of span u)
+// ============================================================================
+constexpr int NS_SUM = 2;
+constexpr uint32_t SOFF_KV = 0;
+constexpr uint32_t SOFF_KT = SOFF_KV + NS_SUM * 2 * TILE_B;  // one buffer (hi, lo)
+constexpr uint32_t SOFF_DS = SOFF_KV;                        // scratch: stage 0, after the MMAs
+constexpr uint32_t SOFF_BAR = SOFF_KT + 2 * TILE_B;
+constexpr uint32_t SMEM_SUM = SOFF_BAR + 128 + 1024;         // ~97 KB: two CTAs per SM
+
+__global__ void __launch_bounds__(192, 2)
+    span_summary_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
+                        SumParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                              ~uintptr_t(1023));
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + SOFF_BAR);
+    uint64_t *kv_full = bars, *kv_empty = bars + NS_SUM;
+    uint64_t *kt_full = bars + 2 * NS_SUM, *kt_empty = kt_full + 1, *done = kt_empty + 1;
+    uint32_t *tmem_base = reinterpret_cast<uint32_t *>(done + 1);
+    volatile int *abort = reinterpret_cast<volatile int *>(tmem_base + 1);
+    float *sDS = reinterpret_cast<float *>(sm + SOFF_DS);
+
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const int per_head = p.n_s - 1;
+    const int bh = blockIdx.x / per_head, js = blockIdx.x % per_head;
+    const int h = bh % p.H;
+    int i0, i1;
+    span_range(js, p.nT, p.n_s, i0, i1);
+    const int E = p.T > p.W ? p.T - p.W : 0;
+    const int ev_first = i0 > p.W / BM ? i0 : p.W / BM;  // first tile with evictions
+    const int ne = i1 > ev_first ? i1 - ev_first : 0;
+    const int e_end = ne > 0 ? min(E, i1 * BM - p.W) : 0;
+
+    if (tid == 0) {
+        for (int s = 0; s < NS_SUM; ++s) {
+            mbar_init(&kv_full[s], 1);
+            mbar_init(&kv_empty[s], 1);
+        }
+        mbar_init(kt_full, 128);
+        mbar_init(kt_empty, 1);
+        mbar_init(done, 1);
+        *abort = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_base, 64);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tb = *tmem_base;
+    float *out = p.dA + (size_t)(bh * p.n_s + js) * HD * HD;
+
+    if (ne == 0) {
+        for (int x = tid; x < HD * HD; x += blockDim.x) out[x] = 0.f;
+    } else if (warp == 0) {
+        if (tid == 0) {
+            tma_prefetch_desc(&tk);
+            tma_prefetch_desc(&tv);
+            int issued = 0;
+            for (int e = 0; e < ne; ++e) {
+                const int s = e % NS_SUM;
+                if (!mbar_wait(&kv_empty[s], ((e / NS_SUM) & 1) ^ 1, abort, p.status)) break;
+                const int n0 = (ev_first + e) * BM - p.W;
+                uint8_t *dst = sm + SOFF_KV + s * 2 * TILE_B;
+                mbar_expect_tx(&kv_full[s], 2 * TILE_B);
+                tma_load_3d(dst, &tk, &kv_full[s], 0, n0, bh);
+                tma_load_3d(dst + TILE_B, &tv, &kv_full[s], 0, n0, bh);
+                issued = e + 1;
+            }
+            for (int st = 0; st < NS_SUM; ++st) {
+                const int fills = issued > st ? (issued - 1 - st) / NS_SUM + 1 : 0;
+                if (fills) mbar_wait_drain(&kv_full[st], (fills - 1) & 1);
+            }
+        }
+    } else if (warp == 1) {
+        if (tid == 32) {
+            const uint32_t id_ds = idesc_bf16(128, 64, true, true);
+            for (int e = 0; e < ne; ++e) {
+                const int s = e % NS_SUM;
+                if (!mbar_wait(kt_full, e & 1, abort, p.status)) break;
+                tc_fence_after();
+                const uint32_t kt = smem_u32(sm + SOFF_KT);
+                const uint32_t vv = smem_u32(sm + SOFF_KV + s * 2 * TILE_B + TILE_B);
+#pragma unroll
+                for (int k = 0; k < 8; ++k)
+                    mma_ss(tb, sdesc_sw128(kt + 2048 * k, TILE_B, 1024),
+                           sdesc_sw128(vv + 2048 * k, TILE_B, 1024), id_ds, (e > 0 || k > 0));
+                mma_commit(kt_empty);
+                mma_commit(&kv_empty[s]);
+            }
+            mma_commit(done);
+            mbar_wait_drain(done, 0);
+        }
+    } else {
+        // builders: warps 2-5, thread u builds key row u
+        const int u = tid - 64;
+        const double lam = p.lam[h];
+        const float eta = p.eta[h];
+        const double l2l = log2(lam);
+        for (int e = 0; e < ne; ++e) {
+            const int s = e % NS_SUM;
+            if (!mbar_wait(&kv_full[s], (e / NS_SUM) & 1, abort, p.status)) break;
+            if (!mbar_wait(kt_empty, (e & 1) ^ 1, abort, p.status)) break;
+            const int n0 = (ev_first + e) * BM - p.W;
+            const int ev = n0 + u;
+            const float w = ev < e_end ? eta * (float)exp2((double)(e_end - 1 - ev) * l2l) : 0.f;
+            uint8_t *kt = sm + SOFF_KT;
+            build_scaled_key_row(sm + SOFF_KV + s * 2 * TILE_B, kt, kt + TILE_B, u, w);
+            fence_async_smem();
+            mbar_arrive(kt_full);
+        }
+        // read the accumulated [hi; lo] rows and add the halves
+        const bool ok = warp_wait(done, 0, abort, p.status);
+        tc_fence_after();
+        const int lane_base = 32 * (warp & 3);
+        const int L = lane_base + (tid & 31);
+        float v[64];
+        if (ok) {
+            uint32_t r[32];
+            tmem_ld32(tmem_addr(tb, lane_base, 0), r);
+            tmem_wait_ld();
+#pragma unroll
+            for (int c = 0; c < 32; ++c) v[c] = __uint_as_float(r[c]);
+            tmem_ld32(tmem_addr(tb, lane_base, 32), r);
+            tmem_wait_ld();
+#pragma unroll
+            for (int c = 0; c < 32; ++c) v[32 + c] = __uint_as_float(r[c]);
+        }
+        if (L >= 64) {
+#pragma unroll
+            for (int c = 0; c < 64; ++c) sDS[c * 64 + (L - 64)] = ok ? v[c] : 0.f;
+        }
+        named_bar(1, 128);
+        if (L < 64) {
+#pragma unroll
+            for (int c = 0; c < 64; ++c) out[L * HD + c] = ok ? v[c] + sDS[c * 64 + L] : 0.f;
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tb, 64);
+}
+
+// ============================================================================
+// Main kernel
+// ============================================================================
+__global__ void __launch_bounds__(kMainThreads, 1)
+    prefill_main_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
+                        const __grid_constant__ CUtensorMap tv, MainParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                              ~uintptr_t(1023));
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + OFF_BAR);
+    uint64_t *q_full = bars, *q_empty = bars + 2;
+    uint64_t *kv_full = bars + 4, *kv_empty = kv_full + NS;
+    uint64_t *s_full = kv_empty + NS, *p_full = s_full + 2, *s_empty = p_full + 2;
+    uint64_t *o_prog = s_empty + 2, *o_full = o_prog + 1, *o_empty = o_full + 1;
+    uint64_t *sst_full = o_empty + 1, *kt_full = sst_full + 1, *ds_full = kt_full + 1;
+    uint64_t *lead_ready = ds_full + 1, *mma_done = lead_ready + 1;
+    uint64_t *sm_sync = mma_done + 1, *st_sync = sm_sync + 1;  // group barriers (256, 128)
+    uint32_t *tmem_base = reinterpret_cast<uint32_t *>(st_sync + 1);
+    volatile int *abort = reinterpret_cast<volatile int *>(tmem_base + 1);
+    float *epw = reinterpret_cast<float *>(sm + OFF_EPW);
+    float *sDS = reinterpret_cast<float *>(sm + OFF_DS);
+
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const bool l1_only = p.l1_only != 0;
+    const int n_spans = p.BH * p.n_s;
+    const int E = p.T > p.W ? p.T - p.W : 0;
+
+    if (tid == 0) {
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&q_full[b], 1);
+            mbar_init(&q_empty[b], 1);
+            mbar_init(&s_full[b], 1);
+            mbar_init(&p_full[b], 256);
+            mbar_init(&s_empty[b], 1);
+        }
+        for (int s = 0; s < NS; ++s) {
+            mbar_init(&kv_full[s], 1);
+            mbar_init(&kv_empty[s], 1);
+        }
+        mbar_init(o_prog, 1);
+        mbar_init(o_full, 1);
+        mbar_init(o_empty, 256);
+        mbar_init(sst_full, 128);
+        mbar_init(kt_full, 128);
+        mbar_init(ds_full, 1);
+        mbar_init(lead_ready, 1);
+        mbar_init(mma_done, 1);
+        mbar_init(sm_sync, 256);
+        mbar_init(st_sync, 128);
+        *abort = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_base, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tb = *tmem_base;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer
+        if (tid == 0) {
+            tma_prefetch_desc(&tq);
+            tma_prefetch_desc(&tk);
+            tma_prefetch_desc(&tv);
+            uint32_t tile = 0, kc = 0;
+            bool ok = true;
+            for (int sp = blockIdx.x; sp < n_spans && ok; sp += gridDim.x) {
+                const int bh = sp / p.n_s;
+                int i0, i1;
+                span_range(sp % p.n_s, p.nT, p.n_s, i0, i1);
+                for (int i = i0; i < i1 && ok; ++i, ++tile) {
+                    const TileInfo ti = tile_info(i, p.W, l1_only);
+                    const int qb = tile & 1;
+                    if (!(ok = mbar_wait(&q_empty[qb], ((tile >> 1) & 1) ^ 1, abort, p.status))) break;
+                    mbar_expect_tx(&q_full[qb], TILE_B);
+                    tma_load_3d(sm + OFF_Q + qb * TILE_B, &tq, &q_full[qb], 0, ti.t0, bh);
+                    for (int j = 0; j < ti.nk; ++j, ++kc) {
+                        const int s = kc % NS;
+                        if (!(ok = mbar_wait(&kv_empty[s], ((kc / NS) & 1) ^ 1, abort, p.status))) break;
+                        uint8_t *dst = sm + OFF_KV + s * 2 * TILE_B;
+                        const int row = (ti.kt0 + j) * BM;
+                        mbar_expect_tx(&kv_full[s], 2 * TILE_B);
+                        tma_load_3d(dst, &tk, &kv_full[s], 0, row, bh);
+                        tma_load_3d(dst + TILE_B, &tv, &kv_full[s], 0, row, bh);
+                    }
+                }
+            }
+            // every issued copy must land before the CTA exits (normally the
+            // MMA side has already waited for all of them)
+            for (uint32_t st = 0; st < NS; ++st) {
+                const uint32_t fills = kc > st ? (kc - 1 - st) / NS + 1 : 0;
+                if (fills) mbar_wait_drain(&kv_full[st], (fills - 1) & 1);
+            }
+            for (uint32_t b = 0; b < 2; ++b) {
+                const uint32_t fills = tile > b ? (tile - 1 - b) / 2 + 1 : 0;
+                if (fills) mbar_wait_drain(&q_full[b], (fills - 1) & 1);
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (tid == 32) {
+            const uint32_t id_qk = idesc_bf16(128, 128, false, false);
+            const uint32_t id_pv = idesc_bf16(128, 64, false, true);
+            const uint32_t id_qs = idesc_bf16(128, 64, false, true);
+            const uint32_t id_ds = idesc_bf16(128, 64, true, true);
+            const uint32_t sb_addr = smem_u32(sm + OFF_SB);
+            const uint32_t kt_addr = smem_u32(sm + OFF_KT);
+            uint32_t tile = 0, kc = 0, lc = 0;
+            bool ok = true;
+            for (int sp = blockIdx.x; sp < n_spans && ok; sp += gridDim.x) {
+                int i0, i1;
+                span_range(sp % p.n_s, p.nT, p.n_s, i0, i1);
+                for (int i = i0; i < i1 && ok; ++i, ++tile) {
+                    const TileInfo ti = tile_info(i, p.W, l1_only);
+                    const int qb = tile & 1;
+                    const uint32_t q_addr = smem_u32(sm + OFF_Q + qb * TILE_B);
+                    if (!(ok = mbar_wait(&q_full[qb], (tile >> 1) & 1, abort, p.status))) break;
+                    const uint32_t kc0 = kc;
+                    auto pv_step = [&](int j) -> bool {
+                        const uint32_t g = kc0 + j;
+                        const int sb = g & 1, s = g % NS;
+                        if (!mbar_wait(&p_full[sb], (g >> 1) & 1, abort, p.status)) return false;
+                        if (j == 0 && !mbar_wait(o_empty, (tile & 1) ^ 1, abort, p.status)) return false;
+                        tc_fence_after();
+                        const uint32_t v_addr = smem_u32(sm + OFF_KV + s * 2 * TILE_B + TILE_B);
+                        const uint32_t s_col = tb + TM_S + sb * 128;
+#pragma unroll
+                        for (int k = 0; k < 8; ++k)
+                            mma_ts(tb + TM_O, s_col + 8 * k, sdesc_sw128(v_addr + 2048 * k, TILE_B, 1024),
+                                   id_pv, (j > 0 || k > 0));
+                        if (j == 0 && ti.l2) {
+#pragma unroll
+                            for (int k = 0; k < 8; ++k)
+                                mma_ts(tb + TM_MI, s_col + 64 + 8 * k,
+                                       sdesc_sw128(v_addr + 2048 * k, TILE_B, 1024), id_pv, k > 0);
+                            if (!mbar_wait(sst_full, lc & 1, abort, p.status)) return false;
+                            tc_fence_after();
+#pragma unroll
+                            for (int k = 0; k < 4; ++k)
+                                mma_ss(tb + TM_MX, sdesc_sw128(q_addr + 32 * k, 16, 1024),
+                                       sdesc_sw128(sb_addr + 2048 * k, 8192, 1024), id_qs, k > 0);
+                            if (!mbar_wait(kt_full, lc & 1, abort, p.status)) return false;
+                            tc_fence_after();
+#pragma unroll
+                            for (int k = 0; k < 8; ++k)
+                                mma_ss(tb + TM_DS, sdesc_sw128(kt_addr + 2048 * k, TILE_B, 1024),
+                                       sdesc_sw128(v_addr + 2048 * k, TILE_B, 1024), id_ds, k > 0);
+                            mma_commit(ds_full);
+                            ++lc;
+                        }
+                        mma_commit(&s_empty[sb]);
+                        mma_commit(o_prog);
+                        mma_commit(&kv_empty[s]);
+                        return true;
+                    };
+                    for (int j = 0; j < ti.nk && ok; ++j) {
+                        const uint32_t g = kc0 + j;
+                        const int s = g % NS, sb = g & 1;
+                        if (!(ok = mbar_wait(&kv_full[s], (g / NS) & 1, abort, p.status))) break;
+                        // the state warps read the leading key tile: hand it on
+                        if (j == 0 && ti.l2) mbar_arrive(lead_ready);
+                        if (!(ok = mbar_wait(&s_empty[sb], ((g >> 1) & 1) ^ 1, abort, p.status))) break;
+                        tc_fence_after();
+                        const uint32_t k_addr = smem_u32(sm + OFF_KV + s * 2 * TILE_B);
+#pragma unroll
+                        for (int k = 0; k < 4; ++k)
+                            mma_ss(tb + TM_S + sb * 128, sdesc_sw128(q_addr + 32 * k, 16, 1024),
+                                   sdesc_sw128(k_addr + 32 * k, 16, 1024), id_qk, k > 0);
+                        mma_commit(&s_full[sb]);
+                        if (j >= 1) ok = pv_step(j - 1);
+                    }
+                    if (ok) ok = pv_step(ti.nk - 1);
+                    mma_commit(&q_empty[qb]);
+                    mma_commit(o_full);
+                    kc = kc0 + ti.nk;
+                }
+            }
+            // nothing may still run on the tensor cores when TMEM is released
+            mma_commit(mma_done);
+            mbar_wait_drain(mma_done, 0);
+        }
+    } else if (warp >= 4 && warp < 12) {
+        // ------------------------------------------------------------ softmax + epilogue
+        // two warpgroups; half h = 0 (warps 4-7) / 1 (warps 8-11) owns score
+        // columns 64h.., output columns 32h..; both see every row r (TMEM lane)
+        const int half = (warp - 4) >> 2;
+        const int r = tid - 128 - 128 * half;
+        const int lane_base = 32 * (warp & 3);
+        const float sl2 = kLog2e * rsqrtf((float)HD);
+        float *xm = reinterpret_cast<float *>(sm + OFF_XM);
+        float *xl = reinterpret_cast<float *>(sm + OFF_XL);
+        uint32_t tile = 0, kc = 0, sync_phase = 0;
+        bool ok = true;
+        for (int sp = blockIdx.x; sp < n_spans && ok; sp += gridDim.x) {
+            const int bh = sp / p.n_s, h = bh % p.H;
+            int i0, i1;
+            span_range(sp % p.n_s, p.nT, p.n_s, i0, i1);
+            const double lam = p.lam[h];
+            const float gate = 1.0f / (1.0f + expf(-p.g[h]));
+            const float pw_r1 = (float)pow(lam, (double)(r + 1));
+            // previous span done with epw, then publish this head's table
+            if (!(ok = group_sync(sm_sync, sync_phase, abort, p.status))) break;
+            if (half == 0)
+                epw[128 + r] = (float)((double)p.eta[h] * pow(lam, (double)r));
+            else
+                epw[r] = 0.f;
+            if (!(ok = group_sync(sm_sync, sync_phase, abort, p.status))) break;
+            for (int i = i0; i < i1 && ok; ++i, ++tile) {
+                const TileInfo ti = tile_info(i, p.W, l1_only);
+                float m_used = -INFINITY, l = 0.f;
+                for (int j = 0; j < ti.nk && ok; ++j, ++kc) {
+                    const int sb = kc & 1;
+                    if (!(ok = warp_wait(&s_full[sb], (kc >> 1) & 1, abort, p.status))) break;
+                    tc_fence_after();
+                    const uint32_t s_col = TM_S + sb * 128;
+                    float s[64];
+                    {
+                        uint32_t ra[32], rb[32];
+                        tmem_ld32(tmem_addr(tb, lane_base, s_col + 64 * half), ra);
+                        tmem_ld32(tmem_addr(tb, lane_base, s_col + 64 * half + 32), rb);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int c = 0; c < 32; ++c) {
+                            s[c] = __uint_as_float(ra[c]);
+                            s[32 + c] = __uint_as_float(rb[c]);
+                        }
+                    }
+                    const int kind = (j == 0 && ti.lead) ? (ti.l2 ? KIND_LEAD_L2 : KIND_LEAD)
+                                                         : (j == ti.nk - 1 ? KIND_DIAG : KIND_FULL);
+                    const float mh = half == 0 ? half_max<0>(kind, s, r) : half_max<64>(kind, s, r);
+                    float *xmk = xm + (kc & 1) * 256;
+                    xmk[half * 128 + r] = mh;
+                    if (!(ok = group_sync(sm_sync, sync_phase, abort, p.status))) break;
+                    const float mt = fmaxf(mh, xmk[(1 - half) * 128 + r]) * sl2;  // sl2 > 0
+                    // Raise the row's reference max only when it grew by more than
+                    // 2^kRescale; rows whose O already holds earlier P V products
+                    // are rescaled in TMEM (each half its 32 columns of O).  TMEM
+                    // access is warp-collective, so the warp rescales together.
+                    const bool raise = mt > m_used + kRescale;
+                    const bool resc = raise && m_used != -INFINITY && j > 0;
+                    const float fo = resc ? ex2(m_used - mt) : 1.0f;
+                    if (__any_sync(0xffffffffu, resc)) {
+                        if (!(ok = warp_wait(o_prog, (kc - 1) & 1, abort, p.status))) break;
+                        tc_fence_after();
+                        uint32_t rr[32];
+                        tmem_ld32(tmem_addr(tb, lane_base, TM_O + 32 * half), rr);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int c = 0; c < 32; ++c)
+                            rr[c] = __float_as_uint(__uint_as_float(rr[c]) * fo);
+                        tmem_st32(tmem_addr(tb, lane_base, TM_O + 32 * half), rr);
+                    }
+                    l *= fo;
+                    if (raise) m_used = mt;
+                    const uint32_t p_addr = tmem_addr(tb, lane_base, s_col + 32 * half);
+                    l += half == 0 ? half_p<0>(kind, s, r, sl2, m_used, p_addr)
+                                   : half_p<64>(kind, s, r, sl2, m_used, p_addr);
+                    if (kind == KIND_LEAD_L2) {
+                        if (half == 0)
+                            write_plin<0>(s, r, epw, p_addr + 64);
+                        else
+                            write_plin<64>(s, r, epw, p_addr + 64);
+                    }
+                    tmem_wait_st();
+                    tc_fence_before();
+                    mbar_arrive(&p_full[sb]);
+                }
+                if (!ok) break;
+                // ---- epilogue: y = O / l + sigmoid(g) (m_intra + lam^(r+1) m_inter)
+                xl[half * 128 + r] = l;
+                if (!(ok = group_sync(sm_sync, sync_phase, abort, p.status))) break;
+                const float inv_l = 1.0f / (l + xl[(1 - half) * 128 + r]);
+                if (!(ok = warp_wait(o_full, tile & 1, abort, p.status))) break;
+                tc_fence_after();
+                float yv[32];
+                {
+                    uint32_t rr[32];
+                    tmem_ld32(tmem_addr(tb, lane_base, TM_O + 32 * half), rr);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) yv[c] = __uint_as_float(rr[c]) * inv_l;
+                    if (ti.l2) {
+                        uint32_t rx[32];
+                        tmem_ld32(tmem_addr(tb, lane_base, TM_MI + 32 * half), rr);
+                        tmem_ld32(tmem_addr(tb, lane_base, TM_MX + 32 * half), rx);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int c = 0; c < 32; ++c)
+                            yv[c] += gate * (__uint_as_float(rr[c]) + pw_r1 * __uint_as_float(rx[c]));
+                    }
+                }
+                tc_fence_before();
+                mbar_arrive(o_empty);
+                const int t = ti.t0 + r;
+                if (t < p.T) {
+                    uint4 *dst = reinterpret_cast<uint4 *>(reinterpret_cast<__nv_bfloat16 *>(p.y) +
+                                                           ((size_t)bh * p.T + t) * HD + 32 * half);
+#pragma unroll
+                    for (int c = 0; c < 4; ++c)
+                        dst[c] = make_uint4(pack_bf16(yv[8 * c], yv[8 * c + 1]),
+                                            pack_bf16(yv[8 * c + 2], yv[8 * c + 3]),
+                                            pack_bf16(yv[8 * c + 4], yv[8 * c + 5]),
+                                            pack_bf16(yv[8 * c + 6], yv[8 * c + 7]));
+                }
+            }
+        }
+    } else if (warp >= 12) {
+        // ------------------------------------------------------------ state
+        const int u = tid - 384;  // TMEM lane; u < 64 owns row u of S
+        uint32_t kc = 0, lc = 0, sync_phase = 0;
+        bool ok = true;
+        uint8_t *sb_tile = sm + OFF_SB;
+        uint8_t *kt_hi = sm + OFF_KT, *kt_lo = sm + OFF_KT + TILE_B;
+        float S[64];
+        for (int sp = blockIdx.x; sp < n_spans && ok; sp += gridDim.x) {
+            const int bh = sp / p.n_s, h = bh % p.H, js = sp % p.n_s;
+            int i0, i1;
+            span_range(js, p.nT, p.n_s, i0, i1);
+            const double lam = p.lam[h];
+            const double l2l = log2(lam);
+            const float eta = p.eta[h];
+            // state at the span start from the predecessors' summaries
+            const int n_start = max(0, i0 * BM - p.W);
+#pragma unroll
+            for (int c = 0; c < 64; ++c) S[c] = 0.f;
+            if (!l1_only && u < 64 && n_start > 0) {
+                for (int jj = 0; jj < js; ++jj) {
+                    int a0, a1;
+                    span_range(jj, p.nT, p.n_s, a0, a1);
+                    const int e_end = max(0, min(E, a1 * BM - p.W));
+                    if (e_end <= 0) continue;
+                    const float coef = (float)exp2((double)(n_start - e_end) * l2l);
+                    const float *src = p.dA + ((size_t)(bh * p.n_s + jj) * HD + u) * HD;
+#pragma unroll
+                    for (int c = 0; c < 64; ++c) S[c] = fmaf(coef, src[c], S[c]);
+                }
+            }
+            bool have_prev = false;
+            int c_prev = 0;
+            auto consume = [&](int c_eff) -> bool {
+                // rows 64..127 of the increment (lo parts) go through shared
+                // memory to the owners of rows 0..63 (hi parts)
+                if (!warp_wait(ds_full, (lc - 1) & 1, abort, p.status)) return false;
+                tc_fence_after();
+                uint32_t rr[32];
+                if (u >= 64) {
+#pragma unroll
+                    for (int c0 = 0; c0 < 64; c0 += 32) {
+                        tmem_ld32(tmem_addr(tb, 32 * (warp & 3), TM_DS + c0), rr);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int c = 0; c < 32; ++c) sDS[(c0 + c) * 64 + (u - 64)] = __uint_as_float(rr[c]);
+                    }
+                }
+                if (!group_sync(st_sync, sync_phase, abort, p.status)) return false;
+                if (u < 64) {
+                    const float dec = (float)exp2((double)c_eff * l2l);
+#pragma unroll
+                    for (int c0 = 0; c0 < 64; c0 += 32) {
+                        tmem_ld32(tmem_addr(tb, 32 * (warp & 3), TM_DS + c0), rr);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int c = 0; c < 32; ++c)
+                            S[c0 + c] = fmaf(dec, S[c0 + c],
+                                             __uint_as_float(rr[c]) + sDS[(c0 + c) * 64 + u]);
+                    }
+                }
+                return group_sync(st_sync, sync_phase, abort, p.status);
+            };
+            for (int i = i0; i < i1 && ok; ++i) {
+                const TileInfo ti = tile_info(i, p.W, l1_only);
+                if (ti.l2) {
+                    if (have_prev && !(ok = consume(c_prev))) break;
+                    // stage S(n0) as bf16 for the inter read (row k = u, 64 columns n)
+                    if (u < 64) {
+#pragma unroll
+                        for (int ch = 0; ch < 8; ++ch)
+                            *reinterpret_cast<uint4 *>(sb_tile + sw128_offset(u, ch * 8)) =
+                                make_uint4(pack_bf16(S[8 * ch], S[8 * ch + 1]),
+                                           pack_bf16(S[8 * ch + 2], S[8 * ch + 3]),
+                                           pack_bf16(S[8 * ch + 4], S[8 * ch + 5]),
+                                           pack_bf16(S[8 * ch + 6], S[8 * ch + 7]));
+                    }
+                    fence_async_smem();
+                    mbar_arrive(sst_full);
+                    // scaled keys of the leading tile for the state MMA
+                    const int s = kc % NS;
+                    if (!(ok = warp_wait(lead_ready, lc & 1, abort, p.status))) break;
+                    const int n0 = ti.t0 - p.W;
+                    const int c_eff = min(BM, E - n0);
+                    const float w =
+                        u < c_eff ? eta * (float)exp2((double)(c_eff - 1 - u) * l2l) : 0.f;
+                    build_scaled_key_row(sm + OFF_KV + s * 2 * TILE_B, kt_hi, kt_lo, u, w);
+                    fence_async_smem();
+                    mbar_arrive(kt_full);
+                    have_prev = true;
+                    c_prev = c_eff;
+                    ++lc;
+                }
+                kc += ti.nk;
+            }
+            if (!ok) break;
+            if (have_prev && !(ok = consume(c_prev))) break;
+            if (!l1_only && js == p.n_s - 1 && u < 64 && p.A_final) {
+                float4 *dst = reinterpret_cast<float4 *>(p.A_final + ((size_t)bh * HD + u) * HD);
+#pragma unroll
+                for (int c = 0; c < 16; ++c)
+                    dst[c] = make_float4(S[4 * c], S[4 * c + 1], S[4 * c + 2], S[4 * c + 3]);
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tb, 512);
+}
+
+// ---------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        cudaDriverEntryPointQueryResult q;
+        void *ptr = nullptr;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) !=
+                cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return nullptr;
+        fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    }
+    return fn;
+}
+
+// [BH][T][64] bf16 -> 3D map with 64 x 128 x 1 boxes, 128-byte swizzle;
+// rows past T read as zero.
+bool make_map(CUtensorMap *m, const void *base, int T, int BH) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[3] = {(cuuint64_t)HD, (cuuint64_t)T, (cuuint64_t)BH};
+    cuuint64_t strides[2] = {(cuuint64_t)HD * 2, (cuuint64_t)T * HD * 2};
+    cuuint32_t box[3] = {HD, BM, 1};
+    cuuint32_t es[3] = {1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides,
+              box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+           CUDA_SUCCESS;
+}
+
+// Spans per head: minimise the work of the busiest CTA, counting each span as
+// its tiles plus a fixed start-up cost (pipeline fill, the pre-pass summary it
+// needs and the combine of its predecessors' summaries); ties go to fewer spans.
+constexpr int kSpanOverheadTiles = 2;
+int choose_spans(int64_t BH, int nT, int num_sms) {
+    int best = 1;
+    int64_t best_cost = INT64_MAX;
+    for (int ns = 1; ns <= nT && ns <= 64; ++ns) {
+        const int64_t spans = BH * ns;
+        const int64_t G = spans < num_sms ? spans : num_sms;
+        const int64_t per_cta = (spans + G - 1) / G;
+        const int64_t cost = per_cta * ((nT + ns - 1) / ns + kSpanOverheadTiles);
+        if (cost < best_cost) {
+            best_cost = cost;
+            best = ns;
+        }
+    }
+    return best;
+}
+
+}  // namespace
 
 bool sm100_supported(const tc_prefill_desc &d) {
-    (void)d;
-    return false;
+    return d.dtype == TC_BF16 && d.dk == HD && d.dv == HD && d.W >= BM && d.W % BM == 0 &&
+           d.T >= 1 && d.T <= (int64_t(1) << 30) && d.B * d.H <= 65535;
+}
+
+static int spans_for(const tc_prefill_desc &d, int num_sms) {
+    const int nT = (int)((d.T + BM - 1) / BM);
+    return choose_spans(d.B * d.H, nT, num_sms);
 }
 
 size_t sm100_workspace_bytes(const tc_prefill_desc &d, int num_sms) {
-    (void)d;
-    (void)num_sms;
-    return 0;
+    if (d.flags & TC_PREFILL_L1_ONLY) return 0;
+    const int ns = spans_for(d, num_sms);
+    if (ns <= 1) return 0;
+    return (size_t)(d.B * d.H * ns) * HD * HD * sizeof(float);
 }
 
 int sm100_launch_count(const tc_prefill_desc &d) {
-    (void)d;
-    return 0;
+    const bool l1 = (d.flags & TC_PREFILL_L1_ONLY) != 0;
+    int sms = 148;
+    int dev = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess)
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    else
+        cudaGetLastError();
+    return 1 + ((!l1 && spans_for(d, sms) > 1) ? 1 : 0);
 }
 
 cudaError_t launch_prefill_sm100(const PrefillParams &p, int num_sms, cudaStream_t s) {
-    (void)p;
-    (void)num_sms;
-    (void)s;
-    return cudaErrorNotSupported;
+    const int64_t BH = p.B * p.H;
+    const int nT = (int)((p.T + BM - 1) / BM);
+    const int ns = choose_spans(BH, nT, num_sms);
+    CUtensorMap tq, tk, tv;
+    if (!make_map(&tq, p.q, (int)p.T, (int)BH) || !make_map(&tk, p.k, (int)p.T, (int)BH) ||
+        !make_map(&tv, p.v, (int)p.T, (int)BH))
+        return cudaErrorInvalidValue;
+    cudaError_t e = cudaFuncSetAttribute(prefill_main_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_MAIN);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(span_summary_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             SMEM_SUM);
+    if (e != cudaSuccess) return e;
+    float *dA = reinterpret_cast<float *>(p.workspace);
+    if (!p.l1_only && ns > 1) {
+        SumParams sp{dA, p.lam, p.eta, (int)p.T, (int)p.W, (int)p.H, (int)BH, nT, ns, p.status};
+        span_summary_kernel<<<(unsigned)(BH * (ns - 1)), 192, SMEM_SUM, s>>>(tk, tv, sp);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    MainParams mp{p.y, p.A_final, p.lam, p.eta, p.g, dA, (int)p.T, (int)p.W, (int)p.H, (int)BH,
+                  nT, ns, p.l1_only ? 1 : 0, p.status};
+    const int64_t spans = BH * ns;
+    const unsigned grid = (unsigned)(spans < num_sms ? spans : num_sms);
+    prefill_main_kernel<<<grid, kMainThreads, SMEM_MAIN, s>>>(tq, tk, tv, mp);
+    return cudaGetLastError();
 }
 
 }  // namespace tc
