@@ -139,6 +139,30 @@ TC_API tc_status tc_prefill_host(const tc_prefill_desc *desc, const void *q, con
                           void *y, float *A_final, void *workspace, size_t workspace_bytes,
                           tc_stream_t stream);
 
+/* Size of the scratch array compiled into the library for
+ * tc_prefill_no_alloc: 16 MiB per GPU that loads the library. */
+#define TC_NO_ALLOC_SCRATCH_BYTES (16u << 20)
+
+/* tc_prefill without a workspace, for callers that cannot allocate device
+ * memory (a host framework that owns every allocation, a real-time path that
+ * must not block in an allocator, a plugin with no allocator to call).  The
+ * paper has no counterpart: this is a deployment convenience of this library.
+ *
+ * Same arguments, results and errors as tc_prefill, except that the scratch
+ * space is a fixed array inside the library (TC_NO_ALLOC_SCRATCH_BYTES,
+ * resident on every GPU that loads the library until the process exits).
+ * Returns TC_ERR_WORKSPACE, enqueuing nothing, when desc would need more
+ * scratch than that (tc_prefill_workspace_size(desc) tells how much).
+ * The first call on each device looks up the array's device address with
+ * that device current; make that first call before any stream capture.
+ * All calls share the array and leave their data in it; no call depends on
+ * what an earlier one left, but calls whose kernels may overlap on the GPU
+ * (unordered streams) race on it and must not be issued that way.
+ * Allocates nothing: no cudaMalloc, cudaFree or allocating library call. */
+TC_API tc_status tc_prefill_no_alloc(const tc_prefill_desc *desc, const void *q, const void *k,
+                                     const void *v, const float *lambda, const float *eta,
+                                     const float *g, void *y, float *A_final, tc_stream_t stream);
+
 /* Streaming state of one layer: the L1 ring buffer, the L2 matrix and the
  * clock.  All arrays are caller-owned device memory, updated in place.
  *   ring_k [B,H,W,d_k], ring_v [B,H,W,d_v] in kv_dtype: slot s holds the

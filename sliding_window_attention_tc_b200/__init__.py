@@ -43,7 +43,8 @@ TC_PREFILL_L1_ONLY = 1
 # Exported C symbols declared in include/tc.h.
 EXPORTED = ("tc_prefill_workspace_size", "tc_prefill", "tc_prefill_launch_count", "tc_prefill_host_workspace_size",
             "tc_prefill_host", "tc_decode_step", "tc_decode_step_host_workspace_size",
-            "tc_decode_step_host", "tc_get_device_status", "tc_status_string", "tc_version")
+            "tc_decode_step_host", "tc_get_device_status", "tc_status_string", "tc_version",
+            "tc_prefill_no_alloc")
 
 
 class PrefillDesc(ctypes.Structure):
@@ -73,6 +74,8 @@ _lib.tc_prefill_host_workspace_size.argtypes = [_PD]
 _lib.tc_prefill_host_workspace_size.restype = _sz
 _lib.tc_prefill_host.argtypes = [_PD] + [_vp] * 9 + [_sz, _vp]
 _lib.tc_prefill_host.restype = _int
+_lib.tc_prefill_no_alloc.argtypes = [_PD] + [_vp] * 8 + [_vp]
+_lib.tc_prefill_no_alloc.restype = _int
 _lib.tc_decode_step.argtypes = [_DS] + [_vp] * 4 + [_vp]
 _lib.tc_decode_step.restype = _int
 _lib.tc_decode_step_host_workspace_size.argtypes = [_DS]
@@ -187,6 +190,28 @@ def prefill_launch_count(desc: PrefillDesc) -> int:
     if n < 0:
         raise TCError(1, "tc_prefill_launch_count")
     return int(n)
+
+
+NO_ALLOC_SCRATCH_BYTES = 16 << 20
+
+
+def prefill_no_alloc(q, k, v, lam, eta, g, W, C, *, l1_only=False, y=None, A_final=None,
+                     stream=None):
+    """tc_prefill_no_alloc: tc_prefill using the library's built-in scratch
+    array (no workspace argument) for callers that cannot allocate device
+    memory.  y / A_final are allocated here by PyTorch only when not given."""
+    desc = _desc_of(q, v, W, C, l1_only)
+    B, H, T, dk = q.shape
+    dv = v.shape[-1]
+    if y is None:
+        y = torch.empty((B, H, T, dv), dtype=q.dtype, device=q.device)
+    if A_final is None and not l1_only:
+        A_final = torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device)
+    _contig(q, k, v, lam, eta, g, y, A_final)
+    st = _lib.tc_prefill_no_alloc(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(lam),
+                                  _ptr(eta), _ptr(g), _ptr(y), _ptr(A_final), _stream(stream))
+    _check(st, "tc_prefill_no_alloc")
+    return y, A_final
 
 
 def prefill_host_workspace_size(desc: PrefillDesc) -> int:
