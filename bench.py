@@ -159,6 +159,34 @@ def _max_over_ranks(x: float, world: int, dev) -> float:
     return float(t.item())
 
 
+def timed_region(step, steps: int, world: int, dev) -> float:
+    """Run step(i) for i < steps between barriers; return the elapsed time in
+    ms, maximised over ranks.  On a CUDA device the time comes from CUDA
+    events on the current stream with a synchronize on both sides; on the
+    CPU (gloo ranks in tests) from a monotonic clock."""
+    cuda = torch.device(dev).type == "cuda"
+    if cuda:
+        stream = torch.cuda.current_stream()
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        _barrier(world)
+        torch.cuda.synchronize()
+        start.record(stream)
+        for i in range(steps):
+            step(i)
+        end.record(stream)
+        torch.cuda.synchronize()
+        _barrier(world)
+        ms = start.elapsed_time(end)
+    else:
+        _barrier(world)
+        t0 = time.perf_counter()
+        for i in range(steps):
+            step(i)
+        ms = (time.perf_counter() - t0) * 1e3
+        _barrier(world)
+    return _max_over_ranks(ms, world, dev)
+
+
 def _prefill_device_inputs(name, dev, copies):
     x = wl.prefill_config(name)
     sets = []

@@ -65,7 +65,8 @@ constexpr uint32_t OFF_DS = OFF_SB + 8192;             // float32 64x64 scratch
 constexpr uint32_t OFF_EPW = OFF_DS + 16384;           // [256]: eta lam^(i-128), 0 for i < 128
 constexpr uint32_t OFF_XM = OFF_EPW + 1024;            // [2 parity][2 halves][128] row maxima
 constexpr uint32_t OFF_XL = OFF_XM + 2048;             // [2 halves][128] row sums
-constexpr uint32_t OFF_BAR = OFF_XL + 1024;
+constexpr uint32_t OFF_STT = OFF_XL + 1024;            // state tables: eta lam^k, lam^k
+constexpr uint32_t OFF_BAR = OFF_STT + 1536;
 constexpr uint32_t SMEM_MAIN = OFF_BAR + 256 + 1024;
 
 // TMEM columns (512 allocated)
@@ -154,23 +155,32 @@ __device__ __forceinline__ TileInfo tile_info(int i, int W, bool l1_only) {
 //   LEAD_L2  ... plus the linear read eta lam^(r-c) <q,k> for c <= r (P')
 enum { KIND_FULL = 0, KIND_DIAG = 1, KIND_LEAD = 2, KIND_LEAD_L2 = 3 };
 
+// rc = r - cb: the row index relative to this half's first column cb, so a
+// local column c is global column cb + c.  One instance of each kind serves
+// both halves (smaller code, fewer instruction-cache misses).
 template <int KIND>
-__device__ __forceinline__ bool in_window(int c, int r) {
-    return KIND == KIND_FULL ? true : (KIND == KIND_DIAG ? c <= r : c > r);
+__device__ __forceinline__ bool in_window(int c, int rc) {
+    return KIND == KIND_FULL ? true : (KIND == KIND_DIAG ? c <= rc : c > rc);
 }
 
-// The 128 columns of a score tile are split between two softmax warpgroups:
-// half h owns columns 64h .. 64h+63 (CB = 64h) of every row.
+// x on window columns, -inf elsewhere, without predicate registers: the sign
+// of (rc - c) or (c - rc - 1) selects the bits of x or of -inf (one LOP3).
+template <int KIND>
+__device__ __forceinline__ float mask_window(float x, int c, int rc) {
+    if (KIND == KIND_FULL) return x;
+    const int d = KIND == KIND_DIAG ? rc - c : c - rc - 1;
+    const int m = d >> 31;  // 0 in the window, -1 outside
+    return __int_as_float((__float_as_int(x) & ~m) | (int(0xff800000u) & m));
+}
 
 // Row maximum of the raw scores over this half's window columns (-inf if none).
-template <int KIND, int CB>
-__device__ __forceinline__ float window_max(const float (&s)[64], int r) {
+template <int KIND>
+__device__ __forceinline__ float window_max(const float (&s)[64], int rc) {
     float m[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) m[i] = -INFINITY;
 #pragma unroll
-    for (int c = 0; c < 64; ++c)
-        m[c & 7] = fmaxf(m[c & 7], in_window<KIND>(CB + c, r) ? s[c] : -INFINITY);
+    for (int c = 0; c < 64; ++c) m[c & 7] = fmaxf(m[c & 7], in_window<KIND>(c, rc) ? s[c] : -INFINITY);
 #pragma unroll
     for (int i = 4; i >= 1; i >>= 1)
 #pragma unroll
@@ -180,9 +190,9 @@ __device__ __forceinline__ float window_max(const float (&s)[64], int r) {
 
 // P = exp2(s * sl2 - m) on window columns (0 elsewhere) as bf16 pairs into 32
 // TMEM columns starting at taddr; returns this half's row sum of P.
-template <int KIND, int CB>
-__device__ __forceinline__ float write_p(const float (&s)[64], int r, float sl2, float m,
-                                         uint32_t taddr) {
+template <int KIND>
+__device__ __forceinline__ float write_p(const float (&s)[64], int rc, float sl2, float m,
+                                      uint32_t taddr) {
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int c0 = 0; c0 < 64; c0 += 32) {
@@ -190,8 +200,8 @@ __device__ __forceinline__ float write_p(const float (&s)[64], int r, float sl2,
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
             const int c = c0 + 2 * e;
-            const float x0 = in_window<KIND>(CB + c, r) ? fmaf(s[c], sl2, -m) : -INFINITY;
-            const float x1 = in_window<KIND>(CB + c + 1, r) ? fmaf(s[c + 1], sl2, -m) : -INFINITY;
+            const float x0 = mask_window<KIND>(fmaf(s[c], sl2, -m), c, rc);
+            const float x1 = mask_window<KIND>(fmaf(s[c + 1], sl2, -m), c + 1, rc);
             const float p0 = ex2(x0), p1 = ex2(x1);
             acc[e & 3] += p0 + p1;
             pk[e] = pack_bf16(p0, p1);
@@ -203,10 +213,9 @@ __device__ __forceinline__ float write_p(const float (&s)[64], int r, float sl2,
 
 // P' = eta lam^(r-c) s for c <= r (the zero-padded table gives 0 for c > r)
 // as bf16 pairs into 32 TMEM columns starting at taddr.
-template <int CB>
-__device__ __forceinline__ void write_plin(const float (&s)[64], int r, const float *epw_pad,
-                                           uint32_t taddr) {
-    const float *w = epw_pad + 128 + r - CB;  // w[-c] = eta lam^(r-CB-c), or 0
+__device__ __forceinline__ void write_plin(const float (&s)[64], int rc, const float *epw_pad,
+                                        uint32_t taddr) {
+    const float *w = epw_pad + 128 + rc;  // w[-c] = eta lam^(rc-c), or 0 when c > rc
 #pragma unroll
     for (int c0 = 0; c0 < 64; c0 += 32) {
         uint32_t pk[16];
@@ -219,21 +228,42 @@ __device__ __forceinline__ void write_plin(const float (&s)[64], int r, const fl
     }
 }
 
-template <int CB>
-__device__ __forceinline__ float half_max(int kind, const float (&s)[64], int r) {
+// A masked kind reduces to FULL (every column inside) or to nothing (every
+// column outside) for the whole warp when all its rows agree; such warps skip
+// the per-column masks, and fully masked ones skip the exponentials.
+enum { SLICE_NONE = -1 };
+__device__ __forceinline__ int slice_kind(int kind, int rc) {
+    if (kind == KIND_FULL) return KIND_FULL;
+    const bool lead = kind != KIND_DIAG;
+    const bool all_in = lead ? (rc < 0) : (rc >= 63);
+    const bool all_out = lead ? (rc >= 63) : (rc < 0);
+    if (__all_sync(0xffffffffu, all_in)) return KIND_FULL;
+    if (__all_sync(0xffffffffu, all_out)) return SLICE_NONE;
+    return lead ? KIND_LEAD : KIND_DIAG;
+}
+
+__device__ __forceinline__ float half_max(int kind, const float (&s)[64], int rc) {
     switch (kind) {
-        case KIND_FULL: return window_max<KIND_FULL, CB>(s, r);
-        case KIND_DIAG: return window_max<KIND_DIAG, CB>(s, r);
-        default: return window_max<KIND_LEAD, CB>(s, r);
+        case SLICE_NONE: return -INFINITY;
+        case KIND_FULL: return window_max<KIND_FULL>(s, rc);
+        case KIND_DIAG: return window_max<KIND_DIAG>(s, rc);
+        default: return window_max<KIND_LEAD>(s, rc);
     }
 }
-template <int CB>
-__device__ __forceinline__ float half_p(int kind, const float (&s)[64], int r, float sl2, float m,
+__device__ __forceinline__ float half_p(int kind, const float (&s)[64], int rc, float sl2, float m,
                                         uint32_t taddr) {
     switch (kind) {
-        case KIND_FULL: return write_p<KIND_FULL, CB>(s, r, sl2, m, taddr);
-        case KIND_DIAG: return write_p<KIND_DIAG, CB>(s, r, sl2, m, taddr);
-        default: return write_p<KIND_LEAD, CB>(s, r, sl2, m, taddr);
+        case SLICE_NONE: {
+            uint32_t z[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) z[e] = 0u;
+            tmem_st16(taddr, z);
+            tmem_st16(taddr + 16, z);
+            return 0.f;
+        }
+        case KIND_FULL: return write_p<KIND_FULL>(s, rc, sl2, m, taddr);
+        case KIND_DIAG: return write_p<KIND_DIAG>(s, rc, sl2, m, taddr);
+        default: return write_p<KIND_LEAD>(s, rc, sl2, m, taddr);
     }
 }
 
@@ -512,6 +542,10 @@ __global__ void __launch_bounds__(kMainThreads, 1)
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
+        // One flat stream over the CTA's key tiles: Q K^T of key tile g is
+        // issued before P V of key tile g-1, also across query tiles, so the
+        // next tile's first scores are ready when the softmax side finishes
+        // the current tile.
         if (tid == 32) {
             const uint32_t id_qk = idesc_bf16(128, 128, false, false);
             const uint32_t id_pv = idesc_bf16(128, 64, false, true);
@@ -519,76 +553,82 @@ __global__ void __launch_bounds__(kMainThreads, 1)
             const uint32_t id_ds = idesc_bf16(128, 64, true, true);
             const uint32_t sb_addr = smem_u32(sm + OFF_SB);
             const uint32_t kt_addr = smem_u32(sm + OFF_KT);
-            uint32_t tile = 0, kc = 0, lc = 0;
+            const uint32_t q_base = smem_u32(sm + OFF_Q), kv_base = smem_u32(sm + OFF_KV);
+            uint32_t tile = 0, g = 0, lc = 0;
             bool ok = true;
+            // the key tile whose P V is still to be issued
+            struct Pending {
+                bool valid, first, last, l2;
+                uint32_t g, tile;
+            } pend = {false, false, false, false, 0, 0};
+            auto pv_step = [&](const Pending &pv) -> bool {
+                const int sb = pv.g & 1, s = pv.g % NS;
+                if (!mbar_wait(&p_full[sb], (pv.g >> 1) & 1, abort, p.status)) return false;
+                if (pv.first && !mbar_wait(o_empty, (pv.tile & 1) ^ 1, abort, p.status)) return false;
+                tc_fence_after();
+                const uint32_t v_addr = kv_base + s * 2 * TILE_B + TILE_B;
+                const uint32_t s_col = tb + TM_S + sb * 128;
+#pragma unroll
+                for (int k = 0; k < 8; ++k)
+                    mma_ts(tb + TM_O, s_col + 8 * k, sdesc_sw128(v_addr + 2048 * k, TILE_B, 1024),
+                           id_pv, (!pv.first || k > 0));
+                if (pv.first && pv.l2) {
+                    const uint32_t q_addr = q_base + (pv.tile & 1) * TILE_B;
+#pragma unroll
+                    for (int k = 0; k < 8; ++k)
+                        mma_ts(tb + TM_MI, s_col + 64 + 8 * k,
+                               sdesc_sw128(v_addr + 2048 * k, TILE_B, 1024), id_pv, k > 0);
+                    if (!mbar_wait(sst_full, lc & 1, abort, p.status)) return false;
+                    tc_fence_after();
+#pragma unroll
+                    for (int k = 0; k < 4; ++k)
+                        mma_ss(tb + TM_MX, sdesc_sw128(q_addr + 32 * k, 16, 1024),
+                               sdesc_sw128(sb_addr + 2048 * k, 8192, 1024), id_qs, k > 0);
+                    if (!mbar_wait(kt_full, lc & 1, abort, p.status)) return false;
+                    tc_fence_after();
+#pragma unroll
+                    for (int k = 0; k < 8; ++k)
+                        mma_ss(tb + TM_DS, sdesc_sw128(kt_addr + 2048 * k, TILE_B, 1024),
+                               sdesc_sw128(v_addr + 2048 * k, TILE_B, 1024), id_ds, k > 0);
+                    mma_commit(ds_full);
+                    ++lc;
+                }
+                mma_commit(&s_empty[sb]);
+                mma_commit(o_prog);
+                mma_commit(&kv_empty[s]);
+                if (pv.last) {
+                    mma_commit(&q_empty[pv.tile & 1]);
+                    mma_commit(o_full);
+                }
+                return true;
+            };
             for (int sp = blockIdx.x; sp < n_spans && ok; sp += gridDim.x) {
                 int i0, i1;
                 span_range(sp % p.n_s, p.nT, p.n_s, i0, i1);
                 for (int i = i0; i < i1 && ok; ++i, ++tile) {
                     const TileInfo ti = tile_info(i, p.W, l1_only);
                     const int qb = tile & 1;
-                    const uint32_t q_addr = smem_u32(sm + OFF_Q + qb * TILE_B);
+                    const uint32_t q_addr = q_base + qb * TILE_B;
                     if (!(ok = mbar_wait(&q_full[qb], (tile >> 1) & 1, abort, p.status))) break;
-                    const uint32_t kc0 = kc;
-                    auto pv_step = [&](int j) -> bool {
-                        const uint32_t g = kc0 + j;
-                        const int sb = g & 1, s = g % NS;
-                        if (!mbar_wait(&p_full[sb], (g >> 1) & 1, abort, p.status)) return false;
-                        if (j == 0 && !mbar_wait(o_empty, (tile & 1) ^ 1, abort, p.status)) return false;
-                        tc_fence_after();
-                        const uint32_t v_addr = smem_u32(sm + OFF_KV + s * 2 * TILE_B + TILE_B);
-                        const uint32_t s_col = tb + TM_S + sb * 128;
-#pragma unroll
-                        for (int k = 0; k < 8; ++k)
-                            mma_ts(tb + TM_O, s_col + 8 * k, sdesc_sw128(v_addr + 2048 * k, TILE_B, 1024),
-                                   id_pv, (j > 0 || k > 0));
-                        if (j == 0 && ti.l2) {
-#pragma unroll
-                            for (int k = 0; k < 8; ++k)
-                                mma_ts(tb + TM_MI, s_col + 64 + 8 * k,
-                                       sdesc_sw128(v_addr + 2048 * k, TILE_B, 1024), id_pv, k > 0);
-                            if (!mbar_wait(sst_full, lc & 1, abort, p.status)) return false;
-                            tc_fence_after();
-#pragma unroll
-                            for (int k = 0; k < 4; ++k)
-                                mma_ss(tb + TM_MX, sdesc_sw128(q_addr + 32 * k, 16, 1024),
-                                       sdesc_sw128(sb_addr + 2048 * k, 8192, 1024), id_qs, k > 0);
-                            if (!mbar_wait(kt_full, lc & 1, abort, p.status)) return false;
-                            tc_fence_after();
-#pragma unroll
-                            for (int k = 0; k < 8; ++k)
-                                mma_ss(tb + TM_DS, sdesc_sw128(kt_addr + 2048 * k, TILE_B, 1024),
-                                       sdesc_sw128(v_addr + 2048 * k, TILE_B, 1024), id_ds, k > 0);
-                            mma_commit(ds_full);
-                            ++lc;
-                        }
-                        mma_commit(&s_empty[sb]);
-                        mma_commit(o_prog);
-                        mma_commit(&kv_empty[s]);
-                        return true;
-                    };
-                    for (int j = 0; j < ti.nk && ok; ++j) {
-                        const uint32_t g = kc0 + j;
+                    for (int j = 0; j < ti.nk && ok; ++j, ++g) {
                         const int s = g % NS, sb = g & 1;
                         if (!(ok = mbar_wait(&kv_full[s], (g / NS) & 1, abort, p.status))) break;
                         // the state warps read the leading key tile: hand it on
                         if (j == 0 && ti.l2) mbar_arrive(lead_ready);
                         if (!(ok = mbar_wait(&s_empty[sb], ((g >> 1) & 1) ^ 1, abort, p.status))) break;
                         tc_fence_after();
-                        const uint32_t k_addr = smem_u32(sm + OFF_KV + s * 2 * TILE_B);
+                        const uint32_t k_addr = kv_base + s * 2 * TILE_B;
 #pragma unroll
                         for (int k = 0; k < 4; ++k)
                             mma_ss(tb + TM_S + sb * 128, sdesc_sw128(q_addr + 32 * k, 16, 1024),
                                    sdesc_sw128(k_addr + 32 * k, 16, 1024), id_qk, k > 0);
                         mma_commit(&s_full[sb]);
-                        if (j >= 1) ok = pv_step(j - 1);
+                        if (pend.valid && !(ok = pv_step(pend))) break;
+                        pend = {true, j == 0, j == ti.nk - 1, ti.l2, g, tile};
                     }
-                    if (ok) ok = pv_step(ti.nk - 1);
-                    mma_commit(&q_empty[qb]);
-                    mma_commit(o_full);
-                    kc = kc0 + ti.nk;
                 }
             }
+            if (ok && pend.valid) ok = pv_step(pend);
             // nothing may still run on the tensor cores when TMEM is released
             mma_commit(mma_done);
             mbar_wait_drain(mma_done, 0);
@@ -605,6 +645,51 @@ __global__ void __launch_bounds__(kMainThreads, 1)
         float *xl = reinterpret_cast<float *>(sm + OFF_XL);
         uint32_t tile = 0, kc = 0, sync_phase = 0;
         bool ok = true;
+        // The epilogue of a tile runs after the first key tile of the next one,
+        // so the wait for the tile's last P V product overlaps useful work.
+        struct Epi {
+            bool valid, l2;
+            int t0, bh;
+            float gate, pw_r1, l;
+            uint32_t tile;
+        } pe = {false, false, 0, 0, 0.f, 0.f, 0.f, 0};
+        auto epilogue = [&](const Epi &e) -> bool {
+            // y = O / l + sigmoid(g) (m_intra + lam^(r+1) m_inter)
+            xl[half * 128 + r] = e.l;
+            if (!group_sync(sm_sync, sync_phase, abort, p.status)) return false;
+            const float inv_l = 1.0f / (e.l + xl[(1 - half) * 128 + r]);
+            if (!warp_wait(o_full, e.tile & 1, abort, p.status)) return false;
+            tc_fence_after();
+            float yv[32];
+            uint32_t rr[32];
+            tmem_ld32(tmem_addr(tb, lane_base, TM_O + 32 * half), rr);
+            tmem_wait_ld();
+#pragma unroll
+            for (int c = 0; c < 32; ++c) yv[c] = __uint_as_float(rr[c]) * inv_l;
+            if (e.l2) {
+                uint32_t rx[32];
+                tmem_ld32(tmem_addr(tb, lane_base, TM_MI + 32 * half), rr);
+                tmem_ld32(tmem_addr(tb, lane_base, TM_MX + 32 * half), rx);
+                tmem_wait_ld();
+#pragma unroll
+                for (int c = 0; c < 32; ++c)
+                    yv[c] += e.gate * (__uint_as_float(rr[c]) + e.pw_r1 * __uint_as_float(rx[c]));
+            }
+            tc_fence_before();
+            mbar_arrive(o_empty);
+            const int t = e.t0 + r;
+            if (t < p.T) {
+                uint4 *dst = reinterpret_cast<uint4 *>(reinterpret_cast<__nv_bfloat16 *>(p.y) +
+                                                       ((size_t)e.bh * p.T + t) * HD + 32 * half);
+#pragma unroll
+                for (int c = 0; c < 4; ++c)
+                    dst[c] = make_uint4(pack_bf16(yv[8 * c], yv[8 * c + 1]),
+                                        pack_bf16(yv[8 * c + 2], yv[8 * c + 3]),
+                                        pack_bf16(yv[8 * c + 4], yv[8 * c + 5]),
+                                        pack_bf16(yv[8 * c + 6], yv[8 * c + 7]));
+            }
+            return true;
+        };
         for (int sp = blockIdx.x; sp < n_spans && ok; sp += gridDim.x) {
             const int bh = sp / p.n_s, h = bh % p.H;
             int i0, i1;
@@ -641,7 +726,8 @@ __global__ void __launch_bounds__(kMainThreads, 1)
                     }
                     const int kind = (j == 0 && ti.lead) ? (ti.l2 ? KIND_LEAD_L2 : KIND_LEAD)
                                                          : (j == ti.nk - 1 ? KIND_DIAG : KIND_FULL);
-                    const float mh = half == 0 ? half_max<0>(kind, s, r) : half_max<64>(kind, s, r);
+                    const int skind = slice_kind(kind, r - 64 * half);
+                    const float mh = half_max(skind, s, r - 64 * half);
                     float *xmk = xm + (kc & 1) * 256;
                     xmk[half * 128 + r] = mh;
                     if (!(ok = group_sync(sm_sync, sync_phase, abort, p.status))) break;
@@ -667,57 +753,22 @@ __global__ void __launch_bounds__(kMainThreads, 1)
                     l *= fo;
                     if (raise) m_used = mt;
                     const uint32_t p_addr = tmem_addr(tb, lane_base, s_col + 32 * half);
-                    l += half == 0 ? half_p<0>(kind, s, r, sl2, m_used, p_addr)
-                                   : half_p<64>(kind, s, r, sl2, m_used, p_addr);
-                    if (kind == KIND_LEAD_L2) {
-                        if (half == 0)
-                            write_plin<0>(s, r, epw, p_addr + 64);
-                        else
-                            write_plin<64>(s, r, epw, p_addr + 64);
-                    }
+                    l += half_p(skind, s, r - 64 * half, sl2, m_used, p_addr);
+                    if (kind == KIND_LEAD_L2) write_plin(s, r - 64 * half, epw, p_addr + 64);
                     tmem_wait_st();
                     tc_fence_before();
                     mbar_arrive(&p_full[sb]);
-                }
-                if (!ok) break;
-                // ---- epilogue: y = O / l + sigmoid(g) (m_intra + lam^(r+1) m_inter)
-                xl[half * 128 + r] = l;
-                if (!(ok = group_sync(sm_sync, sync_phase, abort, p.status))) break;
-                const float inv_l = 1.0f / (l + xl[(1 - half) * 128 + r]);
-                if (!(ok = warp_wait(o_full, tile & 1, abort, p.status))) break;
-                tc_fence_after();
-                float yv[32];
-                {
-                    uint32_t rr[32];
-                    tmem_ld32(tmem_addr(tb, lane_base, TM_O + 32 * half), rr);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int c = 0; c < 32; ++c) yv[c] = __uint_as_float(rr[c]) * inv_l;
-                    if (ti.l2) {
-                        uint32_t rx[32];
-                        tmem_ld32(tmem_addr(tb, lane_base, TM_MI + 32 * half), rr);
-                        tmem_ld32(tmem_addr(tb, lane_base, TM_MX + 32 * half), rx);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int c = 0; c < 32; ++c)
-                            yv[c] += gate * (__uint_as_float(rr[c]) + pw_r1 * __uint_as_float(rx[c]));
+                    if (j == 0 && pe.valid) {
+                        if (!(ok = epilogue(pe))) break;
+                        pe.valid = false;
                     }
                 }
-                tc_fence_before();
-                mbar_arrive(o_empty);
-                const int t = ti.t0 + r;
-                if (t < p.T) {
-                    uint4 *dst = reinterpret_cast<uint4 *>(reinterpret_cast<__nv_bfloat16 *>(p.y) +
-                                                           ((size_t)bh * p.T + t) * HD + 32 * half);
-#pragma unroll
-                    for (int c = 0; c < 4; ++c)
-                        dst[c] = make_uint4(pack_bf16(yv[8 * c], yv[8 * c + 1]),
-                                            pack_bf16(yv[8 * c + 2], yv[8 * c + 3]),
-                                            pack_bf16(yv[8 * c + 4], yv[8 * c + 5]),
-                                            pack_bf16(yv[8 * c + 6], yv[8 * c + 7]));
-                }
+                if (!ok) break;
+                pe = {true, ti.l2, ti.t0, bh, gate, pw_r1, l, tile};
             }
         }
+        if (ok && pe.valid) ok = epilogue(pe);
+
     } else if (warp >= 12) {
         // ------------------------------------------------------------ state
         const int u = tid - 384;  // TMEM lane; u < 64 owns row u of S
@@ -732,7 +783,13 @@ __global__ void __launch_bounds__(kMainThreads, 1)
             span_range(js, p.nT, p.n_s, i0, i1);
             const double lam = p.lam[h];
             const double l2l = log2(lam);
-            const float eta = p.eta[h];
+            // per-span tables (float math in the tile loop only): ew[k] = eta lam^k,
+            // lp[k] = lam^k; the previous span is done with them after its last consume
+            float *ew = reinterpret_cast<float *>(sm + OFF_STT), *lp = ew + 128;
+            ew[u] = (float)((double)p.eta[h] * exp2((double)u * l2l));
+            lp[u] = (float)exp2((double)u * l2l);
+            if (u == 0) lp[128] = (float)exp2(128.0 * l2l);
+            if (!(ok = group_sync(st_sync, sync_phase, abort, p.status))) break;
             // state at the span start from the predecessors' summaries
             const int n_start = max(0, i0 * BM - p.W);
 #pragma unroll
@@ -768,7 +825,7 @@ __global__ void __launch_bounds__(kMainThreads, 1)
                 }
                 if (!group_sync(st_sync, sync_phase, abort, p.status)) return false;
                 if (u < 64) {
-                    const float dec = (float)exp2((double)c_eff * l2l);
+                    const float dec = lp[c_eff];
 #pragma unroll
                     for (int c0 = 0; c0 < 64; c0 += 32) {
                         tmem_ld32(tmem_addr(tb, 32 * (warp & 3), TM_DS + c0), rr);
@@ -802,8 +859,7 @@ __global__ void __launch_bounds__(kMainThreads, 1)
                     if (!(ok = warp_wait(lead_ready, lc & 1, abort, p.status))) break;
                     const int n0 = ti.t0 - p.W;
                     const int c_eff = min(BM, E - n0);
-                    const float w =
-                        u < c_eff ? eta * (float)exp2((double)(c_eff - 1 - u) * l2l) : 0.f;
+                    const float w = u < c_eff ? ew[c_eff - 1 - u] : 0.f;
                     build_scaled_key_row(sm + OFF_KV + s * 2 * TILE_B, kt_hi, kt_lo, u, w);
                     fence_async_smem();
                     mbar_arrive(kt_full);
