@@ -63,16 +63,17 @@ constexpr uint32_t OFF_KT = OFF_KV + NS * 2 * TILE_B;  // scaled keys hi | lo
 constexpr uint32_t OFF_SB = OFF_KT + 2 * TILE_B;       // state bf16 [64 k][64 n]
 constexpr uint32_t OFF_DS = OFF_SB + 8192;             // float32 64x64 scratch
 constexpr uint32_t OFF_EPW = OFF_DS + 16384;           // [256]: eta lam^(i-128), 0 for i < 128
-constexpr uint32_t OFF_XM = OFF_EPW + 1024;            // [2 tile parity][2 halves][128] row maxima
-constexpr uint32_t OFF_XL = OFF_XM + 2048;             // [2 tile parity][2 halves][128] row sums
-constexpr uint32_t OFF_STT = OFF_XL + 2048;            // state tables: eta lam^k, lam^k
+constexpr uint32_t OFF_XM = OFF_EPW + 1024;            // [2 parity][2 halves][128] row maxima
+constexpr uint32_t OFF_XL = OFF_XM + 2048;             // [2 halves][128] row sums
+constexpr uint32_t OFF_STT = OFF_XL + 1024;            // state tables: eta lam^k, lam^k
 constexpr uint32_t OFF_BAR = OFF_STT + 1536;
 constexpr uint32_t SMEM_MAIN = OFF_BAR + 256 + 1024;
 
 // TMEM columns (512 allocated)
 constexpr uint32_t TM_S = 0;    // two 128-column score buffers (P / P' alias them)
-constexpr uint32_t TM_O = 256;  // O_0 | O_1: one 64-column accumulator per softmax half
-constexpr uint32_t TM_M = 384;  // memory read: intra-chunk P' V plus inter-chunk (lam^(r+1) q) S
+constexpr uint32_t TM_O = 256;  // O accumulator, 64 columns
+constexpr uint32_t TM_MI = 320; // intra-chunk memory read
+constexpr uint32_t TM_MX = 384; // inter-chunk memory read q S(n0)
 constexpr uint32_t TM_DS = 448; // state increment: rows 0-63 hi part, 64-127 lo part
 
 constexpr float kLog2e = 1.4426950408889634f;
@@ -154,30 +155,82 @@ __device__ __forceinline__ TileInfo tile_info(int i, int W, bool l1_only) {
 //   LEAD_L2  ... plus the linear read eta lam^(r-c) <q,k> for c <= r (P')
 enum { KIND_FULL = 0, KIND_DIAG = 1, KIND_LEAD = 2, KIND_LEAD_L2 = 3 };
 
-// Window test for one half (64 columns) of a score tile, as an affine
-// function of the column: column c (0..63 within the half) is in the window
-// iff  off + sgn * c >= 0.  rc = r - 64 h is the row relative to the half:
-//   FULL  sgn = 0,  off = 0       (every column)
-//   DIAG  sgn = -1, off = rc      (c <= rc: causal diagonal)
-//   LEAD  sgn = +1, off = -rc - 1 (c > rc: the evicted columns c <= rc are
-//                                  read linearly instead)
-// One code path serves every kind (small code, no predicate registers): the
-// sign of the affine value selects the score or -inf with one LOP3.
-struct WindowMask {
-    int sgn, off;
-};
-__device__ __forceinline__ WindowMask window_mask(int kind, int rc) {
-    if (kind == KIND_FULL) return {0, 0};
-    if (kind == KIND_DIAG) return {-1, rc};
-    return {1, -rc - 1};
+// rc = r - cb: the row index relative to this half's first column cb, so a
+// local column c is global column cb + c.  One instance of each kind serves
+// both halves (smaller code, fewer instruction-cache misses).
+template <int KIND>
+__device__ __forceinline__ bool in_window(int c, int rc) {
+    return KIND == KIND_FULL ? true : (KIND == KIND_DIAG ? c <= rc : c > rc);
 }
-__device__ __forceinline__ float masked(float x, WindowMask wm, int c) {
-    const int m = (wm.off + wm.sgn * c) >> 31;  // 0 in the window, -1 outside
+
+// x on window columns, -inf elsewhere, without predicate registers: the sign
+// of (rc - c) or (c - rc - 1) selects the bits of x or of -inf (one LOP3).
+template <int KIND>
+__device__ __forceinline__ float mask_window(float x, int c, int rc) {
+    if (KIND == KIND_FULL) return x;
+    const int d = KIND == KIND_DIAG ? rc - c : c - rc - 1;
+    const int m = d >> 31;  // 0 in the window, -1 outside
     return __int_as_float((__float_as_int(x) & ~m) | (int(0xff800000u) & m));
 }
 
-// Whole-warp shortcuts: every row of the warp has all (or none) of the half's
-// columns in the window.  SLICE_NONE skips the exponentials.
+// Row maximum of the raw scores over this half's window columns (-inf if none).
+template <int KIND>
+__device__ __forceinline__ float window_max(const float (&s)[64], int rc) {
+    float m[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) m[i] = -INFINITY;
+#pragma unroll
+    for (int c = 0; c < 64; ++c) m[c & 7] = fmaxf(m[c & 7], in_window<KIND>(c, rc) ? s[c] : -INFINITY);
+#pragma unroll
+    for (int i = 4; i >= 1; i >>= 1)
+#pragma unroll
+        for (int j = 0; j < i; ++j) m[j] = fmaxf(m[j], m[j + i]);
+    return m[0];
+}
+
+// P = exp2(s * sl2 - m) on window columns (0 elsewhere) as bf16 pairs into 32
+// TMEM columns starting at taddr; returns this half's row sum of P.
+template <int KIND>
+__device__ __forceinline__ float write_p(const float (&s)[64], int rc, float sl2, float m,
+                                      uint32_t taddr) {
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int c0 = 0; c0 < 64; c0 += 32) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+            const int c = c0 + 2 * e;
+            const float x0 = mask_window<KIND>(fmaf(s[c], sl2, -m), c, rc);
+            const float x1 = mask_window<KIND>(fmaf(s[c + 1], sl2, -m), c + 1, rc);
+            const float p0 = ex2(x0), p1 = ex2(x1);
+            acc[e & 3] += p0 + p1;
+            pk[e] = pack_bf16(p0, p1);
+        }
+        tmem_st16(taddr + c0 / 2, pk);
+    }
+    return (acc[0] + acc[1]) + (acc[2] + acc[3]);
+}
+
+// P' = eta lam^(r-c) s for c <= r (the zero-padded table gives 0 for c > r)
+// as bf16 pairs into 32 TMEM columns starting at taddr.
+__device__ __forceinline__ void write_plin(const float (&s)[64], int rc, const float *epw_pad,
+                                        uint32_t taddr) {
+    const float *w = epw_pad + 128 + rc;  // w[-c] = eta lam^(rc-c), or 0 when c > rc
+#pragma unroll
+    for (int c0 = 0; c0 < 64; c0 += 32) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+            const int c = c0 + 2 * e;
+            pk[e] = pack_bf16(s[c] * w[-c], s[c + 1] * w[-c - 1]);
+        }
+        tmem_st16(taddr + c0 / 2, pk);
+    }
+}
+
+// A masked kind reduces to FULL (every column inside) or to nothing (every
+// column outside) for the whole warp when all its rows agree; such warps skip
+// the per-column masks, and fully masked ones skip the exponentials.
 enum { SLICE_NONE = -1 };
 __device__ __forceinline__ int slice_kind(int kind, int rc) {
     if (kind == KIND_FULL) return KIND_FULL;
@@ -189,112 +242,36 @@ __device__ __forceinline__ int slice_kind(int kind, int rc) {
     return lead ? KIND_LEAD : KIND_DIAG;
 }
 
-// One pass over this half's two 32-column score chunks.  Each chunk is read
-// from TMEM and then overwritten in place by its results, packed as bf16
-// pairs: P = exp2(s * sl2 - m) on window columns (0 elsewhere; all 0 when
-// `none`) in the chunk's first 16 columns and, for a leading tile with the
-// memory path, P' = eta lam^(r-c) s on the evicted columns c <= r (0 for
-// c > r via the zero-padded table) in its last 16.  So half h's 64 columns
-// end up as [P cols 0-31 | P' 0-31 | P cols 32-63 | P' 32-63] of its keys.
-// The second chunk's load is in flight while the first is processed.
-// Returns this half's row sum of P.
-template <bool PLIN>
-__device__ __forceinline__ float half_softmax(uint32_t s_addr, WindowMask wm, bool none, float sl2,
-                                              float m, int rc, const float *epw_pad) {
-    const float *w = epw_pad + 128 + rc;  // w[-c] = eta lam^(rc-c), or 0 when c > rc
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-    uint32_t ra[32], rb[32];
-    tmem_ld32(s_addr, ra);
-    tmem_wait_ld();
-    tmem_ld32(s_addr + 32, rb);
-#pragma unroll
-    for (int chunk = 0; chunk < 2; ++chunk) {
-        uint32_t(&rr)[32] = chunk == 0 ? ra : rb;
-        const int c0 = 32 * chunk;
-        if (chunk == 1) tmem_wait_ld();
-        uint32_t pk[16];
-        if (none) {
-#pragma unroll
-            for (int e = 0; e < 16; ++e) pk[e] = 0u;
-        } else {
-#pragma unroll
-            for (int e = 0; e < 16; ++e) {
-                const int c = c0 + 2 * e;
-                // mask after the FMA: -inf even when m is still -inf
-                const float p0 = ex2(masked(fmaf(__uint_as_float(rr[2 * e]), sl2, -m), wm, c));
-                const float p1 = ex2(masked(fmaf(__uint_as_float(rr[2 * e + 1]), sl2, -m), wm, c + 1));
-                acc[e & 3] += p0 + p1;
-                pk[e] = pack_bf16_rna(p0, p1);
-            }
-        }
-        if (PLIN) {
-            uint32_t pl[16];
-#pragma unroll
-            for (int e = 0; e < 16; ++e) {
-                const int c = c0 + 2 * e;
-                pl[e] = pack_bf16_rna(__uint_as_float(rr[2 * e]) * w[-c],
-                                      __uint_as_float(rr[2 * e + 1]) * w[-c - 1]);
-            }
-            tmem_st16(s_addr + c0 + 16, pl);
-        }
-        tmem_st16(s_addr + c0, pk);
+__device__ __forceinline__ float half_max(int kind, const float (&s)[64], int rc) {
+    switch (kind) {
+        case SLICE_NONE: return -INFINITY;
+        case KIND_FULL: return window_max<KIND_FULL>(s, rc);
+        case KIND_DIAG: return window_max<KIND_DIAG>(s, rc);
+        default: return window_max<KIND_LEAD>(s, rc);
     }
-    return (acc[0] + acc[1]) + (acc[2] + acc[3]);
 }
-
-// P for this half against a given finite (possibly stale) reference m, kept
-// in registers: the scores stay in TMEM until the caller stores pk, so it can
-// still fall back to the max-first path.  Returns the row sum; *max_l2 gets the
-// row's window maximum in log2 units (max of s * sl2), -inf if none.
-__device__ __forceinline__ float half_p_regs(uint32_t s_addr, WindowMask wm, float sl2, float m,
-                                             uint32_t (&pk)[32], float *max_l2) {
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-    float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-    uint32_t ra[32], rb[32];
-    tmem_ld32(s_addr, ra);
-    tmem_ld32(s_addr + 32, rb);
-    tmem_wait_ld();
+__device__ __forceinline__ float half_p(int kind, const float (&s)[64], int rc, float sl2, float m,
+                                        uint32_t taddr) {
+    switch (kind) {
+        case SLICE_NONE: {
+            uint32_t z[16];
 #pragma unroll
-    for (int e = 0; e < 32; ++e) {
-        const int c = 2 * e;
-        const uint32_t u0 = c < 32 ? ra[c] : rb[c - 32], u1 = c < 32 ? ra[c + 1] : rb[c - 31];
-        const float x0 = masked(fmaf(__uint_as_float(u0), sl2, -m), wm, c);
-        const float x1 = masked(fmaf(__uint_as_float(u1), sl2, -m), wm, c + 1);
-        mx[e & 3] = fmaxf(mx[e & 3], fmaxf(x0, x1));
-        const float p0 = ex2(x0), p1 = ex2(x1);
-        acc[e & 3] += p0 + p1;
-        pk[e] = pack_bf16_rna(p0, p1);
+            for (int e = 0; e < 16; ++e) z[e] = 0u;
+            tmem_st16(taddr, z);
+            tmem_st16(taddr + 16, z);
+            return 0.f;
+        }
+        case KIND_FULL: return write_p<KIND_FULL>(s, rc, sl2, m, taddr);
+        case KIND_DIAG: return write_p<KIND_DIAG>(s, rc, sl2, m, taddr);
+        default: return write_p<KIND_LEAD>(s, rc, sl2, m, taddr);
     }
-    *max_l2 = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) + m;
-    return (acc[0] + acc[1]) + (acc[2] + acc[3]);
-}
-
-// Raw-score row maximum over this half's window columns (-inf if none).
-__device__ __forceinline__ float half_max(uint32_t s_addr, WindowMask wm) {
-    uint32_t ra[32], rb[32];
-    tmem_ld32(s_addr, ra);
-    tmem_ld32(s_addr + 32, rb);
-    tmem_wait_ld();
-    float m[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) m[i] = -INFINITY;
-#pragma unroll
-    for (int e = 0; e < 32; ++e) {
-        m[e & 7] = fmaxf(m[e & 7], masked(__uint_as_float(ra[e]), wm, e));
-        m[(e + 4) & 7] = fmaxf(m[(e + 4) & 7], masked(__uint_as_float(rb[e]), wm, 32 + e));
-    }
-#pragma unroll
-    for (int i = 4; i >= 1; i >>= 1)
-#pragma unroll
-        for (int j = 0; j < i; ++j) m[j] = fmaxf(m[j], m[j + i]);
-    return m[0];
 }
 
 // Scaled key row for the state MMA: row u of the key tile times w, split into
 // bf16 hi and lo = bf16(x - hi), written to two SWIZZLE_128B tiles.
 __device__ __forceinline__ void build_scaled_key_row(const uint8_t *ktile, uint8_t *hi_tile,
                                                      uint8_t *lo_tile, int u, float w) {
-#pragma unroll 1
+#pragma unroll
     for (int ch = 0; ch < 8; ++ch) {
         const uint32_t off = sw128_offset(u, ch * 8);
         const uint4 raw = *reinterpret_cast<const uint4 *>(ktile + off);
@@ -311,21 +288,6 @@ __device__ __forceinline__ void build_scaled_key_row(const uint8_t *ktile, uint8
         }
         *reinterpret_cast<uint4 *>(hi_tile + off) = make_uint4(h[0], h[1], h[2], h[3]);
         *reinterpret_cast<uint4 *>(lo_tile + off) = make_uint4(l[0], l[1], l[2], l[3]);
-    }
-}
-
-// Row u of a SWIZZLE_128B bf16 tile times w, rounded to bf16, into the same
-// position of another tile.
-__device__ __forceinline__ void scale_row(const uint8_t *src, uint8_t *dst, int u, float w) {
-#pragma unroll 1
-    for (int ch = 0; ch < 8; ++ch) {
-        const uint32_t off = sw128_offset(u, ch * 8);
-        const uint4 raw = *reinterpret_cast<const uint4 *>(src + off);
-        float f[8];
-        Vec16<__nv_bfloat16>::unpack(raw, f);
-        *reinterpret_cast<uint4 *>(dst + off) =
-            make_uint4(pack_bf16(f[0] * w, f[1] * w), pack_bf16(f[2] * w, f[3] * w),
-                       pack_bf16(f[4] * w, f[5] * w), pack_bf16(f[6] * w, f[7] * w));
     }
 }
 
@@ -553,25 +515,6 @@ __global__ void __launch_bounds__(kMainThreads, 1)
                 for (int i = i0; i < i1 && ok; ++i, ++tile) {
                     const TileInfo ti = tile_info(i, p.W, l1_only);
                     const int qb = tile & 1;
-                    // Each query tile brings one new K/V tile (its diagonal) and its Q
-                    // from HBM; the others were loaded by earlier tiles and sit in L2.
-                    // Start the HBM reads two tiles ahead.
-                    if (i + 2 < i1) {
-                        const int ta = (i + 2) * BM;
-                        tma_prefetch_l2_3d(&tq, 0, ta, bh);
-                        tma_prefetch_l2_3d(&tk, 0, ta, bh);
-                        tma_prefetch_l2_3d(&tv, 0, ta, bh);
-                    }
-                    if (i == i0) {  // first tile of a span: everything it reads is new
-                        for (int a = 0; a < 2 && i + a < i1; ++a) {
-                            const TileInfo ta = tile_info(i + a, p.W, l1_only);
-                            tma_prefetch_l2_3d(&tq, 0, ta.t0, bh);
-                            for (int j = 0; j < ta.nk; ++j) {
-                                tma_prefetch_l2_3d(&tk, 0, (ta.kt0 + j) * BM, bh);
-                                tma_prefetch_l2_3d(&tv, 0, (ta.kt0 + j) * BM, bh);
-                            }
-                        }
-                    }
                     if (!(ok = mbar_wait(&q_empty[qb], ((tile >> 1) & 1) ^ 1, abort, p.status))) break;
                     mbar_expect_tx(&q_full[qb], TILE_B);
                     tma_load_3d(sm + OFF_Q + qb * TILE_B, &tq, &q_full[qb], 0, ti.t0, bh);
@@ -610,7 +553,6 @@ __global__ void __launch_bounds__(kMainThreads, 1)
             const uint32_t id_ds = idesc_bf16(128, 64, true, true);
             const uint32_t sb_addr = smem_u32(sm + OFF_SB);
             const uint32_t kt_addr = smem_u32(sm + OFF_KT);
-            const uint32_t qs_addr = smem_u32(sm + OFF_DS);  // scaled Q (state warps)
             const uint32_t q_base = smem_u32(sm + OFF_Q), kv_base = smem_u32(sm + OFF_KV);
             uint32_t tile = 0, g = 0, lc = 0;
             bool ok = true;
@@ -619,36 +561,6 @@ __global__ void __launch_bounds__(kMainThreads, 1)
                 bool valid, first, last, l2;
                 uint32_t g, tile;
             } pend = {false, false, false, false, 0, 0};
-            // The two state MMAs of a tile (inter read Qs S(n0) into M, state
-            // increment into DS) wait for the state warps' operands; they are
-            // issued as soon as those are ready, tested without blocking at
-            // every key tile, and the leading K/V stage is held until then.
-            struct StateMma {
-                bool valid;
-                uint32_t stage;
-            } smma = {false, 0};
-            auto issue_state = [&](bool block) -> bool {
-                if (!smma.valid) return true;
-                if (!block && !(mbar_test_wait(sst_full, lc & 1) && mbar_test_wait(kt_full, lc & 1)))
-                    return true;
-                if (!mbar_wait(sst_full, lc & 1, abort, p.status)) return false;
-                if (!mbar_wait(kt_full, lc & 1, abort, p.status)) return false;
-                tc_fence_after();
-                const uint32_t v_addr = kv_base + smma.stage * 2 * TILE_B + TILE_B;
-#pragma unroll
-                for (int k = 0; k < 4; ++k)
-                    mma_ss(tb + TM_M, sdesc_sw128(qs_addr + 32 * k, 16, 1024),
-                           sdesc_sw128(sb_addr + 2048 * k, 8192, 1024), id_qs, 1);
-#pragma unroll
-                for (int k = 0; k < 8; ++k)
-                    mma_ss(tb + TM_DS, sdesc_sw128(kt_addr + 2048 * k, TILE_B, 1024),
-                           sdesc_sw128(v_addr + 2048 * k, TILE_B, 1024), id_ds, k > 0);
-                mma_commit(ds_full);
-                mma_commit(&kv_empty[smma.stage]);
-                ++lc;
-                smma.valid = false;
-                return true;
-            };
             auto pv_step = [&](const Pending &pv) -> bool {
                 const int sb = pv.g & 1, s = pv.g % NS;
                 if (!mbar_wait(&p_full[sb], (pv.g >> 1) & 1, abort, p.status)) return false;
@@ -656,32 +568,34 @@ __global__ void __launch_bounds__(kMainThreads, 1)
                 tc_fence_after();
                 const uint32_t v_addr = kv_base + s * 2 * TILE_B + TILE_B;
                 const uint32_t s_col = tb + TM_S + sb * 128;
-                // O_h += P_h V_h: half h holds keys 64h.. of the tile; its score
-                // columns 64h.. hold [P keys 0-31 | P' 0-31 | P 32-63 | P' 32-63]
 #pragma unroll
-                for (int hh = 0; hh < 2; ++hh)
+                for (int k = 0; k < 8; ++k)
+                    mma_ts(tb + TM_O, s_col + 8 * k, sdesc_sw128(v_addr + 2048 * k, TILE_B, 1024),
+                           id_pv, (!pv.first || k > 0));
+                if (pv.first && pv.l2) {
+                    const uint32_t q_addr = q_base + (pv.tile & 1) * TILE_B;
+#pragma unroll
+                    for (int k = 0; k < 8; ++k)
+                        mma_ts(tb + TM_MI, s_col + 64 + 8 * k,
+                               sdesc_sw128(v_addr + 2048 * k, TILE_B, 1024), id_pv, k > 0);
+                    if (!mbar_wait(sst_full, lc & 1, abort, p.status)) return false;
+                    tc_fence_after();
 #pragma unroll
                     for (int k = 0; k < 4; ++k)
-                        mma_ts(tb + TM_O + 64 * hh, s_col + 64 * hh + 32 * (k >> 1) + 8 * (k & 1),
-                               sdesc_sw128(v_addr + 8192 * hh + 2048 * k, TILE_B, 1024), id_pv,
-                               (!pv.first || k > 0));
-                const bool lead_l2 = pv.first && pv.l2;
-                if (lead_l2) {
-                    // m = P' V (intra-chunk) now; + Qs S(n0) with Qs = diag(lam^(r+1)) Q
-                    // when the state warps are ready (issue_state)
+                        mma_ss(tb + TM_MX, sdesc_sw128(q_addr + 32 * k, 16, 1024),
+                               sdesc_sw128(sb_addr + 2048 * k, 8192, 1024), id_qs, k > 0);
+                    if (!mbar_wait(kt_full, lc & 1, abort, p.status)) return false;
+                    tc_fence_after();
 #pragma unroll
-                    for (int hh = 0; hh < 2; ++hh)
-#pragma unroll
-                        for (int k = 0; k < 4; ++k)
-                            mma_ts(tb + TM_M, s_col + 64 * hh + 32 * (k >> 1) + 16 + 8 * (k & 1),
-                                   sdesc_sw128(v_addr + 8192 * hh + 2048 * k, TILE_B, 1024), id_pv,
-                                   (hh > 0 || k > 0));
-                    smma = {true, (uint32_t)s};
+                    for (int k = 0; k < 8; ++k)
+                        mma_ss(tb + TM_DS, sdesc_sw128(kt_addr + 2048 * k, TILE_B, 1024),
+                               sdesc_sw128(v_addr + 2048 * k, TILE_B, 1024), id_ds, k > 0);
+                    mma_commit(ds_full);
+                    ++lc;
                 }
                 mma_commit(&s_empty[sb]);
                 mma_commit(o_prog);
-                if (!lead_l2) mma_commit(&kv_empty[s]);
-                if (!issue_state(pv.last)) return false;
+                mma_commit(&kv_empty[s]);
                 if (pv.last) {
                     mma_commit(&q_empty[pv.tile & 1]);
                     mma_commit(o_full);
@@ -698,9 +612,6 @@ __global__ void __launch_bounds__(kMainThreads, 1)
                     if (!(ok = mbar_wait(&q_full[qb], (tile >> 1) & 1, abort, p.status))) break;
                     for (int j = 0; j < ti.nk && ok; ++j, ++g) {
                         const int s = g % NS, sb = g & 1;
-                        // stage s may be the held leading stage: the producer refills
-                        // it only after the state MMAs are issued
-                        if (smma.valid && smma.stage == (uint32_t)s && !(ok = issue_state(true))) break;
                         if (!(ok = mbar_wait(&kv_full[s], (g / NS) & 1, abort, p.status))) break;
                         // the state warps read the leading key tile: hand it on
                         if (j == 0 && ti.l2) mbar_arrive(lead_ready);
@@ -712,7 +623,6 @@ __global__ void __launch_bounds__(kMainThreads, 1)
                             mma_ss(tb + TM_S + sb * 128, sdesc_sw128(q_addr + 32 * k, 16, 1024),
                                    sdesc_sw128(k_addr + 32 * k, 16, 1024), id_qk, k > 0);
                         mma_commit(&s_full[sb]);
-                        if (!(ok = issue_state(false))) break;
                         if (pend.valid && !(ok = pv_step(pend))) break;
                         pend = {true, j == 0, j == ti.nk - 1, ti.l2, g, tile};
                     }
@@ -740,40 +650,30 @@ __global__ void __launch_bounds__(kMainThreads, 1)
         struct Epi {
             bool valid, l2;
             int t0, bh;
-            float gate, m, l;
+            float gate, pw_r1, l;
             uint32_t tile;
         } pe = {false, false, 0, 0, 0.f, 0.f, 0.f, 0};
         auto epilogue = [&](const Epi &e) -> bool {
-            // the two halves kept separate running maxima and sums: combine
-            //   y = (O_0 2^(m_0-m) + O_1 2^(m_1-m)) / (l_0 2^(m_0-m) + l_1 2^(m_1-m))
-            //       + sigmoid(g) M
-            // double-buffered by tile parity: a half can be one epilogue ahead
-            float *xmt = xm + (e.tile & 1) * 256, *xlt = xl + (e.tile & 1) * 256;
-            xmt[half * 128 + r] = e.m;
-            xlt[half * 128 + r] = e.l;
+            // y = O / l + sigmoid(g) (m_intra + lam^(r+1) m_inter)
+            xl[half * 128 + r] = e.l;
             if (!group_sync(sm_sync, sync_phase, abort, p.status)) return false;
-            const float m0 = xmt[r], m1 = xmt[128 + r];
-            const float mm = fmaxf(m0, m1);
-            const float f0 = ex2(m0 - mm), f1 = ex2(m1 - mm);
-            const float inv_l = 1.0f / (xlt[r] * f0 + xlt[128 + r] * f1);
+            const float inv_l = 1.0f / (e.l + xl[(1 - half) * 128 + r]);
             if (!warp_wait(o_full, e.tile & 1, abort, p.status)) return false;
             tc_fence_after();
             float yv[32];
-            uint32_t ra[32];
-            const float g0 = f0 * inv_l, g1 = f1 * inv_l;
-            tmem_ld32(tmem_addr(tb, lane_base, TM_O + 32 * half), ra);
+            uint32_t rr[32];
+            tmem_ld32(tmem_addr(tb, lane_base, TM_O + 32 * half), rr);
             tmem_wait_ld();
 #pragma unroll
-            for (int c = 0; c < 32; ++c) yv[c] = __uint_as_float(ra[c]) * g0;
-            tmem_ld32(tmem_addr(tb, lane_base, TM_O + 64 + 32 * half), ra);
-            tmem_wait_ld();
-#pragma unroll
-            for (int c = 0; c < 32; ++c) yv[c] = fmaf(__uint_as_float(ra[c]), g1, yv[c]);
+            for (int c = 0; c < 32; ++c) yv[c] = __uint_as_float(rr[c]) * inv_l;
             if (e.l2) {
-                tmem_ld32(tmem_addr(tb, lane_base, TM_M + 32 * half), ra);
+                uint32_t rx[32];
+                tmem_ld32(tmem_addr(tb, lane_base, TM_MI + 32 * half), rr);
+                tmem_ld32(tmem_addr(tb, lane_base, TM_MX + 32 * half), rx);
                 tmem_wait_ld();
 #pragma unroll
-                for (int c = 0; c < 32; ++c) yv[c] = fmaf(e.gate, __uint_as_float(ra[c]), yv[c]);
+                for (int c = 0; c < 32; ++c)
+                    yv[c] += e.gate * (__uint_as_float(rr[c]) + e.pw_r1 * __uint_as_float(rx[c]));
             }
             tc_fence_before();
             mbar_arrive(o_empty);
@@ -796,6 +696,7 @@ __global__ void __launch_bounds__(kMainThreads, 1)
             span_range(sp % p.n_s, p.nT, p.n_s, i0, i1);
             const double lam = p.lam[h];
             const float gate = 1.0f / (1.0f + expf(-p.g[h]));
+            const float pw_r1 = (float)pow(lam, (double)(r + 1));
             // previous span done with epw, then publish this head's table
             if (!(ok = group_sync(sm_sync, sync_phase, abort, p.status))) break;
             if (half == 0)
@@ -811,62 +712,49 @@ __global__ void __launch_bounds__(kMainThreads, 1)
                     if (!(ok = warp_wait(&s_full[sb], (kc >> 1) & 1, abort, p.status))) break;
                     tc_fence_after();
                     const uint32_t s_col = TM_S + sb * 128;
-                    const uint32_t s_addr = tmem_addr(tb, lane_base, s_col + 64 * half);
+                    float s[64];
+                    {
+                        uint32_t ra[32], rb[32];
+                        tmem_ld32(tmem_addr(tb, lane_base, s_col + 64 * half), ra);
+                        tmem_ld32(tmem_addr(tb, lane_base, s_col + 64 * half + 32), rb);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int c = 0; c < 32; ++c) {
+                            s[c] = __uint_as_float(ra[c]);
+                            s[32 + c] = __uint_as_float(rb[c]);
+                        }
+                    }
                     const int kind = (j == 0 && ti.lead) ? (ti.l2 ? KIND_LEAD_L2 : KIND_LEAD)
                                                          : (j == ti.nk - 1 ? KIND_DIAG : KIND_FULL);
-                    const int rc = r - 64 * half;
-                    const int skind = slice_kind(kind, rc);
-                    const WindowMask wm = window_mask(skind, rc);
-                    const bool none = skind == SLICE_NONE;
-                    // The reference max m_used (log2 units) rises only when a row's
-                    // maximum grows by more than 2^kRescale; rows whose O_h already
-                    // holds earlier P V products are then rescaled in TMEM.  When
-                    // every row of the warp has a reference, P is computed in one
-                    // pass against it and the pass is redone in the rare case that
-                    // the tile raised it; otherwise the maximum is taken first.
-                    // TMEM access is warp-collective, so these choices are made per
-                    // warp (factor 1 for rows that need no rescale).
-                    const float l_in = l;
-                    float mt = -INFINITY, fo = 1.0f;
-                    bool pass_done = false;
-                    // (a leading tile is always key tile 0, where m_used is -inf)
-                    if (!none && !__any_sync(0xffffffffu, m_used == -INFINITY)) {
-                        uint32_t pk[32];
-                        const float lp = half_p_regs(s_addr, wm, sl2, m_used, pk, &mt);
-                        pass_done = !__any_sync(0xffffffffu, mt > m_used + kRescale);
-                        if (pass_done) {
-                            l = l_in + lp;
-                            tmem_st16(s_addr, *reinterpret_cast<uint32_t(*)[16]>(&pk[0]));
-                            tmem_st16(s_addr + 32, *reinterpret_cast<uint32_t(*)[16]>(&pk[16]));
-                        }
-                    }
-                    if (!pass_done && !none) mt = half_max(s_addr, wm) * sl2;
-                    if (!pass_done) {
-                        const bool raise = mt > m_used + kRescale;
-                        const bool resc = raise && m_used != -INFINITY && j > 0;
-                        fo = resc ? ex2(m_used - mt) : 1.0f;
-                        if (__any_sync(0xffffffffu, resc)) {
-                            if (!(ok = warp_wait(o_prog, (kc - 1) & 1, abort, p.status))) break;
-                            tc_fence_after();
-#pragma unroll 1
-                            for (int c0 = 0; c0 < 64; c0 += 32) {
-                                uint32_t rr[32];
-                                tmem_ld32(tmem_addr(tb, lane_base, TM_O + 64 * half + c0), rr);
-                                tmem_wait_ld();
+                    const int skind = slice_kind(kind, r - 64 * half);
+                    const float mh = half_max(skind, s, r - 64 * half);
+                    float *xmk = xm + (kc & 1) * 256;
+                    xmk[half * 128 + r] = mh;
+                    if (!(ok = group_sync(sm_sync, sync_phase, abort, p.status))) break;
+                    const float mt = fmaxf(mh, xmk[(1 - half) * 128 + r]) * sl2;  // sl2 > 0
+                    // Raise the row's reference max only when it grew by more than
+                    // 2^kRescale; rows whose O already holds earlier P V products
+                    // are rescaled in TMEM (each half its 32 columns of O).  TMEM
+                    // access is warp-collective, so the warp rescales together.
+                    const bool raise = mt > m_used + kRescale;
+                    const bool resc = raise && m_used != -INFINITY && j > 0;
+                    const float fo = resc ? ex2(m_used - mt) : 1.0f;
+                    if (__any_sync(0xffffffffu, resc)) {
+                        if (!(ok = warp_wait(o_prog, (kc - 1) & 1, abort, p.status))) break;
+                        tc_fence_after();
+                        uint32_t rr[32];
+                        tmem_ld32(tmem_addr(tb, lane_base, TM_O + 32 * half), rr);
+                        tmem_wait_ld();
 #pragma unroll
-                                for (int c = 0; c < 32; ++c)
-                                    rr[c] = __float_as_uint(__uint_as_float(rr[c]) * fo);
-                                tmem_st32(tmem_addr(tb, lane_base, TM_O + 64 * half + c0), rr);
-                            }
-                        }
-                        if (raise) m_used = mt;
-                        // P_h and P'_h overwrite this half's own 64 score columns only
-                        // (the other half may still be reading its scores)
-                        const float lp = kind == KIND_LEAD_L2
-                                             ? half_softmax<true>(s_addr, wm, none, sl2, m_used, rc, epw)
-                                             : half_softmax<false>(s_addr, wm, none, sl2, m_used, rc, epw);
-                        l = l_in * fo + lp;
+                        for (int c = 0; c < 32; ++c)
+                            rr[c] = __float_as_uint(__uint_as_float(rr[c]) * fo);
+                        tmem_st32(tmem_addr(tb, lane_base, TM_O + 32 * half), rr);
                     }
+                    l *= fo;
+                    if (raise) m_used = mt;
+                    const uint32_t p_addr = tmem_addr(tb, lane_base, s_col + 32 * half);
+                    l += half_p(skind, s, r - 64 * half, sl2, m_used, p_addr);
+                    if (kind == KIND_LEAD_L2) write_plin(s, r - 64 * half, epw, p_addr + 64);
                     tmem_wait_st();
                     tc_fence_before();
                     mbar_arrive(&p_full[sb]);
@@ -876,7 +764,7 @@ __global__ void __launch_bounds__(kMainThreads, 1)
                     }
                 }
                 if (!ok) break;
-                pe = {true, ti.l2, ti.t0, bh, gate, m_used, l, tile};
+                pe = {true, ti.l2, ti.t0, bh, gate, pw_r1, l, tile};
             }
         }
         if (ok && pe.valid) ok = epilogue(pe);
@@ -884,7 +772,7 @@ __global__ void __launch_bounds__(kMainThreads, 1)
     } else if (warp >= 12) {
         // ------------------------------------------------------------ state
         const int u = tid - 384;  // TMEM lane; u < 64 owns row u of S
-        uint32_t kc = 0, lc = 0, tile = 0, sync_phase = 0;
+        uint32_t kc = 0, lc = 0, sync_phase = 0;
         bool ok = true;
         uint8_t *sb_tile = sm + OFF_SB;
         uint8_t *kt_hi = sm + OFF_KT, *kt_lo = sm + OFF_KT + TILE_B;
@@ -973,8 +861,6 @@ __global__ void __launch_bounds__(kMainThreads, 1)
                     const int c_eff = min(BM, E - n0);
                     const float w = u < c_eff ? ew[c_eff - 1 - u] : 0.f;
                     build_scaled_key_row(sm + OFF_KV + s * 2 * TILE_B, kt_hi, kt_lo, u, w);
-                    // Qs = diag(lam^(r+1)) Q for the inter-chunk read (row r = u)
-                    scale_row(sm + OFF_Q + (tile & 1) * TILE_B, sm + OFF_DS, u, lp[u + 1]);
                     fence_async_smem();
                     mbar_arrive(kt_full);
                     have_prev = true;
@@ -982,7 +868,6 @@ __global__ void __launch_bounds__(kMainThreads, 1)
                     ++lc;
                 }
                 kc += ti.nk;
-                ++tile;
             }
             if (!ok) break;
             if (have_prev && !(ok = consume(c_prev))) break;

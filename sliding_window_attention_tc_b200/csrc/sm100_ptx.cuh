@@ -46,28 +46,11 @@ __device__ __forceinline__ void mbar_expect_tx(uint64_t *bar, uint32_t bytes) {
                  "r"(bytes)
                  : "memory");
 }
-// One try_wait: the thread sleeps until the phase completes or about
-// kSuspendHintNs passes (then the caller re-checks its abort flag and clock),
-// so waiting warps do not spin on the issue slots.
-constexpr uint32_t kSuspendHintNs = 1000000;
 __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity), "r"(kSuspendHintNs)
-        : "memory");
-    return ok != 0;
-}
-
-// Non-blocking test of a phase (no suspend).
-__device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
         : "r"(smem_u32(bar)), "r"(parity)
@@ -85,7 +68,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
     const uint64_t t0 = globaltimer();
     for (uint32_t i = 1;; ++i) {
         if (mbar_try_wait(bar, parity)) return true;
-        if ((i & 3u) == 0) {
+        if ((i & 255u) == 0) {
             if (*abort) return false;
             if (globaltimer() - t0 > kWaitTimeoutNs) {
                 *abort = 1;
@@ -104,7 +87,7 @@ __device__ __forceinline__ void mbar_wait_drain(uint64_t *bar, uint32_t parity) 
     const uint64_t t0 = globaltimer();
     for (uint32_t i = 1;; ++i) {
         if (mbar_try_wait(bar, parity)) return;
-        if ((i & 3u) == 0 && globaltimer() - t0 > kWaitTimeoutNs) return;
+        if ((i & 255u) == 0 && globaltimer() - t0 > kWaitTimeoutNs) return;
     }
 }
 
@@ -115,14 +98,6 @@ __device__ __forceinline__ void tma_load_3d(void *dst, const void *tmap, uint64_
         "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
         "[%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(dst)),
         "l"(reinterpret_cast<uint64_t>(tmap)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2)
-        : "memory");
-}
-// Bring one tile into L2 ahead of its TMA load (no shared memory, no barrier).
-__device__ __forceinline__ void tma_prefetch_l2_3d(const void *tmap, int c0, int c1, int c2) {
-    asm volatile(
-        "cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(
-            reinterpret_cast<uint64_t>(tmap)),
-        "r"(c0), "r"(c1), "r"(c2)
         : "memory");
 }
 __device__ __forceinline__ void tma_prefetch_desc(const void *tmap) {
@@ -252,13 +227,6 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     uint32_t r;
     asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
     return r;
-}
-
-// Two finite floats -> bf16x2 (lo in the low half), rounded to nearest with
-// ties away from zero, using integer operations only (keeps the XU pipe free
-// for the exponentials).
-__device__ __forceinline__ uint32_t pack_bf16_rna(float lo, float hi) {
-    return __byte_perm(__float_as_uint(lo) + 0x8000u, __float_as_uint(hi) + 0x8000u, 0x7632);
 }
 
 // Byte offset of element (row, col) in a SWIZZLE_128B tile of 64-element
