@@ -40,6 +40,13 @@ sys.path.insert(0, ROOT)
 import workloads as wl  # noqa: E402
 
 HEADLINE = "lm_prefill_bf16"
+
+# DRAM bytes (read + write) per launch from one ncu capture of the current
+# kernels; they must be re-measured (or set to None) whenever a kernel changes.
+#   prefill_main_kernel, LM workload: profiles/prefill_main_kernel_lm_prefill_bf16.md
+#   decode_kernel, 256 x 32 heads (captured at 32 x 32, scaled by heads):
+#     profiles/decode_kernel_b32_w2048_d128.md
+NCU_TRAFFIC_BYTES = {"prefill_main_kernel": 192.0e6, "decode_kernel": 9.28e9}
 METRIC = "prefill tokens/s & decode tok/s per B200; % of TC/HBM roofline"
 UNIT = "tokens/s"
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -481,7 +488,9 @@ def main():
         achieved_tflops = (l1f + l2f) / (mean_ms * 1e-3) / 1e12
         peak_tf = float(peaks["bf16_tflops"])
         roofline = {"bound": "tensor", "achieved": achieved_tflops, "peak": peak_tf,
-                    "unit": "TFLOP/s", "frac": achieved_tflops / peak_tf, "traffic": None,
+                    "unit": "TFLOP/s", "frac": achieved_tflops / peak_tf,
+                    "traffic": NCU_TRAFFIC_BYTES["prefill_main_kernel"],
+                    "traffic_kernel": "prefill_main_kernel (ncu, one launch)",
                     "peak_source": f"{peak_src} bf16 burst",
                     "kernel": "tc_prefill (all launches of one call)",
                     "algorithmic_flops_per_launch": l1f + l2f}
@@ -519,7 +528,7 @@ def main():
                 "tokens_per_s": dec["B"] / (dms * 1e-3),
                 "roofline": {"bound": "hbm", "achieved": gbs, "peak": float(peaks["hbm_gbs"]),
                              "unit": "GB/s", "frac": gbs / float(peaks["hbm_gbs"]),
-                             "traffic": None, "peak_source": f"{peak_src} copy bandwidth",
+                             "traffic": NCU_TRAFFIC_BYTES["decode_kernel"], "peak_source": f"{peak_src} copy bandwidth",
                              "algorithmic_bytes_per_launch": dec["bytes_per_step"]},
                 "e2e": {"ms_per_step": dec["e2e_ms_per_step"],
                         "tokens_per_s": dec["B"] / (dec["e2e_ms_per_step"] * 1e-3),
