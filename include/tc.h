@@ -74,8 +74,12 @@ typedef enum tc_dtype {
 } tc_dtype;
 
 /* tc_prefill_desc.flags */
-#define TC_PREFILL_L1_ONLY 1u /* skip L2 entirely: y = y_local (sigmoid(g) = 0
-                                 taken literally, no A work); A_final unused */
+#define TC_PREFILL_L1_ONLY 1u    /* skip L2 entirely: y = y_local (sigmoid(g) = 0
+                                    taken literally, no A work); A_final unused */
+#define TC_PREFILL_STATE_ONLY 2u /* L2 write path alone: only A_final is
+                                    computed (the chunk scan over the call's
+                                    evictions); q and y are not used and may be
+                                    NULL.  Not combinable with L1_ONLY. */
 
 /* Shapes of one prefill call.  Supported: B, H >= 1; T >= 0; 1 <= d_k, d_v
  * <= 128; W >= 1; C >= 1. */
@@ -117,6 +121,52 @@ TC_API size_t tc_prefill_workspace_size(const tc_prefill_desc *desc);
 TC_API tc_status tc_prefill(const tc_prefill_desc *desc, const void *q, const void *k, const void *v,
                      const float *lambda, const float *eta, const float *g, void *y,
                      float *A_final, void *workspace, size_t workspace_bytes, tc_stream_t stream);
+
+/* Continuation of a sequence: the same layer over desc->T new tokens that
+ * start at global position t0 >= 0, given what the tokens before t0 left
+ * behind.  It serves chunked prefill, a prefill that resumes after decode
+ * steps, and sequence sharding across GPUs (each rank continues from the
+ * previous ranks' tokens).  The paper defines the layer token by token (Fig. 2:
+ * evict, write A, insert, read); this entry point computes exactly what that
+ * loop computes for tokens t0 .. t0+T-1 when started from:
+ *
+ *   halo_k, halo_v  [B,H,n,d_k] / [B,H,n,d_v], dtype of desc, device: the keys
+ *                   and values of tokens t0-n .. t0-1, oldest first, where
+ *                   n = min(t0, W) (the window content at t0).  NULL allowed
+ *                   when n = 0.
+ *   A_init          [B,H,d_k,d_v] float32 device: A after every eviction before
+ *                   t0 (evictions e < t0 - W).  NULL means A = 0.
+ *
+ * q, k, v, y are the new tokens' rows [B,H,T,d].  A_final is A after the
+ * last eviction of the call.  With TC_PREFILL_STATE_ONLY only A_final is
+ * computed.  The tensor-core path takes bf16, d_k = d_v = 64, W a multiple of
+ * 128 and t0 = 0 or t0 >= W; other calls run on the portable float32 path.
+ * Workspace: tc_prefill_from_state_workspace_size(desc, t0) bytes.  Errors
+ * as tc_prefill, plus TC_ERR_INVALID_ARG for t0 < 0 or a missing halo. */
+TC_API size_t tc_prefill_from_state_workspace_size(const tc_prefill_desc *desc, int64_t t0);
+TC_API tc_status tc_prefill_from_state(const tc_prefill_desc *desc, int64_t t0,
+                                       const void *halo_k, const void *halo_v,
+                                       const float *A_init, const void *q, const void *k,
+                                       const void *v, const float *lambda, const float *eta,
+                                       const float *g, void *y, float *A_final, void *workspace,
+                                       size_t workspace_bytes, tc_stream_t stream);
+
+/* Exclusive prefix of L2 states over consecutive pieces of one sequence
+ * (sequence sharding: piece s is the part of the sequence held by rank s).
+ * Piece s alone, started from A = 0, leaves dA_s after its E_s evictions
+ * (tc_prefill_from_state with TC_PREFILL_STATE_ONLY and A_init = NULL).
+ * Every eviction does A <- lambda A + eta k v^T (§3.2, Fig. 2 step (3)), so
+ * the state before piece n_parts is
+ *   A_out = sum_s lambda^(E_{s+1} + ... + E_{n_parts-1}) dA_s,
+ * computed as A <- lambda^{E_s} A + dA_s for s = 0 .. n_parts-1.
+ *   dA     [n_parts][B,H,d_k,d_v] float32 device
+ *   E      [n_parts] int64 device (eviction counts)
+ *   lambda [H] float32 device;  A_out [B,H,d_k,d_v] float32 device.
+ * n_parts = 0 gives A_out = 0.  Errors: TC_ERR_INVALID_ARG, TC_ERR_NO_DEVICE,
+ * TC_ERR_CUDA.  Asynchronous on stream. */
+TC_API tc_status tc_state_fold(int64_t B, int64_t H, int64_t dk, int64_t dv, int64_t n_parts,
+                               const float *dA, const int64_t *E, const float *lambda,
+                               float *A_out, tc_stream_t stream);
 
 /* Number of kernel launches one tc_prefill call enqueues for desc on the
  * current device (the path depends on shapes and dtype), or -1 when desc is

@@ -39,12 +39,14 @@ STATUS_NAMES = {0: "TC_OK", 1: "TC_ERR_INVALID_ARG", 2: "TC_ERR_UNSUPPORTED",
                 6: "TC_ERR_DEVICE_TIMEOUT", 7: "TC_ERR_WORKSPACE"}
 TC_F32, TC_BF16 = 0, 1
 TC_PREFILL_L1_ONLY = 1
+TC_PREFILL_STATE_ONLY = 2
 
 # Exported C symbols declared in include/tc.h.
 EXPORTED = ("tc_prefill_workspace_size", "tc_prefill", "tc_prefill_launch_count", "tc_prefill_host_workspace_size",
             "tc_prefill_host", "tc_decode_step", "tc_decode_step_host_workspace_size",
             "tc_decode_step_host", "tc_get_device_status", "tc_status_string", "tc_version",
-            "tc_prefill_no_alloc")
+            "tc_prefill_no_alloc", "tc_prefill_from_state", "tc_prefill_from_state_workspace_size",
+            "tc_state_fold")
 
 
 class PrefillDesc(ctypes.Structure):
@@ -76,6 +78,12 @@ _lib.tc_prefill_host.argtypes = [_PD] + [_vp] * 9 + [_sz, _vp]
 _lib.tc_prefill_host.restype = _int
 _lib.tc_prefill_no_alloc.argtypes = [_PD] + [_vp] * 8 + [_vp]
 _lib.tc_prefill_no_alloc.restype = _int
+_lib.tc_prefill_from_state_workspace_size.argtypes = [_PD, ctypes.c_int64]
+_lib.tc_prefill_from_state_workspace_size.restype = _sz
+_lib.tc_prefill_from_state.argtypes = [_PD, ctypes.c_int64] + [_vp] * 12 + [_sz, _vp]
+_lib.tc_prefill_from_state.restype = _int
+_lib.tc_state_fold.argtypes = [ctypes.c_int64] * 5 + [_vp] * 4 + [_vp]
+_lib.tc_state_fold.restype = _int
 _lib.tc_decode_step.argtypes = [_DS] + [_vp] * 4 + [_vp]
 _lib.tc_decode_step.restype = _int
 _lib.tc_decode_step_host_workspace_size.argtypes = [_DS]
@@ -141,9 +149,11 @@ def _contig(*ts):
             raise ValueError("tensors must be contiguous")
 
 
-def make_prefill_desc(B, H, T, dk, dv, W, C, dtype: int, l1_only: bool = False) -> PrefillDesc:
+def make_prefill_desc(B, H, T, dk, dv, W, C, dtype: int, l1_only: bool = False,
+                      state_only: bool = False) -> PrefillDesc:
+    flags = (TC_PREFILL_L1_ONLY if l1_only else 0) | (TC_PREFILL_STATE_ONLY if state_only else 0)
     return PrefillDesc(int(B), int(H), int(T), int(dk), int(dv), int(W), int(C), int(dtype),
-                       TC_PREFILL_L1_ONLY if l1_only else 0)
+                       flags)
 
 
 def prefill_workspace_size(desc: PrefillDesc) -> int:
@@ -182,6 +192,57 @@ def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, lam: torch.Tensor
                          _stream(stream))
     _check(st, "tc_prefill")
     return y, A_final
+
+
+def prefill_from_state(q: Optional[torch.Tensor], k: torch.Tensor, v: torch.Tensor,
+                       lam: torch.Tensor, eta: torch.Tensor, g: torch.Tensor, W: int, C: int,
+                       t0: int, halo_k: Optional[torch.Tensor] = None,
+                       halo_v: Optional[torch.Tensor] = None, A_init: Optional[torch.Tensor] = None,
+                       *, state_only: bool = False, l1_only: bool = False,
+                       y: Optional[torch.Tensor] = None, A_final: Optional[torch.Tensor] = None,
+                       workspace: Optional[torch.Tensor] = None, stream=None):
+    """tc_prefill_from_state: the layer over the new tokens k, v [B,H,T,d]
+    (queries q, unless state_only) starting at global position t0, given the
+    halo (keys / values of tokens t0 - min(t0, W) .. t0 - 1, oldest first) and
+    A_init (A after the evictions before t0; None = zero).  Returns
+    (y, A_final); y is None with state_only."""
+    B, H, T, dk = k.shape
+    dv = v.shape[-1]
+    desc = make_prefill_desc(B, H, T, dk, dv, W, C, _dtype_code(k), l1_only, state_only)
+    if y is None and not state_only:
+        y = torch.empty((B, H, T, dv), dtype=k.dtype, device=k.device)
+    if A_final is None and not l1_only:
+        A_final = torch.empty((B, H, dk, dv), dtype=torch.float32, device=k.device)
+    need = _lib.tc_prefill_from_state_workspace_size(ctypes.byref(desc), int(t0))
+    if need == SIZE_ERROR:
+        raise TCError(1, "tc_prefill_from_state_workspace_size")
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=k.device)
+    _contig(q, k, v, lam, eta, g, y, A_final, workspace, halo_k, halo_v, A_init)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = _lib.tc_prefill_from_state(ctypes.byref(desc), int(t0), _ptr(halo_k), _ptr(halo_v),
+                                    _ptr(A_init), _ptr(q), _ptr(k), _ptr(v), _ptr(lam),
+                                    _ptr(eta), _ptr(g), _ptr(y), _ptr(A_final), _ptr(workspace),
+                                    ws_bytes, _stream(stream))
+    _check(st, "tc_prefill_from_state")
+    return y, A_final
+
+
+def state_fold(dA: torch.Tensor, E: torch.Tensor, lam: torch.Tensor,
+               A_out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """tc_state_fold: dA [n_parts,B,H,dk,dv] float32, E [n_parts] int64,
+    lam [H] float32 (all on the device).  Returns the state before piece
+    n_parts."""
+    n, B, H, dk, dv = dA.shape
+    if A_out is None:
+        A_out = torch.empty((B, H, dk, dv), dtype=torch.float32, device=lam.device)
+    _contig(dA, E, lam, A_out)
+    if dA.dtype != torch.float32 or E.dtype != torch.int64:
+        raise TypeError("dA must be float32 and E int64")
+    st = _lib.tc_state_fold(B, H, dk, dv, n, _ptr(dA) if n else None, _ptr(E) if n else None,
+                            _ptr(lam), _ptr(A_out), _stream(stream))
+    _check(st, "tc_state_fold")
+    return A_out
 
 
 def prefill_launch_count(desc: PrefillDesc) -> int:

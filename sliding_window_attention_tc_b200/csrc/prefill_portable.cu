@@ -28,6 +28,14 @@ constexpr int kMaxPerThread = kMaxD * kMaxD / kThreads;  // 64
 __host__ __device__ inline int64_t evictions(int64_t T, int64_t W) { return T > W ? T - W : 0; }
 __host__ __device__ inline int64_t num_chunks(int64_t E, int64_t C) { return (E + C - 1) / C; }
 
+// Row tau of the combined halo + new sequence of one (b,h): halo rows first.
+template <typename T>
+__device__ __forceinline__ const T *kv_row(const void *halo, const void *base, int64_t bh,
+                                           int64_t n_halo, int64_t T_new, int d, int64_t tau) {
+    return tau < n_halo ? reinterpret_cast<const T *>(halo) + (bh * n_halo + tau) * d
+                        : reinterpret_cast<const T *>(base) + (bh * T_new + (tau - n_halo)) * d;
+}
+
 // Chunk scan over one head's evictions; stores S_c (state at the start of
 // chunk c) for c = 0..nC-1 and A_final = the state after all evictions.
 template <typename T>
@@ -40,10 +48,8 @@ __global__ void __launch_bounds__(kThreads) chunk_state_kernel(PrefillParams p, 
     const int64_t bh = blockIdx.x;
     const int h = (int)(bh % p.H);
     const int dk = p.dk, dv = p.dv, nel = dk * dv;
-    const int64_t E = evictions(p.T, p.W), C = p.C;
+    const int64_t E = evictions(p.T + p.n_halo, p.W), C = p.C;
     const double lam = p.lam[h], eta = p.eta[h];
-    const T *kb = reinterpret_cast<const T *>(p.k) + bh * p.T * dk;
-    const T *vb = reinterpret_cast<const T *>(p.v) + bh * p.T * dv;
 
     // thread -> column col, rows row0 + i * rstep
     const int rstep = kThreads / dv;
@@ -51,7 +57,10 @@ __global__ void __launch_bounds__(kThreads) chunk_state_kernel(PrefillParams p, 
     const bool active = tid < rstep * dv;
     float S[kMaxPerThread], D[kMaxPerThread];
 #pragma unroll
-    for (int i = 0; i < kMaxPerThread; ++i) S[i] = 0.f;
+    for (int i = 0; i < kMaxPerThread; ++i) {
+        const int r = row0 + i * rstep;
+        S[i] = (p.A_init && active && r < dk) ? p.A_init[bh * nel + r * dv + col] : 0.f;
+    }
 
     for (int64_t c = 0; c < nC; ++c) {
         float *Sc = states + (bh * nC + c) * nel;
@@ -70,9 +79,11 @@ __global__ void __launch_bounds__(kThreads) chunk_state_kernel(PrefillParams p, 
             const int nt = (int)((Cc - i0 < KT) ? Cc - i0 : KT);
             __syncthreads();
             for (int x = tid; x < nt * dk; x += kThreads)
-                sk[x / dk][x % dk] = to_f32(kb[(c0 + i0 + x / dk) * dk + x % dk]);
+                sk[x / dk][x % dk] = to_f32(
+                    kv_row<T>(p.halo_k, p.k, bh, p.n_halo, p.T, dk, c0 + i0 + x / dk)[x % dk]);
             for (int x = tid; x < nt * dv; x += kThreads)
-                sv[x / dv][x % dv] = to_f32(vb[(c0 + i0 + x / dv) * dv + x % dv]);
+                sv[x / dv][x % dv] = to_f32(
+                    kv_row<T>(p.halo_v, p.v, bh, p.n_halo, p.T, dv, c0 + i0 + x / dv)[x % dv]);
             if (tid < nt) sw[tid] = (float)(eta * pow(lam, (double)(Cc - 1 - (i0 + tid))));
             __syncthreads();
             if (active) {
@@ -122,18 +133,18 @@ __global__ void __launch_bounds__(kThreads) prefill_rows_kernel(PrefillParams p,
     const int64_t bh = blockIdx.y;
     const int h = (int)(bh % p.H);
     const int dk = p.dk, dv = p.dv;
-    const int64_t T = p.T, W = p.W, C = p.C;
-    const int64_t t0 = (int64_t)blockIdx.x * ROWS;
+    // rows of q and y are the new tokens; positions t below are in the
+    // combined halo + new sequence (t = row + n_halo)
+    const int64_t T_new = p.T, nh = p.n_halo, T = T_new + nh, W = p.W, C = p.C;
+    const int64_t t0 = nh + (int64_t)blockIdx.x * ROWS;
     const int64_t t = t0 + warp;
     const bool row_ok = t < T;
     const bool use_l2 = !p.l1_only;
-    const Tin *qb = reinterpret_cast<const Tin *>(p.q) + bh * T * dk;
-    const Tin *kb = reinterpret_cast<const Tin *>(p.k) + bh * T * dk;
-    const Tin *vb = reinterpret_cast<const Tin *>(p.v) + bh * T * dv;
+    const Tin *qb = reinterpret_cast<const Tin *>(p.q) + bh * T_new * dk;
 
     for (int x = tid; x < ROWS * dk; x += kThreads) {
         const int64_t tt = t0 + x / dk;
-        sq[x / dk][x % dk] = tt < T ? to_f32(qb[tt * dk + x % dk]) : 0.f;
+        sq[x / dk][x % dk] = tt < T ? to_f32(qb[(tt - nh) * dk + x % dk]) : 0.f;
     }
 
     const float lam = p.lam[h], eta = p.eta[h];
@@ -163,9 +174,9 @@ __global__ void __launch_bounds__(kThreads) prefill_rows_kernel(PrefillParams p,
         const int nt = (int)((t_last - j0 + 1 < KT) ? t_last - j0 + 1 : KT);
         __syncthreads();
         for (int x = tid; x < nt * dk; x += kThreads)
-            sk[x / dk][x % dk] = to_f32(kb[(j0 + x / dk) * dk + x % dk]);
+            sk[x / dk][x % dk] = to_f32(kv_row<Tin>(p.halo_k, p.k, bh, nh, T_new, dk, j0 + x / dk)[x % dk]);
         for (int x = tid; x < nt * dv; x += kThreads)
-            sv[x / dv][x % dv] = to_f32(vb[(j0 + x / dv) * dv + x % dv]);
+            sv[x / dv][x % dv] = to_f32(kv_row<Tin>(p.halo_v, p.v, bh, nh, T_new, dv, j0 + x / dv)[x % dv]);
         __syncthreads();
         if (!row_ok) continue;
         const int64_t j = j0 + lane;
@@ -219,7 +230,7 @@ __global__ void __launch_bounds__(kThreads) prefill_rows_kernel(PrefillParams p,
             }
         }
     }
-    Tin *y = reinterpret_cast<Tin *>(p.y) + (bh * T + t) * dv;
+    Tin *y = reinterpret_cast<Tin *>(p.y) + (bh * T_new + (t - nh)) * dv;
     const float inv_l = 1.0f / l_run;
 #pragma unroll
     for (int i = 0; i < CPL; ++i) {
@@ -232,14 +243,14 @@ template <typename T>
 cudaError_t launch_t(const PrefillParams &p, cudaStream_t s) {
     const int64_t BH = p.B * p.H;
     if (BH == 0) return cudaSuccess;
-    const int64_t nC = p.l1_only ? 0 : num_chunks(evictions(p.T, p.W), p.C);
+    const int64_t nC = p.l1_only ? 0 : num_chunks(evictions(p.T + p.n_halo, p.W), p.C);
     float *states = reinterpret_cast<float *>(p.workspace);
     if (!p.l1_only) {
         chunk_state_kernel<T><<<(unsigned)BH, kThreads, 0, s>>>(p, states, nC);
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
-    if (p.T > 0) {
+    if (p.T > 0 && !p.state_only) {
         const dim3 grid((unsigned)((p.T + 7) / 8), (unsigned)BH);
         prefill_rows_kernel<T><<<grid, kThreads, 0, s>>>(p, states, nC);
     }
@@ -248,9 +259,9 @@ cudaError_t launch_t(const PrefillParams &p, cudaStream_t s) {
 
 }  // namespace
 
-size_t portable_workspace_bytes(const tc_prefill_desc &d) {
+size_t portable_workspace_bytes(const tc_prefill_desc &d, int64_t n_halo) {
     if (d.flags & TC_PREFILL_L1_ONLY) return 0;
-    const int64_t nC = num_chunks(evictions(d.T, d.W), d.C);
+    const int64_t nC = num_chunks(evictions(d.T + n_halo, d.W), d.C);
     return (size_t)(d.B * d.H * nC * d.dk * d.dv) * sizeof(float);
 }
 

@@ -79,25 +79,48 @@ constexpr uint32_t TM_DS = 448; // state increment: rows 0-63 hi part, 64-127 lo
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescale = 8.0f;  // rescale O only when the running max grows by > 2^8
 
+// Token coordinates.  The kernels run over a combined sequence of T tokens:
+// the first q_off are a halo (the keys and values of the tokens just before
+// a continued sequence, read through their own tensor maps), the rest are the
+// new tokens, whose queries and outputs are rows 0.. of q and y.  Query tiles
+// start at i_begin = q_off / 128; q_off is 0 or W, a multiple of 128.
 struct MainParams {
     void *y;
     float *A_final;
     const float *lam, *eta, *g;
-    const float *dA;  // [BH * n_s][64][64] span summaries
-    int T, W, H, BH, nT, n_s, l1_only;
+    const float *dA;      // [BH * n_s][64][64] span summaries
+    const float *A_init;  // [BH][64][64] state before the first eviction, or null
+    int T, W, H, BH, nT, n_s, l1_only, q_off;
     int *status;
 };
 
 struct SumParams {
     float *dA;
     const float *lam, *eta;
-    int T, W, H, BH, nT, n_s;
+    int T, W, H, BH, nT, n_s, q_off;
     int *status;
 };
 
-__device__ __forceinline__ void span_range(int j, int nT, int n_s, int &i0, int &i1) {
-    i0 = (int)((long long)j * nT / n_s);
-    i1 = (int)((long long)(j + 1) * nT / n_s);
+// Query tiles [i0, i1) of span j: the tiles i_begin .. nT-1 cut into n_s parts.
+__device__ __forceinline__ void span_range(int j, int nT, int n_s, int i_begin, int &i0, int &i1) {
+    const int n = nT - i_begin;
+    i0 = i_begin + (int)((long long)j * n / n_s);
+    i1 = i_begin + (int)((long long)(j + 1) * n / n_s);
+}
+
+// Key / value tile u of the combined sequence: halo maps for u < q_off/128.
+__device__ __forceinline__ void load_kv_tile(uint8_t *dst, const CUtensorMap *tk,
+                                             const CUtensorMap *tv, const CUtensorMap *tkh,
+                                             const CUtensorMap *tvh, uint64_t *bar, int u,
+                                             int q_off, int bh) {
+    const int row = u * 128;
+    if (row < q_off) {
+        tma_load_3d(dst, tkh, bar, 0, row, bh);
+        tma_load_3d(dst + 128 * 64 * 2, tvh, bar, 0, row, bh);
+    } else {
+        tma_load_3d(dst, tk, bar, 0, row - q_off, bh);
+        tma_load_3d(dst + 128 * 64 * 2, tv, bar, 0, row - q_off, bh);
+    }
 }
 
 __device__ __forceinline__ void named_bar(int id, int n) {
@@ -304,7 +327,8 @@ constexpr uint32_t SMEM_SUM = SOFF_BAR + 128 + 1024;         // ~97 KB: two CTAs
 
 __global__ void __launch_bounds__(192, 2)
     span_summary_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
-                        SumParams p) {
+                        const __grid_constant__ CUtensorMap tkh,
+                        const __grid_constant__ CUtensorMap tvh, SumParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~uintptr_t(1023));
@@ -320,7 +344,7 @@ __global__ void __launch_bounds__(192, 2)
     const int bh = blockIdx.x / per_head, js = blockIdx.x % per_head;
     const int h = bh % p.H;
     int i0, i1;
-    span_range(js, p.nT, p.n_s, i0, i1);
+    span_range(js, p.nT, p.n_s, p.q_off / BM, i0, i1);
     const int E = p.T > p.W ? p.T - p.W : 0;
     const int ev_first = i0 > p.W / BM ? i0 : p.W / BM;  // first tile with evictions
     const int ne = i1 > ev_first ? i1 - ev_first : 0;
@@ -360,8 +384,7 @@ __global__ void __launch_bounds__(192, 2)
                 const int n0 = (ev_first + e) * BM - p.W;
                 uint8_t *dst = sm + SOFF_KV + s * 2 * TILE_B;
                 mbar_expect_tx(&kv_full[s], 2 * TILE_B);
-                tma_load_3d(dst, &tk, &kv_full[s], 0, n0, bh);
-                tma_load_3d(dst + TILE_B, &tv, &kv_full[s], 0, n0, bh);
+                load_kv_tile(dst, &tk, &tv, &tkh, &tvh, &kv_full[s], n0 / BM, p.q_off, bh);
                 issued = e + 1;
             }
             for (int st = 0; st < NS_SUM; ++st) {
@@ -444,7 +467,8 @@ __global__ void __launch_bounds__(192, 2)
 // ============================================================================
 __global__ void __launch_bounds__(kMainThreads, 1)
     prefill_main_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
-                        const __grid_constant__ CUtensorMap tv, MainParams p) {
+                        const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tkh,
+                        const __grid_constant__ CUtensorMap tvh, MainParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~uintptr_t(1023));
@@ -506,26 +530,28 @@ __global__ void __launch_bounds__(kMainThreads, 1)
             tma_prefetch_desc(&tq);
             tma_prefetch_desc(&tk);
             tma_prefetch_desc(&tv);
+            if (p.q_off > 0) {
+                tma_prefetch_desc(&tkh);
+                tma_prefetch_desc(&tvh);
+            }
             uint32_t tile = 0, kc = 0;
             bool ok = true;
             for (int sp = blockIdx.x; sp < n_spans && ok; sp += gridDim.x) {
                 const int bh = sp / p.n_s;
                 int i0, i1;
-                span_range(sp % p.n_s, p.nT, p.n_s, i0, i1);
+                span_range(sp % p.n_s, p.nT, p.n_s, p.q_off / BM, i0, i1);
                 for (int i = i0; i < i1 && ok; ++i, ++tile) {
                     const TileInfo ti = tile_info(i, p.W, l1_only);
                     const int qb = tile & 1;
                     if (!(ok = mbar_wait(&q_empty[qb], ((tile >> 1) & 1) ^ 1, abort, p.status))) break;
                     mbar_expect_tx(&q_full[qb], TILE_B);
-                    tma_load_3d(sm + OFF_Q + qb * TILE_B, &tq, &q_full[qb], 0, ti.t0, bh);
+                    tma_load_3d(sm + OFF_Q + qb * TILE_B, &tq, &q_full[qb], 0, ti.t0 - p.q_off, bh);
                     for (int j = 0; j < ti.nk; ++j, ++kc) {
                         const int s = kc % NS;
                         if (!(ok = mbar_wait(&kv_empty[s], ((kc / NS) & 1) ^ 1, abort, p.status))) break;
                         uint8_t *dst = sm + OFF_KV + s * 2 * TILE_B;
-                        const int row = (ti.kt0 + j) * BM;
                         mbar_expect_tx(&kv_full[s], 2 * TILE_B);
-                        tma_load_3d(dst, &tk, &kv_full[s], 0, row, bh);
-                        tma_load_3d(dst + TILE_B, &tv, &kv_full[s], 0, row, bh);
+                        load_kv_tile(dst, &tk, &tv, &tkh, &tvh, &kv_full[s], ti.kt0 + j, p.q_off, bh);
                     }
                 }
             }
@@ -604,7 +630,7 @@ __global__ void __launch_bounds__(kMainThreads, 1)
             };
             for (int sp = blockIdx.x; sp < n_spans && ok; sp += gridDim.x) {
                 int i0, i1;
-                span_range(sp % p.n_s, p.nT, p.n_s, i0, i1);
+                span_range(sp % p.n_s, p.nT, p.n_s, p.q_off / BM, i0, i1);
                 for (int i = i0; i < i1 && ok; ++i, ++tile) {
                     const TileInfo ti = tile_info(i, p.W, l1_only);
                     const int qb = tile & 1;
@@ -679,8 +705,10 @@ __global__ void __launch_bounds__(kMainThreads, 1)
             mbar_arrive(o_empty);
             const int t = e.t0 + r;
             if (t < p.T) {
+                const size_t T_new = (size_t)(p.T - p.q_off);
                 uint4 *dst = reinterpret_cast<uint4 *>(reinterpret_cast<__nv_bfloat16 *>(p.y) +
-                                                       ((size_t)e.bh * p.T + t) * HD + 32 * half);
+                                                       ((size_t)e.bh * T_new + (t - p.q_off)) * HD +
+                                                       32 * half);
 #pragma unroll
                 for (int c = 0; c < 4; ++c)
                     dst[c] = make_uint4(pack_bf16(yv[8 * c], yv[8 * c + 1]),
@@ -693,7 +721,7 @@ __global__ void __launch_bounds__(kMainThreads, 1)
         for (int sp = blockIdx.x; sp < n_spans && ok; sp += gridDim.x) {
             const int bh = sp / p.n_s, h = bh % p.H;
             int i0, i1;
-            span_range(sp % p.n_s, p.nT, p.n_s, i0, i1);
+            span_range(sp % p.n_s, p.nT, p.n_s, p.q_off / BM, i0, i1);
             const double lam = p.lam[h];
             const float gate = 1.0f / (1.0f + expf(-p.g[h]));
             const float pw_r1 = (float)pow(lam, (double)(r + 1));
@@ -780,7 +808,7 @@ __global__ void __launch_bounds__(kMainThreads, 1)
         for (int sp = blockIdx.x; sp < n_spans && ok; sp += gridDim.x) {
             const int bh = sp / p.n_s, h = bh % p.H, js = sp % p.n_s;
             int i0, i1;
-            span_range(js, p.nT, p.n_s, i0, i1);
+            span_range(js, p.nT, p.n_s, p.q_off / BM, i0, i1);
             const double lam = p.lam[h];
             const double l2l = log2(lam);
             // per-span tables (float math in the tile loop only): ew[k] = eta lam^k,
@@ -794,10 +822,17 @@ __global__ void __launch_bounds__(kMainThreads, 1)
             const int n_start = max(0, i0 * BM - p.W);
 #pragma unroll
             for (int c = 0; c < 64; ++c) S[c] = 0.f;
+            if (!l1_only && u < 64 && p.A_init) {
+                // the given state before the first eviction, decayed to the span start
+                const float coef = (float)exp2((double)n_start * l2l);
+                const float *src = p.A_init + ((size_t)bh * HD + u) * HD;
+#pragma unroll
+                for (int c = 0; c < 64; ++c) S[c] = coef * src[c];
+            }
             if (!l1_only && u < 64 && n_start > 0) {
                 for (int jj = 0; jj < js; ++jj) {
                     int a0, a1;
-                    span_range(jj, p.nT, p.n_s, a0, a1);
+                    span_range(jj, p.nT, p.n_s, p.q_off / BM, a0, a1);
                     const int e_end = max(0, min(E, a1 * BM - p.W));
                     if (e_end <= 0) continue;
                     const float coef = (float)exp2((double)(n_start - e_end) * l2l);
@@ -943,14 +978,16 @@ int choose_spans(int64_t BH, int nT, int num_sms) {
 
 }  // namespace
 
-bool sm100_supported(const tc_prefill_desc &d) {
+bool sm100_supported(const tc_prefill_desc &d, int64_t n_halo) {
     return d.dtype == TC_BF16 && d.dk == HD && d.dv == HD && d.W >= BM && d.W % BM == 0 &&
-           d.T >= 1 && d.T <= (int64_t(1) << 30) && d.B * d.H <= 65535;
+           d.T >= 1 && d.T + n_halo <= (int64_t(1) << 30) && d.B * d.H <= 65535 &&
+           (n_halo == 0 || n_halo == d.W) && !(d.flags & TC_PREFILL_STATE_ONLY);
 }
 
+// Spans are cut over the new query tiles only (the halo has no queries).
 static int spans_for(const tc_prefill_desc &d, int num_sms) {
-    const int nT = (int)((d.T + BM - 1) / BM);
-    return choose_spans(d.B * d.H, nT, num_sms);
+    const int nT_new = (int)((d.T + BM - 1) / BM);
+    return choose_spans(d.B * d.H, nT_new, num_sms);
 }
 
 size_t sm100_workspace_bytes(const tc_prefill_desc &d, int num_sms) {
@@ -973,12 +1010,21 @@ int sm100_launch_count(const tc_prefill_desc &d) {
 
 cudaError_t launch_prefill_sm100(const PrefillParams &p, int num_sms, cudaStream_t s) {
     const int64_t BH = p.B * p.H;
-    const int nT = (int)((p.T + BM - 1) / BM);
-    const int ns = choose_spans(BH, nT, num_sms);
-    CUtensorMap tq, tk, tv;
+    const int q_off = (int)p.n_halo;
+    const int T_all = (int)(p.T + p.n_halo);  // combined sequence
+    const int nT = (T_all + BM - 1) / BM;
+    const int ns = choose_spans(BH, nT - q_off / BM, num_sms);
+    CUtensorMap tq, tk, tv, tkh, tvh;
     if (!make_map(&tq, p.q, (int)p.T, (int)BH) || !make_map(&tk, p.k, (int)p.T, (int)BH) ||
         !make_map(&tv, p.v, (int)p.T, (int)BH))
         return cudaErrorInvalidValue;
+    if (q_off > 0) {
+        if (!make_map(&tkh, p.halo_k, q_off, (int)BH) || !make_map(&tvh, p.halo_v, q_off, (int)BH))
+            return cudaErrorInvalidValue;
+    } else {
+        tkh = tk;  // never read
+        tvh = tv;
+    }
     cudaError_t e = cudaFuncSetAttribute(prefill_main_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_MAIN);
     if (e != cudaSuccess) return e;
@@ -987,16 +1033,16 @@ cudaError_t launch_prefill_sm100(const PrefillParams &p, int num_sms, cudaStream
     if (e != cudaSuccess) return e;
     float *dA = reinterpret_cast<float *>(p.workspace);
     if (!p.l1_only && ns > 1) {
-        SumParams sp{dA, p.lam, p.eta, (int)p.T, (int)p.W, (int)p.H, (int)BH, nT, ns, p.status};
-        span_summary_kernel<<<(unsigned)(BH * (ns - 1)), 192, SMEM_SUM, s>>>(tk, tv, sp);
+        SumParams sp{dA, p.lam, p.eta, T_all, (int)p.W, (int)p.H, (int)BH, nT, ns, q_off, p.status};
+        span_summary_kernel<<<(unsigned)(BH * (ns - 1)), 192, SMEM_SUM, s>>>(tk, tv, tkh, tvh, sp);
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
-    MainParams mp{p.y, p.A_final, p.lam, p.eta, p.g, dA, (int)p.T, (int)p.W, (int)p.H, (int)BH,
-                  nT, ns, p.l1_only ? 1 : 0, p.status};
+    MainParams mp{p.y,      p.A_final, p.lam, p.eta, p.g,  dA, p.A_init, T_all, (int)p.W, (int)p.H,
+                  (int)BH, nT,        ns,    p.l1_only ? 1 : 0, q_off, p.status};
     const int64_t spans = BH * ns;
     const unsigned grid = (unsigned)(spans < num_sms ? spans : num_sms);
-    prefill_main_kernel<<<grid, kMainThreads, SMEM_MAIN, s>>>(tq, tk, tv, mp);
+    prefill_main_kernel<<<grid, kMainThreads, SMEM_MAIN, s>>>(tq, tk, tv, tkh, tvh, mp);
     return cudaGetLastError();
 }
 

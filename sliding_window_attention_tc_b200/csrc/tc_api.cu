@@ -33,7 +33,9 @@ tc_status check_desc(const tc_prefill_desc *d) {
     if (d->B < 1 || d->H < 1 || d->T < 0 || d->dk < 1 || d->dv < 1 || d->W < 1 || d->C < 1)
         return TC_ERR_INVALID_ARG;
     if (!valid_dtype(d->dtype)) return TC_ERR_INVALID_ARG;
-    if (d->flags & ~TC_PREFILL_L1_ONLY) return TC_ERR_INVALID_ARG;
+    if (d->flags & ~(TC_PREFILL_L1_ONLY | TC_PREFILL_STATE_ONLY)) return TC_ERR_INVALID_ARG;
+    if ((d->flags & TC_PREFILL_L1_ONLY) && (d->flags & TC_PREFILL_STATE_ONLY))
+        return TC_ERR_INVALID_ARG;
     if (d->dk > kMaxDim || d->dv > kMaxDim) return TC_ERR_UNSUPPORTED;
     // grid limits of the portable path and 32-bit-safe element counts
     if (d->B * d->H > 65535) return TC_ERR_UNSUPPORTED;
@@ -80,10 +82,14 @@ int *status_ptr() {
     return static_cast<int *>(p);
 }
 
-bool use_sm100(const tc_prefill_desc &d) { return tc::sm100_supported(d); }
+// Halo length of a call that continues at global position t0.
+int64_t halo_len(const tc_prefill_desc &d, int64_t t0) { return t0 < d.W ? t0 : d.W; }
 
-size_t prefill_ws(const tc_prefill_desc &d, int num_sms) {
-    return use_sm100(d) ? tc::sm100_workspace_bytes(d, num_sms) : tc::portable_workspace_bytes(d);
+bool use_sm100(const tc_prefill_desc &d, int64_t n_halo) { return tc::sm100_supported(d, n_halo); }
+
+size_t prefill_ws(const tc_prefill_desc &d, int64_t n_halo, int num_sms) {
+    return use_sm100(d, n_halo) ? tc::sm100_workspace_bytes(d, num_sms)
+                                : tc::portable_workspace_bytes(d, n_halo);
 }
 
 int sm_count_or_default() {
@@ -128,32 +134,54 @@ const char *tc_status_string(tc_status s) {
 
 size_t tc_prefill_workspace_size(const tc_prefill_desc *d) {
     if (check_desc(d) != TC_OK) return (size_t)-1;
-    return prefill_ws(*d, sm_count_or_default());
+    return prefill_ws(*d, 0, sm_count_or_default());
 }
 
-tc_status tc_prefill(const tc_prefill_desc *d, const void *q, const void *k, const void *v,
-                     const float *lambda, const float *eta, const float *g, void *y,
-                     float *A_final, void *workspace, size_t workspace_bytes,
-                     tc_stream_t stream) {
+size_t tc_prefill_from_state_workspace_size(const tc_prefill_desc *d, int64_t t0) {
+    if (check_desc(d) != TC_OK || t0 < 0) return (size_t)-1;
+    return prefill_ws(*d, halo_len(*d, t0), sm_count_or_default());
+}
+
+}  // extern "C"
+
+namespace {
+
+// Shared body of tc_prefill (t0 = 0) and tc_prefill_from_state.
+tc_status prefill_impl(const tc_prefill_desc *d, int64_t t0, const void *halo_k,
+                       const void *halo_v, const float *A_init, const void *q, const void *k,
+                       const void *v, const float *lambda, const float *eta, const float *g,
+                       void *y, float *A_final, void *workspace, size_t workspace_bytes,
+                       tc_stream_t stream) {
     tc_status st = check_desc(d);
     if (st != TC_OK) return st;
+    if (t0 < 0 || t0 > (int64_t(1) << 31)) return TC_ERR_INVALID_ARG;
     const bool l1_only = (d->flags & TC_PREFILL_L1_ONLY) != 0;
-    // With T = 0 the token tensors are empty and may be NULL.
+    const bool state_only = (d->flags & TC_PREFILL_STATE_ONLY) != 0;
+    const int64_t n_halo = halo_len(*d, t0);
+    // With T = 0 the token tensors are empty and may be NULL; a state-only
+    // call reads no queries and writes no outputs.
     const bool empty = d->T == 0;
-    if ((!empty && (!q || !k || !v || !y)) || !lambda || !eta || !g || (!l1_only && !A_final))
+    const bool need_q = !empty && !state_only;
+    if ((need_q && (!q || !y)) || (!empty && (!k || !v)) || !lambda || !eta || !g ||
+        (!l1_only && !A_final) || (n_halo > 0 && (!halo_k || !halo_v)))
         return TC_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(y) ||
-        (A_final && !aligned16(A_final)) || (workspace && !aligned16(workspace)))
+        (A_final && !aligned16(A_final)) || (workspace && !aligned16(workspace)) ||
+        !aligned16(halo_k) || !aligned16(halo_v) || !aligned16(A_init))
         return TC_ERR_INVALID_ARG;
     int dev = 0, sms = 0;
     st = current_device(&dev, &sms);
     if (st != TC_OK) return st;
-    const size_t need = prefill_ws(*d, sms);
+    const size_t need = prefill_ws(*d, n_halo, sms);
     if (need > 0 && (!workspace || workspace_bytes < need)) return TC_ERR_WORKSPACE;
-    const void *ptrs[] = {q, k, v, y, lambda, eta, g};
-    for (int i = 0; i < 7; ++i)
-        if (!(empty && i < 4 && !ptrs[i]) && !is_device_ptr(ptrs[i])) return TC_ERR_INVALID_ARG;
+    const void *ptrs[] = {q, y, k, v, lambda, eta, g};
+    for (int i = 0; i < 7; ++i) {
+        const bool may_be_null = (i < 2 && !need_q) || (i < 4 && empty);
+        if (!(may_be_null && !ptrs[i]) && !is_device_ptr(ptrs[i])) return TC_ERR_INVALID_ARG;
+    }
     if (A_final && !is_device_ptr(A_final)) return TC_ERR_INVALID_ARG;
+    if (A_init && !is_device_ptr(A_init)) return TC_ERR_INVALID_ARG;
+    if (n_halo > 0 && (!is_device_ptr(halo_k) || !is_device_ptr(halo_v))) return TC_ERR_INVALID_ARG;
     if (need > 0 && !is_device_ptr(workspace)) return TC_ERR_INVALID_ARG;
 
     tc::PrefillParams p{};
@@ -173,20 +201,47 @@ tc_status tc_prefill(const tc_prefill_desc *d, const void *q, const void *k, con
     p.dk = (int)d->dk;
     p.dv = (int)d->dv;
     p.l1_only = l1_only;
+    p.state_only = state_only;
+    p.halo_k = n_halo > 0 ? halo_k : nullptr;
+    p.halo_v = n_halo > 0 ? halo_v : nullptr;
+    p.n_halo = n_halo;
+    p.A_init = l1_only ? nullptr : A_init;
     p.workspace = workspace;
     p.workspace_bytes = workspace_bytes;
     p.status = status_ptr();
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    cudaError_t e = use_sm100(*d) ? tc::launch_prefill_sm100(p, sms, s)
-                                  : tc::launch_prefill_portable(p, d->dtype, s);
+    cudaError_t e = use_sm100(*d, n_halo) ? tc::launch_prefill_sm100(p, sms, s)
+                                          : tc::launch_prefill_portable(p, d->dtype, s);
     return e == cudaSuccess ? TC_OK : TC_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+tc_status tc_prefill(const tc_prefill_desc *d, const void *q, const void *k, const void *v,
+                     const float *lambda, const float *eta, const float *g, void *y,
+                     float *A_final, void *workspace, size_t workspace_bytes,
+                     tc_stream_t stream) {
+    return prefill_impl(d, 0, nullptr, nullptr, nullptr, q, k, v, lambda, eta, g, y, A_final,
+                        workspace, workspace_bytes, stream);
+}
+
+tc_status tc_prefill_from_state(const tc_prefill_desc *d, int64_t t0, const void *halo_k,
+                                const void *halo_v, const float *A_init, const void *q,
+                                const void *k, const void *v, const float *lambda,
+                                const float *eta, const float *g, void *y, float *A_final,
+                                void *workspace, size_t workspace_bytes, tc_stream_t stream) {
+    return prefill_impl(d, t0, halo_k, halo_v, A_init, q, k, v, lambda, eta, g, y, A_final,
+                        workspace, workspace_bytes, stream);
 }
 
 int tc_prefill_launch_count(const tc_prefill_desc *d) {
     if (check_desc(d) != TC_OK) return -1;
-    if (use_sm100(*d)) return tc::sm100_launch_count(*d);
+    if (use_sm100(*d, 0)) return tc::sm100_launch_count(*d);
     const bool l1_only = (d->flags & TC_PREFILL_L1_ONLY) != 0;
-    return (l1_only ? 0 : 1) + (d->T > 0 ? 1 : 0);
+    const bool state_only = (d->flags & TC_PREFILL_STATE_ONLY) != 0;
+    return (l1_only ? 0 : 1) + (d->T > 0 && !state_only ? 1 : 0);
 }
 
 size_t tc_prefill_host_workspace_size(const tc_prefill_desc *d) {
@@ -196,7 +251,7 @@ size_t tc_prefill_host_workspace_size(const tc_prefill_desc *d) {
     const size_t nv = (size_t)(d->B * d->H * d->T * d->dv) * es;
     const size_t na = (size_t)(d->B * d->H * d->dk * d->dv) * sizeof(float);
     const size_t np = (size_t)d->H * sizeof(float);
-    return round_up(prefill_ws(*d, sm_count_or_default())) + 2 * round_up(nq) + 2 * round_up(nv) +
+    return round_up(prefill_ws(*d, 0, sm_count_or_default())) + 2 * round_up(nq) + 2 * round_up(nv) +
            3 * round_up(np) + round_up(na);
 }
 
@@ -221,7 +276,7 @@ tc_status tc_prefill_host(const tc_prefill_desc *d, const void *q, const void *k
     const size_t na = (size_t)(d->B * d->H * d->dk * d->dv) * sizeof(float);
     const size_t np = (size_t)d->H * sizeof(float);
     char *base = static_cast<char *>(workspace);
-    const size_t ws = round_up(prefill_ws(*d, sms));
+    const size_t ws = round_up(prefill_ws(*d, 0, sms));
     char *dq = base + ws;
     char *dk_ = dq + round_up(nq);
     char *dv_ = dk_ + round_up(nq);

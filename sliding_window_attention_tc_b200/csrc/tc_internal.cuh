@@ -72,6 +72,11 @@ struct DecodeParams {
     int *status;
 };
 
+// T new tokens (q, k, v, y rows), continuing after n_halo earlier tokens whose
+// keys and values are halo_k / halo_v ([BH][n_halo][d], oldest first), with
+// the state A_init ([BH][dk][dv] float32, null = zero) holding every eviction
+// before the first one of the combined halo + new sequence.  A plain prefill
+// has n_halo = 0 and A_init = null.
 struct PrefillParams {
     const void *q, *k, *v;
     void *y;
@@ -80,6 +85,10 @@ struct PrefillParams {
     int64_t B, H, T, W, C;
     int dk, dv;
     bool l1_only;
+    bool state_only;  // A_final only (the chunk scan); q and y unused
+    const void *halo_k, *halo_v;
+    int64_t n_halo;
+    const float *A_init;
     void *workspace;
     size_t workspace_bytes;
     int *status;
@@ -90,11 +99,11 @@ cudaError_t launch_decode(const DecodeParams &p, tc_dtype dtype, int64_t BH, cud
 bool decode_supported(int dk, int dv, tc_dtype dtype);
 
 // prefill_portable.cu: any shape in the supported range, SIMT float32 math.
-size_t portable_workspace_bytes(const tc_prefill_desc &d);
+size_t portable_workspace_bytes(const tc_prefill_desc &d, int64_t n_halo);
 cudaError_t launch_prefill_portable(const PrefillParams &p, tc_dtype dtype, cudaStream_t s);
 
 // prefill_sm100.cu: tcgen05 / TMA path for bf16, d_k = d_v = 64.
-bool sm100_supported(const tc_prefill_desc &d);
+bool sm100_supported(const tc_prefill_desc &d, int64_t n_halo);
 size_t sm100_workspace_bytes(const tc_prefill_desc &d, int num_sms);
 cudaError_t launch_prefill_sm100(const PrefillParams &p, int num_sms, cudaStream_t s);
 int sm100_launch_count(const tc_prefill_desc &d);
