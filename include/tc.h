@@ -246,6 +246,21 @@ typedef struct tc_decode_state {
 TC_API tc_status tc_decode_step(tc_decode_state *state, const void *q_t, const void *k_t,
                          const void *v_t, void *y_t, tc_stream_t stream);
 
+/* tc_decode_step for a ragged batch: every batch row b has its own clock
+ * t_rows[b] (device int64 [B]) instead of the shared state->t (which is
+ * ignored and not advanced).  Row b takes one step of Fig. 2 at t_rows[b]:
+ * its ring slot is t_rows[b] mod W, it evicts only when t_rows[b] >= W, and
+ * its window covers min(t_rows[b] + 1, W) filled slots.  A row with a
+ * negative clock is empty: its ring, A and y are left untouched.  After the
+ * step the library advances every non-negative clock by one on the device
+ * (a second, small kernel on the same stream), so the caller can start rows
+ * (write their clock) and retire them (write -1) between steps without host
+ * synchronisation.  Errors as tc_decode_step; t_rows must be 8-byte aligned
+ * device memory. */
+TC_API tc_status tc_decode_step_ragged(tc_decode_state *state, int64_t *t_rows, const void *q_t,
+                                       const void *k_t, const void *v_t, void *y_t,
+                                       tc_stream_t stream);
+
 /* Device staging bytes tc_decode_step_host needs (q_t, k_t, v_t, y_t).
  * Returns (size_t)-1 when state is NULL or invalid. */
 TC_API size_t tc_decode_step_host_workspace_size(const tc_decode_state *state);

@@ -46,7 +46,7 @@ EXPORTED = ("tc_prefill_workspace_size", "tc_prefill", "tc_prefill_launch_count"
             "tc_prefill_host", "tc_decode_step", "tc_decode_step_host_workspace_size",
             "tc_decode_step_host", "tc_get_device_status", "tc_status_string", "tc_version",
             "tc_prefill_no_alloc", "tc_prefill_from_state", "tc_prefill_from_state_workspace_size",
-            "tc_state_fold")
+            "tc_state_fold", "tc_decode_step_ragged")
 
 
 class PrefillDesc(ctypes.Structure):
@@ -86,6 +86,8 @@ _lib.tc_state_fold.argtypes = [ctypes.c_int64] * 5 + [_vp] * 4 + [_vp]
 _lib.tc_state_fold.restype = _int
 _lib.tc_decode_step.argtypes = [_DS] + [_vp] * 4 + [_vp]
 _lib.tc_decode_step.restype = _int
+_lib.tc_decode_step_ragged.argtypes = [_DS] + [_vp] * 5 + [_vp]
+_lib.tc_decode_step_ragged.restype = _int
 _lib.tc_decode_step_host_workspace_size.argtypes = [_DS]
 _lib.tc_decode_step_host_workspace_size.restype = _sz
 _lib.tc_decode_step_host.argtypes = [_DS] + [_vp] * 5 + [_sz, _vp]
@@ -338,6 +340,25 @@ def decode_step(state: DecodeState, q: torch.Tensor, k: torch.Tensor, v: torch.T
                              _stream(stream))
     _check(st, "tc_decode_step")
     state.t = int(cs.t)
+    return y
+
+
+def decode_step_ragged(state: DecodeState, t_rows: torch.Tensor, q: torch.Tensor,
+                       k: torch.Tensor, v: torch.Tensor, y: Optional[torch.Tensor] = None,
+                       stream=None) -> torch.Tensor:
+    """tc_decode_step_ragged: one step for every batch row b at its own clock
+    t_rows[b] (device int64 [B]; negative = empty row, left untouched).  The
+    library advances the non-negative clocks on the device; state.t is not
+    used."""
+    cs = state.c_struct()
+    if y is None:
+        y = torch.empty(v.shape, dtype=v.dtype, device=v.device)
+    _contig(q, k, v, y, t_rows)
+    if t_rows.dtype != torch.int64:
+        raise TypeError("t_rows must be int64")
+    st = _lib.tc_decode_step_ragged(ctypes.byref(cs), _ptr(t_rows), _ptr(q), _ptr(k), _ptr(v),
+                                    _ptr(y), _stream(stream))
+    _check(st, "tc_decode_step_ragged")
     return y
 
 

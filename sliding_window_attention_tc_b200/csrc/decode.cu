@@ -47,7 +47,11 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(DecodeParams p) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int64_t bh = blockIdx.x;
     const int h = (int)(bh % p.H);
-    const int64_t W = p.W, t = p.t;
+    const int64_t W = p.W;
+    // ragged batches: each batch row has its own clock; a negative clock is an
+    // empty row, which this step leaves untouched
+    const int64_t t = p.t_rows ? p.t_rows[bh / p.H] : p.t;
+    if (t < 0) return;
     const int64_t pos = t % W;
     const bool evict = t >= W;
     const int64_t n = evict ? W : t + 1;  // filled slots after the insert
@@ -218,6 +222,18 @@ cudaError_t launch_t(const DecodeParams &p, int64_t BH, cudaStream_t s) {
 bool decode_supported(int dk, int dv, tc_dtype dtype) {
     (void)dtype;
     return dk == dv && (dk == 16 || dk == 32 || dk == 64 || dk == 128);
+}
+
+__global__ void advance_clocks_kernel(int64_t *t_rows, int64_t B) {
+    for (int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; b < B;
+         b += (int64_t)gridDim.x * blockDim.x)
+        if (t_rows[b] >= 0) t_rows[b] += 1;
+}
+
+cudaError_t launch_advance_clocks(int64_t *t_rows, int64_t B, cudaStream_t s) {
+    const int64_t blocks = (B + 255) / 256;
+    advance_clocks_kernel<<<(unsigned)(blocks < 1024 ? blocks : 1024), 256, 0, s>>>(t_rows, B);
+    return cudaGetLastError();
 }
 
 cudaError_t launch_decode(const DecodeParams &p, tc_dtype dtype, int64_t BH, cudaStream_t s) {

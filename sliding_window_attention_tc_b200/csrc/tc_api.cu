@@ -304,12 +304,19 @@ tc_status tc_prefill_host(const tc_prefill_desc *d, const void *q, const void *k
     return TC_OK;
 }
 
-tc_status tc_decode_step(tc_decode_state *s, const void *q_t, const void *k_t, const void *v_t,
-                         void *y_t, tc_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+// Shared body of tc_decode_step (one clock, s->t) and tc_decode_step_ragged
+// (a device clock per batch row).
+tc_status decode_impl(tc_decode_state *s, int64_t *t_rows, const void *q_t, const void *k_t,
+                      const void *v_t, void *y_t, tc_stream_t stream) {
     tc_status st = check_decode_state(s);
     if (st != TC_OK) return st;
     if (!q_t || !k_t || !v_t || !y_t) return TC_ERR_INVALID_ARG;
-    if (!aligned16(q_t) || !aligned16(k_t) || !aligned16(v_t) || !aligned16(y_t))
+    if (!aligned16(q_t) || !aligned16(k_t) || !aligned16(v_t) || !aligned16(y_t) ||
+        (t_rows && (reinterpret_cast<uintptr_t>(t_rows) & 7u)))
         return TC_ERR_INVALID_ARG;
     int dev = 0;
     st = current_device(&dev, nullptr);
@@ -317,6 +324,7 @@ tc_status tc_decode_step(tc_decode_state *s, const void *q_t, const void *k_t, c
     const void *ptrs[] = {q_t, k_t, v_t, y_t, s->ring_k, s->ring_v, s->A, s->lambda, s->eta, s->g};
     for (const void *p : ptrs)
         if (!is_device_ptr(p)) return TC_ERR_INVALID_ARG;
+    if (t_rows && !is_device_ptr(t_rows)) return TC_ERR_INVALID_ARG;
     tc::DecodeParams p{};
     p.q = q_t;
     p.k = k_t;
@@ -331,14 +339,34 @@ tc_status tc_decode_step(tc_decode_state *s, const void *q_t, const void *k_t, c
     p.H = s->H;
     p.W = s->W;
     p.t = s->t;
+    p.t_rows = t_rows;
     p.dk = (int)s->dk;
     p.dv = (int)s->dv;
     p.status = status_ptr();
-    cudaError_t e = tc::launch_decode(p, s->kv_dtype, s->B * s->H,
-                                      reinterpret_cast<cudaStream_t>(stream));
+    cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = tc::launch_decode(p, s->kv_dtype, s->B * s->H, cs);
     if (e != cudaSuccess) return TC_ERR_CUDA;
-    s->t += 1;
+    if (t_rows) {
+        if (tc::launch_advance_clocks(t_rows, s->B, cs) != cudaSuccess) return TC_ERR_CUDA;
+    } else {
+        s->t += 1;
+    }
     return TC_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+tc_status tc_decode_step(tc_decode_state *s, const void *q_t, const void *k_t, const void *v_t,
+                         void *y_t, tc_stream_t stream) {
+    return decode_impl(s, nullptr, q_t, k_t, v_t, y_t, stream);
+}
+
+tc_status tc_decode_step_ragged(tc_decode_state *s, int64_t *t_rows, const void *q_t,
+                                const void *k_t, const void *v_t, void *y_t, tc_stream_t stream) {
+    if (!t_rows) return TC_ERR_INVALID_ARG;
+    return decode_impl(s, t_rows, q_t, k_t, v_t, y_t, stream);
 }
 
 size_t tc_decode_step_host_workspace_size(const tc_decode_state *s) {

@@ -68,6 +68,7 @@ struct DecodeParams {
     float *A;
     const float *lam, *eta, *g;
     int64_t H, W, t;
+    const int64_t *t_rows;  // per batch row clocks (device), or null: every row at t
     int dk, dv;
     int *status;
 };
@@ -96,6 +97,8 @@ struct PrefillParams {
 
 // decode.cu
 cudaError_t launch_decode(const DecodeParams &p, tc_dtype dtype, int64_t BH, cudaStream_t s);
+// t_rows[b] += 1 for every active row (t_rows[b] >= 0), after a ragged step.
+cudaError_t launch_advance_clocks(int64_t *t_rows, int64_t B, cudaStream_t s);
 bool decode_supported(int dk, int dv, tc_dtype dtype);
 
 // prefill_portable.cu: any shape in the supported range, SIMT float32 math.
