@@ -572,7 +572,7 @@ __global__ void __launch_bounds__(kMainThreads, 1)
         // issued before P V of key tile g-1, also across query tiles, so the
         // next tile's first scores are ready when the softmax side finishes
         // the current tile.
-        if (tid == 32) {
+        {
             const uint32_t id_qk = idesc_bf16(128, 128, false, false);
             const uint32_t id_pv = idesc_bf16(128, 64, false, true);
             const uint32_t id_qs = idesc_bf16(128, 64, false, true);
@@ -589,42 +589,42 @@ __global__ void __launch_bounds__(kMainThreads, 1)
             } pend = {false, false, false, false, 0, 0};
             auto pv_step = [&](const Pending &pv) -> bool {
                 const int sb = pv.g & 1, s = pv.g % NS;
-                if (!mbar_wait(&p_full[sb], (pv.g >> 1) & 1, abort, p.status)) return false;
-                if (pv.first && !mbar_wait(o_empty, (pv.tile & 1) ^ 1, abort, p.status)) return false;
+                if (!warp_wait(&p_full[sb], (pv.g >> 1) & 1, abort, p.status)) return false;
+                if (pv.first && !warp_wait(o_empty, (pv.tile & 1) ^ 1, abort, p.status)) return false;
                 tc_fence_after();
                 const uint32_t v_addr = kv_base + s * 2 * TILE_B + TILE_B;
                 const uint32_t s_col = tb + TM_S + sb * 128;
 #pragma unroll
                 for (int k = 0; k < 8; ++k)
-                    mma_ts(tb + TM_O, s_col + 8 * k, sdesc_sw128(v_addr + 2048 * k, TILE_B, 1024),
+                    mma_ts_w(tb + TM_O, s_col + 8 * k, sdesc_sw128(v_addr + 2048 * k, TILE_B, 1024),
                            id_pv, (!pv.first || k > 0));
                 if (pv.first && pv.l2) {
                     const uint32_t q_addr = q_base + (pv.tile & 1) * TILE_B;
 #pragma unroll
                     for (int k = 0; k < 8; ++k)
-                        mma_ts(tb + TM_MI, s_col + 64 + 8 * k,
+                        mma_ts_w(tb + TM_MI, s_col + 64 + 8 * k,
                                sdesc_sw128(v_addr + 2048 * k, TILE_B, 1024), id_pv, k > 0);
-                    if (!mbar_wait(sst_full, lc & 1, abort, p.status)) return false;
+                    if (!warp_wait(sst_full, lc & 1, abort, p.status)) return false;
                     tc_fence_after();
 #pragma unroll
                     for (int k = 0; k < 4; ++k)
-                        mma_ss(tb + TM_MX, sdesc_sw128(q_addr + 32 * k, 16, 1024),
+                        mma_ss_w(tb + TM_MX, sdesc_sw128(q_addr + 32 * k, 16, 1024),
                                sdesc_sw128(sb_addr + 2048 * k, 8192, 1024), id_qs, k > 0);
-                    if (!mbar_wait(kt_full, lc & 1, abort, p.status)) return false;
+                    if (!warp_wait(kt_full, lc & 1, abort, p.status)) return false;
                     tc_fence_after();
 #pragma unroll
                     for (int k = 0; k < 8; ++k)
-                        mma_ss(tb + TM_DS, sdesc_sw128(kt_addr + 2048 * k, TILE_B, 1024),
+                        mma_ss_w(tb + TM_DS, sdesc_sw128(kt_addr + 2048 * k, TILE_B, 1024),
                                sdesc_sw128(v_addr + 2048 * k, TILE_B, 1024), id_ds, k > 0);
-                    mma_commit(ds_full);
+                    mma_commit_w(ds_full);
                     ++lc;
                 }
-                mma_commit(&s_empty[sb]);
-                mma_commit(o_prog);
-                mma_commit(&kv_empty[s]);
+                mma_commit_w(&s_empty[sb]);
+                mma_commit_w(o_prog);
+                mma_commit_w(&kv_empty[s]);
                 if (pv.last) {
-                    mma_commit(&q_empty[pv.tile & 1]);
-                    mma_commit(o_full);
+                    mma_commit_w(&q_empty[pv.tile & 1]);
+                    mma_commit_w(o_full);
                 }
                 return true;
             };
@@ -635,20 +635,20 @@ __global__ void __launch_bounds__(kMainThreads, 1)
                     const TileInfo ti = tile_info(i, p.W, l1_only);
                     const int qb = tile & 1;
                     const uint32_t q_addr = q_base + qb * TILE_B;
-                    if (!(ok = mbar_wait(&q_full[qb], (tile >> 1) & 1, abort, p.status))) break;
+                    if (!(ok = warp_wait(&q_full[qb], (tile >> 1) & 1, abort, p.status))) break;
                     for (int j = 0; j < ti.nk && ok; ++j, ++g) {
                         const int s = g % NS, sb = g & 1;
-                        if (!(ok = mbar_wait(&kv_full[s], (g / NS) & 1, abort, p.status))) break;
+                        if (!(ok = warp_wait(&kv_full[s], (g / NS) & 1, abort, p.status))) break;
                         // the state warps read the leading key tile: hand it on
-                        if (j == 0 && ti.l2) mbar_arrive(lead_ready);
-                        if (!(ok = mbar_wait(&s_empty[sb], ((g >> 1) & 1) ^ 1, abort, p.status))) break;
+                        if (j == 0 && ti.l2) mbar_arrive_w(lead_ready);
+                        if (!(ok = warp_wait(&s_empty[sb], ((g >> 1) & 1) ^ 1, abort, p.status))) break;
                         tc_fence_after();
                         const uint32_t k_addr = kv_base + s * 2 * TILE_B;
 #pragma unroll
                         for (int k = 0; k < 4; ++k)
-                            mma_ss(tb + TM_S + sb * 128, sdesc_sw128(q_addr + 32 * k, 16, 1024),
+                            mma_ss_w(tb + TM_S + sb * 128, sdesc_sw128(q_addr + 32 * k, 16, 1024),
                                    sdesc_sw128(k_addr + 32 * k, 16, 1024), id_qk, k > 0);
-                        mma_commit(&s_full[sb]);
+                        mma_commit_w(&s_full[sb]);
                         if (pend.valid && !(ok = pv_step(pend))) break;
                         pend = {true, j == 0, j == ti.nk - 1, ti.l2, g, tile};
                     }
@@ -656,7 +656,7 @@ __global__ void __launch_bounds__(kMainThreads, 1)
             }
             if (ok && pend.valid) ok = pv_step(pend);
             // nothing may still run on the tensor cores when TMEM is released
-            mma_commit(mma_done);
+            mma_commit_w(mma_done);
             mbar_wait_drain(mma_done, 0);
         }
     } else if (warp >= 4 && warp < 12) {
