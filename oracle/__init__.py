@@ -46,10 +46,10 @@ def _load():
         build()
         lib = ctypes.CDLL(_LIB)
         i64, dp, c_int, c_double = ctypes.c_int64, ctypes.c_void_p, ctypes.c_int, ctypes.c_double
-        lib.oracle_prefill.argtypes = [i64] * 6 + [dp] * 10 + [c_int]
-        lib.oracle_prefill.restype = c_int
-        lib.oracle_decode.argtypes = [i64] * 7 + [dp] * 10 + [c_int]
-        lib.oracle_decode.restype = c_int
+        lib.oracle_prefill_rule.argtypes = [i64] * 6 + [dp] * 10 + [c_int, c_int]
+        lib.oracle_prefill_rule.restype = c_int
+        lib.oracle_decode_rule.argtypes = [i64] * 7 + [dp] * 10 + [c_int, c_int]
+        lib.oracle_decode_rule.restype = c_int
         lib.oracle_scan_tokens.argtypes = [i64, i64, i64, dp, dp, c_double, c_double, c_int, dp]
         lib.oracle_scan_chunks.argtypes = [i64, i64, i64, i64, dp, dp, c_double, c_double, c_int, dp]
         lib.oracle_scan_chunk_mean.argtypes = [i64, i64, i64, i64, dp, dp, c_double, c_double, dp]
@@ -79,12 +79,19 @@ def threads(nthreads: int = 0) -> int:
     return int(_load().oracle_max_threads(int(nthreads)))
 
 
-def prefill(q, k, v, lam, eta, g, W: int, *, parts: bool = False, nthreads: int = 0):
+# Write rules of Fig. 2 step (3): the outer product (the layer as the paper
+# trains it) or the optional delta rule (update = k (x) (v - k^T A)).
+RULES = {"outer": 0, "delta": 1}
+
+
+def prefill(q, k, v, lam, eta, g, W: int, *, parts: bool = False, nthreads: int = 0,
+            rule: str = "outer"):
     """Token-by-token prefill from an empty state.
 
     q, k: [B,H,T,dk]; v: [B,H,T,dv]; lam, eta, g: [H].  Returns
     ``(y [B,H,T,dv], A_final [B,H,dk,dv])`` in float64, plus
     ``(y_local, m)`` when ``parts`` is set (y = y_local + sigmoid(g) m).
+    ``rule`` selects the write of step (3): "outer" or "delta".
     """
     q, k, v = _f64(q), _f64(k), _f64(v)
     lam, eta, g = _f64(lam), _f64(eta), _f64(g)
@@ -96,15 +103,16 @@ def prefill(q, k, v, lam, eta, g, W: int, *, parts: bool = False, nthreads: int 
     A = np.empty((B, H, dk, dv))
     yl = np.empty_like(y) if parts else None
     m = np.empty_like(y) if parts else None
-    rc = _load().oracle_prefill(B, H, T, dk, dv, int(W), _p(q), _p(k), _p(v), _p(lam), _p(eta),
-                                _p(g), _p(y), _p(A), _p(yl) if parts else None,
-                                _p(m) if parts else None, int(nthreads))
+    rc = _load().oracle_prefill_rule(B, H, T, dk, dv, int(W), _p(q), _p(k), _p(v), _p(lam),
+                                     _p(eta), _p(g), _p(y), _p(A), _p(yl) if parts else None,
+                                     _p(m) if parts else None, RULES[rule], int(nthreads))
     if rc != 0:
         raise RuntimeError("oracle_prefill failed")
     return (y, A, yl, m) if parts else (y, A)
 
 
-def decode(ring_k, ring_v, A, t0: int, q, k, v, lam, eta, g, *, nthreads: int = 0):
+def decode(ring_k, ring_v, A, t0: int, q, k, v, lam, eta, g, *, nthreads: int = 0,
+           rule: str = "outer"):
     """``nsteps`` streaming steps from the state (ring_k [B,H,W,dk],
     ring_v [B,H,W,dv], A [B,H,dk,dv], clock t0).  q, k: [nsteps,B,H,dk];
     v: [nsteps,B,H,dv].  Returns ``(y [nsteps,B,H,dv], ring_k, ring_v, A)``
@@ -118,9 +126,9 @@ def decode(ring_k, ring_v, A, t0: int, q, k, v, lam, eta, g, *, nthreads: int = 
     assert q.shape == (n, B, H, dk) and k.shape == (n, B, H, dk) and v.shape == (n, B, H, dv)
     assert A.shape == (B, H, dk, dv)
     y = np.empty((n, B, H, dv))
-    rc = _load().oracle_decode(B, H, dk, dv, W, int(t0), n, _p(ring_k), _p(ring_v), _p(A),
-                               _p(q), _p(k), _p(v), _p(lam), _p(eta), _p(g), _p(y),
-                               int(nthreads))
+    rc = _load().oracle_decode_rule(B, H, dk, dv, W, int(t0), n, _p(ring_k), _p(ring_v), _p(A),
+                                    _p(q), _p(k), _p(v), _p(lam), _p(eta), _p(g), _p(y),
+                                    RULES[rule], int(nthreads))
     if rc != 0:
         raise RuntimeError("oracle_decode failed")
     return y, ring_k, ring_v, A

@@ -45,11 +45,20 @@
 /* One streaming step for one (batch, head): Fig. 2 steps (2)-(5) in order.
  * ring_k [W, dk], ring_v [W, dv], A [dk, dv] are updated in place.
  * s is scratch of length W.  y_local and m may be NULL. */
+/* Write rules of step (3), A <- lam A + eta update(k_old, v_old) (Fig. 2):
+ *   RULE_OUTER: update = k_old (x) v_old, the outer product;
+ *   RULE_DELTA: update = k_old (x) (v_old - k_old^T A), the optional delta
+ *     (Widrow-Hoff error-correcting) rule the figure mentions; the pages give
+ *     no formula, and k_old^T A is read from A before this write (the memory's
+ *     current prediction of v_old from k_old). */
+enum { RULE_OUTER = 0, RULE_DELTA = 1 };
+
 static void tc_step(int64_t t, int64_t dk, int64_t dv, int64_t W,
                     double *ring_k, double *ring_v, double *A,
                     const double *q, const double *k, const double *v,
                     double lam, double eta, double g,
-                    double *y, double *y_local, double *m, double *s)
+                    double *y, double *y_local, double *m, double *s,
+                    int rule, double *u)
 {
     const int64_t pos = t % W;
 
@@ -58,9 +67,18 @@ static void tc_step(int64_t t, int64_t dk, int64_t dv, int64_t W,
     if (t >= W) {
         const double *k_old = ring_k + pos * dk;
         const double *v_old = ring_v + pos * dv;
+        if (rule == RULE_DELTA) {
+            for (int64_t c = 0; c < dv; ++c) {
+                double pred = 0.0;
+                for (int64_t r = 0; r < dk; ++r) pred += k_old[r] * A[r * dv + c];
+                u[c] = v_old[c] - pred;
+            }
+        } else {
+            for (int64_t c = 0; c < dv; ++c) u[c] = v_old[c];
+        }
         for (int64_t r = 0; r < dk; ++r)
             for (int64_t c = 0; c < dv; ++c)
-                A[r * dv + c] = lam * A[r * dv + c] + eta * (k_old[r] * v_old[c]);
+                A[r * dv + c] = lam * A[r * dv + c] + eta * (k_old[r] * u[c]);
     }
 
     /* (4): the new pair takes the freed slot. */
@@ -124,13 +142,14 @@ int oracle_max_threads(int nthreads)
  * A = 0 (§3.2: A_0 = 0).  q,k: [B,H,T,dk]; v: [B,H,T,dv]; lam, eta, g: [H].
  * Outputs y: [B,H,T,dv], A_final: [B,H,dk,dv]; y_local and m (same shape as
  * y) may be NULL.  Returns 0, or -1 on bad sizes / allocation failure. */
-int oracle_prefill(int64_t B, int64_t H, int64_t T, int64_t dk, int64_t dv, int64_t W,
-                   const double *q, const double *k, const double *v,
-                   const double *lam, const double *eta, const double *g,
-                   double *y, double *A_final, double *y_local, double *m,
-                   int nthreads)
+int oracle_prefill_rule(int64_t B, int64_t H, int64_t T, int64_t dk, int64_t dv, int64_t W,
+                        const double *q, const double *k, const double *v,
+                        const double *lam, const double *eta, const double *g,
+                        double *y, double *A_final, double *y_local, double *m,
+                        int rule, int nthreads)
 {
     if (B < 0 || H < 0 || T < 0 || dk < 1 || dv < 1 || W < 1) return -1;
+    if (rule != RULE_OUTER && rule != RULE_DELTA) return -1;
     set_threads(nthreads);
     int err = 0;
 #pragma omp parallel for schedule(dynamic, 1) reduction(| : err)
@@ -139,8 +158,9 @@ int oracle_prefill(int64_t B, int64_t H, int64_t T, int64_t dk, int64_t dv, int6
         double *ring_k = (double *)calloc((size_t)(W * dk), sizeof(double));
         double *ring_v = (double *)calloc((size_t)(W * dv), sizeof(double));
         double *s = (double *)malloc((size_t)W * sizeof(double));
+        double *u = (double *)malloc((size_t)dv * sizeof(double));
         double *A = A_final + bh * dk * dv;
-        if (!ring_k || !ring_v || !s) {
+        if (!ring_k || !ring_v || !s || !u) {
             err |= 1;
         } else {
             memset(A, 0, (size_t)(dk * dv) * sizeof(double));
@@ -148,14 +168,25 @@ int oracle_prefill(int64_t B, int64_t H, int64_t T, int64_t dk, int64_t dv, int6
                 const int64_t rq = (bh * T + t) * dk, rv = (bh * T + t) * dv;
                 tc_step(t, dk, dv, W, ring_k, ring_v, A, q + rq, k + rq, v + rv,
                         lam[h], eta[h], g[h], y + rv,
-                        y_local ? y_local + rv : NULL, m ? m + rv : NULL, s);
+                        y_local ? y_local + rv : NULL, m ? m + rv : NULL, s, rule, u);
             }
         }
         free(ring_k);
         free(ring_v);
         free(s);
+        free(u);
     }
     return err ? -1 : 0;
+}
+
+int oracle_prefill(int64_t B, int64_t H, int64_t T, int64_t dk, int64_t dv, int64_t W,
+                   const double *q, const double *k, const double *v,
+                   const double *lam, const double *eta, const double *g,
+                   double *y, double *A_final, double *y_local, double *m,
+                   int nthreads)
+{
+    return oracle_prefill_rule(B, H, T, dk, dv, W, q, k, v, lam, eta, g, y, A_final, y_local, m,
+                               RULE_OUTER, nthreads);
 }
 
 /* Decode: nsteps streaming steps starting at clock t0 from a given state.
@@ -163,6 +194,38 @@ int oracle_prefill(int64_t B, int64_t H, int64_t T, int64_t dk, int64_t dv, int6
  * q,k: [nsteps,B,H,dk]; v: [nsteps,B,H,dv]; y: [nsteps,B,H,dv].
  * Slot j of the ring holds token j when t0 < W and token t with t mod W = j
  * otherwise (the layout a streaming run leaves behind). */
+int oracle_decode_rule(int64_t B, int64_t H, int64_t dk, int64_t dv, int64_t W,
+                       int64_t t0, int64_t nsteps,
+                       double *ring_k, double *ring_v, double *A,
+                       const double *q, const double *k, const double *v,
+                       const double *lam, const double *eta, const double *g,
+                       double *y, int rule, int nthreads)
+{
+    if (B < 0 || H < 0 || dk < 1 || dv < 1 || W < 1 || t0 < 0 || nsteps < 0) return -1;
+    if (rule != RULE_OUTER && rule != RULE_DELTA) return -1;
+    set_threads(nthreads);
+    int err = 0;
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : err)
+    for (int64_t bh = 0; bh < B * H; ++bh) {
+        const int64_t h = bh % H;
+        double *s = (double *)malloc((size_t)W * sizeof(double));
+        double *u = (double *)malloc((size_t)dv * sizeof(double));
+        if (!s || !u) {
+            err |= 1;
+        } else {
+            for (int64_t i = 0; i < nsteps; ++i) {
+                const int64_t rq = (i * B * H + bh) * dk, rv = (i * B * H + bh) * dv;
+                tc_step(t0 + i, dk, dv, W, ring_k + bh * W * dk, ring_v + bh * W * dv,
+                        A + bh * dk * dv, q + rq, k + rq, v + rv, lam[h], eta[h], g[h],
+                        y + rv, NULL, NULL, s, rule, u);
+            }
+        }
+        free(s);
+        free(u);
+    }
+    return err ? -1 : 0;
+}
+
 int oracle_decode(int64_t B, int64_t H, int64_t dk, int64_t dv, int64_t W,
                   int64_t t0, int64_t nsteps,
                   double *ring_k, double *ring_v, double *A,
@@ -170,26 +233,8 @@ int oracle_decode(int64_t B, int64_t H, int64_t dk, int64_t dv, int64_t W,
                   const double *lam, const double *eta, const double *g,
                   double *y, int nthreads)
 {
-    if (B < 0 || H < 0 || dk < 1 || dv < 1 || W < 1 || t0 < 0 || nsteps < 0) return -1;
-    set_threads(nthreads);
-    int err = 0;
-#pragma omp parallel for schedule(dynamic, 1) reduction(| : err)
-    for (int64_t bh = 0; bh < B * H; ++bh) {
-        const int64_t h = bh % H;
-        double *s = (double *)malloc((size_t)W * sizeof(double));
-        if (!s) {
-            err |= 1;
-        } else {
-            for (int64_t i = 0; i < nsteps; ++i) {
-                const int64_t rq = (i * B * H + bh) * dk, rv = (i * B * H + bh) * dv;
-                tc_step(t0 + i, dk, dv, W, ring_k + bh * W * dk, ring_v + bh * W * dv,
-                        A + bh * dk * dv, q + rq, k + rq, v + rv, lam[h], eta[h], g[h],
-                        y + rv, NULL, NULL, s);
-            }
-        }
-        free(s);
-    }
-    return err ? -1 : 0;
+    return oracle_decode_rule(B, H, dk, dv, W, t0, nsteps, ring_k, ring_v, A, q, k, v, lam, eta,
+                              g, y, RULE_OUTER, nthreads);
 }
 
 /* ------------------------------------------------------------------------

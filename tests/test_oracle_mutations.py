@@ -23,8 +23,16 @@ MUTATIONS = {
     "missing 1/sqrt(d_k)":
         ("const double scale = 1.0 / sqrt((double)dk);", "const double scale = 1.0;"),
     "dropped decay":
-        ("A[r * dv + c] = lam * A[r * dv + c] + eta * (k_old[r] * v_old[c]);",
-         "A[r * dv + c] = A[r * dv + c] + eta * (k_old[r] * v_old[c]);"),
+        ("A[r * dv + c] = lam * A[r * dv + c] + eta * (k_old[r] * u[c]);",
+         "A[r * dv + c] = A[r * dv + c] + eta * (k_old[r] * u[c]);"),
+    "delta rule: correction with the wrong sign":
+        ("u[c] = v_old[c] - pred;", "u[c] = v_old[c] + pred;"),
+    "delta rule: prediction from the decayed state":
+        ("for (int64_t r = 0; r < dk; ++r) pred += k_old[r] * A[r * dv + c];",
+         "for (int64_t r = 0; r < dk; ++r) pred += k_old[r] * lam * A[r * dv + c];"),
+    "delta rule: transposed prediction":
+        ("for (int64_t r = 0; r < dk; ++r) pred += k_old[r] * A[r * dv + c];",
+         "for (int64_t r = 0; r < dk && r < dv && c < dk; ++r) pred += k_old[r] * A[c * dv + r];"),
     "gate sign":
         ("const double gate = 1.0 / (1.0 + exp(-g));", "const double gate = 1.0 / (1.0 + exp(g));"),
     "window one key short":
@@ -57,6 +65,10 @@ PIN_CALLS = [
     pins.test_chunk_mean_with_decay_drops_per_token_weights,
     pins.test_golden_hand_d1_w1,
     pins.test_golden_hand_d2_w2,
+    lambda: pins.test_delta_rule_repeated_write_closed_form(1.0, 1.0, 3),
+    lambda: pins.test_delta_rule_repeated_write_closed_form(1.0, 0.5, 4),
+    lambda: pins.test_delta_rule_repeated_write_closed_form(0.9, 0.3, 6),
+    pins.test_delta_rule_equals_outer_product_on_orthonormal_keys,
 ]
 
 
@@ -84,8 +96,8 @@ def test_pins_catch_planted_mistake(name, tmp_path):
     so = _build_mutant(tmp_path, old, new)
     good = oracle._load()
     mut = ctypes.CDLL(so)
-    for fn in ("oracle_prefill", "oracle_decode", "oracle_scan_tokens", "oracle_scan_chunks",
-               "oracle_scan_chunk_mean", "oracle_max_threads"):
+    for fn in ("oracle_prefill_rule", "oracle_decode_rule", "oracle_scan_tokens",
+               "oracle_scan_chunks", "oracle_scan_chunk_mean", "oracle_max_threads"):
         getattr(mut, fn).argtypes = getattr(good, fn).argtypes
         getattr(mut, fn).restype = getattr(good, fn).restype
     failed = []

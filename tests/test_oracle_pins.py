@@ -166,6 +166,72 @@ def test_exact_recall_orthonormal_keys():
         np.testing.assert_allclose(m[0, h, T - 1], vals[h], rtol=0, atol=1e-14)
 
 
+# --- the optional delta-rule write (Fig. 2 step (3)) ------------------------
+
+@pytest.mark.parametrize("lam,eta,n", [(1.0, 1.0, 3), (1.0, 0.5, 4), (0.9, 0.3, 6)])
+def test_delta_rule_repeated_write_closed_form(lam, eta, n):
+    """The same pair (unit key k, value v) written n times: with A = a k v^T
+    the delta write gives a_n = (lam - eta) a_{n-1} + eta, so a_n =
+    eta (1 - (lam - eta)^n) / (1 - (lam - eta)).  The outer product gives
+    a_n = lam a_{n-1} + eta instead.  W = 1: token t evicts token t-1, so
+    n + 1 identical tokens make n writes."""
+    dk, dv = 4, 3
+    rng = np.random.default_rng(11)
+    kvec = rng.standard_normal(dk)
+    kvec /= np.linalg.norm(kvec)
+    vvec = rng.standard_normal(dv)
+    T = n + 1
+    q = np.zeros((1, 1, T, dk))
+    k = np.tile(kvec, (1, 1, T, 1))
+    v = np.tile(vvec, (1, 1, T, 1))
+    prm = [np.array([lam]), np.array([eta]), np.zeros(1)]
+    r = lam - eta
+    a_delta = eta * n if abs(1 - r) < 1e-15 else eta * (1 - r ** n) / (1 - r)
+    a_outer = sum(eta * lam ** j for j in range(n))
+    _, A_d = oracle.prefill(q, k, v, *prm, 1, rule="delta")
+    _, A_o = oracle.prefill(q, k, v, *prm, 1, rule="outer")
+    np.testing.assert_allclose(A_d[0, 0], a_delta * np.outer(kvec, vvec), rtol=0, atol=1e-13)
+    np.testing.assert_allclose(A_o[0, 0], a_outer * np.outer(kvec, vvec), rtol=0, atol=1e-13)
+
+
+def test_delta_rule_equals_outer_product_on_orthonormal_keys():
+    """Each evicted key orthogonal to every earlier one: k^T A = 0 before each
+    write, so the delta write adds the same k v^T as the outer product."""
+    dk, dv, E, W = 8, 3, 6, 2
+    rng = np.random.default_rng(12)
+    Qm, _ = np.linalg.qr(rng.standard_normal((dk, dk)))
+    T = E + W
+    q = rng.standard_normal((1, 2, T, dk))
+    k = np.zeros((1, 2, T, dk))
+    k[0, :, :E] = Qm.T[:E]
+    v = rng.standard_normal((1, 2, T, dv))
+    prm = [np.array([1.0, 1.0]), np.array([1.0, 1.0]), np.array([0.3, -0.2])]
+    y_d, A_d = oracle.prefill(q, k, v, *prm, W, rule="delta")
+    y_o, A_o = oracle.prefill(q, k, v, *prm, W, rule="outer")
+    np.testing.assert_allclose(A_d, A_o, rtol=0, atol=1e-13)
+    np.testing.assert_allclose(y_d, y_o, rtol=0, atol=1e-13)
+
+
+def test_delta_rule_decode_continues_prefill():
+    """The streaming form and the prefill form run the same token loop."""
+    x = wl.random_prefill(1, 2, 50, 6, 5, 7, 4, dtype="f32", seed=13)
+    T0 = 30
+    y_full, A_full = oracle.prefill(x.q, x.k, x.v, x.lam, x.eta, x.g, 7, rule="delta")
+    _, A0 = oracle.prefill(x.q[:, :, :T0], x.k[:, :, :T0], x.v[:, :, :T0], x.lam, x.eta, x.g,
+                           7, rule="delta")
+    ring_k = np.zeros((1, 2, 7, 6))
+    ring_v = np.zeros((1, 2, 7, 5))
+    for j in range(T0 - 7, T0):
+        ring_k[:, :, j % 7] = x.k[:, :, j].double().numpy()
+        ring_v[:, :, j % 7] = x.v[:, :, j].double().numpy()
+    y, _, _, A = oracle.decode(ring_k, ring_v, A0, T0, x.q[:, :, T0:].permute(2, 0, 1, 3),
+                               x.k[:, :, T0:].permute(2, 0, 1, 3),
+                               x.v[:, :, T0:].permute(2, 0, 1, 3), x.lam, x.eta, x.g,
+                               rule="delta")
+    np.testing.assert_allclose(y.transpose(1, 2, 0, 3), y_full[:, :, T0:], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(A, A_full, rtol=0, atol=1e-12)
+
+
 # --- training form: chunk scan and the chunk-mean shortcut -----------------
 
 @pytest.mark.parametrize("C", [1, 7, 16, 64, 300])
