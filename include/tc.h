@@ -80,6 +80,11 @@ typedef enum tc_dtype {
                                     computed (the chunk scan over the call's
                                     evictions); q and y are not used and may be
                                     NULL.  Not combinable with L1_ONLY. */
+#define TC_PREFILL_DELTA_RULE 4u /* write evictions with the delta rule
+                                    (TC_WRITE_DELTA below) instead of the outer
+                                    product.  Each write then reads A, so the
+                                    chunk scan does not apply: the portable path
+                                    runs the writes of a head in token order. */
 
 /* Shapes of one prefill call.  Supported: B, H >= 1; T >= 0; 1 <= d_k, d_v
  * <= 128; W >= 1; C >= 1. */
@@ -221,6 +226,15 @@ TC_API tc_status tc_prefill_no_alloc(const tc_prefill_desc *desc, const void *q,
  *   t: number of tokens consumed so far (the next step's clock).
  * A prefill over T tokens continues as a stream with t = T, A = A_final and
  * token j (for the last min(T,W) tokens) copied to slot j mod W. */
+/* Write rule of Fig. 2 step (3), A <- lambda A + eta update(k_old, v_old):
+ *   TC_WRITE_OUTER  update = k_old v_old^T (the paper's layer);
+ *   TC_WRITE_DELTA  update = k_old (v_old - k_old^T A)^T, the optional delta
+ *                   (Widrow-Hoff error-correcting) rule the figure mentions.
+ *                   The pages give no formula; k_old^T A is read from A
+ *                   before the write, i.e. the memory's current prediction
+ *                   of v_old from k_old. */
+typedef enum tc_write_rule { TC_WRITE_OUTER = 0, TC_WRITE_DELTA = 1 } tc_write_rule;
+
 typedef struct tc_decode_state {
     int64_t B, H, dk, dv, W;
     int64_t t;
@@ -231,11 +245,13 @@ typedef struct tc_decode_state {
     const float *lambda; /* [H] */
     const float *eta;    /* [H] */
     const float *g;      /* [H] */
+    tc_write_rule write_rule; /* TC_WRITE_OUTER (0, the paper's layer) or TC_WRITE_DELTA */
 } tc_decode_state;
 
 /* One streaming step (§3.2, Fig. 2) for every (b,h), in the paper's order:
  * (2) if t >= W the pair in slot pos = t mod W is evicted, (3) written
- * A <- lambda A + eta k_old v_old^T, (4) (k_t, v_t) is stored in slot pos,
+ * A <- lambda A + eta k_old v_old^T (or the delta update of write_rule),
+ * (4) (k_t, v_t) is stored in slot pos,
  * (5) y_t = softmax-attention(q_t, filled slots) + sigmoid(g) q_t A.
  * Before the ring fills (t < W) slots t+1..W-1 are masked out.
  *

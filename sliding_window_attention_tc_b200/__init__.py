@@ -40,6 +40,8 @@ STATUS_NAMES = {0: "TC_OK", 1: "TC_ERR_INVALID_ARG", 2: "TC_ERR_UNSUPPORTED",
 TC_F32, TC_BF16 = 0, 1
 TC_PREFILL_L1_ONLY = 1
 TC_PREFILL_STATE_ONLY = 2
+TC_PREFILL_DELTA_RULE = 4
+TC_WRITE_OUTER, TC_WRITE_DELTA = 0, 1
 
 # Exported C symbols declared in include/tc.h.
 EXPORTED = ("tc_prefill_workspace_size", "tc_prefill", "tc_prefill_launch_count", "tc_prefill_host_workspace_size",
@@ -60,7 +62,8 @@ class DecodeStateC(ctypes.Structure):
                 ("dv", ctypes.c_int64), ("W", ctypes.c_int64), ("t", ctypes.c_int64),
                 ("kv_dtype", ctypes.c_int), ("ring_k", ctypes.c_void_p),
                 ("ring_v", ctypes.c_void_p), ("A", ctypes.c_void_p),
-                ("lam", ctypes.c_void_p), ("eta", ctypes.c_void_p), ("g", ctypes.c_void_p)]
+                ("lam", ctypes.c_void_p), ("eta", ctypes.c_void_p), ("g", ctypes.c_void_p),
+                ("write_rule", ctypes.c_int)]
 
 
 _vp, _sz, _int = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int
@@ -152,8 +155,9 @@ def _contig(*ts):
 
 
 def make_prefill_desc(B, H, T, dk, dv, W, C, dtype: int, l1_only: bool = False,
-                      state_only: bool = False) -> PrefillDesc:
-    flags = (TC_PREFILL_L1_ONLY if l1_only else 0) | (TC_PREFILL_STATE_ONLY if state_only else 0)
+                      state_only: bool = False, delta_rule: bool = False) -> PrefillDesc:
+    flags = ((TC_PREFILL_L1_ONLY if l1_only else 0) | (TC_PREFILL_STATE_ONLY if state_only else 0)
+             | (TC_PREFILL_DELTA_RULE if delta_rule else 0))
     return PrefillDesc(int(B), int(H), int(T), int(dk), int(dv), int(W), int(C), int(dtype),
                        flags)
 
@@ -165,19 +169,21 @@ def prefill_workspace_size(desc: PrefillDesc) -> int:
     return int(n)
 
 
-def _desc_of(q, v, W, C, l1_only):
+def _desc_of(q, v, W, C, l1_only, delta_rule=False):
     B, H, T, dk = q.shape
-    return make_prefill_desc(B, H, T, dk, v.shape[-1], W, C, _dtype_code(q), l1_only)
+    return make_prefill_desc(B, H, T, dk, v.shape[-1], W, C, _dtype_code(q), l1_only,
+                             delta_rule=delta_rule)
 
 
 def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, lam: torch.Tensor,
             eta: torch.Tensor, g: torch.Tensor, W: int, C: int, *, l1_only: bool = False,
-            y: Optional[torch.Tensor] = None, A_final: Optional[torch.Tensor] = None,
-            workspace: Optional[torch.Tensor] = None, stream=None):
+            delta_rule: bool = False, y: Optional[torch.Tensor] = None,
+            A_final: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+            stream=None):
     """tc_prefill on device tensors q, k [B,H,T,dk], v [B,H,T,dv] (float32 or
     bfloat16), lam, eta, g [H] float32.  Returns (y, A_final); A_final is
-    None with l1_only."""
-    desc = _desc_of(q, v, W, C, l1_only)
+    None with l1_only.  delta_rule selects the delta-rule write."""
+    desc = _desc_of(q, v, W, C, l1_only, delta_rule)
     B, H, T, dk = q.shape
     dv = v.shape[-1]
     if y is None:
@@ -201,7 +207,8 @@ def prefill_from_state(q: Optional[torch.Tensor], k: torch.Tensor, v: torch.Tens
                        t0: int, halo_k: Optional[torch.Tensor] = None,
                        halo_v: Optional[torch.Tensor] = None, A_init: Optional[torch.Tensor] = None,
                        *, state_only: bool = False, l1_only: bool = False,
-                       y: Optional[torch.Tensor] = None, A_final: Optional[torch.Tensor] = None,
+                       delta_rule: bool = False, y: Optional[torch.Tensor] = None,
+                       A_final: Optional[torch.Tensor] = None,
                        workspace: Optional[torch.Tensor] = None, stream=None):
     """tc_prefill_from_state: the layer over the new tokens k, v [B,H,T,d]
     (queries q, unless state_only) starting at global position t0, given the
@@ -210,7 +217,8 @@ def prefill_from_state(q: Optional[torch.Tensor], k: torch.Tensor, v: torch.Tens
     (y, A_final); y is None with state_only."""
     B, H, T, dk = k.shape
     dv = v.shape[-1]
-    desc = make_prefill_desc(B, H, T, dk, dv, W, C, _dtype_code(k), l1_only, state_only)
+    desc = make_prefill_desc(B, H, T, dk, dv, W, C, _dtype_code(k), l1_only, state_only,
+                             delta_rule)
     if y is None and not state_only:
         y = torch.empty((B, H, T, dv), dtype=k.dtype, device=k.device)
     if A_final is None and not l1_only:
@@ -303,7 +311,8 @@ def prefill_host(q, k, v, lam, eta, g, W, C, y, A_final=None, *, workspace, l1_o
 class DecodeState:
     """Streaming state (caller-owned device tensors, updated in place):
     ring_k [B,H,W,dk], ring_v [B,H,W,dv], A [B,H,dk,dv] float32, lam/eta/g
-    [H] float32 and the clock t (tokens consumed so far)."""
+    [H] float32, the clock t (tokens consumed so far) and the write rule
+    (TC_WRITE_OUTER, the paper's layer, or TC_WRITE_DELTA)."""
     ring_k: torch.Tensor
     ring_v: torch.Tensor
     A: torch.Tensor
@@ -311,6 +320,7 @@ class DecodeState:
     eta: torch.Tensor
     g: torch.Tensor
     t: int
+    write_rule: int = 0
 
     def c_struct(self) -> DecodeStateC:
         B, H, W, dk = self.ring_k.shape
@@ -318,7 +328,8 @@ class DecodeState:
         _contig(self.ring_k, self.ring_v, self.A, self.lam, self.eta, self.g)
         return DecodeStateC(B, H, dk, dv, W, int(self.t), _dtype_code(self.ring_k),
                             self.ring_k.data_ptr(), self.ring_v.data_ptr(), self.A.data_ptr(),
-                            self.lam.data_ptr(), self.eta.data_ptr(), self.g.data_ptr())
+                            self.lam.data_ptr(), self.eta.data_ptr(), self.g.data_ptr(),
+                            int(self.write_rule))
 
     @staticmethod
     def empty(B, H, W, dk, dv, lam, eta, g, dtype=torch.bfloat16, device="cuda"):

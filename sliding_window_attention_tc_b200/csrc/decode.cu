@@ -41,6 +41,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(DecodeParams p) {
 
     __shared__ float s_q[D], s_kn[D], s_vn[D], s_ko[D], s_vo[D];
     __shared__ float s_mp[RG][D];
+    __shared__ float s_pd[RG][D];  // delta rule: partial predictions k_old^T A
     __shared__ float s_gm[NG], s_gl[NG];
     __shared__ __align__(16) float s_acc[NG][D];
 
@@ -83,7 +84,33 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(DecodeParams p) {
             if (r < D) a[i] = A4[r * CG + cg];
         }
         float4 mp = make_float4(0.f, 0.f, 0.f, 0.f);
-        const float4 vo = reinterpret_cast<const float4 *>(s_vo)[cg];
+        float4 vo = reinterpret_cast<const float4 *>(s_vo)[cg];
+        if (p.write_rule == TC_WRITE_DELTA && evict) {
+            // delta rule: the written value is v_old - k_old^T A, with A read
+            // before this write (uniform branch: rule and clock are per CTA)
+            float4 pp = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+            for (int i = 0; i < RPT; ++i) {
+                const int r = rg + i * RG;
+                if (r < D) {
+                    const float kr = s_ko[r];
+                    pp.x = fmaf(kr, a[i].x, pp.x);
+                    pp.y = fmaf(kr, a[i].y, pp.y);
+                    pp.z = fmaf(kr, a[i].z, pp.z);
+                    pp.w = fmaf(kr, a[i].w, pp.w);
+                }
+            }
+            reinterpret_cast<float4 *>(&s_pd[rg][0])[cg] = pp;
+            __syncthreads();
+#pragma unroll
+            for (int g = 0; g < RG; ++g) {
+                const float4 x = reinterpret_cast<const float4 *>(&s_pd[g][0])[cg];
+                vo.x -= x.x;
+                vo.y -= x.y;
+                vo.z -= x.z;
+                vo.w -= x.w;
+            }
+        }
 #pragma unroll
         for (int i = 0; i < RPT; ++i) {
             const int r = rg + i * RG;

@@ -123,9 +123,13 @@ __device__ __forceinline__ float warp_sum(float x) {
 }
 
 // One warp per query row, ROWS consecutive rows per CTA sharing key tiles.
+// mrow: with the delta-rule write, m_t of every new row from
+// delta_l2_kernel (the L2 read is then taken from there, not from chunk
+// states); null for the outer-product write.
 template <typename Tin>
 __global__ void __launch_bounds__(kThreads) prefill_rows_kernel(PrefillParams p,
-                                                                const float *states, int64_t nC) {
+                                                                const float *states, int64_t nC,
+                                                                const float *mrow) {
     constexpr int ROWS = kThreads / 32, KT = 32, CPL = kMaxD / 32;
     __shared__ float sk[KT][kMaxD + 1], sv[KT][kMaxD + 1];
     __shared__ float sq[ROWS][kMaxD];
@@ -152,7 +156,7 @@ __global__ void __launch_bounds__(kThreads) prefill_rows_kernel(PrefillParams p,
     const float scale = (float)(1.4426950408889634 / sqrt((double)dk));
     const int64_t win_lo = t - W + 1 > 0 ? t - W + 1 : 0;
     const int64_t e = t - W;                       // eviction read at step t
-    const bool has_l2 = use_l2 && row_ok && e >= 0;
+    const bool has_l2 = use_l2 && row_ok && e >= 0 && !mrow;
     const int64_t ch = has_l2 ? e / C : 0;
     const int64_t intra_lo = ch * C;
 
@@ -214,6 +218,15 @@ __global__ void __launch_bounds__(kThreads) prefill_rows_kernel(PrefillParams p,
     if (!row_ok) return;
 
     float gate = 0.f;
+    if (mrow && use_l2 && e >= 0) {
+        gate = sigmoidf_acc(p.g[h]);
+        const float *mr = mrow + (bh * T_new + (t - nh)) * dv;
+#pragma unroll
+        for (int i = 0; i < CPL; ++i) {
+            const int c = lane + 32 * i;
+            if (c < dv) macc[i] = mr[c];
+        }
+    }
     if (has_l2) {
         // inter-chunk read: lambda^{r+1} q_t S_c
         gate = sigmoidf_acc(p.g[h]);
@@ -239,10 +252,79 @@ __global__ void __launch_bounds__(kThreads) prefill_rows_kernel(PrefillParams p,
     }
 }
 
+// Delta-rule write (Fig. 2 step (3) with update = k_old (v_old - k_old^T A)^T):
+// each write reads A, so the writes of one (b,h) run in token order here.  A
+// lives in shared memory; for every new row t with an eviction behind it the
+// kernel records m_t = q_t A_t in mrow, and it leaves A_final.
+template <typename T>
+__global__ void __launch_bounds__(kThreads) delta_l2_kernel(PrefillParams p, float *mrow) {
+    extern __shared__ float sA[];  // [dk][dv]
+    __shared__ float sk[kMaxD], sv[kMaxD], sq[kMaxD], su[kMaxD];
+    const int tid = threadIdx.x;
+    const int64_t bh = blockIdx.x;
+    const int h = (int)(bh % p.H);
+    const int dk = p.dk, dv = p.dv, nel = dk * dv;
+    const int64_t nh = p.n_halo, T_new = p.T, T_all = nh + T_new, W = p.W;
+    const float lam = p.lam[h], eta = p.eta[h];
+    for (int x = tid; x < nel; x += kThreads) sA[x] = p.A_init ? p.A_init[bh * nel + x] : 0.f;
+    const T *qb = reinterpret_cast<const T *>(p.q) + bh * T_new * dk;
+    // tokens before max(W, n_halo) neither evict nor have a query to answer
+    for (int64_t tau = (W > nh ? W : nh) < T_all ? (W > nh ? W : nh) : T_all; tau < T_all; ++tau) {
+        const bool evict = tau >= W;
+        const bool query = !p.state_only;
+        __syncthreads();
+        if (evict) {
+            for (int x = tid; x < dk; x += kThreads)
+                sk[x] = to_f32(kv_row<T>(p.halo_k, p.k, bh, nh, T_new, dk, tau - W)[x]);
+            for (int x = tid; x < dv; x += kThreads)
+                sv[x] = to_f32(kv_row<T>(p.halo_v, p.v, bh, nh, T_new, dv, tau - W)[x]);
+        }
+        if (query)
+            for (int x = tid; x < dk; x += kThreads) sq[x] = to_f32(qb[(tau - nh) * dk + x]);
+        __syncthreads();
+        if (evict) {
+            for (int c = tid; c < dv; c += kThreads) {
+                float pred = 0.f;
+                for (int r = 0; r < dk; ++r) pred = fmaf(sk[r], sA[r * dv + c], pred);
+                su[c] = sv[c] - pred;
+            }
+            __syncthreads();
+            for (int x = tid; x < nel; x += kThreads)
+                sA[x] = fmaf(lam, sA[x], eta * sk[x / dv] * su[x % dv]);
+            __syncthreads();
+        }
+        if (query) {
+            for (int c = tid; c < dv; c += kThreads) {
+                float m = 0.f;
+                for (int r = 0; r < dk; ++r) m = fmaf(sq[r], sA[r * dv + c], m);
+                mrow[(bh * T_new + (tau - nh)) * dv + c] = m;
+            }
+        }
+    }
+    __syncthreads();
+    if (p.A_final)
+        for (int x = tid; x < nel; x += kThreads) p.A_final[bh * nel + x] = sA[x];
+}
+
 template <typename T>
 cudaError_t launch_t(const PrefillParams &p, cudaStream_t s) {
     const int64_t BH = p.B * p.H;
     if (BH == 0) return cudaSuccess;
+    if (p.delta_rule && !p.l1_only) {
+        float *mrow = reinterpret_cast<float *>(p.workspace);
+        const size_t smem = (size_t)p.dk * p.dv * sizeof(float);
+        cudaError_t e = cudaFuncSetAttribute(delta_l2_kernel<T>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        delta_l2_kernel<T><<<(unsigned)BH, kThreads, smem, s>>>(p, mrow);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+        if (p.T > 0 && !p.state_only) {
+            const dim3 grid((unsigned)((p.T + 7) / 8), (unsigned)BH);
+            prefill_rows_kernel<T><<<grid, kThreads, 0, s>>>(p, nullptr, 0, mrow);
+        }
+        return cudaGetLastError();
+    }
     const int64_t nC = p.l1_only ? 0 : num_chunks(evictions(p.T + p.n_halo, p.W), p.C);
     float *states = reinterpret_cast<float *>(p.workspace);
     if (!p.l1_only) {
@@ -252,7 +334,7 @@ cudaError_t launch_t(const PrefillParams &p, cudaStream_t s) {
     }
     if (p.T > 0 && !p.state_only) {
         const dim3 grid((unsigned)((p.T + 7) / 8), (unsigned)BH);
-        prefill_rows_kernel<T><<<grid, kThreads, 0, s>>>(p, states, nC);
+        prefill_rows_kernel<T><<<grid, kThreads, 0, s>>>(p, states, nC, nullptr);
     }
     return cudaGetLastError();
 }
@@ -261,6 +343,8 @@ cudaError_t launch_t(const PrefillParams &p, cudaStream_t s) {
 
 size_t portable_workspace_bytes(const tc_prefill_desc &d, int64_t n_halo) {
     if (d.flags & TC_PREFILL_L1_ONLY) return 0;
+    if (d.flags & TC_PREFILL_DELTA_RULE)  // m_t of every new row
+        return (d.flags & TC_PREFILL_STATE_ONLY) ? 0 : (size_t)(d.B * d.H * d.T * d.dv) * sizeof(float);
     const int64_t nC = num_chunks(evictions(d.T + n_halo, d.W), d.C);
     return (size_t)(d.B * d.H * nC * d.dk * d.dv) * sizeof(float);
 }

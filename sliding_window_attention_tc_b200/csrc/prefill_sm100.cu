@@ -981,7 +981,8 @@ int choose_spans(int64_t BH, int nT, int num_sms) {
 bool sm100_supported(const tc_prefill_desc &d, int64_t n_halo) {
     return d.dtype == TC_BF16 && d.dk == HD && d.dv == HD && d.W >= BM && d.W % BM == 0 &&
            d.T >= 1 && d.T + n_halo <= (int64_t(1) << 30) && d.B * d.H <= 65535 &&
-           (n_halo == 0 || n_halo == d.W) && !(d.flags & TC_PREFILL_STATE_ONLY);
+           (n_halo == 0 || n_halo == d.W) &&
+           !(d.flags & (TC_PREFILL_STATE_ONLY | TC_PREFILL_DELTA_RULE));
 }
 
 // Spans are cut over the new query tiles only (the halo has no queries).

@@ -33,7 +33,8 @@ tc_status check_desc(const tc_prefill_desc *d) {
     if (d->B < 1 || d->H < 1 || d->T < 0 || d->dk < 1 || d->dv < 1 || d->W < 1 || d->C < 1)
         return TC_ERR_INVALID_ARG;
     if (!valid_dtype(d->dtype)) return TC_ERR_INVALID_ARG;
-    if (d->flags & ~(TC_PREFILL_L1_ONLY | TC_PREFILL_STATE_ONLY)) return TC_ERR_INVALID_ARG;
+    if (d->flags & ~(TC_PREFILL_L1_ONLY | TC_PREFILL_STATE_ONLY | TC_PREFILL_DELTA_RULE))
+        return TC_ERR_INVALID_ARG;
     if ((d->flags & TC_PREFILL_L1_ONLY) && (d->flags & TC_PREFILL_STATE_ONLY))
         return TC_ERR_INVALID_ARG;
     if (d->dk > kMaxDim || d->dv > kMaxDim) return TC_ERR_UNSUPPORTED;
@@ -103,6 +104,7 @@ tc_status check_decode_state(const tc_decode_state *s) {
     if (s->B < 1 || s->H < 1 || s->dk < 1 || s->dv < 1 || s->W < 1 || s->t < 0)
         return TC_ERR_INVALID_ARG;
     if (!valid_dtype(s->kv_dtype)) return TC_ERR_INVALID_ARG;
+    if (s->write_rule != TC_WRITE_OUTER && s->write_rule != TC_WRITE_DELTA) return TC_ERR_INVALID_ARG;
     if (!s->ring_k || !s->ring_v || !s->A || !s->lambda || !s->eta || !s->g)
         return TC_ERR_INVALID_ARG;
     if (!aligned16(s->ring_k) || !aligned16(s->ring_v) || !aligned16(s->A))
@@ -202,6 +204,7 @@ tc_status prefill_impl(const tc_prefill_desc *d, int64_t t0, const void *halo_k,
     p.dv = (int)d->dv;
     p.l1_only = l1_only;
     p.state_only = state_only;
+    p.delta_rule = (d->flags & TC_PREFILL_DELTA_RULE) != 0;
     p.halo_k = n_halo > 0 ? halo_k : nullptr;
     p.halo_v = n_halo > 0 ? halo_v : nullptr;
     p.n_halo = n_halo;
@@ -340,6 +343,7 @@ tc_status decode_impl(tc_decode_state *s, int64_t *t_rows, const void *q_t, cons
     p.W = s->W;
     p.t = s->t;
     p.t_rows = t_rows;
+    p.write_rule = (int)s->write_rule;
     p.dk = (int)s->dk;
     p.dv = (int)s->dv;
     p.status = status_ptr();

@@ -69,6 +69,7 @@ struct DecodeParams {
     const float *lam, *eta, *g;
     int64_t H, W, t;
     const int64_t *t_rows;  // per batch row clocks (device), or null: every row at t
+    int write_rule;         // TC_WRITE_OUTER or TC_WRITE_DELTA
     int dk, dv;
     int *status;
 };
@@ -87,6 +88,7 @@ struct PrefillParams {
     int dk, dv;
     bool l1_only;
     bool state_only;  // A_final only (the chunk scan); q and y unused
+    bool delta_rule;  // write of Fig. 2 step (3): delta rule instead of the outer product
     const void *halo_k, *halo_v;
     int64_t n_halo;
     const float *A_init;
