@@ -85,6 +85,14 @@ typedef enum tc_dtype {
                                     product.  Each write then reads A, so the
                                     chunk scan does not apply: the portable path
                                     runs the writes of a head in token order. */
+#define TC_PREFILL_CHUNK_MEAN 8u /* ablation, with TC_PREFILL_STATE_ONLY only:
+                                    the chunk-mean shortcut the paper warns
+                                    against (abstract; §1), A <- lambda A +
+                                    eta kbar vbar^T once per chunk of C
+                                    evictions (kbar, vbar the chunk's means),
+                                    instead of the exact weighted sum.  It adds
+                                    C^2 - C spurious cross terms per chunk; it
+                                    exists to measure that error. */
 
 /* Shapes of one prefill call.  Supported: B, H >= 1; T >= 0; 1 <= d_k, d_v
  * <= 128; W >= 1; C >= 1. */

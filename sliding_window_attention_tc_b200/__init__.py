@@ -41,6 +41,7 @@ TC_F32, TC_BF16 = 0, 1
 TC_PREFILL_L1_ONLY = 1
 TC_PREFILL_STATE_ONLY = 2
 TC_PREFILL_DELTA_RULE = 4
+TC_PREFILL_CHUNK_MEAN = 8
 TC_WRITE_OUTER, TC_WRITE_DELTA = 0, 1
 
 # Exported C symbols declared in include/tc.h.
@@ -155,9 +156,11 @@ def _contig(*ts):
 
 
 def make_prefill_desc(B, H, T, dk, dv, W, C, dtype: int, l1_only: bool = False,
-                      state_only: bool = False, delta_rule: bool = False) -> PrefillDesc:
+                      state_only: bool = False, delta_rule: bool = False,
+                      chunk_mean: bool = False) -> PrefillDesc:
     flags = ((TC_PREFILL_L1_ONLY if l1_only else 0) | (TC_PREFILL_STATE_ONLY if state_only else 0)
-             | (TC_PREFILL_DELTA_RULE if delta_rule else 0))
+             | (TC_PREFILL_DELTA_RULE if delta_rule else 0)
+             | (TC_PREFILL_CHUNK_MEAN if chunk_mean else 0))
     return PrefillDesc(int(B), int(H), int(T), int(dk), int(dv), int(W), int(C), int(dtype),
                        flags)
 
@@ -207,7 +210,8 @@ def prefill_from_state(q: Optional[torch.Tensor], k: torch.Tensor, v: torch.Tens
                        t0: int, halo_k: Optional[torch.Tensor] = None,
                        halo_v: Optional[torch.Tensor] = None, A_init: Optional[torch.Tensor] = None,
                        *, state_only: bool = False, l1_only: bool = False,
-                       delta_rule: bool = False, y: Optional[torch.Tensor] = None,
+                       delta_rule: bool = False, chunk_mean: bool = False,
+                       y: Optional[torch.Tensor] = None,
                        A_final: Optional[torch.Tensor] = None,
                        workspace: Optional[torch.Tensor] = None, stream=None):
     """tc_prefill_from_state: the layer over the new tokens k, v [B,H,T,d]
@@ -218,7 +222,7 @@ def prefill_from_state(q: Optional[torch.Tensor], k: torch.Tensor, v: torch.Tens
     B, H, T, dk = k.shape
     dv = v.shape[-1]
     desc = make_prefill_desc(B, H, T, dk, dv, W, C, _dtype_code(k), l1_only, state_only,
-                             delta_rule)
+                             delta_rule, chunk_mean)
     if y is None and not state_only:
         y = torch.empty((B, H, T, dv), dtype=k.dtype, device=k.device)
     if A_final is None and not l1_only:

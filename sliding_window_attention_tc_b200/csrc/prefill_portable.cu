@@ -75,6 +75,7 @@ __global__ void __launch_bounds__(kThreads) chunk_state_kernel(PrefillParams p, 
         const int64_t Cc = (E - c0 < C) ? E - c0 : C;
 #pragma unroll
         for (int i = 0; i < kMaxPerThread; ++i) D[i] = 0.f;
+        float Vs = 0.f;  // chunk-mean ablation: sum of the chunk's values in column col
         for (int64_t i0 = 0; i0 < Cc; i0 += KT) {
             const int nt = (int)((Cc - i0 < KT) ? Cc - i0 : KT);
             __syncthreads();
@@ -84,9 +85,21 @@ __global__ void __launch_bounds__(kThreads) chunk_state_kernel(PrefillParams p, 
             for (int x = tid; x < nt * dv; x += kThreads)
                 sv[x / dv][x % dv] = to_f32(
                     kv_row<T>(p.halo_v, p.v, bh, p.n_halo, p.T, dv, c0 + i0 + x / dv)[x % dv]);
-            if (tid < nt) sw[tid] = (float)(eta * pow(lam, (double)(Cc - 1 - (i0 + tid))));
+            if (tid < nt)
+                sw[tid] = p.chunk_mean ? 1.0f
+                                       : (float)(eta * pow(lam, (double)(Cc - 1 - (i0 + tid))));
             __syncthreads();
-            if (active) {
+            if (p.chunk_mean && active) {
+                // ablation: sums of the chunk's keys and values (their means below)
+                for (int j = 0; j < nt; ++j) {
+#pragma unroll
+                    for (int i = 0; i < kMaxPerThread; ++i) {
+                        const int r = row0 + i * rstep;
+                        if (r < dk) D[i] += sk[j][r];
+                    }
+                    Vs += sv[j][col];
+                }
+            } else if (active) {
                 for (int j = 0; j < nt; ++j) {
                     const float wv = sw[j] * sv[j][col];
 #pragma unroll
@@ -97,9 +110,16 @@ __global__ void __launch_bounds__(kThreads) chunk_state_kernel(PrefillParams p, 
                 }
             }
         }
-        const float dec = (float)pow(lam, (double)Cc);
+        if (p.chunk_mean) {
+            // the chunk-mean shortcut: A <- lam A + eta kbar vbar^T once per chunk
+            const float w = (float)(eta / ((double)Cc * (double)Cc)) * Vs;
 #pragma unroll
-        for (int i = 0; i < kMaxPerThread; ++i) S[i] = fmaf(dec, S[i], D[i]);
+            for (int i = 0; i < kMaxPerThread; ++i) S[i] = fmaf((float)lam, S[i], w * D[i]);
+        } else {
+            const float dec = (float)pow(lam, (double)Cc);
+#pragma unroll
+            for (int i = 0; i < kMaxPerThread; ++i) S[i] = fmaf(dec, S[i], D[i]);
+        }
     }
     if (p.A_final && active) {
         float *A = p.A_final + bh * nel;

@@ -33,7 +33,11 @@ tc_status check_desc(const tc_prefill_desc *d) {
     if (d->B < 1 || d->H < 1 || d->T < 0 || d->dk < 1 || d->dv < 1 || d->W < 1 || d->C < 1)
         return TC_ERR_INVALID_ARG;
     if (!valid_dtype(d->dtype)) return TC_ERR_INVALID_ARG;
-    if (d->flags & ~(TC_PREFILL_L1_ONLY | TC_PREFILL_STATE_ONLY | TC_PREFILL_DELTA_RULE))
+    if (d->flags & ~(TC_PREFILL_L1_ONLY | TC_PREFILL_STATE_ONLY | TC_PREFILL_DELTA_RULE |
+                     TC_PREFILL_CHUNK_MEAN))
+        return TC_ERR_INVALID_ARG;
+    if ((d->flags & TC_PREFILL_CHUNK_MEAN) &&
+        (!(d->flags & TC_PREFILL_STATE_ONLY) || (d->flags & TC_PREFILL_DELTA_RULE)))
         return TC_ERR_INVALID_ARG;
     if ((d->flags & TC_PREFILL_L1_ONLY) && (d->flags & TC_PREFILL_STATE_ONLY))
         return TC_ERR_INVALID_ARG;
@@ -205,6 +209,7 @@ tc_status prefill_impl(const tc_prefill_desc *d, int64_t t0, const void *halo_k,
     p.l1_only = l1_only;
     p.state_only = state_only;
     p.delta_rule = (d->flags & TC_PREFILL_DELTA_RULE) != 0;
+    p.chunk_mean = (d->flags & TC_PREFILL_CHUNK_MEAN) != 0;
     p.halo_k = n_halo > 0 ? halo_k : nullptr;
     p.halo_v = n_halo > 0 ? halo_v : nullptr;
     p.n_halo = n_halo;

@@ -89,6 +89,7 @@ struct PrefillParams {
     bool l1_only;
     bool state_only;  // A_final only (the chunk scan); q and y unused
     bool delta_rule;  // write of Fig. 2 step (3): delta rule instead of the outer product
+    bool chunk_mean;  // ablation: the chunk-mean shortcut instead of the weighted sum
     const void *halo_k, *halo_v;
     int64_t n_halo;
     const float *A_init;
