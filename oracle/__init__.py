@@ -53,6 +53,8 @@ def _load():
         lib.oracle_scan_tokens.argtypes = [i64, i64, i64, dp, dp, c_double, c_double, c_int, dp]
         lib.oracle_scan_chunks.argtypes = [i64, i64, i64, i64, dp, dp, c_double, c_double, c_int, dp]
         lib.oracle_scan_chunk_mean.argtypes = [i64, i64, i64, i64, dp, dp, c_double, c_double, dp]
+        lib.oracle_backward.argtypes = [i64] * 6 + [dp] * 13 + [c_int]
+        lib.oracle_backward.restype = c_int
         lib.oracle_max_threads.argtypes = [c_int]
         lib.oracle_max_threads.restype = c_int
         _lib = lib
@@ -163,3 +165,22 @@ def scan_chunk_mean(k, v, lam: float, eta: float, C: int) -> np.ndarray:
     A = np.empty((dk, dv))
     _load().oracle_scan_chunk_mean(E, int(C), dk, dv, _p(k), _p(v), float(lam), float(eta), _p(A))
     return A
+
+
+def backward(q, k, v, lam, eta, g, W: int, dy, *, nthreads: int = 0):
+    """Gradients of L = sum_t <dy_t, y_t> for the layer from an empty state
+    (outer-product write): returns (dq, dk, dv [B,H,T,d], dlam, deta, dg [H])
+    in float64.  Reverse-mode through the token loop; small inputs only (it
+    keeps every state A_t)."""
+    q, k, v, dy = _f64(q), _f64(k), _f64(v), _f64(dy)
+    lam, eta, g = _f64(lam), _f64(eta), _f64(g)
+    B, H, T, dk = q.shape
+    dv = v.shape[-1]
+    dq, dkk, dvv = np.empty_like(q), np.empty_like(k), np.empty_like(v)
+    dl, de, dg_ = np.empty(H), np.empty(H), np.empty(H)
+    rc = _load().oracle_backward(B, H, T, dk, dv, int(W), _p(q), _p(k), _p(v), _p(lam), _p(eta),
+                                 _p(g), _p(dy), _p(dq), _p(dkk), _p(dvv), _p(dl), _p(de), _p(dg_),
+                                 int(nthreads))
+    if rc != 0:
+        raise RuntimeError("oracle_backward failed")
+    return dq, dkk, dvv, dl, de, dg_

@@ -354,3 +354,161 @@ void oracle_scan_chunk_mean(int64_t E, int64_t C, int64_t dk, int64_t dv,
     free(kb);
     free(vb);
 }
+
+/* ------------------------------------------------------------------------
+ * Backward of the layer (outer-product write), by reverse-mode through the
+ * token loop of Fig. 2.  For the scalar L = sum_t <dy_t, y_t> it returns
+ * dq, dk, dv ([B,H,T,d], same layout as the inputs) and the per-head
+ * dlam, deta, dg ([H], summed over the batch).  The forward is replayed with
+ * every state A_t kept (T*dk*dv doubles per head: small inputs only).
+ *   y_t = y_local_t + s m_t,  s = sigmoid(g),  m_t = q_t A_t,
+ *   A_t = lam A_{t-1} + eta k_{t-W} v_{t-W}^T  (t >= W),  A_t = A_{t-1} else.
+ * Reverse pass: G_t = dL/dA_t = q_t^T (s dy_t) + [t+1 >= W] lam G_{t+1}
+ * (G_{t+1} unscaled when step t+1 has no write); each write at step t gives
+ * dk_e += eta G_t v_e, dv_e += eta G_t^T k_e, deta += <G_t, k_e v_e^T>,
+ * dlam += <G_t, A_{t-1}>.  The window softmax backward is the usual one:
+ * dp_j = <dy_t, v_j>, ds_j = p_j (dp_j - sum_i p_i dp_i),
+ * dq_t += sum_j ds_j k_j / sqrt(dk), dk_j += ds_j q_t / sqrt(dk), dv_j += p_j dy_t.
+ * ------------------------------------------------------------------------ */
+int oracle_backward(int64_t B, int64_t H, int64_t T, int64_t dk, int64_t dv, int64_t W,
+                    const double *q, const double *k, const double *v,
+                    const double *lam, const double *eta, const double *g,
+                    const double *dy, double *dq, double *dkk, double *dvv,
+                    double *dlam, double *deta, double *dg, int nthreads)
+{
+    if (B < 0 || H < 0 || T < 0 || dk < 1 || dv < 1 || W < 1) return -1;
+    set_threads(nthreads);
+    const int64_t nel = dk * dv;
+    memset(dq, 0, (size_t)(B * H * T * dk) * sizeof(double));
+    memset(dkk, 0, (size_t)(B * H * T * dk) * sizeof(double));
+    memset(dvv, 0, (size_t)(B * H * T * dv) * sizeof(double));
+    double *pdl = (double *)calloc((size_t)(B * H), sizeof(double));
+    double *pde = (double *)calloc((size_t)(B * H), sizeof(double));
+    double *pdg = (double *)calloc((size_t)(B * H), sizeof(double));
+    if (!pdl || !pde || !pdg) {
+        free(pdl); free(pde); free(pdg);
+        return -1;
+    }
+    int err = 0;
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : err)
+    for (int64_t bh = 0; bh < B * H; ++bh) {
+        const int64_t h = bh % H;
+        const double *qh = q + bh * T * dk, *kh = k + bh * T * dk, *vh = v + bh * T * dv;
+        const double *dyh = dy + bh * T * dv;
+        double *dqh = dq + bh * T * dk, *dkh = dkk + bh * T * dk, *dvh = dvv + bh * T * dv;
+        double *As = (double *)calloc((size_t)((T + 1) * nel), sizeof(double)); /* As[t+1] = A_t */
+        double *G = (double *)calloc((size_t)nel, sizeof(double));
+        double *p = (double *)malloc((size_t)W * sizeof(double));
+        if (!As || !G || !p) {
+            err |= 1;
+        } else {
+            const double s = 1.0 / (1.0 + exp(-g[h]));
+            const double scale = 1.0 / sqrt((double)dk);
+            /* forward states */
+            for (int64_t t = 0; t < T; ++t) {
+                const double *Ap = As + t * nel;
+                double *An = As + (t + 1) * nel;
+                if (t >= W) {
+                    const double *ke = kh + (t - W) * dk, *ve = vh + (t - W) * dv;
+                    for (int64_t r = 0; r < dk; ++r)
+                        for (int64_t c = 0; c < dv; ++c)
+                            An[r * dv + c] = lam[h] * Ap[r * dv + c] + eta[h] * ke[r] * ve[c];
+                } else {
+                    memcpy(An, Ap, (size_t)nel * sizeof(double));
+                }
+            }
+            /* L2: gate, dq, and the reverse state gradient */
+            for (int64_t t = T - 1; t >= 0; --t) {
+                const double *At = As + (t + 1) * nel;
+                const double *qt = qh + t * dk, *dyt = dyh + t * dv;
+                double mdy = 0.0;
+                for (int64_t c = 0; c < dv; ++c) {
+                    double mc = 0.0;
+                    for (int64_t r = 0; r < dk; ++r) mc += qt[r] * At[r * dv + c];
+                    mdy += mc * dyt[c];
+                }
+                pdg[bh] += s * (1.0 - s) * mdy;
+                for (int64_t r = 0; r < dk; ++r) {
+                    double acc = 0.0;
+                    for (int64_t c = 0; c < dv; ++c) acc += At[r * dv + c] * s * dyt[c];
+                    dqh[t * dk + r] += acc;
+                }
+                for (int64_t r = 0; r < dk; ++r)
+                    for (int64_t c = 0; c < dv; ++c) G[r * dv + c] += qt[r] * s * dyt[c];
+                if (t >= W) {
+                    const int64_t e = t - W;
+                    const double *ke = kh + e * dk, *ve = vh + e * dv;
+                    const double *Ap = As + t * nel; /* A_{t-1} */
+                    for (int64_t r = 0; r < dk; ++r) {
+                        double acc = 0.0;
+                        for (int64_t c = 0; c < dv; ++c) acc += G[r * dv + c] * ve[c];
+                        dkh[e * dk + r] += eta[h] * acc;
+                    }
+                    for (int64_t c = 0; c < dv; ++c) {
+                        double acc = 0.0;
+                        for (int64_t r = 0; r < dk; ++r) acc += G[r * dv + c] * ke[r];
+                        dvh[e * dv + c] += eta[h] * acc;
+                    }
+                    double gkv = 0.0, ga = 0.0;
+                    for (int64_t r = 0; r < dk; ++r)
+                        for (int64_t c = 0; c < dv; ++c) {
+                            gkv += G[r * dv + c] * ke[r] * ve[c];
+                            ga += G[r * dv + c] * Ap[r * dv + c];
+                        }
+                    pde[bh] += gkv;
+                    pdl[bh] += ga;
+                    for (int64_t x = 0; x < nel; ++x) G[x] *= lam[h];
+                }
+            }
+            /* L1: window softmax backward */
+            for (int64_t t = 0; t < T; ++t) {
+                const double *qt = qh + t * dk, *dyt = dyh + t * dv;
+                const int64_t j0 = t - W + 1 > 0 ? t - W + 1 : 0, n = t - j0 + 1;
+                double smax = -INFINITY, den = 0.0;
+                for (int64_t i = 0; i < n; ++i) {
+                    double dot = 0.0;
+                    for (int64_t r = 0; r < dk; ++r) dot += qt[r] * kh[(j0 + i) * dk + r];
+                    p[i] = dot * scale;
+                    if (p[i] > smax) smax = p[i];
+                }
+                for (int64_t i = 0; i < n; ++i) {
+                    p[i] = exp(p[i] - smax);
+                    den += p[i];
+                }
+                double Dt = 0.0;
+                for (int64_t i = 0; i < n; ++i) {
+                    p[i] /= den;
+                    double dp = 0.0;
+                    for (int64_t c = 0; c < dv; ++c) dp += dyt[c] * vh[(j0 + i) * dv + c];
+                    Dt += p[i] * dp;
+                }
+                for (int64_t i = 0; i < n; ++i) {
+                    const int64_t j = j0 + i;
+                    double dp = 0.0;
+                    for (int64_t c = 0; c < dv; ++c) dp += dyt[c] * vh[j * dv + c];
+                    const double ds = p[i] * (dp - Dt);
+                    for (int64_t r = 0; r < dk; ++r) {
+                        dqh[t * dk + r] += ds * kh[j * dk + r] * scale;
+                        dkh[j * dk + r] += ds * qt[r] * scale;
+                    }
+                    for (int64_t c = 0; c < dv; ++c) dvh[j * dv + c] += p[i] * dyt[c];
+                }
+            }
+        }
+        free(As);
+        free(G);
+        free(p);
+    }
+    for (int64_t h = 0; h < H; ++h) {
+        dlam[h] = deta[h] = dg[h] = 0.0;
+        for (int64_t b = 0; b < B; ++b) {
+            dlam[h] += pdl[b * H + h];
+            deta[h] += pde[b * H + h];
+            dg[h] += pdg[b * H + h];
+        }
+    }
+    free(pdl);
+    free(pde);
+    free(pdg);
+    return err ? -1 : 0;
+}

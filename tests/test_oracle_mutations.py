@@ -19,9 +19,10 @@ SRC = os.path.join(os.path.dirname(oracle.__file__), "tc_oracle.c")
 
 MUTATIONS = {
     "first eviction one step late (read before write)":
-        ("if (t >= W) {", "if (t > W) {"),
+        ("if (t >= W) {\n        const double *k_old", "if (t > W) {\n        const double *k_old"),
     "missing 1/sqrt(d_k)":
-        ("const double scale = 1.0 / sqrt((double)dk);", "const double scale = 1.0;"),
+        ("    const double scale = 1.0 / sqrt((double)dk);\n    double smax",
+         "    const double scale = 1.0;\n    double smax"),
     "dropped decay":
         ("A[r * dv + c] = lam * A[r * dv + c] + eta * (k_old[r] * u[c]);",
          "A[r * dv + c] = A[r * dv + c] + eta * (k_old[r] * u[c]);"),
@@ -45,6 +46,12 @@ MUTATIONS = {
         ("    memcpy(ring_k + pos * dk, k, (size_t)dk * sizeof(double));\n"
          "    memcpy(ring_v + pos * dv, v, (size_t)dv * sizeof(double));\n",
          ""),
+    "backward: state gradient not decayed through a write":
+        ("for (int64_t x = 0; x < nel; ++x) G[x] *= lam[h];", "for (int64_t x = 0; x < nel; ++x) G[x] *= 1.0;"),
+    "backward: softmax gradient without the mean term":
+        ("const double ds = p[i] * (dp - Dt);", "const double ds = p[i] * dp;"),
+    "backward: lambda gradient against A_t instead of A_{t-1}":
+        ("const double *Ap = As + t * nel; /* A_{t-1} */", "const double *Ap = As + (t + 1) * nel;"),
     "chunk decay exponent off by one":
         ("const double wd = eta * pow(lam, (double)(Cc - 1 - i));",
          "const double wd = eta * pow(lam, (double)(Cc - i));"),
@@ -69,6 +76,7 @@ PIN_CALLS = [
     lambda: pins.test_delta_rule_repeated_write_closed_form(1.0, 0.5, 4),
     lambda: pins.test_delta_rule_repeated_write_closed_form(0.9, 0.3, 6),
     pins.test_delta_rule_equals_outer_product_on_orthonormal_keys,
+    pins.test_backward_matches_central_differences,
 ]
 
 
@@ -97,7 +105,8 @@ def test_pins_catch_planted_mistake(name, tmp_path):
     good = oracle._load()
     mut = ctypes.CDLL(so)
     for fn in ("oracle_prefill_rule", "oracle_decode_rule", "oracle_scan_tokens",
-               "oracle_scan_chunks", "oracle_scan_chunk_mean", "oracle_max_threads"):
+               "oracle_scan_chunks", "oracle_scan_chunk_mean", "oracle_backward",
+               "oracle_max_threads"):
         getattr(mut, fn).argtypes = getattr(good, fn).argtypes
         getattr(mut, fn).restype = getattr(good, fn).restype
     failed = []

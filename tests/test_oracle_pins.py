@@ -232,6 +232,36 @@ def test_delta_rule_decode_continues_prefill():
     np.testing.assert_allclose(A, A_full, rtol=0, atol=1e-12)
 
 
+# --- backward: reverse-mode gradients against finite differences -----------
+
+def test_backward_matches_central_differences():
+    """Every gradient element of L = sum <dy, y> (q, k, v, lam, eta, g) agrees
+    with a central difference of the forward oracle, on an input where the
+    window fills and many pairs are evicted."""
+    rng = np.random.default_rng(21)
+    B, H, T, dk, dv, W = 1, 2, 11, 3, 2, 3
+    q, k = (rng.standard_normal((B, H, T, dk)) * 0.6 for _ in range(2))
+    v, dy = (rng.standard_normal((B, H, T, dv)) * 0.6 for _ in range(2))
+    lam, eta, g = np.array([0.9, 0.75]), np.array([0.6, 1.2]), np.array([0.4, -0.7])
+    grads = dict(zip(("q", "k", "v", "lam", "eta", "g"), oracle.backward(q, k, v, lam, eta, g, W, dy)))
+    x = {"q": q, "k": k, "v": v, "lam": lam, "eta": eta, "g": g}
+
+    def loss(**over):
+        a = {**x, **over}
+        y, _ = oracle.prefill(a["q"], a["k"], a["v"], a["lam"], a["eta"], a["g"], W)
+        return float((y * dy).sum())
+
+    h = 1e-6
+    for name, base in x.items():
+        fd = np.empty_like(base)
+        for idx in np.ndindex(base.shape):
+            xp, xm = base.copy(), base.copy()
+            xp[idx] += h
+            xm[idx] -= h
+            fd[idx] = (loss(**{name: xp}) - loss(**{name: xm})) / (2 * h)
+        np.testing.assert_allclose(grads[name], fd, rtol=0, atol=5e-8, err_msg=name)
+
+
 # --- training form: chunk scan and the chunk-mean shortcut -----------------
 
 @pytest.mark.parametrize("C", [1, 7, 16, 64, 300])
