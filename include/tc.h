@@ -181,6 +181,25 @@ TC_API tc_status tc_state_fold(int64_t B, int64_t H, int64_t dk, int64_t dv, int
                                const float *dA, const int64_t *E, const float *lambda,
                                float *A_out, tc_stream_t stream);
 
+/* Backward of the layer (outer-product write) over T tokens from an empty
+ * state, for training: with L = sum_t <dy_t, y_t> it computes
+ *   dq, dk, dv  [B,H,T,d] float32 (gradients of q, k, v; input layout),
+ *   dlambda, deta, dg  [H] float32 (summed over the batch).
+ * The pages train lambda, eta and g end to end (§2 training
+ * considerations); the formulas are reverse mode through the token loop of
+ * Fig. 2.  The window part is the usual softmax backward over the W keys;
+ * the memory part is a reverse scan of dL/dA_t, replayed from checkpoints of
+ * A every 64 tokens.  q, k, v, dy: device, dtype of desc (dy has y's layout);
+ * desc->flags must be 0 (C is not used).  Float32 SIMT kernels; four
+ * launches.  Workspace: tc_backward_workspace_size(desc) bytes (about
+ * B*H*(2T + 64*d_k*d_v*(1 + ceil(T/64))) floats).  Errors as tc_prefill. */
+TC_API size_t tc_backward_workspace_size(const tc_prefill_desc *desc);
+TC_API tc_status tc_backward(const tc_prefill_desc *desc, const void *q, const void *k,
+                             const void *v, const float *lambda, const float *eta, const float *g,
+                             const void *dy, float *dq, float *dk, float *dv, float *dlambda,
+                             float *deta, float *dg, void *workspace, size_t workspace_bytes,
+                             tc_stream_t stream);
+
 /* Number of kernel launches one tc_prefill call enqueues for desc on the
  * current device (the path depends on shapes and dtype), or -1 when desc is
  * NULL or invalid.  tc_decode_step always enqueues exactly one. */

@@ -49,7 +49,7 @@ EXPORTED = ("tc_prefill_workspace_size", "tc_prefill", "tc_prefill_launch_count"
             "tc_prefill_host", "tc_decode_step", "tc_decode_step_host_workspace_size",
             "tc_decode_step_host", "tc_get_device_status", "tc_status_string", "tc_version",
             "tc_prefill_no_alloc", "tc_prefill_from_state", "tc_prefill_from_state_workspace_size",
-            "tc_state_fold", "tc_decode_step_ragged")
+            "tc_state_fold", "tc_decode_step_ragged", "tc_backward", "tc_backward_workspace_size")
 
 
 class PrefillDesc(ctypes.Structure):
@@ -86,6 +86,10 @@ _lib.tc_prefill_from_state_workspace_size.argtypes = [_PD, ctypes.c_int64]
 _lib.tc_prefill_from_state_workspace_size.restype = _sz
 _lib.tc_prefill_from_state.argtypes = [_PD, ctypes.c_int64] + [_vp] * 12 + [_sz, _vp]
 _lib.tc_prefill_from_state.restype = _int
+_lib.tc_backward_workspace_size.argtypes = [_PD]
+_lib.tc_backward_workspace_size.restype = _sz
+_lib.tc_backward.argtypes = [_PD] + [_vp] * 14 + [_sz, _vp]
+_lib.tc_backward.restype = _int
 _lib.tc_state_fold.argtypes = [ctypes.c_int64] * 5 + [_vp] * 4 + [_vp]
 _lib.tc_state_fold.restype = _int
 _lib.tc_decode_step.argtypes = [_DS] + [_vp] * 4 + [_vp]
@@ -257,6 +261,32 @@ def state_fold(dA: torch.Tensor, E: torch.Tensor, lam: torch.Tensor,
                             _ptr(lam), _ptr(A_out), _stream(stream))
     _check(st, "tc_state_fold")
     return A_out
+
+
+def backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, lam: torch.Tensor,
+             eta: torch.Tensor, g: torch.Tensor, W: int, dy: torch.Tensor, *,
+             workspace: Optional[torch.Tensor] = None, stream=None):
+    """tc_backward: gradients of L = sum <dy, y> for the layer over q, k, v
+    [B,H,T,d] (from an empty state, outer-product write).  Returns
+    (dq, dk, dv [float32, input layout], dlam, deta, dg [H] float32)."""
+    B, H, T, dk = q.shape
+    dv = v.shape[-1]
+    desc = make_prefill_desc(B, H, T, dk, dv, W, 1, _dtype_code(q))
+    f = dict(dtype=torch.float32, device=q.device)
+    dq, dkk, dvv = torch.empty(B, H, T, dk, **f), torch.empty(B, H, T, dk, **f), torch.empty(B, H, T, dv, **f)
+    dl, de, dg_ = torch.empty(H, **f), torch.empty(H, **f), torch.empty(H, **f)
+    need = _lib.tc_backward_workspace_size(ctypes.byref(desc))
+    if need == SIZE_ERROR:
+        raise TCError(1, "tc_backward_workspace_size")
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    _contig(q, k, v, lam, eta, g, dy, workspace)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = _lib.tc_backward(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(lam), _ptr(eta),
+                          _ptr(g), _ptr(dy), _ptr(dq), _ptr(dkk), _ptr(dvv), _ptr(dl), _ptr(de),
+                          _ptr(dg_), _ptr(workspace), ws_bytes, _stream(stream))
+    _check(st, "tc_backward")
+    return dq, dkk, dvv, dl, de, dg_
 
 
 def prefill_launch_count(desc: PrefillDesc) -> int:

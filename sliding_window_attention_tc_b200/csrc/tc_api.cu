@@ -244,6 +244,41 @@ tc_status tc_prefill_from_state(const tc_prefill_desc *d, int64_t t0, const void
                         workspace, workspace_bytes, stream);
 }
 
+size_t tc_backward_workspace_size(const tc_prefill_desc *d) {
+    if (check_desc(d) != TC_OK || d->flags != 0) return (size_t)-1;
+    return tc::backward_workspace_bytes(*d);
+}
+
+tc_status tc_backward(const tc_prefill_desc *d, const void *q, const void *k, const void *v,
+                      const float *lambda, const float *eta, const float *g, const void *dy,
+                      float *dq, float *dk, float *dv, float *dlambda, float *deta, float *dg,
+                      void *workspace, size_t workspace_bytes, tc_stream_t stream) {
+    tc_status st = check_desc(d);
+    if (st != TC_OK) return st;
+    if (d->flags != 0) return TC_ERR_UNSUPPORTED;
+    const bool empty = d->T == 0;
+    const void *tok[] = {q, k, v, dy, dq, dk, dv};
+    const void *hd[] = {lambda, eta, g, dlambda, deta, dg};
+    for (const void *x : tok)
+        if ((!x && !empty) || !aligned16(x)) return TC_ERR_INVALID_ARG;
+    for (const void *x : hd)
+        if (!x) return TC_ERR_INVALID_ARG;
+    if (workspace && !aligned16(workspace)) return TC_ERR_INVALID_ARG;
+    int dev = 0;
+    st = current_device(&dev, nullptr);
+    if (st != TC_OK) return st;
+    const size_t need = tc::backward_workspace_bytes(*d);
+    if (need > 0 && (!workspace || workspace_bytes < need)) return TC_ERR_WORKSPACE;
+    for (const void *x : tok)
+        if (x && !is_device_ptr(x)) return TC_ERR_INVALID_ARG;
+    for (const void *x : hd)
+        if (!is_device_ptr(x)) return TC_ERR_INVALID_ARG;
+    if (need > 0 && !is_device_ptr(workspace)) return TC_ERR_INVALID_ARG;
+    cudaError_t e = tc::launch_backward(*d, q, k, v, lambda, eta, g, dy, dq, dk, dv, dlambda, deta,
+                                        dg, workspace, reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? TC_OK : TC_ERR_CUDA;
+}
+
 int tc_prefill_launch_count(const tc_prefill_desc *d) {
     if (check_desc(d) != TC_OK) return -1;
     if (use_sm100(*d, 0)) return tc::sm100_launch_count(*d);

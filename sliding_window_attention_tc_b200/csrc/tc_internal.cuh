@@ -108,6 +108,13 @@ bool decode_supported(int dk, int dv, tc_dtype dtype);
 size_t portable_workspace_bytes(const tc_prefill_desc &d, int64_t n_halo);
 cudaError_t launch_prefill_portable(const PrefillParams &p, tc_dtype dtype, cudaStream_t s);
 
+// backward.cu: gradients of the layer (outer-product write), float32 SIMT.
+size_t backward_workspace_bytes(const tc_prefill_desc &d);
+cudaError_t launch_backward(const tc_prefill_desc &d, const void *q, const void *k, const void *v,
+                            const float *lam, const float *eta, const float *g, const void *dy,
+                            float *dq, float *dk, float *dv, float *dlam, float *deta, float *dg,
+                            void *workspace, cudaStream_t s);
+
 // prefill_sm100.cu: tcgen05 / TMA path for bf16, d_k = d_v = 64.
 bool sm100_supported(const tc_prefill_desc &d, int64_t n_halo);
 size_t sm100_workspace_bytes(const tc_prefill_desc &d, int num_sms);
