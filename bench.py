@@ -337,6 +337,55 @@ def time_prefill_e2e(tc, name, dev, steps):
     return {"ms_per_step": ms, "tokens_per_s": B * H * T / (ms * 1e-3), "h2d": h2d, "d2h": d2h}
 
 
+def time_calls(fn, steps, warmup):
+    """Per-call device times (ms) of fn() on the current stream, CUDA events."""
+    stream = torch.cuda.current_stream()
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps)]
+    for a, b in ev:
+        a.record(stream)
+        fn()
+        b.record(stream)
+    torch.cuda.synchronize()
+    return [a.elapsed_time(b) for a, b in ev]
+
+
+# float32 FMA peak of the SIMT kernels (backward, delta rule): 148 SMs x 128
+# FMA lanes x 2 FLOP x 1965 MHz, the nominal unit count and clock.
+FP32_SIMT_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+
+
+def time_training_extras(tc, dev):
+    """The backward pass and the delta-rule prefill on the LM workload (both
+    float32 SIMT paths): ms per call and tokens/s."""
+    x, sets, prm = _prefill_device_inputs(HEADLINE, dev, copies=1)
+    q, k, v = sets[0]
+    B, H, T, d = q.shape
+    gen = torch.Generator(device=dev).manual_seed(7)
+    dy = (torch.randn(B, H, T, d, generator=gen, device=dev) / 8).to(q.dtype)
+    out = {}
+    l1f, l2f = prefill_flops(B, H, T, d, d, x.W)
+    bwd_ms = statistics.median(time_calls(lambda: tc.backward(q, k, v, *prm, x.W, dy), 3, 1))
+    # algorithmic work of the backward: twice the forward's (the usual count
+    # for an attention backward: scores recomputed, dq, dk, dv)
+    tf = 2 * (l1f + l2f) / (bwd_ms * 1e-3) / 1e12
+    out["backward"] = {"workload": HEADLINE, "ms": bwd_ms, "tokens_per_s": B * H * T / (bwd_ms * 1e-3),
+                       "roofline": {"bound": "alu", "achieved": tf, "peak": FP32_SIMT_PEAK_TFLOPS,
+                                    "unit": "TFLOP/s", "frac": tf / FP32_SIMT_PEAK_TFLOPS,
+                                    "traffic": None, "peak_source": "nominal fp32 FMA rate",
+                                    "algorithmic_flops_per_call": 2 * (l1f + l2f)}}
+    delta_ms = statistics.median(time_calls(
+        lambda: tc.prefill(q, k, v, *prm, x.W, x.C, delta_rule=True), 3, 1))
+    out["delta_rule_prefill"] = {"workload": HEADLINE, "ms": delta_ms,
+                                 "tokens_per_s": B * H * T / (delta_ms * 1e-3)}
+    del dy, sets
+    torch.cuda.empty_cache()
+    return out
+
+
 # ---------------------------------------------------------------------------
 def oracle_sample(name, budget_s=12.0):
     """Time the CPU oracle as it stands on a bounded sample of a prefill
@@ -534,6 +583,7 @@ def main():
                         "tokens_per_s": dec["B"] / (dec["e2e_ms_per_step"] * 1e-3),
                         "h2d_bytes_per_step": dec["e2e_h2d_bytes"],
                         "d2h_bytes_per_step": dec["e2e_d2h_bytes"]}}
+            extras.update(time_training_extras(tc, dev))
         e2e = time_prefill_e2e(tc, HEADLINE, dev, max(5, min(20, args.steps // 10)))
     finally:
         clocks.stop()

@@ -20,10 +20,10 @@
 //   step t (eviction e = t - W) gives dk_e += eta G_t v_e,
 //   dv_e += eta G_t^T k_e, deta += <G_t, k_e v_e^T>, dlam += <G_t, A_{t-1}>;
 //   also dq_t += A_t (s dy_t) and dg += s (1 - s) <dy_t, q_t A_t>.
-//   bwd_l2_kernel (a CTA per (b,h)) replays A from checkpoints every kCk
-//   tokens and walks the tokens backwards; it adds to dq, dk, dv and leaves
-//   per-(b,h) partials of dlam, deta, dg, which bwd_reduce_kernel sums over
-//   the batch.
+//   bwd_l2_kernel (CTAs of 8 rows of A per (b,h)) replays A from
+//   checkpoints every kCk tokens and walks the tokens backwards; it adds to
+//   dq, dk, dv and leaves partials of dlam, deta, dg, which
+//   bwd_reduce_kernel sums over the batch and the row blocks in a fixed order.
 
 #include <cuda_runtime.h>
 
@@ -260,165 +260,145 @@ __global__ void __launch_bounds__(kThreads) bwd_keys_kernel(BwdParams p) {
 }
 
 // ---------------------------------------------------------------------------
-// L2 reverse scan, one CTA per (b,h).  Thread layout over the dk x dv
-// matrices: warp w owns rows r = w, w + 8, ...; lane l owns columns
-// c = l, l + 32, ... (row sums by shuffles, column sums through shared memory).
+// L2 reverse scan.  Row r of G_t = dL/dA_t and of A_t only involves q_t[r],
+// k_e[r] and whole rows of dy / v, so each (b,h) is split over CTAs of
+// kRows rows (one row per warp; lane l owns columns l, l+32, ...).  A is
+// replayed from checkpoints every kCk tokens; a segment's q, dy, k, v are
+// staged in shared memory once.  dv_e sums over all rows: the CTAs of a head
+// add their parts with atomics.
 template <typename Tin>
 __global__ void __launch_bounds__(kThreads) bwd_l2_kernel(BwdParams p) {
-    constexpr int RPW = kMaxD / kRows;  // rows per warp (at most)
-    constexpr int CPL = kMaxD / 32;     // columns per lane (at most)
-    __shared__ float sq[kMaxD], sdm[kMaxD], sk[kMaxD], svv[kMaxD];
-    __shared__ float scol[kRows][kMaxD];
-    __shared__ float sred[3][kRows];
+    constexpr int CPL = kMaxD / 32;
+    extern __shared__ float sh[];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int64_t bh = blockIdx.x;
+    const int64_t bh = blockIdx.y;
     const int h = (int)(bh % p.H);
-    const int dk = p.dk, dv = p.dv, nel = dk * dv;
+    const int dk = p.dk, dv = p.dv;
+    const int r0 = blockIdx.x * kRows, r = r0 + warp;
+    const bool row_ok = r < dk;
     const int64_t T = p.T, W = p.W;
     const float lam = p.lam[h], eta = p.eta[h];
     const float sg = 1.f / (1.f + expf(-p.g[h]));
+    // shared: q rows [kCk][kRows], k rows [kCk][kRows], dy [kCk][dv], v [kCk][dv], column sums [kRows][dv]
+    float *sQ = sh, *sK = sQ + kCk * kRows, *sDY = sK + kCk * kRows, *sV = sDY + kCk * dv;
+    float *scol = sV + kCk * dv;
     const Tin *qb = reinterpret_cast<const Tin *>(p.q) + bh * T * dk;
     const Tin *kb = reinterpret_cast<const Tin *>(p.k) + bh * T * dk;
     const Tin *vb = reinterpret_cast<const Tin *>(p.v) + bh * T * dv;
     const Tin *db = reinterpret_cast<const Tin *>(p.dy) + bh * T * dv;
     const int64_t nCk = (T + kCk - 1) / kCk;
-    float *ck = p.ckpt + bh * nCk * nel;
-    float *seg = p.seg + bh * (int64_t)kCk * nel;
-    auto el = [&](int i, int jx) -> int { return (warp + kRows * i) * dv + lane + 32 * jx; };
-    auto in_m = [&](int i, int jx) -> bool { return warp + kRows * i < dk && lane + 32 * jx < dv; };
+    const int nrs = gridDim.x;
+    // this CTA's slices: [nCk][kRows][dv] checkpoints, [kCk][kRows][dv] segment
+    float *ck = p.ckpt + ((bh * nrs + blockIdx.x) * nCk) * (int64_t)kRows * dv;
+    float *seg = p.seg + ((bh * nrs + blockIdx.x) * (int64_t)kCk) * kRows * dv;
+    auto at = [&](int jx) { return warp * dv + lane + 32 * jx; };  // element of a [kRows][dv] slab
+    auto col_ok = [&](int jx) { return lane + 32 * jx < dv; };
 
-    // forward replay storing A before every kCk-th token
-    float A[RPW][CPL];
-#pragma unroll
-    for (int i = 0; i < RPW; ++i)
-#pragma unroll
-        for (int jx = 0; jx < CPL; ++jx) A[i][jx] = 0.f;
-    auto load_kv = [&](int64_t e) {
+    // stage q, dy (tokens tb..te-1) and k, v of their evictions
+    auto stage = [&](int64_t tb, int64_t te, bool with_q) {
         __syncthreads();
-        for (int x = tid; x < dk; x += kThreads) sk[x] = to_f32(kb[e * dk + x]);
-        for (int x = tid; x < dv; x += kThreads) svv[x] = to_f32(vb[e * dv + x]);
+        const int n = (int)(te - tb);
+        for (int x = tid; x < n * kRows; x += kThreads) {
+            const int64_t t = tb + x / kRows;
+            const int rr = r0 + x % kRows;
+            sK[x] = (t >= W && rr < dk) ? to_f32(kb[(t - W) * dk + rr]) : 0.f;
+            if (with_q) sQ[x] = rr < dk ? to_f32(qb[t * dk + rr]) : 0.f;
+        }
+        for (int x = tid; x < n * dv; x += kThreads) {
+            const int64_t t = tb + x / dv;
+            sV[x] = t >= W ? to_f32(vb[(t - W) * dv + x % dv]) : 0.f;
+            if (with_q) sDY[x] = to_f32(db[t * dv + x % dv]);
+        }
         __syncthreads();
     };
-    auto write = [&]() {
+
+    float A[CPL];
 #pragma unroll
-        for (int i = 0; i < RPW; ++i)
+    for (int jx = 0; jx < CPL; ++jx) A[jx] = 0.f;
+    // forward replay: checkpoints of A before every kCk-th token
+    for (int64_t s = 0; s < nCk; ++s) {
+        const int64_t tb = s * kCk, te = tb + kCk < T ? tb + kCk : T;
+#pragma unroll
+        for (int jx = 0; jx < CPL; ++jx)
+            if (col_ok(jx)) ck[s * kRows * dv + at(jx)] = A[jx];
+        stage(tb, te, false);
+        for (int64_t t = tb; t < te; ++t) {
+            if (t < W) continue;
+            const float ek = eta * sK[(t - tb) * kRows + warp];
 #pragma unroll
             for (int jx = 0; jx < CPL; ++jx)
-                if (in_m(i, jx)) A[i][jx] = fmaf(lam, A[i][jx], eta * sk[warp + kRows * i] * svv[lane + 32 * jx]);
-    };
-    for (int64_t t = 0; t < T; ++t) {
-        if (t % kCk == 0) {
-#pragma unroll
-            for (int i = 0; i < RPW; ++i)
-#pragma unroll
-                for (int jx = 0; jx < CPL; ++jx)
-                    if (in_m(i, jx)) ck[(t / kCk) * nel + el(i, jx)] = A[i][jx];
-        }
-        if (t >= W) {
-            load_kv(t - W);
-            write();
+                if (col_ok(jx)) A[jx] = fmaf(lam, A[jx], ek * sV[(t - tb) * dv + lane + 32 * jx]);
         }
     }
 
-    // reverse pass
-    float G[RPW][CPL];
+    float G[CPL];
 #pragma unroll
-    for (int i = 0; i < RPW; ++i)
-#pragma unroll
-        for (int jx = 0; jx < CPL; ++jx) G[i][jx] = 0.f;
-    float pl = 0.f, pe = 0.f, pg = 0.f;  // partials: dlam, deta, dg
+    for (int jx = 0; jx < CPL; ++jx) G[jx] = 0.f;
+    float pl = 0.f, pe = 0.f, pg = 0.f;  // dlam, deta, dg partials
     for (int64_t s = nCk - 1; s >= 0; --s) {
         const int64_t tb = s * kCk, te = tb + kCk < T ? tb + kCk : T;
-        // replay A_t for t in [tb, te) into seg
+        stage(tb, te, true);
+        // replay the segment, keeping every A_t of this CTA's rows
 #pragma unroll
-        for (int i = 0; i < RPW; ++i)
-#pragma unroll
-            for (int jx = 0; jx < CPL; ++jx)
-                if (in_m(i, jx)) A[i][jx] = ck[s * nel + el(i, jx)];
+        for (int jx = 0; jx < CPL; ++jx)
+            if (col_ok(jx)) A[jx] = ck[s * kRows * dv + at(jx)];
         for (int64_t t = tb; t < te; ++t) {
             if (t >= W) {
-                load_kv(t - W);
-                write();
-            }
-#pragma unroll
-            for (int i = 0; i < RPW; ++i)
+                const float ek = eta * sK[(t - tb) * kRows + warp];
 #pragma unroll
                 for (int jx = 0; jx < CPL; ++jx)
-                    if (in_m(i, jx)) seg[(t - tb) * nel + el(i, jx)] = A[i][jx];
+                    if (col_ok(jx)) A[jx] = fmaf(lam, A[jx], ek * sV[(t - tb) * dv + lane + 32 * jx]);
+            }
+#pragma unroll
+            for (int jx = 0; jx < CPL; ++jx)
+                if (col_ok(jx)) seg[(t - tb) * kRows * dv + at(jx)] = A[jx];
         }
         for (int64_t t = te - 1; t >= tb; --t) {
-            __syncthreads();
-            for (int x = tid; x < dk; x += kThreads) sq[x] = to_f32(qb[t * dk + x]);
-            for (int x = tid; x < dv; x += kThreads) sdm[x] = sg * to_f32(db[t * dv + x]);
-            if (t >= W) {
-                for (int x = tid; x < dk; x += kThreads) sk[x] = to_f32(kb[(t - W) * dk + x]);
-                for (int x = tid; x < dv; x += kThreads) svv[x] = to_f32(vb[(t - W) * dv + x]);
-            }
-            __syncthreads();
-            // dq_t += A_t dm_t (row sums); dg partial (1 - s) <q_t, A_t dm_t>
+            const int i = (int)(t - tb);
+            const float qr = sQ[i * kRows + warp];
+            // dq_t[r] += sum_c A_t[r][c] dm_t[c];  dg partial (1 - s) q_t[r] (that)
+            float acc = 0.f;
 #pragma unroll
-            for (int i = 0; i < RPW; ++i) {
-                const int r = warp + kRows * i;
-                float acc = 0.f;
-#pragma unroll
-                for (int jx = 0; jx < CPL; ++jx)
-                    if (in_m(i, jx)) acc = fmaf(seg[(t - tb) * nel + el(i, jx)], sdm[lane + 32 * jx], acc);
-                acc = warp_sum(acc);
-                if (r < dk) {
-                    if (lane == 0) p.gq[(bh * T + t) * dk + r] += acc;
-                    pg = fmaf((1.f - sg) * sq[r], acc, pg);  // same value in every lane
-                }
-            }
+            for (int jx = 0; jx < CPL; ++jx)
+                if (col_ok(jx)) acc = fmaf(seg[i * kRows * dv + at(jx)], sg * sDY[i * dv + lane + 32 * jx], acc);
+            acc = warp_sum(acc);
+            if (row_ok && lane == 0) p.gq[(bh * T + t) * dk + r] += acc;
+            pg = fmaf((1.f - sg) * qr, acc, pg);
             // G += q_t (x) dm_t
 #pragma unroll
-            for (int i = 0; i < RPW; ++i)
-#pragma unroll
-                for (int jx = 0; jx < CPL; ++jx)
-                    if (in_m(i, jx)) G[i][jx] = fmaf(sq[warp + kRows * i], sdm[lane + 32 * jx], G[i][jx]);
+            for (int jx = 0; jx < CPL; ++jx)
+                if (col_ok(jx)) G[jx] = fmaf(qr, sg * sDY[i * dv + lane + 32 * jx], G[jx]);
             if (t >= W) {
                 const int64_t e = t - W;
-                // dk_e += eta G v_e (row sums), deta += <G, k_e v_e^T>
-#pragma unroll
-                for (int i = 0; i < RPW; ++i) {
-                    const int r = warp + kRows * i;
-                    float acc = 0.f;
-#pragma unroll
-                    for (int jx = 0; jx < CPL; ++jx)
-                        if (in_m(i, jx)) acc = fmaf(G[i][jx], svv[lane + 32 * jx], acc);
-                    acc = warp_sum(acc);
-                    if (r < dk) {
-                        if (lane == 0) p.gk[(bh * T + e) * dk + r] += eta * acc;
-                        pe = fmaf(sk[r], acc, pe);
-                    }
-                }
-                // dv_e += eta G^T k_e (column sums), dlam += <G, A_{t-1}>
-                const float *Aprev = t > tb ? seg + (t - 1 - tb) * nel : ck + s * nel;
+                const float kr = sK[i * kRows + warp];
+                float a2 = 0.f;
 #pragma unroll
                 for (int jx = 0; jx < CPL; ++jx) {
-                    float acc = 0.f;
-#pragma unroll
-                    for (int i = 0; i < RPW; ++i)
-                        if (in_m(i, jx)) {
-                            acc = fmaf(G[i][jx], sk[warp + kRows * i], acc);
-                            pl = fmaf(G[i][jx], Aprev[el(i, jx)], pl);
-                        }
-                    if (lane + 32 * jx < dv) scol[warp][lane + 32 * jx] = acc;
+                    if (!col_ok(jx)) continue;
+                    a2 = fmaf(G[jx], sV[i * dv + lane + 32 * jx], a2);
+                    const float Ap = t > tb ? seg[(i - 1) * kRows * dv + at(jx)]
+                                            : ck[s * kRows * dv + at(jx)];
+                    pl = fmaf(G[jx], Ap, pl);
+                    scol[at(jx)] = G[jx] * kr;
                 }
+                a2 = warp_sum(a2);
+                if (row_ok && lane == 0) p.gk[(bh * T + e) * dk + r] += eta * a2;
+                pe = fmaf(kr, a2, pe);
                 __syncthreads();
                 for (int c = tid; c < dv; c += kThreads) {
-                    float acc = 0.f;
-                    for (int w = 0; w < kRows; ++w) acc += scol[w][c];
-                    p.gv[(bh * T + e) * dv + c] += eta * acc;
+                    float sum = 0.f;
+                    for (int w = 0; w < kRows; ++w) sum += scol[w * dv + c];
+                    atomicAdd(&p.gv[(bh * T + e) * dv + c], eta * sum);
                 }
+                __syncthreads();
 #pragma unroll
-                for (int i = 0; i < RPW; ++i)
-#pragma unroll
-                    for (int jx = 0; jx < CPL; ++jx) G[i][jx] *= lam;
+                for (int jx = 0; jx < CPL; ++jx) G[jx] *= lam;
             }
         }
     }
-    // block sums of the partials (pl per thread; pe and pg are the same in
-    // every lane of a warp, so only lane 0 contributes them)
+    // partials of this CTA: pl differs per lane; pe and pg are equal in all
+    // lanes of a warp (only lane 0's count); rows past dk hold zeros
+    __shared__ float sred[3][kRows];
     pl = warp_sum(pl);
     if (lane == 0) {
         sred[0][warp] = pl;
@@ -429,21 +409,23 @@ __global__ void __launch_bounds__(kThreads) bwd_l2_kernel(BwdParams p) {
     if (tid < 3) {
         float a = 0.f;
         for (int w = 0; w < kRows; ++w) a += sred[tid][w];
-        p.part[bh * 3 + tid] = a;
+        p.part[(bh * nrs + blockIdx.x) * 3 + tid] = a;
     }
 }
 
 // dlam, deta, dg per head: the (b,h) partials summed over the batch in a
 // fixed order.
-__global__ void bwd_reduce_kernel(BwdParams p) {
+__global__ void bwd_reduce_kernel(BwdParams p, int nrs) {
     const int64_t h = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (h >= p.H) return;
     float a = 0.f, b_ = 0.f, c = 0.f;
-    for (int64_t b = 0; b < p.B; ++b) {
-        a += p.part[(b * p.H + h) * 3 + 0];
-        b_ += p.part[(b * p.H + h) * 3 + 1];
-        c += p.part[(b * p.H + h) * 3 + 2];
-    }
+    for (int64_t b = 0; b < p.B; ++b)
+        for (int x = 0; x < nrs; ++x) {
+            const float *pp = p.part + ((b * p.H + h) * nrs + x) * 3;
+            a += pp[0];
+            b_ += pp[1];
+            c += pp[2];
+        }
     p.dlam[h] = a;
     p.deta[h] = b_;
     p.dg[h] = c;
@@ -455,15 +437,16 @@ struct BwdLayout {
     size_t lse, Dt, ckpt, seg, part, total;
 };
 BwdLayout bwd_layout(const tc_prefill_desc &d) {
-    const int64_t BH = d.B * d.H, nel = d.dk * d.dv;
+    const int64_t BH = d.B * d.H, nrs = (d.dk + kRows - 1) / kRows;
+    const int64_t slab = nrs * kRows * d.dv;  // rows of A / G padded to whole CTAs
     const int64_t nCk = (d.T + kCk - 1) / kCk;
     BwdLayout L;
     L.lse = 0;
     L.Dt = L.lse + align256((size_t)(BH * d.T) * sizeof(float));
     L.ckpt = L.Dt + align256((size_t)(BH * d.T) * sizeof(float));
-    L.seg = L.ckpt + align256((size_t)(BH * nCk * nel) * sizeof(float));
-    L.part = L.seg + align256((size_t)(BH * kCk * nel) * sizeof(float));
-    L.total = L.part + align256((size_t)(BH * 3) * sizeof(float));
+    L.seg = L.ckpt + align256((size_t)(BH * nCk * slab) * sizeof(float));
+    L.part = L.seg + align256((size_t)(BH * kCk * slab) * sizeof(float));
+    L.total = L.part + align256((size_t)(BH * nrs * 3) * sizeof(float));
     return L;
 }
 
@@ -479,10 +462,15 @@ cudaError_t launch_t(const BwdParams &p, cudaStream_t s) {
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
-    bwd_l2_kernel<Tin><<<(unsigned)BH, kThreads, 0, s>>>(p);
-    cudaError_t e = cudaGetLastError();
+    const int nrs = (p.dk + kRows - 1) / kRows;
+    const size_t smem = (size_t)(2 * kCk * kRows + 2 * kCk * p.dv + kRows * p.dv) * sizeof(float);
+    cudaError_t e = cudaFuncSetAttribute(bwd_l2_kernel<Tin>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    bwd_reduce_kernel<<<(unsigned)((p.H + 127) / 128), 128, 0, s>>>(p);
+    bwd_l2_kernel<Tin><<<dim3((unsigned)nrs, (unsigned)BH), kThreads, smem, s>>>(p);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    bwd_reduce_kernel<<<(unsigned)((p.H + 127) / 128), 128, 0, s>>>(p, nrs);
     return cudaGetLastError();
 }
 
