@@ -32,7 +32,7 @@
 //
 // Roles in the main kernel (384 threads):
 //   warp 0        TMA producer: Q tile, then K/V tiles through an NS-stage ring
-//   warp 1        MMA issuer: S = Q K^T into TMEM (double buffered), O += P V
+//   warp 1        MMA issuer: S = Q K^T into TMEM (two buffers), O += P V
 //                 with P read from TMEM, the L2 MMAs; owns TMEM
 //   warps 4-7     softmax + epilogue: one thread per query row / TMEM lane
 //   warps 8-11    state: keeps S (float32, registers), stages it as bf16 for
@@ -145,6 +145,30 @@ __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volati
     return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort, status));
 }
 
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
+// Two-wide float32 arithmetic (fma / add on register pairs).
+__device__ __forceinline__ uint64_t f2pack(float a, float b) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+    return r;
+}
+__device__ __forceinline__ void ffma2(float &d0, float &d1, float a0, float a1, uint64_t b, uint64_t c) {
+    asm("{\n\t.reg .b64 a, d;\n\tmov.b64 a, {%2, %3};\n\tfma.rn.f32x2 d, a, %4, %5;\n\t"
+        "mov.b64 {%0, %1}, d;\n\t}"
+        : "=f"(d0), "=f"(d1)
+        : "f"(a0), "f"(a1), "l"(b), "l"(c));
+}
+__device__ __forceinline__ void fadd2_acc(uint64_t &acc, float a0, float a1) {
+    asm("{\n\t.reg .b64 a;\n\tmov.b64 a, {%1, %2};\n\tadd.rn.f32x2 %0, %0, a;\n\t}"
+        : "+l"(acc)
+        : "f"(a0), "f"(a1));
+}
+
 __device__ __forceinline__ float ex2(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -203,12 +227,10 @@ __device__ __forceinline__ float window_max(const float (&s)[64], int rc) {
 #pragma unroll
     for (int i = 0; i < 8; ++i) m[i] = -INFINITY;
 #pragma unroll
-    for (int c = 0; c < 64; ++c) m[c & 7] = fmaxf(m[c & 7], in_window<KIND>(c, rc) ? s[c] : -INFINITY);
-#pragma unroll
-    for (int i = 4; i >= 1; i >>= 1)
-#pragma unroll
-        for (int j = 0; j < i; ++j) m[j] = fmaxf(m[j], m[j + i]);
-    return m[0];
+    for (int c = 0; c < 64; c += 2)
+        m[(c >> 1) & 7] = fmax3(m[(c >> 1) & 7], in_window<KIND>(c, rc) ? s[c] : -INFINITY,
+                                in_window<KIND>(c + 1, rc) ? s[c + 1] : -INFINITY);
+    return fmax3(fmax3(m[0], m[1], m[2]), fmax3(m[3], m[4], m[5]), fmaxf(m[6], m[7]));
 }
 
 // P = exp2(s * sl2 - m) on window columns (0 elsewhere) as bf16 pairs into 32
@@ -216,22 +238,28 @@ __device__ __forceinline__ float window_max(const float (&s)[64], int rc) {
 template <int KIND>
 __device__ __forceinline__ float write_p(const float (&s)[64], int rc, float sl2, float m,
                                       uint32_t taddr) {
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    uint64_t acc[2] = {0ull, 0ull};  // (0.f, 0.f) pairs
+    const uint64_t sl2p = f2pack(sl2, sl2), negm = f2pack(-m, -m);
 #pragma unroll
     for (int c0 = 0; c0 < 64; c0 += 32) {
         uint32_t pk[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
             const int c = c0 + 2 * e;
-            const float x0 = mask_window<KIND>(fmaf(s[c], sl2, -m), c, rc);
-            const float x1 = mask_window<KIND>(fmaf(s[c + 1], sl2, -m), c + 1, rc);
+            float x0, x1;
+            ffma2(x0, x1, s[c], s[c + 1], sl2p, negm);
+            x0 = mask_window<KIND>(x0, c, rc);
+            x1 = mask_window<KIND>(x1, c + 1, rc);
             const float p0 = ex2(x0), p1 = ex2(x1);
-            acc[e & 3] += p0 + p1;
+            fadd2_acc(acc[e & 1], p0, p1);
             pk[e] = pack_bf16(p0, p1);
         }
         tmem_st16(taddr + c0 / 2, pk);
     }
-    return (acc[0] + acc[1]) + (acc[2] + acc[3]);
+    float a0, a1, b0, b1;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(a0), "=f"(a1) : "l"(acc[0]));
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(b0), "=f"(b1) : "l"(acc[1]));
+    return (a0 + b0) + (a1 + b1);
 }
 
 // P' = eta lam^(r-c) s for c <= r (the zero-padded table gives 0 for c > r)
@@ -475,8 +503,8 @@ __global__ void __launch_bounds__(kMainThreads, 1)
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + OFF_BAR);
     uint64_t *q_full = bars, *q_empty = bars + 2;
     uint64_t *kv_full = bars + 4, *kv_empty = kv_full + NS;
-    uint64_t *s_full = kv_empty + NS, *p_full = s_full + 2, *s_empty = p_full + 2;
-    uint64_t *o_prog = s_empty + 2, *o_full = o_prog + 1, *o_empty = o_full + 1;
+    uint64_t *s_full = kv_empty + NS, *p_full = s_full + 2;
+    uint64_t *o_prog = p_full + 2, *o_full = o_prog + 1, *o_empty = o_full + 1;
     uint64_t *sst_full = o_empty + 1, *kt_full = sst_full + 1, *ds_full = kt_full + 1;
     uint64_t *lead_ready = ds_full + 1, *mma_done = lead_ready + 1;
     uint64_t *sm_sync = mma_done + 1, *st_sync = sm_sync + 1;  // group barriers (256, 128)
@@ -496,7 +524,6 @@ __global__ void __launch_bounds__(kMainThreads, 1)
             mbar_init(&q_empty[b], 1);
             mbar_init(&s_full[b], 1);
             mbar_init(&p_full[b], 256);
-            mbar_init(&s_empty[b], 1);
         }
         for (int s = 0; s < NS; ++s) {
             mbar_init(&kv_full[s], 1);
@@ -571,7 +598,10 @@ __global__ void __launch_bounds__(kMainThreads, 1)
         // One flat stream over the CTA's key tiles: Q K^T of key tile g is
         // issued before P V of key tile g-1, also across query tiles, so the
         // next tile's first scores are ready when the softmax side finishes
-        // the current tile.
+        // the current tile.  Q K^T of tile g+1 overwrites the score buffer
+        // whose P (and P') the P V (and P'V) of tile g-1 reads; it is issued
+        // right after them without waiting for their completion, because the
+        // tensor core runs one thread's MMAs in issue order.
         {
             const uint32_t id_qk = idesc_bf16(128, 128, false, false);
             const uint32_t id_pv = idesc_bf16(128, 64, false, true);
@@ -619,7 +649,6 @@ __global__ void __launch_bounds__(kMainThreads, 1)
                     mma_commit_w(ds_full);
                     ++lc;
                 }
-                mma_commit_w(&s_empty[sb]);
                 mma_commit_w(o_prog);
                 mma_commit_w(&kv_empty[s]);
                 if (pv.last) {
@@ -641,7 +670,6 @@ __global__ void __launch_bounds__(kMainThreads, 1)
                         if (!(ok = warp_wait(&kv_full[s], (g / NS) & 1, abort, p.status))) break;
                         // the state warps read the leading key tile: hand it on
                         if (j == 0 && ti.l2) mbar_arrive_w(lead_ready);
-                        if (!(ok = warp_wait(&s_empty[sb], ((g >> 1) & 1) ^ 1, abort, p.status))) break;
                         tc_fence_after();
                         const uint32_t k_addr = kv_base + s * 2 * TILE_B;
 #pragma unroll
