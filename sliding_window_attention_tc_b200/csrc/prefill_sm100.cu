@@ -204,40 +204,43 @@ enum { KIND_FULL = 0, KIND_DIAG = 1, KIND_LEAD = 2, KIND_LEAD_L2 = 3 };
 
 // rc = r - cb: the row index relative to this half's first column cb, so a
 // local column c is global column cb + c.  One instance of each kind serves
-// both halves (smaller code, fewer instruction-cache misses).
+// both halves, and DIAG and LEAD share one masked instance: column c is in
+// the window iff rcx - sgn * c >= 0, with (rcx, sgn) = (rc, 1) for DIAG
+// (c <= rc) and (-rc - 1, -1) for LEAD (c > rc).  The kernel's code exceeds
+// the SM instruction cache, so smaller code is faster.
 template <int KIND>
-__device__ __forceinline__ bool in_window(int c, int rc) {
-    return KIND == KIND_FULL ? true : (KIND == KIND_DIAG ? c <= rc : c > rc);
+__device__ __forceinline__ bool in_window(int c, int rcx, int sgn) {
+    return KIND == KIND_FULL ? true : rcx - sgn * c >= 0;
 }
 
 // x on window columns, -inf elsewhere, without predicate registers: the sign
 // of (rc - c) or (c - rc - 1) selects the bits of x or of -inf (one LOP3).
 template <int KIND>
-__device__ __forceinline__ float mask_window(float x, int c, int rc) {
+__device__ __forceinline__ float mask_window(float x, int c, int rcx, int sgn) {
     if (KIND == KIND_FULL) return x;
-    const int d = KIND == KIND_DIAG ? rc - c : c - rc - 1;
+    const int d = rcx - sgn * c;
     const int m = d >> 31;  // 0 in the window, -1 outside
     return __int_as_float((__float_as_int(x) & ~m) | (int(0xff800000u) & m));
 }
 
 // Row maximum of the raw scores over this half's window columns (-inf if none).
 template <int KIND>
-__device__ __forceinline__ float window_max(const float (&s)[64], int rc) {
+__device__ __forceinline__ float window_max(const float (&s)[64], int rc, int sgn) {
     float m[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) m[i] = -INFINITY;
 #pragma unroll
     for (int c = 0; c < 64; c += 2)
-        m[(c >> 1) & 7] = fmax3(m[(c >> 1) & 7], in_window<KIND>(c, rc) ? s[c] : -INFINITY,
-                                in_window<KIND>(c + 1, rc) ? s[c + 1] : -INFINITY);
+        m[(c >> 1) & 7] = fmax3(m[(c >> 1) & 7], in_window<KIND>(c, rc, sgn) ? s[c] : -INFINITY,
+                                in_window<KIND>(c + 1, rc, sgn) ? s[c + 1] : -INFINITY);
     return fmax3(fmax3(m[0], m[1], m[2]), fmax3(m[3], m[4], m[5]), fmaxf(m[6], m[7]));
 }
 
 // P = exp2(s * sl2 - m) on window columns (0 elsewhere) as bf16 pairs into 32
 // TMEM columns starting at taddr; returns this half's row sum of P.
 template <int KIND>
-__device__ __forceinline__ float write_p(const float (&s)[64], int rc, float sl2, float m,
-                                      uint32_t taddr) {
+__device__ __forceinline__ float write_p(const float (&s)[64], int rc, int sgn, float sl2,
+                                      float m, uint32_t taddr) {
     uint64_t acc[2] = {0ull, 0ull};  // (0.f, 0.f) pairs
     const uint64_t sl2p = f2pack(sl2, sl2), negm = f2pack(-m, -m);
 #pragma unroll
@@ -248,8 +251,8 @@ __device__ __forceinline__ float write_p(const float (&s)[64], int rc, float sl2
             const int c = c0 + 2 * e;
             float x0, x1;
             ffma2(x0, x1, s[c], s[c + 1], sl2p, negm);
-            x0 = mask_window<KIND>(x0, c, rc);
-            x1 = mask_window<KIND>(x1, c + 1, rc);
+            x0 = mask_window<KIND>(x0, c, rc, sgn);
+            x1 = mask_window<KIND>(x1, c + 1, rc, sgn);
             const float p0 = ex2(x0), p1 = ex2(x1);
             fadd2_acc(acc[e & 1], p0, p1);
             pk[e] = pack_bf16(p0, p1);
@@ -296,9 +299,9 @@ __device__ __forceinline__ int slice_kind(int kind, int rc) {
 __device__ __forceinline__ float half_max(int kind, const float (&s)[64], int rc) {
     switch (kind) {
         case SLICE_NONE: return -INFINITY;
-        case KIND_FULL: return window_max<KIND_FULL>(s, rc);
-        case KIND_DIAG: return window_max<KIND_DIAG>(s, rc);
-        default: return window_max<KIND_LEAD>(s, rc);
+        case KIND_FULL: return window_max<KIND_FULL>(s, rc, 1);
+        case KIND_DIAG: return window_max<KIND_DIAG>(s, rc, 1);
+        default: return window_max<KIND_DIAG>(s, -rc - 1, -1);
     }
 }
 __device__ __forceinline__ float half_p(int kind, const float (&s)[64], int rc, float sl2, float m,
@@ -312,9 +315,9 @@ __device__ __forceinline__ float half_p(int kind, const float (&s)[64], int rc, 
             tmem_st16(taddr + 16, z);
             return 0.f;
         }
-        case KIND_FULL: return write_p<KIND_FULL>(s, rc, sl2, m, taddr);
-        case KIND_DIAG: return write_p<KIND_DIAG>(s, rc, sl2, m, taddr);
-        default: return write_p<KIND_LEAD>(s, rc, sl2, m, taddr);
+        case KIND_FULL: return write_p<KIND_FULL>(s, rc, 1, sl2, m, taddr);
+        case KIND_DIAG: return write_p<KIND_DIAG>(s, rc, 1, sl2, m, taddr);
+        default: return write_p<KIND_DIAG>(s, -rc - 1, -1, sl2, m, taddr);
     }
 }
 
@@ -601,7 +604,9 @@ __global__ void __launch_bounds__(kMainThreads, 1)
         // the current tile.  Q K^T of tile g+1 overwrites the score buffer
         // whose P (and P') the P V (and P'V) of tile g-1 reads; it is issued
         // right after them without waiting for their completion, because the
-        // tensor core runs one thread's MMAs in issue order.
+        // tensor core runs one thread's MMAs in issue order.  The MMA loops
+        // are not unrolled: the issue is nearly synchronous anyway, and the
+        // smaller code misses the instruction cache less often.
         {
             const uint32_t id_qk = idesc_bf16(128, 128, false, false);
             const uint32_t id_pv = idesc_bf16(128, 64, false, true);
@@ -624,25 +629,25 @@ __global__ void __launch_bounds__(kMainThreads, 1)
                 tc_fence_after();
                 const uint32_t v_addr = kv_base + s * 2 * TILE_B + TILE_B;
                 const uint32_t s_col = tb + TM_S + sb * 128;
-#pragma unroll
+#pragma unroll 1
                 for (int k = 0; k < 8; ++k)
                     mma_ts_w(tb + TM_O, s_col + 8 * k, sdesc_sw128(v_addr + 2048 * k, TILE_B, 1024),
                            id_pv, (!pv.first || k > 0));
                 if (pv.first && pv.l2) {
                     const uint32_t q_addr = q_base + (pv.tile & 1) * TILE_B;
-#pragma unroll
+#pragma unroll 1
                     for (int k = 0; k < 8; ++k)
                         mma_ts_w(tb + TM_MI, s_col + 64 + 8 * k,
                                sdesc_sw128(v_addr + 2048 * k, TILE_B, 1024), id_pv, k > 0);
                     if (!warp_wait(sst_full, lc & 1, abort, p.status)) return false;
                     tc_fence_after();
-#pragma unroll
+#pragma unroll 1
                     for (int k = 0; k < 4; ++k)
                         mma_ss_w(tb + TM_MX, sdesc_sw128(q_addr + 32 * k, 16, 1024),
                                sdesc_sw128(sb_addr + 2048 * k, 8192, 1024), id_qs, k > 0);
                     if (!warp_wait(kt_full, lc & 1, abort, p.status)) return false;
                     tc_fence_after();
-#pragma unroll
+#pragma unroll 1
                     for (int k = 0; k < 8; ++k)
                         mma_ss_w(tb + TM_DS, sdesc_sw128(kt_addr + 2048 * k, TILE_B, 1024),
                                sdesc_sw128(v_addr + 2048 * k, TILE_B, 1024), id_ds, k > 0);
@@ -672,7 +677,7 @@ __global__ void __launch_bounds__(kMainThreads, 1)
                         if (j == 0 && ti.l2) mbar_arrive_w(lead_ready);
                         tc_fence_after();
                         const uint32_t k_addr = kv_base + s * 2 * TILE_B;
-#pragma unroll
+#pragma unroll 1
                         for (int k = 0; k < 4; ++k)
                             mma_ss_w(tb + TM_S + sb * 128, sdesc_sw128(q_addr + 32 * k, 16, 1024),
                                    sdesc_sw128(k_addr + 32 * k, 16, 1024), id_qk, k > 0);
