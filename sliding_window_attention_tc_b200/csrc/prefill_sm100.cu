@@ -55,6 +55,7 @@ constexpr int HD = 64;                   // head dimension handled here
 constexpr int NS = 4;                    // K/V stages (main kernel)
 constexpr uint32_t TILE_B = BM * HD * 2; // 16 KB bf16 tile
 constexpr int kMainThreads = 512;
+constexpr int kMaxSpans = 64;           // spans per head at most (choose_spans)
 
 // main-kernel shared memory (offsets from a 1024-aligned base)
 constexpr uint32_t OFF_Q = 0;                          // 2 Q tiles
@@ -79,6 +80,13 @@ constexpr uint32_t TM_DS = 448; // state increment: rows 0-63 hi part, 64-127 lo
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescale = 8.0f;  // rescale O only when the running max grows by > 2^8
 
+struct PrefixParams {
+    float *dA;            // [BH * (n_s - 1) * n_parts][64][64]: partial summaries in,
+                          // span start states out (over part 0 of the previous span)
+    const float *lam;
+    int T, W, H, nT, n_s, n_parts, q_off;
+};
+
 // Token coordinates.  The kernels run over a combined sequence of T tokens:
 // the first q_off are a halo (the keys and values of the tokens just before
 // a continued sequence, read through their own tensor maps), the rest are the
@@ -88,16 +96,16 @@ struct MainParams {
     void *y;
     float *A_final;
     const float *lam, *eta, *g;
-    const float *dA;      // [BH * n_s][64][64] span summaries
+    const float *S_pre;   // state at the start of span js >= 1: matrix (bh (n_s-1) + js-1) n_parts
     const float *A_init;  // [BH][64][64] state before the first eviction, or null
-    int T, W, H, BH, nT, n_s, l1_only, q_off;
+    int T, W, H, BH, nT, n_s, n_parts, l1_only, q_off;
     int *status;
 };
 
 struct SumParams {
-    float *dA;
+    float *dA;            // [BH * (n_s - 1) * n_parts][64][64] partial span summaries
     const float *lam, *eta;
-    int T, W, H, BH, nT, n_s, q_off;
+    int T, W, H, BH, nT, n_s, n_parts, q_off;
     int *status;
 };
 
@@ -346,10 +354,59 @@ __device__ __forceinline__ void build_scaled_key_row(const uint8_t *ktile, uint8
 }
 
 // ============================================================================
+// Span start states: S_pre(js) = sum over the spans u < js of
+//   lam^(n_start(js) - e_end(u)) dA_u,  dA_u = sum of its parts,
+// as the recurrence S_pre(js) = lam^(n_start(js) - n_start(js-1)) S_pre(js-1)
+//                               + lam^(n_start(js) - e_end(js-1)) dA_(js-1).
+// One thread per (b,h, element); spans in order, parts in index order.  The
+// start state of span js is written over part 0 of span js-1 (the same thread
+// has read that element already).
+// ============================================================================
+__global__ void __launch_bounds__(256) span_prefix_kernel(PrefixParams p) {
+    // decay coefficients per span, once per block: c1 for the previous start
+    // state, c2 for the previous span's summary (lam^0 = 1 also for lam = 0)
+    __shared__ float c1s[kMaxSpans], c2s[kMaxSpans];
+    const int bh = blockIdx.y;
+    const int h = bh % p.H;
+    const int per_head = p.n_s - 1;
+    if (threadIdx.x >= 1 && (int)threadIdx.x < p.n_s) {
+        const int js = threadIdx.x;
+        const double l2l = log2((double)p.lam[h]);
+        const int E = p.T > p.W ? p.T - p.W : 0;
+        int a0, a1, b0, b1, z0, z1;
+        span_range(js - 1, p.nT, p.n_s, p.q_off / BM, a0, a1);
+        span_range(js, p.nT, p.n_s, p.q_off / BM, b0, b1);
+        const int n_start = max(0, b0 * BM - p.W);
+        const int e_end = max(0, min(E, a1 * BM - p.W));
+        int n_prev = 0;
+        if (js > 1) {
+            span_range(js - 1, p.nT, p.n_s, p.q_off / BM, z0, z1);
+            n_prev = max(0, z0 * BM - p.W);
+        }
+        const int n1 = n_start - n_prev, n2 = n_start - e_end;
+        c1s[js] = n1 == 0 ? 1.f : (float)exp2((double)n1 * l2l);
+        c2s[js] = n2 == 0 ? 1.f : (float)exp2((double)n2 * l2l);
+    }
+    __syncthreads();
+    const int x = blockIdx.x * blockDim.x + threadIdx.x;  // element of the 64 x 64 state
+    if (x >= HD * HD) return;
+    float acc = 0.f;
+#pragma unroll 4
+    for (int js = 1; js < p.n_s; ++js) {
+        float *src = p.dA + ((size_t)(bh * per_head + js - 1) * p.n_parts) * HD * HD + x;
+        float d = 0.f;
+        for (int q = 0; q < p.n_parts; ++q) d += src[(size_t)q * HD * HD];
+        acc = c1s[js] * acc + c2s[js] * d;
+        src[0] = acc;
+    }
+}
+
+// ============================================================================
 // Pre-pass: dA_u = sum over the evictions e of span u of
 //           eta lam^(e_end - 1 - e) k_e v_e^T     (e_end = end of span u)
 // ============================================================================
 constexpr int NS_SUM = 2;
+constexpr int kSumTilesPerPart = 3;  // eviction tiles per span-summary CTA
 constexpr uint32_t SOFF_KV = 0;
 constexpr uint32_t SOFF_KT = SOFF_KV + NS_SUM * 2 * TILE_B;  // one buffer (hi, lo)
 constexpr uint32_t SOFF_DS = SOFF_KV;                        // scratch: stage 0, after the MMAs
@@ -372,14 +429,20 @@ __global__ void __launch_bounds__(192, 2)
 
     const int tid = threadIdx.x, warp = tid >> 5;
     const int per_head = p.n_s - 1;
-    const int bh = blockIdx.x / per_head, js = blockIdx.x % per_head;
+    const int slot = blockIdx.x;  // (bh, js, part)
+    const int part = slot % p.n_parts;
+    const int bh = slot / (per_head * p.n_parts), js = (slot / p.n_parts) % per_head;
     const int h = bh % p.H;
     int i0, i1;
     span_range(js, p.nT, p.n_s, p.q_off / BM, i0, i1);
     const int E = p.T > p.W ? p.T - p.W : 0;
-    const int ev_first = i0 > p.W / BM ? i0 : p.W / BM;  // first tile with evictions
-    const int ne = i1 > ev_first ? i1 - ev_first : 0;
-    const int e_end = ne > 0 ? min(E, i1 * BM - p.W) : 0;
+    const int ev_span = i0 > p.W / BM ? i0 : p.W / BM;  // first tile of the span with evictions
+    const int ne_span = i1 > ev_span ? i1 - ev_span : 0;
+    // this CTA's share of the span's eviction tiles; every part decays to
+    // the span's end e_end, so the parts add up to the span's summary
+    const int ev_first = ev_span + (int)((long long)ne_span * part / p.n_parts);
+    const int ne = ev_span + (int)((long long)ne_span * (part + 1) / p.n_parts) - ev_first;
+    const int e_end = ne_span > 0 ? min(E, i1 * BM - p.W) : 0;
 
     if (tid == 0) {
         for (int s = 0; s < NS_SUM; ++s) {
@@ -400,7 +463,7 @@ __global__ void __launch_bounds__(192, 2)
     __syncthreads();
     tc_fence_after();
     const uint32_t tb = *tmem_base;
-    float *out = p.dA + (size_t)(bh * p.n_s + js) * HD * HD;
+    float *out = p.dA + (size_t)slot * HD * HD;
 
     if (ne == 0) {
         for (int x = tid; x < HD * HD; x += blockDim.x) out[x] = 0.f;
@@ -862,17 +925,12 @@ __global__ void __launch_bounds__(kMainThreads, 1)
 #pragma unroll
                 for (int c = 0; c < 64; ++c) S[c] = coef * src[c];
             }
-            if (!l1_only && u < 64 && n_start > 0) {
-                for (int jj = 0; jj < js; ++jj) {
-                    int a0, a1;
-                    span_range(jj, p.nT, p.n_s, p.q_off / BM, a0, a1);
-                    const int e_end = max(0, min(E, a1 * BM - p.W));
-                    if (e_end <= 0) continue;
-                    const float coef = (float)exp2((double)(n_start - e_end) * l2l);
-                    const float *src = p.dA + ((size_t)(bh * p.n_s + jj) * HD + u) * HD;
+            if (!l1_only && u < 64 && js > 0) {
+                // the predecessors' evictions, from span_prefix_kernel
+                const float *src =
+                    p.S_pre + (((size_t)(bh * (p.n_s - 1) + js - 1) * p.n_parts) * HD + u) * HD;
 #pragma unroll
-                    for (int c = 0; c < 64; ++c) S[c] = fmaf(coef, src[c], S[c]);
-                }
+                for (int c = 0; c < 64; ++c) S[c] += src[c];
             }
             bool have_prev = false;
             int c_prev = 0;
@@ -996,7 +1054,7 @@ constexpr int kSpanOverheadTiles = 2;
 int choose_spans(int64_t BH, int nT, int num_sms) {
     int best = 1;
     int64_t best_cost = INT64_MAX;
-    for (int ns = 1; ns <= nT && ns <= 64; ++ns) {
+    for (int ns = 1; ns <= nT && ns <= kMaxSpans; ++ns) {
         const int64_t spans = BH * ns;
         const int64_t G = spans < num_sms ? spans : num_sms;
         const int64_t per_cta = (spans + G - 1) / G;
@@ -1024,11 +1082,24 @@ static int spans_for(const tc_prefill_desc &d, int num_sms) {
     return choose_spans(d.B * d.H, nT_new, num_sms);
 }
 
+// Parts per span summary: about kSumTilesPerPart eviction tiles per CTA, and
+// at most about 4 CTAs per SM in all (which also bounds the workspace).
+static int parts_for(int nT_new, int ns, int64_t BH, int num_sms) {
+    const int tiles = (nT_new + ns - 1) / ns;
+    int parts = (tiles + kSumTilesPerPart - 1) / kSumTilesPerPart;
+    const int64_t cap = (int64_t)4 * num_sms / (BH * (ns - 1));
+    if (parts > cap) parts = (int)cap;
+    return parts < 1 ? 1 : (parts > 16 ? 16 : parts);
+}
+
 size_t sm100_workspace_bytes(const tc_prefill_desc &d, int num_sms) {
     if (d.flags & TC_PREFILL_L1_ONLY) return 0;
     const int ns = spans_for(d, num_sms);
     if (ns <= 1) return 0;
-    return (size_t)(d.B * d.H * ns) * HD * HD * sizeof(float);
+    const int nT_new = (int)((d.T + BM - 1) / BM);
+    const int64_t BH = d.B * d.H;
+    const size_t mats = (size_t)BH * (ns - 1) * parts_for(nT_new, ns, BH, num_sms);
+    return mats * HD * HD * sizeof(float);
 }
 
 int sm100_launch_count(const tc_prefill_desc &d) {
@@ -1039,7 +1110,7 @@ int sm100_launch_count(const tc_prefill_desc &d) {
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     else
         cudaGetLastError();
-    return 1 + ((!l1 && spans_for(d, sms) > 1) ? 1 : 0);
+    return 1 + ((!l1 && spans_for(d, sms) > 1) ? 2 : 0);
 }
 
 cudaError_t launch_prefill_sm100(const PrefillParams &p, int num_sms, cudaStream_t s) {
@@ -1065,15 +1136,22 @@ cudaError_t launch_prefill_sm100(const PrefillParams &p, int num_sms, cudaStream
     e = cudaFuncSetAttribute(span_summary_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              SMEM_SUM);
     if (e != cudaSuccess) return e;
+    const int n_parts = ns > 1 ? parts_for(nT - q_off / BM, ns, BH, num_sms) : 1;
     float *dA = reinterpret_cast<float *>(p.workspace);
     if (!p.l1_only && ns > 1) {
-        SumParams sp{dA, p.lam, p.eta, T_all, (int)p.W, (int)p.H, (int)BH, nT, ns, q_off, p.status};
-        span_summary_kernel<<<(unsigned)(BH * (ns - 1)), 192, SMEM_SUM, s>>>(tk, tv, tkh, tvh, sp);
+        SumParams sp{dA, p.lam, p.eta, T_all, (int)p.W, (int)p.H, (int)BH, nT, ns, n_parts, q_off,
+                     p.status};
+        span_summary_kernel<<<(unsigned)(BH * (ns - 1) * n_parts), 192, SMEM_SUM, s>>>(tk, tv, tkh,
+                                                                                    tvh, sp);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+        PrefixParams pp{dA, p.lam, T_all, (int)p.W, (int)p.H, nT, ns, n_parts, q_off};
+        span_prefix_kernel<<<dim3(HD * HD / 256, (unsigned)BH), 256, 0, s>>>(pp);
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
     MainParams mp{p.y,      p.A_final, p.lam, p.eta, p.g,  dA, p.A_init, T_all, (int)p.W, (int)p.H,
-                  (int)BH, nT,        ns,    p.l1_only ? 1 : 0, q_off, p.status};
+                  (int)BH, nT,        ns,    n_parts,         p.l1_only ? 1 : 0, q_off, p.status};
     const int64_t spans = BH * ns;
     const unsigned grid = (unsigned)(spans < num_sms ? spans : num_sms);
     prefill_main_kernel<<<grid, kMainThreads, SMEM_MAIN, s>>>(tq, tk, tv, tkh, tvh, mp);
