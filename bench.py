@@ -73,6 +73,25 @@ def prefill_flops(B, H, T, dk, dv, W):
     return l1, l2
 
 
+def prefill_executed_flops(B, H, T, W, tile=128, d=64):
+    """Tensor-core FLOPs that prefill_main_kernel issues for one call (the
+    bf16, d = 64 path): Q K^T and P V on every computed tile x tile block,
+    masked parts included, plus the leading tile's P'V, Q S(n0) and hi/lo state
+    MMAs for every query tile that has evictions.  (span_summary_kernel adds
+    2*tile*d*tile*2 per eviction tile of the spans it summarises.)"""
+    nT = (T + tile - 1) // tile
+    wt = W // tile
+    mma_tile = 2 * tile * tile * d                   # one 128 x 128 x 64 product
+    l1 = l2 = 0
+    for i in range(nT):
+        lead = i >= wt
+        nk = wt + 1 if lead else i + 1
+        l1 += nk * 2 * mma_tile                      # Q K^T and P V
+        if lead:
+            l2 += mma_tile + tile * d * d * 2 + mma_tile  # P'V, Q S(n0), [hi; lo] K^T V
+    return l1 * B * H, l2 * B * H
+
+
 def decode_bytes(B, H, W, dk, dv, esz=2):
     ring = B * H * W * (dk + dv) * esz
     A = 2 * B * H * dk * dv * 4
@@ -543,6 +562,9 @@ def main():
                     "peak_source": f"{peak_src} bf16 burst",
                     "kernel": "tc_prefill (all launches of one call)",
                     "algorithmic_flops_per_launch": l1f + l2f}
+        e1, e2 = prefill_executed_flops(B, H, T, x.W)
+        roofline["executed_flops_per_launch"] = e1 + e2
+        roofline["executed_tflops"] = (e1 + e2) / (mean_ms * 1e-3) / 1e12
         extras = {}
         if not args.no_extras:
             l1 = time_prefill(tc, HEADLINE, dev, max(20, args.steps // 4), 3, world,
@@ -565,7 +587,8 @@ def main():
                 "achieved_tflops": (f1 + f2) / (t_lp * 1e-3) / 1e12,
                 "frac_of_bf16_peak": (f1 + f2) / (t_lp * 1e-3) / 1e12 / peak_tf,
                 "l1_only_ms": t_lp1, "l2_overhead_ratio": t_lp / t_lp1 - 1.0,
-                "algorithmic_floor": f2 / f1}
+                "algorithmic_floor": f2 / f1,
+                "executed_tflops": sum(prefill_executed_flops(Bl, Hl, Tl, xl.W)) / (t_lp * 1e-3) / 1e12}
             del lp, lp1
             dec = time_decode(tc, dev, world, clocks=clocks)
             dms = statistics.mean(dec["per_step_ms"])

@@ -1,0 +1,53 @@
+"""Host-side work counts that bench.py reports next to its timings.
+
+The algorithmic FLOPs follow the definitions of the layer: L1 counts
+2 (d_k + d_v) per (query, key in window) pair, and L2 counts 2 d_k d_v per
+eviction plus 2 d_k d_v per token that reads the memory.  The executed counts
+follow the tiling of the bf16 tensor-core kernel: 128 x 128 tiles, and each
+query tile past the first W tokens has W/128 + 1 key tiles.  Each count is
+checked against brute-force enumeration on small shapes and against the
+closed form for the LM workload.
+"""
+import os
+import sys
+
+sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+
+import bench  # noqa: E402
+
+
+def _pairs_brute(T, W):
+    return sum(min(t + 1, W) for t in range(T))
+
+
+def test_algorithmic_flops_match_enumeration():
+    for T, W, dk, dv in [(1, 4, 8, 8), (5, 8, 4, 2), (100, 7, 16, 32), (256, 32, 16, 16)]:
+        l1, l2 = bench.prefill_flops(1, 1, T, dk, dv, W)
+        assert l1 == 2 * (dk + dv) * _pairs_brute(T, W)
+        assert l2 == 4 * dk * dv * max(0, T - W)
+
+
+def test_executed_tiles_match_enumeration():
+    # every (query tile, key tile) pair that overlaps the causal band is computed once
+    for T, W in [(128, 128), (1000, 256), (4096, 512), (32768, 1024)]:
+        nT = (T + 127) // 128
+        blocks = 0
+        lead_tiles = 0
+        for i in range(nT):
+            lo = max(0, i * 128 - W)  # first key any row of tile i sees (row 0 sees i*128-W+1..)
+            first = lo // 128
+            blocks += i - first + 1
+            lead_tiles += i * 128 >= W
+        e1, e2 = bench.prefill_executed_flops(1, 1, T, W)
+        mma_tile = 2 * 128 * 128 * 64
+        assert e1 == blocks * 2 * mma_tile, (T, W)
+        assert e2 == lead_tiles * (2 * mma_tile + 128 * 64 * 64 * 2), (T, W)
+
+
+def test_lm_workload_counts():
+    l1, l2 = bench.prefill_flops(8, 12, 4096, 64, 64, 512)
+    assert l1 + l2 == 53961818112
+    e1, e2 = bench.prefill_executed_flops(8, 12, 4096, 512)
+    # 150 computed tiles and 28 leading tiles per head
+    assert e1 == 96 * 150 * 2 * (2 * 128 * 128 * 64)
+    assert e2 == 96 * 28 * (2 * (2 * 128 * 128 * 64) + 128 * 64 * 64 * 2)
