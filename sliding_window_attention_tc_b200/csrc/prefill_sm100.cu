@@ -25,17 +25,22 @@
 //
 // Work split.  Each head's query tiles are cut into n_s contiguous spans; a
 // persistent CTA (one per SM) runs spans.  A span that starts after other
-// evictions of its head needs S at its start: a small pre-pass kernel
-// (span_summary_kernel) computes for every span u the state its own
-// evictions add, dA_u; the main kernel combines the predecessors' dA_u with
-// the decay between them.
+// evictions of its head needs S at its start.  Two small pre-pass kernels
+// provide it: span_summary_kernel computes, in parts spread over CTAs, the
+// state dA_u that the evictions of span u add (decayed to the span's end),
+// and span_prefix_kernel folds the parts and the predecessors into one start
+// state per span.
 //
-// Roles in the main kernel (384 threads):
+// Roles in the main kernel (512 threads):
 //   warp 0        TMA producer: Q tile, then K/V tiles through an NS-stage ring
 //   warp 1        MMA issuer: S = Q K^T into TMEM (two buffers), O += P V
 //                 with P read from TMEM, the L2 MMAs; owns TMEM
-//   warps 4-7     softmax + epilogue: one thread per query row / TMEM lane
-//   warps 8-11    state: keeps S (float32, registers), stages it as bf16 for
+//   warps 2-3     idle
+//   warps 4-11    softmax + epilogue, two column halves: warps 4-7 take score
+//                 columns 0-63, warps 8-11 columns 64-127; one thread per
+//                 query row / TMEM lane in each half; the halves exchange
+//                 their row maxima once per key tile
+//   warps 12-15   state: keeps S (float32, registers), stages it as bf16 for
 //                 the inter read, builds the scaled hi/lo keys
 // All waits are bounded (mbar_wait); on timeout every role drains and the
 // kernel returns with TC_ERR_DEVICE_TIMEOUT in the status word.
