@@ -11,9 +11,9 @@
 //   p = softmax(q k / sqrt(dk)), dp_j = <dy_t, v_j>, D_t = <dy_t, y_local_t>,
 //   ds_j = p_j (dp_j - D_t); dq_t += sum_j ds_j k_j / sqrt(dk),
 //   dk_j += ds_j q_t / sqrt(dk), dv_j += p_j dy_t.
-//   bwd_rows_kernel (a warp per query row) writes dq and the per-row
-//   log-sum-exp and D_t; bwd_keys_kernel (a warp per key row, over the W
-//   queries that see it) writes dk and dv.
+//   bwd_rows_kernel (a warp per 4 query rows) writes dq and the per-row
+//   log-sum-exp and D_t; bwd_keys_kernel (a warp per 4 key rows, over the W
+//   queries that see them) writes dk and dv.
 //
 // Memory (L2), a reverse scan of G_t = dL/dA_t:
 //   G_t = q_t^T (s dy_t) + [step t+1 writes] lam G_{t+1}, and each write at
@@ -37,7 +37,7 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kMaxD = 128;
-constexpr int kRows = kThreads / 32;  // query or key rows per CTA in the L1 kernels
+constexpr int kRows = kThreads / 32;  // rows of A per CTA in the L2 kernel
 constexpr int kKT = 32;               // key / query tile of the L1 kernels
 constexpr int kCk = 64;               // checkpoint interval of the L2 replay
 constexpr float kLog2e = 1.4426950408889634f;
@@ -66,197 +66,318 @@ __device__ __forceinline__ float warp_sum(float x) {
 }
 
 // ---------------------------------------------------------------------------
-// dq (window part), log-sum-exp and D_t, one warp per query row.
+// Register tiling of the window kernels.  A warp owns kQR query rows (or key
+// rows): every key (or query) value read from shared memory serves kQR
+// FMAs, and the dot products read 16 bytes at a time.  Shared rows are
+// padded to a 16-byte stride whose quads fall in distinct banks for 8
+// consecutive lanes; the padding columns are zero, so dots over them add 0.
+constexpr int kQR = 4;                        // rows per warp
+constexpr int kTileR = (kThreads / 32) * kQR;  // rows per CTA
+
+__host__ __device__ __forceinline__ int pad_stride(int d) {
+    int s = (d + 3) & ~3;
+    if (((s >> 2) & 1) == 0) s += 4;  // odd number of quads: conflict-free float4 rows
+    return s;
+}
+
+// n rows of width d from global (row stride d) into shared rows of stride sp,
+// zero past n rows of src_rows and in the padding columns.
 template <typename Tin>
+__device__ __forceinline__ void load_rows(float *dst, int sp, const Tin *src, int64_t row0,
+                                          int64_t n_valid, int n_rows, int d, int tid) {
+    const int lane = tid & 31;
+    for (int rr = tid >> 5; rr < n_rows; rr += kThreads / 32) {
+        const bool ok = rr < n_valid;
+        const Tin *s = src + (row0 + rr) * d;
+        for (int c = lane; c < sp; c += 32) dst[rr * sp + c] = (ok && c < d) ? to_f32(s[c]) : 0.f;
+    }
+}
+
+// Four dot products of one lane's row `a` (stride-1, padded to quads) with four
+// broadcast rows b[i] (same padding), over dp4 columns.
+__device__ __forceinline__ void dot4(const float *a, const float *b, int sb, int dp4, float (&out)[kQR]) {
+#pragma unroll
+    for (int i = 0; i < kQR; ++i) out[i] = 0.f;
+    for (int r = 0; r < dp4; r += 4) {
+        const float4 x = *reinterpret_cast<const float4 *>(a + r);
+#pragma unroll
+        for (int i = 0; i < kQR; ++i) {
+            const float4 y = *reinterpret_cast<const float4 *>(b + i * sb + r);
+            out[i] = fmaf(x.x, y.x, out[i]);
+            out[i] = fmaf(x.y, y.y, out[i]);
+            out[i] = fmaf(x.z, y.z, out[i]);
+            out[i] = fmaf(x.w, y.w, out[i]);
+        }
+    }
+}
+
+// dq (window part), log-sum-exp and D_t; a warp owns kQR query rows, a lane
+// one key of the current 32-key tile (scores) or output columns lane, lane+32,
+// ... (products with V and K).
+template <typename Tin, int CPL>  // CPL: output columns per lane, >= d / 32
 __global__ void __launch_bounds__(kThreads) bwd_rows_kernel(BwdParams p) {
-    constexpr int CPL = kMaxD / 32;
-    __shared__ float sk[kKT][kMaxD + 1], sv[kKT][kMaxD + 1];
-    __shared__ float sq[kRows][kMaxD], sdy[kRows][kMaxD];
+    extern __shared__ __align__(16) float shr[];
+    const int dk = p.dk, dv = p.dv;
+    const int skp = pad_stride(dk), svp = pad_stride(dv);
+    const int dk4 = (dk + 3) & ~3, dv4 = (dv + 3) & ~3;
+    float *sk = shr;                      // [kKT][skp]
+    float *sv = sk + kKT * skp;           // [kKT][svp]
+    float *sq = sv + kKT * svp;           // [kTileR][skp]
+    float *sdy = sq + kTileR * skp;       // [kTileR][svp]
+    float *spt = sdy + kTileR * svp;      // [warps][kKT][kQR]: P or dS of the warp's rows
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int64_t bh = blockIdx.y;
-    const int dk = p.dk, dv = p.dv;
     const int64_t T = p.T, W = p.W;
-    const int64_t t0 = (int64_t)blockIdx.x * kRows, t = t0 + warp;
-    const bool row_ok = t < T;
+    const int64_t t0 = (int64_t)blockIdx.x * kTileR;  // first row of the CTA
+    const int64_t tw = t0 + warp * kQR;               // first row of the warp
     const Tin *qb = reinterpret_cast<const Tin *>(p.q) + bh * T * dk;
     const Tin *kb = reinterpret_cast<const Tin *>(p.k) + bh * T * dk;
     const Tin *vb = reinterpret_cast<const Tin *>(p.v) + bh * T * dv;
     const Tin *db = reinterpret_cast<const Tin *>(p.dy) + bh * T * dv;
-    for (int x = tid; x < kRows * dk; x += kThreads) {
-        const int64_t tt = t0 + x / dk;
-        sq[x / dk][x % dk] = tt < T ? to_f32(qb[tt * dk + x % dk]) : 0.f;
-    }
-    for (int x = tid; x < kRows * dv; x += kThreads) {
-        const int64_t tt = t0 + x / dv;
-        sdy[x / dv][x % dv] = tt < T ? to_f32(db[tt * dv + x % dv]) : 0.f;
-    }
+    const int64_t n_here = T - t0 < kTileR ? T - t0 : kTileR;
+    load_rows(sq, skp, qb, t0, n_here, kTileR, dk, tid);
+    load_rows(sdy, svp, db, t0, n_here, kTileR, dv, tid);
+    float *my_p = spt + warp * kKT * kQR;
     const float scale2 = kLog2e / sqrtf((float)dk);
-    const int64_t win_lo = t - W + 1 > 0 ? t - W + 1 : 0;
-    const int64_t t_last = (t0 + kRows - 1 < T - 1) ? t0 + kRows - 1 : T - 1;
+    const int64_t t_last = (t0 + kTileR - 1 < T - 1) ? t0 + kTileR - 1 : T - 1;
     const int64_t lo = t0 - W + 1 > 0 ? t0 - W + 1 : 0;
+    const float *q_w = sq + warp * kQR * skp, *dy_w = sdy + warp * kQR * svp;
 
-    // pass 1: softmax statistics and y_local (online)
-    float m_run = -INFINITY, l_run = 0.f, acc[CPL];
+    // pass 1: softmax statistics and y_local (online), per row
+    float m_run[kQR], l_run[kQR], acc[kQR][CPL];
 #pragma unroll
-    for (int i = 0; i < CPL; ++i) acc[i] = 0.f;
+    for (int i = 0; i < kQR; ++i) {
+        m_run[i] = -INFINITY;
+        l_run[i] = 0.f;
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) acc[i][c] = 0.f;
+    }
     for (int64_t j0 = lo; j0 <= t_last; j0 += kKT) {
         const int nt = (int)((t_last - j0 + 1 < kKT) ? t_last - j0 + 1 : kKT);
         __syncthreads();
-        for (int x = tid; x < nt * dk; x += kThreads) sk[x / dk][x % dk] = to_f32(kb[(j0 + x / dk) * dk + x % dk]);
-        for (int x = tid; x < nt * dv; x += kThreads) sv[x / dv][x % dv] = to_f32(vb[(j0 + x / dv) * dv + x % dv]);
+        load_rows(sk, skp, kb, j0, nt, kKT, dk, tid);
+        load_rows(sv, svp, vb, j0, nt, kKT, dv, tid);
         __syncthreads();
-        if (!row_ok) continue;
         const int64_t j = j0 + lane;
-        const bool in_win = lane < nt && j >= win_lo && j <= t;
-        float dot = 0.f;
-        if (in_win)
-            for (int r = 0; r < dk; ++r) dot = fmaf(sq[warp][r], sk[lane][r], dot);
-        const float s = in_win ? dot * scale2 : -INFINITY;
-        const float m_new = fmaxf(m_run, warp_max(s));
-        if (m_new == -INFINITY) continue;
-        const float corr = exp2f(m_run - m_new);
-        const float pj = exp2f(s - m_new);
-        l_run = l_run * corr + warp_sum(pj);
+        float dot[kQR];
+        dot4(sk + lane * skp, q_w, skp, dk4, dot);
+        float pr[kQR];
 #pragma unroll
-        for (int i = 0; i < CPL; ++i) acc[i] *= corr;
-        m_run = m_new;
+        for (int i = 0; i < kQR; ++i) {
+            const int64_t t = tw + i;
+            const bool in_win = t < T && lane < nt && j > t - W && j <= t;
+            const float s = in_win ? dot[i] * scale2 : -INFINITY;
+            const float m_new = fmaxf(m_run[i], warp_max(s));
+            if (m_new == -INFINITY) {  // no key of this tile in the row's window yet
+                pr[i] = 0.f;
+                continue;
+            }
+            const float corr = exp2f(m_run[i] - m_new);
+            pr[i] = exp2f(s - m_new);
+            l_run[i] = l_run[i] * corr + warp_sum(pr[i]);
+#pragma unroll
+            for (int c = 0; c < CPL; ++c) acc[i][c] *= corr;
+            m_run[i] = m_new;
+        }
+        *reinterpret_cast<float4 *>(my_p + lane * kQR) = make_float4(pr[0], pr[1], pr[2], pr[3]);
+        __syncwarp();
         for (int jj = 0; jj < nt; ++jj) {
-            const float pb = __shfl_sync(0xffffffffu, pj, jj);
+            const float4 pb = *reinterpret_cast<const float4 *>(my_p + jj * kQR);
 #pragma unroll
-            for (int i = 0; i < CPL; ++i) {
-                const int c = lane + 32 * i;
-                if (c < dv) acc[i] = fmaf(pb, sv[jj][c], acc[i]);
+            for (int c = 0; c < CPL; ++c) {
+                const int col = lane + 32 * c;
+                if (col < dv) {
+                    const float vv = sv[jj * svp + col];
+                    acc[0][c] = fmaf(pb.x, vv, acc[0][c]);
+                    acc[1][c] = fmaf(pb.y, vv, acc[1][c]);
+                    acc[2][c] = fmaf(pb.z, vv, acc[2][c]);
+                    acc[3][c] = fmaf(pb.w, vv, acc[3][c]);
+                }
             }
         }
+        __syncwarp();
     }
-    float lse2 = 0.f, Dt = 0.f;
-    if (row_ok) {
-        lse2 = m_run + log2f(l_run);
+    float lse2[kQR], Dt[kQR];
+#pragma unroll
+    for (int i = 0; i < kQR; ++i) {
+        const int64_t t = tw + i;
+        lse2[i] = m_run[i] + log2f(l_run[i]);
         float d = 0.f;
 #pragma unroll
-        for (int i = 0; i < CPL; ++i) {
-            const int c = lane + 32 * i;
-            if (c < dv) d = fmaf(sdy[warp][c], acc[i] / l_run, d);
+        for (int c = 0; c < CPL; ++c) {
+            const int col = lane + 32 * c;
+            if (col < dv) d = fmaf(dy_w[i * svp + col], acc[i][c] / l_run[i], d);
         }
-        Dt = warp_sum(d);
-        if (lane == 0) {
-            p.lse[bh * T + t] = lse2;
-            p.Dt[bh * T + t] = Dt;
+        Dt[i] = warp_sum(d);
+        if (t < T && lane == 0) {
+            p.lse[bh * T + t] = lse2[i];
+            p.Dt[bh * T + t] = Dt[i];
         }
     }
     // pass 2: ds_j = p_j (dp_j - D_t); dq_t = sum_j ds_j k_j / sqrt(dk)
-    float dqa[CPL];
+    float dqa[kQR][CPL];
 #pragma unroll
-    for (int i = 0; i < CPL; ++i) dqa[i] = 0.f;
+    for (int i = 0; i < kQR; ++i)
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) dqa[i][c] = 0.f;
     const float inv_sqrt = 1.f / sqrtf((float)dk);
     for (int64_t j0 = lo; j0 <= t_last; j0 += kKT) {
         const int nt = (int)((t_last - j0 + 1 < kKT) ? t_last - j0 + 1 : kKT);
         __syncthreads();
-        for (int x = tid; x < nt * dk; x += kThreads) sk[x / dk][x % dk] = to_f32(kb[(j0 + x / dk) * dk + x % dk]);
-        for (int x = tid; x < nt * dv; x += kThreads) sv[x / dv][x % dv] = to_f32(vb[(j0 + x / dv) * dv + x % dv]);
+        load_rows(sk, skp, kb, j0, nt, kKT, dk, tid);
+        load_rows(sv, svp, vb, j0, nt, kKT, dv, tid);
         __syncthreads();
-        if (!row_ok) continue;
         const int64_t j = j0 + lane;
-        const bool in_win = lane < nt && j >= win_lo && j <= t;
-        float ds = 0.f;
-        if (in_win) {
-            float dot = 0.f, dp = 0.f;
-            for (int r = 0; r < dk; ++r) dot = fmaf(sq[warp][r], sk[lane][r], dot);
-            for (int c = 0; c < dv; ++c) dp = fmaf(sdy[warp][c], sv[lane][c], dp);
-            ds = exp2f(dot * scale2 - lse2) * (dp - Dt);
-        }
-        for (int jj = 0; jj < nt; ++jj) {
-            const float db_ = __shfl_sync(0xffffffffu, ds, jj);
+        float dot[kQR], dp[kQR], ds[kQR];
+        dot4(sk + lane * skp, q_w, skp, dk4, dot);
+        dot4(sv + lane * svp, dy_w, svp, dv4, dp);
 #pragma unroll
-            for (int i = 0; i < CPL; ++i) {
-                const int r = lane + 32 * i;
-                if (r < dk) dqa[i] = fmaf(db_, sk[jj][r], dqa[i]);
+        for (int i = 0; i < kQR; ++i) {
+            const int64_t t = tw + i;
+            const bool in_win = t < T && lane < nt && j > t - W && j <= t;
+            ds[i] = in_win ? exp2f(dot[i] * scale2 - lse2[i]) * (dp[i] - Dt[i]) : 0.f;
+        }
+        *reinterpret_cast<float4 *>(my_p + lane * kQR) = make_float4(ds[0], ds[1], ds[2], ds[3]);
+        __syncwarp();
+        for (int jj = 0; jj < nt; ++jj) {
+            const float4 db4 = *reinterpret_cast<const float4 *>(my_p + jj * kQR);
+#pragma unroll
+            for (int c = 0; c < CPL; ++c) {
+                const int r = lane + 32 * c;
+                if (r < dk) {
+                    const float kk = sk[jj * skp + r];
+                    dqa[0][c] = fmaf(db4.x, kk, dqa[0][c]);
+                    dqa[1][c] = fmaf(db4.y, kk, dqa[1][c]);
+                    dqa[2][c] = fmaf(db4.z, kk, dqa[2][c]);
+                    dqa[3][c] = fmaf(db4.w, kk, dqa[3][c]);
+                }
             }
         }
+        __syncwarp();
     }
-    if (row_ok) {
 #pragma unroll
-        for (int i = 0; i < CPL; ++i) {
-            const int r = lane + 32 * i;
-            if (r < dk) p.gq[(bh * T + t) * dk + r] = dqa[i] * inv_sqrt;
+    for (int i = 0; i < kQR; ++i) {
+        const int64_t t = tw + i;
+        if (t >= T) continue;
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) {
+            const int r = lane + 32 * c;
+            if (r < dk) p.gq[(bh * T + t) * dk + r] = dqa[i][c] * inv_sqrt;
         }
     }
 }
 
 // ---------------------------------------------------------------------------
-// dk, dv (window part), one warp per key row j over the queries t = j .. j+W-1.
-template <typename Tin>
+// dk, dv (window part); a warp owns kQR key rows j over the queries
+// t = j .. j+W-1, a lane one query of the current 32-query tile (scores) or
+// output columns lane, lane+32, ... (products with Q and dY).
+template <typename Tin, int CPL>  // CPL: output columns per lane, >= d / 32
 __global__ void __launch_bounds__(kThreads) bwd_keys_kernel(BwdParams p) {
-    constexpr int CPL = kMaxD / 32;
-    __shared__ float sq[kKT][kMaxD + 1], sdy[kKT][kMaxD + 1];
-    __shared__ float slse[kKT], sD[kKT];
-    __shared__ float sk[kRows][kMaxD], sv[kRows][kMaxD];
+    extern __shared__ __align__(16) float shr[];
+    const int dk = p.dk, dv = p.dv;
+    const int skp = pad_stride(dk), svp = pad_stride(dv);
+    const int dk4 = (dk + 3) & ~3, dv4 = (dv + 3) & ~3;
+    float *sq = shr;                      // [kKT][skp]   queries of the tile
+    float *sdy = sq + kKT * skp;          // [kKT][svp]
+    float *sk = sdy + kKT * svp;          // [kTileR][skp] keys of the CTA
+    float *sv = sk + kTileR * skp;        // [kTileR][svp]
+    float *spt = sv + kTileR * svp;       // [warps][kKT][2 kQR]: P and dS of the warp's keys
+    float *slse = spt + (kThreads / 32) * kKT * 2 * kQR;  // [kKT]
+    float *sD = slse + kKT;                               // [kKT]
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int64_t bh = blockIdx.y;
-    const int dk = p.dk, dv = p.dv;
     const int64_t T = p.T, W = p.W;
-    const int64_t j0k = (int64_t)blockIdx.x * kRows, j = j0k + warp;
-    const bool row_ok = j < T;
+    const int64_t j0k = (int64_t)blockIdx.x * kTileR;  // first key of the CTA
+    const int64_t jw = j0k + warp * kQR;               // first key of the warp
     const Tin *qb = reinterpret_cast<const Tin *>(p.q) + bh * T * dk;
     const Tin *kb = reinterpret_cast<const Tin *>(p.k) + bh * T * dk;
     const Tin *vb = reinterpret_cast<const Tin *>(p.v) + bh * T * dv;
     const Tin *db = reinterpret_cast<const Tin *>(p.dy) + bh * T * dv;
-    for (int x = tid; x < kRows * dk; x += kThreads) {
-        const int64_t jj = j0k + x / dk;
-        sk[x / dk][x % dk] = jj < T ? to_f32(kb[jj * dk + x % dk]) : 0.f;
-    }
-    for (int x = tid; x < kRows * dv; x += kThreads) {
-        const int64_t jj = j0k + x / dv;
-        sv[x / dv][x % dv] = jj < T ? to_f32(vb[jj * dv + x % dv]) : 0.f;
-    }
+    const int64_t n_here = T - j0k < kTileR ? T - j0k : kTileR;
+    load_rows(sk, skp, kb, j0k, n_here, kTileR, dk, tid);
+    load_rows(sv, svp, vb, j0k, n_here, kTileR, dv, tid);
+    float *my_p = spt + warp * kKT * 2 * kQR;
     const float scale2 = kLog2e / sqrtf((float)dk);
     const float inv_sqrt = 1.f / sqrtf((float)dk);
-    // queries that see any key of this CTA: j0k .. j0k + kRows - 1 + W - 1
-    const int64_t q_hi_all = j0k + kRows - 1 + W - 1 < T - 1 ? j0k + kRows - 1 + W - 1 : T - 1;
-    const int64_t q_hi = j + W - 1 < T - 1 ? j + W - 1 : T - 1;
-    float dka[CPL], dva[CPL];
+    // queries that see any key of this CTA: j0k .. j0k + kTileR - 1 + W - 1
+    const int64_t q_hi_all = j0k + kTileR - 1 + W - 1 < T - 1 ? j0k + kTileR - 1 + W - 1 : T - 1;
+    const float *k_w = sk + warp * kQR * skp, *v_w = sv + warp * kQR * svp;
+    float dka[kQR][CPL], dva[kQR][CPL];
 #pragma unroll
-    for (int i = 0; i < CPL; ++i) dka[i] = dva[i] = 0.f;
+    for (int i = 0; i < kQR; ++i)
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) dka[i][c] = dva[i][c] = 0.f;
     for (int64_t q0 = j0k; q0 <= q_hi_all; q0 += kKT) {
         const int nt = (int)((q_hi_all - q0 + 1 < kKT) ? q_hi_all - q0 + 1 : kKT);
         __syncthreads();
-        for (int x = tid; x < nt * dk; x += kThreads) sq[x / dk][x % dk] = to_f32(qb[(q0 + x / dk) * dk + x % dk]);
-        for (int x = tid; x < nt * dv; x += kThreads) sdy[x / dv][x % dv] = to_f32(db[(q0 + x / dv) * dv + x % dv]);
+        load_rows(sq, skp, qb, q0, nt, kKT, dk, tid);
+        load_rows(sdy, svp, db, q0, nt, kKT, dv, tid);
         if (tid < nt) {
             slse[tid] = p.lse[bh * T + q0 + tid];
             sD[tid] = p.Dt[bh * T + q0 + tid];
         }
         __syncthreads();
-        if (!row_ok) continue;
         const int64_t t = q0 + lane;
-        const bool sees = lane < nt && t >= j && t <= q_hi;
-        float pj = 0.f, ds = 0.f;
-        if (sees) {
-            float dot = 0.f, dp = 0.f;
-            for (int r = 0; r < dk; ++r) dot = fmaf(sq[lane][r], sk[warp][r], dot);
-            for (int c = 0; c < dv; ++c) dp = fmaf(sdy[lane][c], sv[warp][c], dp);
-            pj = exp2f(dot * scale2 - slse[lane]);
-            ds = pj * (dp - sD[lane]);
-        }
-        for (int tt = 0; tt < nt; ++tt) {
-            const float pb = __shfl_sync(0xffffffffu, pj, tt);
-            const float dsb = __shfl_sync(0xffffffffu, ds, tt);
+        float dot[kQR], dp[kQR], pj[kQR], ds[kQR];
+        dot4(sq + lane * skp, k_w, skp, dk4, dot);
+        dot4(sdy + lane * svp, v_w, svp, dv4, dp);
+        const float lse_t = lane < nt ? slse[lane] : 0.f, D_t = lane < nt ? sD[lane] : 0.f;
 #pragma unroll
-            for (int i = 0; i < CPL; ++i) {
-                const int r = lane + 32 * i;
-                if (r < dk) dka[i] = fmaf(dsb, sq[tt][r], dka[i]);
-                if (r < dv) dva[i] = fmaf(pb, sdy[tt][r], dva[i]);
+        for (int i = 0; i < kQR; ++i) {
+            const int64_t j = jw + i;
+            const bool sees = j < T && lane < nt && t >= j && t < j + W;
+            pj[i] = sees ? exp2f(dot[i] * scale2 - lse_t) : 0.f;
+            ds[i] = pj[i] * (dp[i] - D_t);
+        }
+        *reinterpret_cast<float4 *>(my_p + lane * 2 * kQR) = make_float4(pj[0], pj[1], pj[2], pj[3]);
+        *reinterpret_cast<float4 *>(my_p + lane * 2 * kQR + kQR) = make_float4(ds[0], ds[1], ds[2], ds[3]);
+        __syncwarp();
+        for (int tt = 0; tt < nt; ++tt) {
+            const float4 pb = *reinterpret_cast<const float4 *>(my_p + tt * 2 * kQR);
+            const float4 dsb = *reinterpret_cast<const float4 *>(my_p + tt * 2 * kQR + kQR);
+#pragma unroll
+            for (int c = 0; c < CPL; ++c) {
+                const int r = lane + 32 * c;
+                if (r < dk) {
+                    const float qq = sq[tt * skp + r];
+                    dka[0][c] = fmaf(dsb.x, qq, dka[0][c]);
+                    dka[1][c] = fmaf(dsb.y, qq, dka[1][c]);
+                    dka[2][c] = fmaf(dsb.z, qq, dka[2][c]);
+                    dka[3][c] = fmaf(dsb.w, qq, dka[3][c]);
+                }
+                if (r < dv) {
+                    const float yy = sdy[tt * svp + r];
+                    dva[0][c] = fmaf(pb.x, yy, dva[0][c]);
+                    dva[1][c] = fmaf(pb.y, yy, dva[1][c]);
+                    dva[2][c] = fmaf(pb.z, yy, dva[2][c]);
+                    dva[3][c] = fmaf(pb.w, yy, dva[3][c]);
+                }
             }
         }
+        __syncwarp();
     }
-    if (row_ok) {
 #pragma unroll
-        for (int i = 0; i < CPL; ++i) {
-            const int r = lane + 32 * i;
-            if (r < dk) p.gk[(bh * T + j) * dk + r] = dka[i] * inv_sqrt;
-            if (r < dv) p.gv[(bh * T + j) * dv + r] = dva[i];
+    for (int i = 0; i < kQR; ++i) {
+        const int64_t j = jw + i;
+        if (j >= T) continue;
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) {
+            const int r = lane + 32 * c;
+            if (r < dk) p.gk[(bh * T + j) * dk + r] = dka[i][c] * inv_sqrt;
+            if (r < dv) p.gv[(bh * T + j) * dv + r] = dva[i][c];
         }
     }
+}
+
+// Dynamic shared memory of the two window kernels.
+__host__ __forceinline__ size_t rows_smem(int dk, int dv) {
+    return (size_t)((kKT + kTileR) * (pad_stride(dk) + pad_stride(dv)) + (kThreads / 32) * kKT * kQR) *
+           sizeof(float);
+}
+__host__ __forceinline__ size_t keys_smem(int dk, int dv) {
+    return (size_t)((kKT + kTileR) * (pad_stride(dk) + pad_stride(dv)) +
+                    (kThreads / 32) * kKT * 2 * kQR + 2 * kKT) *
+           sizeof(float);
 }
 
 // ---------------------------------------------------------------------------
@@ -450,16 +571,30 @@ BwdLayout bwd_layout(const tc_prefill_desc &d) {
     return L;
 }
 
+// The two window kernels, CPL output columns per lane.
+template <typename Tin, int CPL>
+cudaError_t launch_window(const BwdParams &p, cudaStream_t s) {
+    const dim3 grid((unsigned)((p.T + kTileR - 1) / kTileR), (unsigned)(p.B * p.H));
+    const size_t s_rows = rows_smem(p.dk, p.dv), s_keys = keys_smem(p.dk, p.dv);
+    cudaError_t e = cudaFuncSetAttribute(bwd_rows_kernel<Tin, CPL>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s_rows);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(bwd_keys_kernel<Tin, CPL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)s_keys);
+    if (e != cudaSuccess) return e;
+    bwd_rows_kernel<Tin, CPL><<<grid, kThreads, s_rows, s>>>(p);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    bwd_keys_kernel<Tin, CPL><<<grid, kThreads, s_keys, s>>>(p);
+    return cudaGetLastError();
+}
+
 template <typename Tin>
 cudaError_t launch_t(const BwdParams &p, cudaStream_t s) {
     const int64_t BH = p.B * p.H;
     if (p.T > 0) {
-        const dim3 grid((unsigned)((p.T + kRows - 1) / kRows), (unsigned)BH);
-        bwd_rows_kernel<Tin><<<grid, kThreads, 0, s>>>(p);
-        cudaError_t e = cudaGetLastError();
-        if (e != cudaSuccess) return e;
-        bwd_keys_kernel<Tin><<<grid, kThreads, 0, s>>>(p);
-        e = cudaGetLastError();
+        const cudaError_t e = (p.dk <= 64 && p.dv <= 64) ? launch_window<Tin, 2>(p, s)
+                                                          : launch_window<Tin, kMaxD / 32>(p, s);
         if (e != cudaSuccess) return e;
     }
     const int nrs = (p.dk + kRows - 1) / kRows;
