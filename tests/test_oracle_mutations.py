@@ -7,7 +7,6 @@ oracle is mutated; nothing here touches a GPU.
 """
 import ctypes
 import os
-import shutil
 import subprocess
 
 import pytest
