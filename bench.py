@@ -619,7 +619,8 @@ def main():
     launches = head["launches_per_step"]
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+        "warmup": args.warmup, "ms_per_step": ms_step,
+        "ms_per_step_p50": statistics.median(head["per_step_ms"]), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": HEADLINE, "B": B, "H": H, "T": T, "d": dk, "W": x.W, "C": x.C,
                    "parallelism": f"replicas x{world} (heads independent, no collective)",
