@@ -192,7 +192,8 @@ TC_API tc_status tc_state_fold(int64_t B, int64_t H, int64_t dk, int64_t dv, int
  * A every 64 tokens.  q, k, v, dy: device, dtype of desc (dy has y's layout);
  * desc->flags must be 0 (C is not used).  Float32 SIMT kernels; four
  * launches.  Workspace: tc_backward_workspace_size(desc) bytes (about
- * B*H*(2T + 64*d_k*d_v*(1 + ceil(T/64))) floats).  Errors as tc_prefill. */
+ * B*H*(2T + d_k'*d_v*(64 + ceil(T/64))) floats, d_k' = d_k rounded up to a
+ * multiple of 8).  Errors as tc_prefill. */
 TC_API size_t tc_backward_workspace_size(const tc_prefill_desc *desc);
 TC_API tc_status tc_backward(const tc_prefill_desc *desc, const void *q, const void *k,
                              const void *v, const float *lambda, const float *eta, const float *g,
