@@ -406,31 +406,51 @@ def time_training_extras(tc, dev):
 
 
 # ---------------------------------------------------------------------------
+def _rows_per_call(B, H, threads):
+    """Batch rows per oracle call: the fewest (at least one item per thread)
+    whose B' * H items split evenly over the threads, else the most even."""
+    best, best_eff = 1, -1.0
+    for r in range(max(1, min(B, -(-threads // H))), B + 1):
+        items = r * H
+        eff = items / (-(-items // threads) * threads)
+        if eff > best_eff + 1e-9:
+            best, best_eff = r, eff
+        if eff > 0.999:
+            break
+    return best
+
+
+def _oracle_rows(x, b0, b1):
+    """The oracle over batch rows b0..b1-1 and every head: one call, so that
+    its OpenMP loop over (b, h) has (b1 - b0) * H items to share out."""
+    import oracle
+    oracle.prefill(x.q[b0:b1], x.k[b0:b1], x.v[b0:b1], x.lam, x.eta, x.g, x.W)
+
+
 def oracle_sample(name, budget_s=12.0):
     """Time the CPU oracle as it stands on a bounded sample of a prefill
-    workload: whole heads (from t = 0, as the layer requires) until about
-    budget_s seconds are spent.  Returns tokens/s and the sample used."""
+    workload: calls over whole batch rows (every head, from t = 0, as the
+    layer requires), cycling through the rows until about budget_s seconds
+    are spent.  Each call holds at least as many (b, h) items as the oracle
+    has threads.  Returns tokens/s, the threads used and the sample."""
     import oracle
     x = wl.prefill_config(name)
     B, H, T = x.q.shape[:3]
-    cores = oracle.threads()
-    n_heads, spent, tokens = 0, 0.0, 0
-    order = [(b, h) for b in range(B) for h in range(H)]
-    batch = max(1, cores)
-    while spent < budget_s and n_heads < len(order):
-        group = order[n_heads:n_heads + batch]
-        hs = sorted({h for _, h in group})
+    threads = oracle.threads(len(os.sched_getaffinity(0)))  # every core this process may use
+    rows = _rows_per_call(B, H, threads)
+    used = min(threads, rows * H)
+    b0, spent, heads = 0, 0.0, 0
+    while spent < budget_s:
+        b1 = min(B, b0 + rows)
         t0 = time.perf_counter()
-        for h in hs:
-            bs = [b for b, hh in group if hh == h]
-            oracle.prefill(x.q[bs, h:h + 1], x.k[bs, h:h + 1], x.v[bs, h:h + 1],
-                           x.lam[h:h + 1], x.eta[h:h + 1], x.g[h:h + 1], x.W)
+        _oracle_rows(x, b0, b1)
         spent += time.perf_counter() - t0
-        n_heads += len(group)
-        tokens += len(group) * T
-    return {"value": tokens / spent, "unit": UNIT, "cores": cores, "kind": "oracle",
-            "sample": f"{n_heads} of {B * H} heads x {T} tokens of {name} "
-                      f"(float64 token loop, OpenMP over heads), {spent:.1f} s"}
+        heads += (b1 - b0) * H
+        b0 = 0 if b1 == B else b1
+    return {"value": heads * T / spent, "unit": UNIT, "cores": used, "kind": "oracle",
+            "sample": f"{heads} heads x {T} tokens of {name} ({heads / (B * H):.2f} passes over "
+                      f"its {B * H} heads; float64 token loop, OpenMP over heads on {used} "
+                      f"threads), {spent:.1f} s"}
 
 
 def run_reference(args):
@@ -441,34 +461,30 @@ def run_reference(args):
     oracle.build()
     x = wl.prefill_config(HEADLINE)
     B, H, T = x.q.shape[:3]
-    cores = oracle.threads()
+    threads = oracle.threads(len(os.sched_getaffinity(0)))  # every core this process may use
     total_budget = 150.0
     per_step = total_budget / max(1, args.steps + args.warmup)
-    # calibrate: one head for the whole sequence
+    # calibrate on one call that occupies every thread: seconds per batch row
+    rows_cal = _rows_per_call(B, H, threads)
     t0 = time.perf_counter()
-    oracle.prefill(x.q[:1, :1], x.k[:1, :1], x.v[:1, :1], x.lam[:1], x.eta[:1], x.g[:1], x.W,
-                   nthreads=1)
-    one = time.perf_counter() - t0
-    heads = max(1, min(B * H, int(per_step / one * cores)))
-    order = [(b, h) for b in range(B) for h in range(H)][:heads]
+    _oracle_rows(x, 0, rows_cal)
+    per_row = (time.perf_counter() - t0) / rows_cal
+    rows = max(1, min(B, int(per_step / per_row)))  # batch rows (every head) per step
+    cores = min(threads, rows * H)
 
     def step():
-        by_h = {}
-        for b, h in order:
-            by_h.setdefault(h, []).append(b)
-        for h, bs in by_h.items():
-            oracle.prefill(x.q[bs, h:h + 1], x.k[bs, h:h + 1], x.v[bs, h:h + 1],
-                           x.lam[h:h + 1], x.eta[h:h + 1], x.g[h:h + 1], x.W)
+        _oracle_rows(x, 0, rows)
     for _ in range(args.warmup):
         step()
     t0 = time.perf_counter()
     for _ in range(args.steps):
         step()
     el = time.perf_counter() - t0
+    heads = rows * H
     tokens = heads * T * args.steps
     value = tokens / el
     sample = (f"{heads} of {B * H} heads x {T} tokens of {HEADLINE} per step "
-              f"(float64 token loop, OpenMP over heads)")
+              f"(float64 token loop, OpenMP over heads on {cores} threads)")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": el / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
