@@ -51,3 +51,22 @@ def test_lm_workload_counts():
     # 150 computed tiles and 28 leading tiles per head
     assert e1 == 96 * 150 * 2 * (2 * 128 * 128 * 64)
     assert e2 == 96 * 28 * (2 * (2 * 128 * 128 * 64) + 128 * 64 * 64 * 2)
+
+
+def test_oracle_calls_split_evenly_over_threads():
+    # rows per call: at least one (b, h) item per thread, and whole waves where possible
+    for B, H, threads in [(8, 12, 1), (8, 12, 8), (8, 12, 16), (8, 12, 32), (1, 16, 64), (8, 4, 6)]:
+        r = bench._rows_per_call(B, H, threads)
+        assert 1 <= r <= B
+        items = r * H
+        assert items >= min(threads, B * H)
+        if any((k * H) % threads == 0 for k in range(-(-threads // H), B + 1)):
+            assert items % threads == 0, (B, H, threads, r)
+
+
+def test_cpu_baseline_reports_threads_used():
+    out = bench.oracle_sample("lm_prefill_bf16", budget_s=0.05)
+    cores = len(os.sched_getaffinity(0))
+    assert 1 <= out["cores"] <= cores
+    assert out["kind"] == "oracle" and out["value"] > 0
+    assert "heads x 4096 tokens" in out["sample"]
