@@ -44,9 +44,9 @@ HEADLINE = "lm_prefill_bf16"
 # DRAM bytes (read + write) per launch from one ncu capture of the current
 # kernels; they must be re-measured (or set to None) whenever a kernel changes.
 #   prefill_main_kernel, LM workload: profiles/prefill_main_kernel_lm_prefill_bf16.md
-#   decode_kernel, 256 x 32 heads (captured at 32 x 32, scaled by heads):
-#     profiles/decode_kernel_b32_w2048_d128.md
-NCU_TRAFFIC_BYTES = {"prefill_main_kernel": 190.8e6, "decode_kernel": 9.28e9}
+#   decode_kernel: None, the kernel gained the ragged clocks and the delta-rule
+#     branch after its capture (profiles/decode_kernel_b32_w2048_d128.md)
+NCU_TRAFFIC_BYTES = {"prefill_main_kernel": 190.8e6, "decode_kernel": None}
 METRIC = "prefill tokens/s & decode tok/s per B200; % of TC/HBM roofline"
 UNIT = "tokens/s"
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
