@@ -25,7 +25,7 @@
  *     A <- lambda*A + eta*(kbar (x) vbar) and the parallel weighted-sum chunk
  *     scan that equals per-token writes.
  *
- * Readings where the pages leave a step open (each is listed in the design doc):
+ * Readings where the pages leave a step open:
  *   - the write (step 3) precedes the read (step 5) inside a step, so the query
  *     at step t sees token t-W through A and tokens t-W+1..t through the window;
  *   - the window includes the current token (inserted at step 4 before the
