@@ -21,7 +21,7 @@ Compute per rank: one state-only chunk scan and one prefill from the state,
 both in libtc (tc_prefill_from_state), plus tc_state_fold.  No remote memory
 is read by a kernel; the collectives carry all data between GPUs.
 
-The driver works in phases, so the single-process tests can run the same
+The sharded prefill works in phases, so the single-process tests can run the same
 code for several ranks in turn:
     tail      -> all-gather -> piece_state -> all-gather -> finish
 """
