@@ -159,6 +159,32 @@ def _contig(*ts):
             raise ValueError("tensors must be contiguous")
 
 
+# The C-ABI sees only addresses, so a tensor of the wrong size or element type
+# would have a kernel read or write past its end: shapes and dtypes are
+# checked here, before any call.
+def _expect(t: Optional[torch.Tensor], name: str, shape, dtype):
+    if t is None:
+        return
+    if t.dtype != dtype:
+        raise TypeError(f"{name} has dtype {t.dtype}; expected {dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}; expected {tuple(shape)}")
+
+
+def _expect_layer(B, H, T, dk, dv, dt, q, k, v, lam, eta, g, y=None, A_final=None):
+    """q, k [B,H,T,dk], v (and y) [B,H,T,dv] in dt; lam, eta, g [H] float32;
+    A_final [B,H,dk,dv] float32 (None entries are not checked)."""
+    _expect(q, "q", (B, H, T, dk), dt)
+    _expect(k, "k", (B, H, T, dk), dt)
+    _expect(v, "v", (B, H, T, dv), dt)
+    for name, t in (("lam", lam), ("eta", eta), ("g", g)):
+        if t is None:
+            raise ValueError(f"{name} is required")
+        _expect(t, name, (H,), torch.float32)
+    _expect(y, "y", (B, H, T, dv), dt)
+    _expect(A_final, "A_final", (B, H, dk, dv), torch.float32)
+
+
 def make_prefill_desc(B, H, T, dk, dv, W, C, dtype: int, l1_only: bool = False,
                       state_only: bool = False, delta_rule: bool = False,
                       chunk_mean: bool = False) -> PrefillDesc:
@@ -193,6 +219,7 @@ def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, lam: torch.Tensor
     desc = _desc_of(q, v, W, C, l1_only, delta_rule)
     B, H, T, dk = q.shape
     dv = v.shape[-1]
+    _expect_layer(B, H, T, dk, dv, q.dtype, q, k, v, lam, eta, g, y, A_final)
     if y is None:
         y = torch.empty((B, H, T, dv), dtype=q.dtype, device=q.device)
     if A_final is None and not l1_only:
@@ -227,6 +254,11 @@ def prefill_from_state(q: Optional[torch.Tensor], k: torch.Tensor, v: torch.Tens
     dv = v.shape[-1]
     desc = make_prefill_desc(B, H, T, dk, dv, W, C, _dtype_code(k), l1_only, state_only,
                              delta_rule, chunk_mean)
+    _expect_layer(B, H, T, dk, dv, k.dtype, q, k, v, lam, eta, g, y, A_final)
+    n_halo = min(int(t0), int(W))
+    _expect(halo_k, "halo_k", (B, H, n_halo, dk), k.dtype)
+    _expect(halo_v, "halo_v", (B, H, n_halo, dv), k.dtype)
+    _expect(A_init, "A_init", (B, H, dk, dv), torch.float32)
     if y is None and not state_only:
         y = torch.empty((B, H, T, dv), dtype=k.dtype, device=k.device)
     if A_final is None and not l1_only:
@@ -257,6 +289,9 @@ def state_fold(dA: torch.Tensor, E: torch.Tensor, lam: torch.Tensor,
     _contig(dA, E, lam, A_out)
     if dA.dtype != torch.float32 or E.dtype != torch.int64:
         raise TypeError("dA must be float32 and E int64")
+    _expect(E, "E", (n,), torch.int64)
+    _expect(lam, "lam", (H,), torch.float32)
+    _expect(A_out, "A_out", (B, H, dk, dv), torch.float32)
     st = _lib.tc_state_fold(B, H, dk, dv, n, _ptr(dA) if n else None, _ptr(E) if n else None,
                             _ptr(lam), _ptr(A_out), _stream(stream))
     _check(st, "tc_state_fold")
@@ -272,6 +307,8 @@ def backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, lam: torch.Tenso
     B, H, T, dk = q.shape
     dv = v.shape[-1]
     desc = make_prefill_desc(B, H, T, dk, dv, W, 1, _dtype_code(q))
+    _expect_layer(B, H, T, dk, dv, q.dtype, q, k, v, lam, eta, g)
+    _expect(dy, "dy", (B, H, T, dv), q.dtype)
     f = dict(dtype=torch.float32, device=q.device)
     dq, dkk, dvv = torch.empty(B, H, T, dk, **f), torch.empty(B, H, T, dk, **f), torch.empty(B, H, T, dv, **f)
     dl, de, dg_ = torch.empty(H, **f), torch.empty(H, **f), torch.empty(H, **f)
@@ -308,6 +345,7 @@ def prefill_no_alloc(q, k, v, lam, eta, g, W, C, *, l1_only=False, y=None, A_fin
     desc = _desc_of(q, v, W, C, l1_only)
     B, H, T, dk = q.shape
     dv = v.shape[-1]
+    _expect_layer(B, H, T, dk, dv, q.dtype, q, k, v, lam, eta, g, y, A_final)
     if y is None:
         y = torch.empty((B, H, T, dv), dtype=q.dtype, device=q.device)
     if A_final is None and not l1_only:
@@ -333,6 +371,10 @@ def prefill_host(q, k, v, lam, eta, g, W, C, y, A_final=None, *, workspace, l1_o
     prefill_host_workspace_size bytes.  Enqueued on stream; synchronize
     before reading y."""
     desc = _desc_of(q, v, W, C, l1_only)
+    B, H, T, dk = q.shape
+    _expect_layer(B, H, T, dk, v.shape[-1], q.dtype, q, k, v, lam, eta, g, y, A_final)
+    if y is None:
+        raise ValueError("y (a host tensor) is required")
     _contig(q, k, v, lam, eta, g, y, A_final, workspace)
     st = _lib.tc_prefill_host(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(lam),
                               _ptr(eta), _ptr(g), _ptr(y), _ptr(A_final), _ptr(workspace),
@@ -359,6 +401,11 @@ class DecodeState:
     def c_struct(self) -> DecodeStateC:
         B, H, W, dk = self.ring_k.shape
         dv = self.ring_v.shape[-1]
+        _dtype_code(self.ring_k)
+        _expect(self.ring_v, "ring_v", (B, H, W, dv), self.ring_k.dtype)
+        _expect(self.A, "A", (B, H, dk, dv), torch.float32)
+        for name, t in (("lam", self.lam), ("eta", self.eta), ("g", self.g)):
+            _expect(t, name, (H,), torch.float32)
         _contig(self.ring_k, self.ring_v, self.A, self.lam, self.eta, self.g)
         return DecodeStateC(B, H, dk, dv, W, int(self.t), _dtype_code(self.ring_k),
                             self.ring_k.data_ptr(), self.ring_v.data_ptr(), self.A.data_ptr(),
@@ -373,11 +420,23 @@ class DecodeState:
                            lam, eta, g, 0)
 
 
+def _expect_step(state: DecodeState, q, k, v, y):
+    """q, k [B,H,dk], v and y [B,H,dv] in the ring's dtype."""
+    B, H, _, dk = state.ring_k.shape
+    dv = state.ring_v.shape[-1]
+    dt = state.ring_k.dtype
+    _expect(q, "q", (B, H, dk), dt)
+    _expect(k, "k", (B, H, dk), dt)
+    _expect(v, "v", (B, H, dv), dt)
+    _expect(y, "y", (B, H, dv), dt)
+
+
 def decode_step(state: DecodeState, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
                 y: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
     """tc_decode_step: q, k [B,H,dk], v [B,H,dv] device tensors in the ring's
     dtype.  Updates the ring and A in place, advances state.t, returns y."""
     cs = state.c_struct()
+    _expect_step(state, q, k, v, y)
     if y is None:
         y = torch.empty(v.shape, dtype=v.dtype, device=v.device)
     _contig(q, k, v, y)
@@ -396,11 +455,11 @@ def decode_step_ragged(state: DecodeState, t_rows: torch.Tensor, q: torch.Tensor
     library advances the non-negative clocks on the device; state.t is not
     used."""
     cs = state.c_struct()
+    _expect_step(state, q, k, v, y)
+    _expect(t_rows, "t_rows", (state.ring_k.shape[0],), torch.int64)
     if y is None:
         y = torch.empty(v.shape, dtype=v.dtype, device=v.device)
     _contig(q, k, v, y, t_rows)
-    if t_rows.dtype != torch.int64:
-        raise TypeError("t_rows must be int64")
     st = _lib.tc_decode_step_ragged(ctypes.byref(cs), _ptr(t_rows), _ptr(q), _ptr(k), _ptr(v),
                                     _ptr(y), _stream(stream))
     _check(st, "tc_decode_step_ragged")
@@ -419,6 +478,7 @@ def decode_step_host(state: DecodeState, q, k, v, y, *, workspace, stream=None):
     """tc_decode_step_host: q, k, v, y are HOST tensors (pinned); the state
     stays on the device.  Enqueued on stream; synchronize before reading y."""
     cs = state.c_struct()
+    _expect_step(state, q, k, v, y)
     _contig(q, k, v, y, workspace)
     st = _lib.tc_decode_step_host(ctypes.byref(cs), _ptr(q), _ptr(k), _ptr(v), _ptr(y),
                                   _ptr(workspace), workspace.numel(), _stream(stream))
