@@ -237,7 +237,10 @@ TC_API tc_status tc_prefill_host(const tc_prefill_desc *desc, const void *q, con
  * Returns TC_ERR_WORKSPACE, enqueuing nothing, when desc would need more
  * scratch than that (tc_prefill_workspace_size(desc) tells how much).
  * The first call on each device looks up the array's device address with
- * that device current; make that first call before any stream capture.
+ * that device current; make that first call before any stream capture.  The
+ * address is cached until a call fails with TC_ERR_CUDA; after a
+ * cudaDeviceReset the array may sit elsewhere, so treat the next call as a
+ * first call again (outside any capture).
  * All calls share the array and leave their data in it; no call depends on
  * what an earlier one left, but calls whose kernels may overlap on the GPU
  * (unordered streams) race on it and must not be issued that way.
@@ -315,6 +318,17 @@ TC_API size_t tc_decode_step_host_workspace_size(const tc_decode_state *state);
 TC_API tc_status tc_decode_step_host(tc_decode_state *state, const void *q_t, const void *k_t,
                               const void *v_t, void *y_t, void *workspace,
                               size_t workspace_bytes, tc_stream_t stream);
+
+/* Limit, in nanoseconds, of every bounded wait inside the tensor-core prefill
+ * kernels (an mbarrier wait for a copy, a tensor-core product or another warp).
+ * A wait that runs out makes the kernel drain its copies and products, record
+ * TC_ERR_DEVICE_TIMEOUT in the device status word and return, so a stalled
+ * pipeline ends with an error instead of a hung GPU.  0 restores the default
+ * of 2 s, far beyond any legitimate wait.  Process-wide; it applies to calls
+ * made after it and is meant for tests of that failure path (a limit of a
+ * microsecond makes the first wait of a real call run out).  Not thread-safe
+ * against concurrent calls. */
+TC_API void tc_set_wait_limit_ns(uint64_t ns);
 
 /* Synchronizes stream, then returns and clears the device status word of the
  * current device: TC_OK, TC_ERR_DEVICE_BOUNDS or TC_ERR_DEVICE_TIMEOUT. */

@@ -49,7 +49,8 @@ EXPORTED = ("tc_prefill_workspace_size", "tc_prefill", "tc_prefill_launch_count"
             "tc_prefill_host", "tc_decode_step", "tc_decode_step_host_workspace_size",
             "tc_decode_step_host", "tc_get_device_status", "tc_status_string", "tc_version",
             "tc_prefill_no_alloc", "tc_prefill_from_state", "tc_prefill_from_state_workspace_size",
-            "tc_state_fold", "tc_decode_step_ragged", "tc_backward", "tc_backward_workspace_size")
+            "tc_state_fold", "tc_decode_step_ragged", "tc_backward", "tc_backward_workspace_size",
+            "tc_set_wait_limit_ns")
 
 
 class PrefillDesc(ctypes.Structure):
@@ -106,6 +107,8 @@ _lib.tc_status_string.argtypes = [_int]
 _lib.tc_status_string.restype = ctypes.c_char_p
 _lib.tc_version.argtypes = []
 _lib.tc_version.restype = ctypes.c_char_p
+_lib.tc_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
+_lib.tc_set_wait_limit_ns.restype = None
 
 SIZE_ERROR = ctypes.c_size_t(-1).value
 
@@ -157,6 +160,22 @@ def _contig(*ts):
     for t in ts:
         if t is not None and not t.is_contiguous():
             raise ValueError("tensors must be contiguous")
+
+
+def _on_device(current: int, *ts):
+    """Every CUDA tensor must live on the current device `current`: the
+    kernels run there, and another GPU's buffer would be read over the peer
+    link (or fault without peer access).  The library refuses such pointers
+    too; checking here gives a clear Python error first."""
+    for t in ts:
+        if t is not None and t.device.type == "cuda" and t.device.index != current:
+            raise ValueError(f"tensor on {t.device} but the current CUDA device is cuda:{current}; "
+                             "call under torch.cuda.device(...) of the tensors' device")
+
+
+def _dev_check(*ts):
+    if any(t is not None and t.device.type == "cuda" for t in ts):
+        _on_device(torch.cuda.current_device(), *ts)
 
 
 # The C-ABI sees only addresses, so a tensor of the wrong size or element type
@@ -228,6 +247,7 @@ def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, lam: torch.Tensor
     if workspace is None and need > 0:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     _contig(q, k, v, lam, eta, g, y, A_final, workspace)
+    _dev_check(q, k, v, lam, eta, g, y, A_final, workspace)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     st = _lib.tc_prefill(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(lam), _ptr(eta),
                          _ptr(g), _ptr(y), _ptr(A_final), _ptr(workspace), ws_bytes,
@@ -269,6 +289,7 @@ def prefill_from_state(q: Optional[torch.Tensor], k: torch.Tensor, v: torch.Tens
     if workspace is None and need > 0:
         workspace = torch.empty(need, dtype=torch.uint8, device=k.device)
     _contig(q, k, v, lam, eta, g, y, A_final, workspace, halo_k, halo_v, A_init)
+    _dev_check(q, k, v, lam, eta, g, y, A_final, workspace, halo_k, halo_v, A_init)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     st = _lib.tc_prefill_from_state(ctypes.byref(desc), int(t0), _ptr(halo_k), _ptr(halo_v),
                                     _ptr(A_init), _ptr(q), _ptr(k), _ptr(v), _ptr(lam),
@@ -287,6 +308,7 @@ def state_fold(dA: torch.Tensor, E: torch.Tensor, lam: torch.Tensor,
     if A_out is None:
         A_out = torch.empty((B, H, dk, dv), dtype=torch.float32, device=lam.device)
     _contig(dA, E, lam, A_out)
+    _dev_check(dA, E, lam, A_out)
     if dA.dtype != torch.float32 or E.dtype != torch.int64:
         raise TypeError("dA must be float32 and E int64")
     _expect(E, "E", (n,), torch.int64)
@@ -318,6 +340,7 @@ def backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, lam: torch.Tenso
     if workspace is None and need > 0:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     _contig(q, k, v, lam, eta, g, dy, workspace)
+    _dev_check(q, k, v, lam, eta, g, dy, workspace)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     st = _lib.tc_backward(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(lam), _ptr(eta),
                           _ptr(g), _ptr(dy), _ptr(dq), _ptr(dkk), _ptr(dvv), _ptr(dl), _ptr(de),
@@ -351,6 +374,7 @@ def prefill_no_alloc(q, k, v, lam, eta, g, W, C, *, l1_only=False, y=None, A_fin
     if A_final is None and not l1_only:
         A_final = torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device)
     _contig(q, k, v, lam, eta, g, y, A_final)
+    _dev_check(q, k, v, lam, eta, g, y, A_final)
     st = _lib.tc_prefill_no_alloc(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(lam),
                                   _ptr(eta), _ptr(g), _ptr(y), _ptr(A_final), _stream(stream))
     _check(st, "tc_prefill_no_alloc")
@@ -376,9 +400,10 @@ def prefill_host(q, k, v, lam, eta, g, W, C, y, A_final=None, *, workspace, l1_o
     if y is None:
         raise ValueError("y (a host tensor) is required")
     _contig(q, k, v, lam, eta, g, y, A_final, workspace)
+    _dev_check(workspace)
     st = _lib.tc_prefill_host(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(lam),
                               _ptr(eta), _ptr(g), _ptr(y), _ptr(A_final), _ptr(workspace),
-                              workspace.numel(), _stream(stream))
+                              workspace.numel() * workspace.element_size(), _stream(stream))
     _check(st, "tc_prefill_host")
     return y, A_final
 
@@ -407,6 +432,7 @@ class DecodeState:
         for name, t in (("lam", self.lam), ("eta", self.eta), ("g", self.g)):
             _expect(t, name, (H,), torch.float32)
         _contig(self.ring_k, self.ring_v, self.A, self.lam, self.eta, self.g)
+        _dev_check(self.ring_k, self.ring_v, self.A, self.lam, self.eta, self.g)
         return DecodeStateC(B, H, dk, dv, W, int(self.t), _dtype_code(self.ring_k),
                             self.ring_k.data_ptr(), self.ring_v.data_ptr(), self.A.data_ptr(),
                             self.lam.data_ptr(), self.eta.data_ptr(), self.g.data_ptr(),
@@ -440,6 +466,7 @@ def decode_step(state: DecodeState, q: torch.Tensor, k: torch.Tensor, v: torch.T
     if y is None:
         y = torch.empty(v.shape, dtype=v.dtype, device=v.device)
     _contig(q, k, v, y)
+    _dev_check(q, k, v, y)
     st = _lib.tc_decode_step(ctypes.byref(cs), _ptr(q), _ptr(k), _ptr(v), _ptr(y),
                              _stream(stream))
     _check(st, "tc_decode_step")
@@ -460,6 +487,7 @@ def decode_step_ragged(state: DecodeState, t_rows: torch.Tensor, q: torch.Tensor
     if y is None:
         y = torch.empty(v.shape, dtype=v.dtype, device=v.device)
     _contig(q, k, v, y, t_rows)
+    _dev_check(q, k, v, y, t_rows)
     st = _lib.tc_decode_step_ragged(ctypes.byref(cs), _ptr(t_rows), _ptr(q), _ptr(k), _ptr(v),
                                     _ptr(y), _stream(stream))
     _check(st, "tc_decode_step_ragged")
@@ -480,11 +508,20 @@ def decode_step_host(state: DecodeState, q, k, v, y, *, workspace, stream=None):
     cs = state.c_struct()
     _expect_step(state, q, k, v, y)
     _contig(q, k, v, y, workspace)
+    _dev_check(workspace)
     st = _lib.tc_decode_step_host(ctypes.byref(cs), _ptr(q), _ptr(k), _ptr(v), _ptr(y),
-                                  _ptr(workspace), workspace.numel(), _stream(stream))
+                                  _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                  _stream(stream))
     _check(st, "tc_decode_step_host")
     state.t = int(cs.t)
     return y
+
+
+def set_wait_limit_ns(ns: int) -> None:
+    """tc_set_wait_limit_ns: limit of the tensor-core kernels' bounded waits
+    (0 restores the 2 s default).  Process-wide; meant for tests of the
+    timeout path."""
+    _lib.tc_set_wait_limit_ns(int(ns))
 
 
 def device_status(stream=None) -> int:

@@ -11,9 +11,13 @@ plain associative memory), once by the exact scan and once by the shortcut
 reads the memory, m_i = k_i A.  Reported per N:
   recall_cos   mean cosine between m_i and v_i
   recall_top1  fraction of keys whose read is closest (cosine) to its own value
-The writes run in libtc (tc_prefill_from_state, state only: the N pairs are
-the evictions of an N + 1 token sequence with W = 1); the read-out and the
-scores are analysis and use PyTorch.
+Both the writes and the reads run in libtc.  The writes are
+tc_prefill_from_state, state only: the N pairs are the evictions of an N + 1
+token sequence with W = 1.  The reads are the layer's own L2 read: a
+continuation (t0 = 1, W = 1) from A_init = A whose window holds only zero
+values and whose writes add nothing (eta = 0), with the keys as queries and
+sigmoid(g) = 1, so that y_i = k_i A.  Only the scores (cosines, argmax) are
+computed here, with PyTorch, as analysis.
 """
 from __future__ import annotations
 
@@ -35,8 +39,24 @@ def _state(k: torch.Tensor, v: torch.Tensor, C: int, chunk_mean: bool) -> torch.
     return A[0, 0]
 
 
+def _read(k: torch.Tensor, A: torch.Tensor) -> torch.Tensor:
+    """m_i = k_i A through the layer: every window value is zero (y_local =
+    0), eta = 0 keeps A fixed over the call, and g = 40 makes sigmoid(g) = 1
+    in float32, so the output is the memory read alone."""
+    from . import prefill_from_state
+    N, d = k.shape
+    dev = k.device
+    zeros = torch.zeros(1, 1, N, d, device=dev)
+    halo = torch.zeros(1, 1, 1, d, device=dev)
+    y, _ = prefill_from_state(k.contiguous().view(1, 1, N, d), zeros, zeros,
+                              torch.ones(1, device=dev), torch.zeros(1, device=dev),
+                              torch.full((1,), 40.0, device=dev), 1, 1, 1, halo, halo,
+                              A.contiguous().view(1, 1, d, d))
+    return y[0, 0]
+
+
 def _scores(k, v, A) -> Dict[str, float]:
-    m = k @ A
+    m = _read(k, A)
     mn = torch.nn.functional.normalize(m, dim=-1)
     vn = torch.nn.functional.normalize(v, dim=-1)
     cos = (mn * vn).sum(-1)

@@ -105,6 +105,7 @@ struct MainParams {
     const float *A_init;  // [BH][64][64] state before the first eviction, or null
     int T, W, H, BH, nT, n_s, n_parts, l1_only, q_off;
     int *status;
+    unsigned long long wait_ns;  // limit of every bounded wait
 };
 
 struct SumParams {
@@ -112,6 +113,7 @@ struct SumParams {
     const float *lam, *eta;
     int T, W, H, BH, nT, n_s, n_parts, q_off;
     int *status;
+    unsigned long long wait_ns;  // limit of every bounded wait
 };
 
 // Query tiles [i0, i1) of span j: the tiles i_begin .. nT-1 cut into n_s parts.
@@ -144,9 +146,9 @@ __device__ __forceinline__ void named_bar(int id, int n) {
 // bar.sync it gives up with the bounded wait, so an aborting thread cannot
 // leave the rest of its group blocked.
 __device__ __forceinline__ bool group_sync(uint64_t *bar, uint32_t &phase, volatile int *abort,
-                                           int *status) {
+                                           int *status, uint64_t limit = kWaitTimeoutNs) {
     mbar_arrive(bar);
-    const bool ok = __all_sync(0xffffffffu, mbar_wait(bar, phase & 1, abort, status));
+    const bool ok = __all_sync(0xffffffffu, mbar_wait(bar, phase & 1, abort, status, limit));
     ++phase;
     return ok;
 }
@@ -154,8 +156,8 @@ __device__ __forceinline__ bool group_sync(uint64_t *bar, uint32_t &phase, volat
 // mbar_wait with one answer for the whole warp, so that warps which go on to
 // warp-collective tcgen05.ld / st never diverge on a failed wait.
 __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volatile int *abort,
-                                          int *status) {
-    return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort, status));
+                                          int *status, uint64_t limit = kWaitTimeoutNs) {
+    return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort, status, limit));
 }
 
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
@@ -423,8 +425,10 @@ __global__ void __launch_bounds__(192, 2)
                         const __grid_constant__ CUtensorMap tkh,
                         const __grid_constant__ CUtensorMap tvh, SumParams p) {
     extern __shared__ uint8_t smem_raw[];
-    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                              ~uintptr_t(1023));
+    // 1024-aligned base by pointer arithmetic on the shared array itself, so
+    // that the compiler keeps the shared address space (ld/st.shared) for
+    // every access derived from it
+    uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + SOFF_BAR);
     uint64_t *kv_full = bars, *kv_empty = bars + NS_SUM;
     uint64_t *kt_full = bars + 2 * NS_SUM, *kt_empty = kt_full + 1, *done = kt_empty + 1;
@@ -479,7 +483,7 @@ __global__ void __launch_bounds__(192, 2)
             int issued = 0;
             for (int e = 0; e < ne; ++e) {
                 const int s = e % NS_SUM;
-                if (!mbar_wait(&kv_empty[s], ((e / NS_SUM) & 1) ^ 1, abort, p.status)) break;
+                if (!mbar_wait(&kv_empty[s], ((e / NS_SUM) & 1) ^ 1, abort, p.status, p.wait_ns)) break;
                 const int n0 = (ev_first + e) * BM - p.W;
                 uint8_t *dst = sm + SOFF_KV + s * 2 * TILE_B;
                 mbar_expect_tx(&kv_full[s], 2 * TILE_B);
@@ -496,7 +500,7 @@ __global__ void __launch_bounds__(192, 2)
             const uint32_t id_ds = idesc_bf16(128, 64, true, true);
             for (int e = 0; e < ne; ++e) {
                 const int s = e % NS_SUM;
-                if (!mbar_wait(kt_full, e & 1, abort, p.status)) break;
+                if (!mbar_wait(kt_full, e & 1, abort, p.status, p.wait_ns)) break;
                 tc_fence_after();
                 const uint32_t kt = smem_u32(sm + SOFF_KT);
                 const uint32_t vv = smem_u32(sm + SOFF_KV + s * 2 * TILE_B + TILE_B);
@@ -518,8 +522,8 @@ __global__ void __launch_bounds__(192, 2)
         const double l2l = log2(lam);
         for (int e = 0; e < ne; ++e) {
             const int s = e % NS_SUM;
-            if (!mbar_wait(&kv_full[s], (e / NS_SUM) & 1, abort, p.status)) break;
-            if (!mbar_wait(kt_empty, (e & 1) ^ 1, abort, p.status)) break;
+            if (!mbar_wait(&kv_full[s], (e / NS_SUM) & 1, abort, p.status, p.wait_ns)) break;
+            if (!mbar_wait(kt_empty, (e & 1) ^ 1, abort, p.status, p.wait_ns)) break;
             const int n0 = (ev_first + e) * BM - p.W;
             const int ev = n0 + u;
             const float w = ev < e_end ? eta * (float)exp2((double)(e_end - 1 - ev) * l2l) : 0.f;
@@ -529,7 +533,7 @@ __global__ void __launch_bounds__(192, 2)
             mbar_arrive(kt_full);
         }
         // read the accumulated [hi; lo] rows and add the halves
-        const bool ok = warp_wait(done, 0, abort, p.status);
+        const bool ok = warp_wait(done, 0, abort, p.status, p.wait_ns);
         tc_fence_after();
         const int lane_base = 32 * (warp & 3);
         const int L = lane_base + (tid & 31);
@@ -569,8 +573,10 @@ __global__ void __launch_bounds__(kMainThreads, 1)
                         const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tkh,
                         const __grid_constant__ CUtensorMap tvh, MainParams p) {
     extern __shared__ uint8_t smem_raw[];
-    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                              ~uintptr_t(1023));
+    // 1024-aligned base by pointer arithmetic on the shared array itself, so
+    // that the compiler keeps the shared address space (ld/st.shared) for
+    // every access derived from it
+    uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + OFF_BAR);
     uint64_t *q_full = bars, *q_empty = bars + 2;
     uint64_t *kv_full = bars + 4, *kv_empty = kv_full + NS;
@@ -641,12 +647,12 @@ __global__ void __launch_bounds__(kMainThreads, 1)
                 for (int i = i0; i < i1 && ok; ++i, ++tile) {
                     const TileInfo ti = tile_info(i, p.W, l1_only);
                     const int qb = tile & 1;
-                    if (!(ok = mbar_wait(&q_empty[qb], ((tile >> 1) & 1) ^ 1, abort, p.status))) break;
+                    if (!(ok = mbar_wait(&q_empty[qb], ((tile >> 1) & 1) ^ 1, abort, p.status, p.wait_ns))) break;
                     mbar_expect_tx(&q_full[qb], TILE_B);
                     tma_load_3d(sm + OFF_Q + qb * TILE_B, &tq, &q_full[qb], 0, ti.t0 - p.q_off, bh);
                     for (int j = 0; j < ti.nk; ++j, ++kc) {
                         const int s = kc % NS;
-                        if (!(ok = mbar_wait(&kv_empty[s], ((kc / NS) & 1) ^ 1, abort, p.status))) break;
+                        if (!(ok = mbar_wait(&kv_empty[s], ((kc / NS) & 1) ^ 1, abort, p.status, p.wait_ns))) break;
                         uint8_t *dst = sm + OFF_KV + s * 2 * TILE_B;
                         mbar_expect_tx(&kv_full[s], 2 * TILE_B);
                         load_kv_tile(dst, &tk, &tv, &tkh, &tvh, &kv_full[s], ti.kt0 + j, p.q_off, bh);
@@ -692,33 +698,34 @@ __global__ void __launch_bounds__(kMainThreads, 1)
             } pend = {false, false, false, false, 0, 0};
             auto pv_step = [&](const Pending &pv) -> bool {
                 const int sb = pv.g & 1, s = pv.g % NS;
-                if (!warp_wait(&p_full[sb], (pv.g >> 1) & 1, abort, p.status)) return false;
-                if (pv.first && !warp_wait(o_empty, (pv.tile & 1) ^ 1, abort, p.status)) return false;
+                if (!warp_wait(&p_full[sb], (pv.g >> 1) & 1, abort, p.status, p.wait_ns)) return false;
+                if (pv.first && !warp_wait(o_empty, (pv.tile & 1) ^ 1, abort, p.status, p.wait_ns)) return false;
                 tc_fence_after();
                 const uint32_t v_addr = kv_base + s * 2 * TILE_B + TILE_B;
                 const uint32_t s_col = tb + TM_S + sb * 128;
-#pragma unroll 1
-                for (int k = 0; k < 8; ++k)
-                    mma_ts_w(tb + TM_O, s_col + 8 * k, sdesc_sw128(v_addr + 2048 * k, TILE_B, 1024),
-                           id_pv, (!pv.first || k > 0));
+                // Issue loops are unrolled with the descriptors stepped by
+                // constants (+2048 bytes of a K/V tile = +128 in the address
+                // field): a rolled loop that rebuilds each descriptor takes more
+                // than twice as long to issue the same MMAs.
+                const uint64_t vd = sdesc_sw128(v_addr, TILE_B, 1024);
+                mma_ts_w(tb + TM_O, s_col, vd, id_pv, !pv.first);
+#pragma unroll
+                for (int k = 1; k < 8; ++k) mma_ts_w(tb + TM_O, s_col + 8 * k, vd + 128 * k, id_pv, 1);
                 if (pv.first && pv.l2) {
                     const uint32_t q_addr = q_base + (pv.tile & 1) * TILE_B;
-#pragma unroll 1
+#pragma unroll
                     for (int k = 0; k < 8; ++k)
-                        mma_ts_w(tb + TM_MI, s_col + 64 + 8 * k,
-                               sdesc_sw128(v_addr + 2048 * k, TILE_B, 1024), id_pv, k > 0);
-                    if (!warp_wait(sst_full, lc & 1, abort, p.status)) return false;
+                        mma_ts_w(tb + TM_MI, s_col + 64 + 8 * k, vd + 128 * k, id_pv, k > 0);
+                    if (!warp_wait(sst_full, lc & 1, abort, p.status, p.wait_ns)) return false;
                     tc_fence_after();
-#pragma unroll 1
-                    for (int k = 0; k < 4; ++k)
-                        mma_ss_w(tb + TM_MX, sdesc_sw128(q_addr + 32 * k, 16, 1024),
-                               sdesc_sw128(sb_addr + 2048 * k, 8192, 1024), id_qs, k > 0);
-                    if (!warp_wait(kt_full, lc & 1, abort, p.status)) return false;
+                    const uint64_t qd = sdesc_sw128(q_addr, 16, 1024), sd = sdesc_sw128(sb_addr, 8192, 1024);
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) mma_ss_w(tb + TM_MX, qd + 2 * k, sd + 128 * k, id_qs, k > 0);
+                    if (!warp_wait(kt_full, lc & 1, abort, p.status, p.wait_ns)) return false;
                     tc_fence_after();
-#pragma unroll 1
-                    for (int k = 0; k < 8; ++k)
-                        mma_ss_w(tb + TM_DS, sdesc_sw128(kt_addr + 2048 * k, TILE_B, 1024),
-                               sdesc_sw128(v_addr + 2048 * k, TILE_B, 1024), id_ds, k > 0);
+                    const uint64_t ktd = sdesc_sw128(kt_addr, TILE_B, 1024);
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) mma_ss_w(tb + TM_DS, ktd + 128 * k, vd + 128 * k, id_ds, k > 0);
                     mma_commit_w(ds_full);
                     ++lc;
                 }
@@ -737,18 +744,18 @@ __global__ void __launch_bounds__(kMainThreads, 1)
                     const TileInfo ti = tile_info(i, p.W, l1_only);
                     const int qb = tile & 1;
                     const uint32_t q_addr = q_base + qb * TILE_B;
-                    if (!(ok = warp_wait(&q_full[qb], (tile >> 1) & 1, abort, p.status))) break;
+                    if (!(ok = warp_wait(&q_full[qb], (tile >> 1) & 1, abort, p.status, p.wait_ns))) break;
                     for (int j = 0; j < ti.nk && ok; ++j, ++g) {
                         const int s = g % NS, sb = g & 1;
-                        if (!(ok = warp_wait(&kv_full[s], (g / NS) & 1, abort, p.status))) break;
+                        if (!(ok = warp_wait(&kv_full[s], (g / NS) & 1, abort, p.status, p.wait_ns))) break;
                         // the state warps read the leading key tile: hand it on
                         if (j == 0 && ti.l2) mbar_arrive_w(lead_ready);
                         tc_fence_after();
                         const uint32_t k_addr = kv_base + s * 2 * TILE_B;
-#pragma unroll 1
+                        const uint64_t qd = sdesc_sw128(q_addr, 16, 1024), kd = sdesc_sw128(k_addr, 16, 1024);
+#pragma unroll
                         for (int k = 0; k < 4; ++k)
-                            mma_ss_w(tb + TM_S + sb * 128, sdesc_sw128(q_addr + 32 * k, 16, 1024),
-                                   sdesc_sw128(k_addr + 32 * k, 16, 1024), id_qk, k > 0);
+                            mma_ss_w(tb + TM_S + sb * 128, qd + 2 * k, kd + 2 * k, id_qk, k > 0);
                         mma_commit_w(&s_full[sb]);
                         if (pend.valid && !(ok = pv_step(pend))) break;
                         pend = {true, j == 0, j == ti.nk - 1, ti.l2, g, tile};
@@ -783,9 +790,9 @@ __global__ void __launch_bounds__(kMainThreads, 1)
         auto epilogue = [&](const Epi &e) -> bool {
             // y = O / l + sigmoid(g) (m_intra + lam^(r+1) m_inter)
             xl[half * 128 + r] = e.l;
-            if (!group_sync(sm_sync, sync_phase, abort, p.status)) return false;
+            if (!group_sync(sm_sync, sync_phase, abort, p.status, p.wait_ns)) return false;
             const float inv_l = 1.0f / (e.l + xl[(1 - half) * 128 + r]);
-            if (!warp_wait(o_full, e.tile & 1, abort, p.status)) return false;
+            if (!warp_wait(o_full, e.tile & 1, abort, p.status, p.wait_ns)) return false;
             tc_fence_after();
             float yv[32];
             uint32_t rr[32];
@@ -827,18 +834,18 @@ __global__ void __launch_bounds__(kMainThreads, 1)
             const float gate = 1.0f / (1.0f + expf(-p.g[h]));
             const float pw_r1 = (float)pow(lam, (double)(r + 1));
             // previous span done with epw, then publish this head's table
-            if (!(ok = group_sync(sm_sync, sync_phase, abort, p.status))) break;
+            if (!(ok = group_sync(sm_sync, sync_phase, abort, p.status, p.wait_ns))) break;
             if (half == 0)
                 epw[128 + r] = (float)((double)p.eta[h] * pow(lam, (double)r));
             else
                 epw[r] = 0.f;
-            if (!(ok = group_sync(sm_sync, sync_phase, abort, p.status))) break;
+            if (!(ok = group_sync(sm_sync, sync_phase, abort, p.status, p.wait_ns))) break;
             for (int i = i0; i < i1 && ok; ++i, ++tile) {
                 const TileInfo ti = tile_info(i, p.W, l1_only);
                 float m_used = -INFINITY, l = 0.f;
                 for (int j = 0; j < ti.nk && ok; ++j, ++kc) {
                     const int sb = kc & 1;
-                    if (!(ok = warp_wait(&s_full[sb], (kc >> 1) & 1, abort, p.status))) break;
+                    if (!(ok = warp_wait(&s_full[sb], (kc >> 1) & 1, abort, p.status, p.wait_ns))) break;
                     tc_fence_after();
                     const uint32_t s_col = TM_S + sb * 128;
                     float s[64];
@@ -859,7 +866,7 @@ __global__ void __launch_bounds__(kMainThreads, 1)
                     const float mh = half_max(skind, s, r - 64 * half);
                     float *xmk = xm + (kc & 1) * 256;
                     xmk[half * 128 + r] = mh;
-                    if (!(ok = group_sync(sm_sync, sync_phase, abort, p.status))) break;
+                    if (!(ok = group_sync(sm_sync, sync_phase, abort, p.status, p.wait_ns))) break;
                     const float mt = fmaxf(mh, xmk[(1 - half) * 128 + r]) * sl2;  // sl2 > 0
                     // Raise the row's reference max only when it grew by more than
                     // 2^kRescale; rows whose O already holds earlier P V products
@@ -869,7 +876,7 @@ __global__ void __launch_bounds__(kMainThreads, 1)
                     const bool resc = raise && m_used != -INFINITY && j > 0;
                     const float fo = resc ? ex2(m_used - mt) : 1.0f;
                     if (__any_sync(0xffffffffu, resc)) {
-                        if (!(ok = warp_wait(o_prog, (kc - 1) & 1, abort, p.status))) break;
+                        if (!(ok = warp_wait(o_prog, (kc - 1) & 1, abort, p.status, p.wait_ns))) break;
                         tc_fence_after();
                         uint32_t rr[32];
                         tmem_ld32(tmem_addr(tb, lane_base, TM_O + 32 * half), rr);
@@ -918,7 +925,7 @@ __global__ void __launch_bounds__(kMainThreads, 1)
             ew[u] = (float)((double)p.eta[h] * exp2((double)u * l2l));
             lp[u] = (float)exp2((double)u * l2l);
             if (u == 0) lp[128] = (float)exp2(128.0 * l2l);
-            if (!(ok = group_sync(st_sync, sync_phase, abort, p.status))) break;
+            if (!(ok = group_sync(st_sync, sync_phase, abort, p.status, p.wait_ns))) break;
             // state at the span start from the predecessors' summaries
             const int n_start = max(0, i0 * BM - p.W);
 #pragma unroll
@@ -942,7 +949,7 @@ __global__ void __launch_bounds__(kMainThreads, 1)
             auto consume = [&](int c_eff) -> bool {
                 // rows 64..127 of the increment (lo parts) go through shared
                 // memory to the owners of rows 0..63 (hi parts)
-                if (!warp_wait(ds_full, (lc - 1) & 1, abort, p.status)) return false;
+                if (!warp_wait(ds_full, (lc - 1) & 1, abort, p.status, p.wait_ns)) return false;
                 tc_fence_after();
                 uint32_t rr[32];
                 if (u >= 64) {
@@ -954,7 +961,7 @@ __global__ void __launch_bounds__(kMainThreads, 1)
                         for (int c = 0; c < 32; ++c) sDS[(c0 + c) * 64 + (u - 64)] = __uint_as_float(rr[c]);
                     }
                 }
-                if (!group_sync(st_sync, sync_phase, abort, p.status)) return false;
+                if (!group_sync(st_sync, sync_phase, abort, p.status, p.wait_ns)) return false;
                 if (u < 64) {
                     const float dec = lp[c_eff];
 #pragma unroll
@@ -967,7 +974,7 @@ __global__ void __launch_bounds__(kMainThreads, 1)
                                              __uint_as_float(rr[c]) + sDS[(c0 + c) * 64 + u]);
                     }
                 }
-                return group_sync(st_sync, sync_phase, abort, p.status);
+                return group_sync(st_sync, sync_phase, abort, p.status, p.wait_ns);
             };
             for (int i = i0; i < i1 && ok; ++i) {
                 const TileInfo ti = tile_info(i, p.W, l1_only);
@@ -987,7 +994,7 @@ __global__ void __launch_bounds__(kMainThreads, 1)
                     mbar_arrive(sst_full);
                     // scaled keys of the leading tile for the state MMA
                     const int s = kc % NS;
-                    if (!(ok = warp_wait(lead_ready, lc & 1, abort, p.status))) break;
+                    if (!(ok = warp_wait(lead_ready, lc & 1, abort, p.status, p.wait_ns))) break;
                     const int n0 = ti.t0 - p.W;
                     const int c_eff = min(BM, E - n0);
                     const float w = u < c_eff ? ew[c_eff - 1 - u] : 0.f;
@@ -1145,7 +1152,7 @@ cudaError_t launch_prefill_sm100(const PrefillParams &p, int num_sms, cudaStream
     float *dA = reinterpret_cast<float *>(p.workspace);
     if (!p.l1_only && ns > 1) {
         SumParams sp{dA, p.lam, p.eta, T_all, (int)p.W, (int)p.H, (int)BH, nT, ns, n_parts, q_off,
-                     p.status};
+                     p.status, p.wait_ns};
         span_summary_kernel<<<(unsigned)(BH * (ns - 1) * n_parts), 192, SMEM_SUM, s>>>(tk, tv, tkh,
                                                                                     tvh, sp);
         e = cudaGetLastError();
@@ -1156,7 +1163,8 @@ cudaError_t launch_prefill_sm100(const PrefillParams &p, int num_sms, cudaStream
         if (e != cudaSuccess) return e;
     }
     MainParams mp{p.y,      p.A_final, p.lam, p.eta, p.g,  dA, p.A_init, T_all, (int)p.W, (int)p.H,
-                  (int)BH, nT,        ns,    n_parts,         p.l1_only ? 1 : 0, q_off, p.status};
+                  (int)BH, nT,        ns,    n_parts,         p.l1_only ? 1 : 0, q_off, p.status,
+                  p.wait_ns};
     const int64_t spans = BH * ns;
     const unsigned grid = (unsigned)(spans < num_sms ? spans : num_sms);
     prefill_main_kernel<<<grid, kMainThreads, SMEM_MAIN, s>>>(tq, tk, tv, tkh, tvh, mp);

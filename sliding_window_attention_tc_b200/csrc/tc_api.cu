@@ -68,15 +68,23 @@ tc_status current_device(int *dev, int *num_sms) {
     return TC_OK;
 }
 
-// A pointer the device can dereference (device or managed memory).
-bool is_device_ptr(const void *p) {
+// A pointer the current device dev can dereference: managed memory, or
+// device memory allocated on dev itself.  Memory of another GPU is refused:
+// a kernel on dev would otherwise read it over the peer link, or fault when
+// peer access is off.
+bool is_device_ptr(const void *p, int dev) {
     cudaPointerAttributes a;
     if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
         cudaGetLastError();
         return false;
     }
-    return a.type == cudaMemoryTypeDevice || a.type == cudaMemoryTypeManaged;
+    return a.type == cudaMemoryTypeManaged || (a.type == cudaMemoryTypeDevice && a.device == dev);
 }
+
+// Limit of the bounded waits inside the tensor-core kernels (0 = default).
+unsigned long long g_wait_limit_ns = 0;
+constexpr unsigned long long kDefaultWaitNs = 2000000000ull;  // 2 s
+unsigned long long wait_limit_ns() { return g_wait_limit_ns ? g_wait_limit_ns : kDefaultWaitNs; }
 
 int *status_ptr() {
     void *p = nullptr;
@@ -123,6 +131,8 @@ tc_status check_decode_state(const tc_decode_state *s) {
 extern "C" {
 
 const char *tc_version(void) { return "0.1.0"; }
+
+void tc_set_wait_limit_ns(uint64_t ns) { g_wait_limit_ns = ns; }
 
 const char *tc_status_string(tc_status s) {
     switch (s) {
@@ -183,12 +193,12 @@ tc_status prefill_impl(const tc_prefill_desc *d, int64_t t0, const void *halo_k,
     const void *ptrs[] = {q, y, k, v, lambda, eta, g};
     for (int i = 0; i < 7; ++i) {
         const bool may_be_null = (i < 2 && !need_q) || (i < 4 && empty);
-        if (!(may_be_null && !ptrs[i]) && !is_device_ptr(ptrs[i])) return TC_ERR_INVALID_ARG;
+        if (!(may_be_null && !ptrs[i]) && !is_device_ptr(ptrs[i], dev)) return TC_ERR_INVALID_ARG;
     }
-    if (A_final && !is_device_ptr(A_final)) return TC_ERR_INVALID_ARG;
-    if (A_init && !is_device_ptr(A_init)) return TC_ERR_INVALID_ARG;
-    if (n_halo > 0 && (!is_device_ptr(halo_k) || !is_device_ptr(halo_v))) return TC_ERR_INVALID_ARG;
-    if (need > 0 && !is_device_ptr(workspace)) return TC_ERR_INVALID_ARG;
+    if (A_final && !is_device_ptr(A_final, dev)) return TC_ERR_INVALID_ARG;
+    if (A_init && !is_device_ptr(A_init, dev)) return TC_ERR_INVALID_ARG;
+    if (n_halo > 0 && (!is_device_ptr(halo_k, dev) || !is_device_ptr(halo_v, dev))) return TC_ERR_INVALID_ARG;
+    if (need > 0 && !is_device_ptr(workspace, dev)) return TC_ERR_INVALID_ARG;
 
     tc::PrefillParams p{};
     p.q = q;
@@ -217,6 +227,7 @@ tc_status prefill_impl(const tc_prefill_desc *d, int64_t t0, const void *halo_k,
     p.workspace = workspace;
     p.workspace_bytes = workspace_bytes;
     p.status = status_ptr();
+    p.wait_ns = wait_limit_ns();
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     cudaError_t e = use_sm100(*d, n_halo) ? tc::launch_prefill_sm100(p, sms, s)
                                           : tc::launch_prefill_portable(p, d->dtype, s);
@@ -270,10 +281,10 @@ tc_status tc_backward(const tc_prefill_desc *d, const void *q, const void *k, co
     const size_t need = tc::backward_workspace_bytes(*d);
     if (need > 0 && (!workspace || workspace_bytes < need)) return TC_ERR_WORKSPACE;
     for (const void *x : tok)
-        if (x && !is_device_ptr(x)) return TC_ERR_INVALID_ARG;
+        if (x && !is_device_ptr(x, dev)) return TC_ERR_INVALID_ARG;
     for (const void *x : hd)
-        if (!is_device_ptr(x)) return TC_ERR_INVALID_ARG;
-    if (need > 0 && !is_device_ptr(workspace)) return TC_ERR_INVALID_ARG;
+        if (!is_device_ptr(x, dev)) return TC_ERR_INVALID_ARG;
+    if (need > 0 && !is_device_ptr(workspace, dev)) return TC_ERR_INVALID_ARG;
     cudaError_t e = tc::launch_backward(*d, q, k, v, lambda, eta, g, dy, dq, dk, dv, dlambda, deta,
                                         dg, workspace, reinterpret_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? TC_OK : TC_ERR_CUDA;
@@ -311,7 +322,7 @@ tc_status tc_prefill_host(const tc_prefill_desc *d, const void *q, const void *k
     if (st != TC_OK) return st;
     const size_t need = tc_prefill_host_workspace_size(d);
     if (!workspace || workspace_bytes < need) return TC_ERR_WORKSPACE;
-    if (!aligned16(workspace) || !is_device_ptr(workspace)) return TC_ERR_INVALID_ARG;
+    if (!aligned16(workspace) || !is_device_ptr(workspace, dev)) return TC_ERR_INVALID_ARG;
 
     const size_t es = elem_size(d->dtype);
     const size_t nq = (size_t)(d->B * d->H * d->T * d->dk) * es;
@@ -366,8 +377,8 @@ tc_status decode_impl(tc_decode_state *s, int64_t *t_rows, const void *q_t, cons
     if (st != TC_OK) return st;
     const void *ptrs[] = {q_t, k_t, v_t, y_t, s->ring_k, s->ring_v, s->A, s->lambda, s->eta, s->g};
     for (const void *p : ptrs)
-        if (!is_device_ptr(p)) return TC_ERR_INVALID_ARG;
-    if (t_rows && !is_device_ptr(t_rows)) return TC_ERR_INVALID_ARG;
+        if (!is_device_ptr(p, dev)) return TC_ERR_INVALID_ARG;
+    if (t_rows && !is_device_ptr(t_rows, dev)) return TC_ERR_INVALID_ARG;
     tc::DecodeParams p{};
     p.q = q_t;
     p.k = k_t;
@@ -431,7 +442,7 @@ tc_status tc_decode_step_host(tc_decode_state *s, const void *q_t, const void *k
     if (st != TC_OK) return st;
     const size_t need = tc_decode_step_host_workspace_size(s);
     if (!workspace || workspace_bytes < need) return TC_ERR_WORKSPACE;
-    if (!aligned16(workspace) || !is_device_ptr(workspace)) return TC_ERR_INVALID_ARG;
+    if (!aligned16(workspace) || !is_device_ptr(workspace, dev)) return TC_ERR_INVALID_ARG;
     const size_t es = elem_size(s->kv_dtype);
     const size_t nk = (size_t)(s->B * s->H * s->dk) * es, nv = (size_t)(s->B * s->H * s->dv) * es;
     char *dq = static_cast<char *>(workspace);

@@ -96,6 +96,7 @@ struct PrefillParams {
     void *workspace;
     size_t workspace_bytes;
     int *status;
+    unsigned long long wait_ns;  // limit of the tensor-core kernels' bounded waits
 };
 
 // decode.cu

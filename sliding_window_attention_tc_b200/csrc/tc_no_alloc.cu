@@ -13,7 +13,11 @@
 // Its device address is looked up once per device with cudaGetSymbolAddress
 // (a host-side use of the array's name is not a device address) on the first
 // call made while that device is current; that first call should therefore
-// happen before any stream capture.  All calls share the one array: its
+// happen before any stream capture.  The address is cached for the life of
+// the context: after cudaDeviceReset the array may move, so the cache entry
+// is dropped when a call fails with a CUDA error, and callers should not rely
+// on the entry point across a device reset without making a fresh first call.
+// All calls share the one array: its
 // contents are whatever the previous call left there, which is harmless
 // because the prefill writes every scratch byte before reading it, and two
 // calls whose kernels overlap on the GPU (different streams, no ordering
@@ -65,6 +69,13 @@ extern "C" tc_status tc_prefill_no_alloc(const tc_prefill_desc *desc, const void
     }
     void *scratch = scratch_address(dev);
     if (!scratch) return TC_ERR_CUDA;
-    return tc_prefill(desc, q, k, v, lambda, eta, g, y, A_final, scratch,
-                      (size_t)TC_NO_ALLOC_SCRATCH_BYTES, stream);
+    const tc_status st = tc_prefill(desc, q, k, v, lambda, eta, g, y, A_final, scratch,
+                                    (size_t)TC_NO_ALLOC_SCRATCH_BYTES, stream);
+    if (st == TC_ERR_CUDA) {
+        // the cached address may belong to a context that no longer exists
+        // (cudaDeviceReset): look it up again on the next call
+        std::lock_guard<std::mutex> lock(g_mutex);
+        g_scratch_ptr[dev] = nullptr;
+    }
+    return st;
 }

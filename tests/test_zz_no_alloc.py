@@ -4,9 +4,10 @@ tc_prefill_no_alloc serves callers that cannot allocate device memory: it
 runs the same prefill with the library's built-in scratch array in place of
 a caller workspace.  These tests call it through the C-ABI twice in a row
 with different inputs (the second call finds the first call's data in the
-shared scratch) and compare each result with tc_prefill's, using the same
-tolerances as the parity tests.  This file is named so that pytest collects
-it last.
+shared scratch) and require each result to equal tc_prefill's bit for bit:
+both run the same deterministic kernels on the same inputs, so any
+difference would be scratch data leaking from one call into the next.  This
+file is named so that pytest collects it last.
 """
 import ctypes
 
@@ -60,14 +61,9 @@ def test_no_alloc_matches_workspace_entry_point(cuda_device, case):
         y_ref, A_ref = tc.prefill(*args, W, C)
         torch.cuda.synchronize()
         assert tc.device_status() == 0
-        y_na, y_ref = y_na.double().cpu().numpy(), y_ref.double().cpu().numpy()
-        A_na, A_ref = A_na.double().cpu().numpy(), A_ref.double().cpu().numpy()
-        if dtype == "f32":
-            assert np.abs(y_na - y_ref).max() <= 1e-5 * np.abs(y_ref).max()
-            assert np.abs(A_na - A_ref).max() <= 1e-5 * np.abs(A_ref).max()
-        else:
-            assert np.linalg.norm(y_na - y_ref) <= 1e-2 * np.linalg.norm(y_ref)
-            assert np.linalg.norm(A_na - A_ref) <= 1e-3 * np.linalg.norm(A_ref)
+        assert torch.equal(y_na, y_ref)
+        assert torch.equal(A_na, A_ref)
+        assert np.isfinite(y_ref.float().cpu().numpy()).all()
 
 
 def test_no_alloc_rejects_more_scratch_than_it_has(cuda_device):
