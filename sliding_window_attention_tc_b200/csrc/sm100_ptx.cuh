@@ -66,9 +66,12 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
                                           int *status, uint64_t limit_ns = kWaitTimeoutNs) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer();
+    // the timer is read every 256 failed tries, or on every try when the
+    // limit is short (a test of the timeout path)
+    const uint32_t every = limit_ns < 1000000u ? 0u : 255u;
     for (uint32_t i = 1;; ++i) {
         if (mbar_try_wait(bar, parity)) return true;
-        if ((i & 255u) == 0) {
+        if ((i & every) == 0) {
             if (*abort) return false;
             if (globaltimer() - t0 > limit_ns) {
                 *abort = 1;
@@ -120,9 +123,12 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
                                           int *status, uint64_t limit_ns = kWaitTimeoutNs) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer();
+    // the timer is read every 256 failed tries, or on every try when the
+    // limit is short (a test of the timeout path)
+    const uint32_t every = limit_ns < 1000000u ? 0u : 255u;
     for (uint32_t i = 1;; ++i) {
         if (mbar_try_wait(bar, parity)) return true;
-        if ((i & 255u) == 0) {
+        if ((i & every) == 0) {
             if (*abort) return false;
             if (globaltimer() - t0 > limit_ns) {
                 *abort = 1;
