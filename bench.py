@@ -24,6 +24,7 @@ same JSON line with "impl": "reference".
 from __future__ import annotations
 
 import argparse
+import ctypes
 import json
 import os
 import statistics
@@ -406,6 +407,41 @@ def time_training_extras(tc, dev):
     return out
 
 
+def time_varlen(tc, dev, steps=20, warmup=3):
+    """The variable-length workload in one tc_prefill_varlen call, against the
+    same sequences run as one tc_prefill call each (device-resident inputs,
+    CUDA events, ms per whole batch)."""
+    x = wl.varlen_config()
+    q, k, v, cu = (t.to(dev) for t in (x.q, x.k, x.v, x.cu_seqlens))
+    prm = tuple(t.to(dev) for t in (x.lam, x.eta, x.g))
+    total, H, d = q.shape
+    n = len(x.cu_seqlens) - 1
+    y = torch.empty_like(v)
+    A = torch.empty(n, H, d, d, dtype=torch.float32, device=dev)
+    desc = tc.make_prefill_desc(n, H, x.max_seqlen, d, d, x.W, x.C, tc.TC_BF16)
+    ws_n = tc.lib_handle().tc_prefill_varlen_workspace_size(ctypes.byref(desc))
+    ws = torch.empty(max(ws_n, 1), dtype=torch.uint8, device=dev)
+    one = statistics.median(time_calls(
+        lambda: tc.prefill_varlen(q, k, v, cu, x.max_seqlen, *prm, x.W, x.C, y=y, A_final=A,
+                                  workspace=ws if ws_n else None), steps, warmup))
+    seqs = [tuple(t.to(dev) for t in x.sequence(b)) for b in range(n)]
+    outs = [(torch.empty_like(s[2]), torch.empty(1, H, d, d, dtype=torch.float32, device=dev))
+            for s in seqs]
+
+    def per_sequence():
+        for s, (ys, As) in zip(seqs, outs):
+            tc.prefill(*s, *prm, x.W, x.C, y=ys, A_final=As)
+
+    many = statistics.median(time_calls(per_sequence, max(5, steps // 4), warmup))
+    tokens = total * H
+    return {"workload": "varlen prefill, 15 sequences of 55..8192 tokens (32768 in all), "
+                        "H=12, d=64, W=512, bf16",
+            "lengths": list(wl.VARLEN_CONFIG["lengths"]), "ms": one, "tokens_per_s": tokens / (one * 1e-3),
+            "launches_per_call": tc.prefill_launch_count(desc),
+            "per_sequence_calls_ms": many,
+            "per_sequence_calls_tokens_per_s": tokens / (many * 1e-3)}
+
+
 # ---------------------------------------------------------------------------
 def _rows_per_call(B, H, threads):
     """Batch rows per oracle call: the fewest (at least one item per thread)
@@ -510,6 +546,9 @@ def run_only(args, tc, dev, world, peaks):
         print(json.dumps({"only": "decode", "B": d["B"], "steps": d["steps"], "ms_per_step": ms,
                           "GB_per_s": d["bytes_per_step"] / (ms * 1e-3) / 1e9}))
         return 0
+    if args.only == "varlen":
+        print(json.dumps({"only": "varlen", **time_varlen(tc, dev, args.steps, args.warmup)}))
+        return 0
     name = HEADLINE if args.only == "prefill" else "long_prefill_bf16"
     r = time_prefill(tc, name, dev, args.steps, args.warmup, world)
     x = r["x"]
@@ -531,7 +570,7 @@ def main():
     ap.add_argument("--impl", default="tc", choices=["tc", "reference"])
     ap.add_argument("--no-extras", action="store_true",
                     help="headline prefill only (skip decode, long prefill, oracle)")
-    ap.add_argument("--only", choices=["prefill", "long", "decode"], default=None,
+    ap.add_argument("--only", choices=["prefill", "long", "decode", "varlen"], default=None,
                     help="time one workload only and print its numbers (profiling runs)")
     ap.add_argument("--decode-batch", type=int, default=None,
                     help="batch of the decode workload (default 256)")
@@ -623,6 +662,7 @@ def main():
                         "tokens_per_s": dec["B"] / (dec["e2e_ms_per_step"] * 1e-3),
                         "h2d_bytes_per_step": dec["e2e_h2d_bytes"],
                         "d2h_bytes_per_step": dec["e2e_d2h_bytes"]}}
+            extras["varlen_prefill"] = time_varlen(tc, dev)
             extras.update(time_training_extras(tc, dev))
         e2e = time_prefill_e2e(tc, HEADLINE, dev, max(5, min(20, args.steps // 10)))
     finally:

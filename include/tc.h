@@ -164,6 +164,40 @@ TC_API tc_status tc_prefill_from_state(const tc_prefill_desc *desc, int64_t t0,
                                        const float *g, void *y, float *A_final, void *workspace,
                                        size_t workspace_bytes, tc_stream_t stream);
 
+/* Variable-length prefill: desc->B sequences of different lengths in one
+ * call, each the layer over its own tokens from an empty state (ring empty,
+ * A = 0), exactly as tc_prefill would run it alone.  Each sequence runs its
+ * own streaming step (§3.2, Fig. 2); nothing passes between sequences.
+ *
+ *   cu_seqlens  int64 device [desc->B + 1], 8-byte aligned: sequence b holds
+ *               the packed token rows cu_seqlens[b] .. cu_seqlens[b+1]-1.
+ *               cu_seqlens[0] = 0, non-decreasing, cu_seqlens[B] = total,
+ *               every length <= desc->T.  Empty sequences are allowed.
+ *   total       packed token rows, 0 <= total <= 2^30.
+ *   desc->T     the longest length (it sizes the schedule and workspace).
+ *   q, k, v, y  packed token-major [total, H, d] (head rows of one token
+ *               adjacent); may be NULL when total = 0.
+ *   A_final     [B, H, d_k, d_v] float32, A after each sequence's last
+ *               eviction (0 for a sequence of at most W tokens); may be NULL
+ *               only with TC_PREFILL_L1_ONLY.
+ *   workspace   tc_prefill_varlen_workspace_size(desc) bytes.
+ *
+ * Supported: the tensor-core path only (bf16, d_k = d_v = 64, W a multiple
+ * of 128, flags 0 or TC_PREFILL_L1_ONLY); other descriptions return
+ * TC_ERR_UNSUPPORTED (and (size_t)-1 from the size query).  The offsets are
+ * device data, so the host cannot check them: the kernels do.  A sequence
+ * whose offsets are negative, decreasing, past total or longer than desc->T
+ * is skipped (its rows of y are not written, its A_final is zero) and the
+ * call sets TC_ERR_DEVICE_BOUNDS in the device status word
+ * (tc_get_device_status); nothing outside the buffers is read or written.
+ * Other errors as tc_prefill. */
+TC_API size_t tc_prefill_varlen_workspace_size(const tc_prefill_desc *desc);
+TC_API tc_status tc_prefill_varlen(const tc_prefill_desc *desc, const int64_t *cu_seqlens,
+                                   int64_t total, const void *q, const void *k, const void *v,
+                                   const float *lambda, const float *eta, const float *g, void *y,
+                                   float *A_final, void *workspace, size_t workspace_bytes,
+                                   tc_stream_t stream);
+
 /* Exclusive prefix of L2 states over consecutive pieces of one sequence
  * (sequence sharding: piece s is the part of the sequence held by rank s).
  * Piece s alone, started from A = 0, leaves dA_s after its E_s evictions

@@ -50,7 +50,7 @@ EXPORTED = ("tc_prefill_workspace_size", "tc_prefill", "tc_prefill_launch_count"
             "tc_decode_step_host", "tc_get_device_status", "tc_status_string", "tc_version",
             "tc_prefill_no_alloc", "tc_prefill_from_state", "tc_prefill_from_state_workspace_size",
             "tc_state_fold", "tc_decode_step_ragged", "tc_backward", "tc_backward_workspace_size",
-            "tc_set_wait_limit_ns")
+            "tc_set_wait_limit_ns", "tc_prefill_varlen", "tc_prefill_varlen_workspace_size")
 
 
 class PrefillDesc(ctypes.Structure):
@@ -87,6 +87,10 @@ _lib.tc_prefill_from_state_workspace_size.argtypes = [_PD, ctypes.c_int64]
 _lib.tc_prefill_from_state_workspace_size.restype = _sz
 _lib.tc_prefill_from_state.argtypes = [_PD, ctypes.c_int64] + [_vp] * 12 + [_sz, _vp]
 _lib.tc_prefill_from_state.restype = _int
+_lib.tc_prefill_varlen_workspace_size.argtypes = [_PD]
+_lib.tc_prefill_varlen_workspace_size.restype = _sz
+_lib.tc_prefill_varlen.argtypes = [_PD, _vp, ctypes.c_int64] + [_vp] * 9 + [_sz, _vp]
+_lib.tc_prefill_varlen.restype = _int
 _lib.tc_backward_workspace_size.argtypes = [_PD]
 _lib.tc_backward_workspace_size.restype = _sz
 _lib.tc_backward.argtypes = [_PD] + [_vp] * 14 + [_sz, _vp]
@@ -253,6 +257,49 @@ def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, lam: torch.Tensor
                          _ptr(g), _ptr(y), _ptr(A_final), _ptr(workspace), ws_bytes,
                          _stream(stream))
     _check(st, "tc_prefill")
+    return y, A_final
+
+
+def prefill_varlen(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlens: torch.Tensor,
+                   max_seqlen: int, lam: torch.Tensor, eta: torch.Tensor, g: torch.Tensor,
+                   W: int, C: int, *, l1_only: bool = False, y: Optional[torch.Tensor] = None,
+                   A_final: Optional[torch.Tensor] = None,
+                   workspace: Optional[torch.Tensor] = None, stream=None):
+    """tc_prefill_varlen: len(cu_seqlens) - 1 sequences packed token-major,
+    q, k [total,H,dk], v [total,H,dv] bfloat16; sequence b is rows
+    cu_seqlens[b] .. cu_seqlens[b+1]-1 (cu_seqlens int64 on the device),
+    max_seqlen its longest length.  Each sequence starts from an empty
+    state.  Returns (y [total,H,dv], A_final [B,H,dk,dv] float32 or None with
+    l1_only)."""
+    total, H, dk = k.shape
+    dv = v.shape[-1]
+    B = cu_seqlens.numel() - 1
+    if B < 1:
+        raise ValueError("cu_seqlens needs at least two entries")
+    _expect(cu_seqlens, "cu_seqlens", (B + 1,), torch.int64)
+    _expect(q, "q", (total, H, dk), k.dtype)
+    _expect(v, "v", (total, H, dv), k.dtype)
+    for name, t in (("lam", lam), ("eta", eta), ("g", g)):
+        _expect(t, name, (H,), torch.float32)
+    _expect(y, "y", (total, H, dv), k.dtype)
+    _expect(A_final, "A_final", (B, H, dk, dv), torch.float32)
+    desc = make_prefill_desc(B, H, int(max_seqlen), dk, dv, W, C, _dtype_code(k), l1_only)
+    if y is None:
+        y = torch.empty((total, H, dv), dtype=k.dtype, device=k.device)
+    if A_final is None and not l1_only:
+        A_final = torch.empty((B, H, dk, dv), dtype=torch.float32, device=k.device)
+    need = _lib.tc_prefill_varlen_workspace_size(ctypes.byref(desc))
+    if need == SIZE_ERROR:
+        raise TCError(2, "tc_prefill_varlen_workspace_size")
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=k.device)
+    _contig(q, k, v, cu_seqlens, lam, eta, g, y, A_final, workspace)
+    _dev_check(q, k, v, cu_seqlens, lam, eta, g, y, A_final, workspace)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = _lib.tc_prefill_varlen(ctypes.byref(desc), _ptr(cu_seqlens), int(total), _ptr(q),
+                                _ptr(k), _ptr(v), _ptr(lam), _ptr(eta), _ptr(g), _ptr(y),
+                                _ptr(A_final), _ptr(workspace), ws_bytes, _stream(stream))
+    _check(st, "tc_prefill_varlen")
     return y, A_final
 
 

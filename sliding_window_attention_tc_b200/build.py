@@ -1,6 +1,6 @@
 """Build libtc.so in-tree with nvcc for sm_100a.
 
-    python sliding_window_attention_tc_b200/build.py [--force] [--debug] [-v]
+    python sliding_window_attention_tc_b200/build.py [--force] [-v]
 
 Each .cu file under csrc/ is compiled to an object with
 ``-gencode arch=compute_100a,code=sm_100a -lineinfo -O3`` and the objects are
@@ -52,14 +52,12 @@ def needs_build() -> bool:
     return any(os.path.getmtime(f) > t for f in _deps())
 
 
-def build(force: bool = False, debug: bool = False, verbose: bool = False) -> str:
+def build(force: bool = False, verbose: bool = False) -> str:
     if not force and not needs_build():
         return LIB
     os.makedirs(OBJDIR, exist_ok=True)
     nvcc = _nvcc()
     flags = list(NVCC_FLAGS)
-    if debug:
-        flags.append("-DTC_DEBUG_BOUNDS=1")
     if verbose:
         flags += ["-Xptxas", "-v"]
     objs = []
@@ -78,5 +76,5 @@ def build(force: bool = False, debug: bool = False, verbose: bool = False) -> st
 
 
 if __name__ == "__main__":
-    build(force="--force" in sys.argv, debug="--debug" in sys.argv, verbose="-v" in sys.argv)
+    build(force="--force" in sys.argv, verbose="-v" in sys.argv)
     print(LIB)

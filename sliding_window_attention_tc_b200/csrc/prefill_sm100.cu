@@ -85,11 +85,20 @@ constexpr uint32_t TM_DS = 448; // state increment: rows 0-63 hi part, 64-127 lo
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescale = 8.0f;  // rescale O only when the running max grows by > 2^8
 
+// Variable-length calls: sequence b of the batch is tokens cu[b] .. cu[b+1]-1
+// of packed [total][H][64] tensors; cu == null for fixed-length calls.
+struct Varlen {
+    const int64_t *cu;   // device [n_seq + 1]
+    int total, max_len;
+};
+
 struct PrefixParams {
     float *dA;            // [BH * (n_s - 1) * n_parts][64][64]: partial summaries in,
                           // span start states out (over part 0 of the previous span)
     const float *lam;
     int T, W, H, nT, n_s, n_parts, q_off;
+    Varlen vl;
+    int *status;
 };
 
 // Token coordinates.  The kernels run over a combined sequence of T tokens:
@@ -106,6 +115,7 @@ struct MainParams {
     int T, W, H, BH, nT, n_s, n_parts, l1_only, q_off;
     int *status;
     unsigned long long wait_ns;  // limit of every bounded wait
+    Varlen vl;
 };
 
 struct SumParams {
@@ -114,6 +124,7 @@ struct SumParams {
     int T, W, H, BH, nT, n_s, n_parts, q_off;
     int *status;
     unsigned long long wait_ns;  // limit of every bounded wait
+    Varlen vl;
 };
 
 // Query tiles [i0, i1) of span j: the tiles i_begin .. nT-1 cut into n_s parts.
@@ -123,18 +134,62 @@ __device__ __forceinline__ void span_range(int j, int nT, int n_s, int i_begin, 
     i1 = i_begin + (int)((long long)(j + 1) * n / n_s);
 }
 
+// The sequence of row bh (one head of one sequence).  Fixed-length calls: T
+// tokens (halo included) in the row's own [T][64] slab.  Variable-length
+// calls: sequence b = bh / H, tokens cu[b] .. cu[b+1]-1 of the packed
+// [total][H][64] tensors, head z = bh % H.  Offsets that are inconsistent
+// (decreasing, past total, or longer than max_len) are reported as
+// TC_ERR_DEVICE_BOUNDS and the row is treated as empty, so nothing outside
+// the tensors is read or written.
+struct SeqView {
+    int T, nT, row0, z;
+};
+__device__ __forceinline__ SeqView seq_view(const Varlen &vl, int bh, int H, int T_fixed,
+                                            int *status) {
+    SeqView v;
+    if (!vl.cu) {
+        v.T = T_fixed;
+        v.row0 = 0;
+        v.z = bh;
+    } else {
+        const int b = bh / H;
+        const int64_t a = vl.cu[b], e = vl.cu[b + 1];
+        if (a < 0 || e < a || e > vl.total || e - a > vl.max_len) {
+            report(status, 5);
+            v.T = 0;
+            v.row0 = 0;
+        } else {
+            v.T = (int)(e - a);
+            v.row0 = (int)a;
+        }
+        v.z = bh % H;
+    }
+    v.nT = (v.T + BM - 1) / BM;
+    return v;
+}
+
+// 128 rows starting at sequence row `row` of a [.][64] tensor map: (0, row, z)
+// for fixed-length maps, (0, z, row0 + row) for the packed (d, H, total) maps.
+__device__ __forceinline__ void tma_rows(void *dst, const CUtensorMap *m, uint64_t *bar, int row,
+                                         const SeqView &v, bool varlen) {
+    if (varlen)
+        tma_load_3d(dst, m, bar, 0, v.z, v.row0 + row);
+    else
+        tma_load_3d(dst, m, bar, 0, row, v.z);
+}
+
 // Key / value tile u of the combined sequence: halo maps for u < q_off/128.
 __device__ __forceinline__ void load_kv_tile(uint8_t *dst, const CUtensorMap *tk,
                                              const CUtensorMap *tv, const CUtensorMap *tkh,
                                              const CUtensorMap *tvh, uint64_t *bar, int u,
-                                             int q_off, int bh) {
+                                             int q_off, const SeqView &v, bool varlen) {
     const int row = u * 128;
     if (row < q_off) {
-        tma_load_3d(dst, tkh, bar, 0, row, bh);
-        tma_load_3d(dst + 128 * 64 * 2, tvh, bar, 0, row, bh);
+        tma_load_3d(dst, tkh, bar, 0, row, v.z);
+        tma_load_3d(dst + 128 * 64 * 2, tvh, bar, 0, row, v.z);
     } else {
-        tma_load_3d(dst, tk, bar, 0, row - q_off, bh);
-        tma_load_3d(dst + 128 * 64 * 2, tv, bar, 0, row - q_off, bh);
+        tma_rows(dst, tk, bar, row - q_off, v, varlen);
+        tma_rows(dst + 128 * 64 * 2, tv, bar, row - q_off, v, varlen);
     }
 }
 
@@ -378,16 +433,17 @@ __global__ void __launch_bounds__(256) span_prefix_kernel(PrefixParams p) {
     const int per_head = p.n_s - 1;
     if (threadIdx.x >= 1 && (int)threadIdx.x < p.n_s) {
         const int js = threadIdx.x;
+        const SeqView sv = seq_view(p.vl, bh, p.H, p.T, js == 1 ? p.status : nullptr);
         const double l2l = log2((double)p.lam[h]);
-        const int E = p.T > p.W ? p.T - p.W : 0;
+        const int E = sv.T > p.W ? sv.T - p.W : 0;
         int a0, a1, b0, b1, z0, z1;
-        span_range(js - 1, p.nT, p.n_s, p.q_off / BM, a0, a1);
-        span_range(js, p.nT, p.n_s, p.q_off / BM, b0, b1);
+        span_range(js - 1, sv.nT, p.n_s, p.q_off / BM, a0, a1);
+        span_range(js, sv.nT, p.n_s, p.q_off / BM, b0, b1);
         const int n_start = max(0, b0 * BM - p.W);
         const int e_end = max(0, min(E, a1 * BM - p.W));
         int n_prev = 0;
         if (js > 1) {
-            span_range(js - 1, p.nT, p.n_s, p.q_off / BM, z0, z1);
+            span_range(js - 1, sv.nT, p.n_s, p.q_off / BM, z0, z1);
             n_prev = max(0, z0 * BM - p.W);
         }
         const int n1 = n_start - n_prev, n2 = n_start - e_end;
@@ -442,9 +498,11 @@ __global__ void __launch_bounds__(192, 2)
     const int part = slot % p.n_parts;
     const int bh = slot / (per_head * p.n_parts), js = (slot / p.n_parts) % per_head;
     const int h = bh % p.H;
+    const bool varlen = p.vl.cu != nullptr;
+    const SeqView sv = seq_view(p.vl, bh, p.H, p.T, tid == 0 ? p.status : nullptr);
     int i0, i1;
-    span_range(js, p.nT, p.n_s, p.q_off / BM, i0, i1);
-    const int E = p.T > p.W ? p.T - p.W : 0;
+    span_range(js, sv.nT, p.n_s, p.q_off / BM, i0, i1);
+    const int E = sv.T > p.W ? sv.T - p.W : 0;
     const int ev_span = i0 > p.W / BM ? i0 : p.W / BM;  // first tile of the span with evictions
     const int ne_span = i1 > ev_span ? i1 - ev_span : 0;
     // this CTA's share of the span's eviction tiles; every part decays to
@@ -487,7 +545,7 @@ __global__ void __launch_bounds__(192, 2)
                 const int n0 = (ev_first + e) * BM - p.W;
                 uint8_t *dst = sm + SOFF_KV + s * 2 * TILE_B;
                 mbar_expect_tx(&kv_full[s], 2 * TILE_B);
-                load_kv_tile(dst, &tk, &tv, &tkh, &tvh, &kv_full[s], n0 / BM, p.q_off, bh);
+                load_kv_tile(dst, &tk, &tv, &tkh, &tvh, &kv_full[s], n0 / BM, p.q_off, sv, varlen);
                 issued = e + 1;
             }
             for (int st = 0; st < NS_SUM; ++st) {
@@ -593,7 +651,7 @@ __global__ void __launch_bounds__(kMainThreads, 1)
     const int tid = threadIdx.x, warp = tid >> 5;
     const bool l1_only = p.l1_only != 0;
     const int n_spans = p.BH * p.n_s;
-    const int E = p.T > p.W ? p.T - p.W : 0;
+    const bool varlen = p.vl.cu != nullptr;
 
     if (tid == 0) {
         for (int b = 0; b < 2; ++b) {
@@ -642,20 +700,21 @@ __global__ void __launch_bounds__(kMainThreads, 1)
             bool ok = true;
             for (int sp = blockIdx.x; sp < n_spans && ok; sp += gridDim.x) {
                 const int bh = sp / p.n_s;
+                const SeqView sv = seq_view(p.vl, bh, p.H, p.T, nullptr);
                 int i0, i1;
-                span_range(sp % p.n_s, p.nT, p.n_s, p.q_off / BM, i0, i1);
+                span_range(sp % p.n_s, sv.nT, p.n_s, p.q_off / BM, i0, i1);
                 for (int i = i0; i < i1 && ok; ++i, ++tile) {
                     const TileInfo ti = tile_info(i, p.W, l1_only);
                     const int qb = tile & 1;
                     if (!(ok = mbar_wait(&q_empty[qb], ((tile >> 1) & 1) ^ 1, abort, p.status, p.wait_ns))) break;
                     mbar_expect_tx(&q_full[qb], TILE_B);
-                    tma_load_3d(sm + OFF_Q + qb * TILE_B, &tq, &q_full[qb], 0, ti.t0 - p.q_off, bh);
+                    tma_rows(sm + OFF_Q + qb * TILE_B, &tq, &q_full[qb], ti.t0 - p.q_off, sv, varlen);
                     for (int j = 0; j < ti.nk; ++j, ++kc) {
                         const int s = kc % NS;
                         if (!(ok = mbar_wait(&kv_empty[s], ((kc / NS) & 1) ^ 1, abort, p.status, p.wait_ns))) break;
                         uint8_t *dst = sm + OFF_KV + s * 2 * TILE_B;
                         mbar_expect_tx(&kv_full[s], 2 * TILE_B);
-                        load_kv_tile(dst, &tk, &tv, &tkh, &tvh, &kv_full[s], ti.kt0 + j, p.q_off, bh);
+                        load_kv_tile(dst, &tk, &tv, &tkh, &tvh, &kv_full[s], ti.kt0 + j, p.q_off, sv, varlen);
                     }
                 }
             }
@@ -678,9 +737,7 @@ __global__ void __launch_bounds__(kMainThreads, 1)
         // the current tile.  Q K^T of tile g+1 overwrites the score buffer
         // whose P (and P') the P V (and P'V) of tile g-1 reads; it is issued
         // right after them without waiting for their completion, because the
-        // tensor core runs one thread's MMAs in issue order.  The MMA loops
-        // are not unrolled: the issue is nearly synchronous anyway, and the
-        // smaller code misses the instruction cache less often.
+        // tensor core runs one thread's MMAs in issue order.
         {
             const uint32_t id_qk = idesc_bf16(128, 128, false, false);
             const uint32_t id_pv = idesc_bf16(128, 64, false, true);
@@ -738,8 +795,9 @@ __global__ void __launch_bounds__(kMainThreads, 1)
                 return true;
             };
             for (int sp = blockIdx.x; sp < n_spans && ok; sp += gridDim.x) {
+                const SeqView sv = seq_view(p.vl, sp / p.n_s, p.H, p.T, nullptr);
                 int i0, i1;
-                span_range(sp % p.n_s, p.nT, p.n_s, p.q_off / BM, i0, i1);
+                span_range(sp % p.n_s, sv.nT, p.n_s, p.q_off / BM, i0, i1);
                 for (int i = i0; i < i1 && ok; ++i, ++tile) {
                     const TileInfo ti = tile_info(i, p.W, l1_only);
                     const int qb = tile & 1;
@@ -783,10 +841,10 @@ __global__ void __launch_bounds__(kMainThreads, 1)
         // so the wait for the tile's last P V product overlaps useful work.
         struct Epi {
             bool valid, l2;
-            int t0, bh;
+            int t0, bh, T, row0;  // T, row0: the row's sequence (SeqView)
             float gate, pw_r1, l;
             uint32_t tile;
-        } pe = {false, false, 0, 0, 0.f, 0.f, 0.f, 0};
+        } pe = {false, false, 0, 0, 0, 0, 0.f, 0.f, 0.f, 0};
         auto epilogue = [&](const Epi &e) -> bool {
             // y = O / l + sigmoid(g) (m_intra + lam^(r+1) m_inter)
             xl[half * 128 + r] = e.l;
@@ -812,11 +870,12 @@ __global__ void __launch_bounds__(kMainThreads, 1)
             tc_fence_before();
             mbar_arrive(o_empty);
             const int t = e.t0 + r;
-            if (t < p.T) {
-                const size_t T_new = (size_t)(p.T - p.q_off);
+            if (t < e.T) {
+                // fixed length: [BH][T_new][64]; variable length: [total][H][64]
+                const size_t row = varlen ? ((size_t)(e.row0 + t) * p.H + e.bh % p.H)
+                                          : ((size_t)e.bh * (size_t)(p.T - p.q_off) + (t - p.q_off));
                 uint4 *dst = reinterpret_cast<uint4 *>(reinterpret_cast<__nv_bfloat16 *>(p.y) +
-                                                       ((size_t)e.bh * T_new + (t - p.q_off)) * HD +
-                                                       32 * half);
+                                                       row * HD + 32 * half);
 #pragma unroll
                 for (int c = 0; c < 4; ++c)
                     dst[c] = make_uint4(pack_bf16(yv[8 * c], yv[8 * c + 1]),
@@ -828,8 +887,9 @@ __global__ void __launch_bounds__(kMainThreads, 1)
         };
         for (int sp = blockIdx.x; sp < n_spans && ok; sp += gridDim.x) {
             const int bh = sp / p.n_s, h = bh % p.H;
+            const SeqView sv = seq_view(p.vl, bh, p.H, p.T, nullptr);
             int i0, i1;
-            span_range(sp % p.n_s, p.nT, p.n_s, p.q_off / BM, i0, i1);
+            span_range(sp % p.n_s, sv.nT, p.n_s, p.q_off / BM, i0, i1);
             const double lam = p.lam[h];
             const float gate = 1.0f / (1.0f + expf(-p.g[h]));
             const float pw_r1 = (float)pow(lam, (double)(r + 1));
@@ -900,7 +960,7 @@ __global__ void __launch_bounds__(kMainThreads, 1)
                     }
                 }
                 if (!ok) break;
-                pe = {true, ti.l2, ti.t0, bh, gate, pw_r1, l, tile};
+                pe = {true, ti.l2, ti.t0, bh, sv.T, sv.row0, gate, pw_r1, l, tile};
             }
         }
         if (ok && pe.valid) ok = epilogue(pe);
@@ -915,8 +975,11 @@ __global__ void __launch_bounds__(kMainThreads, 1)
         float S[64];
         for (int sp = blockIdx.x; sp < n_spans && ok; sp += gridDim.x) {
             const int bh = sp / p.n_s, h = bh % p.H, js = sp % p.n_s;
+            // the state warps report rows with inconsistent offsets (once per span)
+            const SeqView sv = seq_view(p.vl, bh, p.H, p.T, u == 0 ? p.status : nullptr);
+            const int E = sv.T > p.W ? sv.T - p.W : 0;
             int i0, i1;
-            span_range(js, p.nT, p.n_s, p.q_off / BM, i0, i1);
+            span_range(js, sv.nT, p.n_s, p.q_off / BM, i0, i1);
             const double lam = p.lam[h];
             const double l2l = log2(lam);
             // per-span tables (float math in the tile loop only): ew[k] = eta lam^k,
@@ -1059,6 +1122,22 @@ bool make_map(CUtensorMap *m, const void *base, int T, int BH) {
            CUDA_SUCCESS;
 }
 
+// Packed [total][H][64] bf16 (variable-length calls) -> 3D map over
+// (column, head, token) with 64 x 1 x 128 boxes: the same shared-memory tile
+// as make_map's, 128 token rows of one head; rows past total read as zero.
+bool make_map_packed(CUtensorMap *m, const void *base, int64_t total, int H) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[3] = {(cuuint64_t)HD, (cuuint64_t)H, (cuuint64_t)total};
+    cuuint64_t strides[2] = {(cuuint64_t)HD * 2, (cuuint64_t)H * HD * 2};
+    cuuint32_t box[3] = {HD, 1, BM};
+    cuuint32_t es[3] = {1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides,
+              box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+           CUDA_SUCCESS;
+}
+
 // Spans per head: minimise the work of the busiest CTA, counting each span as
 // its tiles plus a fixed start-up cost (pipeline fill, the pre-pass summary it
 // needs and the combine of its predecessors' summaries); ties go to fewer spans.
@@ -1131,10 +1210,20 @@ cudaError_t launch_prefill_sm100(const PrefillParams &p, int num_sms, cudaStream
     const int T_all = (int)(p.T + p.n_halo);  // combined sequence
     const int nT = (T_all + BM - 1) / BM;
     const int ns = choose_spans(BH, nT - q_off / BM, num_sms);
+    // variable length: B sequences of at most T tokens packed in [total][H][64],
+    // one row bh = (sequence, head) per B * H, spans cut over the longest
+    const bool varlen = p.cu_seqlens != nullptr;
+    const Varlen vl{p.cu_seqlens, (int)p.total, (int)p.T};
     CUtensorMap tq, tk, tv, tkh, tvh;
-    if (!make_map(&tq, p.q, (int)p.T, (int)BH) || !make_map(&tk, p.k, (int)p.T, (int)BH) ||
-        !make_map(&tv, p.v, (int)p.T, (int)BH))
+    if (varlen) {
+        if (!make_map_packed(&tq, p.q, p.total, (int)p.H) ||
+            !make_map_packed(&tk, p.k, p.total, (int)p.H) ||
+            !make_map_packed(&tv, p.v, p.total, (int)p.H))
+            return cudaErrorInvalidValue;
+    } else if (!make_map(&tq, p.q, (int)p.T, (int)BH) || !make_map(&tk, p.k, (int)p.T, (int)BH) ||
+               !make_map(&tv, p.v, (int)p.T, (int)BH)) {
         return cudaErrorInvalidValue;
+    }
     if (q_off > 0) {
         if (!make_map(&tkh, p.halo_k, q_off, (int)BH) || !make_map(&tvh, p.halo_v, q_off, (int)BH))
             return cudaErrorInvalidValue;
@@ -1152,19 +1241,19 @@ cudaError_t launch_prefill_sm100(const PrefillParams &p, int num_sms, cudaStream
     float *dA = reinterpret_cast<float *>(p.workspace);
     if (!p.l1_only && ns > 1) {
         SumParams sp{dA, p.lam, p.eta, T_all, (int)p.W, (int)p.H, (int)BH, nT, ns, n_parts, q_off,
-                     p.status, p.wait_ns};
+                     p.status, p.wait_ns, vl};
         span_summary_kernel<<<(unsigned)(BH * (ns - 1) * n_parts), 192, SMEM_SUM, s>>>(tk, tv, tkh,
                                                                                     tvh, sp);
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
-        PrefixParams pp{dA, p.lam, T_all, (int)p.W, (int)p.H, nT, ns, n_parts, q_off};
+        PrefixParams pp{dA, p.lam, T_all, (int)p.W, (int)p.H, nT, ns, n_parts, q_off, vl, p.status};
         span_prefix_kernel<<<dim3(HD * HD / 256, (unsigned)BH), 256, 0, s>>>(pp);
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
     MainParams mp{p.y,      p.A_final, p.lam, p.eta, p.g,  dA, p.A_init, T_all, (int)p.W, (int)p.H,
                   (int)BH, nT,        ns,    n_parts,         p.l1_only ? 1 : 0, q_off, p.status,
-                  p.wait_ns};
+                  p.wait_ns,  vl};
     const int64_t spans = BH * ns;
     const unsigned grid = (unsigned)(spans < num_sms ? spans : num_sms);
     prefill_main_kernel<<<grid, kMainThreads, SMEM_MAIN, s>>>(tq, tk, tv, tkh, tvh, mp);

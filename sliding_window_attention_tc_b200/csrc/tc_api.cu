@@ -105,6 +105,15 @@ size_t prefill_ws(const tc_prefill_desc &d, int64_t n_halo, int num_sms) {
                                 : tc::portable_workspace_bytes(d, n_halo);
 }
 
+// Variable-length calls run on the tensor-core path only (any longest
+// length, 0 included), without the state-only, delta-rule and chunk-mean
+// variants.
+bool varlen_supported(const tc_prefill_desc &d) {
+    tc_prefill_desc c = d;
+    if (c.T < 1) c.T = 1;
+    return use_sm100(c, 0) && !(d.flags & ~TC_PREFILL_L1_ONLY);
+}
+
 int sm_count_or_default() {
     int dev = 0, sms = 0;
     if (current_device(&dev, &sms) != TC_OK) return 148;
@@ -253,6 +262,76 @@ tc_status tc_prefill_from_state(const tc_prefill_desc *d, int64_t t0, const void
                                 void *workspace, size_t workspace_bytes, tc_stream_t stream) {
     return prefill_impl(d, t0, halo_k, halo_v, A_init, q, k, v, lambda, eta, g, y, A_final,
                         workspace, workspace_bytes, stream);
+}
+
+size_t tc_prefill_varlen_workspace_size(const tc_prefill_desc *d) {
+    if (check_desc(d) != TC_OK || !varlen_supported(*d)) return (size_t)-1;
+    return tc::sm100_workspace_bytes(*d, sm_count_or_default());
+}
+
+tc_status tc_prefill_varlen(const tc_prefill_desc *d, const int64_t *cu_seqlens, int64_t total,
+                            const void *q, const void *k, const void *v, const float *lambda,
+                            const float *eta, const float *g, void *y, float *A_final,
+                            void *workspace, size_t workspace_bytes, tc_stream_t stream) {
+    tc_status st = check_desc(d);
+    if (st != TC_OK) return st;
+    const bool l1_only = (d->flags & TC_PREFILL_L1_ONLY) != 0;
+    if (total < 0 || total > (int64_t(1) << 30) || !cu_seqlens ||
+        (reinterpret_cast<uintptr_t>(cu_seqlens) & 7u))
+        return TC_ERR_INVALID_ARG;
+    if ((total > 0 && (!q || !k || !v || !y)) || !lambda || !eta || !g || (!l1_only && !A_final))
+        return TC_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(y) ||
+        (A_final && !aligned16(A_final)) || (workspace && !aligned16(workspace)))
+        return TC_ERR_INVALID_ARG;
+    // the tensor-core path only: bf16, d = 64, W a multiple of 128, no state-only,
+    // delta-rule or chunk-mean variants
+    if (!varlen_supported(*d)) return TC_ERR_UNSUPPORTED;
+    if (d->H * total > (int64_t(1) << 31)) return TC_ERR_UNSUPPORTED;
+    int dev = 0, sms = 0;
+    st = current_device(&dev, &sms);
+    if (st != TC_OK) return st;
+    const size_t need = tc::sm100_workspace_bytes(*d, sms);
+    if (need > 0 && (!workspace || workspace_bytes < need)) return TC_ERR_WORKSPACE;
+    const void *ptrs[] = {q, k, v, y};
+    for (const void *x : ptrs)
+        if (total > 0 && !is_device_ptr(x, dev)) return TC_ERR_INVALID_ARG;
+    const void *hd[] = {lambda, eta, g, cu_seqlens};
+    for (const void *x : hd)
+        if (!is_device_ptr(x, dev)) return TC_ERR_INVALID_ARG;
+    if (A_final && !l1_only && !is_device_ptr(A_final, dev)) return TC_ERR_INVALID_ARG;
+    if (need > 0 && !is_device_ptr(workspace, dev)) return TC_ERR_INVALID_ARG;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (total == 0) {
+        // every sequence is empty: no tokens to read, A_final = 0
+        if (l1_only) return TC_OK;
+        const size_t na = (size_t)(d->B * d->H * d->dk * d->dv) * sizeof(float);
+        return cudaMemsetAsync(A_final, 0, na, s) == cudaSuccess ? TC_OK : TC_ERR_CUDA;
+    }
+    tc::PrefillParams p{};
+    p.q = q;
+    p.k = k;
+    p.v = v;
+    p.y = y;
+    p.A_final = l1_only ? nullptr : A_final;
+    p.lam = lambda;
+    p.eta = eta;
+    p.g = g;
+    p.B = d->B;
+    p.H = d->H;
+    p.T = d->T;
+    p.W = d->W;
+    p.C = d->C;
+    p.dk = (int)d->dk;
+    p.dv = (int)d->dv;
+    p.l1_only = l1_only;
+    p.workspace = workspace;
+    p.workspace_bytes = workspace_bytes;
+    p.status = status_ptr();
+    p.wait_ns = wait_limit_ns();
+    p.cu_seqlens = cu_seqlens;
+    p.total = total;
+    return tc::launch_prefill_sm100(p, sms, s) == cudaSuccess ? TC_OK : TC_ERR_CUDA;
 }
 
 size_t tc_backward_workspace_size(const tc_prefill_desc *d) {

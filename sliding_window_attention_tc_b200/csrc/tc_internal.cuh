@@ -97,6 +97,11 @@ struct PrefillParams {
     size_t workspace_bytes;
     int *status;
     unsigned long long wait_ns;  // limit of the tensor-core kernels' bounded waits
+    // variable-length calls (tc_prefill_varlen): B sequences packed along the
+    // token axis, sequence b = tokens cu_seqlens[b] .. cu_seqlens[b+1]-1 of
+    // [total][H][d] q, k, v, y; T is the longest length.  Null: fixed length.
+    const int64_t *cu_seqlens;
+    int64_t total;
 };
 
 // decode.cu

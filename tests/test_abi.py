@@ -134,3 +134,51 @@ def test_valid_decode_without_device_reports_no_device():
     assert st.t == 5  # the clock only advances on success
     n = tc.lib_handle().tc_decode_step_host_workspace_size(ctypes.byref(st))
     assert n == 4 * 2 * 2 * 64 * 2 + 0 or n >= 4 * 2 * 2 * 64 * 2
+
+
+def _call_varlen(desc, cu=FAKE, total=300, **ptrs):
+    p = dict(q=FAKE, k=FAKE, v=FAKE, lam=FAKE, eta=FAKE, g=FAKE, y=FAKE, A=FAKE, ws=FAKE)
+    p.update(ptrs)
+    return tc.lib_handle().tc_prefill_varlen(
+        ctypes.byref(desc) if desc is not None else None, cu, total, p["q"], p["k"], p["v"],
+        p["lam"], p["eta"], p["g"], p["y"], p["A"], p["ws"], 1 << 40, None)
+
+
+def _varlen_desc(**kw):
+    base = dict(B=3, H=2, T=200, dk=64, dv=64, W=128, C=64, dtype=tc.TC_BF16)
+    base.update(kw)
+    return _desc(**base)
+
+
+def test_varlen_rejects_invalid_arguments():
+    lib = tc.lib_handle()
+    assert _call_varlen(None) == 1
+    assert _call_varlen(_varlen_desc(), cu=None) == 1
+    assert _call_varlen(_varlen_desc(), cu=ctypes.c_void_p(0x10004)) == 1  # not 8-byte aligned
+    assert _call_varlen(_varlen_desc(), total=-1) == 1
+    assert _call_varlen(_varlen_desc(), total=(1 << 30) + 1) == 1
+    assert _call_varlen(_varlen_desc(), q=None) == 1
+    assert _call_varlen(_varlen_desc(), A=None) == 1
+    assert _call_varlen(_varlen_desc(), k=ctypes.c_void_p(0x10008)) == 1
+    # total = 0: the token tensors may be NULL (then only the device is missing)
+    st = _call_varlen(_varlen_desc(), total=0, q=None, k=None, v=None, y=None)
+    assert st in (0, 3)
+    assert lib.tc_prefill_varlen_workspace_size(None) == tc.SIZE_ERROR
+
+
+@pytest.mark.parametrize("kw", [dict(dtype=tc.TC_F32), dict(dk=32, dv=32), dict(W=100),
+                                dict(W=64), dict(flags=tc.TC_PREFILL_STATE_ONLY)])
+def test_varlen_outside_the_tensor_core_path_is_unsupported(kw):
+    flags = kw.pop("flags", 0)
+    d = _varlen_desc(**kw)
+    d.flags = flags
+    assert _call_varlen(d) == 2
+    assert tc.lib_handle().tc_prefill_varlen_workspace_size(ctypes.byref(d)) == tc.SIZE_ERROR
+
+
+@pytest.mark.skipif(HAS_GPU, reason="checks the no-device answer")
+def test_valid_varlen_without_device_reports_no_device():
+    assert _call_varlen(_varlen_desc()) == 3
+    d = _varlen_desc(l1_only=True)
+    assert _call_varlen(d, A=None) == 3
+    assert tc.lib_handle().tc_prefill_varlen_workspace_size(ctypes.byref(_varlen_desc())) >= 0

@@ -97,3 +97,21 @@ def test_valid_tensors_pass_the_checks():
     q, k, v, lam, eta, g = _layer()
     with pytest.raises(RuntimeError):
         tc.prefill(q, k, v, lam, eta, g, W, 8)
+
+
+def test_prefill_varlen_checks_the_packed_layout():
+    total = 50
+    q, k, v = (torch.randn(total, H, 64).to(torch.bfloat16) for _ in range(3))
+    lam, eta, g = torch.full((H,), 0.9), torch.full((H,), 0.5), torch.zeros(H)
+    cu = torch.tensor([0, 20, 50], dtype=torch.int64)
+    with pytest.raises(TypeError):  # offsets must be int64
+        tc.prefill_varlen(q, k, v, cu.int(), 30, lam, eta, g, 128, 64)
+    with pytest.raises(ValueError):  # q one token short
+        tc.prefill_varlen(q[1:], k, v, cu, 30, lam, eta, g, 128, 64)
+    with pytest.raises(TypeError):  # v in another dtype
+        tc.prefill_varlen(q, k, v.float(), cu, 30, lam, eta, g, 128, 64)
+    with pytest.raises(ValueError):  # A_final for the wrong number of sequences
+        tc.prefill_varlen(q, k, v, cu, 30, lam, eta, g, 128, 64,
+                          A_final=torch.empty(3, H, 64, 64))
+    with pytest.raises(ValueError):  # no sequence at all
+        tc.prefill_varlen(q, k, v, cu[:1], 30, lam, eta, g, 128, 64)

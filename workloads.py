@@ -34,6 +34,11 @@ PREFILL_CONFIGS = {
     "long_prefill_bf16": dict(B=1, H=16, T=32768, dk=64, dv=64, W=1024, C=128, dtype="bf16",
                               seed=1004),
 }
+# variable-length prefill: the LM workload's 32768 tokens per head cut into
+# 15 sequences of mixed lengths (shorter than W, ragged, and much longer)
+VARLEN_CONFIG = dict(lengths=[8192, 6000, 4096, 3000, 2500, 2048, 1777, 1500, 1200, 1000, 700,
+                              400, 200, 100, 55],
+                     H=12, dk=64, dv=64, W=512, C=64, dtype="bf16", seed=1006)
 DECODE_CONFIG = dict(B=256, H=32, dk=128, dv=128, W=2048, steps=512, history=10240,
                      prewarm_evictions=8192, dtype="bf16", seed=1005)
 
@@ -145,6 +150,56 @@ def random_prefill(B, H, T, dk, dv, W, C, *, dtype="f32", seed=0, scale=None,
     return PrefillInputs(q.to(dt).contiguous(), k.to(dt).contiguous(), v.to(dt).contiguous(),
                          lam.float(), eta.float(), g.float(), W, C,
                          {"name": "random", "seed": seed, "dtype": dtype})
+
+
+@dataclass
+class VarlenInputs:
+    q: torch.Tensor  # [total, H, dk], sequences packed token-major
+    k: torch.Tensor
+    v: torch.Tensor  # [total, H, dv]
+    cu_seqlens: torch.Tensor  # int64 [n_seq + 1]
+    lam: torch.Tensor  # [H] float32, shared by every sequence
+    eta: torch.Tensor
+    g: torch.Tensor
+    W: int
+    C: int
+
+    @property
+    def max_seqlen(self) -> int:
+        return int((self.cu_seqlens[1:] - self.cu_seqlens[:-1]).max()) if len(self.cu_seqlens) > 1 else 0
+
+    def sequence(self, b: int):
+        """q, k, v of sequence b as [1, H, T_b, d] (the fixed-length layout)."""
+        a, e = int(self.cu_seqlens[b]), int(self.cu_seqlens[b + 1])
+        return tuple(t[a:e].permute(1, 0, 2).unsqueeze(0).contiguous()
+                     for t in (self.q, self.k, self.v))
+
+
+def random_varlen(lengths, H, dk, dv, W, C, *, dtype="bf16", seed=0, scale=None,
+                  lam_range=(0.9, 0.999), eta_range=(0.1, 1.0)) -> VarlenInputs:
+    """Seeded packed inputs: sequences of the given lengths, one after the
+    other along the token axis, with the same per-head parameters."""
+    gen = _gen(seed)
+    s = scale if scale is not None else 1.0 / math.sqrt(dk)
+    total = int(sum(lengths))
+    q = torch.randn(total, H, dk, generator=gen, dtype=torch.float64) * s
+    k = torch.randn(total, H, dk, generator=gen, dtype=torch.float64) * s
+    v = torch.randn(total, H, dv, generator=gen, dtype=torch.float64) * s
+    lam = _uniform(gen, H, *lam_range)
+    eta = _uniform(gen, H, *eta_range)
+    g = torch.randn(H, generator=gen, dtype=torch.float64)
+    cu = torch.zeros(len(lengths) + 1, dtype=torch.int64)
+    cu[1:] = torch.cumsum(torch.tensor(lengths, dtype=torch.int64), 0)
+    dt = _TDTYPE[dtype]
+    return VarlenInputs(q.to(dt).contiguous(), k.to(dt).contiguous(), v.to(dt).contiguous(), cu,
+                        lam.float(), eta.float(), g.float(), W, C)
+
+
+def varlen_config() -> "VarlenInputs":
+    """Inputs of the variable-length prefill workload (CPU tensors)."""
+    c = VARLEN_CONFIG
+    return random_varlen(c["lengths"], c["H"], c["dk"], c["dv"], c["W"], c["C"],
+                         dtype=c["dtype"], seed=c["seed"])
 
 
 @dataclass
