@@ -193,19 +193,29 @@ __device__ __forceinline__ void load_kv_tile(uint8_t *dst, const CUtensorMap *tk
     }
 }
 
-__device__ __forceinline__ void named_bar(int id, int n) {
-    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+// Named barrier over n threads that also ORs pred over them; returns true if
+// any passed true.  A hardware barrier has no time limit, so a role group
+// that syncs with it follows one rule: a bounded wait that gives up only sets
+// a flag, the thread still reaches the group's next barrier with it, and all
+// threads leave their loops together right after a barrier that reported
+// one.  Every thread of the group then passes the same sequence of barriers.
+// (Per query key tile it costs a few tens of cycles, against a few hundred
+// for an mbarrier that 256 threads arrive on and poll.)
+__device__ __forceinline__ bool bar_any(int id, int n, bool pred) {
+    uint32_t res;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 q, %1, 0;\n\t"
+        "bar.red.or.pred p, %2, %3, q;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(res)
+        : "r"((uint32_t)pred), "r"(id), "r"(n)
+        : "memory");
+    return res != 0;
 }
 
-// Barrier for one 128-thread role group on an mbarrier (count 128): unlike
-// bar.sync it gives up with the bounded wait, so an aborting thread cannot
-// leave the rest of its group blocked.
-__device__ __forceinline__ bool group_sync(uint64_t *bar, uint32_t &phase, volatile int *abort,
-                                           int *status, uint64_t limit = kWaitTimeoutNs) {
-    mbar_arrive(bar);
-    const bool ok = __all_sync(0xffffffffu, mbar_wait(bar, phase & 1, abort, status, limit));
-    ++phase;
-    return ok;
+__device__ __forceinline__ void named_bar(int id, int n) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
 }
 
 // mbar_wait with one answer for the whole warp, so that warps which go on to
@@ -642,8 +652,7 @@ __global__ void __launch_bounds__(kMainThreads, 1)
     uint64_t *o_prog = p_full + 2, *o_full = o_prog + 1, *o_empty = o_full + 1;
     uint64_t *sst_full = o_empty + 1, *kt_full = sst_full + 1, *ds_full = kt_full + 1;
     uint64_t *lead_ready = ds_full + 1, *mma_done = lead_ready + 1;
-    uint64_t *sm_sync = mma_done + 1, *st_sync = sm_sync + 1;  // group barriers (256, 128)
-    uint32_t *tmem_base = reinterpret_cast<uint32_t *>(st_sync + 1);
+    uint32_t *tmem_base = reinterpret_cast<uint32_t *>(mma_done + 1);
     volatile int *abort = reinterpret_cast<volatile int *>(tmem_base + 1);
     float *epw = reinterpret_cast<float *>(sm + OFF_EPW);
     float *sDS = reinterpret_cast<float *>(sm + OFF_DS);
@@ -672,8 +681,6 @@ __global__ void __launch_bounds__(kMainThreads, 1)
         mbar_init(ds_full, 1);
         mbar_init(lead_ready, 1);
         mbar_init(mma_done, 1);
-        mbar_init(sm_sync, 256);
-        mbar_init(st_sync, 128);
         *abort = 0;
         fence_mbar_init();
     }
@@ -835,7 +842,7 @@ __global__ void __launch_bounds__(kMainThreads, 1)
         const float sl2 = kLog2e * rsqrtf((float)HD);
         float *xm = reinterpret_cast<float *>(sm + OFF_XM);
         float *xl = reinterpret_cast<float *>(sm + OFF_XL);
-        uint32_t tile = 0, kc = 0, sync_phase = 0;
+        uint32_t tile = 0, kc = 0;
         bool ok = true;
         // The epilogue of a tile runs after the first key tile of the next one,
         // so the wait for the tile's last P V product overlaps useful work.
@@ -845,12 +852,22 @@ __global__ void __launch_bounds__(kMainThreads, 1)
             float gate, pw_r1, l;
             uint32_t tile;
         } pe = {false, false, 0, 0, 0, 0, 0.f, 0.f, 0.f, 0};
-        auto epilogue = [&](const Epi &e) -> bool {
+        // A bounded wait that gives up sets `failed`; the thread carries on to
+        // the next softmax barrier, which tells every softmax thread, and all
+        // 256 leave their loops right after that barrier.  So every one of them
+        // passes the same sequence of barriers.
+        bool failed = false;
+        auto epilogue = [&](const Epi &e) -> bool {  // false: all softmax threads stop
             // y = O / l + sigmoid(g) (m_intra + lam^(r+1) m_inter)
+            // (between two epilogues every thread passes a key-tile barrier, so
+            // one xl buffer suffices)
             xl[half * 128 + r] = e.l;
-            if (!group_sync(sm_sync, sync_phase, abort, p.status, p.wait_ns)) return false;
+            if (bar_any(1, 256, failed)) return false;
             const float inv_l = 1.0f / (e.l + xl[(1 - half) * 128 + r]);
-            if (!warp_wait(o_full, e.tile & 1, abort, p.status, p.wait_ns)) return false;
+            if (!warp_wait(o_full, e.tile & 1, abort, p.status, p.wait_ns)) {
+                failed = true;
+                return true;
+            }
             tc_fence_after();
             float yv[32];
             uint32_t rr[32];
@@ -894,18 +911,25 @@ __global__ void __launch_bounds__(kMainThreads, 1)
             const float gate = 1.0f / (1.0f + expf(-p.g[h]));
             const float pw_r1 = (float)pow(lam, (double)(r + 1));
             // previous span done with epw, then publish this head's table
-            if (!(ok = group_sync(sm_sync, sync_phase, abort, p.status, p.wait_ns))) break;
+            if (bar_any(1, 256, failed)) {
+                ok = false;
+                break;
+            }
             if (half == 0)
                 epw[128 + r] = (float)((double)p.eta[h] * pow(lam, (double)r));
             else
                 epw[r] = 0.f;
-            if (!(ok = group_sync(sm_sync, sync_phase, abort, p.status, p.wait_ns))) break;
+            if (bar_any(1, 256, failed)) {
+                ok = false;
+                break;
+            }
             for (int i = i0; i < i1 && ok; ++i, ++tile) {
                 const TileInfo ti = tile_info(i, p.W, l1_only);
                 float m_used = -INFINITY, l = 0.f;
                 for (int j = 0; j < ti.nk && ok; ++j, ++kc) {
                     const int sb = kc & 1;
-                    if (!(ok = warp_wait(&s_full[sb], (kc >> 1) & 1, abort, p.status, p.wait_ns))) break;
+                    // (on a timeout the scores read below are stale, and unused)
+                    if (!warp_wait(&s_full[sb], (kc >> 1) & 1, abort, p.status, p.wait_ns)) failed = true;
                     tc_fence_after();
                     const uint32_t s_col = TM_S + sb * 128;
                     float s[64];
@@ -926,7 +950,10 @@ __global__ void __launch_bounds__(kMainThreads, 1)
                     const float mh = half_max(skind, s, r - 64 * half);
                     float *xmk = xm + (kc & 1) * 256;
                     xmk[half * 128 + r] = mh;
-                    if (!(ok = group_sync(sm_sync, sync_phase, abort, p.status, p.wait_ns))) break;
+                    if (bar_any(1, 256, failed)) {
+                        ok = false;
+                        break;
+                    }
                     const float mt = fmaxf(mh, xmk[(1 - half) * 128 + r]) * sl2;  // sl2 > 0
                     // Raise the row's reference max only when it grew by more than
                     // 2^kRescale; rows whose O already holds earlier P V products
@@ -936,40 +963,49 @@ __global__ void __launch_bounds__(kMainThreads, 1)
                     const bool resc = raise && m_used != -INFINITY && j > 0;
                     const float fo = resc ? ex2(m_used - mt) : 1.0f;
                     if (__any_sync(0xffffffffu, resc)) {
-                        if (!(ok = warp_wait(o_prog, (kc - 1) & 1, abort, p.status, p.wait_ns))) break;
-                        tc_fence_after();
-                        uint32_t rr[32];
-                        tmem_ld32(tmem_addr(tb, lane_base, TM_O + 32 * half), rr);
-                        tmem_wait_ld();
+                        if (warp_wait(o_prog, (kc - 1) & 1, abort, p.status, p.wait_ns)) {
+                            tc_fence_after();
+                            uint32_t rr[32];
+                            tmem_ld32(tmem_addr(tb, lane_base, TM_O + 32 * half), rr);
+                            tmem_wait_ld();
 #pragma unroll
-                        for (int c = 0; c < 32; ++c)
-                            rr[c] = __float_as_uint(__uint_as_float(rr[c]) * fo);
-                        tmem_st32(tmem_addr(tb, lane_base, TM_O + 32 * half), rr);
+                            for (int c = 0; c < 32; ++c)
+                                rr[c] = __float_as_uint(__uint_as_float(rr[c]) * fo);
+                            tmem_st32(tmem_addr(tb, lane_base, TM_O + 32 * half), rr);
+                        } else {
+                            failed = true;  // skip the P work, still reach every barrier
+                        }
                     }
-                    l *= fo;
-                    if (raise) m_used = mt;
-                    const uint32_t p_addr = tmem_addr(tb, lane_base, s_col + 32 * half);
-                    l += half_p(skind, s, r - 64 * half, sl2, m_used, p_addr);
-                    if (kind == KIND_LEAD_L2) write_plin(s, r - 64 * half, epw, p_addr + 64);
-                    tmem_wait_st();
-                    tc_fence_before();
-                    mbar_arrive(&p_full[sb]);
+                    if (!failed) {
+                        l *= fo;
+                        if (raise) m_used = mt;
+                        const uint32_t p_addr = tmem_addr(tb, lane_base, s_col + 32 * half);
+                        l += half_p(skind, s, r - 64 * half, sl2, m_used, p_addr);
+                        if (kind == KIND_LEAD_L2) write_plin(s, r - 64 * half, epw, p_addr + 64);
+                        tmem_wait_st();
+                        tc_fence_before();
+                        mbar_arrive(&p_full[sb]);
+                    }
                     if (j == 0 && pe.valid) {
-                        if (!(ok = epilogue(pe))) break;
                         pe.valid = false;
+                        if (!(ok = epilogue(pe))) break;
                     }
                 }
                 if (!ok) break;
                 pe = {true, ti.l2, ti.t0, bh, sv.T, sv.row0, gate, pw_r1, l, tile};
             }
         }
-        if (ok && pe.valid) ok = epilogue(pe);
+        if (pe.valid) epilogue(pe);  // every softmax thread: pe.valid is the same for all
 
     } else if (warp >= 12) {
         // ------------------------------------------------------------ state
         const int u = tid - 384;  // TMEM lane; u < 64 owns row u of S
-        uint32_t kc = 0, lc = 0, sync_phase = 0;
+        uint32_t kc = 0, lc = 0;
         bool ok = true;
+        // as in the softmax warps: a wait that gives up sets `failed`, the next
+        // state barrier (named barrier 2, 128 threads) tells all, and all leave
+        // right after it
+        bool failed = false;
         uint8_t *sb_tile = sm + OFF_SB;
         uint8_t *kt_hi = sm + OFF_KT, *kt_lo = sm + OFF_KT + TILE_B;
         float S[64];
@@ -988,7 +1024,10 @@ __global__ void __launch_bounds__(kMainThreads, 1)
             ew[u] = (float)((double)p.eta[h] * exp2((double)u * l2l));
             lp[u] = (float)exp2((double)u * l2l);
             if (u == 0) lp[128] = (float)exp2(128.0 * l2l);
-            if (!(ok = group_sync(st_sync, sync_phase, abort, p.status, p.wait_ns))) break;
+            if (bar_any(2, 128, failed)) {
+                ok = false;
+                break;
+            }
             // state at the span start from the predecessors' summaries
             const int n_start = max(0, i0 * BM - p.W);
 #pragma unroll
@@ -1009,13 +1048,13 @@ __global__ void __launch_bounds__(kMainThreads, 1)
             }
             bool have_prev = false;
             int c_prev = 0;
-            auto consume = [&](int c_eff) -> bool {
+            auto consume = [&](int c_eff) -> bool {  // false: all state threads stop
                 // rows 64..127 of the increment (lo parts) go through shared
                 // memory to the owners of rows 0..63 (hi parts)
-                if (!warp_wait(ds_full, (lc - 1) & 1, abort, p.status, p.wait_ns)) return false;
+                if (!warp_wait(ds_full, (lc - 1) & 1, abort, p.status, p.wait_ns)) failed = true;
                 tc_fence_after();
                 uint32_t rr[32];
-                if (u >= 64) {
+                if (u >= 64 && !failed) {
 #pragma unroll
                     for (int c0 = 0; c0 < 64; c0 += 32) {
                         tmem_ld32(tmem_addr(tb, 32 * (warp & 3), TM_DS + c0), rr);
@@ -1024,7 +1063,7 @@ __global__ void __launch_bounds__(kMainThreads, 1)
                         for (int c = 0; c < 32; ++c) sDS[(c0 + c) * 64 + (u - 64)] = __uint_as_float(rr[c]);
                     }
                 }
-                if (!group_sync(st_sync, sync_phase, abort, p.status, p.wait_ns)) return false;
+                if (bar_any(2, 128, failed)) return false;
                 if (u < 64) {
                     const float dec = lp[c_eff];
 #pragma unroll
@@ -1037,7 +1076,7 @@ __global__ void __launch_bounds__(kMainThreads, 1)
                                              __uint_as_float(rr[c]) + sDS[(c0 + c) * 64 + u]);
                     }
                 }
-                return group_sync(st_sync, sync_phase, abort, p.status, p.wait_ns);
+                return !bar_any(2, 128, false);
             };
             for (int i = i0; i < i1 && ok; ++i) {
                 const TileInfo ti = tile_info(i, p.W, l1_only);
@@ -1057,13 +1096,15 @@ __global__ void __launch_bounds__(kMainThreads, 1)
                     mbar_arrive(sst_full);
                     // scaled keys of the leading tile for the state MMA
                     const int s = kc % NS;
-                    if (!(ok = warp_wait(lead_ready, lc & 1, abort, p.status, p.wait_ns))) break;
+                    if (!warp_wait(lead_ready, lc & 1, abort, p.status, p.wait_ns)) failed = true;
                     const int n0 = ti.t0 - p.W;
                     const int c_eff = min(BM, E - n0);
-                    const float w = u < c_eff ? ew[c_eff - 1 - u] : 0.f;
-                    build_scaled_key_row(sm + OFF_KV + s * 2 * TILE_B, kt_hi, kt_lo, u, w);
-                    fence_async_smem();
-                    mbar_arrive(kt_full);
+                    if (!failed) {
+                        const float w = u < c_eff ? ew[c_eff - 1 - u] : 0.f;
+                        build_scaled_key_row(sm + OFF_KV + s * 2 * TILE_B, kt_hi, kt_lo, u, w);
+                        fence_async_smem();
+                        mbar_arrive(kt_full);
+                    }
                     have_prev = true;
                     c_prev = c_eff;
                     ++lc;
