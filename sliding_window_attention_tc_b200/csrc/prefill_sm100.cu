@@ -29,7 +29,10 @@
 // provide it: span_summary_kernel computes, in parts spread over CTAs, the
 // state dA_u that the evictions of span u add (decayed to the span's end),
 // and span_prefix_kernel folds the parts and the predecessors into one start
-// state per span.
+// state per span.  The prefix and main kernels are launched as programmatic
+// dependents of the kernel before them: each may start as its predecessor's
+// CTAs finish, and waits for the predecessor's results (griddep_wait) only
+// where it reads them.
 //
 // Roles in the main kernel (512 threads):
 //   warp 0        TMA producer: Q tile, then K/V tiles through an NS-stage ring
@@ -435,6 +438,7 @@ __device__ __forceinline__ void build_scaled_key_row(const uint8_t *ktile, uint8
 // has read that element already).
 // ============================================================================
 __global__ void __launch_bounds__(256) span_prefix_kernel(PrefixParams p) {
+    griddep_launch_dependents();
     // decay coefficients per span, once per block: c1 for the previous start
     // state, c2 for the previous span's summary (lam^0 = 1 also for lam = 0)
     __shared__ float c1s[kMaxSpans], c2s[kMaxSpans];
@@ -463,6 +467,7 @@ __global__ void __launch_bounds__(256) span_prefix_kernel(PrefixParams p) {
     __syncthreads();
     const int x = blockIdx.x * blockDim.x + threadIdx.x;  // element of the 64 x 64 state
     if (x >= HD * HD) return;
+    griddep_wait();  // the span summaries
     float acc = 0.f;
 #pragma unroll 4
     for (int js = 1; js < p.n_s; ++js) {
@@ -502,6 +507,7 @@ __global__ void __launch_bounds__(192, 2)
     volatile int *abort = reinterpret_cast<volatile int *>(tmem_base + 1);
     float *sDS = reinterpret_cast<float *>(sm + SOFF_DS);
 
+    griddep_launch_dependents();
     const int tid = threadIdx.x, warp = tid >> 5;
     const int per_head = p.n_s - 1;
     const int slot = blockIdx.x;  // (bh, js, part)
@@ -1041,6 +1047,7 @@ __global__ void __launch_bounds__(kMainThreads, 1)
             }
             if (!l1_only && u < 64 && js > 0) {
                 // the predecessors' evictions, from span_prefix_kernel
+                griddep_wait();
                 const float *src =
                     p.S_pre + (((size_t)(bh * (p.n_s - 1) + js - 1) * p.n_parts) * HD + u) * HD;
 #pragma unroll
@@ -1280,7 +1287,16 @@ cudaError_t launch_prefill_sm100(const PrefillParams &p, int num_sms, cudaStream
     if (e != cudaSuccess) return e;
     const int n_parts = ns > 1 ? parts_for(nT - q_off / BM, ns, BH, num_sms) : 1;
     float *dA = reinterpret_cast<float *>(p.workspace);
-    if (!p.l1_only && ns > 1) {
+    // The summary kernel waits for all earlier work of the stream, as usual.
+    // The prefix and main kernels after it may start early (programmatic
+    // stream serialization); they read their predecessor's results only
+    // after griddep_wait, and everything else they read was complete before
+    // the summary kernel started.
+    cudaLaunchAttribute early[1];
+    early[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    early[0].val.programmaticStreamSerializationAllowed = 1;
+    const bool summaries = !p.l1_only && ns > 1;
+    if (summaries) {
         SumParams sp{dA, p.lam, p.eta, T_all, (int)p.W, (int)p.H, (int)BH, nT, ns, n_parts, q_off,
                      p.status, p.wait_ns, vl};
         span_summary_kernel<<<(unsigned)(BH * (ns - 1) * n_parts), 192, SMEM_SUM, s>>>(tk, tv, tkh,
@@ -1288,17 +1304,27 @@ cudaError_t launch_prefill_sm100(const PrefillParams &p, int num_sms, cudaStream
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
         PrefixParams pp{dA, p.lam, T_all, (int)p.W, (int)p.H, nT, ns, n_parts, q_off, vl, p.status};
-        span_prefix_kernel<<<dim3(HD * HD / 256, (unsigned)BH), 256, 0, s>>>(pp);
-        e = cudaGetLastError();
+        cudaLaunchConfig_t pc = {};
+        pc.gridDim = dim3(HD * HD / 256, (unsigned)BH);
+        pc.blockDim = dim3(256);
+        pc.stream = s;
+        pc.attrs = early;
+        pc.numAttrs = 1;
+        e = cudaLaunchKernelEx(&pc, span_prefix_kernel, pp);
         if (e != cudaSuccess) return e;
     }
     MainParams mp{p.y,      p.A_final, p.lam, p.eta, p.g,  dA, p.A_init, T_all, (int)p.W, (int)p.H,
                   (int)BH, nT,        ns,    n_parts,         p.l1_only ? 1 : 0, q_off, p.status,
                   p.wait_ns,  vl};
     const int64_t spans = BH * ns;
-    const unsigned grid = (unsigned)(spans < num_sms ? spans : num_sms);
-    prefill_main_kernel<<<grid, kMainThreads, SMEM_MAIN, s>>>(tq, tk, tv, tkh, tvh, mp);
-    return cudaGetLastError();
+    cudaLaunchConfig_t mc = {};
+    mc.gridDim = dim3((unsigned)(spans < num_sms ? spans : num_sms));
+    mc.blockDim = dim3(kMainThreads);
+    mc.dynamicSmemBytes = SMEM_MAIN;
+    mc.stream = s;
+    mc.attrs = early;
+    mc.numAttrs = summaries ? 1 : 0;
+    return cudaLaunchKernelEx(&mc, prefill_main_kernel, tq, tk, tv, tkh, tvh, mp);
 }
 
 }  // namespace tc

@@ -173,6 +173,17 @@ __device__ __forceinline__ void fence_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// ---- programmatic dependent launch ---------------------------------------
+// A kernel launched with programmatic stream serialization may start before
+// the previous kernel in the stream has finished; griddep_wait blocks the
+// calling thread until that kernel has completed and its memory writes are
+// visible.  griddep_launch_dependents lets the dependent kernel start once
+// every CTA of this one has issued it (or exited).
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---- TMEM -------------------------------------------------------------------
 __device__ __forceinline__ void tmem_alloc(uint32_t *dst, uint32_t ncols) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
