@@ -358,6 +358,17 @@ def time_prefill_e2e(tc, name, dev, steps):
     return {"ms_per_step": ms, "tokens_per_s": B * H * T / (ms * 1e-3), "h2d": h2d, "d2h": d2h}
 
 
+def state_size_ratio(T, W, d):
+    """Per-head decode state of the layer (a W-slot bf16 ring of keys and
+    values plus the d x d float32 A) against a full bf16 KV cache of T tokens:
+    elements (W*2d + d^2) / (T*2d), and bytes.  Context only: the pages'
+    2.4x figure is a whole-model peak-memory measurement."""
+    elems = (W * 2 * d + d * d) / (T * 2 * d)
+    nbytes = (W * 2 * d * 2 + d * d * 4) / (T * 2 * d * 2)
+    return {"T": T, "W": W, "d": d, "elements_ratio": elems, "bytes_ratio": nbytes,
+            "full_kv_over_state_bytes": 1.0 / nbytes}
+
+
 def time_calls(fn, steps, warmup):
     """Per-call device times (ms) of fn() on the current stream, CUDA events."""
     stream = torch.cuda.current_stream()
@@ -644,7 +655,8 @@ def main():
                 "frac_of_bf16_peak": (f1 + f2) / (t_lp * 1e-3) / 1e12 / peak_tf,
                 "l1_only_ms": t_lp1, "l2_overhead_ratio": t_lp / t_lp1 - 1.0,
                 "algorithmic_floor": f2 / f1,
-                "executed_tflops": sum(prefill_executed_flops(Bl, Hl, Tl, xl.W)) / (t_lp * 1e-3) / 1e12}
+                "executed_tflops": sum(prefill_executed_flops(Bl, Hl, Tl, xl.W)) / (t_lp * 1e-3) / 1e12,
+                "state_size": state_size_ratio(Tl, xl.W, dl)}
             del lp, lp1
             dec = time_decode(tc, dev, world, clocks=clocks)
             dms = statistics.mean(dec["per_step_ms"])

@@ -20,11 +20,17 @@
 //   step t (eviction e = t - W) gives dk_e += eta G_t v_e,
 //   dv_e += eta G_t^T k_e, deta += <G_t, k_e v_e^T>, dlam += <G_t, A_{t-1}>;
 //   also dq_t += A_t (s dy_t) and dg += s (1 - s) <dy_t, q_t A_t>.
-//   bwd_l2_kernel (CTAs of 8 rows of A per (b,h)) replays A from
-//   checkpoints every kCk tokens and walks the tokens backwards; it adds to
-//   dq, dk, dv and leaves partials of dlam, deta, dg, which
-//   bwd_reduce_kernel sums over the batch and the row blocks in a fixed order.
+//   bwd_l2_kernel (CTAs of 8 rows of A per (b,h), one thread-block cluster
+//   per (b,h)) replays A from checkpoints every kCk tokens and walks the
+//   tokens backwards; it adds to dq, dk, dv and leaves partials of dlam,
+//   deta, dg, which bwd_reduce_kernel sums over the batch and the row blocks
+//   in a fixed order.  dv_e sums over all rows of G: each CTA keeps its rows'
+//   part for a segment's evictions in shared memory, and the cluster adds
+//   the parts rank by rank through distributed shared memory.  No step
+//   depends on the order in which CTAs run, so the gradients are the same
+//   bit for bit on every run.
 
+#include <cooperative_groups.h>
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -386,7 +392,8 @@ __host__ __forceinline__ size_t keys_smem(int dk, int dv) {
 // kRows rows (one row per warp; lane l owns columns l, l+32, ...).  A is
 // replayed from checkpoints every kCk tokens; a segment's q, dy, k, v are
 // staged in shared memory once.  dv_e sums over all rows: the CTAs of a head
-// add their parts with atomics.
+// are one cluster, and after each segment every CTA adds one slice of the
+// segment's evictions over the cluster's parts, rank by rank.
 template <typename Tin>
 __global__ void __launch_bounds__(kThreads) bwd_l2_kernel(BwdParams p) {
     constexpr int CPL = kMaxD / 32;
@@ -400,9 +407,13 @@ __global__ void __launch_bounds__(kThreads) bwd_l2_kernel(BwdParams p) {
     const int64_t T = p.T, W = p.W;
     const float lam = p.lam[h], eta = p.eta[h];
     const float sg = 1.f / (1.f + expf(-p.g[h]));
-    // shared: q rows [kCk][kRows], k rows [kCk][kRows], dy [kCk][dv], v [kCk][dv], column sums [kRows][dv]
+    // shared: q rows [kCk][kRows], k rows [kCk][kRows], dy [kCk][dv], v [kCk][dv], column sums
+    // [kRows][dv], this CTA's part of dv for the segment's evictions [kCk][dv]
     float *sQ = sh, *sK = sQ + kCk * kRows, *sDY = sK + kCk * kRows, *sV = sDY + kCk * dv;
     float *scol = sV + kCk * dv;
+    float *sDV = scol + kRows * dv;
+    namespace cg = cooperative_groups;
+    cg::cluster_group cluster = cg::this_cluster();
     const Tin *qb = reinterpret_cast<const Tin *>(p.q) + bh * T * dk;
     const Tin *kb = reinterpret_cast<const Tin *>(p.k) + bh * T * dk;
     const Tin *vb = reinterpret_cast<const Tin *>(p.v) + bh * T * dv;
@@ -509,13 +520,27 @@ __global__ void __launch_bounds__(kThreads) bwd_l2_kernel(BwdParams p) {
                 for (int c = tid; c < dv; c += kThreads) {
                     float sum = 0.f;
                     for (int w = 0; w < kRows; ++w) sum += scol[w * dv + c];
-                    atomicAdd(&p.gv[(bh * T + e) * dv + c], eta * sum);
+                    sDV[i * dv + c] = sum;
                 }
                 __syncthreads();
 #pragma unroll
                 for (int jx = 0; jx < CPL; ++jx) G[jx] *= lam;
             }
         }
+        // dv of the segment's evictions e = t - W (t in [max(tb, W), te)): the
+        // parts of all row blocks, added in rank order; CTA x of the cluster
+        // takes every nrs-th eviction starting at x
+        cluster.sync();
+        const int64_t t_first = tb > W ? tb : W;
+        for (int64_t t = t_first + blockIdx.x; t < te; t += nrs) {
+            const int i = (int)(t - tb);
+            for (int c = tid; c < dv; c += kThreads) {
+                float sum = 0.f;
+                for (int q = 0; q < nrs; ++q) sum += cluster.map_shared_rank(sDV, q)[i * dv + c];
+                p.gv[(bh * T + (t - W)) * dv + c] += eta * sum;
+            }
+        }
+        cluster.sync();  // the parts are read before the next segment overwrites them
     }
     // partials of this CTA: pl differs per lane; pe and pg are equal in all
     // lanes of a warp (only lane 0's count); rows past dk hold zeros
@@ -597,13 +622,30 @@ cudaError_t launch_t(const BwdParams &p, cudaStream_t s) {
                                                           : launch_window<Tin, kMaxD / 32>(p, s);
         if (e != cudaSuccess) return e;
     }
-    const int nrs = (p.dk + kRows - 1) / kRows;
-    const size_t smem = (size_t)(2 * kCk * kRows + 2 * kCk * p.dv + kRows * p.dv) * sizeof(float);
+    const int nrs = (p.dk + kRows - 1) / kRows;  // row blocks = CTAs of one cluster (<= 16)
+    const size_t smem =
+        (size_t)(2 * kCk * kRows + 2 * kCk * p.dv + kRows * p.dv + kCk * p.dv) * sizeof(float);
     cudaError_t e = cudaFuncSetAttribute(bwd_l2_kernel<Tin>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    bwd_l2_kernel<Tin><<<dim3((unsigned)nrs, (unsigned)BH), kThreads, smem, s>>>(p);
-    e = cudaGetLastError();
+    if (nrs > 8) {
+        e = cudaFuncSetAttribute(bwd_l2_kernel<Tin>,
+                                 cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+        if (e != cudaSuccess) return e;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)nrs, (unsigned)BH);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)nrs;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, bwd_l2_kernel<Tin>, p);
     if (e != cudaSuccess) return e;
     bwd_reduce_kernel<<<(unsigned)((p.H + 127) / 128), 128, 0, s>>>(p, nrs);
     return cudaGetLastError();

@@ -26,6 +26,8 @@ CASES = [
     (1, 1, 100, 16, 8, 5, "f32"),       # d_k != d_v
     (1, 2, 40, 16, 16, 64, "f32"),      # T < W: no eviction, L2 gradients of lambda, eta are 0
     (1, 2, 300, 64, 64, 128, "bf16"),   # checkpoints in several segments
+    (1, 2, 200, 128, 128, 64, "bf16"),  # d = 128: 16 row blocks per head in one cluster
+    (1, 1, 150, 128, 40, 16, "f32"),    # d_k = 128, d_v not a multiple of 32
 ]
 
 
@@ -47,3 +49,21 @@ def test_backward_matches_oracle(cuda_device, case):
             assert float(a.abs().max()) <= 1e-6, name
         else:
             assert max_rel(a.cpu().numpy(), b) <= 2e-4, (name, max_rel(a.cpu().numpy(), b))
+
+
+def test_backward_is_bit_for_bit_repeatable(cuda_device):
+    """Every gradient is a fixed-order sum (no atomics): two calls on the
+    same inputs give identical bits."""
+    import sliding_window_attention_tc_b200 as tc
+    B, H, T, d, W = 2, 4, 1100, 64, 128
+    x = wl.random_prefill(B, H, T, d, d, W, 8, dtype="bf16", seed=5)
+    gen = torch.Generator().manual_seed(6)
+    dy = (torch.randn(B, H, T, d, generator=gen) / 4).to(x.q.dtype)
+    dev = cuda_device
+    args = [t.to(dev).contiguous() for t in (x.q, x.k, x.v, x.lam, x.eta, x.g)]
+    a = tc.backward(*args, W, dy.to(dev))
+    b = tc.backward(*args, W, dy.to(dev))
+    torch.cuda.synchronize()
+    assert tc.device_status() == 0
+    for name, u, w in zip(("dq", "dk", "dv", "dlam", "deta", "dg"), a, b):
+        assert torch.equal(u, w), name

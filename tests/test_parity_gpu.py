@@ -140,6 +140,22 @@ def test_prefill_long_bf16_full_size_sampled_heads(cuda_device):
     print("long_prefill_bf16", out)
 
 
+def test_prefill_long_bf16_every_head(cuda_device):
+    """All 16 heads of the long-context workload (1 x 16 x 32768, W = 1024),
+    y and A_final, against one oracle call that runs the heads in parallel."""
+    x = wl.prefill_config("long_prefill_bf16")
+    y, A = run_prefill(x, cuda_device)
+    yo, Ao = oracle.prefill(x.q, x.k, x.v, x.lam, x.eta, x.g, x.W)
+    H = x.q.shape[1]
+    worst = {"y": 0.0, "A": 0.0}
+    for h in range(H):
+        ey, eA = rel_l2(y[0, h], yo[0, h]), rel_l2(A[0, h], Ao[0, h])
+        assert ey <= BF16_Y_TOL and eA <= BF16_A_TOL, (h, ey, eA)
+        worst = {"y": max(worst["y"], ey), "A": max(worst["A"], eA)}
+    assert np.isfinite(y).all()
+    print("long_prefill_bf16, every head", worst)
+
+
 # --- edge shapes ----------------------------------------------------------
 
 EDGE = [
