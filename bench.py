@@ -44,11 +44,11 @@ HEADLINE = "lm_prefill_bf16"
 
 # DRAM bytes (read + write) per launch from one ncu capture of the current
 # kernels; they must be re-measured (or set to None) whenever a kernel changes.
-#   prefill_main_kernel: None until the kernel as it now stands is captured
-#     again (its MMA issue loops changed after profiles/prefill_main_kernel_*)
+#   prefill_main_kernel: one LM launch, 159.2 MB read + 31.9 MB written
+#     (profiles/prefill_main_kernel_lm_prefill_bf16.md)
 #   decode_kernel: the B = 32 capture scaled by heads to the 256 x 32 launch,
 #     (1.1417 + 0.0172) GB x 8 (profiles/decode_kernel_b32_w2048_d128.md)
-NCU_TRAFFIC_BYTES = {"prefill_main_kernel": None, "decode_kernel": 9.27e9}
+NCU_TRAFFIC_BYTES = {"prefill_main_kernel": 1.911e8, "decode_kernel": 9.27e9}
 METRIC = "prefill tokens/s & decode tok/s per B200; % of TC/HBM roofline"
 UNIT = "tokens/s"
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
