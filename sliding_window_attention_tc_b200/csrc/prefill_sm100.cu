@@ -217,10 +217,6 @@ __device__ __forceinline__ bool bar_any(int id, int n, bool pred) {
     return res != 0;
 }
 
-__device__ __forceinline__ void named_bar(int id, int n) {
-    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
-}
-
 // mbar_wait with one answer for the whole warp, so that warps which go on to
 // warp-collective tcgen05.ld / st never diverge on a failed wait.
 __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volatile int *abort,
@@ -428,6 +424,29 @@ __device__ __forceinline__ void build_scaled_key_row(const uint8_t *ktile, uint8
     }
 }
 
+// The same for half a row: 16-byte chunks [4 half, 4 half + 4) of row u.
+__device__ __forceinline__ void build_scaled_key_half(const uint8_t *ktile, uint8_t *hi_tile,
+                                                      uint8_t *lo_tile, int u, int half, float w) {
+#pragma unroll
+    for (int cc = 0; cc < 4; ++cc) {
+        const uint32_t off = sw128_offset(u, (4 * half + cc) * 8);
+        const uint4 raw = *reinterpret_cast<const uint4 *>(ktile + off);
+        float f[8];
+        Vec16<__nv_bfloat16>::unpack(raw, f);
+        uint32_t h[4], l[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const float x0 = f[2 * e] * w, x1 = f[2 * e + 1] * w;
+            const uint32_t hp = pack_bf16(x0, x1);
+            const float h0 = __uint_as_float(hp << 16), h1 = __uint_as_float(hp & 0xffff0000u);
+            h[e] = hp;
+            l[e] = pack_bf16(x0 - h0, x1 - h1);
+        }
+        *reinterpret_cast<uint4 *>(hi_tile + off) = make_uint4(h[0], h[1], h[2], h[3]);
+        *reinterpret_cast<uint4 *>(lo_tile + off) = make_uint4(l[0], l[1], l[2], l[3]);
+    }
+}
+
 // ============================================================================
 // Span start states: S_pre(js) = sum over the spans u < js of
 //   lam^(n_start(js) - e_end(u)) dA_u,  dA_u = sum of its parts,
@@ -483,15 +502,50 @@ __global__ void __launch_bounds__(256) span_prefix_kernel(PrefixParams p) {
 // Pre-pass: dA_u = sum over the evictions e of span u of
 //           eta lam^(e_end - 1 - e) k_e v_e^T     (e_end = end of span u)
 // ============================================================================
-constexpr int NS_SUM = 2;
-constexpr int kSumTilesPerPart = 3;  // eviction tiles per span-summary CTA
+constexpr int NS_SUM = 3;            // K/V stages of the summary kernel
+constexpr int kSumTilesPerPart = 3;  // eviction tiles per span-summary part
+constexpr int kSumThreads = 448;     // producer, MMA, 8 builder and 4 epilogue warps
 constexpr uint32_t SOFF_KV = 0;
-constexpr uint32_t SOFF_KT = SOFF_KV + NS_SUM * 2 * TILE_B;  // one buffer (hi, lo)
-constexpr uint32_t SOFF_DS = SOFF_KV;                        // scratch: stage 0, after the MMAs
-constexpr uint32_t SOFF_BAR = SOFF_KT + 2 * TILE_B;
-constexpr uint32_t SMEM_SUM = SOFF_BAR + 128 + 1024;         // ~97 KB: two CTAs per SM
+constexpr uint32_t SOFF_KT = SOFF_KV + NS_SUM * 2 * TILE_B;  // two buffers (hi, lo)
+constexpr uint32_t SOFF_DS = SOFF_KT + 2 * 2 * TILE_B;       // float32 64x64 exchange
+constexpr uint32_t SOFF_BAR = SOFF_DS + 16384;
+constexpr uint32_t SMEM_SUM = SOFF_BAR + 256 + 1024;         // ~177 KB: one CTA per SM
 
-__global__ void __launch_bounds__(192, 2)
+// Where the evictions of one summary part lie: span js of row bh, part
+// `part` of its n_parts; ev_first / ne its eviction tiles, e_end the end of
+// the span's evictions (every part decays to it, so the parts add up to the
+// span's summary).
+struct SumSlot {
+    SeqView sv;
+    int bh, ev_first, ne, e_end;
+};
+__device__ __forceinline__ SumSlot sum_slot(const SumParams &p, int slot, int *status) {
+    SumSlot q;
+    const int per_head = p.n_s - 1;
+    const int part = slot % p.n_parts;
+    const int js = (slot / p.n_parts) % per_head;
+    q.bh = slot / (per_head * p.n_parts);
+    q.sv = seq_view(p.vl, q.bh, p.H, p.T, status);
+    int i0, i1;
+    span_range(js, q.sv.nT, p.n_s, p.q_off / BM, i0, i1);
+    const int E = q.sv.T > p.W ? q.sv.T - p.W : 0;
+    const int ev_span = i0 > p.W / BM ? i0 : p.W / BM;  // first tile of the span with evictions
+    const int ne_span = i1 > ev_span ? i1 - ev_span : 0;
+    q.ev_first = ev_span + (int)((long long)ne_span * part / p.n_parts);
+    q.ne = ev_span + (int)((long long)ne_span * (part + 1) / p.n_parts) - q.ev_first;
+    q.e_end = ne_span > 0 ? min(E, i1 * BM - p.W) : 0;
+    return q;
+}
+
+// Persistent CTAs, one per SM, each taking parts blockIdx.x, + gridDim.x, ...
+// Roles: warp 0 loads K/V tiles through an NS_SUM-stage ring; warps 2-9
+// build the scaled hi/lo keys (half a row per thread, two warps per SM
+// sub-partition to hide the build's latency) into two alternating buffers;
+// warp 1 accumulates a part's tiles into one of two TMEM accumulators;
+// warps 10-13 read a finished accumulator, add its hi and lo rows and store
+// the part.  So the loads, builds, MMAs and stores of consecutive tiles and
+// parts overlap.
+__global__ void __launch_bounds__(kSumThreads, 1)
     span_summary_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
                         const __grid_constant__ CUtensorMap tkh,
                         const __grid_constant__ CUtensorMap tvh, SumParams p) {
@@ -502,141 +556,179 @@ __global__ void __launch_bounds__(192, 2)
     uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + SOFF_BAR);
     uint64_t *kv_full = bars, *kv_empty = bars + NS_SUM;
-    uint64_t *kt_full = bars + 2 * NS_SUM, *kt_empty = kt_full + 1, *done = kt_empty + 1;
+    uint64_t *kt_full = bars + 2 * NS_SUM, *kt_empty = kt_full + 2;
+    uint64_t *acc_full = kt_empty + 2, *acc_empty = acc_full + 2, *done = acc_empty + 2;
     uint32_t *tmem_base = reinterpret_cast<uint32_t *>(done + 1);
     volatile int *abort = reinterpret_cast<volatile int *>(tmem_base + 1);
     float *sDS = reinterpret_cast<float *>(sm + SOFF_DS);
 
     griddep_launch_dependents();
     const int tid = threadIdx.x, warp = tid >> 5;
-    const int per_head = p.n_s - 1;
-    const int slot = blockIdx.x;  // (bh, js, part)
-    const int part = slot % p.n_parts;
-    const int bh = slot / (per_head * p.n_parts), js = (slot / p.n_parts) % per_head;
-    const int h = bh % p.H;
+    const int n_slots = p.BH * (p.n_s - 1) * p.n_parts;
     const bool varlen = p.vl.cu != nullptr;
-    const SeqView sv = seq_view(p.vl, bh, p.H, p.T, tid == 0 ? p.status : nullptr);
-    int i0, i1;
-    span_range(js, sv.nT, p.n_s, p.q_off / BM, i0, i1);
-    const int E = sv.T > p.W ? sv.T - p.W : 0;
-    const int ev_span = i0 > p.W / BM ? i0 : p.W / BM;  // first tile of the span with evictions
-    const int ne_span = i1 > ev_span ? i1 - ev_span : 0;
-    // this CTA's share of the span's eviction tiles; every part decays to
-    // the span's end e_end, so the parts add up to the span's summary
-    const int ev_first = ev_span + (int)((long long)ne_span * part / p.n_parts);
-    const int ne = ev_span + (int)((long long)ne_span * (part + 1) / p.n_parts) - ev_first;
-    const int e_end = ne_span > 0 ? min(E, i1 * BM - p.W) : 0;
 
     if (tid == 0) {
         for (int s = 0; s < NS_SUM; ++s) {
             mbar_init(&kv_full[s], 1);
             mbar_init(&kv_empty[s], 1);
         }
-        mbar_init(kt_full, 128);
-        mbar_init(kt_empty, 1);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&kt_full[b], 256);
+            mbar_init(&kt_empty[b], 1);
+            mbar_init(&acc_full[b], 1);
+            mbar_init(&acc_empty[b], 128);
+        }
         mbar_init(done, 1);
         *abort = 0;
         fence_mbar_init();
     }
     if (warp == 1) {
-        tmem_alloc(tmem_base, 64);
+        tmem_alloc(tmem_base, 128);
         tmem_relinquish();
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tb = *tmem_base;
-    float *out = p.dA + (size_t)slot * HD * HD;
 
-    if (ne == 0) {
-        for (int x = tid; x < HD * HD; x += blockDim.x) out[x] = 0.f;
-    } else if (warp == 0) {
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer
         if (tid == 0) {
             tma_prefetch_desc(&tk);
             tma_prefetch_desc(&tv);
-            int issued = 0;
-            for (int e = 0; e < ne; ++e) {
-                const int s = e % NS_SUM;
-                if (!mbar_wait(&kv_empty[s], ((e / NS_SUM) & 1) ^ 1, abort, p.status, p.wait_ns)) break;
-                const int n0 = (ev_first + e) * BM - p.W;
-                uint8_t *dst = sm + SOFF_KV + s * 2 * TILE_B;
-                mbar_expect_tx(&kv_full[s], 2 * TILE_B);
-                load_kv_tile(dst, &tk, &tv, &tkh, &tvh, &kv_full[s], n0 / BM, p.q_off, sv, varlen);
-                issued = e + 1;
+            uint32_t g = 0;
+            bool ok = true;
+            for (int slot = blockIdx.x; slot < n_slots && ok; slot += gridDim.x) {
+                const SumSlot q = sum_slot(p, slot, nullptr);
+                for (int e = 0; e < q.ne; ++e, ++g) {
+                    const int s = g % NS_SUM;
+                    if (!(ok = mbar_wait(&kv_empty[s], ((g / NS_SUM) & 1) ^ 1, abort, p.status, p.wait_ns))) break;
+                    const int n0 = (q.ev_first + e) * BM - p.W;
+                    mbar_expect_tx(&kv_full[s], 2 * TILE_B);
+                    load_kv_tile(sm + SOFF_KV + s * 2 * TILE_B, &tk, &tv, &tkh, &tvh, &kv_full[s],
+                                 n0 / BM, p.q_off, q.sv, varlen);
+                }
             }
-            for (int st = 0; st < NS_SUM; ++st) {
-                const int fills = issued > st ? (issued - 1 - st) / NS_SUM + 1 : 0;
+            // every issued copy lands before the CTA exits
+            for (uint32_t st = 0; st < NS_SUM; ++st) {
+                const uint32_t fills = g > st ? (g - 1 - st) / NS_SUM + 1 : 0;
                 if (fills) mbar_wait_drain(&kv_full[st], (fills - 1) & 1);
             }
         }
     } else if (warp == 1) {
-        if (tid == 32) {
-            const uint32_t id_ds = idesc_bf16(128, 64, true, true);
-            for (int e = 0; e < ne; ++e) {
-                const int s = e % NS_SUM;
-                if (!mbar_wait(kt_full, e & 1, abort, p.status, p.wait_ns)) break;
+        // ------------------------------------------------------------ MMA issuer
+        const uint32_t id_ds = idesc_bf16(128, 64, true, true);
+        uint32_t g = 0, nz = 0;
+        bool ok = true;
+        for (int slot = blockIdx.x; slot < n_slots && ok; slot += gridDim.x) {
+            const SumSlot q = sum_slot(p, slot, nullptr);
+            if (q.ne == 0) continue;
+            const uint32_t acc = tb + 64 * (nz & 1);
+            for (int e = 0; e < q.ne; ++e, ++g) {
+                const int s = g % NS_SUM, b = g & 1;
+                if (!(ok = warp_wait(&kt_full[b], (g >> 1) & 1, abort, p.status, p.wait_ns))) break;
+                if (e == 0 && !(ok = warp_wait(&acc_empty[nz & 1], ((nz >> 1) & 1) ^ 1, abort, p.status, p.wait_ns))) break;
                 tc_fence_after();
-                const uint32_t kt = smem_u32(sm + SOFF_KT);
-                const uint32_t vv = smem_u32(sm + SOFF_KV + s * 2 * TILE_B + TILE_B);
+                const uint64_t ktd = sdesc_sw128(smem_u32(sm + SOFF_KT + b * 2 * TILE_B), TILE_B, 1024);
+                const uint64_t vd = sdesc_sw128(smem_u32(sm + SOFF_KV + s * 2 * TILE_B + TILE_B), TILE_B, 1024);
+                mma_ss_w(acc, ktd, vd, id_ds, e > 0);
 #pragma unroll
-                for (int k = 0; k < 8; ++k)
-                    mma_ss(tb, sdesc_sw128(kt + 2048 * k, TILE_B, 1024),
-                           sdesc_sw128(vv + 2048 * k, TILE_B, 1024), id_ds, (e > 0 || k > 0));
-                mma_commit(kt_empty);
-                mma_commit(&kv_empty[s]);
+                for (int k = 1; k < 8; ++k) mma_ss_w(acc, ktd + 128 * k, vd + 128 * k, id_ds, 1);
+                mma_commit_w(&kt_empty[b]);
+                mma_commit_w(&kv_empty[s]);
+                if (e == q.ne - 1) mma_commit_w(&acc_full[nz & 1]);
             }
-            mma_commit(done);
-            mbar_wait_drain(done, 0);
+            ++nz;
+        }
+        // nothing may still run on the tensor cores when TMEM is released
+        mma_commit_w(done);
+        mbar_wait_drain(done, 0);
+    } else if (warp >= 2 && warp < 10) {
+        // ------------------------------------------------------------ key builders
+        const int u = (tid - 64) & 127, half = (tid - 64) >> 7;  // key row, half of it
+        uint32_t g = 0;
+        bool ok = true;
+        for (int slot = blockIdx.x; slot < n_slots && ok; slot += gridDim.x) {
+            const SumSlot q = sum_slot(p, slot, tid == 64 ? p.status : nullptr);
+            if (q.ne == 0) continue;
+            const int h = q.bh % p.H;
+            const float l2l = (float)log2((double)p.lam[h]);
+            const float eta = p.eta[h];
+            for (int e = 0; e < q.ne; ++e, ++g) {
+                const int s = g % NS_SUM, b = g & 1;
+                if (!(ok = mbar_wait(&kv_full[s], (g / NS_SUM) & 1, abort, p.status, p.wait_ns))) break;
+                if (!(ok = mbar_wait(&kt_empty[b], ((g >> 1) & 1) ^ 1, abort, p.status, p.wait_ns))) break;
+                const int ev = (q.ev_first + e) * BM - p.W + u;
+                // float exp2: relative error ~1e-7 for the weights that matter (the
+                // exponent error grows with the decay, and decayed terms are small)
+                const float w = ev < q.e_end ? eta * exp2f((float)(q.e_end - 1 - ev) * l2l) : 0.f;
+                uint8_t *kt = sm + SOFF_KT + b * 2 * TILE_B;
+                build_scaled_key_half(sm + SOFF_KV + s * 2 * TILE_B, kt, kt + TILE_B, u, half, w);
+                fence_async_smem();
+                mbar_arrive(&kt_full[b]);
+            }
         }
     } else {
-        // builders: warps 2-5, thread u builds key row u
-        const int u = tid - 64;
-        const double lam = p.lam[h];
-        const float eta = p.eta[h];
-        const double l2l = log2(lam);
-        for (int e = 0; e < ne; ++e) {
-            const int s = e % NS_SUM;
-            if (!mbar_wait(&kv_full[s], (e / NS_SUM) & 1, abort, p.status, p.wait_ns)) break;
-            if (!mbar_wait(kt_empty, (e & 1) ^ 1, abort, p.status, p.wait_ns)) break;
-            const int n0 = (ev_first + e) * BM - p.W;
-            const int ev = n0 + u;
-            const float w = ev < e_end ? eta * (float)exp2((double)(e_end - 1 - ev) * l2l) : 0.f;
-            uint8_t *kt = sm + SOFF_KT;
-            build_scaled_key_row(sm + SOFF_KV + s * 2 * TILE_B, kt, kt + TILE_B, u, w);
-            fence_async_smem();
-            mbar_arrive(kt_full);
-        }
-        // read the accumulated [hi; lo] rows and add the halves
-        const bool ok = warp_wait(done, 0, abort, p.status, p.wait_ns);
-        tc_fence_after();
-        const int lane_base = 32 * (warp & 3);
-        const int L = lane_base + (tid & 31);
-        float v[64];
-        if (ok) {
-            uint32_t r[32];
-            tmem_ld32(tmem_addr(tb, lane_base, 0), r);
-            tmem_wait_ld();
+        // ------------------------------------------------------------ epilogue
+        // TMEM lane L = row of the accumulator: L < 64 the hi part of state row
+        // L, L >= 64 the lo part of state row L - 64.  A wait that gives up sets
+        // `failed`; the next barrier (named barrier 1, these 128 threads) tells
+        // all, and all leave together.
+        const int L = 32 * (warp & 3) + (tid & 31);
+        uint32_t nz = 0;
+        bool failed = false;
+        for (int slot = blockIdx.x; slot < n_slots; slot += gridDim.x) {
+            const SumSlot q = sum_slot(p, slot, nullptr);
+            float *out = p.dA + (size_t)slot * HD * HD;
+            if (q.ne == 0) {
+                if (L < 64) {
+                    float4 *dst = reinterpret_cast<float4 *>(out + L * HD);
 #pragma unroll
-            for (int c = 0; c < 32; ++c) v[c] = __uint_as_float(r[c]);
-            tmem_ld32(tmem_addr(tb, lane_base, 32), r);
-            tmem_wait_ld();
+                    for (int c = 0; c < 16; ++c) dst[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+                }
+                continue;
+            }
+            if (!failed && !warp_wait(&acc_full[nz & 1], (nz >> 1) & 1, abort, p.status, p.wait_ns))
+                failed = true;
+            tc_fence_after();
+            float v[64];
+            if (!failed) {
+                uint32_t r[32];
+                const uint32_t acc = tb + 64 * (nz & 1);
+                tmem_ld32(tmem_addr(acc, 32 * (warp & 3), 0), r);
+                tmem_wait_ld();
 #pragma unroll
-            for (int c = 0; c < 32; ++c) v[32 + c] = __uint_as_float(r[c]);
-        }
-        if (L >= 64) {
+                for (int c = 0; c < 32; ++c) v[c] = __uint_as_float(r[c]);
+                tmem_ld32(tmem_addr(acc, 32 * (warp & 3), 32), r);
+                tmem_wait_ld();
 #pragma unroll
-            for (int c = 0; c < 64; ++c) sDS[c * 64 + (L - 64)] = ok ? v[c] : 0.f;
-        }
-        named_bar(1, 128);
-        if (L < 64) {
+                for (int c = 0; c < 32; ++c) v[32 + c] = __uint_as_float(r[c]);
+            }
+            // the previous part's readers of sDS are done
+            if (bar_any(1, 128, failed)) break;
+            if (L >= 64) {
 #pragma unroll
-            for (int c = 0; c < 64; ++c) out[L * HD + c] = ok ? v[c] + sDS[c * 64 + L] : 0.f;
+                for (int c = 0; c < 64; ++c) sDS[c * 64 + (L - 64)] = v[c];
+            }
+            // the accumulator is read: the MMA issuer may start the part after next in it
+            tc_fence_before();
+            mbar_arrive(&acc_empty[nz & 1]);
+            if (bar_any(1, 128, false)) break;
+            if (L < 64) {
+                float4 *dst = reinterpret_cast<float4 *>(out + L * HD);
+#pragma unroll
+                for (int c = 0; c < 16; ++c)
+                    dst[c] = make_float4(v[4 * c] + sDS[(4 * c) * 64 + L], v[4 * c + 1] + sDS[(4 * c + 1) * 64 + L],
+                                         v[4 * c + 2] + sDS[(4 * c + 2) * 64 + L],
+                                         v[4 * c + 3] + sDS[(4 * c + 3) * 64 + L]);
+            }
+            ++nz;
         }
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == 1) tmem_dealloc(tb, 64);
+    if (warp == 1) tmem_dealloc(tb, 128);
 }
 
 // ============================================================================
@@ -1299,8 +1391,9 @@ cudaError_t launch_prefill_sm100(const PrefillParams &p, int num_sms, cudaStream
     if (summaries) {
         SumParams sp{dA, p.lam, p.eta, T_all, (int)p.W, (int)p.H, (int)BH, nT, ns, n_parts, q_off,
                      p.status, p.wait_ns, vl};
-        span_summary_kernel<<<(unsigned)(BH * (ns - 1) * n_parts), 192, SMEM_SUM, s>>>(tk, tv, tkh,
-                                                                                    tvh, sp);
+        const int64_t n_slots = BH * (ns - 1) * n_parts;  // persistent: one CTA per SM at most
+        span_summary_kernel<<<(unsigned)(n_slots < num_sms ? n_slots : num_sms), kSumThreads, SMEM_SUM,
+                              s>>>(tk, tv, tkh, tvh, sp);
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
         PrefixParams pp{dA, p.lam, T_all, (int)p.W, (int)p.H, nT, ns, n_parts, q_off, vl, p.status};

@@ -57,20 +57,35 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
         : "memory");
     return ok != 0;
 }
+// Non-blocking probe of the phase (try_wait may suspend the thread until the
+// phase completes or a hardware time slice ends).
+__device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
 
 // Waits for the phase with the given parity to complete.  Gives up after
 // limit_ns (or at once if *abort is already set): sets *abort, records
 // TC_ERR_DEVICE_TIMEOUT (6) in the status word and returns false, so every
-// role drains and the kernel ends instead of hanging.
+// role drains and the kernel ends instead of hanging.  A limit under 1 ms
+// is a test of this path: the wait then probes without suspending (try_wait
+// alone could sleep through a short limit and still succeed) and reads the
+// timer after every probe.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort,
                                           int *status, uint64_t limit_ns = kWaitTimeoutNs) {
-    if (mbar_try_wait(bar, parity)) return true;
+    const bool poll = limit_ns < 1000000u;
+    if (poll ? mbar_test_wait(bar, parity) : mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer();
-    // the timer is read every 256 failed tries, or on every try when the
-    // limit is short (a test of the timeout path)
-    const uint32_t every = limit_ns < 1000000u ? 0u : 255u;
+    const uint32_t every = poll ? 0u : 255u;  // timer reads: every try, or every 256
     for (uint32_t i = 1;; ++i) {
-        if (mbar_try_wait(bar, parity)) return true;
+        if (poll ? mbar_test_wait(bar, parity) : mbar_try_wait(bar, parity)) return true;
         if ((i & every) == 0) {
             if (*abort) return false;
             if (globaltimer() - t0 > limit_ns) {
@@ -119,15 +134,25 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
         : "memory");
     return ok != 0;
 }
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int *abort,
                                           int *status, uint64_t limit_ns = kWaitTimeoutNs) {
-    if (mbar_try_wait(bar, parity)) return true;
+    const bool poll = limit_ns < 1000000u;  // as above: a test of the timeout path
+    if (poll ? mbar_test_wait(bar, parity) : mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer();
-    // the timer is read every 256 failed tries, or on every try when the
-    // limit is short (a test of the timeout path)
-    const uint32_t every = limit_ns < 1000000u ? 0u : 255u;
+    const uint32_t every = poll ? 0u : 255u;
     for (uint32_t i = 1;; ++i) {
-        if (mbar_try_wait(bar, parity)) return true;
+        if (poll ? mbar_test_wait(bar, parity) : mbar_try_wait(bar, parity)) return true;
         if ((i & every) == 0) {
             if (*abort) return false;
             if (globaltimer() - t0 > limit_ns) {
