@@ -502,14 +502,14 @@ __global__ void __launch_bounds__(256) span_prefix_kernel(PrefixParams p) {
 // Pre-pass: dA_u = sum over the evictions e of span u of
 //           eta lam^(e_end - 1 - e) k_e v_e^T     (e_end = end of span u)
 // ============================================================================
-constexpr int NS_SUM = 3;            // K/V stages of the summary kernel
+constexpr int NS_SUM = 4;            // K/V stages of the summary kernel
 constexpr int kSumTilesPerPart = 3;  // eviction tiles per span-summary part
 constexpr int kSumThreads = 448;     // producer, MMA, 8 builder and 4 epilogue warps
 constexpr uint32_t SOFF_KV = 0;
 constexpr uint32_t SOFF_KT = SOFF_KV + NS_SUM * 2 * TILE_B;  // two buffers (hi, lo)
 constexpr uint32_t SOFF_DS = SOFF_KT + 2 * 2 * TILE_B;       // float32 64x64 exchange
 constexpr uint32_t SOFF_BAR = SOFF_DS + 16384;
-constexpr uint32_t SMEM_SUM = SOFF_BAR + 256 + 1024;         // ~177 KB: one CTA per SM
+constexpr uint32_t SMEM_SUM = SOFF_BAR + 256 + 1024;         // ~210 KB: one CTA per SM
 
 // Where the evictions of one summary part lie: span js of row bh, part
 // `part` of its n_parts; ev_first / ne its eviction tiles, e_end the end of
