@@ -277,9 +277,25 @@ def tc_launches_per_prefill(tc, desc):
     return fn(desc) if fn else None
 
 
+def decode_state_from_prewarm(tc, x, rows=16):
+    """A of the decode workload: its n_prewarm evicted pairs written through
+    libtc (state-only scan), rows batch rows at a time."""
+    B, H, _, dk = x.ring_k.shape
+    dv = x.ring_v.shape[-1]
+    A = torch.empty((B, H, dk, dv), dtype=torch.float32, device=x.ring_k.device)
+    for b0 in range(0, B, rows):
+        b1 = min(B, b0 + rows)
+        k, v = wl.decode_prewarm_pairs(x, b0, b1)
+        tc.write_pairs(k, v, x.lam, x.eta, A=A[b0:b1])
+        del k, v
+    torch.cuda.synchronize()
+    return A
+
+
 def time_decode(tc, dev, world, clocks=None, steps=None, batch=None, e2e=True):
     x = wl.decode_workload(device=dev, B=batch, steps=None if steps is None else steps + 3)
     n = x.q.shape[0] - 3 if steps is not None else x.q.shape[0]
+    x.A = decode_state_from_prewarm(tc, x)
     st = tc.DecodeState(x.ring_k, x.ring_v, x.A, x.lam, x.eta, x.g, x.t0)
     B, H, W, dk = x.ring_k.shape
     dv = x.ring_v.shape[-1]

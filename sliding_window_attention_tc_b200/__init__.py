@@ -303,6 +303,24 @@ def prefill_varlen(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlens
     return y, A_final
 
 
+def write_pairs(k: torch.Tensor, v: torch.Tensor, lam: torch.Tensor, eta: torch.Tensor,
+                A: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """A after writing the pairs k [B,H,n,dk], v [B,H,n,dv] in order into an
+    empty state with the layer's write, A <- lam A + eta k v^T per pair:
+    tc_prefill_from_state, state only, over the n pairs plus one token with
+    W = 1, so that exactly the n pairs are evicted (one chunk of n)."""
+    B, H, n, dk = k.shape
+    dv = v.shape[-1]
+    pad_k = torch.zeros((B, H, 1, dk), dtype=k.dtype, device=k.device)
+    pad_v = torch.zeros((B, H, 1, dv), dtype=v.dtype, device=v.device)
+    ks = torch.cat([k, pad_k], dim=2).contiguous()
+    vs = torch.cat([v, pad_v], dim=2).contiguous()
+    g = torch.zeros(H, dtype=torch.float32, device=k.device)
+    _, A = prefill_from_state(None, ks, vs, lam, eta, g, 1, max(n, 1), 0, state_only=True,
+                              A_final=A)
+    return A
+
+
 def prefill_from_state(q: Optional[torch.Tensor], k: torch.Tensor, v: torch.Tensor,
                        lam: torch.Tensor, eta: torch.Tensor, g: torch.Tensor, W: int, C: int,
                        t0: int, halo_k: Optional[torch.Tensor] = None,

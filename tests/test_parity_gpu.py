@@ -140,6 +140,22 @@ def test_prefill_long_bf16_full_size_sampled_heads(cuda_device):
     print("long_prefill_bf16", out)
 
 
+def test_prefill_lm_bf16_every_head(cuda_device):
+    """All 96 (b, h) rows of the LM workload (8 x 12 x 4096, W = 512), y and
+    A_final, against one oracle call over every row."""
+    x = wl.prefill_config("lm_prefill_bf16")
+    y, A = run_prefill(x, cuda_device)
+    yo, Ao = oracle.prefill(x.q, x.k, x.v, x.lam, x.eta, x.g, x.W)
+    B, H = x.q.shape[:2]
+    worst = {"y": 0.0, "A": 0.0}
+    for b in range(B):
+        for h in range(H):
+            ey, eA = rel_l2(y[b, h], yo[b, h]), rel_l2(A[b, h], Ao[b, h])
+            assert ey <= BF16_Y_TOL and eA <= BF16_A_TOL, (b, h, ey, eA)
+            worst = {"y": max(worst["y"], ey), "A": max(worst["A"], eA)}
+    print("lm_prefill_bf16, every head", worst)
+
+
 def test_prefill_long_bf16_every_head(cuda_device):
     """All 16 heads of the long-context workload (1 x 16 x 32768, W = 1024),
     y and A_final, against one oracle call that runs the heads in parallel."""
@@ -316,15 +332,32 @@ def test_decode_host_variant_matches_device(cuda_device):
 
 def test_decode_full_size_sampled_heads(cuda_device):
     """The batched-decode workload (256 x 32 heads, d = 128, W = 2048, ring
-    full, A pre-warmed, 512 steps) on the GPU; the oracle replays 32 sampled
-    heads over all 512 steps from the same initial state."""
+    full, A the state left by 8192 evicted pairs, 512 steps) on the GPU; A is
+    written through libtc.  The oracle writes the same pairs for 32 sampled
+    heads with its own token loop, then replays them over all 512 steps."""
+    import bench
     tc = _tc()
     x = wl.decode_workload(device=cuda_device)
     B, H = x.ring_k.shape[:2]
     rng = np.random.default_rng(0)
     flat = rng.choice(B * H, size=32, replace=False)
     sb, sh = torch.as_tensor(flat // H), torch.as_tensor(flat % H)
-    init = [t[sb, sh].cpu() for t in (x.ring_k, x.ring_v, x.A)]
+    x.A = bench.decode_state_from_prewarm(tc, x)
+    prm = [t.cpu()[sh] for t in (x.lam, x.eta, x.g)]
+    # the oracle's A for the sampled heads, from the same pairs (one oracle
+    # "batch" entry, each sampled head with its own parameters)
+    pk, pv = [], []
+    for b, h in zip(sb.tolist(), sh.tolist()):
+        k_ev, v_ev = wl.decode_prewarm_pairs(x, b, b + 1)
+        pk.append(k_ev[0, h].cpu())
+        pv.append(v_ev[0, h].cpu())
+    pk, pv = torch.stack(pk).unsqueeze(0), torch.stack(pv).unsqueeze(0)
+    pad = torch.zeros(1, len(flat), 1, pk.shape[-1], dtype=pk.dtype)
+    kk, vv = torch.cat([pk, pad], dim=2), torch.cat([pv, pad], dim=2)
+    _, A_o = oracle.prefill(torch.zeros_like(kk), kk, vv, prm[0], prm[1], prm[2], 1)
+    A_err0 = rel_l2(x.A[sb, sh].cpu().numpy(), A_o[0])
+    assert A_err0 <= 1e-4, A_err0  # a float32 scan of 8192 writes against float64
+    init = [x.ring_k[sb, sh].cpu(), x.ring_v[sb, sh].cpu(), torch.from_numpy(A_o[0])]
     st = tc.DecodeState(x.ring_k, x.ring_v, x.A, x.lam, x.eta, x.g, x.t0)
     n = x.q.shape[0]
     ys = torch.empty(n, len(flat), x.v.shape[-1], dtype=torch.bfloat16)
@@ -334,8 +367,6 @@ def test_decode_full_size_sampled_heads(cuda_device):
     torch.cuda.synchronize()
     assert tc.device_status() == 0
     q, k, v = (t[:, sb, sh].cpu().unsqueeze(1) for t in (x.q, x.k, x.v))
-    prm = [t.cpu()[sh] for t in (x.lam, x.eta, x.g)]
-    # one oracle "batch" entry per sampled head, each with its own parameters
     yo, rko, rvo, Ao = oracle.decode(init[0].unsqueeze(0), init[1].unsqueeze(0),
                                      init[2].unsqueeze(0), x.t0, q, k, v, *prm)
     y_err = rel_l2(ys.float().numpy(), yo[:, 0])

@@ -18,6 +18,7 @@ callers copy sampled heads to the host for checking.
 from __future__ import annotations
 
 import math
+from typing import Optional
 from dataclasses import dataclass, field
 
 import torch
@@ -206,7 +207,7 @@ def varlen_config() -> "VarlenInputs":
 class DecodeInputs:
     ring_k: torch.Tensor  # [B,H,W,dk]
     ring_v: torch.Tensor  # [B,H,W,dv]
-    A: torch.Tensor  # [B,H,dk,dv] float32
+    A: Optional[torch.Tensor]  # [B,H,dk,dv] float32, or None: build it from prewarm_pairs
     q: torch.Tensor  # [steps,B,H,dk]
     k: torch.Tensor  # [steps,B,H,dk]
     v: torch.Tensor  # [steps,B,H,dv]
@@ -215,18 +216,38 @@ class DecodeInputs:
     g: torch.Tensor
     t0: int
     W: int
+    n_prewarm: int = 0  # evicted pairs before the ring (decode_prewarm_pairs)
+    seed: int = 0
+
+
+def decode_prewarm_pairs(x: "DecodeInputs", b0: int, b1: int):
+    """The n_prewarm (key, value) pairs evicted before the ring's tokens, for
+    batch rows b0 .. b1-1: k [b1-b0, H, n, dk], v [b1-b0, H, n, dv] in the
+    ring's dtype, pair e being token e (tokens n .. n+W-1 fill the ring).
+    Drawn like the stream, N(0,1)/sqrt(d), from a generator seeded per batch
+    row, so any subset of rows can be drawn again."""
+    B, H, W, dk = x.ring_k.shape
+    dv = x.ring_v.shape[-1]
+    n = x.n_prewarm
+    dev = x.ring_k.device
+    gen = torch.Generator(device=dev)
+    ks, vs = [], []
+    for b in range(b0, b1):
+        gen.manual_seed(x.seed * 1000003 + 17 + b)
+        ks.append(torch.randn((H, n, dk), generator=gen, device=dev).mul_(1.0 / math.sqrt(dk)))
+        vs.append(torch.randn((H, n, dv), generator=gen, device=dev).mul_(1.0 / math.sqrt(dv)))
+    dt = x.ring_k.dtype
+    return torch.stack(ks).to(dt), torch.stack(vs).to(dt)
 
 
 def decode_workload(*, B=None, H=None, dk=None, dv=None, W=None, steps=None, history=None,
                     prewarm_evictions=None, dtype=None, seed=None, device="cuda") -> DecodeInputs:
     """Batched-decode workload: a full ring (tokens history-W..history-1 at
-    slot t mod W), a pre-warmed A and ``steps`` fresh (q, k, v) per head.
-
-    The pre-warmed A stands for the state left by ``prewarm_evictions``
-    earlier evictions of N(0,1)/sqrt(dk) keys and values; it is drawn as a
-    Gaussian matrix whose entry scale matches such a state,
-    eta * sqrt(sum_{j<n} lam^(2j)) / sqrt(dk*dv).  Defaults are the full
-    256 x 32 head, d = 128, W = 2048, 512-step workload."""
+    slot t mod W) and ``steps`` fresh (q, k, v) per head.  A is left None:
+    it is the state the ``prewarm_evictions`` pairs before the ring leave
+    (decode_prewarm_pairs draws them; the caller writes them into A).
+    Defaults are the full 256 x 32 head, d = 128, W = 2048, 512-step
+    workload, with 8192 evicted pairs (history = 8192 + W)."""
     c = dict(DECODE_CONFIG)
     for key, val in dict(B=B, H=H, dk=dk, dv=dv, W=W, steps=steps, history=history,
                          prewarm_evictions=prewarm_evictions, dtype=dtype, seed=seed).items():
@@ -249,13 +270,9 @@ def decode_workload(*, B=None, H=None, dk=None, dv=None, W=None, steps=None, his
 
     ring_k = draw((B, H, W, dk), sk)
     ring_v = draw((B, H, W, dv), sv)
-    npre = c["prewarm_evictions"]
-    geo = (1.0 - lam.pow(2 * npre)) / (1.0 - lam.pow(2))
-    a_scale = (eta * geo.sqrt() * sk * sv).float().to(dev)
-    A = torch.randn((B, H, dk, dv), generator=gen, device=dev, dtype=torch.float32)
-    A.mul_(a_scale.view(1, H, 1, 1))
     q = draw((n, B, H, dk), sk)
     k = draw((n, B, H, dk), sk)
     v = draw((n, B, H, dv), sv)
-    return DecodeInputs(ring_k, ring_v, A, q, k, v, lam.float().to(dev), eta.float().to(dev),
-                        g.float().to(dev), int(c["history"]), W)
+    return DecodeInputs(ring_k, ring_v, None, q, k, v, lam.float().to(dev), eta.float().to(dev),
+                        g.float().to(dev), int(c["history"]), W, int(c["prewarm_evictions"]),
+                        int(c["seed"]))
