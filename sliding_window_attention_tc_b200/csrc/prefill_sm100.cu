@@ -119,6 +119,7 @@ struct MainParams {
     int *status;
     unsigned long long wait_ns;  // limit of every bounded wait
     Varlen vl;
+    const int *order;     // rows (bh) in the order their spans are dealt out, or null
 };
 
 struct SumParams {
@@ -135,6 +136,24 @@ __device__ __forceinline__ void span_range(int j, int nT, int n_s, int i_begin, 
     const int n = nT - i_begin;
     i0 = i_begin + (int)((long long)j * n / n_s);
     i1 = i_begin + (int)((long long)(j + 1) * n / n_s);
+}
+
+// The k-th span of this CTA.  Spans are dealt to the persistent CTAs in
+// snake order (round k left to right when k is even, right to left when
+// odd) over the rows in `order` (null: index order), so that with rows
+// sorted longest first the CTAs get nearly equal work.  Returns false past
+// the last span.
+struct Span {
+    int bh, js;
+};
+__device__ __forceinline__ bool cta_span(int k, int n_spans, int n_s, const int *order, Span &sp) {
+    const int G = gridDim.x, c = blockIdx.x;
+    const long long pos = (long long)k * G + ((k & 1) ? (G - 1 - c) : c);
+    if (pos >= n_spans) return false;
+    const int row = (int)(pos / n_s);
+    sp.bh = order ? order[row] : row;
+    sp.js = (int)(pos % n_s);
+    return true;
 }
 
 // The sequence of row bh (one head of one sequence).  Fixed-length calls: T
@@ -803,11 +822,12 @@ __global__ void __launch_bounds__(kMainThreads, 1)
             }
             uint32_t tile = 0, kc = 0;
             bool ok = true;
-            for (int sp = blockIdx.x; sp < n_spans && ok; sp += gridDim.x) {
-                const int bh = sp / p.n_s;
+            Span spn;
+            for (int ks = 0; ok && cta_span(ks, n_spans, p.n_s, p.order, spn); ++ks) {
+                const int bh = spn.bh;
                 const SeqView sv = seq_view(p.vl, bh, p.H, p.T, nullptr);
                 int i0, i1;
-                span_range(sp % p.n_s, sv.nT, p.n_s, p.q_off / BM, i0, i1);
+                span_range(spn.js, sv.nT, p.n_s, p.q_off / BM, i0, i1);
                 for (int i = i0; i < i1 && ok; ++i, ++tile) {
                     const TileInfo ti = tile_info(i, p.W, l1_only);
                     const int qb = tile & 1;
@@ -899,10 +919,11 @@ __global__ void __launch_bounds__(kMainThreads, 1)
                 }
                 return true;
             };
-            for (int sp = blockIdx.x; sp < n_spans && ok; sp += gridDim.x) {
-                const SeqView sv = seq_view(p.vl, sp / p.n_s, p.H, p.T, nullptr);
+            Span spn;
+            for (int ks = 0; ok && cta_span(ks, n_spans, p.n_s, p.order, spn); ++ks) {
+                const SeqView sv = seq_view(p.vl, spn.bh, p.H, p.T, nullptr);
                 int i0, i1;
-                span_range(sp % p.n_s, sv.nT, p.n_s, p.q_off / BM, i0, i1);
+                span_range(spn.js, sv.nT, p.n_s, p.q_off / BM, i0, i1);
                 for (int i = i0; i < i1 && ok; ++i, ++tile) {
                     const TileInfo ti = tile_info(i, p.W, l1_only);
                     const int qb = tile & 1;
@@ -1000,11 +1021,12 @@ __global__ void __launch_bounds__(kMainThreads, 1)
             }
             return true;
         };
-        for (int sp = blockIdx.x; sp < n_spans && ok; sp += gridDim.x) {
-            const int bh = sp / p.n_s, h = bh % p.H;
+        Span spn;
+        for (int ks = 0; ok && cta_span(ks, n_spans, p.n_s, p.order, spn); ++ks) {
+            const int bh = spn.bh, h = bh % p.H;
             const SeqView sv = seq_view(p.vl, bh, p.H, p.T, nullptr);
             int i0, i1;
-            span_range(sp % p.n_s, sv.nT, p.n_s, p.q_off / BM, i0, i1);
+            span_range(spn.js, sv.nT, p.n_s, p.q_off / BM, i0, i1);
             const double lam = p.lam[h];
             const float gate = 1.0f / (1.0f + expf(-p.g[h]));
             const float pw_r1 = (float)pow(lam, (double)(r + 1));
@@ -1107,8 +1129,9 @@ __global__ void __launch_bounds__(kMainThreads, 1)
         uint8_t *sb_tile = sm + OFF_SB;
         uint8_t *kt_hi = sm + OFF_KT, *kt_lo = sm + OFF_KT + TILE_B;
         float S[64];
-        for (int sp = blockIdx.x; sp < n_spans && ok; sp += gridDim.x) {
-            const int bh = sp / p.n_s, h = bh % p.H, js = sp % p.n_s;
+        Span spn;
+        for (int ks = 0; ok && cta_span(ks, n_spans, p.n_s, p.order, spn); ++ks) {
+            const int bh = spn.bh, h = bh % p.H, js = spn.js;
             // the state warps report rows with inconsistent offsets (once per span)
             const SeqView sv = seq_view(p.vl, bh, p.H, p.T, u == 0 ? p.status : nullptr);
             const int E = sv.T > p.W ? sv.T - p.W : 0;
@@ -1227,6 +1250,54 @@ __global__ void __launch_bounds__(kMainThreads, 1)
     if (warp == 1) tmem_dealloc(tb, 512);
 }
 
+// ============================================================================
+// Row order of a variable-length call: the sequences by decreasing length
+// (ties by index), the H heads of each together, so that the main kernel
+// deals the longest spans out first.  One block; for more than kOrderMax
+// sequences the rows keep their index order.
+// ============================================================================
+constexpr int kOrderMax = 4096;
+__global__ void __launch_bounds__(1024) varlen_order_kernel(Varlen vl, int B, int H, int *order) {
+    __shared__ unsigned long long key[kOrderMax];
+    const int tid = threadIdx.x;
+    if (B > kOrderMax) {
+        for (int x = tid; x < B * H; x += blockDim.x) order[x] = x;
+        return;
+    }
+    int n = 1;
+    while (n < B) n <<= 1;
+    for (int b = tid; b < n; b += blockDim.x) {
+        unsigned long long k = ~0ull;  // padding sorts last
+        if (b < B) {
+            const int64_t a = vl.cu[b], e = vl.cu[b + 1];
+            const bool okb = a >= 0 && e >= a && e <= vl.total && e - a <= vl.max_len;
+            const unsigned len = okb ? (unsigned)(e - a) : 0u;
+            k = ((unsigned long long)(0x7fffffffu - len) << 32) | (unsigned)b;
+        }
+        key[b] = k;
+    }
+    __syncthreads();
+    // bitonic sort, ascending keys = descending lengths
+    for (int size = 2; size <= n; size <<= 1) {
+        for (int stride = size >> 1; stride > 0; stride >>= 1) {
+            for (int i = tid; i < n; i += blockDim.x) {
+                const int j = i ^ stride;
+                if (j > i) {
+                    const bool up = (i & size) == 0;
+                    const unsigned long long x = key[i], y = key[j];
+                    if ((x > y) == up) {
+                        key[i] = y;
+                        key[j] = x;
+                    }
+                }
+            }
+            __syncthreads();
+        }
+    }
+    for (int x = tid; x < B * H; x += blockDim.x)
+        order[x] = (int)(key[x / H] & 0xffffffffu) * H + x % H;
+}
+
 // ---------------------------------------------------------------------------
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
@@ -1323,7 +1394,8 @@ static int parts_for(int nT_new, int ns, int64_t BH, int num_sms) {
     return parts < 1 ? 1 : (parts > 16 ? 16 : parts);
 }
 
-size_t sm100_workspace_bytes(const tc_prefill_desc &d, int num_sms) {
+// Summary parts; for a variable-length call the row order follows them.
+static size_t summary_bytes(const tc_prefill_desc &d, int num_sms) {
     if (d.flags & TC_PREFILL_L1_ONLY) return 0;
     const int ns = spans_for(d, num_sms);
     if (ns <= 1) return 0;
@@ -1331,6 +1403,12 @@ size_t sm100_workspace_bytes(const tc_prefill_desc &d, int num_sms) {
     const int64_t BH = d.B * d.H;
     const size_t mats = (size_t)BH * (ns - 1) * parts_for(nT_new, ns, BH, num_sms);
     return mats * HD * HD * sizeof(float);
+}
+
+size_t sm100_workspace_bytes(const tc_prefill_desc &d, int num_sms, bool varlen) {
+    const size_t sum = summary_bytes(d, num_sms);
+    if (!varlen) return sum;
+    return (sum + 255) / 256 * 256 + (size_t)(d.B * d.H) * sizeof(int);
 }
 
 int sm100_launch_count(const tc_prefill_desc &d) {
@@ -1379,6 +1457,19 @@ cudaError_t launch_prefill_sm100(const PrefillParams &p, int num_sms, cudaStream
     if (e != cudaSuccess) return e;
     const int n_parts = ns > 1 ? parts_for(nT - q_off / BM, ns, BH, num_sms) : 1;
     float *dA = reinterpret_cast<float *>(p.workspace);
+    int *order = nullptr;
+    if (varlen) {
+        tc_prefill_desc d{};
+        d.B = p.B;
+        d.H = p.H;
+        d.T = p.T;
+        d.flags = p.l1_only ? TC_PREFILL_L1_ONLY : 0u;
+        const size_t sum = summary_bytes(d, num_sms);
+        order = reinterpret_cast<int *>(static_cast<char *>(p.workspace) + (sum + 255) / 256 * 256);
+        varlen_order_kernel<<<1, 1024, 0, s>>>(vl, (int)p.B, (int)p.H, order);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
     // The summary kernel waits for all earlier work of the stream, as usual.
     // The prefix and main kernels after it may start early (programmatic
     // stream serialization); they read their predecessor's results only
@@ -1408,7 +1499,7 @@ cudaError_t launch_prefill_sm100(const PrefillParams &p, int num_sms, cudaStream
     }
     MainParams mp{p.y,      p.A_final, p.lam, p.eta, p.g,  dA, p.A_init, T_all, (int)p.W, (int)p.H,
                   (int)BH, nT,        ns,    n_parts,         p.l1_only ? 1 : 0, q_off, p.status,
-                  p.wait_ns,  vl};
+                  p.wait_ns,  vl, order};
     const int64_t spans = BH * ns;
     cudaLaunchConfig_t mc = {};
     mc.gridDim = dim3((unsigned)(spans < num_sms ? spans : num_sms));

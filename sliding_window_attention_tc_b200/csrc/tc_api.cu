@@ -266,7 +266,7 @@ tc_status tc_prefill_from_state(const tc_prefill_desc *d, int64_t t0, const void
 
 size_t tc_prefill_varlen_workspace_size(const tc_prefill_desc *d) {
     if (check_desc(d) != TC_OK || !varlen_supported(*d)) return (size_t)-1;
-    return tc::sm100_workspace_bytes(*d, sm_count_or_default());
+    return tc::sm100_workspace_bytes(*d, sm_count_or_default(), true);
 }
 
 tc_status tc_prefill_varlen(const tc_prefill_desc *d, const int64_t *cu_seqlens, int64_t total,
@@ -291,8 +291,8 @@ tc_status tc_prefill_varlen(const tc_prefill_desc *d, const int64_t *cu_seqlens,
     int dev = 0, sms = 0;
     st = current_device(&dev, &sms);
     if (st != TC_OK) return st;
-    const size_t need = tc::sm100_workspace_bytes(*d, sms);
-    if (need > 0 && (!workspace || workspace_bytes < need)) return TC_ERR_WORKSPACE;
+    const size_t need = tc::sm100_workspace_bytes(*d, sms, true);
+    if (!workspace || workspace_bytes < need) return TC_ERR_WORKSPACE;
     const void *ptrs[] = {q, k, v, y};
     for (const void *x : ptrs)
         if (total > 0 && !is_device_ptr(x, dev)) return TC_ERR_INVALID_ARG;
@@ -300,7 +300,7 @@ tc_status tc_prefill_varlen(const tc_prefill_desc *d, const int64_t *cu_seqlens,
     for (const void *x : hd)
         if (!is_device_ptr(x, dev)) return TC_ERR_INVALID_ARG;
     if (A_final && !l1_only && !is_device_ptr(A_final, dev)) return TC_ERR_INVALID_ARG;
-    if (need > 0 && !is_device_ptr(workspace, dev)) return TC_ERR_INVALID_ARG;
+    if (!is_device_ptr(workspace, dev)) return TC_ERR_INVALID_ARG;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if (total == 0) {
         // every sequence is empty: no tokens to read, A_final = 0

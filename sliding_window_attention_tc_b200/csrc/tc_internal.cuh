@@ -123,7 +123,7 @@ cudaError_t launch_backward(const tc_prefill_desc &d, const void *q, const void 
 
 // prefill_sm100.cu: tcgen05 / TMA path for bf16, d_k = d_v = 64.
 bool sm100_supported(const tc_prefill_desc &d, int64_t n_halo);
-size_t sm100_workspace_bytes(const tc_prefill_desc &d, int num_sms);
+size_t sm100_workspace_bytes(const tc_prefill_desc &d, int num_sms, bool varlen = false);
 cudaError_t launch_prefill_sm100(const PrefillParams &p, int num_sms, cudaStream_t s);
 int sm100_launch_count(const tc_prefill_desc &d);
 
