@@ -20,17 +20,16 @@
 //   step t (eviction e = t - W) gives dk_e += eta G_t v_e,
 //   dv_e += eta G_t^T k_e, deta += <G_t, k_e v_e^T>, dlam += <G_t, A_{t-1}>;
 //   also dq_t += A_t (s dy_t) and dg += s (1 - s) <dy_t, q_t A_t>.
-//   bwd_l2_kernel (CTAs of 8 rows of A per (b,h), one thread-block cluster
-//   per (b,h)) replays A from checkpoints every kCk tokens and walks the
-//   tokens backwards; it adds to dq, dk, dv and leaves partials of dlam,
-//   deta, dg, which bwd_reduce_kernel sums over the batch and the row blocks
-//   in a fixed order.  dv_e sums over all rows of G: each CTA keeps its rows'
-//   part for a segment's evictions in shared memory, and the cluster adds
-//   the parts rank by rank through distributed shared memory.  No step
-//   depends on the order in which CTAs run, so the gradients are the same
-//   bit for bit on every run.
+//   Chunked over the evictions (the transpose of the forward chunk scan):
+//   l2b_sums_kernel computes per chunk the state increment and the chunk's
+//   summary of q^T (s dy); l2b_scan_kernel scans both over the chunks, one
+//   thread per state element, giving each chunk's start state A_c and the
+//   G that the later chunks pass back (H_c); l2b_chunk_kernel then forms the
+//   chunk's gradients from C x C products in shared memory; the
+//   bwd_reduce_kernel sums the lambda, eta, g partials over the batch and
+//   the chunks in a fixed order.  No atomics: the gradients are the same bit
+//   for bit on every run.
 
-#include <cooperative_groups.h>
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -43,18 +42,22 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kMaxD = 128;
-constexpr int kRows = kThreads / 32;  // rows of A per CTA in the L2 kernel
 constexpr int kKT = 32;               // key / query tile of the L1 kernels
-constexpr int kCk = 64;               // checkpoint interval of the L2 replay
 constexpr float kLog2e = 1.4426950408889634f;
+
+// Evictions per chunk of the memory backward.  32 keeps l2b_chunk_kernel at
+// about 75 KB of shared memory for d = 64 (three CTAs per SM) and its
+// triangular in-chunk work small; the scan over chunks is cheap either way.
+__host__ __device__ __forceinline__ int l2b_chunk(int, int) { return 32; }
 
 struct BwdParams {
     const void *q, *k, *v, *dy;
     const float *lam, *eta, *g;
     float *gq, *gk, *gv;    // gradients of q, k, v (float32, layout of the inputs)
     float *lse, *Dt;        // [BH][T] per query row (log2 domain), <dy, y_local>
-    float *ckpt, *seg;      // L2 replay: [BH][nCk][dk*dv], [BH][kCk][dk*dv]
-    float *part;            // [BH][3]: dlam, deta, dg
+    float *Ac, *Hc;         // [BH][nC][dk*dv]: increments, then chunk start states A_c;
+                            // summaries, then the G passed back from later chunks H_c
+    float *part;            // [BH][nC][3]: dlam, deta, dg partials
     float *dlam, *deta, *dg;
     int64_t B, H, T, W;
     int dk, dv;
@@ -387,187 +390,340 @@ __host__ __forceinline__ size_t keys_smem(int dk, int dv) {
 }
 
 // ---------------------------------------------------------------------------
-// L2 reverse scan.  Row r of G_t = dL/dA_t and of A_t only involves q_t[r],
-// k_e[r] and whole rows of dy / v, so each (b,h) is split over CTAs of
-// kRows rows (one row per warp; lane l owns columns l, l+32, ...).  A is
-// replayed from checkpoints every kCk tokens; a segment's q, dy, k, v are
-// staged in shared memory once.  dv_e sums over all rows: the CTAs of a head
-// are one cluster, and after each segment every CTA adds one slice of the
-// segment's evictions over the cluster's parts, rank by rank.
+// Memory part, chunked.  Chunk c of row bh holds evictions e = cC .. cC+L-1
+// (L <= C); index i, j, s within it.  Reads at t = e + W: qt_s = q_t,
+// dt_s = s dy_t.  pw(n) = lam^n.
+
+// lam^n for n = 0 .. n_max into shared memory (lam^0 = 1 also for lam = 0).
+__device__ __forceinline__ void lam_powers(float *pw, int n_max, float lam) {
+    const double l2l = log2((double)lam);
+    for (int n = threadIdx.x; n <= n_max; n += blockDim.x)
+        pw[n] = n == 0 ? 1.f : (float)exp2((double)n * l2l);
+}
+
+// Rows r0 .. r0+n-1 (of width d, row stride d in global) into shared rows of
+// stride sp; a row index past `valid` reads as zeros.
 template <typename Tin>
-__global__ void __launch_bounds__(kThreads) bwd_l2_kernel(BwdParams p) {
-    constexpr int CPL = kMaxD / 32;
-    extern __shared__ float sh[];
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int64_t bh = blockIdx.y;
-    const int h = (int)(bh % p.H);
-    const int dk = p.dk, dv = p.dv;
-    const int r0 = blockIdx.x * kRows, r = r0 + warp;
-    const bool row_ok = r < dk;
-    const int64_t T = p.T, W = p.W;
-    const float lam = p.lam[h], eta = p.eta[h];
-    const float sg = 1.f / (1.f + expf(-p.g[h]));
-    // shared: q rows [kCk][kRows], k rows [kCk][kRows], dy [kCk][dv], v [kCk][dv], column sums
-    // [kRows][dv], this CTA's part of dv for the segment's evictions [kCk][dv]
-    float *sQ = sh, *sK = sQ + kCk * kRows, *sDY = sK + kCk * kRows, *sV = sDY + kCk * dv;
-    float *scol = sV + kCk * dv;
-    float *sDV = scol + kRows * dv;
-    namespace cg = cooperative_groups;
-    cg::cluster_group cluster = cg::this_cluster();
-    const Tin *qb = reinterpret_cast<const Tin *>(p.q) + bh * T * dk;
-    const Tin *kb = reinterpret_cast<const Tin *>(p.k) + bh * T * dk;
-    const Tin *vb = reinterpret_cast<const Tin *>(p.v) + bh * T * dv;
-    const Tin *db = reinterpret_cast<const Tin *>(p.dy) + bh * T * dv;
-    const int64_t nCk = (T + kCk - 1) / kCk;
-    const int nrs = gridDim.x;
-    // this CTA's slices: [nCk][kRows][dv] checkpoints, [kCk][kRows][dv] segment
-    float *ck = p.ckpt + ((bh * nrs + blockIdx.x) * nCk) * (int64_t)kRows * dv;
-    float *seg = p.seg + ((bh * nrs + blockIdx.x) * (int64_t)kCk) * kRows * dv;
-    auto at = [&](int jx) { return warp * dv + lane + 32 * jx; };  // element of a [kRows][dv] slab
-    auto col_ok = [&](int jx) { return lane + 32 * jx < dv; };
-
-    // stage q, dy (tokens tb..te-1) and k, v of their evictions
-    auto stage = [&](int64_t tb, int64_t te, bool with_q) {
-        __syncthreads();
-        const int n = (int)(te - tb);
-        for (int x = tid; x < n * kRows; x += kThreads) {
-            const int64_t t = tb + x / kRows;
-            const int rr = r0 + x % kRows;
-            sK[x] = (t >= W && rr < dk) ? to_f32(kb[(t - W) * dk + rr]) : 0.f;
-            if (with_q) sQ[x] = rr < dk ? to_f32(qb[t * dk + rr]) : 0.f;
-        }
-        for (int x = tid; x < n * dv; x += kThreads) {
-            const int64_t t = tb + x / dv;
-            sV[x] = t >= W ? to_f32(vb[(t - W) * dv + x % dv]) : 0.f;
-            if (with_q) sDY[x] = to_f32(db[t * dv + x % dv]);
-        }
-        __syncthreads();
-    };
-
-    float A[CPL];
-#pragma unroll
-    for (int jx = 0; jx < CPL; ++jx) A[jx] = 0.f;
-    // forward replay: checkpoints of A before every kCk-th token
-    for (int64_t s = 0; s < nCk; ++s) {
-        const int64_t tb = s * kCk, te = tb + kCk < T ? tb + kCk : T;
-#pragma unroll
-        for (int jx = 0; jx < CPL; ++jx)
-            if (col_ok(jx)) ck[s * kRows * dv + at(jx)] = A[jx];
-        stage(tb, te, false);
-        for (int64_t t = tb; t < te; ++t) {
-            if (t < W) continue;
-            const float ek = eta * sK[(t - tb) * kRows + warp];
-#pragma unroll
-            for (int jx = 0; jx < CPL; ++jx)
-                if (col_ok(jx)) A[jx] = fmaf(lam, A[jx], ek * sV[(t - tb) * dv + lane + 32 * jx]);
-        }
-    }
-
-    float G[CPL];
-#pragma unroll
-    for (int jx = 0; jx < CPL; ++jx) G[jx] = 0.f;
-    float pl = 0.f, pe = 0.f, pg = 0.f;  // dlam, deta, dg partials
-    for (int64_t s = nCk - 1; s >= 0; --s) {
-        const int64_t tb = s * kCk, te = tb + kCk < T ? tb + kCk : T;
-        stage(tb, te, true);
-        // replay the segment, keeping every A_t of this CTA's rows
-#pragma unroll
-        for (int jx = 0; jx < CPL; ++jx)
-            if (col_ok(jx)) A[jx] = ck[s * kRows * dv + at(jx)];
-        for (int64_t t = tb; t < te; ++t) {
-            if (t >= W) {
-                const float ek = eta * sK[(t - tb) * kRows + warp];
-#pragma unroll
-                for (int jx = 0; jx < CPL; ++jx)
-                    if (col_ok(jx)) A[jx] = fmaf(lam, A[jx], ek * sV[(t - tb) * dv + lane + 32 * jx]);
-            }
-#pragma unroll
-            for (int jx = 0; jx < CPL; ++jx)
-                if (col_ok(jx)) seg[(t - tb) * kRows * dv + at(jx)] = A[jx];
-        }
-        for (int64_t t = te - 1; t >= tb; --t) {
-            const int i = (int)(t - tb);
-            const float qr = sQ[i * kRows + warp];
-            // dq_t[r] += sum_c A_t[r][c] dm_t[c];  dg partial (1 - s) q_t[r] (that)
-            float acc = 0.f;
-#pragma unroll
-            for (int jx = 0; jx < CPL; ++jx)
-                if (col_ok(jx)) acc = fmaf(seg[i * kRows * dv + at(jx)], sg * sDY[i * dv + lane + 32 * jx], acc);
-            acc = warp_sum(acc);
-            if (row_ok && lane == 0) p.gq[(bh * T + t) * dk + r] += acc;
-            pg = fmaf((1.f - sg) * qr, acc, pg);
-            // G += q_t (x) dm_t
-#pragma unroll
-            for (int jx = 0; jx < CPL; ++jx)
-                if (col_ok(jx)) G[jx] = fmaf(qr, sg * sDY[i * dv + lane + 32 * jx], G[jx]);
-            if (t >= W) {
-                const int64_t e = t - W;
-                const float kr = sK[i * kRows + warp];
-                float a2 = 0.f;
-#pragma unroll
-                for (int jx = 0; jx < CPL; ++jx) {
-                    if (!col_ok(jx)) continue;
-                    a2 = fmaf(G[jx], sV[i * dv + lane + 32 * jx], a2);
-                    const float Ap = t > tb ? seg[(i - 1) * kRows * dv + at(jx)]
-                                            : ck[s * kRows * dv + at(jx)];
-                    pl = fmaf(G[jx], Ap, pl);
-                    scol[at(jx)] = G[jx] * kr;
-                }
-                a2 = warp_sum(a2);
-                if (row_ok && lane == 0) p.gk[(bh * T + e) * dk + r] += eta * a2;
-                pe = fmaf(kr, a2, pe);
-                __syncthreads();
-                for (int c = tid; c < dv; c += kThreads) {
-                    float sum = 0.f;
-                    for (int w = 0; w < kRows; ++w) sum += scol[w * dv + c];
-                    sDV[i * dv + c] = sum;
-                }
-                __syncthreads();
-#pragma unroll
-                for (int jx = 0; jx < CPL; ++jx) G[jx] *= lam;
-            }
-        }
-        // dv of the segment's evictions e = t - W (t in [max(tb, W), te)): the
-        // parts of all row blocks, added in rank order; CTA x of the cluster
-        // takes every nrs-th eviction starting at x
-        cluster.sync();
-        const int64_t t_first = tb > W ? tb : W;
-        for (int64_t t = t_first + blockIdx.x; t < te; t += nrs) {
-            const int i = (int)(t - tb);
-            for (int c = tid; c < dv; c += kThreads) {
-                float sum = 0.f;
-                for (int q = 0; q < nrs; ++q) sum += cluster.map_shared_rank(sDV, q)[i * dv + c];
-                p.gv[(bh * T + (t - W)) * dv + c] += eta * sum;
-            }
-        }
-        cluster.sync();  // the parts are read before the next segment overwrites them
-    }
-    // partials of this CTA: pl differs per lane; pe and pg are equal in all
-    // lanes of a warp (only lane 0's count); rows past dk hold zeros
-    __shared__ float sred[3][kRows];
-    pl = warp_sum(pl);
-    if (lane == 0) {
-        sred[0][warp] = pl;
-        sred[1][warp] = pe;
-        sred[2][warp] = pg;
-    }
-    __syncthreads();
-    if (tid < 3) {
-        float a = 0.f;
-        for (int w = 0; w < kRows; ++w) a += sred[tid][w];
-        p.part[(bh * nrs + blockIdx.x) * 3 + tid] = a;
+__device__ __forceinline__ void stage_rows(float *dst, int sp, const Tin *src, int64_t r0, int n,
+                                           int valid, int d, float scale) {
+    for (int x = threadIdx.x; x < n * d; x += blockDim.x) {
+        const int rr = x / d, c = x % d;
+        dst[rr * sp + c] = rr < valid ? scale * to_f32(src[(r0 + rr) * d + c]) : 0.f;
     }
 }
 
-// dlam, deta, dg per head: the (b,h) partials summed over the batch in a
-// fixed order.
-__global__ void bwd_reduce_kernel(BwdParams p, int nrs) {
+// One 4 x 4 block of out[m][n] = sum_k a(m, k) b(k, n) in registers (m0, n0
+// its corner; a and b return 0 outside the ranges they cover).  Each operand
+// loaded from shared memory serves four products.
+template <class FA, class FB>
+__device__ __forceinline__ void tile44(int K, int m0, int n0, FA a, FB b, float (&acc)[4][4]) {
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+#pragma unroll
+        for (int w = 0; w < 4; ++w) acc[u][w] = 0.f;
+    for (int k = 0; k < K; ++k) {
+        float av[4], bv[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) av[u] = a(m0 + u, k);
+#pragma unroll
+        for (int w = 0; w < 4; ++w) bv[w] = b(k, n0 + w);
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+#pragma unroll
+            for (int w = 0; w < 4; ++w) acc[u][w] = fmaf(av[u], bv[w], acc[u][w]);
+    }
+}
+
+// Per chunk: the state increment dA_c = sum_i eta lam^(L-1-i) k_i v_i^T (into
+// Ac) and the summary X_c = sum_s lam^s qt_s^T dt_s (into Hc).
+template <typename Tin>
+__global__ void __launch_bounds__(kThreads) l2b_sums_kernel(BwdParams p) {
+    extern __shared__ float sh[];
+    const int dk = p.dk, dv = p.dv, C = l2b_chunk(dk, dv);
+    const int64_t bh = blockIdx.y, T = p.T, W = p.W, E = T - W;
+    const int c = blockIdx.x, h = (int)(bh % p.H);
+    const int64_t e0 = (int64_t)c * C;
+    const int L = (int)(E - e0 < C ? E - e0 : C);
+    const int nC = (int)((E + C - 1) / C);
+    const float lam = p.lam[h], eta = p.eta[h];
+    const float sg = 1.f / (1.f + expf(-p.g[h]));
+    float *sK = sh, *sV = sK + C * dk, *sQ = sV + C * dv, *sD = sQ + C * dk, *pw = sD + C * dv;
+    const Tin *kb = reinterpret_cast<const Tin *>(p.k) + bh * T * dk;
+    const Tin *vb = reinterpret_cast<const Tin *>(p.v) + bh * T * dv;
+    const Tin *qb = reinterpret_cast<const Tin *>(p.q) + bh * T * dk;
+    const Tin *db = reinterpret_cast<const Tin *>(p.dy) + bh * T * dv;
+    stage_rows(sK, dk, kb, e0, C, L, dk, 1.f);
+    stage_rows(sV, dv, vb, e0, C, L, dv, 1.f);
+    stage_rows(sQ, dk, qb, e0 + W, C, L, dk, 1.f);
+    stage_rows(sD, dv, db, e0 + W, C, L, dv, sg);
+    lam_powers(pw, C, lam);
+    __syncthreads();
+    float *outA = p.Ac + ((size_t)bh * nC + c) * dk * dv;
+    float *outX = p.Hc + ((size_t)bh * nC + c) * dk * dv;
+    const int tm = (dk + 3) / 4, tn = (dv + 3) / 4;
+    for (int t = threadIdx.x; t < tm * tn; t += blockDim.x) {
+        const int r0 = 4 * (t / tn), c0 = 4 * (t % tn);
+        float acc[4][4];
+        tile44(L, r0, c0, [&](int r, int i) { return r < dk ? pw[L - 1 - i] * sK[i * dk + r] : 0.f; },
+               [&](int i, int cc) { return cc < dv ? sV[i * dv + cc] : 0.f; }, acc);
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+#pragma unroll
+            for (int w = 0; w < 4; ++w)
+                if (r0 + u < dk && c0 + w < dv) outA[(r0 + u) * dv + c0 + w] = eta * acc[u][w];
+        tile44(L, r0, c0, [&](int r, int i) { return r < dk ? pw[i] * sQ[i * dk + r] : 0.f; },
+               [&](int i, int cc) { return cc < dv ? sD[i * dv + cc] : 0.f; }, acc);
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+#pragma unroll
+            for (int w = 0; w < 4; ++w)
+                if (r0 + u < dk && c0 + w < dv) outX[(r0 + u) * dv + c0 + w] = acc[u][w];
+    }
+}
+
+// Per (row, state element), over the chunks: A_c = state before chunk c's
+// writes (forward), H_c = G at the start of chunk c+1 (backward), in place.
+// Values are read kScanBatch chunks ahead of their use, so each thread keeps
+// several loads in flight instead of one.
+constexpr int kScanBatch = 8;
+__global__ void __launch_bounds__(kThreads) l2b_scan_kernel(BwdParams p) {
+    __shared__ float decay[2];  // lam^C, lam^(length of the last chunk)
+    const int dk = p.dk, dv = p.dv, C = l2b_chunk(dk, dv);
+    const int64_t bh = blockIdx.y, E = p.T - p.W;
+    const int nC = (int)((E + C - 1) / C);
+    if (threadIdx.x < 2) {
+        const double l2l = log2((double)p.lam[bh % p.H]);
+        const int n = threadIdx.x == 0 ? C : (int)(E - (int64_t)(nC - 1) * C);
+        decay[threadIdx.x] = (float)exp2((double)n * l2l);
+    }
+    __syncthreads();
+    const int x = blockIdx.x * blockDim.x + threadIdx.x;
+    if (x >= dk * dv) return;
+    const float pC = decay[0], pLast = decay[1];
+    const size_t stride = (size_t)dk * dv;
+    float *__restrict__ Ac = p.Ac + (size_t)bh * nC * stride + x;
+    float *__restrict__ Hc = p.Hc + (size_t)bh * nC * stride + x;
+    float A = 0.f;
+    for (int c0 = 0; c0 < nC; c0 += kScanBatch) {
+        float d[kScanBatch];
+#pragma unroll
+        for (int u = 0; u < kScanBatch; ++u) d[u] = c0 + u < nC ? Ac[(size_t)(c0 + u) * stride] : 0.f;
+#pragma unroll
+        for (int u = 0; u < kScanBatch; ++u) {
+            const int c = c0 + u;
+            if (c < nC) {
+                Ac[(size_t)c * stride] = A;
+                A = fmaf(c == nC - 1 ? pLast : pC, A, d[u]);
+            }
+        }
+    }
+    float H = 0.f;
+    for (int c0 = nC - 1; c0 >= 0; c0 -= kScanBatch) {
+        float xs[kScanBatch];
+#pragma unroll
+        for (int u = 0; u < kScanBatch; ++u) xs[u] = c0 - u >= 0 ? Hc[(size_t)(c0 - u) * stride] : 0.f;
+#pragma unroll
+        for (int u = 0; u < kScanBatch; ++u) {
+            const int c = c0 - u;
+            if (c >= 0) {
+                Hc[(size_t)c * stride] = H;
+                H = fmaf(c == nC - 1 ? pLast : pC, H, xs[u]);
+            }
+        }
+    }
+}
+
+// Per chunk, with A = A_c and H = H_c (rows of K, V, qt, dt staged):
+//   dk_i = eta [pw(L-i) H v_i + sum_{s>=i} pw(s-i) (dt_s.v_i) qt_s]
+//   dv_i = eta [pw(L-i) H^T k_i + sum_{s>=i} pw(s-i) (qt_s.k_i) dt_s]
+//   dq_s = pw(s+1) A dt_s + eta sum_{j<=s} pw(s-j) (dt_s.v_j) k_j
+//   m_s  = pw(s+1) qt_s A + eta sum_{j<=s} pw(s-j) (qt_s.k_j) v_j
+//   deta += sum_i <k_i, dk_i> / eta,  dg += (1 - sig) sum_s <dt_s, m_s>,
+//   dlam += L pw(L) <H, A> + sum_s (s+1) pw(s) <qt_s A, dt_s>
+//         + eta sum_j (L-1-j) pw(L-1-j) <k_j, H v_j>
+//         + eta sum_{j<s} (s-j) pw(s-1-j) (qt_s.k_j) (dt_s.v_j)
+// (sum over the chunk's steps e of <G_e, A_{e-1}>, with G_e and A_{e-1}
+// written out in the chunk's terms).  The increments of dq, dk, dv are added
+// to the window part's results; each row belongs to one chunk.
+template <typename Tin>
+__global__ void __launch_bounds__(kThreads) l2b_chunk_kernel(BwdParams p) {
+    extern __shared__ float sh[];
+    const int dk = p.dk, dv = p.dv, C = l2b_chunk(dk, dv);
+    const int sk = dk + 1, sv = dv + 1, sc = C + 1;  // padded strides
+    const int64_t bh = blockIdx.y, T = p.T, W = p.W, E = T - W;
+    const int c = blockIdx.x, h = (int)(bh % p.H);
+    const int64_t e0 = (int64_t)c * C;
+    const int L = (int)(E - e0 < C ? E - e0 : C);
+    const int nC = (int)((E + C - 1) / C);
+    const float eta = p.eta[h];
+    const float sg = 1.f / (1.f + expf(-p.g[h]));
+    float *sK = sh, *sV = sK + C * sk, *sQ = sV + C * sv, *sD = sQ + C * sk;
+    float *sA = sD + C * sv, *sH = sA + dk * sv, *sQK = sH + dk * sv, *sDV = sQK + C * sc;
+    float *pw = sDV + C * sc, *sred = pw + C + 2;
+    const Tin *kb = reinterpret_cast<const Tin *>(p.k) + bh * T * dk;
+    const Tin *vb = reinterpret_cast<const Tin *>(p.v) + bh * T * dv;
+    const Tin *qb = reinterpret_cast<const Tin *>(p.q) + bh * T * dk;
+    const Tin *db = reinterpret_cast<const Tin *>(p.dy) + bh * T * dv;
+    stage_rows(sK, sk, kb, e0, C, L, dk, 1.f);
+    stage_rows(sV, sv, vb, e0, C, L, dv, 1.f);
+    stage_rows(sQ, sk, qb, e0 + W, C, L, dk, 1.f);
+    stage_rows(sD, sv, db, e0 + W, C, L, dv, sg);
+    const float *gA = p.Ac + ((size_t)bh * nC + c) * dk * dv;
+    const float *gH = p.Hc + ((size_t)bh * nC + c) * dk * dv;
+    for (int x = threadIdx.x; x < dk * dv; x += blockDim.x) {
+        sA[(x / dv) * sv + x % dv] = gA[x];
+        sH[(x / dv) * sv + x % dv] = gH[x];
+    }
+    lam_powers(pw, C + 1, p.lam[h]);
+    __syncthreads();
+    // QK[s][j] = qt_s . k_j, DV[s][j] = dt_s . v_j
+    const int tc_ = (C + 3) / 4;
+    for (int t = threadIdx.x; t < tc_ * tc_; t += blockDim.x) {
+        const int s0 = 4 * (t / tc_), j0 = 4 * (t % tc_);
+        float acc[4][4];
+        tile44(dk, s0, j0, [&](int s, int r) { return sQ[s * sk + r]; },
+               [&](int r, int j) { return sK[j * sk + r]; }, acc);
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+#pragma unroll
+            for (int w = 0; w < 4; ++w) sQK[(s0 + u) * sc + j0 + w] = acc[u][w];
+        tile44(dv, s0, j0, [&](int s, int cc) { return sD[s * sv + cc]; },
+               [&](int cc, int j) { return sV[j * sv + cc]; }, acc);
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+#pragma unroll
+            for (int w = 0; w < 4; ++w) sDV[(s0 + u) * sc + j0 + w] = acc[u][w];
+    }
+    __syncthreads();
+    float p_lam = 0.f, p_eta = 0.f, p_g = 0.f;  // this thread's partials
+    float *gq = p.gq + (bh * T + e0 + W) * dk, *gk = p.gk + (bh * T + e0) * dk;
+    float *gv = p.gv + (bh * T + e0) * dv;
+    const int tL = (L + 3) / 4, tk = (dk + 3) / 4, tv = (dv + 3) / 4;
+    // dk and the <k, H v> terms: rows i, columns r
+    for (int t = threadIdx.x; t < tL * tk; t += blockDim.x) {
+        const int i0 = 4 * (t / tk), r0 = 4 * (t % tk);
+        float hv[4][4], in[4][4];
+        tile44(dv, i0, r0, [&](int i, int cc) { return sV[i * sv + cc]; },
+               [&](int cc, int r) { return r < dk ? sH[r * sv + cc] : 0.f; }, hv);
+        tile44(L, i0, r0, [&](int i, int s) { return s >= i ? pw[s - i] * sDV[s * sc + i] : 0.f; },
+               [&](int s, int r) { return r < dk ? sQ[s * sk + r] : 0.f; }, in);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int i = i0 + u;
+            if (i >= L) continue;
+#pragma unroll
+            for (int w = 0; w < 4; ++w) {
+                const int r = r0 + w;
+                if (r >= dk) continue;
+                const float dkr = pw[L - i] * hv[u][w] + in[u][w];  // dk_i[r] / eta
+                gk[(size_t)i * dk + r] += eta * dkr;
+                p_eta = fmaf(sK[i * sk + r], dkr, p_eta);
+                p_lam = fmaf(eta * (float)(L - 1 - i) * pw[L - 1 - i] * sK[i * sk + r], hv[u][w], p_lam);
+            }
+        }
+    }
+    // dv: rows i, columns cc
+    for (int t = threadIdx.x; t < tL * tv; t += blockDim.x) {
+        const int i0 = 4 * (t / tv), c0 = 4 * (t % tv);
+        float hk[4][4], in[4][4];
+        tile44(dk, i0, c0, [&](int i, int r) { return sK[i * sk + r]; },
+               [&](int r, int cc) { return cc < dv ? sH[r * sv + cc] : 0.f; }, hk);
+        tile44(L, i0, c0, [&](int i, int s) { return s >= i ? pw[s - i] * sQK[s * sc + i] : 0.f; },
+               [&](int s, int cc) { return cc < dv ? sD[s * sv + cc] : 0.f; }, in);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int i = i0 + u;
+            if (i >= L) continue;
+#pragma unroll
+            for (int w = 0; w < 4; ++w)
+                if (c0 + w < dv) gv[(size_t)i * dv + c0 + w] += eta * (pw[L - i] * hk[u][w] + in[u][w]);
+        }
+    }
+    // dq: rows s, columns r
+    for (int t = threadIdx.x; t < tL * tk; t += blockDim.x) {
+        const int s0 = 4 * (t / tk), r0 = 4 * (t % tk);
+        float ad[4][4], in[4][4];
+        tile44(dv, s0, r0, [&](int s, int cc) { return sD[s * sv + cc]; },
+               [&](int cc, int r) { return r < dk ? sA[r * sv + cc] : 0.f; }, ad);
+        tile44(L, s0, r0, [&](int s, int j) { return j <= s ? pw[s - j] * sDV[s * sc + j] : 0.f; },
+               [&](int j, int r) { return r < dk ? sK[j * sk + r] : 0.f; }, in);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int s = s0 + u;
+            if (s >= L) continue;
+#pragma unroll
+            for (int w = 0; w < 4; ++w)
+                if (r0 + w < dk) gq[(size_t)s * dk + r0 + w] += pw[s + 1] * ad[u][w] + eta * in[u][w];
+        }
+    }
+    // m (for dg) and the <qt A, dt> terms: rows s, columns cc
+    for (int t = threadIdx.x; t < tL * tv; t += blockDim.x) {
+        const int s0 = 4 * (t / tv), c0 = 4 * (t % tv);
+        float qa[4][4], in[4][4];
+        tile44(dk, s0, c0, [&](int s, int r) { return sQ[s * sk + r]; },
+               [&](int r, int cc) { return cc < dv ? sA[r * sv + cc] : 0.f; }, qa);
+        tile44(L, s0, c0, [&](int s, int j) { return j <= s ? pw[s - j] * sQK[s * sc + j] : 0.f; },
+               [&](int j, int cc) { return cc < dv ? sV[j * sv + cc] : 0.f; }, in);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int s = s0 + u;
+            if (s >= L) continue;
+#pragma unroll
+            for (int w = 0; w < 4; ++w) {
+                const int cc = c0 + w;
+                if (cc >= dv) continue;
+                const float m = pw[s + 1] * qa[u][w] + eta * in[u][w];
+                p_g = fmaf(sD[s * sv + cc], m, p_g);
+                p_lam = fmaf((float)(s + 1) * pw[s] * qa[u][w], sD[s * sv + cc], p_lam);
+            }
+        }
+    }
+    // the pair terms and <H, A>
+    for (int x = threadIdx.x; x < L * L; x += blockDim.x) {
+        const int s = x / L, j = x % L;
+        if (j < s)
+            p_lam = fmaf(eta * (float)(s - j) * pw[s - 1 - j] * sQK[s * sc + j], sDV[s * sc + j], p_lam);
+    }
+    for (int x = threadIdx.x; x < dk * dv; x += blockDim.x)
+        p_lam = fmaf((float)L * pw[L] * sH[(x / dv) * sv + x % dv], sA[(x / dv) * sv + x % dv], p_lam);
+    p_g *= 1.f - sg;
+    // fixed-order block sum of the three partials
+    p_lam = warp_sum(p_lam);
+    p_eta = warp_sum(p_eta);
+    p_g = warp_sum(p_g);
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    if (lane == 0) {
+        sred[warp * 3] = p_lam;
+        sred[warp * 3 + 1] = p_eta;
+        sred[warp * 3 + 2] = p_g;
+    }
+    __syncthreads();
+    if (threadIdx.x < 3) {
+        float a = 0.f;
+        for (int w = 0; w < kThreads / 32; ++w) a += sred[w * 3 + threadIdx.x];
+        p.part[((size_t)bh * nC + c) * 3 + threadIdx.x] = a;
+    }
+}
+
+__host__ __forceinline__ size_t l2b_chunk_smem(int dk, int dv) {
+    const int C = l2b_chunk(dk, dv);
+    return (size_t)(C * (dk + 1) * 2 + C * (dv + 1) * 2 + 2 * dk * (dv + 1) + 2 * C * (C + 1) + C + 2 +
+                    3 * (kThreads / 32)) * sizeof(float);
+}
+__host__ __forceinline__ size_t l2b_sums_smem(int dk, int dv) {
+    const int C = l2b_chunk(dk, dv);
+    return (size_t)(2 * C * dk + 2 * C * dv + C + 1) * sizeof(float);
+}
+
+// dlam, deta, dg per head: the (b, h, chunk) partials summed over the batch
+// and the chunks in a fixed order (zero when nothing is evicted).
+__global__ void bwd_reduce_kernel(BwdParams p, int nC) {
     const int64_t h = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (h >= p.H) return;
     float a = 0.f, b_ = 0.f, c = 0.f;
     for (int64_t b = 0; b < p.B; ++b)
-        for (int x = 0; x < nrs; ++x) {
-            const float *pp = p.part + ((b * p.H + h) * nrs + x) * 3;
+        for (int x = 0; x < nC; ++x) {
+            const float *pp = p.part + ((b * p.H + h) * nC + x) * 3;
             a += pp[0];
             b_ += pp[1];
             c += pp[2];
@@ -579,20 +735,26 @@ __global__ void bwd_reduce_kernel(BwdParams p, int nrs) {
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
+// Chunks of the memory backward: ceil(E / C) over the E = T - W evictions.
+int64_t l2b_chunks(const tc_prefill_desc &d) {
+    const int64_t E = d.T > d.W ? d.T - d.W : 0;
+    const int C = l2b_chunk((int)d.dk, (int)d.dv);
+    return (E + C - 1) / C;
+}
+
 struct BwdLayout {
-    size_t lse, Dt, ckpt, seg, part, total;
+    size_t lse, Dt, Ac, Hc, part, total;
 };
 BwdLayout bwd_layout(const tc_prefill_desc &d) {
-    const int64_t BH = d.B * d.H, nrs = (d.dk + kRows - 1) / kRows;
-    const int64_t slab = nrs * kRows * d.dv;  // rows of A / G padded to whole CTAs
-    const int64_t nCk = (d.T + kCk - 1) / kCk;
+    const int64_t BH = d.B * d.H, nC = l2b_chunks(d);
+    const size_t mats = (size_t)(BH * nC) * d.dk * d.dv * sizeof(float);
     BwdLayout L;
     L.lse = 0;
     L.Dt = L.lse + align256((size_t)(BH * d.T) * sizeof(float));
-    L.ckpt = L.Dt + align256((size_t)(BH * d.T) * sizeof(float));
-    L.seg = L.ckpt + align256((size_t)(BH * nCk * slab) * sizeof(float));
-    L.part = L.seg + align256((size_t)(BH * kCk * slab) * sizeof(float));
-    L.total = L.part + align256((size_t)(BH * nrs * 3) * sizeof(float));
+    L.Ac = L.Dt + align256((size_t)(BH * d.T) * sizeof(float));
+    L.Hc = L.Ac + align256(mats);
+    L.part = L.Hc + align256(mats);
+    L.total = L.part + align256((size_t)(BH * nC * 3) * sizeof(float));
     return L;
 }
 
@@ -622,32 +784,32 @@ cudaError_t launch_t(const BwdParams &p, cudaStream_t s) {
                                                           : launch_window<Tin, kMaxD / 32>(p, s);
         if (e != cudaSuccess) return e;
     }
-    const int nrs = (p.dk + kRows - 1) / kRows;  // row blocks = CTAs of one cluster (<= 16)
-    const size_t smem =
-        (size_t)(2 * kCk * kRows + 2 * kCk * p.dv + kRows * p.dv + kCk * p.dv) * sizeof(float);
-    cudaError_t e = cudaFuncSetAttribute(bwd_l2_kernel<Tin>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    if (nrs > 8) {
-        e = cudaFuncSetAttribute(bwd_l2_kernel<Tin>,
-                                 cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    // memory part, chunked: sums, scan over the chunks, per-chunk gradients
+    const int C = l2b_chunk(p.dk, p.dv);
+    const int64_t E = p.T > p.W ? p.T - p.W : 0;
+    const int nC = (int)((E + C - 1) / C);
+    cudaError_t e = cudaSuccess;
+    if (nC > 0) {
+        const size_t s_sums = l2b_sums_smem(p.dk, p.dv), s_chunk = l2b_chunk_smem(p.dk, p.dv);
+        e = cudaFuncSetAttribute(l2b_sums_kernel<Tin>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)s_sums);
+        if (e != cudaSuccess) return e;
+        e = cudaFuncSetAttribute(l2b_chunk_kernel<Tin>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)s_chunk);
+        if (e != cudaSuccess) return e;
+        const dim3 grid((unsigned)nC, (unsigned)BH);
+        l2b_sums_kernel<Tin><<<grid, kThreads, s_sums, s>>>(p);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+        l2b_scan_kernel<<<dim3((unsigned)((p.dk * p.dv + kThreads - 1) / kThreads), (unsigned)BH),
+                          kThreads, 0, s>>>(p);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+        l2b_chunk_kernel<Tin><<<grid, kThreads, s_chunk, s>>>(p);
+        e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)nrs, (unsigned)BH);
-    cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = s;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = (unsigned)nrs;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, bwd_l2_kernel<Tin>, p);
-    if (e != cudaSuccess) return e;
-    bwd_reduce_kernel<<<(unsigned)((p.H + 127) / 128), 128, 0, s>>>(p, nrs);
+    bwd_reduce_kernel<<<(unsigned)((p.H + 127) / 128), 128, 0, s>>>(p, nC);
     return cudaGetLastError();
 }
 
@@ -674,8 +836,8 @@ cudaError_t launch_backward(const tc_prefill_desc &d, const void *q, const void 
     p.gv = dv;
     p.lse = reinterpret_cast<float *>(ws + L.lse);
     p.Dt = reinterpret_cast<float *>(ws + L.Dt);
-    p.ckpt = reinterpret_cast<float *>(ws + L.ckpt);
-    p.seg = reinterpret_cast<float *>(ws + L.seg);
+    p.Ac = reinterpret_cast<float *>(ws + L.Ac);
+    p.Hc = reinterpret_cast<float *>(ws + L.Hc);
     p.part = reinterpret_cast<float *>(ws + L.part);
     p.dlam = dlam;
     p.deta = deta;
