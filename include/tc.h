@@ -221,13 +221,20 @@ TC_API tc_status tc_state_fold(int64_t B, int64_t H, int64_t dk, int64_t dv, int
  *   dlambda, deta, dg  [H] float32 (summed over the batch).
  * The pages train lambda, eta and g end to end (§2 training
  * considerations); the formulas are reverse mode through the token loop of
- * Fig. 2.  The window part is the usual softmax backward over the W keys;
- * the memory part is a reverse scan of dL/dA_t, replayed from checkpoints of
- * A every 64 tokens.  q, k, v, dy: device, dtype of desc (dy has y's layout);
- * desc->flags must be 0 (C is not used).  Float32 SIMT kernels; four
- * launches.  Workspace: tc_backward_workspace_size(desc) bytes (about
- * B*H*(2T + d_k'*d_v*(64 + ceil(T/64))) floats, d_k' = d_k rounded up to a
- * multiple of 8).  Errors as tc_prefill. */
+ * Fig. 2.  The window part is the usual softmax backward over the W keys:
+ * for bf16 with d_k = d_v = 64 two tcgen05 kernels (scores and their
+ * gradients in TMEM, P and dS fed back to the tensor cores as bf16 hi + lo
+ * pairs, float32 accumulation), otherwise two float32 SIMT kernels.  The
+ * memory part is the reverse scan of dL/dA_t taken in chunks of 32
+ * evictions (per-chunk sums, a scan over the chunks, per-chunk gradients),
+ * float32.  Every sum has a fixed order: two calls give the same bits.
+ * q, k, v, dy: device, dtype of desc (dy has y's layout); desc->flags must
+ * be 0 (C is not used).  Up to six launches.  Workspace:
+ * tc_backward_workspace_size(desc) bytes (about
+ * B*H*(2 T' + 2 d_k d_v ceil((T-W)/32)) floats, T' = T rounded up to a
+ * multiple of 64).  A bounded wait inside the tensor-core kernels that runs
+ * out leaves TC_ERR_DEVICE_TIMEOUT in the device status word.  Errors as
+ * tc_prefill. */
 TC_API size_t tc_backward_workspace_size(const tc_prefill_desc *desc);
 TC_API tc_status tc_backward(const tc_prefill_desc *desc, const void *q, const void *k,
                              const void *v, const float *lambda, const float *eta, const float *g,

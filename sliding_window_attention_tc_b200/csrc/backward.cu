@@ -1,4 +1,4 @@
-// Backward of the Tensor Cache layer (outer-product write), float32 SIMT.
+// Backward of the Tensor Cache layer (outer-product write).
 //
 // "Tensor Cache: Eviction-conditioned Associative Memory for Transformers":
 // the pages train lambda, eta and g end to end through the chunk scan (§2
@@ -11,9 +11,11 @@
 //   p = softmax(q k / sqrt(dk)), dp_j = <dy_t, v_j>, D_t = <dy_t, y_local_t>,
 //   ds_j = p_j (dp_j - D_t); dq_t += sum_j ds_j k_j / sqrt(dk),
 //   dk_j += ds_j q_t / sqrt(dk), dv_j += p_j dy_t.
-//   bwd_rows_kernel (a warp per 4 query rows) writes dq and the per-row
-//   log-sum-exp and D_t; bwd_keys_kernel (a warp per 4 key rows, over the W
-//   queries that see them) writes dk and dv.
+//   For bf16 with d_k = d_v = 64 two tensor-core kernels do this
+//   (backward_sm100.cu); otherwise, in float32 SIMT, bwd_rows_kernel (a warp
+//   per 4 query rows) writes dq and the per-row log-sum-exp and D_t, and
+//   bwd_keys_kernel (a warp per 4 key rows, over the W queries that see
+//   them) writes dk and dv.
 //
 // Memory (L2), a reverse scan of G_t = dL/dA_t:
 //   G_t = q_t^T (s dy_t) + [step t+1 writes] lam G_{t+1}, and each write at
@@ -55,6 +57,7 @@ struct BwdParams {
     const float *lam, *eta, *g;
     float *gq, *gk, *gv;    // gradients of q, k, v (float32, layout of the inputs)
     float *lse, *Dt;        // [BH][T] per query row (log2 domain), <dy, y_local>
+    int64_t stat_stride;    // row stride of lse, Dt (T, or the tensor-core path's Tp)
     float *Ac, *Hc;         // [BH][nC][dk*dv]: increments, then chunk start states A_c;
                             // summaries, then the G passed back from later chunks H_c
     float *part;            // [BH][nC][3]: dlam, deta, dg partials
@@ -219,8 +222,8 @@ __global__ void __launch_bounds__(kThreads) bwd_rows_kernel(BwdParams p) {
         }
         Dt[i] = warp_sum(d);
         if (t < T && lane == 0) {
-            p.lse[bh * T + t] = lse2[i];
-            p.Dt[bh * T + t] = Dt[i];
+            p.lse[bh * p.stat_stride + t] = lse2[i];
+            p.Dt[bh * p.stat_stride + t] = Dt[i];
         }
     }
     // pass 2: ds_j = p_j (dp_j - D_t); dq_t = sum_j ds_j k_j / sqrt(dk)
@@ -322,8 +325,8 @@ __global__ void __launch_bounds__(kThreads) bwd_keys_kernel(BwdParams p) {
         load_rows(sq, skp, qb, q0, nt, kKT, dk, tid);
         load_rows(sdy, svp, db, q0, nt, kKT, dv, tid);
         if (tid < nt) {
-            slse[tid] = p.lse[bh * T + q0 + tid];
-            sD[tid] = p.Dt[bh * T + q0 + tid];
+            slse[tid] = p.lse[bh * p.stat_stride + q0 + tid];
+            sD[tid] = p.Dt[bh * p.stat_stride + q0 + tid];
         }
         __syncthreads();
         const int64_t t = q0 + lane;
@@ -748,10 +751,11 @@ struct BwdLayout {
 BwdLayout bwd_layout(const tc_prefill_desc &d) {
     const int64_t BH = d.B * d.H, nC = l2b_chunks(d);
     const size_t mats = (size_t)(BH * nC) * d.dk * d.dv * sizeof(float);
+    const size_t stats = (size_t)(BH * backward_stat_stride(d.T)) * sizeof(float);
     BwdLayout L;
     L.lse = 0;
-    L.Dt = L.lse + align256((size_t)(BH * d.T) * sizeof(float));
-    L.Ac = L.Dt + align256((size_t)(BH * d.T) * sizeof(float));
+    L.Dt = L.lse + align256(stats);
+    L.Ac = L.Dt + align256(stats);
     L.Hc = L.Ac + align256(mats);
     L.part = L.Hc + align256(mats);
     L.total = L.part + align256((size_t)(BH * nC * 3) * sizeof(float));
@@ -776,14 +780,10 @@ cudaError_t launch_window(const BwdParams &p, cudaStream_t s) {
     return cudaGetLastError();
 }
 
+// Memory part and the final reduction of the scalar gradients.
 template <typename Tin>
-cudaError_t launch_t(const BwdParams &p, cudaStream_t s) {
+cudaError_t launch_memory(const BwdParams &p, cudaStream_t s) {
     const int64_t BH = p.B * p.H;
-    if (p.T > 0) {
-        const cudaError_t e = (p.dk <= 64 && p.dv <= 64) ? launch_window<Tin, 2>(p, s)
-                                                          : launch_window<Tin, kMaxD / 32>(p, s);
-        if (e != cudaSuccess) return e;
-    }
     // memory part, chunked: sums, scan over the chunks, per-chunk gradients
     const int C = l2b_chunk(p.dk, p.dv);
     const int64_t E = p.T > p.W ? p.T - p.W : 0;
@@ -813,6 +813,24 @@ cudaError_t launch_t(const BwdParams &p, cudaStream_t s) {
     return cudaGetLastError();
 }
 
+// The whole backward: window part (tensor cores where they take the shape),
+// then the memory part.
+template <typename Tin>
+cudaError_t launch_t(const tc_prefill_desc &d, const BwdParams &p, int *status,
+                     unsigned long long wait_ns, cudaStream_t s) {
+    if (p.T > 0) {
+        cudaError_t e;
+        if (backward_window_tc_supported(d))
+            e = launch_backward_window_tc(d, p.q, p.k, p.v, p.dy, p.gq, p.gk, p.gv, p.lse, p.Dt, status,
+                                          wait_ns, s);
+        else
+            e = (p.dk <= 64 && p.dv <= 64) ? launch_window<Tin, 2>(p, s)
+                                           : launch_window<Tin, kMaxD / 32>(p, s);
+        if (e != cudaSuccess) return e;
+    }
+    return launch_memory<Tin>(p, s);
+}
+
 }  // namespace
 
 size_t backward_workspace_bytes(const tc_prefill_desc &d) { return bwd_layout(d).total; }
@@ -820,7 +838,8 @@ size_t backward_workspace_bytes(const tc_prefill_desc &d) { return bwd_layout(d)
 cudaError_t launch_backward(const tc_prefill_desc &d, const void *q, const void *k, const void *v,
                             const float *lam, const float *eta, const float *g, const void *dy,
                             float *dq, float *dk, float *dv, float *dlam, float *deta, float *dg,
-                            void *workspace, cudaStream_t s) {
+                            void *workspace, int *status, unsigned long long wait_ns,
+                            cudaStream_t s) {
     const BwdLayout L = bwd_layout(d);
     char *ws = static_cast<char *>(workspace);
     BwdParams p{};
@@ -848,7 +867,14 @@ cudaError_t launch_backward(const tc_prefill_desc &d, const void *q, const void 
     p.W = d.W;
     p.dk = (int)d.dk;
     p.dv = (int)d.dv;
-    return d.dtype == TC_BF16 ? launch_t<__nv_bfloat16>(p, s) : launch_t<float>(p, s);
+    p.stat_stride = backward_window_tc_supported(d) ? backward_stat_stride(d.T) : d.T;
+    return d.dtype == TC_BF16 ? launch_t<__nv_bfloat16>(d, p, status, wait_ns, s)
+                              : launch_t<float>(d, p, status, wait_ns, s);
+}
+
+int backward_launch_count(const tc_prefill_desc &d) {
+    const int window = d.T > 0 ? 2 : 0;
+    return window + (l2b_chunks(d) > 0 ? 3 : 0) + 1;
 }
 
 }  // namespace tc

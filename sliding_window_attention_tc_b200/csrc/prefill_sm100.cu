@@ -1304,19 +1304,7 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t
                                   const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
-EncodeTiledFn encode_fn() {
-    static EncodeTiledFn fn = nullptr;
-    if (!fn) {
-        cudaDriverEntryPointQueryResult q;
-        void *ptr = nullptr;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) !=
-                cudaSuccess ||
-            q != cudaDriverEntryPointSuccess)
-            return nullptr;
-        fn = reinterpret_cast<EncodeTiledFn>(ptr);
-    }
-    return fn;
-}
+EncodeTiledFn encode_fn() { return reinterpret_cast<EncodeTiledFn>(tensor_map_encoder()); }
 
 // [BH][T][64] bf16 -> 3D map with 64 x 128 x 1 boxes, 128-byte swizzle;
 // rows past T read as zero.
@@ -1370,6 +1358,20 @@ int choose_spans(int64_t BH, int nT, int num_sms) {
 }
 
 }  // namespace
+
+void *tensor_map_encoder() {
+    static void *fn = nullptr;
+    if (!fn) {
+        cudaDriverEntryPointQueryResult q;
+        void *ptr = nullptr;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) !=
+                cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return nullptr;
+        fn = ptr;
+    }
+    return fn;
+}
 
 bool sm100_supported(const tc_prefill_desc &d, int64_t n_halo) {
     return d.dtype == TC_BF16 && d.dk == HD && d.dv == HD && d.W >= BM && d.W % BM == 0 &&

@@ -365,7 +365,8 @@ tc_status tc_backward(const tc_prefill_desc *d, const void *q, const void *k, co
         if (!is_device_ptr(x, dev)) return TC_ERR_INVALID_ARG;
     if (need > 0 && !is_device_ptr(workspace, dev)) return TC_ERR_INVALID_ARG;
     cudaError_t e = tc::launch_backward(*d, q, k, v, lambda, eta, g, dy, dq, dk, dv, dlambda, deta,
-                                        dg, workspace, reinterpret_cast<cudaStream_t>(stream));
+                                        dg, workspace, status_ptr(), wait_limit_ns(),
+                                        reinterpret_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? TC_OK : TC_ERR_CUDA;
 }
 

@@ -114,12 +114,30 @@ bool decode_supported(int dk, int dv, tc_dtype dtype);
 size_t portable_workspace_bytes(const tc_prefill_desc &d, int64_t n_halo);
 cudaError_t launch_prefill_portable(const PrefillParams &p, tc_dtype dtype, cudaStream_t s);
 
-// backward.cu: gradients of the layer (outer-product write), float32 SIMT.
+// backward.cu: gradients of the layer (outer-product write); the window part
+// on the tensor cores where backward_sm100.cu takes the shape, else float32
+// SIMT; the memory part as a float32 chunk scan.
 size_t backward_workspace_bytes(const tc_prefill_desc &d);
 cudaError_t launch_backward(const tc_prefill_desc &d, const void *q, const void *k, const void *v,
                             const float *lam, const float *eta, const float *g, const void *dy,
                             float *dq, float *dk, float *dv, float *dlam, float *deta, float *dg,
-                            void *workspace, cudaStream_t s);
+                            void *workspace, int *status, unsigned long long wait_ns,
+                            cudaStream_t s);
+// Kernels of one backward call.
+int backward_launch_count(const tc_prefill_desc &d);
+
+// backward_sm100.cu: window part of the backward, tcgen05 / TMA (bf16, d = 64).
+// dq, dk, dv are written (not accumulated); lse and Dt ([BH][Tp] float32,
+// Tp = backward_stat_stride(T)) receive the per-query statistics.
+bool backward_window_tc_supported(const tc_prefill_desc &d);
+int64_t backward_stat_stride(int64_t T);
+cudaError_t launch_backward_window_tc(const tc_prefill_desc &d, const void *q, const void *k,
+                                      const void *v, const void *dy, float *dq, float *dk, float *dv,
+                                      float *lse, float *Dt, int *status, unsigned long long wait_ns,
+                                      cudaStream_t s);
+
+// cuTensorMapEncodeTiled from the driver (null if unavailable).
+void *tensor_map_encoder();
 
 // prefill_sm100.cu: tcgen05 / TMA path for bf16, d_k = d_v = 64.
 bool sm100_supported(const tc_prefill_desc &d, int64_t n_halo);

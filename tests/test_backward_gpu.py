@@ -25,8 +25,12 @@ CASES = [
     (1, 2, 300, 32, 32, 64, "f32"),
     (1, 1, 100, 16, 8, 5, "f32"),       # d_k != d_v
     (1, 2, 40, 16, 16, 64, "f32"),      # T < W: no eviction, L2 gradients of lambda, eta are 0
-    (1, 2, 300, 64, 64, 128, "bf16"),   # checkpoints in several segments
-    (1, 2, 200, 128, 128, 64, "bf16"),  # d = 128: 16 row blocks per head in one cluster
+    (1, 2, 300, 64, 64, 128, "bf16"),   # bf16, d = 64: tensor-core window part
+    (2, 3, 1000, 64, 64, 200, "bf16"),  # W not a multiple of the 64-row tiles, ragged T
+    (1, 2, 77, 64, 64, 512, "bf16"),    # W > T, one partial 128-row block
+    (1, 1, 700, 64, 64, 1, "bf16"),     # W = 1: every key its own query only
+    (1, 2, 2100, 64, 64, 512, "bf16"),  # many tiles per block, 2 blocks per SM
+    (1, 2, 200, 128, 128, 64, "bf16"),  # d = 128: SIMT window kernels, 4 columns per lane
     (1, 1, 150, 128, 40, 16, "f32"),    # d_k = 128, d_v not a multiple of 32
 ]
 
