@@ -47,10 +47,11 @@ constexpr int kMaxD = 128;
 constexpr int kKT = 32;               // key / query tile of the L1 kernels
 constexpr float kLog2e = 1.4426950408889634f;
 
-// Evictions per chunk of the memory backward.  32 keeps l2b_chunk_kernel at
-// about 75 KB of shared memory for d = 64 (three CTAs per SM) and its
-// triangular in-chunk work small; the scan over chunks is cheap either way.
-__host__ __device__ __forceinline__ int l2b_chunk(int, int) { return 32; }
+// Evictions per chunk of the memory backward.  The tensor-core chunk kernel
+// (bf16, d = 64) takes 128, one MMA tile of rows.  The SIMT one takes 32,
+// which keeps it at about 75 KB of shared memory for d = 64 (three CTAs per
+// SM) and its triangular in-chunk work small.
+int l2b_chunk(const tc_prefill_desc &d) { return backward_memory_tc_supported(d) ? 128 : 32; }
 
 struct BwdParams {
     const void *q, *k, *v, *dy;
@@ -64,6 +65,7 @@ struct BwdParams {
     float *dlam, *deta, *dg;
     int64_t B, H, T, W;
     int dk, dv;
+    int C;                  // evictions per chunk of the memory part
 };
 
 __device__ __forceinline__ float warp_max(float x) {
@@ -442,7 +444,7 @@ __device__ __forceinline__ void tile44(int K, int m0, int n0, FA a, FB b, float 
 template <typename Tin>
 __global__ void __launch_bounds__(kThreads) l2b_sums_kernel(BwdParams p) {
     extern __shared__ float sh[];
-    const int dk = p.dk, dv = p.dv, C = l2b_chunk(dk, dv);
+    const int dk = p.dk, dv = p.dv, C = p.C;
     const int64_t bh = blockIdx.y, T = p.T, W = p.W, E = T - W;
     const int c = blockIdx.x, h = (int)(bh % p.H);
     const int64_t e0 = (int64_t)c * C;
@@ -491,7 +493,7 @@ __global__ void __launch_bounds__(kThreads) l2b_sums_kernel(BwdParams p) {
 constexpr int kScanBatch = 8;
 __global__ void __launch_bounds__(kThreads) l2b_scan_kernel(BwdParams p) {
     __shared__ float decay[2];  // lam^C, lam^(length of the last chunk)
-    const int dk = p.dk, dv = p.dv, C = l2b_chunk(dk, dv);
+    const int dk = p.dk, dv = p.dv, C = p.C;
     const int64_t bh = blockIdx.y, E = p.T - p.W;
     const int nC = (int)((E + C - 1) / C);
     if (threadIdx.x < 2) {
@@ -551,7 +553,7 @@ __global__ void __launch_bounds__(kThreads) l2b_scan_kernel(BwdParams p) {
 template <typename Tin>
 __global__ void __launch_bounds__(kThreads) l2b_chunk_kernel(BwdParams p) {
     extern __shared__ float sh[];
-    const int dk = p.dk, dv = p.dv, C = l2b_chunk(dk, dv);
+    const int dk = p.dk, dv = p.dv, C = p.C;
     const int sk = dk + 1, sv = dv + 1, sc = C + 1;  // padded strides
     const int64_t bh = blockIdx.y, T = p.T, W = p.W, E = T - W;
     const int c = blockIdx.x, h = (int)(bh % p.H);
@@ -708,13 +710,11 @@ __global__ void __launch_bounds__(kThreads) l2b_chunk_kernel(BwdParams p) {
     }
 }
 
-__host__ __forceinline__ size_t l2b_chunk_smem(int dk, int dv) {
-    const int C = l2b_chunk(dk, dv);
+__host__ __forceinline__ size_t l2b_chunk_smem(int dk, int dv, int C) {
     return (size_t)(C * (dk + 1) * 2 + C * (dv + 1) * 2 + 2 * dk * (dv + 1) + 2 * C * (C + 1) + C + 2 +
                     3 * (kThreads / 32)) * sizeof(float);
 }
-__host__ __forceinline__ size_t l2b_sums_smem(int dk, int dv) {
-    const int C = l2b_chunk(dk, dv);
+__host__ __forceinline__ size_t l2b_sums_smem(int dk, int dv, int C) {
     return (size_t)(2 * C * dk + 2 * C * dv + C + 1) * sizeof(float);
 }
 
@@ -741,7 +741,7 @@ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 // Chunks of the memory backward: ceil(E / C) over the E = T - W evictions.
 int64_t l2b_chunks(const tc_prefill_desc &d) {
     const int64_t E = d.T > d.W ? d.T - d.W : 0;
-    const int C = l2b_chunk((int)d.dk, (int)d.dv);
+    const int C = l2b_chunk(d);
     return (E + C - 1) / C;
 }
 
@@ -782,31 +782,45 @@ cudaError_t launch_window(const BwdParams &p, cudaStream_t s) {
 
 // Memory part and the final reduction of the scalar gradients.
 template <typename Tin>
-cudaError_t launch_memory(const BwdParams &p, cudaStream_t s) {
+cudaError_t launch_memory(const tc_prefill_desc &d, const BwdParams &p, int *status,
+                          unsigned long long wait_ns, cudaStream_t s) {
     const int64_t BH = p.B * p.H;
     // memory part, chunked: sums, scan over the chunks, per-chunk gradients
-    const int C = l2b_chunk(p.dk, p.dv);
+    const int C = p.C;
     const int64_t E = p.T > p.W ? p.T - p.W : 0;
     const int nC = (int)((E + C - 1) / C);
+    const bool tc_chunk = backward_memory_tc_supported(d);
     cudaError_t e = cudaSuccess;
     if (nC > 0) {
-        const size_t s_sums = l2b_sums_smem(p.dk, p.dv), s_chunk = l2b_chunk_smem(p.dk, p.dv);
-        e = cudaFuncSetAttribute(l2b_sums_kernel<Tin>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)s_sums);
-        if (e != cudaSuccess) return e;
-        e = cudaFuncSetAttribute(l2b_chunk_kernel<Tin>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)s_chunk);
-        if (e != cudaSuccess) return e;
+        const size_t s_sums = l2b_sums_smem(p.dk, p.dv, C), s_chunk = l2b_chunk_smem(p.dk, p.dv, C);
+        if (!tc_chunk) {
+            e = cudaFuncSetAttribute(l2b_sums_kernel<Tin>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)s_sums);
+            if (e != cudaSuccess) return e;
+            e = cudaFuncSetAttribute(l2b_chunk_kernel<Tin>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)s_chunk);
+            if (e != cudaSuccess) return e;
+        }
         const dim3 grid((unsigned)nC, (unsigned)BH);
-        l2b_sums_kernel<Tin><<<grid, kThreads, s_sums, s>>>(p);
-        e = cudaGetLastError();
+        if (tc_chunk) {
+            e = launch_backward_sums_tc(d, p.q, p.k, p.v, p.dy, p.lam, p.eta, p.g, p.Ac, p.Hc, status,
+                                        wait_ns, s);
+        } else {
+            l2b_sums_kernel<Tin><<<grid, kThreads, s_sums, s>>>(p);
+            e = cudaGetLastError();
+        }
         if (e != cudaSuccess) return e;
         l2b_scan_kernel<<<dim3((unsigned)((p.dk * p.dv + kThreads - 1) / kThreads), (unsigned)BH),
                           kThreads, 0, s>>>(p);
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
-        l2b_chunk_kernel<Tin><<<grid, kThreads, s_chunk, s>>>(p);
-        e = cudaGetLastError();
+        if (tc_chunk) {
+            e = launch_backward_chunks_tc(d, p.q, p.k, p.v, p.dy, p.lam, p.eta, p.g, p.Ac, p.Hc, p.gq,
+                                          p.gk, p.gv, p.part, status, wait_ns, s);
+        } else {
+            l2b_chunk_kernel<Tin><<<grid, kThreads, s_chunk, s>>>(p);
+            e = cudaGetLastError();
+        }
         if (e != cudaSuccess) return e;
     }
     bwd_reduce_kernel<<<(unsigned)((p.H + 127) / 128), 128, 0, s>>>(p, nC);
@@ -828,7 +842,7 @@ cudaError_t launch_t(const tc_prefill_desc &d, const BwdParams &p, int *status,
                                            : launch_window<Tin, kMaxD / 32>(p, s);
         if (e != cudaSuccess) return e;
     }
-    return launch_memory<Tin>(p, s);
+    return launch_memory<Tin>(d, p, status, wait_ns, s);
 }
 
 }  // namespace
@@ -868,6 +882,7 @@ cudaError_t launch_backward(const tc_prefill_desc &d, const void *q, const void 
     p.dk = (int)d.dk;
     p.dv = (int)d.dv;
     p.stat_stride = backward_window_tc_supported(d) ? backward_stat_stride(d.T) : d.T;
+    p.C = l2b_chunk(d);
     return d.dtype == TC_BF16 ? launch_t<__nv_bfloat16>(d, p, status, wait_ns, s)
                               : launch_t<float>(d, p, status, wait_ns, s);
 }

@@ -136,6 +136,24 @@ cudaError_t launch_backward_window_tc(const tc_prefill_desc &d, const void *q, c
                                       float *lse, float *Dt, int *status, unsigned long long wait_ns,
                                       cudaStream_t s);
 
+// Memory part of the backward, per chunk of 128 evictions on the tensor cores
+// (bf16, d = 64).  launch_backward_sums_tc writes each chunk's state
+// increment and gradient summary into Ac, Hc ([BH][nC][64][64] float32); after
+// the scan over chunks these hold each chunk's start state A_c and the G
+// passed back from the later chunks H_c, from which launch_backward_chunks_tc
+// adds the chunk's contributions to dq, dk, dv and writes its partials of
+// dlambda, deta, dg into part [BH][nC][3].
+bool backward_memory_tc_supported(const tc_prefill_desc &d);
+cudaError_t launch_backward_sums_tc(const tc_prefill_desc &d, const void *q, const void *k, const void *v,
+                                    const void *dy, const float *lam, const float *eta, const float *g,
+                                    float *Ac, float *Hc, int *status, unsigned long long wait_ns,
+                                    cudaStream_t s);
+cudaError_t launch_backward_chunks_tc(const tc_prefill_desc &d, const void *q, const void *k,
+                                      const void *v, const void *dy, const float *lam,
+                                      const float *eta, const float *g, const float *Ac,
+                                      const float *Hc, float *dq, float *dk, float *dv, float *part,
+                                      int *status, unsigned long long wait_ns, cudaStream_t s);
+
 // cuTensorMapEncodeTiled from the driver (null if unavailable).
 void *tensor_map_encoder();
 
