@@ -401,30 +401,40 @@ def time_calls(fn, steps, warmup):
     return [a.elapsed_time(b) for a, b in ev]
 
 
-# float32 FMA peak of the SIMT kernels (backward, delta rule): 148 SMs x 128
-# FMA lanes x 2 FLOP x 1965 MHz, the nominal unit count and clock.
-FP32_SIMT_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+def backward_flops(B, H, T, d, W):
+    """Algorithmic FLOPs of one backward call: the window part takes five
+    products per (query, key in window) pair (scores and dP recomputed, dV,
+    dK, dQ) against the forward's two; the memory part twice the forward's
+    write + read (the state's and its gradient's scans)."""
+    l1, l2 = prefill_flops(B, H, T, d, d, W)
+    return 2.5 * l1 + 2 * l2
 
 
-def time_training_extras(tc, dev):
-    """The backward pass and the delta-rule prefill on the LM workload (both
-    float32 SIMT paths): ms per call and tokens/s."""
+def time_training_extras(tc, dev, peaks=None, peak_src="fallback", steps=5):
+    """The backward pass (tensor-core window and memory parts for bf16, d = 64)
+    and the delta-rule prefill (float32 SIMT, token-sequential memory) on the
+    LM workload: ms per call and tokens/s."""
+    peaks = peaks or dict(PEAKS_FALLBACK)
     x, sets, prm = _prefill_device_inputs(HEADLINE, dev, copies=1)
     q, k, v = sets[0]
     B, H, T, d = q.shape
     gen = torch.Generator(device=dev).manual_seed(7)
     dy = (torch.randn(B, H, T, d, generator=gen, device=dev) / 8).to(q.dtype)
     out = {}
-    l1f, l2f = prefill_flops(B, H, T, d, d, x.W)
-    bwd_ms = statistics.median(time_calls(lambda: tc.backward(q, k, v, *prm, x.W, dy), 3, 1))
-    # algorithmic work of the backward: twice the forward's (the usual count
-    # for an attention backward: scores recomputed, dq, dk, dv)
-    tf = 2 * (l1f + l2f) / (bwd_ms * 1e-3) / 1e12
+    bwd_ms = statistics.median(time_calls(lambda: tc.backward(q, k, v, *prm, x.W, dy), steps, 3))
+    fl = backward_flops(B, H, T, d, x.W)
+    tf = fl / (bwd_ms * 1e-3) / 1e12
+    peak_tf = float(peaks["bf16_tflops"])
     out["backward"] = {"workload": HEADLINE, "ms": bwd_ms, "tokens_per_s": B * H * T / (bwd_ms * 1e-3),
-                       "roofline": {"bound": "alu", "achieved": tf, "peak": FP32_SIMT_PEAK_TFLOPS,
-                                    "unit": "TFLOP/s", "frac": tf / FP32_SIMT_PEAK_TFLOPS,
-                                    "traffic": None, "peak_source": "nominal fp32 FMA rate",
-                                    "algorithmic_flops_per_call": 2 * (l1f + l2f)}}
+                       "launches_per_call": tc.backward_launch_count(q, x.W)[0],
+                       "tensor_cores": tc.backward_launch_count(q, x.W)[1],
+                       "roofline": {"bound": "tensor", "achieved": tf, "peak": peak_tf,
+                                    "unit": "TFLOP/s", "frac": tf / peak_tf, "traffic": None,
+                                    "peak_source": f"{peak_src} bf16 burst",
+                                    "algorithmic_flops_per_call": fl,
+                                    "note": "P, dS and the float32 states enter the tensor cores "
+                                            "as bf16 hi + lo pairs, so the executed work is "
+                                            "about twice the algorithmic"}}
     delta_ms = statistics.median(time_calls(
         lambda: tc.prefill(q, k, v, *prm, x.W, x.C, delta_rule=True), 3, 1))
     out["delta_rule_prefill"] = {"workload": HEADLINE, "ms": delta_ms,
@@ -577,6 +587,10 @@ def run_only(args, tc, dev, world, peaks):
     if args.only == "varlen":
         print(json.dumps({"only": "varlen", **time_varlen(tc, dev, args.steps, args.warmup)}))
         return 0
+    if args.only == "backward":
+        print(json.dumps({"only": "backward",
+                          **time_training_extras(tc, dev, peaks, steps=args.steps)["backward"]}))
+        return 0
     name = HEADLINE if args.only == "prefill" else "long_prefill_bf16"
     r = time_prefill(tc, name, dev, args.steps, args.warmup, world)
     x = r["x"]
@@ -598,7 +612,7 @@ def main():
     ap.add_argument("--impl", default="tc", choices=["tc", "reference"])
     ap.add_argument("--no-extras", action="store_true",
                     help="headline prefill only (skip decode, long prefill, oracle)")
-    ap.add_argument("--only", choices=["prefill", "long", "decode", "varlen"], default=None,
+    ap.add_argument("--only", choices=["prefill", "long", "decode", "varlen", "backward"], default=None,
                     help="time one workload only and print its numbers (profiling runs)")
     ap.add_argument("--decode-batch", type=int, default=None,
                     help="batch of the decode workload (default 256)")
@@ -692,7 +706,7 @@ def main():
                         "h2d_bytes_per_step": dec["e2e_h2d_bytes"],
                         "d2h_bytes_per_step": dec["e2e_d2h_bytes"]}}
             extras["varlen_prefill"] = time_varlen(tc, dev)
-            extras.update(time_training_extras(tc, dev))
+            extras.update(time_training_extras(tc, dev, peaks, peak_src))
         e2e = time_prefill_e2e(tc, HEADLINE, dev, max(5, min(20, args.steps // 10)))
     finally:
         clocks.stop()

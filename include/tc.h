@@ -242,6 +242,13 @@ TC_API tc_status tc_backward(const tc_prefill_desc *desc, const void *q, const v
                              float *deta, float *dg, void *workspace, size_t workspace_bytes,
                              tc_stream_t stream);
 
+/* Number of kernel launches one tc_backward call enqueues for desc, or -1
+ * when desc is NULL, invalid or has flags set.  When tensor_cores is not
+ * NULL it receives 1 if the call runs the tcgen05 kernels (bf16,
+ * d_k = d_v = 64, on a device that has them) and 0 for the float32 SIMT
+ * kernels. */
+TC_API int tc_backward_launch_count(const tc_prefill_desc *desc, int *tensor_cores);
+
 /* Number of kernel launches one tc_prefill call enqueues for desc on the
  * current device (the path depends on shapes and dtype), or -1 when desc is
  * NULL or invalid.  tc_decode_step always enqueues exactly one. */

@@ -50,7 +50,8 @@ EXPORTED = ("tc_prefill_workspace_size", "tc_prefill", "tc_prefill_launch_count"
             "tc_decode_step_host", "tc_get_device_status", "tc_status_string", "tc_version",
             "tc_prefill_no_alloc", "tc_prefill_from_state", "tc_prefill_from_state_workspace_size",
             "tc_state_fold", "tc_decode_step_ragged", "tc_backward", "tc_backward_workspace_size",
-            "tc_set_wait_limit_ns", "tc_prefill_varlen", "tc_prefill_varlen_workspace_size")
+            "tc_set_wait_limit_ns", "tc_prefill_varlen", "tc_prefill_varlen_workspace_size",
+            "tc_backward_launch_count")
 
 
 class PrefillDesc(ctypes.Structure):
@@ -75,6 +76,8 @@ _lib.tc_prefill_workspace_size.argtypes = [_PD]
 _lib.tc_prefill_workspace_size.restype = _sz
 _lib.tc_prefill.argtypes = [_PD] + [_vp] * 9 + [_sz, _vp]
 _lib.tc_prefill.restype = _int
+_lib.tc_backward_launch_count.argtypes = [_PD, ctypes.POINTER(_int)]
+_lib.tc_backward_launch_count.restype = _int
 _lib.tc_prefill_launch_count.argtypes = [_PD]
 _lib.tc_prefill_launch_count.restype = _int
 _lib.tc_prefill_host_workspace_size.argtypes = [_PD]
@@ -412,6 +415,19 @@ def backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, lam: torch.Tenso
                           _ptr(dg_), _ptr(workspace), ws_bytes, _stream(stream))
     _check(st, "tc_backward")
     return dq, dkk, dvv, dl, de, dg_
+
+
+def backward_launch_count(q: torch.Tensor, W: int, v: Optional[torch.Tensor] = None):
+    """(launches, tensor_cores) of one tc_backward call on tensors shaped like
+    q [B,H,T,d_k] (and v [B,H,T,d_v], default q's shape) with window W."""
+    B, H, T, dk = q.shape
+    dv = dk if v is None else v.shape[-1]
+    desc = make_prefill_desc(B, H, T, dk, dv, W, 1, _dtype_code(q))
+    tcf = _int(0)
+    n = _lib.tc_backward_launch_count(ctypes.byref(desc), ctypes.byref(tcf))
+    if n < 0:
+        raise TCError(1, "tc_backward_launch_count")
+    return int(n), bool(tcf.value)
 
 
 def prefill_launch_count(desc: PrefillDesc) -> int:

@@ -417,28 +417,6 @@ __device__ __forceinline__ void stage_rows(float *dst, int sp, const Tin *src, i
     }
 }
 
-// One 4 x 4 block of out[m][n] = sum_k a(m, k) b(k, n) in registers (m0, n0
-// its corner; a and b return 0 outside the ranges they cover).  Each operand
-// loaded from shared memory serves four products.
-template <class FA, class FB>
-__device__ __forceinline__ void tile44(int K, int m0, int n0, FA a, FB b, float (&acc)[4][4]) {
-#pragma unroll
-    for (int u = 0; u < 4; ++u)
-#pragma unroll
-        for (int w = 0; w < 4; ++w) acc[u][w] = 0.f;
-    for (int k = 0; k < K; ++k) {
-        float av[4], bv[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) av[u] = a(m0 + u, k);
-#pragma unroll
-        for (int w = 0; w < 4; ++w) bv[w] = b(k, n0 + w);
-#pragma unroll
-        for (int u = 0; u < 4; ++u)
-#pragma unroll
-            for (int w = 0; w < 4; ++w) acc[u][w] = fmaf(av[u], bv[w], acc[u][w]);
-    }
-}
-
 // Per chunk: the state increment dA_c = sum_i eta lam^(L-1-i) k_i v_i^T (into
 // Ac) and the summary X_c = sum_s lam^s qt_s^T dt_s (into Hc).
 template <typename Tin>

@@ -1,0 +1,392 @@
+// Delta-rule write (Fig. 2 step (3) of "Tensor Cache: Eviction-conditioned
+// Associative Memory for Transformers", with the error-correcting update
+// k_old (v_old - k_old^T A)^T) taken in chunks instead of token by token.
+//
+// Chunk c holds evictions e0 .. e0+L-1 (L <= CD), local index i, and S is the
+// state before its first write.  With the error u_i = v_i - A_{i-1}^T k_i the
+// write is A_i = lam A_{i-1} + eta k_i u_i^T, so
+//   A_i = lam^(i+1) S + eta sum_{l<=i} lam^(i-l) k_l u_l^T,
+// and the errors solve a unit lower-triangular system,
+//   u_i + eta sum_{l<i} lam^(i-1-l) (k_i . k_l) u_l = v_i - lam^i S^T k_i,
+// i.e. (I + N) U = V - D K S with D = diag(lam^i).  Its solution splits as
+// U = Ut - Wt S with Ut = (I + N)^-1 V and Wt = (I + N)^-1 D K, neither of
+// which depends on S, and the chunk maps its start state affinely,
+//   S' = lam^L S + eta K^T G U = P S + Q,   G = diag(lam^(L-1-l)),
+//   P = lam^L I - eta K^T G Wt,   Q = eta K^T G Ut.
+// Three kernels: delta_prep_kernel solves for Ut, Wt and forms P, Q (every
+// chunk at once); delta_scan_kernel runs S_{c+1} = P_c S_c + Q_c per head
+// (the only sequential part, one 64 x 64 product per chunk); and
+// delta_read_kernel forms U and the reads of the chunk's rows,
+//   m_i = q'_i A_i = lam^(i+1) q'_i S + eta sum_{l<=i} lam^(i-l) (q'_i . k_l) u_l,
+// with q'_i the query at t = e0 + i + W.  float32 SIMT; no halo (a call that
+// continues a sequence takes the token-order kernel).
+
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "tc.h"
+#include "tc_internal.cuh"
+
+namespace tc {
+namespace {
+
+constexpr int CD = 64;         // evictions per chunk
+constexpr int kDThreads = 256;
+constexpr int kSB = 16;        // rows per block of the forward substitution
+
+struct DeltaBufs {
+    float *Ut, *Wt;  // [BH][E][dv], [BH][E][dk]
+    float *P, *Q;    // [BH][nC][dk][dk], [BH][nC][dk][dv]
+    float *S;        // [BH][nC][dk][dv]: start state of every chunk
+    int64_t E, nC;
+};
+
+size_t al256(size_t x) { return (x + 255) & ~size_t(255); }
+
+struct DeltaLayout {
+    size_t mrow, Ut, Wt, P, Q, S, total;
+};
+DeltaLayout delta_layout(const tc_prefill_desc &d) {
+    const int64_t BH = d.B * d.H, E = d.T > d.W ? d.T - d.W : 0, nC = (E + CD - 1) / CD;
+    const bool reads = !(d.flags & TC_PREFILL_STATE_ONLY);
+    DeltaLayout L;
+    L.mrow = 0;
+    L.Ut = L.mrow + (reads ? al256((size_t)(BH * d.T * d.dv) * sizeof(float)) : 0);
+    L.Wt = L.Ut + al256((size_t)(BH * E * d.dv) * sizeof(float));
+    L.P = L.Wt + al256((size_t)(BH * E * d.dk) * sizeof(float));
+    L.Q = L.P + al256((size_t)(BH * nC * d.dk * d.dk) * sizeof(float));
+    L.S = L.Q + al256((size_t)(BH * nC * d.dk * d.dv) * sizeof(float));
+    L.total = L.S + al256((size_t)(BH * nC * d.dk * d.dv) * sizeof(float));
+    return L;
+}
+
+// lam^n for n = 0 .. n_max (lam^0 = 1 also for lam = 0).
+__device__ __forceinline__ void powers(float *pw, int n_max, float lam) {
+    const double l2l = log2((double)lam);
+    for (int n = threadIdx.x; n <= n_max; n += blockDim.x) pw[n] = n == 0 ? 1.f : (float)exp2((double)n * l2l);
+}
+
+// rows r0 .. r0+n_valid-1 of a [.][d] tensor into shared rows of stride sp,
+// scaled by scale(row); rows n_valid .. CD-1 are zero.
+template <typename Tin, class F>
+__device__ __forceinline__ void load_rows_scaled(float *dst, int sp, const Tin *src, int64_t r0, int n_valid, int d,
+                                                 F scale) {
+    for (int x = threadIdx.x; x < CD * d; x += blockDim.x) {
+        const int i = x / d, c = x % d;
+        dst[i * sp + c] = i < n_valid ? scale(i) * to_f32(src[(r0 + i) * d + c]) : 0.f;
+    }
+}
+
+template <typename Tin>
+__global__ void __launch_bounds__(kDThreads) delta_prep_kernel(PrefillParams p, DeltaBufs w) {
+    extern __shared__ float sh[];
+    const int dk = p.dk, dv = p.dv, nx = dv + dk;
+    const int skp = dk + 1, sxp = nx + 1;
+    float *sK = sh, *X = sK + CD * skp, *sN = X + CD * sxp, *pw = sN + CD * (CD + 1);
+    const int64_t bh = blockIdx.y, T = p.T, E = w.E;
+    const int c = blockIdx.x, h = (int)(bh % p.H);
+    const int64_t e0 = (int64_t)c * CD;
+    const int L = (int)(E - e0 < CD ? E - e0 : CD);
+    const float eta = p.eta[h];
+    powers(pw, CD, p.lam[h]);
+    __syncthreads();
+    const Tin *kb = reinterpret_cast<const Tin *>(p.k) + bh * T * dk;
+    const Tin *vb = reinterpret_cast<const Tin *>(p.v) + bh * T * dv;
+    load_rows_scaled(sK, skp, kb, e0, L, dk, [](int) { return 1.f; });
+    load_rows_scaled(X, sxp, vb, e0, L, dv, [](int) { return 1.f; });
+    load_rows_scaled(X + dv, sxp, kb, e0, L, dk, [&](int i) { return pw[i]; });
+    __syncthreads();
+    // N[i][l] = eta lam^(i-1-l) (k_i . k_l) for l < i < L
+    for (int t = threadIdx.x; t < (CD / 4) * (CD / 4); t += blockDim.x) {
+        const int i0 = 4 * (t / (CD / 4)), l0 = 4 * (t % (CD / 4));
+        float acc[4][4];
+        tile44(dk, i0, l0, [&](int i, int r) { return sK[i * skp + r]; },
+               [&](int r, int l) { return sK[l * skp + r]; }, acc);
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+                const int i = i0 + u, l = l0 + v;
+                sN[i * (CD + 1) + l] = (l < i && i < L) ? eta * pw[i - 1 - l] * acc[u][v] : 0.f;
+            }
+    }
+    __syncthreads();
+    // forward substitution X_i -= sum_{l<i} N[i][l] X_l in blocks of kSB rows:
+    // the earlier blocks' part of a block is one parallel product, then the
+    // block's rows go one by one over at most kSB - 1 earlier rows each
+    for (int b0 = 0; b0 < L; b0 += kSB) {
+        if (b0 > 0) {
+            for (int x = threadIdx.x; x < kSB * nx; x += blockDim.x) {
+                const int i = b0 + x / nx, col = x % nx;
+                float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+                for (int l = 0; l < b0; l += 4) {
+                    a0 = fmaf(sN[i * (CD + 1) + l], X[l * sxp + col], a0);
+                    a1 = fmaf(sN[i * (CD + 1) + l + 1], X[(l + 1) * sxp + col], a1);
+                    a2 = fmaf(sN[i * (CD + 1) + l + 2], X[(l + 2) * sxp + col], a2);
+                    a3 = fmaf(sN[i * (CD + 1) + l + 3], X[(l + 3) * sxp + col], a3);
+                }
+                X[i * sxp + col] -= (a0 + a1) + (a2 + a3);
+            }
+            __syncthreads();
+        }
+        const int b1 = b0 + kSB < L ? b0 + kSB : L;
+        for (int i = b0 + 1; i < b1; ++i) {
+            for (int col = threadIdx.x; col < nx; col += blockDim.x) {
+                float a = X[i * sxp + col];
+                for (int l = b0; l < i; ++l) a = fmaf(-sN[i * (CD + 1) + l], X[l * sxp + col], a);
+                X[i * sxp + col] = a;
+            }
+            __syncthreads();
+        }
+    }
+    // Ut, Wt rows
+    float *Ut = w.Ut + (bh * E + e0) * dv, *Wt = w.Wt + (bh * E + e0) * dk;
+    for (int x = threadIdx.x; x < L * dv; x += blockDim.x) Ut[x] = X[(x / dv) * sxp + x % dv];
+    for (int x = threadIdx.x; x < L * dk; x += blockDim.x) Wt[x] = X[(x / dk) * sxp + dv + x % dk];
+    // P = lam^L I - eta K^T G Wt,  Q = eta K^T G Ut
+    float *P = w.P + ((size_t)bh * w.nC + c) * dk * dk, *Q = w.Q + ((size_t)bh * w.nC + c) * dk * dv;
+    const int tk = (dk + 3) / 4, tv = (dv + 3) / 4;
+    for (int t = threadIdx.x; t < tk * (tk + tv); t += blockDim.x) {
+        const int r0 = 4 * (t / (tk + tv)), cb = t % (tk + tv);
+        const bool isP = cb < tk;
+        const int c0 = 4 * (isP ? cb : cb - tk), off = isP ? dv : 0, ncol = isP ? dk : dv;
+        float acc[4][4];
+        tile44(L, r0, c0, [&](int r, int l) { return r < dk ? pw[L - 1 - l] * sK[l * skp + r] : 0.f; },
+               [&](int l, int cc) { return cc < ncol ? X[l * sxp + off + cc] : 0.f; }, acc);
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+                const int r = r0 + u, cc = c0 + v;
+                if (r >= dk || cc >= ncol) continue;
+                if (isP)
+                    P[r * dk + cc] = (r == cc ? pw[L] : 0.f) - eta * acc[u][v];
+                else
+                    Q[r * dv + cc] = eta * acc[u][v];
+            }
+    }
+}
+
+// S_{c+1} = P_c S_c + Q_c per head, from A_init (or zero); records every
+// chunk's start state and leaves A_final.  Each thread owns 4 x 4 blocks of
+// S; chunk c+1's P and Q are loaded into registers while chunk c is computed.
+constexpr int kScanRegs = 4;  // float4 loads of P per thread and chunk (d_k <= 64)
+__global__ void __launch_bounds__(kDThreads) delta_scan_kernel(PrefillParams p, DeltaBufs w) {
+    extern __shared__ float sh[];
+    const int dk = p.dk, dv = p.dv, nel = dk * dv;
+    float *sS = sh, *sP = sS + nel;
+    const int64_t bh = blockIdx.x;
+    const int tid = threadIdx.x;
+    for (int x = tid; x < nel; x += blockDim.x) sS[x] = p.A_init ? p.A_init[bh * nel + x] : 0.f;
+    const int tk = (dk + 3) / 4, tv = (dv + 3) / 4;
+    const bool small = dk * dk <= kScanRegs * 4 * kDThreads;
+    float4 pre[kScanRegs];
+    auto fetch = [&](int64_t c) {
+        const float4 *P4 = reinterpret_cast<const float4 *>(w.P + ((size_t)bh * w.nC + c) * dk * dk);
+#pragma unroll
+        for (int u = 0; u < kScanRegs; ++u) {
+            const int x = tid + u * kDThreads;
+            if (x < dk * dk / 4) pre[u] = P4[x];
+        }
+    };
+    if (small && w.nC > 0) fetch(0);
+    for (int64_t c = 0; c < w.nC; ++c) {
+        const float *Q = w.Q + ((size_t)bh * w.nC + c) * nel;
+        float *S_out = w.S + ((size_t)bh * w.nC + c) * nel;
+        __syncthreads();
+        if (small) {
+#pragma unroll
+            for (int u = 0; u < kScanRegs; ++u) {
+                const int x = tid + u * kDThreads;
+                if (x < dk * dk / 4) reinterpret_cast<float4 *>(sP)[x] = pre[u];
+            }
+            if (c + 1 < w.nC) fetch(c + 1);
+        } else {
+            const float *P = w.P + ((size_t)bh * w.nC + c) * dk * dk;
+            for (int x = tid; x < dk * dk; x += blockDim.x) sP[x] = P[x];
+        }
+        for (int x = tid; x < nel; x += blockDim.x) S_out[x] = sS[x];
+        __syncthreads();
+        // new S in registers (this thread's blocks), written back after a barrier
+        float acc[4][4][4];  // up to 4 blocks per thread (d = 128)
+        const int nb = tk * tv;
+#pragma unroll
+        for (int bb = 0; bb < 4; ++bb) {
+            const int t = tid + bb * kDThreads;
+            if (t < nb) {
+                const int r0 = 4 * (t / tv), c0 = 4 * (t % tv);
+                tile44(dk, r0, c0, [&](int r, int rr) { return r < dk ? sP[r * dk + rr] : 0.f; },
+                       [&](int rr, int cc) { return cc < dv ? sS[rr * dv + cc] : 0.f; }, acc[bb]);
+            }
+        }
+        __syncthreads();
+#pragma unroll
+        for (int bb = 0; bb < 4; ++bb) {
+            const int t = tid + bb * kDThreads;
+            if (t < nb) {
+                const int r0 = 4 * (t / tv), c0 = 4 * (t % tv);
+#pragma unroll
+                for (int u = 0; u < 4; ++u)
+#pragma unroll
+                    for (int v = 0; v < 4; ++v)
+                        if (r0 + u < dk && c0 + v < dv) {
+                            const int x = (r0 + u) * dv + c0 + v;
+                            sS[x] = acc[bb][u][v] + Q[x];
+                        }
+            }
+        }
+    }
+    __syncthreads();
+    if (p.A_final)
+        for (int x = tid; x < nel; x += blockDim.x) p.A_final[bh * nel + x] = sS[x];
+}
+
+// m of the chunk's read rows: into mrow ([BH][T][dv] float32), or, with
+// add_y, y = y + sigma(g) m in place (y already holds the window part).
+template <typename Tin>
+__global__ void __launch_bounds__(kDThreads) delta_read_kernel(PrefillParams p, DeltaBufs w, float *mrow,
+                                                               int add_y) {
+    extern __shared__ float sh[];
+    const int dk = p.dk, dv = p.dv;
+    const int skp = dk + 1, svp = dv + 1, sgp = CD + 1;
+    float *sS = sh, *sU = sS + dk * dv, *sK = sU + CD * svp, *sQ = sK + CD * skp;
+    float *sWt = sQ + CD * skp, *sG = sWt + CD * skp, *pw = sG + CD * sgp;
+    const int64_t bh = blockIdx.y, T = p.T, W = p.W, E = w.E;
+    const int c = blockIdx.x, h = (int)(bh % p.H);
+    const int64_t e0 = (int64_t)c * CD;
+    const int L = (int)(E - e0 < CD ? E - e0 : CD);
+    const float eta = p.eta[h];
+    powers(pw, CD, p.lam[h]);
+    const float *S = w.S + ((size_t)bh * w.nC + c) * dk * dv;
+    for (int x = threadIdx.x; x < dk * dv; x += blockDim.x) sS[x] = S[x];
+    const Tin *kb = reinterpret_cast<const Tin *>(p.k) + bh * T * dk;
+    const Tin *qb = reinterpret_cast<const Tin *>(p.q) + bh * T * dk;
+    load_rows_scaled(sK, skp, kb, e0, L, dk, [](int) { return 1.f; });
+    load_rows_scaled(sQ, skp, qb, e0 + W, L, dk, [](int) { return 1.f; });
+    load_rows_scaled(sWt, skp, w.Wt + bh * E * dk, e0, L, dk, [](int) { return 1.f; });
+    load_rows_scaled(sU, svp, w.Ut + bh * E * dv, e0, L, dv, [](int) { return 1.f; });
+    __syncthreads();
+    const int tv = (dv + 3) / 4;
+    // U = Ut - Wt S (each thread updates only the entries it computed)
+    for (int t = threadIdx.x; t < (CD / 4) * tv; t += blockDim.x) {
+        const int i0 = 4 * (t / tv), c0 = 4 * (t % tv);
+        float acc[4][4];
+        tile44(dk, i0, c0, [&](int i, int r) { return sWt[i * skp + r]; },
+               [&](int r, int cc) { return cc < dv ? sS[r * dv + cc] : 0.f; }, acc);
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+#pragma unroll
+            for (int v = 0; v < 4; ++v)
+                if (c0 + v < dv) sU[(i0 + u) * svp + c0 + v] -= acc[u][v];
+    }
+    // G[i][l] = eta lam^(i-l) (q'_i . k_l) for l <= i < L
+    for (int t = threadIdx.x; t < (CD / 4) * (CD / 4); t += blockDim.x) {
+        const int i0 = 4 * (t / (CD / 4)), l0 = 4 * (t % (CD / 4));
+        float acc[4][4];
+        tile44(dk, i0, l0, [&](int i, int r) { return sQ[i * skp + r]; },
+               [&](int r, int l) { return sK[l * skp + r]; }, acc);
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+                const int i = i0 + u, l = l0 + v;
+                sG[i * sgp + l] = (l <= i && i < L) ? eta * pw[i - l] * acc[u][v] : 0.f;
+            }
+    }
+    __syncthreads();
+    // m = diag(lam^(i+1)) Q' S + G U
+    const float sg = sigmoidf_acc(p.g[h]);
+    for (int t = threadIdx.x; t < (CD / 4) * tv; t += blockDim.x) {
+        const int i0 = 4 * (t / tv), c0 = 4 * (t % tv);
+        float qs[4][4], gu[4][4];
+        tile44(dk, i0, c0, [&](int i, int r) { return sQ[i * skp + r]; },
+               [&](int r, int cc) { return cc < dv ? sS[r * dv + cc] : 0.f; }, qs);
+        tile44(CD, i0, c0, [&](int i, int l) { return sG[i * sgp + l]; },
+               [&](int l, int cc) { return cc < dv ? sU[l * svp + cc] : 0.f; }, gu);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int i = i0 + u;
+            if (i >= L) continue;
+            const int64_t row = bh * T + e0 + W + i;
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+                const int cc = c0 + v;
+                if (cc >= dv) continue;
+                const float m = fmaf(pw[i + 1], qs[u][v], gu[u][v]);
+                if (add_y) {
+                    Tin *y = reinterpret_cast<Tin *>(p.y) + row * dv + cc;
+                    *y = from_f32<Tin>(fmaf(sg, m, to_f32(*y)));
+                } else {
+                    mrow[row * dv + cc] = m;
+                }
+            }
+        }
+    }
+}
+
+template <typename Tin>
+cudaError_t launch_delta_t(const PrefillParams &p, bool add_y, cudaStream_t s) {
+    tc_prefill_desc d{};
+    d.B = p.B;
+    d.H = p.H;
+    d.T = p.T;
+    d.dk = p.dk;
+    d.dv = p.dv;
+    d.W = p.W;
+    d.flags = p.state_only ? TC_PREFILL_STATE_ONLY : 0;
+    const DeltaLayout Lo = delta_layout(d);
+    char *ws = static_cast<char *>(p.workspace);
+    DeltaBufs w;
+    w.Ut = reinterpret_cast<float *>(ws + Lo.Ut);
+    w.Wt = reinterpret_cast<float *>(ws + Lo.Wt);
+    w.P = reinterpret_cast<float *>(ws + Lo.P);
+    w.Q = reinterpret_cast<float *>(ws + Lo.Q);
+    w.S = reinterpret_cast<float *>(ws + Lo.S);
+    w.E = p.T > p.W ? p.T - p.W : 0;
+    w.nC = (w.E + CD - 1) / CD;
+    const int64_t BH = p.B * p.H;
+    const int dk = p.dk, dv = p.dv;
+    cudaError_t e;
+    if (w.nC > 0) {
+        const size_t sm_prep = (size_t)(CD * (dk + 1) + CD * (dk + dv + 1) + CD * (CD + 1) + CD + 1) * sizeof(float);
+        e = cudaFuncSetAttribute(delta_prep_kernel<Tin>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_prep);
+        if (e != cudaSuccess) return e;
+        delta_prep_kernel<Tin><<<dim3((unsigned)w.nC, (unsigned)BH), kDThreads, sm_prep, s>>>(p, w);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    const size_t sm_scan = (size_t)(dk * dv + dk * dk) * sizeof(float);
+    e = cudaFuncSetAttribute(delta_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_scan);
+    if (e != cudaSuccess) return e;
+    delta_scan_kernel<<<(unsigned)BH, kDThreads, sm_scan, s>>>(p, w);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    if (w.nC > 0 && !p.state_only) {
+        const size_t sm_read = (size_t)(dk * dv + CD * (dv + 1) + 3 * CD * (dk + 1) + CD * (CD + 1) + CD + 1) *
+                               sizeof(float);
+        e = cudaFuncSetAttribute(delta_read_kernel<Tin>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_read);
+        if (e != cudaSuccess) return e;
+        float *mrow = reinterpret_cast<float *>(ws + Lo.mrow);
+        delta_read_kernel<Tin><<<dim3((unsigned)w.nC, (unsigned)BH), kDThreads, sm_read, s>>>(p, w, mrow,
+                                                                                          add_y ? 1 : 0);
+        e = cudaGetLastError();
+    }
+    return e;
+}
+
+}  // namespace
+
+size_t delta_chunked_workspace_bytes(const tc_prefill_desc &d) { return delta_layout(d).total; }
+
+int delta_chunked_launch_count(const tc_prefill_desc &d) {
+    const int64_t E = d.T > d.W ? d.T - d.W : 0;
+    const bool reads = !(d.flags & TC_PREFILL_STATE_ONLY);
+    return (E > 0 ? 2 : 1) + (E > 0 && reads ? 1 : 0);
+}
+
+cudaError_t launch_delta_chunked(const PrefillParams &p, tc_dtype dtype, bool add_y, cudaStream_t s) {
+    return dtype == TC_BF16 ? launch_delta_t<__nv_bfloat16>(p, add_y, s) : launch_delta_t<float>(p, add_y, s);
+}
+
+}  // namespace tc

@@ -330,7 +330,19 @@ template <typename T>
 cudaError_t launch_t(const PrefillParams &p, cudaStream_t s) {
     const int64_t BH = p.B * p.H;
     if (BH == 0) return cudaSuccess;
+    if (p.delta_rule && !p.l1_only && p.n_halo == 0) {
+        // chunked delta-rule memory, then the window part reads m from mrow
+        cudaError_t e = launch_delta_chunked(p, std::is_same<T, float>::value ? TC_F32 : TC_BF16, false, s);
+        if (e != cudaSuccess) return e;
+        if (p.T > 0 && !p.state_only) {
+            const dim3 grid((unsigned)((p.T + 7) / 8), (unsigned)BH);
+            prefill_rows_kernel<T><<<grid, kThreads, 0, s>>>(p, nullptr, 0,
+                                                             reinterpret_cast<const float *>(p.workspace));
+        }
+        return cudaGetLastError();
+    }
     if (p.delta_rule && !p.l1_only) {
+        // a continued sequence (halo): the writes in token order
         float *mrow = reinterpret_cast<float *>(p.workspace);
         const size_t smem = (size_t)p.dk * p.dv * sizeof(float);
         cudaError_t e = cudaFuncSetAttribute(delta_l2_kernel<T>,
@@ -363,8 +375,11 @@ cudaError_t launch_t(const PrefillParams &p, cudaStream_t s) {
 
 size_t portable_workspace_bytes(const tc_prefill_desc &d, int64_t n_halo) {
     if (d.flags & TC_PREFILL_L1_ONLY) return 0;
-    if (d.flags & TC_PREFILL_DELTA_RULE)  // m_t of every new row
+    if (d.flags & TC_PREFILL_DELTA_RULE) {
+        if (n_halo == 0) return delta_chunked_workspace_bytes(d);  // m_t rows and the chunk buffers
+        // token order: m_t of every new row
         return (d.flags & TC_PREFILL_STATE_ONLY) ? 0 : (size_t)(d.B * d.H * d.T * d.dv) * sizeof(float);
+    }
     const int64_t nC = num_chunks(evictions(d.T + n_halo, d.W), d.C);
     return (size_t)(d.B * d.H * nC * d.dk * d.dv) * sizeof(float);
 }

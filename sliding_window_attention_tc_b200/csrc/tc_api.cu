@@ -100,6 +100,18 @@ int64_t halo_len(const tc_prefill_desc &d, int64_t t0) { return t0 < d.W ? t0 : 
 
 bool use_sm100(const tc_prefill_desc &d, int64_t n_halo) { return tc::sm100_supported(d, n_halo); }
 
+// A delta-rule call with queries and no halo whose window part the
+// tensor-core kernel takes (its L1-only form): window part there, memory in
+// chunks (which then adds sigma(g) m into y).
+bool delta_window_on_sm100(const tc_prefill_desc &d, int64_t n_halo) {
+    if (!(d.flags & TC_PREFILL_DELTA_RULE) || (d.flags & (TC_PREFILL_L1_ONLY | TC_PREFILL_STATE_ONLY)) ||
+        n_halo != 0 || d.T < 1)
+        return false;
+    tc_prefill_desc l1 = d;
+    l1.flags = TC_PREFILL_L1_ONLY;
+    return use_sm100(l1, 0);
+}
+
 size_t prefill_ws(const tc_prefill_desc &d, int64_t n_halo, int num_sms) {
     return use_sm100(d, n_halo) ? tc::sm100_workspace_bytes(d, num_sms)
                                 : tc::portable_workspace_bytes(d, n_halo);
@@ -238,6 +250,18 @@ tc_status prefill_impl(const tc_prefill_desc *d, int64_t t0, const void *halo_k,
     p.status = status_ptr();
     p.wait_ns = wait_limit_ns();
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (delta_window_on_sm100(*d, n_halo)) {
+        tc::PrefillParams w = p;
+        w.l1_only = true;
+        w.delta_rule = false;
+        w.A_final = nullptr;
+        w.A_init = nullptr;
+        w.workspace = nullptr;
+        w.workspace_bytes = 0;
+        cudaError_t e = tc::launch_prefill_sm100(w, sms, s);
+        if (e == cudaSuccess) e = tc::launch_delta_chunked(p, d->dtype, true, s);
+        return e == cudaSuccess ? TC_OK : TC_ERR_CUDA;
+    }
     cudaError_t e = use_sm100(*d, n_halo) ? tc::launch_prefill_sm100(p, sms, s)
                                           : tc::launch_prefill_portable(p, d->dtype, s);
     return e == cudaSuccess ? TC_OK : TC_ERR_CUDA;
@@ -370,11 +394,19 @@ tc_status tc_backward(const tc_prefill_desc *d, const void *q, const void *k, co
     return e == cudaSuccess ? TC_OK : TC_ERR_CUDA;
 }
 
+int tc_backward_launch_count(const tc_prefill_desc *d, int *tensor_cores) {
+    if (check_desc(d) != TC_OK || d->flags != 0) return -1;
+    if (tensor_cores) *tensor_cores = tc::backward_window_tc_supported(*d) ? 1 : 0;
+    return tc::backward_launch_count(*d);
+}
+
 int tc_prefill_launch_count(const tc_prefill_desc *d) {
     if (check_desc(d) != TC_OK) return -1;
     if (use_sm100(*d, 0)) return tc::sm100_launch_count(*d);
     const bool l1_only = (d->flags & TC_PREFILL_L1_ONLY) != 0;
     const bool state_only = (d->flags & TC_PREFILL_STATE_ONLY) != 0;
+    if ((d->flags & TC_PREFILL_DELTA_RULE) && !l1_only)  // chunked memory + the window part
+        return tc::delta_chunked_launch_count(*d) + (d->T > 0 && !state_only ? 1 : 0);
     return (l1_only ? 0 : 1) + (d->T > 0 && !state_only ? 1 : 0);
 }
 

@@ -43,6 +43,29 @@ template <> struct Vec16<__nv_bfloat16> {
     }
 };
 
+// One 4 x 4 block of out[m][n] = sum_k a(m, k) b(k, n) in registers (m0, n0
+// its corner; a and b return 0 outside the ranges they cover).  Each operand
+// loaded from shared memory serves four products (float32 SIMT products of
+// the small per-chunk matrices).
+template <class FA, class FB>
+__device__ __forceinline__ void tile44(int K, int m0, int n0, FA a, FB b, float (&acc)[4][4]) {
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+#pragma unroll
+        for (int w = 0; w < 4; ++w) acc[u][w] = 0.f;
+    for (int k = 0; k < K; ++k) {
+        float av[4], bv[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) av[u] = a(m0 + u, k);
+#pragma unroll
+        for (int w = 0; w < 4; ++w) bv[w] = b(k, n0 + w);
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+#pragma unroll
+            for (int w = 0; w < 4; ++w) acc[u][w] = fmaf(av[u], bv[w], acc[u][w]);
+    }
+}
+
 __device__ __forceinline__ uint4 ldg_nc_v4(const void *p) {
     uint4 r;
     asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
@@ -109,6 +132,14 @@ cudaError_t launch_decode(const DecodeParams &p, tc_dtype dtype, int64_t BH, cud
 // t_rows[b] += 1 for every active row (t_rows[b] >= 0), after a ragged step.
 cudaError_t launch_advance_clocks(int64_t *t_rows, int64_t B, cudaStream_t s);
 bool decode_supported(int dk, int dv, tc_dtype dtype);
+
+// delta_chunked.cu: the delta-rule write in chunks (no halo), float32 SIMT.
+// Workspace: m_t rows ([BH][T][dv] float32, at offset 0, unless state-only)
+// and the chunk buffers.  Writes A_final; with add_y it adds sigma(g) m_t into
+// y (which holds the window part), else it leaves m_t in the workspace rows.
+size_t delta_chunked_workspace_bytes(const tc_prefill_desc &d);
+int delta_chunked_launch_count(const tc_prefill_desc &d);
+cudaError_t launch_delta_chunked(const PrefillParams &p, tc_dtype dtype, bool add_y, cudaStream_t s);
 
 // prefill_portable.cu: any shape in the supported range, SIMT float32 math.
 size_t portable_workspace_bytes(const tc_prefill_desc &d, int64_t n_halo);

@@ -60,6 +60,33 @@ def test_launch_counts():
     assert _lib().tc_prefill_launch_count(ctypes.byref(_desc(flags=tc.TC_PREFILL_STATE_ONLY))) == 1
 
 
+def test_backward_launch_counts():
+    """Two window kernels, three for the memory part when something is
+    evicted (sums, scan over chunks, per-chunk gradients), one reduction."""
+    tcf = ctypes.c_int(-1)
+    assert _lib().tc_backward_launch_count(None, None) == -1
+    assert _lib().tc_backward_launch_count(ctypes.byref(_desc(flags=tc.TC_PREFILL_L1_ONLY)), None) == -1
+    assert _lib().tc_backward_launch_count(ctypes.byref(_desc()), ctypes.byref(tcf)) == 6
+    assert tcf.value == 0  # float32: SIMT kernels
+    assert _lib().tc_backward_launch_count(ctypes.byref(_desc(T=20, W=32)), None) == 3
+    lm = _desc(B=8, H=12, T=4096, W=512, C=64, dtype=tc.TC_BF16)
+    assert _lib().tc_backward_launch_count(ctypes.byref(lm), ctypes.byref(tcf)) == 6
+    assert tcf.value == (1 if HAS_GPU else 0)
+
+
+def test_delta_launch_counts():
+    """Chunked memory: prep, scan over chunks, reads; plus the window part
+    (the tensor-core kernel for bf16, d = 64, W a multiple of 128)."""
+    lm = tc.make_prefill_desc(8, 12, 4096, 64, 64, 512, 64, tc.TC_BF16, False)
+    lm.flags = tc.TC_PREFILL_DELTA_RULE
+    assert tc.prefill_launch_count(lm) == 4
+    lm.flags = tc.TC_PREFILL_DELTA_RULE | tc.TC_PREFILL_STATE_ONLY
+    assert tc.prefill_launch_count(lm) == 2
+    short = tc.make_prefill_desc(1, 1, 100, 64, 64, 128, 64, tc.TC_BF16, False)
+    short.flags = tc.TC_PREFILL_DELTA_RULE
+    assert tc.prefill_launch_count(short) == 2  # no eviction: the scan (A_final) and the window part
+
+
 # ---------------------------------------------------------------- tc_prefill_from_state
 def _from_state(desc, t0, halo_k=FAKE, halo_v=FAKE, A_init=FAKE, q=FAKE, y=FAKE, A=FAKE):
     return _lib().tc_prefill_from_state(ctypes.byref(desc), t0, halo_k, halo_v, A_init, q, FAKE,

@@ -1,8 +1,11 @@
 """GPU parity of tc_backward against the float64 oracle backward (itself
 pinned by central differences of the forward oracle).  Both sides read the
-same rounded inputs (bf16 values widened exactly), and the GPU computes in
-float32, so the bound is float32-level for every input dtype: max|x - ref| /
-max|ref| <= 2e-4 per gradient tensor (sums over up to T*d terms)."""
+same rounded inputs (bf16 values widened exactly).  The GPU accumulates in
+float32; on the tensor-core path (bf16, d = 64) the products of the bf16
+inputs are exact and P, dS and the float32 states enter as bf16 hi + lo
+pairs (remainder below 2^-17 relative), so the bound is float32-level for
+every input dtype: max|x - ref| / max|ref| <= 2e-4 per gradient tensor (sums
+over up to T*d terms)."""
 import numpy as np
 import pytest
 import torch
@@ -47,6 +50,8 @@ def test_backward_matches_oracle(cuda_device, case):
     got = tc.backward(d(x.q), d(x.k), d(x.v), d(x.lam), d(x.eta), d(x.g), W, d(dy))
     torch.cuda.synchronize()
     assert tc.device_status() == 0
+    # bf16 with d = 64 takes the tensor-core kernels, every other case SIMT
+    assert tc.backward_launch_count(x.q, W, x.v)[1] == (dtype == "bf16" and dk == dv == 64)
     ref = oracle.backward(x.q, x.k, x.v, x.lam, x.eta, x.g, W, dy)
     for name, a, b in zip(("dq", "dk", "dv", "dlam", "deta", "dg"), got, ref):
         if np.abs(b).max() == 0:
@@ -71,3 +76,31 @@ def test_backward_is_bit_for_bit_repeatable(cuda_device):
     assert tc.device_status() == 0
     for name, u, w in zip(("dq", "dk", "dv", "dlam", "deta", "dg"), a, b):
         assert torch.equal(u, w), name
+
+
+def test_backward_full_lm_shape_one_head(cuda_device):
+    """The LM workload at full size (8 x 12 x 4096, d = 64, W = 512), the
+    launch configuration the benchmark times.  Heads are independent, and
+    dlambda, deta, dg of head h sum over the batch only, so the oracle run on
+    head h alone (all 8 batch rows) checks every output of that head."""
+    import sliding_window_attention_tc_b200 as tc
+    x = wl.prefill_config("lm_prefill_bf16")
+    B, H, T, d = x.q.shape
+    gen = torch.Generator().manual_seed(11)
+    dy = (torch.randn(B, H, T, d, generator=gen) / 8).to(x.q.dtype)
+    dev = cuda_device
+    args = [t.to(dev).contiguous() for t in (x.q, x.k, x.v, x.lam, x.eta, x.g)]
+    assert tc.backward_launch_count(x.q, x.W)[1]
+    got = tc.backward(*args, x.W, dy.to(dev))
+    torch.cuda.synchronize()
+    assert tc.device_status() == 0
+    h = 7
+    sl = lambda t: t[:, h:h + 1]
+    ref = oracle.backward(sl(x.q), sl(x.k), sl(x.v), x.lam[h:h + 1], x.eta[h:h + 1], x.g[h:h + 1],
+                          x.W, sl(dy))
+    for name, a, r in zip(("dq", "dk", "dv"), got[:3], ref[:3]):
+        err = max_rel(sl(a).cpu().numpy(), r)
+        assert err <= 2e-4, (name, err)
+    for name, a, r in zip(("dlam", "deta", "dg"), got[3:], ref[3:]):
+        err = abs(float(a[h]) - float(r[0])) / abs(float(r[0]))
+        assert err <= 2e-4, (name, err)

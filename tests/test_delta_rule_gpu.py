@@ -119,3 +119,27 @@ def test_delta_decode_continues_a_delta_prefill(cuda_device):
     yo, Ao = oracle.prefill(x.q, x.k, x.v, x.lam, x.eta, x.g, W, rule="delta")
     assert max_rel(torch.stack(ys, 2).numpy(), yo[:, :, T:]) <= 1e-5
     assert max_rel(st.A.cpu().numpy(), Ao) <= 1e-5
+
+
+# chunked memory (64 evictions per chunk): several chunks and a ragged last one
+CHUNKED = [
+    (1, 2, 1000, 32, 16, "f32"),    # 16 chunks, the last of 24 evictions
+    (1, 1, 300, 128, 40, "f32"),    # d = 128
+    (2, 2, 700, 64, 200, "bf16"),   # W not a multiple of 128: SIMT window part
+    (1, 3, 1100, 64, 256, "bf16"),  # tensor-core window part, memory added into y
+]
+
+
+@pytest.mark.parametrize("B,H,T,d,W,dtype", CHUNKED, ids=[f"{c[5]}_T{c[2]}_d{c[3]}_W{c[4]}" for c in CHUNKED])
+def test_delta_prefill_chunked(cuda_device, B, H, T, d, W, dtype):
+    tc = _tc()
+    x = wl.random_prefill(B, H, T, d, d, W, 16, dtype=dtype, seed=7 + T + d)
+    dev = cuda_device
+    dd = lambda t: t.to(dev).contiguous()
+    y_ref, A_ref = oracle.prefill(x.q, x.k, x.v, x.lam, x.eta, x.g, W, rule="delta")
+    y, A = tc.prefill(dd(x.q), dd(x.k), dd(x.v), dd(x.lam), dd(x.eta), dd(x.g), W, 16,
+                      delta_rule=True)
+    torch.cuda.synchronize()
+    assert tc.device_status() == 0
+    _close(dtype, y.float().cpu().numpy(), y_ref, A.cpu().numpy(), A_ref)
+
