@@ -67,11 +67,50 @@ __device__ __forceinline__ void powers(float *pw, int n_max, float lam) {
     for (int n = threadIdx.x; n <= n_max; n += blockDim.x) pw[n] = n == 0 ? 1.f : (float)exp2((double)n * l2l);
 }
 
+// Four consecutive elements as float32 (16-byte / 8-byte aligned).
+__device__ __forceinline__ void load4(const float *p, float (&f)[4]) {
+    const float4 a = *reinterpret_cast<const float4 *>(p);
+    f[0] = a.x;
+    f[1] = a.y;
+    f[2] = a.z;
+    f[3] = a.w;
+}
+__device__ __forceinline__ void load4(const __nv_bfloat16 *p, float (&f)[4]) {
+    const uint2 a = *reinterpret_cast<const uint2 *>(p);
+    f[0] = __uint_as_float(a.x << 16);
+    f[1] = __uint_as_float(a.x & 0xffff0000u);
+    f[2] = __uint_as_float(a.y << 16);
+    f[3] = __uint_as_float(a.y & 0xffff0000u);
+}
+__device__ __forceinline__ void store4(float *p, const float (&f)[4]) {
+    *reinterpret_cast<float4 *>(p) = make_float4(f[0], f[1], f[2], f[3]);
+}
+__device__ __forceinline__ void store4(__nv_bfloat16 *p, const float (&f)[4]) {
+    *reinterpret_cast<uint2 *>(p) = make_uint2(pack_bf16_rn(f[0], f[1]), pack_bf16_rn(f[2], f[3]));
+}
+
 // rows r0 .. r0+n_valid-1 of a [.][d] tensor into shared rows of stride sp,
-// scaled by scale(row); rows n_valid .. CD-1 are zero.
+// scaled by scale(row); rows n_valid .. CD-1 are zero.  Four elements per
+// load when d is a multiple of 4.
 template <typename Tin, class F>
 __device__ __forceinline__ void load_rows_scaled(float *dst, int sp, const Tin *src, int64_t r0, int n_valid, int d,
                                                  F scale) {
+    if ((d & 3) == 0) {
+        const int d4 = d >> 2;
+        for (int x = threadIdx.x; x < CD * d4; x += blockDim.x) {
+            const int i = x / d4, c = 4 * (x - i * d4);
+            float f[4] = {0.f, 0.f, 0.f, 0.f};
+            if (i < n_valid) {
+                load4(src + (r0 + i) * d + c, f);
+                const float sc = scale(i);
+#pragma unroll
+                for (int u = 0; u < 4; ++u) f[u] *= sc;
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) dst[i * sp + c + u] = f[u];
+        }
+        return;
+    }
     for (int x = threadIdx.x; x < CD * d; x += blockDim.x) {
         const int i = x / d, c = x % d;
         dst[i * sp + c] = i < n_valid ? scale(i) * to_f32(src[(r0 + i) * d + c]) : 0.f;
@@ -309,16 +348,31 @@ __global__ void __launch_bounds__(kDThreads) delta_read_kernel(PrefillParams p, 
             const int i = i0 + u;
             if (i >= L) continue;
             const int64_t row = bh * T + e0 + W + i;
+            float m[4];
+#pragma unroll
+            for (int v = 0; v < 4; ++v) m[v] = fmaf(pw[i + 1], qs[u][v], gu[u][v]);
+            if ((dv & 3) == 0) {  // four columns at once (c0 + 3 < dv)
+                if (add_y) {
+                    Tin *y = reinterpret_cast<Tin *>(p.y) + row * dv + c0;
+                    float f[4];
+                    load4(y, f);
+#pragma unroll
+                    for (int v = 0; v < 4; ++v) f[v] = fmaf(sg, m[v], f[v]);
+                    store4(y, f);
+                } else {
+                    store4(mrow + row * dv + c0, m);
+                }
+                continue;
+            }
 #pragma unroll
             for (int v = 0; v < 4; ++v) {
                 const int cc = c0 + v;
                 if (cc >= dv) continue;
-                const float m = fmaf(pw[i + 1], qs[u][v], gu[u][v]);
                 if (add_y) {
                     Tin *y = reinterpret_cast<Tin *>(p.y) + row * dv + cc;
-                    *y = from_f32<Tin>(fmaf(sg, m, to_f32(*y)));
+                    *y = from_f32<Tin>(fmaf(sg, m[v], to_f32(*y)));
                 } else {
-                    mrow[row * dv + cc] = m;
+                    mrow[row * dv + cc] = m[v];
                 }
             }
         }

@@ -20,6 +20,12 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(flo
     return __float2bfloat16_rn(x);
 }
 
+// Two floats -> a bf16 pair (round to nearest even), a in the low half.
+__device__ __forceinline__ uint32_t pack_bf16_rn(float a, float b) {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+    return *reinterpret_cast<const uint32_t *>(&h);
+}
+
 // Unpack 16 bytes holding VEC elements of T into floats.
 template <typename T> struct Vec16;
 template <> struct Vec16<float> {
