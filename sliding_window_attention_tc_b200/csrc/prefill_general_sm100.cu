@@ -1,0 +1,835 @@
+// Tensor-core prefill for the shapes the fused prefill_main_kernel does not
+// take: bf16 with d_k = d_v = D in {64, 128}, any window W >= 1, any T, and
+// continuations with any halo (0 < t0 < W included).
+//
+// "Tensor Cache: Eviction-conditioned Associative Memory for Transformers":
+// the window read of §3.1 eq. (1) and the memory of §3.2 / Fig. 2 (write on
+// eviction, A <- lam A + eta k v^T; read m = q A; y = y_local + sigma(g) m),
+// the memory in the chunked form of the abstract and §2 (chunks of CG = 128
+// evictions).  Five kernels, all but the copy and the scan on tcgen05:
+//   gen_combine_kernel   halo + new keys / values into one sequence (only
+//                        when continuing with a halo);
+//   gen_sums_kernel      per chunk dA_c = eta K^T diag(lam^(L-1-i)) V, one
+//                        M = 128 product (two chunks side by side for D = 64);
+//   gen_scan_kernel      A_c = chunk start states from A_init, and A_final;
+//   gen_read_kernel      per chunk the reads m_i = lam^(i+1) q'_i A_c +
+//                        eta sum_{l<=i} lam^(i-l) (q'_i . k_l) v_l into a row
+//                        buffer (q'_i the query at t = e0 + i + W);
+//   gen_window_kernel    the window softmax in one pass (online rescaling of
+//                        the output accumulator in TMEM) and the fusion
+//                        y = y_local + sigma(g) m.
+// Positions are those of the combined sequence (halo first): token tau is a
+// new row when tau >= n_halo, evictions are tau = 0 .. n_halo + T - W - 1 and
+// A_init holds every eviction before the combined sequence.  float32 values
+// that enter the tensor cores (the states, the decayed in-chunk scores) are
+// split into bf16 hi + lo pairs; P of the window softmax is bf16, as in the
+// fused kernel.
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "sm100_ptx.cuh"
+#include "tc.h"
+#include "tc_internal.cuh"
+
+namespace tc {
+namespace {
+
+using namespace sm100;
+
+constexpr int CG = 128;                  // evictions per chunk, query rows per window CTA
+constexpr int GX = 64;                   // key rows per window tile
+constexpr int kGThreads = 192;           // warp 0 TMA, warp 1 MMA, warps 2-5 element-wise
+constexpr uint32_t BLK128 = 128 * 128;   // a 128-row x 64-column bf16 block (16 KB)
+constexpr uint32_t BLK64 = 64 * 128;     // a 64-row x 64-column bf16 block (8 KB)
+constexpr float kLog2eG = 1.4426950408889634f;
+
+struct GenParams {
+    const __nv_bfloat16 *q, *k, *v;  // q: [BH][T][D] new rows; k, v: the combined sequence
+    __nv_bfloat16 *y;
+    float *mrow;                     // [BH][T][D] float32 reads (null: none)
+    float *dA;                       // [BH][nC][D][D]: increments, then start states
+    float *A_final;
+    const float *A_init;
+    const float *lam, *eta, *g;
+    int T, Tc, n_halo, W, H, E, nC;  // new rows, combined rows, halo, window, heads, evictions, chunks
+    int *status;
+    unsigned long long wait_ns;
+};
+
+__device__ __forceinline__ bool gwait(uint64_t *bar, uint32_t parity, volatile int *abort, const GenParams &p) {
+    return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort, p.status, p.wait_ns));
+}
+__device__ __forceinline__ float gex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+__device__ __forceinline__ void gsplit(float x0, float x1, uint32_t &hi, uint32_t &lo) {
+    hi = pack_bf16(x0, x1);
+    lo = pack_bf16(x0 - __uint_as_float(hi << 16), x1 - __uint_as_float(hi & 0xffff0000u));
+}
+// lam^n, n = 0 .. n_max, by the calling 128 threads (index x)
+__device__ __forceinline__ void gpowers(float *pw, int n_max, float lam, int x) {
+    const double l2l = log2((double)lam);
+    for (int n = x; n <= n_max; n += 128) pw[n] = n == 0 ? 1.f : (float)exp2((double)n * l2l);
+}
+__device__ __forceinline__ void gbar128() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+// rows [row, row + rows) of a [.][D] map as NB column blocks of 64
+template <int NB>
+__device__ __forceinline__ void tma_rows_nb(uint8_t *dst, const CUtensorMap *m, uint64_t *bar, int row, int bh,
+                                            uint32_t blk) {
+#pragma unroll
+    for (int b = 0; b < NB; ++b) tma_load_3d(dst + b * blk, m, bar, 64 * b, row, bh);
+}
+
+// ===========================================================================
+// Window part.  A CTA owns 128 new query rows (TMEM lanes); 64-row key
+// tiles stream through NS stages.  Per tile: S = Q K^T into TMEM; the
+// element-wise warps take the row max, rescale O in TMEM when it grew (O is
+// complete then: the scores' commit follows the previous P V), write
+// P = exp2(s - m) as bf16 over S, and O += P V runs from TMEM.
+template <int NB>
+struct WinCfg {
+    static constexpr int D = 64 * NB;
+    static constexpr int NS = NB == 1 ? 4 : 3;
+    static constexpr uint32_t Q_B = NB * BLK128;
+    static constexpr uint32_t X_B = NB * BLK64;   // one K or V tile
+    static constexpr uint32_t OFF_Q = 0;
+    static constexpr uint32_t OFF_X = Q_B;         // NS x (K tile, V tile)
+    static constexpr uint32_t OFF_BAR = OFF_X + NS * 2 * X_B;
+    static constexpr uint32_t SMEM = OFF_BAR + 128 + 1024;
+    static constexpr uint32_t TM_S = 0, TM_O = 64, COLS = NB == 1 ? 128 : 256;
+};
+
+template <int NB>
+__global__ void __launch_bounds__(kGThreads, 1)
+    gen_window_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
+                      const __grid_constant__ CUtensorMap tv, GenParams p) {
+    using C = WinCfg<NB>;
+    constexpr int D = C::D, NS = C::NS;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + C::OFF_BAR);
+    uint64_t *q_full = bars, *x_full = bars + 1, *x_empty = x_full + NS, *s_full = x_empty + NS;
+    uint64_t *p_ready = s_full + 1, *o_full = p_ready + 1, *mma_done = o_full + 1;
+    uint32_t *tmem_base = reinterpret_cast<uint32_t *>(mma_done + 1);
+    volatile int *abort = reinterpret_cast<volatile int *>(tmem_base + 1);
+
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const int bh = blockIdx.y;
+    const int t0 = blockIdx.x * CG;           // first new row
+    const int tau0 = p.n_halo + t0;           // its combined position
+    const int lo = max(0, tau0 - p.W + 1), hi = min(p.Tc - 1, tau0 + CG - 1);
+    const int xs = lo & ~(GX - 1);
+    const int N = (hi - xs) / GX + 1;
+
+    if (tid == 0) {
+        mbar_init(q_full, 1);
+        for (int s = 0; s < NS; ++s) {
+            mbar_init(&x_full[s], 1);
+            mbar_init(&x_empty[s], 1);
+        }
+        mbar_init(s_full, 1);
+        mbar_init(p_ready, 4);
+        mbar_init(o_full, 1);
+        mbar_init(mma_done, 1);
+        *abort = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_base, C::COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tb = *tmem_base;
+
+    if (warp == 0) {
+        if (tid == 0) {
+            mbar_expect_tx(q_full, C::Q_B);
+            tma_rows_nb<NB>(sm + C::OFF_Q, &tq, q_full, t0, bh, BLK128);
+            int n = 0;
+            for (; n < N; ++n) {
+                const int s = n % NS;
+                if (!mbar_wait(&x_empty[s], ((n / NS) & 1) ^ 1, abort, p.status, p.wait_ns)) break;
+                uint8_t *dst = sm + C::OFF_X + s * 2 * C::X_B;
+                mbar_expect_tx(&x_full[s], 2 * C::X_B);
+                tma_rows_nb<NB>(dst, &tk, &x_full[s], xs + GX * n, bh, BLK64);
+                tma_rows_nb<NB>(dst + C::X_B, &tv, &x_full[s], xs + GX * n, bh, BLK64);
+            }
+            mbar_wait_drain(q_full, 0);
+            for (int st = 0; st < NS; ++st) {
+                const int fills = n > st ? (n - 1 - st) / NS + 1 : 0;
+                if (fills) mbar_wait_drain(&x_full[st], (fills - 1) & 1);
+            }
+        }
+    } else if (warp == 1) {
+        const uint32_t id_s = idesc_bf16(128, 64, false, false);
+        const uint32_t id_o = idesc_bf16(128, D, false, true);
+        const uint32_t sq = smem_u32(sm + C::OFF_Q), sx = smem_u32(sm + C::OFF_X);
+        bool ok = gwait(q_full, 0, abort, p);
+        for (int n = 0; ok && n <= N; ++n) {
+            if (n > 0) {
+                const int m = n - 1, sp = m % NS;
+                if (!(ok = gwait(p_ready, m & 1, abort, p))) break;
+                tc_fence_after();
+                // O += P V: P (64 keys) in the score columns, V read MN-major
+                const uint64_t vd = sdesc_sw128(sx + sp * 2 * C::X_B + C::X_B, BLK64, 1024);
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    mma_ts_w(tb + C::TM_O, tb + C::TM_S + 8 * k, vd + 128 * k, id_o, (m > 0 || k > 0) ? 1u : 0u);
+                mma_commit_w(&x_empty[sp]);
+            }
+            if (n == N) break;
+            const int s = n % NS;
+            if (!(ok = gwait(&x_full[s], (n / NS) & 1, abort, p))) break;
+            tc_fence_after();
+            const uint32_t kx = sx + s * 2 * C::X_B;
+#pragma unroll
+            for (int b = 0; b < NB; ++b)
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    mma_ss_w(tb + C::TM_S, sdesc_sw128(sq + b * BLK128, 16, 1024) + 2 * k,
+                             sdesc_sw128(kx + b * BLK64, 16, 1024) + 2 * k, id_s, (b > 0 || k > 0) ? 1u : 0u);
+            mma_commit_w(s_full);
+        }
+        if (ok) mma_commit_w(o_full);
+        mma_commit_w(mma_done);
+        mbar_wait_drain(mma_done, 0);
+    } else {
+        const int q4 = warp & 3;
+        const int r = 32 * q4 + (tid & 31);
+        const uint32_t lanes = tb + ((uint32_t)(32 * q4) << 16);
+        const int t = t0 + r, tau = tau0 + r;
+        const uint32_t wlim = t < p.T ? (uint32_t)p.W : 0u;
+        const float sl2 = kLog2eG * rsqrtf((float)D);
+        float m_run = -INFINITY, l_run = 0.f;
+        bool ok = true;
+        for (int n = 0; n < N; ++n) {
+            if (!(ok = gwait(s_full, n & 1, abort, p))) break;
+            tc_fence_after();
+            const int base = tau - (xs + GX * n);  // tau - j = base - c
+            uint32_t sr[2][32];
+            tmem_ld32(lanes + C::TM_S, sr[0]);
+            tmem_ld32(lanes + C::TM_S + 32, sr[1]);
+            tmem_wait_ld();
+            float mx = -INFINITY;
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+#pragma unroll
+                for (int c = 0; c < 32; ++c) {
+                    const bool in = (uint32_t)(base - (32 * h + c)) < wlim;
+                    const float x = in ? __uint_as_float(sr[h][c]) * sl2 : -INFINITY;
+                    sr[h][c] = __float_as_uint(x);
+                    mx = fmaxf(mx, x);
+                }
+            const float m_new = fmaxf(m_run, mx);
+            const float corr = m_new == -INFINITY ? 1.f : gex2(m_run - m_new);
+            // rescale O (complete: this tile's scores were committed after the previous P V)
+            if (n > 0 && __any_sync(0xffffffffu, corr != 1.f)) {
+#pragma unroll
+                for (int c0 = 0; c0 < D; c0 += 32) {
+                    uint32_t o[32];
+                    tmem_ld32(lanes + C::TM_O + c0, o);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * corr);
+                    tmem_st32(lanes + C::TM_O + c0, o);
+                }
+            }
+            float sum = 0.f;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                uint32_t pk[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                    const float a = m_new == -INFINITY ? 0.f : gex2(__uint_as_float(sr[h][2 * e]) - m_new);
+                    const float b = m_new == -INFINITY ? 0.f : gex2(__uint_as_float(sr[h][2 * e + 1]) - m_new);
+                    sum += a + b;
+                    pk[e] = pack_bf16(a, b);
+                }
+                tmem_st16(lanes + C::TM_S + 16 * h, pk);
+            }
+            l_run = fmaf(l_run, corr, sum);
+            m_run = m_new;
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            mbar_arrive_w(p_ready);
+        }
+        if (ok && gwait(o_full, 0, abort, p)) {
+            tc_fence_after();
+            const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
+            const bool has_m = p.mrow && tau >= p.W && t < p.T;
+            const float sg = has_m ? 1.f / (1.f + expf(-p.g[bh % p.H])) : 0.f;
+            const float *mr = has_m ? p.mrow + ((size_t)bh * p.T + t) * D : nullptr;
+#pragma unroll
+            for (int c0 = 0; c0 < D; c0 += 32) {
+                uint32_t o[32];
+                tmem_ld32(lanes + C::TM_O + c0, o);
+                tmem_wait_ld();
+                if (t < p.T) {
+                    float f[32];
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) f[c] = __uint_as_float(o[c]) * inv_l;
+                    if (has_m) {
+#pragma unroll
+                        for (int c = 0; c < 32; c += 4) {
+                            const float4 mv = *reinterpret_cast<const float4 *>(mr + c0 + c);
+                            f[c] = fmaf(sg, mv.x, f[c]);
+                            f[c + 1] = fmaf(sg, mv.y, f[c + 1]);
+                            f[c + 2] = fmaf(sg, mv.z, f[c + 2]);
+                            f[c + 3] = fmaf(sg, mv.w, f[c + 3]);
+                        }
+                    }
+                    uint4 *dst = reinterpret_cast<uint4 *>(p.y + ((size_t)bh * p.T + t) * D + c0);
+#pragma unroll
+                    for (int u = 0; u < 4; ++u)
+                        dst[u] = make_uint4(pack_bf16(f[8 * u], f[8 * u + 1]), pack_bf16(f[8 * u + 2], f[8 * u + 3]),
+                                            pack_bf16(f[8 * u + 4], f[8 * u + 5]),
+                                            pack_bf16(f[8 * u + 6], f[8 * u + 7]));
+                }
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tb, C::COLS);
+}
+
+// ===========================================================================
+// Per-chunk increments.  A = two 64-row M blocks (K^T of two chunks for
+// D = 64, or the two column halves of one chunk's K^T for D = 128), B = the
+// matching two N blocks of diag(w) V as bf16 hi + lo; D's diagonal blocks
+// (D = 64) or all of it (D = 128) are the increments.
+constexpr uint32_t SUM_OFF_A = 0;                  // 2 blocks (TMA)
+constexpr uint32_t SUM_OFF_B = 2 * BLK128;         // hi: 2 blocks, lo: 2 blocks
+constexpr uint32_t SUM_OFF_PW = SUM_OFF_B + 4 * BLK128;
+constexpr uint32_t SUM_OFF_BAR = SUM_OFF_PW + 136 * 4;
+constexpr uint32_t SUM_SMEM = SUM_OFF_BAR + 64 + 1024;
+
+template <int NB>
+__global__ void __launch_bounds__(kGThreads, 2)
+    gen_sums_kernel(const __grid_constant__ CUtensorMap tk, GenParams p) {
+    constexpr int D = 64 * NB;
+    constexpr int CPB = NB == 1 ? 2 : 1;  // chunks per CTA
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + SUM_OFF_BAR);
+    uint64_t *in_full = bars, *b_ready = bars + 1, *acc_full = bars + 2, *mma_done = bars + 3;
+    uint32_t *tmem_base = reinterpret_cast<uint32_t *>(bars + 4);
+    volatile int *abort = reinterpret_cast<volatile int *>(tmem_base + 1);
+    float *pw = reinterpret_cast<float *>(sm + SUM_OFF_PW);
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const int bh = blockIdx.y, c_first = blockIdx.x * CPB;
+    const int h = bh % p.H;
+
+    if (tid == 0) {
+        mbar_init(in_full, 1);
+        mbar_init(b_ready, 128);
+        mbar_init(acc_full, 1);
+        mbar_init(mma_done, 1);
+        *abort = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_base, 128);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tb = *tmem_base;
+
+    if (warp == 0) {
+        if (tid == 0) {
+            mbar_expect_tx(in_full, 2 * BLK128);
+            if (NB == 1) {  // K of chunks c_first, c_first + 1 (rows past the combined sequence read zero)
+                tma_load_3d(sm + SUM_OFF_A, &tk, in_full, 0, c_first * CG, bh);
+                tma_load_3d(sm + SUM_OFF_A + BLK128, &tk, in_full, 0, (c_first + 1) * CG, bh);
+            } else {
+                tma_load_3d(sm + SUM_OFF_A, &tk, in_full, 0, c_first * CG, bh);
+                tma_load_3d(sm + SUM_OFF_A + BLK128, &tk, in_full, 64, c_first * CG, bh);
+            }
+            mbar_wait_drain(in_full, 0);
+        }
+    } else if (warp == 1) {
+        const uint32_t sa = smem_u32(sm + SUM_OFF_A), sb = smem_u32(sm + SUM_OFF_B);
+        const uint32_t id = idesc_bf16(128, 128, true, true);
+        bool ok = gwait(in_full, 0, abort, p) && gwait(b_ready, 0, abort, p);
+        if (ok) {
+            tc_fence_after();
+#pragma unroll
+            for (int part = 0; part < 2; ++part)
+#pragma unroll
+                for (int k = 0; k < 8; ++k)
+                    mma_ss_w(tb, sdesc_sw128(sa, BLK128, 1024) + 128 * k,
+                             sdesc_sw128(sb + part * 2 * BLK128, BLK128, 1024) + 128 * k, id,
+                             (part > 0 || k > 0) ? 1u : 0u);
+            mma_commit_w(acc_full);
+        }
+        mma_commit_w(mma_done);
+        mbar_wait_drain(mma_done, 0);
+    } else {
+        const int q4 = warp & 3;
+        const int x = 32 * q4 + (tid & 31);
+        const uint32_t lanes = tb + ((uint32_t)(32 * q4) << 16);
+        gpowers(pw, CG, p.lam[h], x);
+        gbar128();
+        // B row x: for each N block b, w * V row of the block's chunk (D = 64) or
+        // columns 64 b .. of the chunk's row (D = 128)
+#pragma unroll
+        for (int b = 0; b < 2; ++b) {
+            const int c = NB == 1 ? c_first + b : c_first;
+            const int e0 = c * CG;
+            const int L = c < p.nC ? min(CG, p.E - e0) : 0;
+            const float w = x < L ? pw[L - 1 - x] : 0.f;
+            const int col0 = NB == 1 ? 0 : 64 * b;
+            const uint4 *src = reinterpret_cast<const uint4 *>(p.v + ((size_t)bh * p.Tc + e0 + x) * D + col0);
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const uint4 a = w != 0.f ? src[u] : make_uint4(0u, 0u, 0u, 0u);
+                const uint32_t ws[4] = {a.x, a.y, a.z, a.w};
+                uint32_t hi[4], lo[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    gsplit(w * __uint_as_float(ws[e] << 16), w * __uint_as_float(ws[e] & 0xffff0000u), hi[e], lo[e]);
+                *reinterpret_cast<uint4 *>(sm + SUM_OFF_B + b * BLK128 + sw128_offset(x, 8 * u)) =
+                    make_uint4(hi[0], hi[1], hi[2], hi[3]);
+                *reinterpret_cast<uint4 *>(sm + SUM_OFF_B + (2 + b) * BLK128 + sw128_offset(x, 8 * u)) =
+                    make_uint4(lo[0], lo[1], lo[2], lo[3]);
+            }
+        }
+        fence_async_smem();
+        mbar_arrive(b_ready);
+        if (gwait(acc_full, 0, abort, p)) {
+            tc_fence_after();
+            const float eta = p.eta[h];
+            // D = 64: lanes 0..63 rows of chunk c_first (columns 0..63), 64..127 of
+            // c_first + 1 (columns 64..127); D = 128: every lane a row, all columns
+            const int c = NB == 1 ? c_first + (x >> 6) : c_first;
+            const int r = NB == 1 ? (x & 63) : x;
+            const uint32_t col0 = NB == 1 ? (uint32_t)(x & 64) : 0u;
+            if (c < p.nC) {
+                float *dst = p.dA + (((size_t)bh * p.nC + c) * D + r) * D;
+#pragma unroll
+                for (int c0 = 0; c0 < (NB == 1 ? 64 : 128); c0 += 32) {
+                    uint32_t v[32];
+                    tmem_ld32(lanes + col0 + c0, v);
+                    tmem_wait_ld();
+                    float4 *d4 = reinterpret_cast<float4 *>(dst + c0);
+#pragma unroll
+                    for (int u = 0; u < 8; ++u)
+                        d4[u] = make_float4(eta * __uint_as_float(v[4 * u]), eta * __uint_as_float(v[4 * u + 1]),
+                                            eta * __uint_as_float(v[4 * u + 2]), eta * __uint_as_float(v[4 * u + 3]));
+                }
+            } else {
+                // the chunk past the end (odd chunk count, D = 64): its lanes still
+                // take part in the collective loads
+                uint32_t v[32];
+                tmem_ld32(lanes + col0, v);
+                tmem_wait_ld();
+                tmem_ld32(lanes + col0 + 32, v);
+                tmem_wait_ld();
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tb, 128);
+}
+
+// ===========================================================================
+// Chunk start states, one thread per state element: A_c (in place over the
+// increments) and A_final.
+__global__ void __launch_bounds__(256) gen_scan_kernel(GenParams p, int D) {
+    __shared__ float decay[2];
+    const int bh = blockIdx.y;
+    if (threadIdx.x < 2) {
+        const double l2l = log2((double)p.lam[bh % p.H]);
+        const int last = p.nC > 0 ? p.E - (p.nC - 1) * CG : 0;
+        const int n = threadIdx.x == 0 ? CG : last;
+        decay[threadIdx.x] = (float)exp2((double)n * l2l);
+    }
+    __syncthreads();
+    const int x = blockIdx.x * blockDim.x + threadIdx.x;
+    const int nel = D * D;
+    if (x >= nel) return;
+    float A = p.A_init ? p.A_init[(size_t)bh * nel + x] : 0.f;
+    float *dA = p.dA + (size_t)bh * p.nC * nel + x;
+    constexpr int kB = 8;
+    for (int c0 = 0; c0 < p.nC; c0 += kB) {
+        float d[kB];
+#pragma unroll
+        for (int u = 0; u < kB; ++u) d[u] = c0 + u < p.nC ? dA[(size_t)(c0 + u) * nel] : 0.f;
+#pragma unroll
+        for (int u = 0; u < kB; ++u) {
+            const int c = c0 + u;
+            if (c < p.nC) {
+                dA[(size_t)c * nel] = A;
+                A = fmaf(c == p.nC - 1 ? decay[1] : decay[0], A, d[u]);
+            }
+        }
+    }
+    if (p.A_final) p.A_final[(size_t)bh * nel + x] = A;
+}
+
+// ===========================================================================
+// Reads of one chunk: QK = Q' K^T (TMEM); Mq = eta lam^(i-l) QK on l <= i < L
+// as bf16 hi + lo over QK; mA = Q' A_c (A_c as bf16 hi + lo in shared
+// memory, read MN-major); mI = Mq V; m = lam^(i+1) mA + mI into mrow.
+template <int NB>
+struct ReadCfg {
+    static constexpr int D = 64 * NB;
+    static constexpr uint32_t IN_B = NB * BLK128;            // a 128-row input tile
+    static constexpr uint32_t OFF_Q = 0, OFF_K = IN_B, OFF_V = 2 * IN_B;
+    static constexpr uint32_t ST_BLK = D * 128;              // D rows x 64 columns of A_c
+    static constexpr uint32_t OFF_A = 3 * IN_B;              // hi: NB blocks, lo: NB blocks
+    static constexpr uint32_t OFF_PW = OFF_A + 2 * NB * ST_BLK;
+    static constexpr uint32_t OFF_BAR = OFF_PW + 136 * 4;
+    static constexpr uint32_t SMEM = OFF_BAR + 64 + 1024;
+    static constexpr uint32_t TM_QK = 0, TM_MA = 128, TM_MI = 128 + D, COLS = NB == 1 ? 256 : 512;
+};
+
+template <int NB>
+__global__ void __launch_bounds__(kGThreads, 1)
+    gen_read_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
+                    const __grid_constant__ CUtensorMap tv, GenParams p) {
+    using C = ReadCfg<NB>;
+    constexpr int D = C::D;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + C::OFF_BAR);
+    uint64_t *in_full = bars, *s_full = bars + 1, *m_ready = bars + 2, *acc_full = bars + 3;
+    uint64_t *mma_done = bars + 4;
+    uint32_t *tmem_base = reinterpret_cast<uint32_t *>(bars + 5);
+    volatile int *abort = reinterpret_cast<volatile int *>(tmem_base + 1);
+    float *pw = reinterpret_cast<float *>(sm + C::OFF_PW);
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const int c = blockIdx.x, bh = blockIdx.y, h = bh % p.H;
+    const int e0 = c * CG, L = min(CG, p.E - e0);
+    const int qrow0 = e0 + p.W - p.n_halo;  // new row of eviction e0's read
+
+    if (tid == 0) {
+        mbar_init(in_full, 1);
+        mbar_init(s_full, 1);
+        mbar_init(m_ready, 128);
+        mbar_init(acc_full, 1);
+        mbar_init(mma_done, 1);
+        *abort = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_base, C::COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tb = *tmem_base;
+
+    if (warp == 0) {
+        if (tid == 0) {
+            mbar_expect_tx(in_full, 3 * C::IN_B);
+            tma_rows_nb<NB>(sm + C::OFF_Q, &tq, in_full, qrow0, bh, BLK128);
+            tma_rows_nb<NB>(sm + C::OFF_K, &tk, in_full, e0, bh, BLK128);
+            tma_rows_nb<NB>(sm + C::OFF_V, &tv, in_full, e0, bh, BLK128);
+            mbar_wait_drain(in_full, 0);
+        }
+    } else if (warp == 1) {
+        const uint32_t base = smem_u32(sm);
+        const uint32_t sq = base + C::OFF_Q, sk = base + C::OFF_K, sv = base + C::OFF_V, sa = base + C::OFF_A;
+        const uint32_t id_qk = idesc_bf16(128, 128, false, false);
+        const uint32_t id_n = idesc_bf16(128, D, false, true);
+        bool ok = gwait(in_full, 0, abort, p);
+        if (ok) {
+            tc_fence_after();
+#pragma unroll
+            for (int b = 0; b < NB; ++b)
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    mma_ss_w(tb + C::TM_QK, sdesc_sw128(sq + b * BLK128, 16, 1024) + 2 * k,
+                             sdesc_sw128(sk + b * BLK128, 16, 1024) + 2 * k, id_qk, (b > 0 || k > 0) ? 1u : 0u);
+            mma_commit_w(s_full);
+            ok = gwait(m_ready, 0, abort, p);
+        }
+        if (ok) {
+            tc_fence_after();
+#pragma unroll
+            for (int part = 0; part < 2; ++part) {
+                // mA += Q' A_part: K = D (Q' column blocks), A_c rows K-steps of 16
+                const uint32_t ap = sa + part * NB * C::ST_BLK;
+#pragma unroll
+                for (int k = 0; k < 4 * NB; ++k)
+                    mma_ss_w(tb + C::TM_MA, sdesc_sw128(sq + (k >> 2) * BLK128, 16, 1024) + 2 * (k & 3),
+                             sdesc_sw128(ap, C::ST_BLK, 1024) + 128 * k, id_n, (part > 0 || k > 0) ? 1u : 0u);
+                // mI += Mq_part V: Mq's K-step k (keys 16k ..) at columns 32 (k/2) + 8 (k%2) (+16 for lo)
+#pragma unroll
+                for (int k = 0; k < 8; ++k)
+                    mma_ts_w(tb + C::TM_MI, tb + C::TM_QK + 32 * (k >> 1) + 8 * (k & 1) + 16 * part,
+                             sdesc_sw128(sv, BLK128, 1024) + 128 * k, id_n, (part > 0 || k > 0) ? 1u : 0u);
+            }
+            mma_commit_w(acc_full);
+        }
+        mma_commit_w(mma_done);
+        mbar_wait_drain(mma_done, 0);
+    } else {
+        const int q4 = warp & 3;
+        const int x = 32 * q4 + (tid & 31);
+        const uint32_t lanes = tb + ((uint32_t)(32 * q4) << 16);
+        const float eta = p.eta[h];
+        gpowers(pw, CG + 1, p.lam[h], x);
+        gbar128();
+        // A_c as bf16 hi + lo, [D rows][D columns] in NB column blocks
+        {
+            const float *Ac = p.dA + ((size_t)bh * p.nC + c) * D * D;
+            for (int u = x; u < D * D / 8; u += 128) {
+                const int r = u / (D / 8), col = 8 * (u % (D / 8));
+                const float4 a0 = *reinterpret_cast<const float4 *>(Ac + r * D + col);
+                const float4 a1 = *reinterpret_cast<const float4 *>(Ac + r * D + col + 4);
+                uint32_t hi[4], lo[4];
+                gsplit(a0.x, a0.y, hi[0], lo[0]);
+                gsplit(a0.z, a0.w, hi[1], lo[1]);
+                gsplit(a1.x, a1.y, hi[2], lo[2]);
+                gsplit(a1.z, a1.w, hi[3], lo[3]);
+                const uint32_t off = (col >> 6) * C::ST_BLK + sw128_offset(r, col & 63);
+                *reinterpret_cast<uint4 *>(sm + C::OFF_A + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+                *reinterpret_cast<uint4 *>(sm + C::OFF_A + NB * C::ST_BLK + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+            }
+        }
+        bool ok = gwait(s_full, 0, abort, p);
+        if (ok) {
+            tc_fence_after();
+            const bool row_in = x < L;
+#pragma unroll 1
+            for (int jb = 0; jb < 4; ++jb) {
+                uint32_t qk[32];
+                tmem_ld32(lanes + C::TM_QK + 32 * jb, qk);
+                tmem_wait_ld();
+                uint32_t hi[16], lo[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                    float v[2];
+#pragma unroll
+                    for (int u = 0; u < 2; ++u) {
+                        const int l = 32 * jb + 2 * e + u;
+                        v[u] = (row_in && l <= x) ? eta * pw[x - l] * __uint_as_float(qk[2 * e + u]) : 0.f;
+                    }
+                    gsplit(v[0], v[1], hi[e], lo[e]);
+                }
+                tmem_st16(lanes + C::TM_QK + 32 * jb, hi);
+                tmem_st16(lanes + C::TM_QK + 32 * jb + 16, lo);
+            }
+            tmem_wait_st();
+        }
+        fence_async_smem();
+        tc_fence_before();
+        mbar_arrive(m_ready);
+        // every lane takes part in the collective loads; rows past L write nothing
+        if (ok && gwait(acc_full, 0, abort, p)) {
+            tc_fence_after();
+            const float dec = pw[min(x + 1, CG + 1)];
+            float *dst = p.mrow + ((size_t)bh * p.T + qrow0 + x) * D;
+#pragma unroll
+            for (int c0 = 0; c0 < D; c0 += 32) {
+                uint32_t a[32], b[32];
+                tmem_ld32(lanes + C::TM_MA + c0, a);
+                tmem_ld32(lanes + C::TM_MI + c0, b);
+                tmem_wait_ld();
+                if (x < L) {
+                    float4 *d4 = reinterpret_cast<float4 *>(dst + c0);
+#pragma unroll
+                    for (int u = 0; u < 8; ++u)
+                        d4[u] = make_float4(fmaf(dec, __uint_as_float(a[4 * u]), __uint_as_float(b[4 * u])),
+                                            fmaf(dec, __uint_as_float(a[4 * u + 1]), __uint_as_float(b[4 * u + 1])),
+                                            fmaf(dec, __uint_as_float(a[4 * u + 2]), __uint_as_float(b[4 * u + 2])),
+                                            fmaf(dec, __uint_as_float(a[4 * u + 3]), __uint_as_float(b[4 * u + 3])));
+                }
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tb, C::COLS);
+}
+
+// ===========================================================================
+// Halo + new rows of keys and values into one [BH][Tc][D] sequence.
+__global__ void gen_combine_kernel(const __nv_bfloat16 *halo, const __nv_bfloat16 *src, __nv_bfloat16 *dst,
+                                   int n_halo, int T, int D, int64_t BH) {
+    const int64_t per = (int64_t)(n_halo + T) * D / 8;  // 16-byte units per head
+    for (int64_t x = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; x < BH * per; x += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t bh = x / per, u = x % per;
+        const int64_t row = u * 8 / D, col = u * 8 % D;
+        const uint4 *s = row < n_halo
+                             ? reinterpret_cast<const uint4 *>(halo + (bh * n_halo + row) * D + col)
+                             : reinterpret_cast<const uint4 *>(src + (bh * T + row - n_halo) * D + col);
+        reinterpret_cast<uint4 *>(dst)[x] = *s;
+    }
+}
+
+typedef CUresult (*EncodeFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                             const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                             CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+// [BH][rows][D] bf16 -> 3D map (D, rows, BH), boxes of 64 columns x box_rows x 1, 128-byte swizzle
+bool gen_map(CUtensorMap *m, const void *base, int rows, int BH, int D, int box_rows) {
+    EncodeFn fn = reinterpret_cast<EncodeFn>(tensor_map_encoder());
+    if (!fn || rows < 1) return false;
+    cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)rows, (cuuint64_t)BH};
+    cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)rows * D * 2};
+    cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 1};
+    cuuint32_t es[3] = {1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, es,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+size_t gal(size_t x) { return (x + 255) & ~size_t(255); }
+
+struct GenLayout {
+    size_t kc, vc, mrow, dA, total;
+};
+GenLayout gen_layout(const tc_prefill_desc &d, int64_t n_halo) {
+    const int64_t BH = d.B * d.H, D = d.dk, Tc = n_halo + d.T;
+    const int64_t E = Tc > d.W ? Tc - d.W : 0, nC = (E + CG - 1) / CG;
+    const bool l1 = (d.flags & TC_PREFILL_L1_ONLY) != 0, state = (d.flags & TC_PREFILL_STATE_ONLY) != 0;
+    const bool delta = (d.flags & TC_PREFILL_DELTA_RULE) != 0;
+    GenLayout L;
+    L.kc = 0;
+    const size_t comb = n_halo > 0 ? gal((size_t)(BH * Tc * D) * 2) : 0;
+    L.vc = L.kc + comb;
+    L.mrow = L.vc + comb;
+    const size_t mrow = (!l1 && !state && !delta) ? gal((size_t)(BH * d.T * D) * sizeof(float)) : 0;
+    L.dA = L.mrow + mrow;
+    const size_t dA = (!l1 && !delta) ? gal((size_t)(BH * nC * D * D) * sizeof(float)) : 0;
+    L.total = L.dA + dA;
+    return L;
+}
+
+template <int NB>
+cudaError_t launch_general_t(const PrefillParams &pp, const float *mrow_in, cudaStream_t s) {
+    constexpr int D = 64 * NB;
+    tc_prefill_desc d{};
+    d.B = pp.B;
+    d.H = pp.H;
+    d.T = pp.T;
+    d.dk = pp.dk;
+    d.dv = pp.dv;
+    d.W = pp.W;
+    d.C = pp.C;
+    d.dtype = TC_BF16;
+    d.flags = (pp.l1_only ? TC_PREFILL_L1_ONLY : 0u) | (pp.state_only ? TC_PREFILL_STATE_ONLY : 0u) |
+              (pp.delta_rule ? TC_PREFILL_DELTA_RULE : 0u);
+    const GenLayout Lo = gen_layout(d, pp.n_halo);
+    char *ws = static_cast<char *>(pp.workspace);
+    const int BH = (int)(pp.B * pp.H);
+    GenParams p{};
+    p.q = static_cast<const __nv_bfloat16 *>(pp.q);
+    p.k = static_cast<const __nv_bfloat16 *>(pp.k);
+    p.v = static_cast<const __nv_bfloat16 *>(pp.v);
+    p.y = static_cast<__nv_bfloat16 *>(pp.y);
+    p.T = (int)pp.T;
+    p.n_halo = (int)pp.n_halo;
+    p.Tc = p.T + p.n_halo;
+    p.W = (int)(pp.W < p.Tc + 1 ? pp.W : p.Tc + 1);  // a window past the sequence changes nothing
+    p.H = (int)pp.H;
+    p.E = p.Tc > p.W ? p.Tc - p.W : 0;
+    p.nC = (p.E + CG - 1) / CG;
+    p.lam = pp.lam;
+    p.eta = pp.eta;
+    p.g = pp.g;
+    p.A_init = pp.A_init;
+    p.A_final = pp.A_final;
+    p.status = pp.status;
+    p.wait_ns = pp.wait_ns;
+    cudaError_t e;
+    if (p.n_halo > 0) {  // one sequence of keys and values, halo first
+        __nv_bfloat16 *kc = reinterpret_cast<__nv_bfloat16 *>(ws + Lo.kc);
+        __nv_bfloat16 *vc = reinterpret_cast<__nv_bfloat16 *>(ws + Lo.vc);
+        gen_combine_kernel<<<1184, 256, 0, s>>>(static_cast<const __nv_bfloat16 *>(pp.halo_k), p.k, kc, p.n_halo,
+                                                p.T, D, BH);
+        gen_combine_kernel<<<1184, 256, 0, s>>>(static_cast<const __nv_bfloat16 *>(pp.halo_v), p.v, vc, p.n_halo,
+                                                p.T, D, BH);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        p.k = kc;
+        p.v = vc;
+    }
+    const bool l2 = !pp.l1_only && !pp.delta_rule;
+    p.dA = l2 ? reinterpret_cast<float *>(ws + Lo.dA) : nullptr;
+    p.mrow = pp.delta_rule ? const_cast<float *>(mrow_in)
+                           : (l2 && !pp.state_only && p.nC > 0 ? reinterpret_cast<float *>(ws + Lo.mrow) : nullptr);
+    const bool queries = !pp.state_only && p.T > 0;
+    CUtensorMap mk128, mv128, mq128, mk64, mv64;
+    if ((queries || (l2 && p.nC > 0)) &&
+        (!gen_map(&mk128, p.k, p.Tc, BH, D, 128) || !gen_map(&mv128, p.v, p.Tc, BH, D, 128) ||
+         !gen_map(&mk64, p.k, p.Tc, BH, D, 64) || !gen_map(&mv64, p.v, p.Tc, BH, D, 64)))
+        return cudaErrorInvalidValue;
+    if (queries && !gen_map(&mq128, p.q, p.T, BH, D, 128)) return cudaErrorInvalidValue;
+    if (l2) {
+        if (p.nC > 0) {
+            e = cudaFuncSetAttribute(gen_sums_kernel<NB>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SUM_SMEM);
+            if (e != cudaSuccess) return e;
+            const int cpb = NB == 1 ? 2 : 1;
+            gen_sums_kernel<NB><<<dim3((unsigned)((p.nC + cpb - 1) / cpb), (unsigned)BH), kGThreads, SUM_SMEM, s>>>(
+                mk128, p);
+            if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        }
+        gen_scan_kernel<<<dim3((unsigned)((D * D + 255) / 256), (unsigned)BH), 256, 0, s>>>(p, D);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        if (queries && p.nC > 0) {
+            using RC = ReadCfg<NB>;
+            e = cudaFuncSetAttribute(gen_read_kernel<NB>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)RC::SMEM);
+            if (e != cudaSuccess) return e;
+            gen_read_kernel<NB><<<dim3((unsigned)p.nC, (unsigned)BH), kGThreads, RC::SMEM, s>>>(mq128, mk128, mv128, p);
+            if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        }
+    }
+    if (queries) {
+        using WC = WinCfg<NB>;
+        e = cudaFuncSetAttribute(gen_window_kernel<NB>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)WC::SMEM);
+        if (e != cudaSuccess) return e;
+        gen_window_kernel<NB><<<dim3((unsigned)((p.T + CG - 1) / CG), (unsigned)BH), kGThreads, WC::SMEM, s>>>(
+            mq128, mk64, mv64, p);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+}
+
+}  // namespace
+
+bool general_supported(const tc_prefill_desc &d, int64_t n_halo) {
+    if (d.dtype != TC_BF16 || d.dk != d.dv || (d.dk != 64 && d.dk != 128)) return false;
+    if (d.flags & TC_PREFILL_CHUNK_MEAN) return false;
+    if ((d.flags & TC_PREFILL_DELTA_RULE) && (n_halo != 0 || (d.flags & (TC_PREFILL_STATE_ONLY | TC_PREFILL_L1_ONLY))))
+        return false;
+    if (d.T + n_halo >= (int64_t(1) << 30) || d.B * d.H > 65535) return false;
+    return tensor_map_encoder() != nullptr;
+}
+
+size_t general_workspace_bytes(const tc_prefill_desc &d, int64_t n_halo) { return gen_layout(d, n_halo).total; }
+
+int general_launch_count(const tc_prefill_desc &d, int64_t n_halo) {
+    const int64_t Tc = n_halo + d.T, W = d.W < Tc + 1 ? d.W : Tc + 1, E = Tc > W ? Tc - W : 0;
+    const bool l1 = (d.flags & TC_PREFILL_L1_ONLY) != 0, state = (d.flags & TC_PREFILL_STATE_ONLY) != 0;
+    const bool delta = (d.flags & TC_PREFILL_DELTA_RULE) != 0;
+    const bool queries = !state && d.T > 0;
+    int n = n_halo > 0 ? 2 : 0;
+    if (!l1 && !delta) n += (E > 0 ? 1 : 0) + 1 + (queries && E > 0 ? 1 : 0);
+    return n + (queries ? 1 : 0);
+}
+
+cudaError_t launch_prefill_general(const PrefillParams &p, const float *mrow, cudaStream_t s) {
+    return p.dk == 64 ? launch_general_t<1>(p, mrow, s) : launch_general_t<2>(p, mrow, s);
+}
+
+}  // namespace tc

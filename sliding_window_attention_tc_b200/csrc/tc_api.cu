@@ -112,9 +112,18 @@ bool delta_window_on_sm100(const tc_prefill_desc &d, int64_t n_halo) {
     return use_sm100(l1, 0);
 }
 
+// Shapes the fused kernel does not take but the general tensor-core path does
+// (bf16, d_k = d_v in {64, 128}: any W, any halo).
+bool use_general(const tc_prefill_desc &d, int64_t n_halo) {
+    return !use_sm100(d, n_halo) && tc::general_supported(d, n_halo);
+}
+
 size_t prefill_ws(const tc_prefill_desc &d, int64_t n_halo, int num_sms) {
-    return use_sm100(d, n_halo) ? tc::sm100_workspace_bytes(d, num_sms)
-                                : tc::portable_workspace_bytes(d, n_halo);
+    if (use_sm100(d, n_halo)) return tc::sm100_workspace_bytes(d, num_sms);
+    if (use_general(d, n_halo))
+        return (d.flags & TC_PREFILL_DELTA_RULE) ? tc::delta_chunked_workspace_bytes(d)
+                                                 : tc::general_workspace_bytes(d, n_halo);
+    return tc::portable_workspace_bytes(d, n_halo);
 }
 
 // Variable-length calls run on the tensor-core path only (any longest
@@ -262,6 +271,16 @@ tc_status prefill_impl(const tc_prefill_desc *d, int64_t t0, const void *halo_k,
         if (e == cudaSuccess) e = tc::launch_delta_chunked(p, d->dtype, true, s);
         return e == cudaSuccess ? TC_OK : TC_ERR_CUDA;
     }
+    if (use_general(*d, n_halo)) {
+        cudaError_t e = cudaSuccess;
+        const float *mrow = nullptr;
+        if (p.delta_rule) {  // chunked delta memory into the workspace rows, then the window part
+            e = tc::launch_delta_chunked(p, d->dtype, false, s);
+            mrow = reinterpret_cast<const float *>(workspace);
+        }
+        if (e == cudaSuccess) e = tc::launch_prefill_general(p, mrow, s);
+        return e == cudaSuccess ? TC_OK : TC_ERR_CUDA;
+    }
     cudaError_t e = use_sm100(*d, n_halo) ? tc::launch_prefill_sm100(p, sms, s)
                                           : tc::launch_prefill_portable(p, d->dtype, s);
     return e == cudaSuccess ? TC_OK : TC_ERR_CUDA;
@@ -405,6 +424,9 @@ int tc_prefill_launch_count(const tc_prefill_desc *d) {
     if (use_sm100(*d, 0)) return tc::sm100_launch_count(*d);
     const bool l1_only = (d->flags & TC_PREFILL_L1_ONLY) != 0;
     const bool state_only = (d->flags & TC_PREFILL_STATE_ONLY) != 0;
+    if (use_general(*d, 0))
+        return ((d->flags & TC_PREFILL_DELTA_RULE) ? tc::delta_chunked_launch_count(*d) : 0) +
+               tc::general_launch_count(*d, 0);
     if ((d->flags & TC_PREFILL_DELTA_RULE) && !l1_only)  // chunked memory + the window part
         return tc::delta_chunked_launch_count(*d) + (d->T > 0 && !state_only ? 1 : 0);
     return (l1_only ? 0 : 1) + (d->T > 0 && !state_only ? 1 : 0);

@@ -191,6 +191,15 @@ cudaError_t launch_backward_chunks_tc(const tc_prefill_desc &d, const void *q, c
                                       const float *Hc, float *dq, float *dk, float *dv, float *part,
                                       int *status, unsigned long long wait_ns, cudaStream_t s);
 
+// prefill_general_sm100.cu: tensor-core prefill for bf16, d_k = d_v in {64,
+// 128}, any W and halo (what prefill_main_kernel does not take).  With the
+// delta rule (no halo) the memory's reads come from mrow ([BH][T][d] float32,
+// written by launch_delta_chunked); otherwise mrow is null.
+bool general_supported(const tc_prefill_desc &d, int64_t n_halo);
+size_t general_workspace_bytes(const tc_prefill_desc &d, int64_t n_halo);
+int general_launch_count(const tc_prefill_desc &d, int64_t n_halo);
+cudaError_t launch_prefill_general(const PrefillParams &p, const float *mrow, cudaStream_t s);
+
 // cuTensorMapEncodeTiled from the driver (null if unavailable).
 void *tensor_map_encoder();
 
