@@ -26,6 +26,7 @@ from __future__ import annotations
 import argparse
 import ctypes
 import json
+import math
 import os
 import statistics
 import subprocess
@@ -444,6 +445,43 @@ def time_training_extras(tc, dev, peaks=None, peak_src="fallback", steps=5):
     return out
 
 
+def time_general(tc, dev, steps=10, warmup=3):
+    """The general tensor-core prefill (the shapes the fused kernel does not
+    take): the LM workload at W = 500 (not a multiple of 128), and d = 128 with
+    W = 2048 (the decode workload's head size and window) over 8 x 32 heads
+    of 4096 tokens.  Device-resident inputs, CUDA events, ms per call."""
+    out = {}
+    x, sets, prm = _prefill_device_inputs(HEADLINE, dev, copies=1)
+    q, k, v = sets[0]
+    B, H, T, d = q.shape
+    W = 500
+    ms = statistics.median(time_calls(lambda: tc.prefill(q, k, v, *prm, W, x.C), steps, warmup))
+    l1f, l2f = prefill_flops(B, H, T, d, d, W)
+    desc = tc.make_prefill_desc(B, H, T, d, d, W, x.C, tc.TC_BF16)
+    out["lm_w500"] = {"B": B, "H": H, "T": T, "d": d, "W": W, "ms": ms,
+                      "tokens_per_s": B * H * T / (ms * 1e-3),
+                      "algorithmic_tflops": (l1f + l2f) / (ms * 1e-3) / 1e12,
+                      "launches_per_call": tc.prefill_launch_count(desc)}
+    del sets, q, k, v
+    B, H, T, d, W = 8, 32, 4096, 128, 2048
+    gen = torch.Generator(device=dev).manual_seed(1005)
+    q, k, v = ((torch.randn(B, H, T, d, generator=gen, device=dev) / math.sqrt(d)).to(torch.bfloat16)
+               for _ in range(3))
+    lam = 0.99 + 0.0099 * torch.rand(H, generator=gen, device=dev)
+    eta = 0.1 + 0.9 * torch.rand(H, generator=gen, device=dev)
+    g = torch.randn(H, generator=gen, device=dev)
+    ms = statistics.median(time_calls(lambda: tc.prefill(q, k, v, lam, eta, g, W, 128), steps, warmup))
+    l1f, l2f = prefill_flops(B, H, T, d, d, W)
+    desc = tc.make_prefill_desc(B, H, T, d, d, W, 128, tc.TC_BF16)
+    out["d128_w2048"] = {"B": B, "H": H, "T": T, "d": d, "W": W, "ms": ms,
+                         "tokens_per_s": B * H * T / (ms * 1e-3),
+                         "algorithmic_tflops": (l1f + l2f) / (ms * 1e-3) / 1e12,
+                         "launches_per_call": tc.prefill_launch_count(desc)}
+    del q, k, v
+    torch.cuda.empty_cache()
+    return out
+
+
 def time_varlen(tc, dev, steps=20, warmup=3):
     """The variable-length workload in one tc_prefill_varlen call, against the
     same sequences run as one tc_prefill call each (device-resident inputs,
@@ -587,6 +625,9 @@ def run_only(args, tc, dev, world, peaks):
     if args.only == "varlen":
         print(json.dumps({"only": "varlen", **time_varlen(tc, dev, args.steps, args.warmup)}))
         return 0
+    if args.only == "general":
+        print(json.dumps({"only": "general", **time_general(tc, dev, args.steps, args.warmup)}))
+        return 0
     if args.only == "backward":
         print(json.dumps({"only": "backward",
                           **time_training_extras(tc, dev, peaks, steps=args.steps)["backward"]}))
@@ -612,7 +653,8 @@ def main():
     ap.add_argument("--impl", default="tc", choices=["tc", "reference"])
     ap.add_argument("--no-extras", action="store_true",
                     help="headline prefill only (skip decode, long prefill, oracle)")
-    ap.add_argument("--only", choices=["prefill", "long", "decode", "varlen", "backward"], default=None,
+    ap.add_argument("--only", choices=["prefill", "long", "decode", "varlen", "backward", "general"],
+                    default=None,
                     help="time one workload only and print its numbers (profiling runs)")
     ap.add_argument("--decode-batch", type=int, default=None,
                     help="batch of the decode workload (default 256)")
@@ -706,6 +748,7 @@ def main():
                         "h2d_bytes_per_step": dec["e2e_h2d_bytes"],
                         "d2h_bytes_per_step": dec["e2e_d2h_bytes"]}}
             extras["varlen_prefill"] = time_varlen(tc, dev)
+            extras["general_prefill"] = time_general(tc, dev)
             extras.update(time_training_extras(tc, dev, peaks, peak_src))
         e2e = time_prefill_e2e(tc, HEADLINE, dev, max(5, min(20, args.steps // 10)))
     finally:
