@@ -628,6 +628,13 @@ def run_only(args, tc, dev, world, peaks):
     if args.only == "general":
         print(json.dumps({"only": "general", **time_general(tc, dev, args.steps, args.warmup)}))
         return 0
+    if args.only == "delta":
+        x, sets, prm = _prefill_device_inputs(HEADLINE, dev, copies=1)
+        q, k, v = sets[0]
+        ms = statistics.median(time_calls(lambda: tc.prefill(q, k, v, *prm, x.W, x.C, delta_rule=True),
+                                          args.steps, args.warmup))
+        print(json.dumps({"only": "delta", "workload": HEADLINE, "ms": ms}))
+        return 0
     if args.only == "backward":
         print(json.dumps({"only": "backward",
                           **time_training_extras(tc, dev, peaks, steps=args.steps)["backward"]}))
@@ -653,7 +660,7 @@ def main():
     ap.add_argument("--impl", default="tc", choices=["tc", "reference"])
     ap.add_argument("--no-extras", action="store_true",
                     help="headline prefill only (skip decode, long prefill, oracle)")
-    ap.add_argument("--only", choices=["prefill", "long", "decode", "varlen", "backward", "general"],
+    ap.add_argument("--only", choices=["prefill", "long", "decode", "varlen", "backward", "general", "delta"],
                     default=None,
                     help="time one workload only and print its numbers (profiling runs)")
     ap.add_argument("--decode-batch", type=int, default=None,

@@ -107,7 +107,7 @@ struct WinCfg {
 };
 
 template <int NB>
-__global__ void __launch_bounds__(kGThreads, 1)
+__global__ void __launch_bounds__(kGThreads, NB == 1 ? 2 : 1)
     gen_window_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                       const __grid_constant__ CUtensorMap tv, GenParams p) {
     using C = WinCfg<NB>;
@@ -215,20 +215,19 @@ __global__ void __launch_bounds__(kGThreads, 1)
             if (!(ok = gwait(s_full, n & 1, abort, p))) break;
             tc_fence_after();
             const int base = tau - (xs + GX * n);  // tau - j = base - c
-            uint32_t sr[2][32];
-            tmem_ld32(lanes + C::TM_S, sr[0]);
-            tmem_ld32(lanes + C::TM_S + 32, sr[1]);
-            tmem_wait_ld();
+            // the row max over both 32-column halves, then the exponentials from a
+            // second read of the scores (fewer live registers)
             float mx = -INFINITY;
 #pragma unroll
-            for (int h = 0; h < 2; ++h)
+            for (int h = 0; h < 2; ++h) {
+                uint32_t sr[32];
+                tmem_ld32(lanes + C::TM_S + 32 * h, sr);
+                tmem_wait_ld();
 #pragma unroll
-                for (int c = 0; c < 32; ++c) {
-                    const bool in = (uint32_t)(base - (32 * h + c)) < wlim;
-                    const float x = in ? __uint_as_float(sr[h][c]) * sl2 : -INFINITY;
-                    sr[h][c] = __float_as_uint(x);
-                    mx = fmaxf(mx, x);
-                }
+                for (int c = 0; c < 32; ++c)
+                    if ((uint32_t)(base - (32 * h + c)) < wlim) mx = fmaxf(mx, __uint_as_float(sr[c]));
+            }
+            mx *= sl2;
             const float m_new = fmaxf(m_run, mx);
             const float corr = m_new == -INFINITY ? 1.f : gex2(m_run - m_new);
             // rescale O (complete: this tile's scores were committed after the previous P V)
@@ -244,13 +243,18 @@ __global__ void __launch_bounds__(kGThreads, 1)
                 }
             }
             float sum = 0.f;
+            const float neg_m = m_new == -INFINITY ? 0.f : -m_new;
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
+                uint32_t sr[32];
+                tmem_ld32(lanes + C::TM_S + 32 * h, sr);
+                tmem_wait_ld();
                 uint32_t pk[16];
 #pragma unroll
                 for (int e = 0; e < 16; ++e) {
-                    const float a = m_new == -INFINITY ? 0.f : gex2(__uint_as_float(sr[h][2 * e]) - m_new);
-                    const float b = m_new == -INFINITY ? 0.f : gex2(__uint_as_float(sr[h][2 * e + 1]) - m_new);
+                    const int c = 32 * h + 2 * e;
+                    const float a = (uint32_t)(base - c) < wlim ? gex2(fmaf(__uint_as_float(sr[2 * e]), sl2, neg_m)) : 0.f;
+                    const float b = (uint32_t)(base - c - 1) < wlim ? gex2(fmaf(__uint_as_float(sr[2 * e + 1]), sl2, neg_m)) : 0.f;
                     sum += a + b;
                     pk[e] = pack_bf16(a, b);
                 }
