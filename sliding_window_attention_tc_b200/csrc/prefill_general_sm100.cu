@@ -89,10 +89,12 @@ __device__ __forceinline__ void tma_rows_nb(uint8_t *dst, const CUtensorMap *m, 
 
 // ===========================================================================
 // Window part.  A CTA owns 128 new query rows (TMEM lanes); 64-row key
-// tiles stream through NS stages.  Per tile: S = Q K^T into TMEM; the
-// element-wise warps take the row max, rescale O in TMEM when it grew (O is
-// complete then: the scores' commit follows the previous P V), write
-// P = exp2(s - m) as bf16 over S, and O += P V runs from TMEM.
+// tiles stream through NS stages.  Scores have two TMEM buffers: S of tile
+// n+1 is issued before P V of tile n, so the element-wise warps find the
+// next scores ready when they finish a tile.  Per tile they take the row max,
+// rescale O in TMEM when it grew (after waiting for the previous P V, which a
+// per-tile commit reports), write P = exp2(s - m) as bf16 over S, and
+// O += P V runs from TMEM.
 template <int NB>
 struct WinCfg {
     static constexpr int D = 64 * NB;
@@ -102,8 +104,8 @@ struct WinCfg {
     static constexpr uint32_t OFF_Q = 0;
     static constexpr uint32_t OFF_X = Q_B;         // NS x (K tile, V tile)
     static constexpr uint32_t OFF_BAR = OFF_X + NS * 2 * X_B;
-    static constexpr uint32_t SMEM = OFF_BAR + 128 + 1024;
-    static constexpr uint32_t TM_S = 0, TM_O = 64, COLS = NB == 1 ? 128 : 256;
+    static constexpr uint32_t SMEM = OFF_BAR + 256 + 1024;  // (8 + 2 NS) barriers, TMEM address, abort flag
+    static constexpr uint32_t TM_S = 0, TM_O = 128, COLS = 256;  // two 64-column score buffers, then O
 };
 
 template <int NB>
@@ -116,7 +118,7 @@ __global__ void __launch_bounds__(kGThreads, NB == 1 ? 2 : 1)
     uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + C::OFF_BAR);
     uint64_t *q_full = bars, *x_full = bars + 1, *x_empty = x_full + NS, *s_full = x_empty + NS;
-    uint64_t *p_ready = s_full + 1, *o_full = p_ready + 1, *mma_done = o_full + 1;
+    uint64_t *p_ready = s_full + 2, *o_done = p_ready + 2, *o_full = o_done + 1, *mma_done = o_full + 1;
     uint32_t *tmem_base = reinterpret_cast<uint32_t *>(mma_done + 1);
     volatile int *abort = reinterpret_cast<volatile int *>(tmem_base + 1);
 
@@ -134,8 +136,11 @@ __global__ void __launch_bounds__(kGThreads, NB == 1 ? 2 : 1)
             mbar_init(&x_full[s], 1);
             mbar_init(&x_empty[s], 1);
         }
-        mbar_init(s_full, 1);
-        mbar_init(p_ready, 4);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&s_full[b], 1);
+            mbar_init(&p_ready[b], 4);
+        }
+        mbar_init(o_done, 1);
         mbar_init(o_full, 1);
         mbar_init(mma_done, 1);
         *abort = 0;
@@ -174,30 +179,34 @@ __global__ void __launch_bounds__(kGThreads, NB == 1 ? 2 : 1)
         const uint32_t id_o = idesc_bf16(128, D, false, true);
         const uint32_t sq = smem_u32(sm + C::OFF_Q), sx = smem_u32(sm + C::OFF_X);
         bool ok = gwait(q_full, 0, abort, p);
-        for (int n = 0; ok && n <= N; ++n) {
-            if (n > 0) {
-                const int m = n - 1, sp = m % NS;
-                if (!(ok = gwait(p_ready, m & 1, abort, p))) break;
-                tc_fence_after();
-                // O += P V: P (64 keys) in the score columns, V read MN-major
-                const uint64_t vd = sdesc_sw128(sx + sp * 2 * C::X_B + C::X_B, BLK64, 1024);
-#pragma unroll
-                for (int k = 0; k < 4; ++k)
-                    mma_ts_w(tb + C::TM_O, tb + C::TM_S + 8 * k, vd + 128 * k, id_o, (m > 0 || k > 0) ? 1u : 0u);
-                mma_commit_w(&x_empty[sp]);
-            }
-            if (n == N) break;
-            const int s = n % NS;
-            if (!(ok = gwait(&x_full[s], (n / NS) & 1, abort, p))) break;
+        // S(n) into score buffer n % 2
+        auto issue_s = [&](int n) -> bool {
+            const int st = n % NS;
+            if (!gwait(&x_full[st], (n / NS) & 1, abort, p)) return false;
             tc_fence_after();
-            const uint32_t kx = sx + s * 2 * C::X_B;
+            const uint32_t kx = sx + st * 2 * C::X_B, sb = tb + C::TM_S + 64 * (n & 1);
 #pragma unroll
             for (int b = 0; b < NB; ++b)
 #pragma unroll
                 for (int k = 0; k < 4; ++k)
-                    mma_ss_w(tb + C::TM_S, sdesc_sw128(sq + b * BLK128, 16, 1024) + 2 * k,
+                    mma_ss_w(sb, sdesc_sw128(sq + b * BLK128, 16, 1024) + 2 * k,
                              sdesc_sw128(kx + b * BLK64, 16, 1024) + 2 * k, id_s, (b > 0 || k > 0) ? 1u : 0u);
-            mma_commit_w(s_full);
+            mma_commit_w(&s_full[n & 1]);
+            return true;
+        };
+        if (ok) ok = issue_s(0);
+        for (int n = 0; ok && n < N; ++n) {
+            // the next scores go out before this tile's P V
+            if (n + 1 < N && !(ok = issue_s(n + 1))) break;
+            if (!(ok = gwait(&p_ready[n & 1], (n >> 1) & 1, abort, p))) break;
+            tc_fence_after();
+            // O += P V: P (64 keys) in score buffer n % 2, V read MN-major
+            const uint64_t vd = sdesc_sw128(sx + (n % NS) * 2 * C::X_B + C::X_B, BLK64, 1024);
+            const uint32_t pb = tb + C::TM_S + 64 * (n & 1);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) mma_ts_w(tb + C::TM_O, pb + 8 * k, vd + 128 * k, id_o, (n > 0 || k > 0) ? 1u : 0u);
+            mma_commit_w(&x_empty[n % NS]);
+            mma_commit_w(o_done);
         }
         if (ok) mma_commit_w(o_full);
         mma_commit_w(mma_done);
@@ -212,8 +221,9 @@ __global__ void __launch_bounds__(kGThreads, NB == 1 ? 2 : 1)
         float m_run = -INFINITY, l_run = 0.f;
         bool ok = true;
         for (int n = 0; n < N; ++n) {
-            if (!(ok = gwait(s_full, n & 1, abort, p))) break;
+            if (!(ok = gwait(&s_full[n & 1], (n >> 1) & 1, abort, p))) break;
             tc_fence_after();
+            const uint32_t sbuf = lanes + C::TM_S + 64 * (n & 1);
             const int base = tau - (xs + GX * n);  // tau - j = base - c
             // the row max over both 32-column halves, then the exponentials from a
             // second read of the scores (fewer live registers)
@@ -221,7 +231,7 @@ __global__ void __launch_bounds__(kGThreads, NB == 1 ? 2 : 1)
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
                 uint32_t sr[32];
-                tmem_ld32(lanes + C::TM_S + 32 * h, sr);
+                tmem_ld32(sbuf + 32 * h, sr);
                 tmem_wait_ld();
 #pragma unroll
                 for (int c = 0; c < 32; ++c)
@@ -230,8 +240,12 @@ __global__ void __launch_bounds__(kGThreads, NB == 1 ? 2 : 1)
             mx *= sl2;
             const float m_new = fmaxf(m_run, mx);
             const float corr = m_new == -INFINITY ? 1.f : gex2(m_run - m_new);
-            // rescale O (complete: this tile's scores were committed after the previous P V)
+            // rescale O once the previous P V is complete (its commit is the
+            // (n-1)-th completion of o_done; the n-th cannot come before this
+            // tile's P, so the parity names it unambiguously)
             if (n > 0 && __any_sync(0xffffffffu, corr != 1.f)) {
+                if (!(ok = gwait(o_done, (n - 1) & 1, abort, p))) break;
+                tc_fence_after();
 #pragma unroll
                 for (int c0 = 0; c0 < D; c0 += 32) {
                     uint32_t o[32];
@@ -247,7 +261,7 @@ __global__ void __launch_bounds__(kGThreads, NB == 1 ? 2 : 1)
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
                 uint32_t sr[32];
-                tmem_ld32(lanes + C::TM_S + 32 * h, sr);
+                tmem_ld32(sbuf + 32 * h, sr);
                 tmem_wait_ld();
                 uint32_t pk[16];
 #pragma unroll
@@ -258,14 +272,14 @@ __global__ void __launch_bounds__(kGThreads, NB == 1 ? 2 : 1)
                     sum += a + b;
                     pk[e] = pack_bf16(a, b);
                 }
-                tmem_st16(lanes + C::TM_S + 16 * h, pk);
+                tmem_st16(sbuf + 16 * h, pk);
             }
             l_run = fmaf(l_run, corr, sum);
             m_run = m_new;
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
-            mbar_arrive_w(p_ready);
+            mbar_arrive_w(&p_ready[n & 1]);
         }
         if (ok && gwait(o_full, 0, abort, p)) {
             tc_fence_after();
