@@ -292,10 +292,7 @@ TC_API tc_status tc_prefill_host(const tc_prefill_desc *desc, const void *q, con
  * All calls share the array and leave their data in it; no call depends on
  * what an earlier one left, but calls whose kernels may overlap on the GPU
  * (unordered streams) race on it and must not be issued that way.
- * Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
- * The array's device address is looked up once per device and kept for the
- * life of the process, so this entry point must not be used after a
- * cudaDeviceReset of that device. */
+ * Allocates nothing: no cudaMalloc, cudaFree or allocating library call. */
 TC_API tc_status tc_prefill_no_alloc(const tc_prefill_desc *desc, const void *q, const void *k,
                                      const void *v, const float *lambda, const float *eta,
                                      const float *g, void *y, float *A_final, tc_stream_t stream);
