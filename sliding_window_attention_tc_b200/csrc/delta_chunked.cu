@@ -89,40 +89,46 @@ __device__ __forceinline__ void store4(__nv_bfloat16 *p, const float (&f)[4]) {
     *reinterpret_cast<uint2 *>(p) = make_uint2(pack_bf16_rn(f[0], f[1]), pack_bf16_rn(f[2], f[3]));
 }
 
-// rows r0 .. r0+n_valid-1 of a [.][d] tensor into shared rows of stride sp,
-// scaled by scale(row); rows n_valid .. CD-1 are zero.  Four elements per
-// load when d is a multiple of 4.
-template <typename Tin, class F>
-__device__ __forceinline__ void load_rows_scaled(float *dst, int sp, const Tin *src, int64_t r0, int n_valid, int d,
-                                                 F scale) {
-    if ((d & 3) == 0) {
-        const int d4 = d >> 2;
-        for (int x = threadIdx.x; x < CD * d4; x += blockDim.x) {
-            const int i = x / d4, c = 4 * (x - i * d4);
-            float f[4] = {0.f, 0.f, 0.f, 0.f};
-            if (i < n_valid) {
-                load4(src + (r0 + i) * d + c, f);
-                const float sc = scale(i);
+// acc[u][v] = sum_k a(k)[u] b(k)[v] over k < K, with a(k), b(k) four
+// consecutive floats of shared memory (16-byte loads): one 4 x 4 block of a
+// product whose operands are stored so that both are contiguous along the
+// block's rows and columns.
+template <class FA, class FB>
+__device__ __forceinline__ void tile44v(int K, FA a, FB b, float (&acc)[4][4]) {
 #pragma unroll
-                for (int u = 0; u < 4; ++u) f[u] *= sc;
-            }
+    for (int u = 0; u < 4; ++u)
 #pragma unroll
-            for (int u = 0; u < 4; ++u) dst[i * sp + c + u] = f[u];
-        }
-        return;
+        for (int v = 0; v < 4; ++v) acc[u][v] = 0.f;
+#pragma unroll 4
+    for (int k = 0; k < K; ++k) {
+        const float4 x = a(k), y = b(k);
+        const float xs[4] = {x.x, x.y, x.z, x.w}, ys[4] = {y.x, y.y, y.z, y.w};
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+#pragma unroll
+            for (int v = 0; v < 4; ++v) acc[u][v] = fmaf(xs[u], ys[v], acc[u][v]);
     }
-    for (int x = threadIdx.x; x < CD * d; x += blockDim.x) {
-        const int i = x / d, c = x % d;
-        dst[i * sp + c] = i < n_valid ? scale(i) * to_f32(src[(r0 + i) * d + c]) : 0.f;
-    }
+}
+__device__ __forceinline__ float4 lds4(const float *p) { return *reinterpret_cast<const float4 *>(p); }
+__host__ __device__ __forceinline__ int up4(int x) { return (x + 3) & ~3; }
+
+// Shared-memory floats of the two per-chunk kernels (head sizes padded to
+// multiples of 4 with zero columns; row pitches multiples of 4).
+__host__ __device__ __forceinline__ int prep_floats(int dk, int dv) {
+    const int dk4 = up4(dk), nx4 = up4(dv) + dk4;
+    return 68 + dk4 * (CD + 4) + CD * (dk4 + 4) + CD * (nx4 + 4) + CD * (CD + 4);
+}
+__host__ __device__ __forceinline__ int read_floats(int dk, int dv) {
+    const int dk4 = up4(dk), dv4 = up4(dv);
+    return 68 + dk4 * (dv4 + 4) + CD * (dv4 + 4) + 3 * dk4 * (CD + 4) + CD * (CD + 4);
 }
 
 template <typename Tin>
 __global__ void __launch_bounds__(kDThreads) delta_prep_kernel(PrefillParams p, DeltaBufs w) {
-    extern __shared__ float sh[];
-    const int dk = p.dk, dv = p.dv, nx = dv + dk;
-    const int skp = dk + 1, sxp = nx + 1;
-    float *sK = sh, *X = sK + CD * skp, *sN = X + CD * sxp, *pw = sN + CD * (CD + 1);
+    extern __shared__ __align__(16) float sh[];
+    const int dk = p.dk, dv = p.dv, dk4 = up4(dk), dv4 = up4(dv), nx4 = dv4 + dk4;
+    const int tp = CD + 4, kgp = dk4 + 4, xp = nx4 + 4, np = CD + 4;
+    float *pw = sh, *sKT = pw + 68, *sKG = sKT + dk4 * tp, *X = sKG + CD * kgp, *sN = X + CD * xp;
     const int64_t bh = blockIdx.y, T = p.T, E = w.E;
     const int c = blockIdx.x, h = (int)(bh % p.H);
     const int64_t e0 = (int64_t)c * CD;
@@ -130,24 +136,33 @@ __global__ void __launch_bounds__(kDThreads) delta_prep_kernel(PrefillParams p, 
     const float eta = p.eta[h];
     powers(pw, CD, p.lam[h]);
     __syncthreads();
-    const Tin *kb = reinterpret_cast<const Tin *>(p.k) + bh * T * dk;
-    const Tin *vb = reinterpret_cast<const Tin *>(p.v) + bh * T * dv;
-    load_rows_scaled(sK, skp, kb, e0, L, dk, [](int) { return 1.f; });
-    load_rows_scaled(X, sxp, vb, e0, L, dv, [](int) { return 1.f; });
-    load_rows_scaled(X + dv, sxp, kb, e0, L, dk, [&](int i) { return pw[i]; });
+    const Tin *kb = reinterpret_cast<const Tin *>(p.k) + (bh * T + e0) * dk;
+    const Tin *vb = reinterpret_cast<const Tin *>(p.v) + (bh * T + e0) * dv;
+    // K^T; K scaled by G = lam^(L-1-i); X = [V | diag(lam^i) K]; zero past L and in the pads
+    for (int x = threadIdx.x; x < CD * dk4; x += blockDim.x) {
+        const int i = x / dk4, r = x - i * dk4;
+        const float kv = (i < L && r < dk) ? to_f32(kb[(int64_t)i * dk + r]) : 0.f;
+        sKT[r * tp + i] = kv;
+        sKG[i * kgp + r] = i < L ? pw[L - 1 - i] * kv : 0.f;
+        X[i * xp + dv4 + r] = pw[i] * kv;
+    }
+    for (int x = threadIdx.x; x < CD * dv4; x += blockDim.x) {
+        const int i = x / dv4, cc = x - i * dv4;
+        X[i * xp + cc] = (i < L && cc < dv) ? to_f32(vb[(int64_t)i * dv + cc]) : 0.f;
+    }
     __syncthreads();
     // N[i][l] = eta lam^(i-1-l) (k_i . k_l) for l < i < L
     for (int t = threadIdx.x; t < (CD / 4) * (CD / 4); t += blockDim.x) {
         const int i0 = 4 * (t / (CD / 4)), l0 = 4 * (t % (CD / 4));
         float acc[4][4];
-        tile44(dk, i0, l0, [&](int i, int r) { return sK[i * skp + r]; },
-               [&](int r, int l) { return sK[l * skp + r]; }, acc);
+        tile44v(dk4, [&](int r) { return lds4(sKT + r * tp + i0); }, [&](int r) { return lds4(sKT + r * tp + l0); },
+                acc);
 #pragma unroll
         for (int u = 0; u < 4; ++u)
 #pragma unroll
             for (int v = 0; v < 4; ++v) {
                 const int i = i0 + u, l = l0 + v;
-                sN[i * (CD + 1) + l] = (l < i && i < L) ? eta * pw[i - 1 - l] * acc[u][v] : 0.f;
+                sN[i * np + l] = (l < i && i < L) ? eta * pw[i - 1 - l] * acc[u][v] : 0.f;
             }
     }
     __syncthreads();
@@ -156,43 +171,44 @@ __global__ void __launch_bounds__(kDThreads) delta_prep_kernel(PrefillParams p, 
     // block's rows go one by one over at most kSB - 1 earlier rows each
     for (int b0 = 0; b0 < L; b0 += kSB) {
         if (b0 > 0) {
-            for (int x = threadIdx.x; x < kSB * nx; x += blockDim.x) {
-                const int i = b0 + x / nx, col = x % nx;
+            for (int x = threadIdx.x; x < kSB * nx4; x += blockDim.x) {
+                const int i = b0 + x / nx4, col = x % nx4;
                 float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
                 for (int l = 0; l < b0; l += 4) {
-                    a0 = fmaf(sN[i * (CD + 1) + l], X[l * sxp + col], a0);
-                    a1 = fmaf(sN[i * (CD + 1) + l + 1], X[(l + 1) * sxp + col], a1);
-                    a2 = fmaf(sN[i * (CD + 1) + l + 2], X[(l + 2) * sxp + col], a2);
-                    a3 = fmaf(sN[i * (CD + 1) + l + 3], X[(l + 3) * sxp + col], a3);
+                    const float4 nv = lds4(sN + i * np + l);
+                    a0 = fmaf(nv.x, X[l * xp + col], a0);
+                    a1 = fmaf(nv.y, X[(l + 1) * xp + col], a1);
+                    a2 = fmaf(nv.z, X[(l + 2) * xp + col], a2);
+                    a3 = fmaf(nv.w, X[(l + 3) * xp + col], a3);
                 }
-                X[i * sxp + col] -= (a0 + a1) + (a2 + a3);
+                X[i * xp + col] -= (a0 + a1) + (a2 + a3);
             }
             __syncthreads();
         }
         const int b1 = b0 + kSB < L ? b0 + kSB : L;
         for (int i = b0 + 1; i < b1; ++i) {
-            for (int col = threadIdx.x; col < nx; col += blockDim.x) {
-                float a = X[i * sxp + col];
-                for (int l = b0; l < i; ++l) a = fmaf(-sN[i * (CD + 1) + l], X[l * sxp + col], a);
-                X[i * sxp + col] = a;
+            for (int col = threadIdx.x; col < nx4; col += blockDim.x) {
+                float a = X[i * xp + col];
+                for (int l = b0; l < i; ++l) a = fmaf(-sN[i * np + l], X[l * xp + col], a);
+                X[i * xp + col] = a;
             }
             __syncthreads();
         }
     }
     // Ut, Wt rows
     float *Ut = w.Ut + (bh * E + e0) * dv, *Wt = w.Wt + (bh * E + e0) * dk;
-    for (int x = threadIdx.x; x < L * dv; x += blockDim.x) Ut[x] = X[(x / dv) * sxp + x % dv];
-    for (int x = threadIdx.x; x < L * dk; x += blockDim.x) Wt[x] = X[(x / dk) * sxp + dv + x % dk];
-    // P = lam^L I - eta K^T G Wt,  Q = eta K^T G Ut
+    for (int x = threadIdx.x; x < L * dv; x += blockDim.x) Ut[x] = X[(x / dv) * xp + x % dv];
+    for (int x = threadIdx.x; x < L * dk; x += blockDim.x) Wt[x] = X[(x / dk) * xp + dv4 + x % dk];
+    // P = lam^L I - eta K^T G Wt,  Q = eta K^T G Ut: rows r of K^T G, columns of [Wt | Ut]
     float *P = w.P + ((size_t)bh * w.nC + c) * dk * dk, *Q = w.Q + ((size_t)bh * w.nC + c) * dk * dv;
-    const int tk = (dk + 3) / 4, tv = (dv + 3) / 4;
+    const int tk = dk4 / 4, tv = dv4 / 4;
     for (int t = threadIdx.x; t < tk * (tk + tv); t += blockDim.x) {
         const int r0 = 4 * (t / (tk + tv)), cb = t % (tk + tv);
         const bool isP = cb < tk;
-        const int c0 = 4 * (isP ? cb : cb - tk), off = isP ? dv : 0, ncol = isP ? dk : dv;
+        const int c0 = 4 * (isP ? cb : cb - tk), off = isP ? dv4 : 0, ncol = isP ? dk : dv;
         float acc[4][4];
-        tile44(L, r0, c0, [&](int r, int l) { return r < dk ? pw[L - 1 - l] * sK[l * skp + r] : 0.f; },
-               [&](int l, int cc) { return cc < ncol ? X[l * sxp + off + cc] : 0.f; }, acc);
+        tile44v(L, [&](int l) { return lds4(sKG + l * kgp + r0); }, [&](int l) { return lds4(X + l * xp + off + c0); },
+                acc);
 #pragma unroll
         for (int u = 0; u < 4; ++u)
 #pragma unroll
@@ -286,11 +302,11 @@ __global__ void __launch_bounds__(kDThreads) delta_scan_kernel(PrefillParams p, 
 template <typename Tin>
 __global__ void __launch_bounds__(kDThreads) delta_read_kernel(PrefillParams p, DeltaBufs w, float *mrow,
                                                                int add_y) {
-    extern __shared__ float sh[];
-    const int dk = p.dk, dv = p.dv;
-    const int skp = dk + 1, svp = dv + 1, sgp = CD + 1;
-    float *sS = sh, *sU = sS + dk * dv, *sK = sU + CD * svp, *sQ = sK + CD * skp;
-    float *sWt = sQ + CD * skp, *sG = sWt + CD * skp, *pw = sG + CD * sgp;
+    extern __shared__ __align__(16) float sh[];
+    const int dk = p.dk, dv = p.dv, dk4 = up4(dk), dv4 = up4(dv);
+    const int sp = dv4 + 4, tp = CD + 4;
+    float *pw = sh, *sS = pw + 68, *sU = sS + dk4 * sp, *sKT = sU + CD * sp, *sQT = sKT + dk4 * tp;
+    float *sWT = sQT + dk4 * tp, *sGT = sWT + dk4 * tp;
     const int64_t bh = blockIdx.y, T = p.T, W = p.W, E = w.E;
     const int c = blockIdx.x, h = (int)(bh % p.H);
     const int64_t e0 = (int64_t)c * CD;
@@ -298,39 +314,49 @@ __global__ void __launch_bounds__(kDThreads) delta_read_kernel(PrefillParams p, 
     const float eta = p.eta[h];
     powers(pw, CD, p.lam[h]);
     const float *S = w.S + ((size_t)bh * w.nC + c) * dk * dv;
-    for (int x = threadIdx.x; x < dk * dv; x += blockDim.x) sS[x] = S[x];
-    const Tin *kb = reinterpret_cast<const Tin *>(p.k) + bh * T * dk;
-    const Tin *qb = reinterpret_cast<const Tin *>(p.q) + bh * T * dk;
-    load_rows_scaled(sK, skp, kb, e0, L, dk, [](int) { return 1.f; });
-    load_rows_scaled(sQ, skp, qb, e0 + W, L, dk, [](int) { return 1.f; });
-    load_rows_scaled(sWt, skp, w.Wt + bh * E * dk, e0, L, dk, [](int) { return 1.f; });
-    load_rows_scaled(sU, svp, w.Ut + bh * E * dv, e0, L, dv, [](int) { return 1.f; });
+    for (int x = threadIdx.x; x < dk4 * dv4; x += blockDim.x) {
+        const int r = x / dv4, cc = x - r * dv4;
+        sS[r * sp + cc] = (r < dk && cc < dv) ? S[r * dv + cc] : 0.f;
+    }
+    const Tin *kb = reinterpret_cast<const Tin *>(p.k) + (bh * T + e0) * dk;
+    const Tin *qb = reinterpret_cast<const Tin *>(p.q) + (bh * T + e0 + W) * dk;
+    const float *wt = w.Wt + (bh * E + e0) * dk, *ut = w.Ut + (bh * E + e0) * dv;
+    for (int x = threadIdx.x; x < CD * dk4; x += blockDim.x) {
+        const int i = x / dk4, r = x - i * dk4;
+        const bool in = i < L && r < dk;
+        sKT[r * tp + i] = in ? to_f32(kb[(int64_t)i * dk + r]) : 0.f;
+        sQT[r * tp + i] = in ? to_f32(qb[(int64_t)i * dk + r]) : 0.f;
+        sWT[r * tp + i] = in ? wt[i * dk + r] : 0.f;
+    }
+    for (int x = threadIdx.x; x < CD * dv4; x += blockDim.x) {
+        const int i = x / dv4, cc = x - i * dv4;
+        sU[i * sp + cc] = (i < L && cc < dv) ? ut[i * dv + cc] : 0.f;
+    }
     __syncthreads();
-    const int tv = (dv + 3) / 4;
+    const int tv = dv4 / 4;
     // U = Ut - Wt S (each thread updates only the entries it computed)
     for (int t = threadIdx.x; t < (CD / 4) * tv; t += blockDim.x) {
         const int i0 = 4 * (t / tv), c0 = 4 * (t % tv);
         float acc[4][4];
-        tile44(dk, i0, c0, [&](int i, int r) { return sWt[i * skp + r]; },
-               [&](int r, int cc) { return cc < dv ? sS[r * dv + cc] : 0.f; }, acc);
+        tile44v(dk4, [&](int r) { return lds4(sWT + r * tp + i0); }, [&](int r) { return lds4(sS + r * sp + c0); },
+                acc);
 #pragma unroll
         for (int u = 0; u < 4; ++u)
 #pragma unroll
-            for (int v = 0; v < 4; ++v)
-                if (c0 + v < dv) sU[(i0 + u) * svp + c0 + v] -= acc[u][v];
+            for (int v = 0; v < 4; ++v) sU[(i0 + u) * sp + c0 + v] -= acc[u][v];
     }
-    // G[i][l] = eta lam^(i-l) (q'_i . k_l) for l <= i < L
+    // G^T[l][i] = eta lam^(i-l) (q'_i . k_l) for l <= i < L
     for (int t = threadIdx.x; t < (CD / 4) * (CD / 4); t += blockDim.x) {
-        const int i0 = 4 * (t / (CD / 4)), l0 = 4 * (t % (CD / 4));
+        const int l0 = 4 * (t / (CD / 4)), i0 = 4 * (t % (CD / 4));
         float acc[4][4];
-        tile44(dk, i0, l0, [&](int i, int r) { return sQ[i * skp + r]; },
-               [&](int r, int l) { return sK[l * skp + r]; }, acc);
+        tile44v(dk4, [&](int r) { return lds4(sKT + r * tp + l0); }, [&](int r) { return lds4(sQT + r * tp + i0); },
+                acc);
 #pragma unroll
         for (int u = 0; u < 4; ++u)
 #pragma unroll
             for (int v = 0; v < 4; ++v) {
-                const int i = i0 + u, l = l0 + v;
-                sG[i * sgp + l] = (l <= i && i < L) ? eta * pw[i - l] * acc[u][v] : 0.f;
+                const int l = l0 + u, i = i0 + v;
+                sGT[l * tp + i] = (l <= i && i < L) ? eta * pw[i - l] * acc[u][v] : 0.f;
             }
     }
     __syncthreads();
@@ -339,10 +365,8 @@ __global__ void __launch_bounds__(kDThreads) delta_read_kernel(PrefillParams p, 
     for (int t = threadIdx.x; t < (CD / 4) * tv; t += blockDim.x) {
         const int i0 = 4 * (t / tv), c0 = 4 * (t % tv);
         float qs[4][4], gu[4][4];
-        tile44(dk, i0, c0, [&](int i, int r) { return sQ[i * skp + r]; },
-               [&](int r, int cc) { return cc < dv ? sS[r * dv + cc] : 0.f; }, qs);
-        tile44(CD, i0, c0, [&](int i, int l) { return sG[i * sgp + l]; },
-               [&](int l, int cc) { return cc < dv ? sU[l * svp + cc] : 0.f; }, gu);
+        tile44v(dk4, [&](int r) { return lds4(sQT + r * tp + i0); }, [&](int r) { return lds4(sS + r * sp + c0); }, qs);
+        tile44v(L, [&](int l) { return lds4(sGT + l * tp + i0); }, [&](int l) { return lds4(sU + l * sp + c0); }, gu);
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
             const int i = i0 + u;
@@ -351,7 +375,7 @@ __global__ void __launch_bounds__(kDThreads) delta_read_kernel(PrefillParams p, 
             float m[4];
 #pragma unroll
             for (int v = 0; v < 4; ++v) m[v] = fmaf(pw[i + 1], qs[u][v], gu[u][v]);
-            if ((dv & 3) == 0) {  // four columns at once (c0 + 3 < dv)
+            if ((dv & 3) == 0) {  // four columns at once
                 if (add_y) {
                     Tin *y = reinterpret_cast<Tin *>(p.y) + row * dv + c0;
                     float f[4];
@@ -403,7 +427,7 @@ cudaError_t launch_delta_t(const PrefillParams &p, bool add_y, cudaStream_t s) {
     const int dk = p.dk, dv = p.dv;
     cudaError_t e;
     if (w.nC > 0) {
-        const size_t sm_prep = (size_t)(CD * (dk + 1) + CD * (dk + dv + 1) + CD * (CD + 1) + CD + 1) * sizeof(float);
+        const size_t sm_prep = (size_t)prep_floats(dk, dv) * sizeof(float);
         e = cudaFuncSetAttribute(delta_prep_kernel<Tin>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_prep);
         if (e != cudaSuccess) return e;
         delta_prep_kernel<Tin><<<dim3((unsigned)w.nC, (unsigned)BH), kDThreads, sm_prep, s>>>(p, w);
@@ -417,8 +441,7 @@ cudaError_t launch_delta_t(const PrefillParams &p, bool add_y, cudaStream_t s) {
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     if (w.nC > 0 && !p.state_only) {
-        const size_t sm_read = (size_t)(dk * dv + CD * (dv + 1) + 3 * CD * (dk + 1) + CD * (CD + 1) + CD + 1) *
-                               sizeof(float);
+        const size_t sm_read = (size_t)read_floats(dk, dv) * sizeof(float);
         e = cudaFuncSetAttribute(delta_read_kernel<Tin>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_read);
         if (e != cudaSuccess) return e;
         float *mrow = reinterpret_cast<float *>(ws + Lo.mrow);
