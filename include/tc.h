@@ -182,9 +182,10 @@ TC_API tc_status tc_prefill_from_state(const tc_prefill_desc *desc, int64_t t0,
  *               only with TC_PREFILL_L1_ONLY.
  *   workspace   tc_prefill_varlen_workspace_size(desc) bytes.
  *
- * Supported: the tensor-core path only (bf16, d_k = d_v = 64, W a multiple
- * of 128, flags 0 or TC_PREFILL_L1_ONLY); other descriptions return
- * TC_ERR_UNSUPPORTED (and (size_t)-1 from the size query).  The offsets are
+ * Supported: the tensor-core paths only (bf16, d_k = d_v in {64, 128}, any
+ * W, flags 0 or TC_PREFILL_L1_ONLY; d = 64 with W a multiple of 128 runs the
+ * fused kernel, the rest the general tensor-core path); other descriptions
+ * return TC_ERR_UNSUPPORTED (and (size_t)-1 from the size query).  The offsets are
  * device data, so the host cannot check them: the kernels do.  A sequence
  * whose offsets are negative, decreasing, past total or longer than desc->T
  * is skipped (its rows of y are not written, its A_final is zero) and the

@@ -56,9 +56,46 @@ struct GenParams {
     const float *A_init;
     const float *lam, *eta, *g;
     int T, Tc, n_halo, W, H, E, nC;  // new rows, combined rows, halo, window, heads, evictions, chunks
+    // variable-length calls: sequence b = packed rows cu[b] .. cu[b+1]-1 of
+    // [total][H][D] q, k, v, y (and m rows); T is then the longest length
+    // and E, nC the largest eviction and chunk counts.  Null: fixed length.
+    const int64_t *cu;
+    int total;
     int *status;
     unsigned long long wait_ns;
 };
+
+// One (sequence, head) row of work: its row origin and length in the tensors
+// (fixed length: rows of [BH][Tc] / [BH][T]; packed: rows of [total][H]).
+struct GSeq {
+    int bh, h, row0, T, Tc, E, nC;
+    bool packed;
+};
+__device__ __forceinline__ GSeq gseq(const GenParams &p, int bh) {
+    GSeq s;
+    s.bh = bh;
+    s.h = bh % p.H;
+    s.packed = p.cu != nullptr;
+    if (!s.packed) {
+        s.row0 = 0;
+        s.T = p.T;
+        s.Tc = p.Tc;
+    } else {
+        const int64_t a = p.cu[bh / p.H], e = p.cu[bh / p.H + 1];
+        const bool ok = a >= 0 && e >= a && e <= p.total && e - a <= p.T;
+        if (!ok && s.h == 0 && threadIdx.x == 0 && blockIdx.x == 0) report(p.status, 5);
+        s.row0 = ok ? (int)a : 0;
+        s.T = s.Tc = ok ? (int)(e - a) : 0;
+    }
+    s.E = s.Tc > p.W ? s.Tc - p.W : 0;
+    s.nC = (s.E + CG - 1) / CG;
+    return s;
+}
+// Element offset of row `row` (of the combined sequence for k and v, else of the
+// new rows) of a [.][D] tensor; rows_fixed is the row count of the fixed layout.
+__device__ __forceinline__ size_t grow(const GSeq &s, int row, int rows_fixed, int H, int D) {
+    return s.packed ? ((size_t)(s.row0 + row) * H + s.h) * D : ((size_t)s.bh * rows_fixed + row) * D;
+}
 
 __device__ __forceinline__ bool gwait(uint64_t *bar, uint32_t parity, volatile int *abort, const GenParams &p) {
     return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort, p.status, p.wait_ns));
@@ -79,12 +116,18 @@ __device__ __forceinline__ void gpowers(float *pw, int n_max, float lam, int x) 
 }
 __device__ __forceinline__ void gbar128() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
-// rows [row, row + rows) of a [.][D] map as NB column blocks of 64
+// rows [row, row + rows) of a [.][D] map as NB column blocks of 64: maps
+// (D, rows, BH) for fixed lengths, (D, H, total) for packed sequences
 template <int NB>
-__device__ __forceinline__ void tma_rows_nb(uint8_t *dst, const CUtensorMap *m, uint64_t *bar, int row, int bh,
-                                            uint32_t blk) {
+__device__ __forceinline__ void tma_rows_nb(uint8_t *dst, const CUtensorMap *m, uint64_t *bar, int row,
+                                            const GSeq &sq, uint32_t blk) {
 #pragma unroll
-    for (int b = 0; b < NB; ++b) tma_load_3d(dst + b * blk, m, bar, 64 * b, row, bh);
+    for (int b = 0; b < NB; ++b) {
+        if (sq.packed)
+            tma_load_3d(dst + b * blk, m, bar, 64 * b, sq.h, sq.row0 + row);
+        else
+            tma_load_3d(dst + b * blk, m, bar, 64 * b, row, sq.bh);
+    }
 }
 
 // ===========================================================================
@@ -123,10 +166,11 @@ __global__ void __launch_bounds__(kGThreads, NB == 1 ? 2 : 1)
     volatile int *abort = reinterpret_cast<volatile int *>(tmem_base + 1);
 
     const int tid = threadIdx.x, warp = tid >> 5;
-    const int bh = blockIdx.y;
+    const GSeq sq = gseq(p, blockIdx.y);
     const int t0 = blockIdx.x * CG;           // first new row
+    if (t0 >= sq.T) return;                   // past this sequence (variable-length calls)
     const int tau0 = p.n_halo + t0;           // its combined position
-    const int lo = max(0, tau0 - p.W + 1), hi = min(p.Tc - 1, tau0 + CG - 1);
+    const int lo = max(0, tau0 - p.W + 1), hi = min(sq.Tc - 1, tau0 + CG - 1);
     const int xs = lo & ~(GX - 1);
     const int N = (hi - xs) / GX + 1;
 
@@ -158,15 +202,15 @@ __global__ void __launch_bounds__(kGThreads, NB == 1 ? 2 : 1)
     if (warp == 0) {
         if (tid == 0) {
             mbar_expect_tx(q_full, C::Q_B);
-            tma_rows_nb<NB>(sm + C::OFF_Q, &tq, q_full, t0, bh, BLK128);
+            tma_rows_nb<NB>(sm + C::OFF_Q, &tq, q_full, t0, sq, BLK128);
             int n = 0;
             for (; n < N; ++n) {
                 const int s = n % NS;
                 if (!mbar_wait(&x_empty[s], ((n / NS) & 1) ^ 1, abort, p.status, p.wait_ns)) break;
                 uint8_t *dst = sm + C::OFF_X + s * 2 * C::X_B;
                 mbar_expect_tx(&x_full[s], 2 * C::X_B);
-                tma_rows_nb<NB>(dst, &tk, &x_full[s], xs + GX * n, bh, BLK64);
-                tma_rows_nb<NB>(dst + C::X_B, &tv, &x_full[s], xs + GX * n, bh, BLK64);
+                tma_rows_nb<NB>(dst, &tk, &x_full[s], xs + GX * n, sq, BLK64);
+                tma_rows_nb<NB>(dst + C::X_B, &tv, &x_full[s], xs + GX * n, sq, BLK64);
             }
             mbar_wait_drain(q_full, 0);
             for (int st = 0; st < NS; ++st) {
@@ -216,7 +260,7 @@ __global__ void __launch_bounds__(kGThreads, NB == 1 ? 2 : 1)
         const int r = 32 * q4 + (tid & 31);
         const uint32_t lanes = tb + ((uint32_t)(32 * q4) << 16);
         const int t = t0 + r, tau = tau0 + r;
-        const uint32_t wlim = t < p.T ? (uint32_t)p.W : 0u;
+        const uint32_t wlim = t < sq.T ? (uint32_t)p.W : 0u;
         const float sl2 = kLog2eG * rsqrtf((float)D);
         float m_run = -INFINITY, l_run = 0.f;
         bool ok = true;
@@ -284,15 +328,15 @@ __global__ void __launch_bounds__(kGThreads, NB == 1 ? 2 : 1)
         if (ok && gwait(o_full, 0, abort, p)) {
             tc_fence_after();
             const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
-            const bool has_m = p.mrow && tau >= p.W && t < p.T;
-            const float sg = has_m ? 1.f / (1.f + expf(-p.g[bh % p.H])) : 0.f;
-            const float *mr = has_m ? p.mrow + ((size_t)bh * p.T + t) * D : nullptr;
+            const bool has_m = p.mrow && tau >= p.W && t < sq.T;
+            const float sg = has_m ? 1.f / (1.f + expf(-p.g[sq.h])) : 0.f;
+            const float *mr = has_m ? p.mrow + grow(sq, t, p.T, p.H, D) : nullptr;
 #pragma unroll
             for (int c0 = 0; c0 < D; c0 += 32) {
                 uint32_t o[32];
                 tmem_ld32(lanes + C::TM_O + c0, o);
                 tmem_wait_ld();
-                if (t < p.T) {
+                if (t < sq.T) {
                     float f[32];
 #pragma unroll
                     for (int c = 0; c < 32; ++c) f[c] = __uint_as_float(o[c]) * inv_l;
@@ -306,7 +350,7 @@ __global__ void __launch_bounds__(kGThreads, NB == 1 ? 2 : 1)
                             f[c + 3] = fmaf(sg, mv.w, f[c + 3]);
                         }
                     }
-                    uint4 *dst = reinterpret_cast<uint4 *>(p.y + ((size_t)bh * p.T + t) * D + c0);
+                    uint4 *dst = reinterpret_cast<uint4 *>(p.y + grow(sq, t, p.T, p.H, D) + c0);
 #pragma unroll
                     for (int u = 0; u < 4; ++u)
                         dst[u] = make_uint4(pack_bf16(f[8 * u], f[8 * u + 1]), pack_bf16(f[8 * u + 2], f[8 * u + 3]),
@@ -346,8 +390,10 @@ __global__ void __launch_bounds__(kGThreads, 2)
     volatile int *abort = reinterpret_cast<volatile int *>(tmem_base + 1);
     float *pw = reinterpret_cast<float *>(sm + SUM_OFF_PW);
     const int tid = threadIdx.x, warp = tid >> 5;
-    const int bh = blockIdx.y, c_first = blockIdx.x * CPB;
-    const int h = bh % p.H;
+    const GSeq sq = gseq(p, blockIdx.y);
+    const int bh = sq.bh, c_first = blockIdx.x * CPB;
+    const int h = sq.h;
+    if (c_first >= sq.nC) return;  // past this sequence's chunks (variable-length calls)
 
     if (tid == 0) {
         mbar_init(in_full, 1);
@@ -369,13 +415,16 @@ __global__ void __launch_bounds__(kGThreads, 2)
     if (warp == 0) {
         if (tid == 0) {
             mbar_expect_tx(in_full, 2 * BLK128);
-            if (NB == 1) {  // K of chunks c_first, c_first + 1 (rows past the combined sequence read zero)
-                tma_load_3d(sm + SUM_OFF_A, &tk, in_full, 0, c_first * CG, bh);
-                tma_load_3d(sm + SUM_OFF_A + BLK128, &tk, in_full, 0, (c_first + 1) * CG, bh);
-            } else {
-                tma_load_3d(sm + SUM_OFF_A, &tk, in_full, 0, c_first * CG, bh);
+            // K of chunks c_first, c_first + 1 (D = 64) or the two column halves of
+            // chunk c_first (D = 128); rows past the data read zero, rows past the
+            // sequence (packed calls) meet zero weights
+            tma_rows_nb<1>(sm + SUM_OFF_A, &tk, in_full, c_first * CG, sq, BLK128);
+            if (NB == 1)
+                tma_rows_nb<1>(sm + SUM_OFF_A + BLK128, &tk, in_full, (c_first + 1) * CG, sq, BLK128);
+            else if (sq.packed)
+                tma_load_3d(sm + SUM_OFF_A + BLK128, &tk, in_full, 64, sq.h, sq.row0 + c_first * CG);
+            else
                 tma_load_3d(sm + SUM_OFF_A + BLK128, &tk, in_full, 64, c_first * CG, bh);
-            }
             mbar_wait_drain(in_full, 0);
         }
     } else if (warp == 1) {
@@ -407,10 +456,10 @@ __global__ void __launch_bounds__(kGThreads, 2)
         for (int b = 0; b < 2; ++b) {
             const int c = NB == 1 ? c_first + b : c_first;
             const int e0 = c * CG;
-            const int L = c < p.nC ? min(CG, p.E - e0) : 0;
+            const int L = c < sq.nC ? min(CG, sq.E - e0) : 0;
             const float w = x < L ? pw[L - 1 - x] : 0.f;
             const int col0 = NB == 1 ? 0 : 64 * b;
-            const uint4 *src = reinterpret_cast<const uint4 *>(p.v + ((size_t)bh * p.Tc + e0 + x) * D + col0);
+            const uint4 *src = reinterpret_cast<const uint4 *>(p.v + grow(sq, x < L ? e0 + x : 0, p.Tc, p.H, D) + col0);
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
                 const uint4 a = w != 0.f ? src[u] : make_uint4(0u, 0u, 0u, 0u);
@@ -435,7 +484,7 @@ __global__ void __launch_bounds__(kGThreads, 2)
             const int c = NB == 1 ? c_first + (x >> 6) : c_first;
             const int r = NB == 1 ? (x & 63) : x;
             const uint32_t col0 = NB == 1 ? (uint32_t)(x & 64) : 0u;
-            if (c < p.nC) {
+            if (c < sq.nC) {
                 float *dst = p.dA + (((size_t)bh * p.nC + c) * D + r) * D;
 #pragma unroll
                 for (int c0 = 0; c0 < (NB == 1 ? 64 : 128); c0 += 32) {
@@ -470,10 +519,11 @@ __global__ void __launch_bounds__(kGThreads, 2)
 // increments) and A_final.
 __global__ void __launch_bounds__(256) gen_scan_kernel(GenParams p, int D) {
     __shared__ float decay[2];
-    const int bh = blockIdx.y;
+    const GSeq sq = gseq(p, blockIdx.y);
+    const int bh = sq.bh, nC = sq.nC;
     if (threadIdx.x < 2) {
-        const double l2l = log2((double)p.lam[bh % p.H]);
-        const int last = p.nC > 0 ? p.E - (p.nC - 1) * CG : 0;
+        const double l2l = log2((double)p.lam[sq.h]);
+        const int last = nC > 0 ? sq.E - (nC - 1) * CG : 0;
         const int n = threadIdx.x == 0 ? CG : last;
         decay[threadIdx.x] = (float)exp2((double)n * l2l);
     }
@@ -482,18 +532,18 @@ __global__ void __launch_bounds__(256) gen_scan_kernel(GenParams p, int D) {
     const int nel = D * D;
     if (x >= nel) return;
     float A = p.A_init ? p.A_init[(size_t)bh * nel + x] : 0.f;
-    float *dA = p.dA + (size_t)bh * p.nC * nel + x;
+    float *dA = p.dA + (size_t)bh * p.nC * nel + x;  // p.nC: chunk slots per row
     constexpr int kB = 8;
-    for (int c0 = 0; c0 < p.nC; c0 += kB) {
+    for (int c0 = 0; c0 < nC; c0 += kB) {
         float d[kB];
 #pragma unroll
-        for (int u = 0; u < kB; ++u) d[u] = c0 + u < p.nC ? dA[(size_t)(c0 + u) * nel] : 0.f;
+        for (int u = 0; u < kB; ++u) d[u] = c0 + u < nC ? dA[(size_t)(c0 + u) * nel] : 0.f;
 #pragma unroll
         for (int u = 0; u < kB; ++u) {
             const int c = c0 + u;
-            if (c < p.nC) {
+            if (c < nC) {
                 dA[(size_t)c * nel] = A;
-                A = fmaf(c == p.nC - 1 ? decay[1] : decay[0], A, d[u]);
+                A = fmaf(c == nC - 1 ? decay[1] : decay[0], A, d[u]);
             }
         }
     }
@@ -532,8 +582,10 @@ __global__ void __launch_bounds__(kGThreads, 1)
     volatile int *abort = reinterpret_cast<volatile int *>(tmem_base + 1);
     float *pw = reinterpret_cast<float *>(sm + C::OFF_PW);
     const int tid = threadIdx.x, warp = tid >> 5;
-    const int c = blockIdx.x, bh = blockIdx.y, h = bh % p.H;
-    const int e0 = c * CG, L = min(CG, p.E - e0);
+    const GSeq sq = gseq(p, blockIdx.y);
+    const int c = blockIdx.x, bh = sq.bh, h = sq.h;
+    if (c >= sq.nC) return;  // past this sequence's chunks (variable-length calls)
+    const int e0 = c * CG, L = min(CG, sq.E - e0);
     const int qrow0 = e0 + p.W - p.n_halo;  // new row of eviction e0's read
 
     if (tid == 0) {
@@ -557,9 +609,9 @@ __global__ void __launch_bounds__(kGThreads, 1)
     if (warp == 0) {
         if (tid == 0) {
             mbar_expect_tx(in_full, 3 * C::IN_B);
-            tma_rows_nb<NB>(sm + C::OFF_Q, &tq, in_full, qrow0, bh, BLK128);
-            tma_rows_nb<NB>(sm + C::OFF_K, &tk, in_full, e0, bh, BLK128);
-            tma_rows_nb<NB>(sm + C::OFF_V, &tv, in_full, e0, bh, BLK128);
+            tma_rows_nb<NB>(sm + C::OFF_Q, &tq, in_full, qrow0, sq, BLK128);
+            tma_rows_nb<NB>(sm + C::OFF_K, &tk, in_full, e0, sq, BLK128);
+            tma_rows_nb<NB>(sm + C::OFF_V, &tv, in_full, e0, sq, BLK128);
             mbar_wait_drain(in_full, 0);
         }
     } else if (warp == 1) {
@@ -655,7 +707,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
         if (ok && gwait(acc_full, 0, abort, p)) {
             tc_fence_after();
             const float dec = pw[min(x + 1, CG + 1)];
-            float *dst = p.mrow + ((size_t)bh * p.T + qrow0 + x) * D;
+            float *dst = p.mrow + grow(sq, x < L ? qrow0 + x : 0, p.T, p.H, D);
 #pragma unroll
             for (int c0 = 0; c0 < D; c0 += 32) {
                 uint32_t a[32], b[32];
@@ -706,6 +758,20 @@ bool gen_map(CUtensorMap *m, const void *base, int rows, int BH, int D, int box_
     cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)rows, (cuuint64_t)BH};
     cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)rows * D * 2};
     cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 1};
+    cuuint32_t es[3] = {1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, es,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Packed [total][H][D] bf16 -> 3D map (D, H, total), boxes of 64 columns x 1 x box_rows:
+// the same shared-memory tile as gen_map's, box_rows token rows of one head
+bool gen_map_packed(CUtensorMap *m, const void *base, int total, int H, int D, int box_rows) {
+    EncodeFn fn = reinterpret_cast<EncodeFn>(tensor_map_encoder());
+    if (!fn || total < 1) return false;
+    cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)total};
+    cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)H * D * 2};
+    cuuint32_t box[3] = {64, 1, (cuuint32_t)box_rows};
     cuuint32_t es[3] = {1, 1, 1};
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, es,
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -770,6 +836,9 @@ cudaError_t launch_general_t(const PrefillParams &pp, const float *mrow_in, cuda
     p.A_final = pp.A_final;
     p.status = pp.status;
     p.wait_ns = pp.wait_ns;
+    p.cu = pp.cu_seqlens;  // variable-length: T is the longest length, no halo
+    p.total = (int)pp.total;
+    const bool packed = p.cu != nullptr;
     cudaError_t e;
     if (p.n_halo > 0) {  // one sequence of keys and values, halo first
         __nv_bfloat16 *kc = reinterpret_cast<__nv_bfloat16 *>(ws + Lo.kc);
@@ -788,11 +857,14 @@ cudaError_t launch_general_t(const PrefillParams &pp, const float *mrow_in, cuda
                            : (l2 && !pp.state_only && p.nC > 0 ? reinterpret_cast<float *>(ws + Lo.mrow) : nullptr);
     const bool queries = !pp.state_only && p.T > 0;
     CUtensorMap mk128, mv128, mq128, mk64, mv64;
+    auto map = [&](CUtensorMap *m, const void *base, int rows, int box) {
+        return packed ? gen_map_packed(m, base, p.total, p.H, D, box) : gen_map(m, base, rows, BH, D, box);
+    };
     if ((queries || (l2 && p.nC > 0)) &&
-        (!gen_map(&mk128, p.k, p.Tc, BH, D, 128) || !gen_map(&mv128, p.v, p.Tc, BH, D, 128) ||
-         !gen_map(&mk64, p.k, p.Tc, BH, D, 64) || !gen_map(&mv64, p.v, p.Tc, BH, D, 64)))
+        (!map(&mk128, p.k, p.Tc, 128) || !map(&mv128, p.v, p.Tc, 128) || !map(&mk64, p.k, p.Tc, 64) ||
+         !map(&mv64, p.v, p.Tc, 64)))
         return cudaErrorInvalidValue;
-    if (queries && !gen_map(&mq128, p.q, p.T, BH, D, 128)) return cudaErrorInvalidValue;
+    if (queries && !map(&mq128, p.q, p.T, 128)) return cudaErrorInvalidValue;
     if (l2) {
         if (p.nC > 0) {
             e = cudaFuncSetAttribute(gen_sums_kernel<NB>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SUM_SMEM);
@@ -825,13 +897,19 @@ cudaError_t launch_general_t(const PrefillParams &pp, const float *mrow_in, cuda
 
 }  // namespace
 
+bool general_varlen_supported(const tc_prefill_desc &d) {
+    tc_prefill_desc c = d;
+    if (c.T < 1) c.T = 1;
+    return !(d.flags & ~TC_PREFILL_L1_ONLY) && general_supported(c, 0);
+}
+
 bool general_supported(const tc_prefill_desc &d, int64_t n_halo) {
     if (d.dtype != TC_BF16 || d.dk != d.dv || (d.dk != 64 && d.dk != 128)) return false;
     if (d.flags & TC_PREFILL_CHUNK_MEAN) return false;
     if ((d.flags & TC_PREFILL_DELTA_RULE) && (n_halo != 0 || (d.flags & (TC_PREFILL_STATE_ONLY | TC_PREFILL_L1_ONLY))))
         return false;
-    if (d.T + n_halo >= (int64_t(1) << 30) || d.B * d.H > 65535) return false;
-    return tensor_map_encoder() != nullptr;
+    // shapes only: a call without a device gets TC_ERR_NO_DEVICE, not UNSUPPORTED
+    return d.T + n_halo < (int64_t(1) << 30) && d.B * d.H <= 65535;
 }
 
 size_t general_workspace_bytes(const tc_prefill_desc &d, int64_t n_halo) { return gen_layout(d, n_halo).total; }

@@ -135,6 +135,15 @@ bool varlen_supported(const tc_prefill_desc &d) {
     return use_sm100(c, 0) && !(d.flags & ~TC_PREFILL_L1_ONLY);
 }
 
+// Workspace of a variable-length call on the general path (at least 256
+// bytes, so that the call always has a device workspace to check).
+size_t varlen_general_ws(const tc_prefill_desc &d) {
+    tc_prefill_desc c = d;
+    if (c.T < 1) c.T = 1;
+    const size_t n = tc::general_workspace_bytes(c, 0);
+    return n < 256 ? 256 : n;
+}
+
 int sm_count_or_default() {
     int dev = 0, sms = 0;
     if (current_device(&dev, &sms) != TC_OK) return 148;
@@ -308,8 +317,10 @@ tc_status tc_prefill_from_state(const tc_prefill_desc *d, int64_t t0, const void
 }
 
 size_t tc_prefill_varlen_workspace_size(const tc_prefill_desc *d) {
-    if (check_desc(d) != TC_OK || !varlen_supported(*d)) return (size_t)-1;
-    return tc::sm100_workspace_bytes(*d, sm_count_or_default(), true);
+    if (check_desc(d) != TC_OK) return (size_t)-1;
+    if (varlen_supported(*d)) return tc::sm100_workspace_bytes(*d, sm_count_or_default(), true);
+    if (tc::general_varlen_supported(*d)) return varlen_general_ws(*d);
+    return (size_t)-1;
 }
 
 tc_status tc_prefill_varlen(const tc_prefill_desc *d, const int64_t *cu_seqlens, int64_t total,
@@ -327,14 +338,16 @@ tc_status tc_prefill_varlen(const tc_prefill_desc *d, const int64_t *cu_seqlens,
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(y) ||
         (A_final && !aligned16(A_final)) || (workspace && !aligned16(workspace)))
         return TC_ERR_INVALID_ARG;
-    // the tensor-core path only: bf16, d = 64, W a multiple of 128, no state-only,
-    // delta-rule or chunk-mean variants
-    if (!varlen_supported(*d)) return TC_ERR_UNSUPPORTED;
+    // tensor-core paths only (the fused kernel, else the general path: bf16,
+    // d_k = d_v in {64, 128}), without the state-only, delta-rule or chunk-mean
+    // variants
+    const bool fused = varlen_supported(*d);
+    if (!fused && !tc::general_varlen_supported(*d)) return TC_ERR_UNSUPPORTED;
     if (d->H * total > (int64_t(1) << 31)) return TC_ERR_UNSUPPORTED;
     int dev = 0, sms = 0;
     st = current_device(&dev, &sms);
     if (st != TC_OK) return st;
-    const size_t need = tc::sm100_workspace_bytes(*d, sms, true);
+    const size_t need = fused ? tc::sm100_workspace_bytes(*d, sms, true) : varlen_general_ws(*d);
     if (!workspace || workspace_bytes < need) return TC_ERR_WORKSPACE;
     const void *ptrs[] = {q, k, v, y};
     for (const void *x : ptrs)
@@ -374,7 +387,8 @@ tc_status tc_prefill_varlen(const tc_prefill_desc *d, const int64_t *cu_seqlens,
     p.wait_ns = wait_limit_ns();
     p.cu_seqlens = cu_seqlens;
     p.total = total;
-    return tc::launch_prefill_sm100(p, sms, s) == cudaSuccess ? TC_OK : TC_ERR_CUDA;
+    const cudaError_t e = fused ? tc::launch_prefill_sm100(p, sms, s) : tc::launch_prefill_general(p, nullptr, s);
+    return e == cudaSuccess ? TC_OK : TC_ERR_CUDA;
 }
 
 size_t tc_backward_workspace_size(const tc_prefill_desc *d) {

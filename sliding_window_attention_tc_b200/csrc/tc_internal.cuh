@@ -196,6 +196,10 @@ cudaError_t launch_backward_chunks_tc(const tc_prefill_desc &d, const void *q, c
 // delta rule (no halo) the memory's reads come from mrow ([BH][T][d] float32,
 // written by launch_delta_chunked); otherwise mrow is null.
 bool general_supported(const tc_prefill_desc &d, int64_t n_halo);
+// Variable-length calls (PrefillParams::cu_seqlens set) on the general path:
+// bf16, d_k = d_v in {64, 128}, any W, flags 0 or L1-only.  Workspace as
+// general_workspace_bytes(d, 0) with d.T the longest length.
+bool general_varlen_supported(const tc_prefill_desc &d);
 size_t general_workspace_bytes(const tc_prefill_desc &d, int64_t n_halo);
 int general_launch_count(const tc_prefill_desc &d, int64_t n_halo);
 cudaError_t launch_prefill_general(const PrefillParams &p, const float *mrow, cudaStream_t s);

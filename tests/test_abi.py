@@ -166,9 +166,10 @@ def test_varlen_rejects_invalid_arguments():
     assert lib.tc_prefill_varlen_workspace_size(None) == tc.SIZE_ERROR
 
 
-@pytest.mark.parametrize("kw", [dict(dtype=tc.TC_F32), dict(dk=32, dv=32), dict(W=100),
-                                dict(W=64), dict(flags=tc.TC_PREFILL_STATE_ONLY)])
-def test_varlen_outside_the_tensor_core_path_is_unsupported(kw):
+@pytest.mark.parametrize("kw", [dict(dtype=tc.TC_F32), dict(dk=32, dv=32), dict(dk=64, dv=128),
+                                dict(flags=tc.TC_PREFILL_STATE_ONLY),
+                                dict(flags=tc.TC_PREFILL_DELTA_RULE)])
+def test_varlen_outside_the_tensor_core_paths_is_unsupported(kw):
     flags = kw.pop("flags", 0)
     d = _varlen_desc(**kw)
     d.flags = flags
@@ -179,6 +180,11 @@ def test_varlen_outside_the_tensor_core_path_is_unsupported(kw):
 @pytest.mark.skipif(HAS_GPU, reason="checks the no-device answer")
 def test_valid_varlen_without_device_reports_no_device():
     assert _call_varlen(_varlen_desc()) == 3
+    # the general tensor-core path: W not a multiple of 128, d = 128
+    for kw in (dict(W=100), dict(W=64), dict(dk=128, dv=128, W=300)):
+        d = _varlen_desc(**kw)
+        assert _call_varlen(d) == 3
+        assert tc.lib_handle().tc_prefill_varlen_workspace_size(ctypes.byref(d)) > 0
     d = _varlen_desc(l1_only=True)
     assert _call_varlen(d, A=None) == 3
     assert tc.lib_handle().tc_prefill_varlen_workspace_size(ctypes.byref(_varlen_desc())) >= 0

@@ -120,3 +120,35 @@ def test_general_decode_shaped_prefill(cuda_device):
     assert tc.prefill_launch_count(desc) == general_launches(T, W)
     y, A = run_prefill(x, cuda_device)
     check_prefill(x, y, A)
+
+
+def test_general_full_size_bench_workloads(cuda_device):
+    """The two general-path workloads bench.py times, at full size, in the
+    launch configuration it uses: the LM workload at W = 500, and d = 128,
+    W = 2048 over 8 x 32 heads of 4096 tokens (inputs seeded as in bench.py).
+    Sampled heads against the oracle run on each sampled head alone."""
+    import math
+    tc = _tc()
+    dev = cuda_device
+    x = wl.prefill_config("lm_prefill_bf16")
+    y, A = tc.prefill(*(t.to(dev).contiguous() for t in (x.q, x.k, x.v, x.lam, x.eta, x.g)), 500, x.C)
+    torch.cuda.synchronize()
+    assert tc.device_status() == 0
+    x500 = wl.PrefillInputs(x.q, x.k, x.v, x.lam, x.eta, x.g, 500, x.C)
+    check_prefill(x500, y.float().cpu().numpy(), A.cpu().numpy(), heads=[(0, 0), (3, 7), (7, 11)])
+    del y, A
+    B, H, T, d, W = 8, 32, 4096, 128, 2048
+    gen = torch.Generator(device=dev).manual_seed(1005)
+    q, k, v = ((torch.randn(B, H, T, d, generator=gen, device=dev) / math.sqrt(d)).to(torch.bfloat16)
+               for _ in range(3))
+    lam = 0.99 + 0.0099 * torch.rand(H, generator=gen, device=dev)
+    eta = 0.1 + 0.9 * torch.rand(H, generator=gen, device=dev)
+    g = torch.randn(H, generator=gen, device=dev)
+    y, A = tc.prefill(q, k, v, lam, eta, g, W, 128)
+    torch.cuda.synchronize()
+    assert tc.device_status() == 0
+    for b, h in [(0, 0), (5, 31)]:
+        sl = lambda t: t[b:b + 1, h:h + 1].cpu()
+        yo, Ao = oracle.prefill(sl(q), sl(k), sl(v), lam[h:h + 1].cpu(), eta[h:h + 1].cpu(), g[h:h + 1].cpu(), W)
+        assert rel_l2(y[b, h].float().cpu().numpy(), yo[0, 0]) <= BF16_Y_TOL
+        assert rel_l2(A[b, h].cpu().numpy(), Ao[0, 0]) <= BF16_A_TOL

@@ -154,3 +154,38 @@ def test_varlen_with_no_tokens_zeroes_the_states(cuda_device):
     assert y.numel() == 0
     assert torch.all(A == 0)
     assert tc.device_status() == 0
+
+
+# general tensor-core path: W not a multiple of 128, d = 128, W = 1
+GENERAL = [
+    ([300, 0, 1000, 77, 2100], 3, 64, 200, 64),
+    ([500, 1, 1300, 129], 2, 128, 256, 64),
+    ([900, 64, 128, 5, 0], 2, 64, 1, 16),
+]
+
+
+@pytest.mark.parametrize("case", GENERAL, ids=[f"d{c[2]}_W{c[3]}" for c in GENERAL])
+def test_varlen_general_path_matches_the_oracle(cuda_device, case):
+    import sliding_window_attention_tc_b200 as tc
+    lengths, H, d, W, C = case
+    x = wl.random_varlen(lengths, H, d, d, W, C, dtype="bf16", seed=W + d)
+    y, A = _run(tc, x, cuda_device)
+    yl1, _ = _run(tc, x, cuda_device, l1_only=True)
+    assert tc.device_status() == 0
+    y, yl1, A = y.float().cpu().numpy(), yl1.float().cpu().numpy(), A.cpu().numpy()
+    assert np.isfinite(y).all() and np.isfinite(A).all()
+    for b in range(len(lengths)):
+        print(b, _check_sequence(x, b, y, A, yl1))
+
+
+def test_varlen_general_path_reports_inconsistent_offsets(cuda_device):
+    import sliding_window_attention_tc_b200 as tc
+    x = wl.random_varlen([300, 200, 300], 2, 64, 64, 200, 64, dtype="bf16", seed=9)
+    bad = torch.tensor([200, 500, 100, 150], dtype=torch.int64)
+    y, A = _run(tc, x, cuda_device, cu=bad, max_seqlen=300)
+    assert tc.device_status() == TC_ERR_DEVICE_BOUNDS
+    y, A = y.float().cpu().numpy(), A.cpu().numpy()
+    assert np.all(A[1] == 0.0)
+    good = wl.VarlenInputs(x.q, x.k, x.v, bad, x.lam, x.eta, x.g, x.W, x.C)
+    _check_sequence(good, 0, y, A)
+    _check_sequence(good, 2, y, A)
