@@ -223,12 +223,13 @@ TC_API tc_status tc_state_fold(int64_t B, int64_t H, int64_t dk, int64_t dv, int
  * The pages train lambda, eta and g end to end (§2 training
  * considerations); the formulas are reverse mode through the token loop of
  * Fig. 2.  The window part is the usual softmax backward over the W keys:
- * for bf16 with d_k = d_v = 64 two tcgen05 kernels (scores and their
+ * for bf16 with d_k = d_v in {64, 128} two tcgen05 kernels (scores and their
  * gradients in TMEM, P and dS fed back to the tensor cores as bf16 hi + lo
  * pairs, float32 accumulation), otherwise two float32 SIMT kernels.  The
- * memory part is the reverse scan of dL/dA_t taken in chunks of 32
- * evictions (per-chunk sums, a scan over the chunks, per-chunk gradients),
- * float32.  Every sum has a fixed order: two calls give the same bits.
+ * memory part is the reverse scan of dL/dA_t taken in chunks (per-chunk
+ * sums, a scan over the chunks, per-chunk gradients): tcgen05 kernels with
+ * chunks of 128 for bf16 with d = 64, float32 SIMT with chunks of 32
+ * otherwise.  Every sum has a fixed order: two calls give the same bits.
  * q, k, v, dy: device, dtype of desc (dy has y's layout); desc->flags must
  * be 0 (C is not used).  Up to six launches.  Workspace:
  * tc_backward_workspace_size(desc) bytes (about

@@ -55,19 +55,27 @@ constexpr int NSX = 4;               // other-side tile stages
 constexpr int kBwdTcThreads = 192;
 constexpr float kLog2eF = 1.4426950408889634f;
 
-constexpr uint32_t OWN_TILE = BO * HDB * 2;  // 16 KB
-constexpr uint32_t X_TILE = BX * HDB * 2;    // 8 KB
-constexpr uint32_t OFF_OWN = 0;                           // own_a, own_b
-constexpr uint32_t OFF_XS = 2 * OWN_TILE;                 // NSX x (x_a, x_b)
-constexpr uint32_t OFF_ST = OFF_XS + NSX * 2 * X_TILE;    // NSX x (lse[64], D[64]) (keys kernel)
-constexpr uint32_t OFF_BARS = OFF_ST + NSX * 2 * BX * 4;
-constexpr uint32_t SMEM_BWD_TC = OFF_BARS + 128 + 1024;   // + slack for the 1024-byte alignment
+constexpr uint32_t BLK_O = BO * 128;  // 16 KB: 128 rows x 64 bf16 columns
+constexpr uint32_t BLK_X = BX * 128;  // 8 KB: 64 rows x 64 bf16 columns
 
-// TMEM columns: S (then P hi/lo), dP (then dS hi/lo), two accumulators.
-constexpr uint32_t TMC_S = 0, TMC_DP = 64, TMC_ACC0 = 128, TMC_ACC1 = 192, TMC_COLS = 256;
+// Layout of the window kernels for head size D = 64 NB: tiles are NB blocks
+// of 64 columns.  TMEM: S (then P hi/lo), dP (then dS hi/lo), two D-column
+// accumulators.
+template <int NB>
+struct BwdCfg {
+    static constexpr int D = 64 * NB;
+    static constexpr uint32_t OWN = NB * BLK_O, XT = NB * BLK_X;
+    static constexpr uint32_t OFF_OWN = 0;                         // own_a, own_b
+    static constexpr uint32_t OFF_XS = 2 * OWN;                    // NSX x (x_a, x_b)
+    static constexpr uint32_t OFF_ST = OFF_XS + NSX * 2 * XT;      // NSX x (lse[64], D[64]) (keys kernel)
+    static constexpr uint32_t OFF_BARS = OFF_ST + NSX * 2 * BX * 4;
+    static constexpr uint32_t SMEM = OFF_BARS + 128 + 1024;        // + slack for the 1024-byte alignment
+    static constexpr uint32_t TMC_S = 0, TMC_DP = 64, TMC_ACC0 = 128, TMC_ACC1 = 128 + D;
+    static constexpr uint32_t COLS = NB == 1 ? 256 : 512;
+};
 
 struct BwdTcParams {
-    float *out0, *out1;  // rows kernel: dq; keys kernel: dk, dv  ([BH][T][64] float32)
+    float *out0, *out1;  // rows kernel: dq; keys kernel: dk, dv  ([BH][T][D] float32)
     float *lse, *Dt;     // [BH][Tp] per query row: log-sum-exp (log2), D_t
     int T, Tp, W;        // W clamped to T
     int *status;
@@ -92,17 +100,22 @@ __device__ __forceinline__ void split_pair(float x0, float x1, uint32_t &hi, uin
     lo = pack_bf16(x0 - h0, x1 - h1);
 }
 
-template <bool KEYS>
-__global__ void __launch_bounds__(kBwdTcThreads, 2)
+template <bool KEYS, int NB>
+__global__ void __launch_bounds__(kBwdTcThreads, NB == 1 ? 2 : 1)
     bwd_window_tc_kernel(const __grid_constant__ CUtensorMap t_own_a,
                          const __grid_constant__ CUtensorMap t_own_b,
                          const __grid_constant__ CUtensorMap t_x_a,
                          const __grid_constant__ CUtensorMap t_x_b,
                          const __grid_constant__ CUtensorMap t_lse,
                          const __grid_constant__ CUtensorMap t_D, BwdTcParams p) {
+    using Cf = BwdCfg<NB>;
+    constexpr int D = Cf::D;
+    constexpr uint32_t OWN_TILE = Cf::OWN, X_TILE = Cf::XT, OFF_OWN = Cf::OFF_OWN, OFF_XS = Cf::OFF_XS;
+    constexpr uint32_t OFF_ST = Cf::OFF_ST, TMC_S = Cf::TMC_S, TMC_DP = Cf::TMC_DP;
+    constexpr uint32_t TMC_ACC0 = Cf::TMC_ACC0, TMC_ACC1 = Cf::TMC_ACC1, TMC_COLS = Cf::COLS;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + OFF_BARS);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + Cf::OFF_BARS);
     uint64_t *own_full = bars, *x_full = bars + 1, *x_empty = x_full + NSX;
     uint64_t *s_full = x_empty + NSX, *ops_ready = s_full + 1, *acc_full = ops_ready + 1;
     uint64_t *mma_done = acc_full + 1;
@@ -157,8 +170,11 @@ __global__ void __launch_bounds__(kBwdTcThreads, 2)
             tma_prefetch_desc(&t_x_a);
             tma_prefetch_desc(&t_x_b);
             mbar_expect_tx(own_full, 2 * OWN_TILE);
-            tma_load_3d(sm + OFF_OWN, &t_own_a, own_full, 0, o0, bh);
-            tma_load_3d(sm + OFF_OWN + OWN_TILE, &t_own_b, own_full, 0, o0, bh);
+#pragma unroll
+            for (int b = 0; b < NB; ++b) {
+                tma_load_3d(sm + OFF_OWN + b * BLK_O, &t_own_a, own_full, 64 * b, o0, bh);
+                tma_load_3d(sm + OFF_OWN + OWN_TILE + b * BLK_O, &t_own_b, own_full, 64 * b, o0, bh);
+            }
             int n = 0;
             for (; n < N; ++n) {
                 const int s = n % NSX;
@@ -166,8 +182,11 @@ __global__ void __launch_bounds__(kBwdTcThreads, 2)
                 const int x0 = xs + BX * (n % nX);
                 uint8_t *dst = sm + OFF_XS + s * 2 * X_TILE;
                 mbar_expect_tx(&x_full[s], 2 * X_TILE + (KEYS ? 2 * BX * 4 : 0));
-                tma_load_3d(dst, &t_x_a, &x_full[s], 0, x0, bh);
-                tma_load_3d(dst + X_TILE, &t_x_b, &x_full[s], 0, x0, bh);
+#pragma unroll
+                for (int b = 0; b < NB; ++b) {
+                    tma_load_3d(dst + b * BLK_X, &t_x_a, &x_full[s], 64 * b, x0, bh);
+                    tma_load_3d(dst + X_TILE + b * BLK_X, &t_x_b, &x_full[s], 64 * b, x0, bh);
+                }
                 if (KEYS) {
                     float *st = reinterpret_cast<float *>(sm + OFF_ST) + s * 2 * BX;
                     tma_load_2d(st, &t_lse, &x_full[s], x0, bh);
@@ -188,7 +207,7 @@ __global__ void __launch_bounds__(kBwdTcThreads, 2)
         // (issued before S of tile n+1, which overwrites their operands: the
         // tensor core runs one thread's MMAs in issue order).
         const uint32_t id_s = idesc_bf16(128, 64, false, false);
-        const uint32_t id_g = idesc_bf16(128, 64, false, true);
+        const uint32_t id_g = idesc_bf16(128, D, false, true);  // N = D over NB column blocks
         const uint32_t own_a = smem_u32(sm + OFF_OWN), own_b = own_a + OWN_TILE;
         const uint32_t xbase = smem_u32(sm + OFF_XS);
         bool ok = warp_wait_b(own_full, 0, abort, p.status, p.wait_ns);
@@ -200,7 +219,7 @@ __global__ void __launch_bounds__(kBwdTcThreads, 2)
                 tc_fence_after();
                 if (KEYS || m >= nX) {
                     const uint32_t xa = xbase + sp * 2 * X_TILE, xb = xa + X_TILE;
-                    const uint64_t da = sdesc_sw128(xa, X_TILE, 1024);
+                    const uint64_t da = sdesc_sw128(xa, BLK_X, 1024);
                     // acc0 += dS x_a: K step k reads dS columns 16k..16k+15,
                     // hi at 32 (k/2) + 8 (k%2), lo 16 columns further
 #pragma unroll
@@ -210,7 +229,7 @@ __global__ void __launch_bounds__(kBwdTcThreads, 2)
                         mma_ts_w(tb + TMC_ACC0, tb + col + 16, da + 128 * k, id_g, 1u);
                     }
                     if (KEYS) {
-                        const uint64_t db = sdesc_sw128(xb, X_TILE, 1024);
+                        const uint64_t db = sdesc_sw128(xb, BLK_X, 1024);
 #pragma unroll
                         for (int k = 0; k < 4; ++k) {
                             const uint32_t col = TMC_S + 32 * (k >> 1) + 8 * (k & 1);
@@ -228,12 +247,18 @@ __global__ void __launch_bounds__(kBwdTcThreads, 2)
             if (!(ok = warp_wait_b(&x_full[s], (n / NSX) & 1, abort, p.status, p.wait_ns))) break;
             tc_fence_after();
             const uint32_t xa = xbase + s * 2 * X_TILE, xb = xa + X_TILE;
-            const uint64_t oa = sdesc_sw128(own_a, 16, 1024), ob = sdesc_sw128(own_b, 16, 1024);
-            const uint64_t ka = sdesc_sw128(xa, 16, 1024), kb = sdesc_sw128(xb, 16, 1024);
 #pragma unroll
-            for (int k = 0; k < 4; ++k) mma_ss_w(tb + TMC_S, oa + 2 * k, ka + 2 * k, id_s, k > 0);
+            for (int b = 0; b < NB; ++b) {
+                const uint64_t oa = sdesc_sw128(own_a + b * BLK_O, 16, 1024), ka = sdesc_sw128(xa + b * BLK_X, 16, 1024);
 #pragma unroll
-            for (int k = 0; k < 4; ++k) mma_ss_w(tb + TMC_DP, ob + 2 * k, kb + 2 * k, id_s, k > 0);
+                for (int k = 0; k < 4; ++k) mma_ss_w(tb + TMC_S, oa + 2 * k, ka + 2 * k, id_s, (b > 0 || k > 0) ? 1u : 0u);
+            }
+#pragma unroll
+            for (int b = 0; b < NB; ++b) {
+                const uint64_t ob = sdesc_sw128(own_b + b * BLK_O, 16, 1024), kb = sdesc_sw128(xb + b * BLK_X, 16, 1024);
+#pragma unroll
+                for (int k = 0; k < 4; ++k) mma_ss_w(tb + TMC_DP, ob + 2 * k, kb + 2 * k, id_s, (b > 0 || k > 0) ? 1u : 0u);
+            }
             mma_commit_w(s_full);
         }
         if (ok) mma_commit_w(acc_full);
@@ -245,7 +270,7 @@ __global__ void __launch_bounds__(kBwdTcThreads, 2)
         const int q4 = warp & 3;
         const int r = 32 * q4 + (tid & 31);
         const uint32_t lanes = tb + ((uint32_t)(32 * q4) << 16);
-        const float sl2 = kLog2eF * 0.125f;  // log2(e) / sqrt(64)
+        const float sl2 = kLog2eF * rsqrtf((float)D);  // log2(e) / sqrt(D)
         const int orow = o0 + r;
         const float *stat = reinterpret_cast<const float *>(sm + OFF_ST);
         // rows kernel: online statistics of query row orow
@@ -347,15 +372,15 @@ __global__ void __launch_bounds__(kBwdTcThreads, 2)
             const size_t row = (size_t)bh * T + orow;
 #pragma unroll
             for (int a = 0; a < (KEYS ? 2 : 1); ++a) {
-                const float scale = a == 0 ? 0.125f : 1.f;  // 1/sqrt(64) on dq, dk
+                const float scale = a == 0 ? rsqrtf((float)D) : 1.f;  // 1/sqrt(D) on dq, dk
                 float *out = a == 0 ? p.out0 : p.out1;
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {
+                for (int h = 0; h < D / 32; ++h) {
                     uint32_t v[32];
                     tmem_ld32(lanes + (a == 0 ? TMC_ACC0 : TMC_ACC1) + 32 * h, v);
                     tmem_wait_ld();
                     if (orow < T) {
-                        float4 *dst = reinterpret_cast<float4 *>(out + row * HDB + 32 * h);
+                        float4 *dst = reinterpret_cast<float4 *>(out + row * D + 32 * h);
 #pragma unroll
                         for (int c = 0; c < 8; ++c)
                             dst[c] = make_float4(__uint_as_float(v[4 * c]) * scale,
@@ -892,12 +917,12 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t
 
 // [BH][T][64] bf16 -> 3D map, boxes of 64 x rows x 1 with the 128-byte swizzle;
 // rows past T read as zero.
-bool rows_map(CUtensorMap *m, const void *base, int T, int BH, int rows) {
+bool rows_map(CUtensorMap *m, const void *base, int T, int BH, int rows, int D = HDB) {
     EncodeTiledFn fn = reinterpret_cast<EncodeTiledFn>(tensor_map_encoder());
     if (!fn) return false;
-    cuuint64_t dims[3] = {(cuuint64_t)HDB, (cuuint64_t)T, (cuuint64_t)BH};
-    cuuint64_t strides[2] = {(cuuint64_t)HDB * 2, (cuuint64_t)T * HDB * 2};
-    cuuint32_t box[3] = {HDB, (cuuint32_t)rows, 1};
+    cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)T, (cuuint64_t)BH};
+    cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)T * D * 2};
+    cuuint32_t box[3] = {64, (cuuint32_t)rows, 1};
     cuuint32_t es[3] = {1, 1, 1};
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box,
               es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -920,23 +945,29 @@ bool stat_map(CUtensorMap *m, const float *base, int Tp, int BH) {
 }  // namespace
 
 bool backward_window_tc_supported(const tc_prefill_desc &d) {
-    return d.dtype == TC_BF16 && d.dk == HDB && d.dv == HDB && d.T >= 1 && d.T < (int64_t(1) << 30) &&
-           d.B * d.H <= 65535 && tensor_map_encoder() != nullptr;
+    return d.dtype == TC_BF16 && d.dk == d.dv && (d.dk == 64 || d.dk == 128) && d.T >= 1 &&
+           d.T < (int64_t(1) << 30) && d.B * d.H <= 65535 && tensor_map_encoder() != nullptr;
+}
+
+bool backward_memory_tc_supported(const tc_prefill_desc &d) {
+    return backward_window_tc_supported(d) && d.dk == HDB;
 }
 
 int64_t backward_stat_stride(int64_t T) { return (T + BX - 1) / BX * BX; }
 
-cudaError_t launch_backward_window_tc(const tc_prefill_desc &d, const void *q, const void *k,
-                                      const void *v, const void *dy, float *dq, float *dk, float *dv,
-                                      float *lse, float *Dt, int *status, unsigned long long wait_ns,
-                                      cudaStream_t s) {
+template <int NB>
+cudaError_t launch_window_tc_t(const tc_prefill_desc &d, const void *q, const void *k, const void *v,
+                               const void *dy, float *dq, float *dk, float *dv, float *lse, float *Dt,
+                               int *status, unsigned long long wait_ns, cudaStream_t s) {
+    using Cf = BwdCfg<NB>;
+    constexpr int D = Cf::D;
     const int T = (int)d.T, BH = (int)(d.B * d.H);
     const int Tp = (int)backward_stat_stride(d.T);
     CUtensorMap mq_o, mdy_o, mk_x, mv_x, mk_o, mv_o, mq_x, mdy_x, mlse, mD;
-    if (!rows_map(&mq_o, q, T, BH, BO) || !rows_map(&mdy_o, dy, T, BH, BO) ||
-        !rows_map(&mk_x, k, T, BH, BX) || !rows_map(&mv_x, v, T, BH, BX) ||
-        !rows_map(&mk_o, k, T, BH, BO) || !rows_map(&mv_o, v, T, BH, BO) ||
-        !rows_map(&mq_x, q, T, BH, BX) || !rows_map(&mdy_x, dy, T, BH, BX) ||
+    if (!rows_map(&mq_o, q, T, BH, BO, D) || !rows_map(&mdy_o, dy, T, BH, BO, D) ||
+        !rows_map(&mk_x, k, T, BH, BX, D) || !rows_map(&mv_x, v, T, BH, BX, D) ||
+        !rows_map(&mk_o, k, T, BH, BO, D) || !rows_map(&mv_o, v, T, BH, BO, D) ||
+        !rows_map(&mq_x, q, T, BH, BX, D) || !rows_map(&mdy_x, dy, T, BH, BX, D) ||
         !stat_map(&mlse, lse, Tp, BH) || !stat_map(&mD, Dt, Tp, BH))
         return cudaErrorInvalidValue;
     BwdTcParams p{};
@@ -948,24 +979,30 @@ cudaError_t launch_backward_window_tc(const tc_prefill_desc &d, const void *q, c
     p.status = status;
     p.wait_ns = wait_ns;
     const dim3 grid((unsigned)((T + BO - 1) / BO), (unsigned)BH);
-    cudaError_t e = cudaFuncSetAttribute(bwd_window_tc_kernel<false>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BWD_TC);
+    cudaError_t e = cudaFuncSetAttribute(bwd_window_tc_kernel<false, NB>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Cf::SMEM);
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(bwd_window_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)SMEM_BWD_TC);
+    e = cudaFuncSetAttribute(bwd_window_tc_kernel<true, NB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)Cf::SMEM);
     if (e != cudaSuccess) return e;
     p.out0 = dq;
     p.out1 = nullptr;
-    bwd_window_tc_kernel<false><<<grid, kBwdTcThreads, SMEM_BWD_TC, s>>>(mq_o, mdy_o, mk_x, mv_x, mlse, mD, p);
+    bwd_window_tc_kernel<false, NB><<<grid, kBwdTcThreads, Cf::SMEM, s>>>(mq_o, mdy_o, mk_x, mv_x, mlse, mD, p);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     p.out0 = dk;
     p.out1 = dv;
-    bwd_window_tc_kernel<true><<<grid, kBwdTcThreads, SMEM_BWD_TC, s>>>(mk_o, mv_o, mq_x, mdy_x, mlse, mD, p);
+    bwd_window_tc_kernel<true, NB><<<grid, kBwdTcThreads, Cf::SMEM, s>>>(mk_o, mv_o, mq_x, mdy_x, mlse, mD, p);
     return cudaGetLastError();
 }
 
-bool backward_memory_tc_supported(const tc_prefill_desc &d) { return backward_window_tc_supported(d); }
+cudaError_t launch_backward_window_tc(const tc_prefill_desc &d, const void *q, const void *k,
+                                      const void *v, const void *dy, float *dq, float *dk, float *dv,
+                                      float *lse, float *Dt, int *status, unsigned long long wait_ns,
+                                      cudaStream_t s) {
+    return d.dk == 128 ? launch_window_tc_t<2>(d, q, k, v, dy, dq, dk, dv, lse, Dt, status, wait_ns, s)
+                       : launch_window_tc_t<1>(d, q, k, v, dy, dq, dk, dv, lse, Dt, status, wait_ns, s);
+}
 
 cudaError_t launch_backward_chunks_tc(const tc_prefill_desc &d, const void *q, const void *k,
                                       const void *v, const void *dy, const float *lam,

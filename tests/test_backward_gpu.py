@@ -33,7 +33,9 @@ CASES = [
     (1, 2, 77, 64, 64, 512, "bf16"),    # W > T, one partial 128-row block
     (1, 1, 700, 64, 64, 1, "bf16"),     # W = 1: every key its own query only
     (1, 2, 2100, 64, 64, 512, "bf16"),  # many tiles per block, 2 blocks per SM
-    (1, 2, 200, 128, 128, 64, "bf16"),  # d = 128: SIMT window kernels, 4 columns per lane
+    (1, 2, 200, 128, 128, 64, "bf16"),  # d = 128: tensor-core window, SIMT memory part
+    (2, 2, 700, 128, 128, 200, "bf16"), # d = 128, W not a multiple of the tiles, several chunks
+    (1, 1, 300, 128, 128, 512, "bf16"), # d = 128, W > T
     (1, 1, 150, 128, 40, 16, "f32"),    # d_k = 128, d_v not a multiple of 32
 ]
 
@@ -50,8 +52,8 @@ def test_backward_matches_oracle(cuda_device, case):
     got = tc.backward(d(x.q), d(x.k), d(x.v), d(x.lam), d(x.eta), d(x.g), W, d(dy))
     torch.cuda.synchronize()
     assert tc.device_status() == 0
-    # bf16 with d = 64 takes the tensor-core kernels, every other case SIMT
-    assert tc.backward_launch_count(x.q, W, x.v)[1] == (dtype == "bf16" and dk == dv == 64)
+    # bf16 with d = 64 or 128 takes the tensor-core window kernels, every other case SIMT
+    assert tc.backward_launch_count(x.q, W, x.v)[1] == (dtype == "bf16" and dk == dv and dk in (64, 128))
     ref = oracle.backward(x.q, x.k, x.v, x.lam, x.eta, x.g, W, dy)
     for name, a, b in zip(("dq", "dk", "dv", "dlam", "deta", "dg"), got, ref):
         if np.abs(b).max() == 0:
