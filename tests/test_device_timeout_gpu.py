@@ -51,3 +51,58 @@ def test_wait_limit_runs_out_and_the_context_stays_usable(cuda_device):
     A = A.cpu().numpy()
     assert np.linalg.norm(y - yo) <= 1e-2 * np.linalg.norm(yo)
     assert np.linalg.norm(A - Ao) <= 1e-3 * np.linalg.norm(Ao)
+
+
+def _rel(x, ref):
+    return float(np.linalg.norm(np.asarray(x, np.float64) - ref) / np.linalg.norm(ref))
+
+
+@pytest.mark.parametrize("d,W", [(64, 200), (128, 256)], ids=["d64_W200", "d128_W256"])
+def test_general_path_wait_limit_runs_out(cuda_device, d, W):
+    """The general tensor-core prefill (window, sums, reads): the same bounded
+    waits and drains, then a clean call on the same context."""
+    import sliding_window_attention_tc_b200 as tc
+    B, H, T = 2, 4, 1500
+    x = wl.random_prefill(B, H, T, d, d, W, 64, dtype="bf16", seed=41)
+    desc = tc.make_prefill_desc(B, H, T, d, d, W, 64, tc.TC_BF16)
+    assert tc.prefill_launch_count(desc) == 4  # sums, scan, reads, window
+    assert tc.device_status() == 0
+    try:
+        tc.set_wait_limit_ns(1)
+        _run(tc, x, cuda_device)
+        assert tc.device_status() == TC_ERR_DEVICE_TIMEOUT
+    finally:
+        tc.set_wait_limit_ns(0)
+    y, A = _run(tc, x, cuda_device)
+    assert tc.device_status() == 0
+    yo, Ao = oracle.prefill(x.q, x.k, x.v, x.lam, x.eta, x.g, x.W)
+    assert _rel(y.float().cpu().numpy(), yo) <= 1e-2
+    assert _rel(A.cpu().numpy(), Ao) <= 1e-3
+
+
+def test_backward_wait_limit_runs_out(cuda_device):
+    """The backward's tensor-core kernels (window, per-chunk sums and
+    gradients): the waits give up and drain, then a clean call matches the
+    oracle backward."""
+    import sliding_window_attention_tc_b200 as tc
+    B, H, T, d, W = 1, 2, 900, 64, 128
+    x = wl.random_prefill(B, H, T, d, d, W, 64, dtype="bf16", seed=43)
+    gen = torch.Generator().manual_seed(44)
+    dy = (torch.randn(B, H, T, d, generator=gen) / 4).to(x.q.dtype)
+    dev = cuda_device
+    args = [t.to(dev).contiguous() for t in (x.q, x.k, x.v, x.lam, x.eta, x.g)]
+    assert tc.backward_launch_count(x.q, W)[1]
+    try:
+        tc.set_wait_limit_ns(1)
+        tc.backward(*args, W, dy.to(dev))
+        torch.cuda.synchronize()
+        assert tc.device_status() == TC_ERR_DEVICE_TIMEOUT
+    finally:
+        tc.set_wait_limit_ns(0)
+    got = tc.backward(*args, W, dy.to(dev))
+    torch.cuda.synchronize()
+    assert tc.device_status() == 0
+    ref = oracle.backward(x.q, x.k, x.v, x.lam, x.eta, x.g, W, dy)
+    for a, b in zip(got[:3], ref[:3]):
+        a = a.cpu().numpy()
+        assert np.abs(a - b).max() <= 2e-4 * np.abs(b).max()
