@@ -152,3 +152,34 @@ def test_general_full_size_bench_workloads(cuda_device):
         yo, Ao = oracle.prefill(sl(q), sl(k), sl(v), lam[h:h + 1].cpu(), eta[h:h + 1].cpu(), g[h:h + 1].cpu(), W)
         assert rel_l2(y[b, h].float().cpu().numpy(), yo[0, 0]) <= BF16_Y_TOL
         assert rel_l2(A[b, h].cpu().numpy(), Ao[0, 0]) <= BF16_A_TOL
+
+
+def test_general_prefill_fills_a_d128_decode_ring(cuda_device):
+    """The decode workload's head size and window (d = 128, W = 256 here to
+    keep the oracle short): a bf16 prefill on the general tensor-core path
+    hands its state to the decode stream (ring slot j mod W holds token j,
+    A = A_final, t = T), which continues; both match the oracle over all
+    tokens."""
+    tc = _tc()
+    B, H, T, n, d, W = 1, 2, 700, 24, 128, 256
+    x = wl.random_prefill(B, H, T + n, d, d, W, 64, dtype="bf16", seed=51)
+    dev = cuda_device
+    dd = lambda t: t.to(dev).contiguous()
+    desc = tc.make_prefill_desc(B, H, T, d, d, W, 64, tc.TC_BF16)
+    assert tc.prefill_launch_count(desc) == general_launches(T, W)
+    lam, eta, g = dd(x.lam), dd(x.eta), dd(x.g)
+    y, A = tc.prefill(dd(x.q[:, :, :T]), dd(x.k[:, :, :T]), dd(x.v[:, :, :T]), lam, eta, g, W, 64)
+    ring_k = torch.zeros(B, H, W, d, dtype=torch.bfloat16, device=dev)
+    ring_v = torch.zeros(B, H, W, d, dtype=torch.bfloat16, device=dev)
+    for j in range(T - W, T):
+        ring_k[:, :, j % W] = x.k[:, :, j].to(dev)
+        ring_v[:, :, j % W] = x.v[:, :, j].to(dev)
+    st = tc.DecodeState(ring_k, ring_v, A, lam, eta, g, T)
+    ys = [tc.decode_step(st, dd(x.q[:, :, j]), dd(x.k[:, :, j]), dd(x.v[:, :, j])).float().cpu()
+          for j in range(T, T + n)]
+    torch.cuda.synchronize()
+    assert tc.device_status() == 0
+    yo, Ao = oracle.prefill(x.q, x.k, x.v, x.lam, x.eta, x.g, W)
+    assert rel_l2(y.float().cpu().numpy(), yo[:, :, :T]) <= BF16_Y_TOL
+    assert rel_l2(torch.stack(ys, 2).numpy(), yo[:, :, T:]) <= BF16_Y_TOL
+    assert rel_l2(st.A.cpu().numpy(), Ao) <= BF16_A_TOL
