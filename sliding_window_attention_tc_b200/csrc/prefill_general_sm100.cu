@@ -5,19 +5,18 @@
 // "Tensor Cache: Eviction-conditioned Associative Memory for Transformers":
 // the window read of §3.1 eq. (1) and the memory of §3.2 / Fig. 2 (write on
 // eviction, A <- lam A + eta k v^T; read m = q A; y = y_local + sigma(g) m),
-// the memory in the chunked form of the abstract and §2 (chunks of CG = 128
-// evictions).  Five kernels, all but the copy and the scan on tcgen05:
+// the memory in the chunked form of the abstract and §2, one chunk per block
+// of 128 new rows: the evictions that block's reads take in.  Four kernels,
+// all but the copy and the scan on tcgen05:
 //   gen_combine_kernel   halo + new keys / values into one sequence (only
 //                        when continuing with a halo);
 //   gen_sums_kernel      per chunk dA_c = eta K^T diag(lam^(L-1-i)) V, one
 //                        M = 128 product (two chunks side by side for D = 64);
 //   gen_scan_kernel      A_c = chunk start states from A_init, and A_final;
-//   gen_read_kernel      per chunk the reads m_i = lam^(i+1) q'_i A_c +
-//                        eta sum_{l<=i} lam^(i-l) (q'_i . k_l) v_l into a row
-//                        buffer (q'_i the query at t = e0 + i + W);
 //   gen_window_kernel    the window softmax in one pass (online rescaling of
-//                        the output accumulator in TMEM) and the fusion
-//                        y = y_local + sigma(g) m.
+//                        the output accumulator in TMEM), the block's reads
+//                        m = lam^(i+1) q A_c + the in-chunk terms from the same
+//                        scores, and the fusion y = y_local + sigma(g) m.
 // Positions are those of the combined sequence (halo first): token tau is a
 // new row when tau >= n_halo, evictions are tau = 0 .. n_halo + T - W - 1 and
 // A_init holds every eviction before the combined sequence.  float32 values
@@ -51,7 +50,8 @@ struct GenParams {
     const __nv_bfloat16 *q, *k, *v;  // q: [BH][T][D] new rows; k, v: the combined sequence
     __nv_bfloat16 *y;
     float *mrow;                     // [BH][T][D] float32 reads (null: none)
-    float *dA;                       // [BH][nC][D][D]: increments, then start states
+    float *dA;                       // [BH][nC][D][D]: per-chunk increments
+    __nv_bfloat16 *ab;               // [BH][nC][2][D][D]: chunk start states as bf16 hi, lo
     float *A_final;
     const float *A_init;
     const float *lam, *eta, *g;
@@ -88,8 +88,18 @@ __device__ __forceinline__ GSeq gseq(const GenParams &p, int bh) {
         s.T = s.Tc = ok ? (int)(e - a) : 0;
     }
     s.E = s.Tc > p.W ? s.Tc - p.W : 0;
-    s.nC = (s.E + CG - 1) / CG;
+    s.nC = (s.T + CG - 1) / CG;  // one chunk per block of 128 new rows
     return s;
+}
+
+// Chunk b holds the evictions that the reads of query block b (new rows
+// 128 b .. 128 b + 127, combined positions n_halo + 128 b + r) take in:
+// [e_lo, e_hi), possibly empty.  Consecutive chunks are adjacent, and since
+// the halo is at most W long the first starts at eviction 0.
+__device__ __forceinline__ void chunk_range(const GenParams &p, const GSeq &s, int b, int &e_lo, int &e_hi) {
+    const int a = p.n_halo + CG * b - p.W;
+    e_lo = max(0, a);
+    e_hi = max(e_lo, min(s.E, a + CG));
 }
 // Element offset of row `row` (of the combined sequence for k and v, else of the
 // new rows) of a [.][D] tensor; rows_fixed is the row count of the fixed layout.
@@ -131,30 +141,46 @@ __device__ __forceinline__ void tma_rows_nb(uint8_t *dst, const CUtensorMap *m, 
 }
 
 // ===========================================================================
-// Window part.  A CTA owns 128 new query rows (TMEM lanes); 64-row key
-// tiles stream through NS stages.  Scores have two TMEM buffers: S of tile
-// n+1 is issued before P V of tile n, so the element-wise warps find the
-// next scores ready when they finish a tile.  Per tile they take the row max,
-// rescale O in TMEM when it grew (after waiting for the previous P V, which a
-// per-tile commit reports), write P = exp2(s - m) as bf16 over S, and
-// O += P V runs from TMEM.
+// Window part, and with it the memory's reads.  A CTA owns 128 new query rows
+// (TMEM lanes, query block b); 64-row key tiles stream through NS stages.
+// Scores have two TMEM buffers: S of tile n+1 is issued before P V of tile
+// n, so the softmax warpgroup finds the next scores ready when it finishes a
+// tile.  Per tile it takes the row max over the band mask 0 <= tau - j < W,
+// rescales O in TMEM when the max grew (after waiting for the previous P V,
+// which a per-tile commit reports), writes P = exp2(s - m) as bf16 over S,
+// and O += P V runs with P as the TMEM operand.
+// With the memory (dA set, no m rows): the reads of block b take in chunk b's
+// evictions [e_lo, e_hi) (the keys just left of the window) and the start
+// state A_b, m_r = lam^(tau-W-e_lo+1) q_r A_b + sum_{e_lo <= j <= tau-W}
+// eta lam^(tau-W-j) <q_r, k_j> v_j.  The key tiles then start at e_lo, the
+// second term is P' V with P' = eta lam^(tau-W-j) s from the same scores
+// (written beside P in the score buffer, accumulated in its own TMEM
+// columns), and the first is one more MMA after the last tile, Q A_b with A_b
+// as bf16 hi + lo in shared memory.  Score buffer layout (bf16 pairs, 64
+// keys): [P keys 0-31 | P' keys 0-31 | P keys 32-63 | P' keys 32-63].
 template <int NB>
 struct WinCfg {
     static constexpr int D = 64 * NB;
     static constexpr int NS = NB == 1 ? 4 : 3;
     static constexpr uint32_t Q_B = NB * BLK128;
     static constexpr uint32_t X_B = NB * BLK64;   // one K or V tile
+    static constexpr uint32_t ST_BLK = D * 128;   // D rows x 64 columns of A_b
     static constexpr uint32_t OFF_Q = 0;
     static constexpr uint32_t OFF_X = Q_B;         // NS x (K tile, V tile)
-    static constexpr uint32_t OFF_BAR = OFF_X + NS * 2 * X_B;
-    static constexpr uint32_t SMEM = OFF_BAR + 256 + 1024;  // (8 + 2 NS) barriers, TMEM address, abort flag
-    static constexpr uint32_t TM_S = 0, TM_O = 128, COLS = 256;  // two 64-column score buffers, then O
+    static constexpr uint32_t OFF_A = OFF_X + NS * 2 * X_B;  // A_b hi: NB blocks, lo: NB blocks
+    static constexpr uint32_t OFF_PW = OFF_A + 2 * NB * ST_BLK;  // lam^n, n = 0 .. 128
+    static constexpr uint32_t OFF_BAR = OFF_PW + 136 * 4;
+    static constexpr uint32_t SMEM = OFF_BAR + 256 + 1024;  // (9 + 2 NS) barriers, TMEM address, abort flag
+    // two 64-column score buffers, O, the reads' accumulator (P' V, then + Q A_b
+    // lands in the score buffers' columns after the last tile)
+    static constexpr uint32_t TM_S = 0, TM_O = 128, TM_MI = 128 + D, COLS = NB == 1 ? 256 : 512;
 };
 
 template <int NB>
 __global__ void __launch_bounds__(kGThreads, NB == 1 ? 2 : 1)
     gen_window_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
-                      const __grid_constant__ CUtensorMap tv, GenParams p) {
+                      const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tab,
+                      GenParams p) {
     using C = WinCfg<NB>;
     constexpr int D = C::D, NS = C::NS;
     extern __shared__ uint8_t smem_raw[];
@@ -162,17 +188,26 @@ __global__ void __launch_bounds__(kGThreads, NB == 1 ? 2 : 1)
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + C::OFF_BAR);
     uint64_t *q_full = bars, *x_full = bars + 1, *x_empty = x_full + NS, *s_full = x_empty + NS;
     uint64_t *p_ready = s_full + 2, *o_done = p_ready + 2, *o_full = o_done + 1, *mma_done = o_full + 1;
-    uint32_t *tmem_base = reinterpret_cast<uint32_t *>(mma_done + 1);
+    uint64_t *a_ready = mma_done + 1;
+    uint32_t *tmem_base = reinterpret_cast<uint32_t *>(a_ready + 1);
     volatile int *abort = reinterpret_cast<volatile int *>(tmem_base + 1);
+    float *pw = reinterpret_cast<float *>(sm + C::OFF_PW);
 
     const int tid = threadIdx.x, warp = tid >> 5;
     const GSeq sq = gseq(p, blockIdx.y);
     const int t0 = blockIdx.x * CG;           // first new row
     if (t0 >= sq.T) return;                   // past this sequence (variable-length calls)
     const int tau0 = p.n_halo + t0;           // its combined position
-    const int lo = max(0, tau0 - p.W + 1), hi = min(sq.Tc - 1, tau0 + CG - 1);
+    // the memory's reads of this block: chunk b = blockIdx.x
+    const bool mem = p.dA != nullptr && p.mrow == nullptr;
+    int e_lo = 0, e_hi = 0;
+    if (mem) chunk_range(p, sq, blockIdx.x, e_lo, e_hi);
+    const bool reads = mem && e_hi > e_lo;
+    const int lo = reads ? e_lo : max(0, tau0 - p.W + 1), hi = min(sq.Tc - 1, tau0 + CG - 1);
     const int xs = lo & ~(GX - 1);
     const int N = (hi - xs) / GX + 1;
+    // key tiles holding evictions of the chunk (CTA-uniform)
+    auto tile_reads = [&](int n) { return reads && xs + GX * n < e_hi && xs + GX * n + GX > e_lo; };
 
     if (tid == 0) {
         mbar_init(q_full, 1);
@@ -187,6 +222,7 @@ __global__ void __launch_bounds__(kGThreads, NB == 1 ? 2 : 1)
         mbar_init(o_done, 1);
         mbar_init(o_full, 1);
         mbar_init(mma_done, 1);
+        mbar_init(a_ready, 1);
         *abort = 0;
         fence_mbar_init();
     }
@@ -203,6 +239,17 @@ __global__ void __launch_bounds__(kGThreads, NB == 1 ? 2 : 1)
         if (tid == 0) {
             mbar_expect_tx(q_full, C::Q_B);
             tma_rows_nb<NB>(sm + C::OFF_Q, &tq, q_full, t0, sq, BLK128);
+            if (reads) {
+                // A_b hi, lo: rows (slot * 2 + part) * D of the [.][D] map, NB column blocks
+                const int slot = sq.bh * p.nC + blockIdx.x;
+                mbar_expect_tx(a_ready, 2 * NB * C::ST_BLK);
+#pragma unroll
+                for (int part = 0; part < 2; ++part)
+#pragma unroll
+                    for (int b = 0; b < NB; ++b)
+                        tma_load_2d(sm + C::OFF_A + (part * NB + b) * C::ST_BLK, &tab, a_ready, 64 * b,
+                                    (slot * 2 + part) * D);
+            }
             int n = 0;
             for (; n < N; ++n) {
                 const int s = n % NS;
@@ -213,6 +260,7 @@ __global__ void __launch_bounds__(kGThreads, NB == 1 ? 2 : 1)
                 tma_rows_nb<NB>(dst + C::X_B, &tv, &x_full[s], xs + GX * n, sq, BLK64);
             }
             mbar_wait_drain(q_full, 0);
+            if (reads) mbar_wait_drain(a_ready, 0);
             for (int st = 0; st < NS; ++st) {
                 const int fills = n > st ? (n - 1 - st) / NS + 1 : 0;
                 if (fills) mbar_wait_drain(&x_full[st], (fills - 1) & 1);
@@ -221,7 +269,7 @@ __global__ void __launch_bounds__(kGThreads, NB == 1 ? 2 : 1)
     } else if (warp == 1) {
         const uint32_t id_s = idesc_bf16(128, 64, false, false);
         const uint32_t id_o = idesc_bf16(128, D, false, true);
-        const uint32_t sq = smem_u32(sm + C::OFF_Q), sx = smem_u32(sm + C::OFF_X);
+        const uint32_t sq_a = smem_u32(sm + C::OFF_Q), sx = smem_u32(sm + C::OFF_X);
         bool ok = gwait(q_full, 0, abort, p);
         // S(n) into score buffer n % 2
         auto issue_s = [&](int n) -> bool {
@@ -233,44 +281,80 @@ __global__ void __launch_bounds__(kGThreads, NB == 1 ? 2 : 1)
             for (int b = 0; b < NB; ++b)
 #pragma unroll
                 for (int k = 0; k < 4; ++k)
-                    mma_ss_w(sb, sdesc_sw128(sq + b * BLK128, 16, 1024) + 2 * k,
+                    mma_ss_w(sb, sdesc_sw128(sq_a + b * BLK128, 16, 1024) + 2 * k,
                              sdesc_sw128(kx + b * BLK64, 16, 1024) + 2 * k, id_s, (b > 0 || k > 0) ? 1u : 0u);
             mma_commit_w(&s_full[n & 1]);
             return true;
         };
         if (ok) ok = issue_s(0);
+        bool first_read = true;
         for (int n = 0; ok && n < N; ++n) {
             // the next scores go out before this tile's P V
             if (n + 1 < N && !(ok = issue_s(n + 1))) break;
             if (!(ok = gwait(&p_ready[n & 1], (n >> 1) & 1, abort, p))) break;
             tc_fence_after();
-            // O += P V: P (64 keys) in score buffer n % 2, V read MN-major
+            // O += P V (and M += P' V): K-step k (keys 16 k ..) at columns 32 (k / 2) + 8 (k % 2)
             const uint64_t vd = sdesc_sw128(sx + (n % NS) * 2 * C::X_B + C::X_B, BLK64, 1024);
             const uint32_t pb = tb + C::TM_S + 64 * (n & 1);
 #pragma unroll
-            for (int k = 0; k < 4; ++k) mma_ts_w(tb + C::TM_O, pb + 8 * k, vd + 128 * k, id_o, (n > 0 || k > 0) ? 1u : 0u);
+            for (int k = 0; k < 4; ++k)
+                mma_ts_w(tb + C::TM_O, pb + 32 * (k >> 1) + 8 * (k & 1), vd + 128 * k, id_o,
+                         (n > 0 || k > 0) ? 1u : 0u);
+            if (tile_reads(n)) {
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    mma_ts_w(tb + C::TM_MI, pb + 32 * (k >> 1) + 16 + 8 * (k & 1), vd + 128 * k, id_o,
+                             (!first_read || k > 0) ? 1u : 0u);
+                first_read = false;
+            }
             mma_commit_w(&x_empty[n % NS]);
             mma_commit_w(o_done);
+        }
+        if (ok && reads) {
+            // Q A_b (hi + lo) into the score columns, after every P V of the loop
+            if ((ok = gwait(a_ready, 0, abort, p))) {
+                tc_fence_after();
+                const uint32_t sa = smem_u32(sm + C::OFF_A);
+#pragma unroll
+                for (int part = 0; part < 2; ++part)
+#pragma unroll
+                    for (int k = 0; k < 4 * NB; ++k)
+                        mma_ss_w(tb + C::TM_S, sdesc_sw128(sq_a + (k >> 2) * BLK128, 16, 1024) + 2 * (k & 3),
+                                 sdesc_sw128(sa + part * NB * C::ST_BLK, C::ST_BLK, 1024) + 128 * k, id_o,
+                                 (part > 0 || k > 0) ? 1u : 0u);
+            }
         }
         if (ok) mma_commit_w(o_full);
         mma_commit_w(mma_done);
         mbar_wait_drain(mma_done, 0);
     } else {
         const int q4 = warp & 3;
-        const int r = 32 * q4 + (tid & 31);
+        const int x = 32 * q4 + (tid & 31);
+        const int r = x;
         const uint32_t lanes = tb + ((uint32_t)(32 * q4) << 16);
         const int t = t0 + r, tau = tau0 + r;
         const uint32_t wlim = t < sq.T ? (uint32_t)p.W : 0u;
         const float sl2 = kLog2eG * rsqrtf((float)D);
+        float eta = 0.f;
+        if (reads) {
+            // lam^n for the reads' weights (A_b arrives by copy)
+            gpowers(pw, CG, p.lam[sq.h], x);
+            eta = p.eta[sq.h];
+            gbar128();  // pw complete
+        }
+        // the reads of row r cover evictions e_lo .. tau - W (none when tau < W or t >= T)
+        const int rd_hi = (reads && t < sq.T) ? tau - p.W : -1;
         float m_run = -INFINITY, l_run = 0.f;
         bool ok = true;
         for (int n = 0; n < N; ++n) {
             if (!(ok = gwait(&s_full[n & 1], (n >> 1) & 1, abort, p))) break;
             tc_fence_after();
             const uint32_t sbuf = lanes + C::TM_S + 64 * (n & 1);
-            const int base = tau - (xs + GX * n);  // tau - j = base - c
-            // the row max over both 32-column halves, then the exponentials from a
-            // second read of the scores (fewer live registers)
+            const int j0 = xs + GX * n;
+            const int base = tau - j0;  // tau - j = base - c
+            const bool tr = tile_reads(n);
+            // the row max over both 32-column halves, then the exponentials (and
+            // the reads' weights) from a second read of the scores
             float mx = -INFINITY;
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
@@ -316,7 +400,19 @@ __global__ void __launch_bounds__(kGThreads, NB == 1 ? 2 : 1)
                     sum += a + b;
                     pk[e] = pack_bf16(a, b);
                 }
-                tmem_st16(sbuf + 16 * h, pk);
+                tmem_st16(sbuf + 32 * h, pk);
+                if (tr) {
+                    // P' = eta lam^(tau-W-j) s for e_lo <= j <= tau - W
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        const int j = j0 + 32 * h + 2 * e;
+                        const int d0 = rd_hi - j, d1 = d0 - 1;
+                        const float a = (d0 >= 0 && j >= e_lo) ? eta * pw[min(d0, CG)] * __uint_as_float(sr[2 * e]) : 0.f;
+                        const float b = (d1 >= 0 && j + 1 >= e_lo) ? eta * pw[min(d1, CG)] * __uint_as_float(sr[2 * e + 1]) : 0.f;
+                        pk[e] = pack_bf16(a, b);
+                    }
+                    tmem_st16(sbuf + 32 * h + 16, pk);
+                }
             }
             l_run = fmaf(l_run, corr, sum);
             m_run = m_new;
@@ -328,19 +424,25 @@ __global__ void __launch_bounds__(kGThreads, NB == 1 ? 2 : 1)
         if (ok && gwait(o_full, 0, abort, p)) {
             tc_fence_after();
             const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
-            const bool has_m = p.mrow && tau >= p.W && t < sq.T;
+            const bool has_m = (p.mrow && tau >= p.W && t < sq.T) || rd_hi >= e_lo;
             const float sg = has_m ? 1.f / (1.f + expf(-p.g[sq.h])) : 0.f;
-            const float *mr = has_m ? p.mrow + grow(sq, t, p.T, p.H, D) : nullptr;
+            const float *mr = (p.mrow && has_m) ? p.mrow + grow(sq, t, p.T, p.H, D) : nullptr;
+            // m = lam^(tau-W-e_lo+1) (q A_b) + (P' V) for the in-kernel reads
+            const float dec = (reads && rd_hi >= e_lo) ? pw[min(rd_hi - e_lo + 1, CG)] : 0.f;
 #pragma unroll
             for (int c0 = 0; c0 < D; c0 += 32) {
-                uint32_t o[32];
+                uint32_t o[32], ma[32], mi[32];
                 tmem_ld32(lanes + C::TM_O + c0, o);
+                if (reads) {
+                    tmem_ld32(lanes + C::TM_S + c0, ma);
+                    tmem_ld32(lanes + C::TM_MI + c0, mi);
+                }
                 tmem_wait_ld();
                 if (t < sq.T) {
                     float f[32];
 #pragma unroll
                     for (int c = 0; c < 32; ++c) f[c] = __uint_as_float(o[c]) * inv_l;
-                    if (has_m) {
+                    if (mr) {
 #pragma unroll
                         for (int c = 0; c < 32; c += 4) {
                             const float4 mv = *reinterpret_cast<const float4 *>(mr + c0 + c);
@@ -349,6 +451,10 @@ __global__ void __launch_bounds__(kGThreads, NB == 1 ? 2 : 1)
                             f[c + 2] = fmaf(sg, mv.z, f[c + 2]);
                             f[c + 3] = fmaf(sg, mv.w, f[c + 3]);
                         }
+                    } else if (reads && has_m) {
+#pragma unroll
+                        for (int c = 0; c < 32; ++c)
+                            f[c] = fmaf(sg, fmaf(dec, __uint_as_float(ma[c]), __uint_as_float(mi[c])), f[c]);
                     }
                     uint4 *dst = reinterpret_cast<uint4 *>(p.y + grow(sq, t, p.T, p.H, D) + c0);
 #pragma unroll
@@ -416,15 +522,18 @@ __global__ void __launch_bounds__(kGThreads, 2)
         if (tid == 0) {
             mbar_expect_tx(in_full, 2 * BLK128);
             // K of chunks c_first, c_first + 1 (D = 64) or the two column halves of
-            // chunk c_first (D = 128); rows past the data read zero, rows past the
-            // sequence (packed calls) meet zero weights
-            tma_rows_nb<1>(sm + SUM_OFF_A, &tk, in_full, c_first * CG, sq, BLK128);
+            // chunk c_first (D = 128), from each chunk's first eviction; rows past
+            // the data read zero, rows past a chunk meet zero weights
+            int lo0, hi0, lo1, hi1;
+            chunk_range(p, sq, c_first, lo0, hi0);
+            chunk_range(p, sq, c_first + 1, lo1, hi1);
+            tma_rows_nb<1>(sm + SUM_OFF_A, &tk, in_full, lo0, sq, BLK128);
             if (NB == 1)
-                tma_rows_nb<1>(sm + SUM_OFF_A + BLK128, &tk, in_full, (c_first + 1) * CG, sq, BLK128);
+                tma_rows_nb<1>(sm + SUM_OFF_A + BLK128, &tk, in_full, lo1, sq, BLK128);
             else if (sq.packed)
-                tma_load_3d(sm + SUM_OFF_A + BLK128, &tk, in_full, 64, sq.h, sq.row0 + c_first * CG);
+                tma_load_3d(sm + SUM_OFF_A + BLK128, &tk, in_full, 64, sq.h, sq.row0 + lo0);
             else
-                tma_load_3d(sm + SUM_OFF_A + BLK128, &tk, in_full, 64, c_first * CG, bh);
+                tma_load_3d(sm + SUM_OFF_A + BLK128, &tk, in_full, 64, lo0, bh);
             mbar_wait_drain(in_full, 0);
         }
     } else if (warp == 1) {
@@ -455,8 +564,9 @@ __global__ void __launch_bounds__(kGThreads, 2)
 #pragma unroll
         for (int b = 0; b < 2; ++b) {
             const int c = NB == 1 ? c_first + b : c_first;
-            const int e0 = c * CG;
-            const int L = c < sq.nC ? min(CG, sq.E - e0) : 0;
+            int e0, e1;
+            chunk_range(p, sq, c, e0, e1);
+            const int L = c < sq.nC ? e1 - e0 : 0;
             const float w = x < L ? pw[L - 1 - x] : 0.f;
             const int col0 = NB == 1 ? 0 : 64 * b;
             const uint4 *src = reinterpret_cast<const uint4 *>(p.v + grow(sq, x < L ? e0 + x : 0, p.Tc, p.H, D) + col0);
@@ -517,15 +627,16 @@ __global__ void __launch_bounds__(kGThreads, 2)
 // ===========================================================================
 // Chunk start states, one thread per state element: A_c (in place over the
 // increments) and A_final.
+constexpr int kMaxScanChunks = 4096;  // chunk decays kept in shared memory (longer rows compute theirs)
 __global__ void __launch_bounds__(256) gen_scan_kernel(GenParams p, int D) {
-    __shared__ float decay[2];
+    __shared__ float decay[kMaxScanChunks];  // lam^(length of chunk c)
     const GSeq sq = gseq(p, blockIdx.y);
     const int bh = sq.bh, nC = sq.nC;
-    if (threadIdx.x < 2) {
-        const double l2l = log2((double)p.lam[sq.h]);
-        const int last = nC > 0 ? sq.E - (nC - 1) * CG : 0;
-        const int n = threadIdx.x == 0 ? CG : last;
-        decay[threadIdx.x] = (float)exp2((double)n * l2l);
+    const double l2l = log2((double)p.lam[sq.h]);
+    for (int c = threadIdx.x; c < nC && c < kMaxScanChunks; c += blockDim.x) {
+        int e0, e1;
+        chunk_range(p, sq, c, e0, e1);
+        decay[c] = (float)exp2((double)(e1 - e0) * l2l);
     }
     __syncthreads();
     const int x = blockIdx.x * blockDim.x + threadIdx.x;
@@ -537,199 +648,29 @@ __global__ void __launch_bounds__(256) gen_scan_kernel(GenParams p, int D) {
     for (int c0 = 0; c0 < nC; c0 += kB) {
         float d[kB];
 #pragma unroll
-        for (int u = 0; u < kB; ++u) d[u] = c0 + u < nC ? dA[(size_t)(c0 + u) * nel] : 0.f;
+        for (int u = 0; u < kB; ++u) d[u] = (c0 + u < nC && sq.E > 0) ? dA[(size_t)(c0 + u) * nel] : 0.f;
 #pragma unroll
         for (int u = 0; u < kB; ++u) {
             const int c = c0 + u;
             if (c < nC) {
-                dA[(size_t)c * nel] = A;
-                A = fmaf(c == nC - 1 ? decay[1] : decay[0], A, d[u]);
+                // the start state as bf16 hi + lo, row-major, for the window kernel's copy
+                const __nv_bfloat16 hi = __float2bfloat16_rn(A);
+                __nv_bfloat16 *o = p.ab + (((size_t)bh * p.nC + c) * 2) * nel + x;
+                o[0] = hi;
+                o[nel] = __float2bfloat16_rn(A - __bfloat162float(hi));
+                float dc;
+                if (c < kMaxScanChunks) {
+                    dc = decay[c];
+                } else {
+                    int e0, e1;
+                    chunk_range(p, sq, c, e0, e1);
+                    dc = (float)exp2((double)(e1 - e0) * l2l);
+                }
+                A = fmaf(dc, A, d[u]);
             }
         }
     }
     if (p.A_final) p.A_final[(size_t)bh * nel + x] = A;
-}
-
-// ===========================================================================
-// Reads of one chunk: QK = Q' K^T (TMEM); Mq = eta lam^(i-l) QK on l <= i < L
-// as bf16 hi + lo over QK; mA = Q' A_c (A_c as bf16 hi + lo in shared
-// memory, read MN-major); mI = Mq V; m = lam^(i+1) mA + mI into mrow.
-template <int NB>
-struct ReadCfg {
-    static constexpr int D = 64 * NB;
-    static constexpr uint32_t IN_B = NB * BLK128;            // a 128-row input tile
-    static constexpr uint32_t OFF_Q = 0, OFF_K = IN_B, OFF_V = 2 * IN_B;
-    static constexpr uint32_t ST_BLK = D * 128;              // D rows x 64 columns of A_c
-    static constexpr uint32_t OFF_A = 3 * IN_B;              // hi: NB blocks, lo: NB blocks
-    static constexpr uint32_t OFF_PW = OFF_A + 2 * NB * ST_BLK;
-    static constexpr uint32_t OFF_BAR = OFF_PW + 136 * 4;
-    static constexpr uint32_t SMEM = OFF_BAR + 64 + 1024;
-    static constexpr uint32_t TM_QK = 0, TM_MA = 128, TM_MI = 128 + D, COLS = NB == 1 ? 256 : 512;
-};
-
-template <int NB>
-__global__ void __launch_bounds__(kGThreads, 1)
-    gen_read_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
-                    const __grid_constant__ CUtensorMap tv, GenParams p) {
-    using C = ReadCfg<NB>;
-    constexpr int D = C::D;
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + C::OFF_BAR);
-    uint64_t *in_full = bars, *s_full = bars + 1, *m_ready = bars + 2, *acc_full = bars + 3;
-    uint64_t *mma_done = bars + 4;
-    uint32_t *tmem_base = reinterpret_cast<uint32_t *>(bars + 5);
-    volatile int *abort = reinterpret_cast<volatile int *>(tmem_base + 1);
-    float *pw = reinterpret_cast<float *>(sm + C::OFF_PW);
-    const int tid = threadIdx.x, warp = tid >> 5;
-    const GSeq sq = gseq(p, blockIdx.y);
-    const int c = blockIdx.x, bh = sq.bh, h = sq.h;
-    if (c >= sq.nC) return;  // past this sequence's chunks (variable-length calls)
-    const int e0 = c * CG, L = min(CG, sq.E - e0);
-    const int qrow0 = e0 + p.W - p.n_halo;  // new row of eviction e0's read
-
-    if (tid == 0) {
-        mbar_init(in_full, 1);
-        mbar_init(s_full, 1);
-        mbar_init(m_ready, 128);
-        mbar_init(acc_full, 1);
-        mbar_init(mma_done, 1);
-        *abort = 0;
-        fence_mbar_init();
-    }
-    if (warp == 1) {
-        tmem_alloc(tmem_base, C::COLS);
-        tmem_relinquish();
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tb = *tmem_base;
-
-    if (warp == 0) {
-        if (tid == 0) {
-            mbar_expect_tx(in_full, 3 * C::IN_B);
-            tma_rows_nb<NB>(sm + C::OFF_Q, &tq, in_full, qrow0, sq, BLK128);
-            tma_rows_nb<NB>(sm + C::OFF_K, &tk, in_full, e0, sq, BLK128);
-            tma_rows_nb<NB>(sm + C::OFF_V, &tv, in_full, e0, sq, BLK128);
-            mbar_wait_drain(in_full, 0);
-        }
-    } else if (warp == 1) {
-        const uint32_t base = smem_u32(sm);
-        const uint32_t sq = base + C::OFF_Q, sk = base + C::OFF_K, sv = base + C::OFF_V, sa = base + C::OFF_A;
-        const uint32_t id_qk = idesc_bf16(128, 128, false, false);
-        const uint32_t id_n = idesc_bf16(128, D, false, true);
-        bool ok = gwait(in_full, 0, abort, p);
-        if (ok) {
-            tc_fence_after();
-#pragma unroll
-            for (int b = 0; b < NB; ++b)
-#pragma unroll
-                for (int k = 0; k < 4; ++k)
-                    mma_ss_w(tb + C::TM_QK, sdesc_sw128(sq + b * BLK128, 16, 1024) + 2 * k,
-                             sdesc_sw128(sk + b * BLK128, 16, 1024) + 2 * k, id_qk, (b > 0 || k > 0) ? 1u : 0u);
-            mma_commit_w(s_full);
-            ok = gwait(m_ready, 0, abort, p);
-        }
-        if (ok) {
-            tc_fence_after();
-#pragma unroll
-            for (int part = 0; part < 2; ++part) {
-                // mA += Q' A_part: K = D (Q' column blocks), A_c rows K-steps of 16
-                const uint32_t ap = sa + part * NB * C::ST_BLK;
-#pragma unroll
-                for (int k = 0; k < 4 * NB; ++k)
-                    mma_ss_w(tb + C::TM_MA, sdesc_sw128(sq + (k >> 2) * BLK128, 16, 1024) + 2 * (k & 3),
-                             sdesc_sw128(ap, C::ST_BLK, 1024) + 128 * k, id_n, (part > 0 || k > 0) ? 1u : 0u);
-                // mI += Mq_part V: Mq's K-step k (keys 16k ..) at columns 32 (k/2) + 8 (k%2) (+16 for lo)
-#pragma unroll
-                for (int k = 0; k < 8; ++k)
-                    mma_ts_w(tb + C::TM_MI, tb + C::TM_QK + 32 * (k >> 1) + 8 * (k & 1) + 16 * part,
-                             sdesc_sw128(sv, BLK128, 1024) + 128 * k, id_n, (part > 0 || k > 0) ? 1u : 0u);
-            }
-            mma_commit_w(acc_full);
-        }
-        mma_commit_w(mma_done);
-        mbar_wait_drain(mma_done, 0);
-    } else {
-        const int q4 = warp & 3;
-        const int x = 32 * q4 + (tid & 31);
-        const uint32_t lanes = tb + ((uint32_t)(32 * q4) << 16);
-        const float eta = p.eta[h];
-        gpowers(pw, CG + 1, p.lam[h], x);
-        gbar128();
-        // A_c as bf16 hi + lo, [D rows][D columns] in NB column blocks
-        {
-            const float *Ac = p.dA + ((size_t)bh * p.nC + c) * D * D;
-            for (int u = x; u < D * D / 8; u += 128) {
-                const int r = u / (D / 8), col = 8 * (u % (D / 8));
-                const float4 a0 = *reinterpret_cast<const float4 *>(Ac + r * D + col);
-                const float4 a1 = *reinterpret_cast<const float4 *>(Ac + r * D + col + 4);
-                uint32_t hi[4], lo[4];
-                gsplit(a0.x, a0.y, hi[0], lo[0]);
-                gsplit(a0.z, a0.w, hi[1], lo[1]);
-                gsplit(a1.x, a1.y, hi[2], lo[2]);
-                gsplit(a1.z, a1.w, hi[3], lo[3]);
-                const uint32_t off = (col >> 6) * C::ST_BLK + sw128_offset(r, col & 63);
-                *reinterpret_cast<uint4 *>(sm + C::OFF_A + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-                *reinterpret_cast<uint4 *>(sm + C::OFF_A + NB * C::ST_BLK + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
-            }
-        }
-        bool ok = gwait(s_full, 0, abort, p);
-        if (ok) {
-            tc_fence_after();
-            const bool row_in = x < L;
-#pragma unroll 1
-            for (int jb = 0; jb < 4; ++jb) {
-                uint32_t qk[32];
-                tmem_ld32(lanes + C::TM_QK + 32 * jb, qk);
-                tmem_wait_ld();
-                uint32_t hi[16], lo[16];
-#pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    float v[2];
-#pragma unroll
-                    for (int u = 0; u < 2; ++u) {
-                        const int l = 32 * jb + 2 * e + u;
-                        v[u] = (row_in && l <= x) ? eta * pw[x - l] * __uint_as_float(qk[2 * e + u]) : 0.f;
-                    }
-                    gsplit(v[0], v[1], hi[e], lo[e]);
-                }
-                tmem_st16(lanes + C::TM_QK + 32 * jb, hi);
-                tmem_st16(lanes + C::TM_QK + 32 * jb + 16, lo);
-            }
-            tmem_wait_st();
-        }
-        fence_async_smem();
-        tc_fence_before();
-        mbar_arrive(m_ready);
-        // every lane takes part in the collective loads; rows past L write nothing
-        if (ok && gwait(acc_full, 0, abort, p)) {
-            tc_fence_after();
-            const float dec = pw[min(x + 1, CG + 1)];
-            float *dst = p.mrow + grow(sq, x < L ? qrow0 + x : 0, p.T, p.H, D);
-#pragma unroll
-            for (int c0 = 0; c0 < D; c0 += 32) {
-                uint32_t a[32], b[32];
-                tmem_ld32(lanes + C::TM_MA + c0, a);
-                tmem_ld32(lanes + C::TM_MI + c0, b);
-                tmem_wait_ld();
-                if (x < L) {
-                    float4 *d4 = reinterpret_cast<float4 *>(dst + c0);
-#pragma unroll
-                    for (int u = 0; u < 8; ++u)
-                        d4[u] = make_float4(fmaf(dec, __uint_as_float(a[4 * u]), __uint_as_float(b[4 * u])),
-                                            fmaf(dec, __uint_as_float(a[4 * u + 1]), __uint_as_float(b[4 * u + 1])),
-                                            fmaf(dec, __uint_as_float(a[4 * u + 2]), __uint_as_float(b[4 * u + 2])),
-                                            fmaf(dec, __uint_as_float(a[4 * u + 3]), __uint_as_float(b[4 * u + 3])));
-                }
-            }
-        }
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    if (warp == 1) tmem_dealloc(tb, C::COLS);
 }
 
 // ===========================================================================
@@ -778,25 +719,39 @@ bool gen_map_packed(CUtensorMap *m, const void *base, int total, int H, int D, i
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// [rows][D] bf16 -> 2D map, boxes of 64 columns x D rows, 128-byte swizzle
+// (the split chunk start states: D rows per part of each slot)
+bool gen_map_rows(CUtensorMap *m, const void *base, int64_t rows, int D) {
+    EncodeFn fn = reinterpret_cast<EncodeFn>(tensor_map_encoder());
+    if (!fn || rows < 1) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)D * 2};
+    cuuint32_t box[2] = {64, (cuuint32_t)D};
+    cuuint32_t es[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, es,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 size_t gal(size_t x) { return (x + 255) & ~size_t(255); }
 
 struct GenLayout {
-    size_t kc, vc, mrow, dA, total;
+    size_t kc, vc, mrow, dA, ab, total;
 };
 GenLayout gen_layout(const tc_prefill_desc &d, int64_t n_halo) {
     const int64_t BH = d.B * d.H, D = d.dk, Tc = n_halo + d.T;
-    const int64_t E = Tc > d.W ? Tc - d.W : 0, nC = (E + CG - 1) / CG;
-    const bool l1 = (d.flags & TC_PREFILL_L1_ONLY) != 0, state = (d.flags & TC_PREFILL_STATE_ONLY) != 0;
+    const int64_t nC = (d.T + CG - 1) / CG;  // one chunk per block of 128 new rows
+    const bool l1 = (d.flags & TC_PREFILL_L1_ONLY) != 0;
     const bool delta = (d.flags & TC_PREFILL_DELTA_RULE) != 0;
     GenLayout L;
     L.kc = 0;
     const size_t comb = n_halo > 0 ? gal((size_t)(BH * Tc * D) * 2) : 0;
     L.vc = L.kc + comb;
-    L.mrow = L.vc + comb;
-    const size_t mrow = (!l1 && !state && !delta) ? gal((size_t)(BH * d.T * D) * sizeof(float)) : 0;
-    L.dA = L.mrow + mrow;
+    L.mrow = L.vc + comb;  // (unused: the reads happen inside the window kernel)
+    L.dA = L.mrow;
     const size_t dA = (!l1 && !delta) ? gal((size_t)(BH * nC * D * D) * sizeof(float)) : 0;
-    L.total = L.dA + dA;
+    L.ab = L.dA + dA;  // the split start states: the same bytes again
+    L.total = L.ab + dA;
     return L;
 }
 
@@ -828,7 +783,7 @@ cudaError_t launch_general_t(const PrefillParams &pp, const float *mrow_in, cuda
     p.W = (int)(pp.W < p.Tc + 1 ? pp.W : p.Tc + 1);  // a window past the sequence changes nothing
     p.H = (int)pp.H;
     p.E = p.Tc > p.W ? p.Tc - p.W : 0;
-    p.nC = (p.E + CG - 1) / CG;
+    p.nC = (p.T + CG - 1) / CG;  // chunk slots per row: one per block of 128 new rows
     p.lam = pp.lam;
     p.eta = pp.eta;
     p.g = pp.g;
@@ -853,20 +808,22 @@ cudaError_t launch_general_t(const PrefillParams &pp, const float *mrow_in, cuda
     }
     const bool l2 = !pp.l1_only && !pp.delta_rule;
     p.dA = l2 ? reinterpret_cast<float *>(ws + Lo.dA) : nullptr;
-    p.mrow = pp.delta_rule ? const_cast<float *>(mrow_in)
-                           : (l2 && !pp.state_only && p.nC > 0 ? reinterpret_cast<float *>(ws + Lo.mrow) : nullptr);
+    p.ab = l2 ? reinterpret_cast<__nv_bfloat16 *>(ws + Lo.ab) : nullptr;
+    p.mrow = pp.delta_rule ? const_cast<float *>(mrow_in) : nullptr;
     const bool queries = !pp.state_only && p.T > 0;
-    CUtensorMap mk128, mv128, mq128, mk64, mv64;
+    CUtensorMap mk128, mq128, mk64, mv64;
     auto map = [&](CUtensorMap *m, const void *base, int rows, int box) {
         return packed ? gen_map_packed(m, base, p.total, p.H, D, box) : gen_map(m, base, rows, BH, D, box);
     };
-    if ((queries || (l2 && p.nC > 0)) &&
-        (!map(&mk128, p.k, p.Tc, 128) || !map(&mv128, p.v, p.Tc, 128) || !map(&mk64, p.k, p.Tc, 64) ||
-         !map(&mv64, p.v, p.Tc, 64)))
+    if ((queries || (l2 && p.E > 0)) &&
+        (!map(&mk128, p.k, p.Tc, 128) || !map(&mk64, p.k, p.Tc, 64) || !map(&mv64, p.v, p.Tc, 64)))
         return cudaErrorInvalidValue;
     if (queries && !map(&mq128, p.q, p.T, 128)) return cudaErrorInvalidValue;
+    CUtensorMap mab = mq128;  // any valid map when the memory is off (not read then)
+    if (queries && l2 && p.nC > 0 && !gen_map_rows(&mab, p.ab, (int64_t)BH * p.nC * 2 * D, D))
+        return cudaErrorInvalidValue;
     if (l2) {
-        if (p.nC > 0) {
+        if (p.E > 0) {
             e = cudaFuncSetAttribute(gen_sums_kernel<NB>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SUM_SMEM);
             if (e != cudaSuccess) return e;
             const int cpb = NB == 1 ? 2 : 1;
@@ -876,20 +833,13 @@ cudaError_t launch_general_t(const PrefillParams &pp, const float *mrow_in, cuda
         }
         gen_scan_kernel<<<dim3((unsigned)((D * D + 255) / 256), (unsigned)BH), 256, 0, s>>>(p, D);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
-        if (queries && p.nC > 0) {
-            using RC = ReadCfg<NB>;
-            e = cudaFuncSetAttribute(gen_read_kernel<NB>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)RC::SMEM);
-            if (e != cudaSuccess) return e;
-            gen_read_kernel<NB><<<dim3((unsigned)p.nC, (unsigned)BH), kGThreads, RC::SMEM, s>>>(mq128, mk128, mv128, p);
-            if ((e = cudaGetLastError()) != cudaSuccess) return e;
-        }
     }
     if (queries) {
         using WC = WinCfg<NB>;
         e = cudaFuncSetAttribute(gen_window_kernel<NB>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)WC::SMEM);
         if (e != cudaSuccess) return e;
         gen_window_kernel<NB><<<dim3((unsigned)((p.T + CG - 1) / CG), (unsigned)BH), kGThreads, WC::SMEM, s>>>(
-            mq128, mk64, mv64, p);
+            mq128, mk64, mv64, mab, p);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     return cudaSuccess;
@@ -908,8 +858,10 @@ bool general_supported(const tc_prefill_desc &d, int64_t n_halo) {
     if (d.flags & TC_PREFILL_CHUNK_MEAN) return false;
     if ((d.flags & TC_PREFILL_DELTA_RULE) && (n_halo != 0 || (d.flags & (TC_PREFILL_STATE_ONLY | TC_PREFILL_L1_ONLY))))
         return false;
-    // shapes only: a call without a device gets TC_ERR_NO_DEVICE, not UNSUPPORTED
-    return d.T + n_halo < (int64_t(1) << 30) && d.B * d.H <= 65535;
+    // shapes only: a call without a device gets TC_ERR_NO_DEVICE, not UNSUPPORTED;
+    // the split start states are addressed by 32-bit copy coordinates
+    const int64_t slots = d.B * d.H * ((d.T + CG - 1) / CG);
+    return d.T + n_halo < (int64_t(1) << 30) && d.B * d.H <= 65535 && slots * 2 * d.dk < (int64_t(1) << 31);
 }
 
 size_t general_workspace_bytes(const tc_prefill_desc &d, int64_t n_halo) { return gen_layout(d, n_halo).total; }
@@ -920,8 +872,8 @@ int general_launch_count(const tc_prefill_desc &d, int64_t n_halo) {
     const bool delta = (d.flags & TC_PREFILL_DELTA_RULE) != 0;
     const bool queries = !state && d.T > 0;
     int n = n_halo > 0 ? 2 : 0;
-    if (!l1 && !delta) n += (E > 0 ? 1 : 0) + 1 + (queries && E > 0 ? 1 : 0);
-    return n + (queries ? 1 : 0);
+    if (!l1 && !delta) n += (E > 0 ? 1 : 0) + 1;  // sums, scan
+    return n + (queries ? 1 : 0);                  // window (with the reads)
 }
 
 cudaError_t launch_prefill_general(const PrefillParams &p, const float *mrow, cudaStream_t s) {

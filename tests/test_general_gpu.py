@@ -5,7 +5,7 @@ against the float64 oracle ("Tensor Cache: Eviction-conditioned Associative
 Memory for Transformers", §3.1 eq. (1) and §3.2 Fig. 2).  Tolerances are the
 bf16 ones of the other parity tests: ||y - ref|| / ||ref|| <= 1e-2 and
 ||A - ref|| / ||ref|| <= 1e-3.  Each case also checks the launch count of
-the general path (combine copies, sums, scan, reads, window), so a silent
+the general path (combine copies, sums, scan, window with the reads), so a silent
 switch to the SIMT kernels fails here."""
 import numpy as np
 import pytest
@@ -39,8 +39,8 @@ def general_launches(T, W, n_halo=0, l1_only=False, state_only=False):
     queries = not state_only and T > 0
     n = 2 if n_halo > 0 else 0
     if not l1_only:
-        n += (1 if E > 0 else 0) + 1 + (1 if queries and E > 0 else 0)
-    return n + (1 if queries else 0)
+        n += (1 if E > 0 else 0) + 1  # sums, scan
+    return n + (1 if queries else 0)  # window (with the reads)
 
 
 CASES = [
