@@ -47,9 +47,12 @@ HEADLINE = "lm_prefill_bf16"
 # kernels; they must be re-measured (or set to None) whenever a kernel changes.
 #   prefill_main_kernel: one LM launch, 159.2 MB read + 31.9 MB written
 #     (profiles/prefill_main_kernel_lm_prefill_bf16.md)
+#   gen_window_kernel: None until captured at the LM shape
 #   decode_kernel: the B = 32 capture scaled by heads to the 256 x 32 launch,
 #     (1.1417 + 0.0172) GB x 8 (profiles/decode_kernel_b32_w2048_d128.md)
-NCU_TRAFFIC_BYTES = {"prefill_main_kernel": 1.911e8, "decode_kernel": 9.27e9}
+NCU_TRAFFIC_BYTES = {"prefill_main_kernel": 1.911e8, "gen_window_kernel": None, "decode_kernel": 9.27e9}
+# the kernel that dominates one prefill call on each tensor-core path
+PATH_KERNEL = {"fused": "prefill_main_kernel", "general": "gen_window_kernel"}
 METRIC = "prefill tokens/s & decode tok/s per B200; % of TC/HBM roofline"
 UNIT = "tokens/s"
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -93,6 +96,37 @@ def prefill_executed_flops(B, H, T, W, tile=128, d=64):
         if lead:
             l2 += mma_tile + tile * d * d * 2 + mma_tile  # P'V, Q S(n0), [hi; lo] K^T V
     return l1 * B * H, l2 * B * H
+
+
+def general_executed_flops(B, H, T, W, d=64, l1_only=False):
+    """Tensor-core FLOPs the general path issues for one call (bf16, no halo):
+    per block of 128 query rows, Q K^T and P V on every 64-key tile from the
+    first key it reads to the block's last row (masked parts included), P'V on
+    the tiles that hold the block's chunk of evictions and Q A_b (hi + lo)
+    after them; per-chunk sums: one 128 x 128 x 128 product pair (hi + lo)
+    per CTA (two chunks of d = 64, or one of d = 128)."""
+    G, X = 128, 64
+    E = max(0, T - W)
+    nC = (T + G - 1) // G
+    win = mem = 0
+    for b in range(nC):
+        tau0 = G * b
+        a = G * b - W
+        e_lo = max(0, a)
+        e_hi = max(e_lo, min(E, a + G))
+        reads = not l1_only and e_hi > e_lo
+        lo = e_lo if reads else max(0, tau0 - W + 1)
+        hi = min(T - 1, tau0 + G - 1)
+        xs = lo & ~(X - 1)
+        n_tiles = (hi - xs) // X + 1
+        win += n_tiles * 2 * (2 * G * X * d)
+        if reads:
+            n_read = sum(1 for n in range(n_tiles) if xs + X * n < e_hi and xs + X * n + X > e_lo)
+            mem += n_read * 2 * G * X * d + 2 * (2 * G * d * d)
+    if not l1_only and E > 0:
+        ctas = (nC + 1) // 2 if d == 64 else nC
+        mem += ctas * 2 * (2 * G * G * G)
+    return win * B * H, mem * B * H
 
 
 def decode_bytes(B, H, W, dk, dv, esz=2):
@@ -702,14 +736,18 @@ def main():
         mean_ms = statistics.mean(head["per_step_ms"])
         achieved_tflops = (l1f + l2f) / (mean_ms * 1e-3) / 1e12
         peak_tf = float(peaks["bf16_tflops"])
+        path = tc.prefill_path_for(tc.make_prefill_desc(B, H, T, dk, dv, x.W, x.C, tc.TC_BF16))
+        kern = PATH_KERNEL[path]
         roofline = {"bound": "tensor", "achieved": achieved_tflops, "peak": peak_tf,
                     "unit": "TFLOP/s", "frac": achieved_tflops / peak_tf,
-                    "traffic": NCU_TRAFFIC_BYTES["prefill_main_kernel"],
-                    "traffic_kernel": "prefill_main_kernel (ncu, one launch)",
+                    "traffic": NCU_TRAFFIC_BYTES[kern],
+                    "traffic_kernel": f"{kern} (ncu, one launch)",
                     "peak_source": f"{peak_src} bf16 burst",
-                    "kernel": "tc_prefill (all launches of one call)",
+                    "kernel": f"tc_prefill (all launches of one call, {path} path)",
+                    "path": path,
                     "algorithmic_flops_per_launch": l1f + l2f}
-        e1, e2 = prefill_executed_flops(B, H, T, x.W)
+        executed = prefill_executed_flops if path == "fused" else general_executed_flops
+        e1, e2 = executed(B, H, T, x.W)
         roofline["executed_flops_per_launch"] = e1 + e2
         roofline["executed_tflops"] = (e1 + e2) / (mean_ms * 1e-3) / 1e12
         extras = {}
@@ -735,7 +773,10 @@ def main():
                 "frac_of_bf16_peak": (f1 + f2) / (t_lp * 1e-3) / 1e12 / peak_tf,
                 "l1_only_ms": t_lp1, "l2_overhead_ratio": t_lp / t_lp1 - 1.0,
                 "algorithmic_floor": f2 / f1,
-                "executed_tflops": sum(prefill_executed_flops(Bl, Hl, Tl, xl.W)) / (t_lp * 1e-3) / 1e12,
+                "path": tc.prefill_path_for(tc.make_prefill_desc(Bl, Hl, Tl, dl, dl, xl.W, xl.C, tc.TC_BF16)),
+                "executed_tflops": sum((prefill_executed_flops if tc.prefill_path_for(
+                    tc.make_prefill_desc(Bl, Hl, Tl, dl, dl, xl.W, xl.C, tc.TC_BF16)) == "fused"
+                    else general_executed_flops)(Bl, Hl, Tl, xl.W)) / (t_lp * 1e-3) / 1e12,
                 "state_size": state_size_ratio(Tl, xl.W, dl)}
             del lp, lp1
             dec = time_decode(tc, dev, world, clocks=clocks)

@@ -285,7 +285,10 @@ TC_API tc_status tc_prefill_host(const tc_prefill_desc *desc, const void *q, con
  * space is a fixed array inside the library (TC_NO_ALLOC_SCRATCH_BYTES,
  * resident on every GPU that loads the library until the process exits).
  * Returns TC_ERR_WORKSPACE, enqueuing nothing, when desc would need more
- * scratch than that (tc_prefill_workspace_size(desc) tells how much).
+ * scratch than that (tc_prefill_workspace_size(desc) tells how much).  Under
+ * TC_PATH_AUTO a call that both tensor-core paths take runs on the fused
+ * kernel when only its scratch fits (the general path keeps per-chunk
+ * states: 100 MiB at B = 8, H = 12, T = 4096, d = 64).
  * The first call on each device looks up the array's device address with
  * that device current; make that first call before any stream capture.  The
  * address is cached until a call fails with TC_ERR_CUDA; after a
@@ -379,6 +382,37 @@ TC_API tc_status tc_decode_step_host(tc_decode_state *state, const void *q_t, co
  * microsecond makes the first wait of a real call run out).  Not thread-safe
  * against concurrent calls. */
 TC_API void tc_set_wait_limit_ns(uint64_t ns);
+
+/* Which tensor-core prefill runs a call that both can take: bf16, d_k = d_v
+ * = 64, W a multiple of 128 and t0 = 0 or t0 >= W (plain, L1-only and
+ * variable-length calls, and the window part of a delta-rule call).
+ *   TC_PATH_AUTO     the faster of the two on B200 (the default): the
+ *                    general path for fixed-length calls, the fused kernel
+ *                    for variable-length calls
+ *   TC_PATH_FUSED    the fused kernel: span summaries, their prefix, and one
+ *                    kernel that carries the memory's state on chip
+ *   TC_PATH_GENERAL  the general path: per-chunk sums, a chunk scan, and the
+ *                    window kernel that also computes the memory's reads
+ * Calls that only one path takes run there whatever the setting.  Both give
+ * results within the same tolerances of the definition (float32 state, bf16
+ * P); they are not bit-identical to each other.  Process-wide; applies to
+ * calls, workspace-size and launch-count queries made after it, so query the
+ * workspace after choosing.  Not thread-safe against concurrent calls.
+ * Returns TC_ERR_INVALID_ARG (and keeps the setting) for any other value. */
+#define TC_PATH_AUTO 0
+#define TC_PATH_FUSED 1
+#define TC_PATH_GENERAL 2
+TC_API tc_status tc_set_prefill_path(int path);
+
+/* The current setting of tc_set_prefill_path. */
+TC_API int tc_get_prefill_path(void);
+
+/* The path (TC_PATH_FUSED or TC_PATH_GENERAL) a fixed-length call described
+ * by desc would take now, continuing at t0 (0 for tc_prefill; the delta
+ * rule's window part counts); -1 when desc is NULL
+ * or invalid or neither tensor-core path takes it (the float32 SIMT path
+ * then runs).  Needs no device. */
+TC_API int tc_prefill_path_for(const tc_prefill_desc *desc, int64_t t0);
 
 /* Synchronizes stream, then returns and clears the device status word of the
  * current device: TC_OK, TC_ERR_DEVICE_BOUNDS or TC_ERR_DEVICE_TIMEOUT. */

@@ -43,6 +43,7 @@ TC_PREFILL_STATE_ONLY = 2
 TC_PREFILL_DELTA_RULE = 4
 TC_PREFILL_CHUNK_MEAN = 8
 TC_WRITE_OUTER, TC_WRITE_DELTA = 0, 1
+TC_PATH_AUTO, TC_PATH_FUSED, TC_PATH_GENERAL = 0, 1, 2
 
 # Exported C symbols declared in include/tc.h.
 EXPORTED = ("tc_prefill_workspace_size", "tc_prefill", "tc_prefill_launch_count", "tc_prefill_host_workspace_size",
@@ -51,7 +52,8 @@ EXPORTED = ("tc_prefill_workspace_size", "tc_prefill", "tc_prefill_launch_count"
             "tc_prefill_no_alloc", "tc_prefill_from_state", "tc_prefill_from_state_workspace_size",
             "tc_state_fold", "tc_decode_step_ragged", "tc_backward", "tc_backward_workspace_size",
             "tc_set_wait_limit_ns", "tc_prefill_varlen", "tc_prefill_varlen_workspace_size",
-            "tc_backward_launch_count")
+            "tc_backward_launch_count", "tc_set_prefill_path", "tc_get_prefill_path",
+            "tc_prefill_path_for")
 
 
 class PrefillDesc(ctypes.Structure):
@@ -116,6 +118,12 @@ _lib.tc_version.argtypes = []
 _lib.tc_version.restype = ctypes.c_char_p
 _lib.tc_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
 _lib.tc_set_wait_limit_ns.restype = None
+_lib.tc_set_prefill_path.argtypes = [_int]
+_lib.tc_set_prefill_path.restype = _int
+_lib.tc_get_prefill_path.argtypes = []
+_lib.tc_get_prefill_path.restype = _int
+_lib.tc_prefill_path_for.argtypes = [_PD, ctypes.c_int64]
+_lib.tc_prefill_path_for.restype = _int
 
 SIZE_ERROR = ctypes.c_size_t(-1).value
 
@@ -436,6 +444,47 @@ def prefill_launch_count(desc: PrefillDesc) -> int:
     if n < 0:
         raise TCError(1, "tc_prefill_launch_count")
     return int(n)
+
+
+_PATHS = {"auto": TC_PATH_AUTO, "fused": TC_PATH_FUSED, "general": TC_PATH_GENERAL}
+
+
+def set_prefill_path(path) -> None:
+    """tc_set_prefill_path: "auto" (default), "fused" or "general" (or the
+    TC_PATH_* value), for calls both tensor-core paths can take.  Process-wide."""
+    code = _PATHS.get(path, path) if isinstance(path, str) else int(path)
+    if not isinstance(code, int):
+        raise TCError(1, "tc_set_prefill_path")
+    _check(_lib.tc_set_prefill_path(code), "tc_set_prefill_path")
+
+
+def get_prefill_path() -> str:
+    """The current tc_set_prefill_path setting, by name."""
+    code = int(_lib.tc_get_prefill_path())
+    return {v: k for k, v in _PATHS.items()}[code]
+
+
+class prefill_path:
+    """Context manager: tc_set_prefill_path(path) inside, the previous setting after."""
+
+    def __init__(self, path):
+        self.path = path
+
+    def __enter__(self):
+        self.prev = get_prefill_path()
+        set_prefill_path(self.path)
+        return self
+
+    def __exit__(self, *exc):
+        set_prefill_path(self.prev)
+        return False
+
+
+def prefill_path_for(desc: PrefillDesc, t0: int = 0):
+    """tc_prefill_path_for: "fused" or "general", the tensor-core path a call
+    described by desc (continuing at t0) would take now; None when neither takes it."""
+    code = int(_lib.tc_prefill_path_for(ctypes.byref(desc), ctypes.c_int64(int(t0))))
+    return None if code < 0 else {TC_PATH_FUSED: "fused", TC_PATH_GENERAL: "general"}[code]
 
 
 NO_ALLOC_SCRATCH_BYTES = 16 << 20

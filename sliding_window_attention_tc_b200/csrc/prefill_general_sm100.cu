@@ -125,6 +125,103 @@ __device__ __forceinline__ void gpowers(float *pw, int n_max, float lam, int x) 
     for (int n = x; n <= n_max; n += 128) pw[n] = n == 0 ? 1.f : (float)exp2((double)n * l2l);
 }
 __device__ __forceinline__ void gbar128() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+// lam^n (n >= 0) by binary powering in double, rounded once to float
+__device__ __forceinline__ float gpow(float lam, int n) {
+    double r = 1.0, b = (double)lam;
+    for (; n > 0; n >>= 1) {
+        if (n & 1) r *= b;
+        b *= b;
+    }
+    return (float)r;
+}
+
+// How the window 0 <= tau - j < W cuts a 64-key tile, for all 32 rows of a
+// warp at once: every column inside (no per-column masks), none inside (P =
+// 0, no exponentials), or masked column by column.
+enum { kTileFull = 0, kTileMasked = 1, kTileNone = 2 };
+// O is rescaled only when a row's max grows by more than 2^8 over the max its
+// P values are taken against, so P <= 2^8 (exact in bf16's float32 range)
+// and most tiles skip the rescale and its wait for the previous P V.
+constexpr float kRescaleG = 8.f;
+// eta lam^d table for the reads' weights, zero-padded: entry 128 + d holds
+// eta lam^d for 0 <= d < 128 and 0 for d < 0 (and for d >= 128, which only
+// the columns before the chunk reach, and those are masked)
+constexpr int kEpw = 384;
+
+__device__ __forceinline__ int tile_kind(int base, uint32_t wlim) {
+    // column c is in the window iff 0 <= base - c < wlim, c in [0, GX)
+    if (__all_sync(0xffffffffu, wlim != 0u && base >= GX - 1 && base < (int)wlim)) return kTileFull;
+    if (__all_sync(0xffffffffu, wlim == 0u || base < 0 || base - (GX - 1) >= (int)wlim)) return kTileNone;
+    return kTileMasked;
+}
+
+// Row max of the raw scores over the window columns (-inf if none), as a tree.
+template <bool MASK>
+__device__ __forceinline__ float tile_max(const float (&s)[GX], int base, uint32_t wlim) {
+    float m[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) m[i] = -INFINITY;
+#pragma unroll
+    for (int c = 0; c < GX; c += 2) {
+        const float a = (!MASK || (uint32_t)(base - c) < wlim) ? s[c] : -INFINITY;
+        const float b = (!MASK || (uint32_t)(base - c - 1) < wlim) ? s[c + 1] : -INFINITY;
+        m[(c >> 1) & 7] = fmax3(m[(c >> 1) & 7], a, b);
+    }
+    return fmax3(fmax3(m[0], m[1], m[2]), fmax3(m[3], m[4], m[5]), fmaxf(m[6], m[7]));
+}
+
+// P = exp2(s sl2 - m) on the window columns (0 elsewhere), bf16 pairs into
+// the P columns of the score buffer (keys 32 h .. 32 h + 31 at column 32 h);
+// returns the row sum of P.
+template <bool MASK>
+__device__ __forceinline__ float tile_p(const float (&s)[GX], int base, uint32_t wlim, float sl2, float m,
+                                        uint32_t sbuf) {
+    uint64_t acc[2] = {0ull, 0ull};  // (0.f, 0.f) pairs
+    const uint64_t sl2p = f2pack(sl2, sl2), negm = f2pack(-m, -m);
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+            const int c = 32 * h + 2 * e;
+            float x0, x1;
+            ffma2(x0, x1, s[c], s[c + 1], sl2p, negm);
+            if (MASK) {
+                x0 = (uint32_t)(base - c) < wlim ? x0 : -INFINITY;
+                x1 = (uint32_t)(base - c - 1) < wlim ? x1 : -INFINITY;
+            }
+            const float p0 = gex2(x0), p1 = gex2(x1);
+            fadd2_acc(acc[e & 1], p0, p1);
+            pk[e] = pack_bf16(p0, p1);
+        }
+        tmem_st16(sbuf + 32 * h, pk);
+    }
+    float a0, a1, b0, b1;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(a0), "=f"(a1) : "l"(acc[0]));
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(b0), "=f"(b1) : "l"(acc[1]));
+    return (a0 + b0) + (a1 + b1);
+}
+
+// P' = eta lam^(off - c) s for off - c >= 0 (w[-c] from the padded table) and
+// c >= cmin, bf16 pairs into the P' columns (keys 32 h .. at column 32 h + 16).
+template <bool CMIN>
+__device__ __forceinline__ void tile_plin(const float (&s)[GX], const float *w, int cmin, uint32_t sbuf) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+            const int c = 32 * h + 2 * e;
+            float w0 = w[-c], w1 = w[-c - 1];
+            if (CMIN) {
+                w0 = c >= cmin ? w0 : 0.f;
+                w1 = c + 1 >= cmin ? w1 : 0.f;
+            }
+            pk[e] = pack_bf16(w0 * s[c], w1 * s[c + 1]);
+        }
+        tmem_st16(sbuf + 32 * h + 16, pk);
+    }
+}
 
 // rows [row, row + rows) of a [.][D] map as NB column blocks of 64: maps
 // (D, rows, BH) for fixed lengths, (D, H, total) for packed sequences
@@ -169,7 +266,8 @@ struct WinCfg {
     static constexpr uint32_t OFF_X = Q_B;         // NS x (K tile, V tile)
     static constexpr uint32_t OFF_A = OFF_X + NS * 2 * X_B;  // A_b hi: NB blocks, lo: NB blocks
     static constexpr uint32_t OFF_PW = OFF_A + 2 * NB * ST_BLK;  // lam^n, n = 0 .. 128
-    static constexpr uint32_t OFF_BAR = OFF_PW + 136 * 4;
+    static constexpr uint32_t OFF_EPW = OFF_PW + 136 * 4;         // padded eta lam^d table
+    static constexpr uint32_t OFF_BAR = OFF_EPW + kEpw * 4;
     static constexpr uint32_t SMEM = OFF_BAR + 256 + 1024;  // (9 + 2 NS) barriers, TMEM address, abort flag
     // two 64-column score buffers, O, the reads' accumulator (P' V, then + Q A_b
     // lands in the score buffers' columns after the last tile)
@@ -192,6 +290,7 @@ __global__ void __launch_bounds__(kGThreads, NB == 1 ? 2 : 1)
     uint32_t *tmem_base = reinterpret_cast<uint32_t *>(a_ready + 1);
     volatile int *abort = reinterpret_cast<volatile int *>(tmem_base + 1);
     float *pw = reinterpret_cast<float *>(sm + C::OFF_PW);
+    float *epw = reinterpret_cast<float *>(sm + C::OFF_EPW);
 
     const int tid = threadIdx.x, warp = tid >> 5;
     const GSeq sq = gseq(p, blockIdx.y);
@@ -239,17 +338,6 @@ __global__ void __launch_bounds__(kGThreads, NB == 1 ? 2 : 1)
         if (tid == 0) {
             mbar_expect_tx(q_full, C::Q_B);
             tma_rows_nb<NB>(sm + C::OFF_Q, &tq, q_full, t0, sq, BLK128);
-            if (reads) {
-                // A_b hi, lo: rows (slot * 2 + part) * D of the [.][D] map, NB column blocks
-                const int slot = sq.bh * p.nC + blockIdx.x;
-                mbar_expect_tx(a_ready, 2 * NB * C::ST_BLK);
-#pragma unroll
-                for (int part = 0; part < 2; ++part)
-#pragma unroll
-                    for (int b = 0; b < NB; ++b)
-                        tma_load_2d(sm + C::OFF_A + (part * NB + b) * C::ST_BLK, &tab, a_ready, 64 * b,
-                                    (slot * 2 + part) * D);
-            }
             int n = 0;
             for (; n < N; ++n) {
                 const int s = n % NS;
@@ -258,6 +346,21 @@ __global__ void __launch_bounds__(kGThreads, NB == 1 ? 2 : 1)
                 mbar_expect_tx(&x_full[s], 2 * C::X_B);
                 tma_rows_nb<NB>(dst, &tk, &x_full[s], xs + GX * n, sq, BLK64);
                 tma_rows_nb<NB>(dst + C::X_B, &tv, &x_full[s], xs + GX * n, sq, BLK64);
+            }
+            if (reads) {
+                // A_b is the scan's output, and this kernel may start while the scan
+                // still runs (it is only needed after the last key tile): wait for
+                // the scan's grid here, then copy A_b hi, lo (rows (slot * 2 + part)
+                // * D of the [.][D] map, NB column blocks)
+                griddep_wait();
+                const int slot = sq.bh * p.nC + blockIdx.x;
+                mbar_expect_tx(a_ready, 2 * NB * C::ST_BLK);
+#pragma unroll
+                for (int part = 0; part < 2; ++part)
+#pragma unroll
+                    for (int b = 0; b < NB; ++b)
+                        tma_load_2d(sm + C::OFF_A + (part * NB + b) * C::ST_BLK, &tab, a_ready, 64 * b,
+                                    (slot * 2 + part) * D);
             }
             mbar_wait_drain(q_full, 0);
             if (reads) mbar_wait_drain(a_ready, 0);
@@ -335,16 +438,18 @@ __global__ void __launch_bounds__(kGThreads, NB == 1 ? 2 : 1)
         const int t = t0 + r, tau = tau0 + r;
         const uint32_t wlim = t < sq.T ? (uint32_t)p.W : 0u;
         const float sl2 = kLog2eG * rsqrtf((float)D);
-        float eta = 0.f;
         if (reads) {
-            // lam^n for the reads' weights (A_b arrives by copy)
+            // lam^n for the reads' weights (A_b arrives by copy), then the
+            // padded eta lam^d table
             gpowers(pw, CG, p.lam[sq.h], x);
-            eta = p.eta[sq.h];
+            const float eta = p.eta[sq.h];
             gbar128();  // pw complete
+            for (int i = x; i < kEpw; i += 128) epw[i] = (i >= 128 && i < 128 + CG) ? eta * pw[i - 128] : 0.f;
+            gbar128();  // epw complete
         }
         // the reads of row r cover evictions e_lo .. tau - W (none when tau < W or t >= T)
         const int rd_hi = (reads && t < sq.T) ? tau - p.W : -1;
-        float m_run = -INFINITY, l_run = 0.f;
+        float m_used = -INFINITY, l_run = 0.f;  // max P is taken against (log2 units), row sum
         bool ok = true;
         for (int n = 0; n < N; ++n) {
             if (!(ok = gwait(&s_full[n & 1], (n >> 1) & 1, abort, p))) break;
@@ -352,26 +457,30 @@ __global__ void __launch_bounds__(kGThreads, NB == 1 ? 2 : 1)
             const uint32_t sbuf = lanes + C::TM_S + 64 * (n & 1);
             const int j0 = xs + GX * n;
             const int base = tau - j0;  // tau - j = base - c
-            const bool tr = tile_reads(n);
-            // the row max over both 32-column halves, then the exponentials (and
-            // the reads' weights) from a second read of the scores
-            float mx = -INFINITY;
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                uint32_t sr[32];
-                tmem_ld32(sbuf + 32 * h, sr);
+            float s[GX];
+            {
+                uint32_t ra[32], rb[32];
+                tmem_ld32(sbuf, ra);
+                tmem_ld32(sbuf + 32, rb);
                 tmem_wait_ld();
 #pragma unroll
-                for (int c = 0; c < 32; ++c)
-                    if ((uint32_t)(base - (32 * h + c)) < wlim) mx = fmaxf(mx, __uint_as_float(sr[c]));
+                for (int c = 0; c < 32; ++c) {
+                    s[c] = __uint_as_float(ra[c]);
+                    s[32 + c] = __uint_as_float(rb[c]);
+                }
             }
-            mx *= sl2;
-            const float m_new = fmaxf(m_run, mx);
-            const float corr = m_new == -INFINITY ? 1.f : gex2(m_run - m_new);
+            const int kind = tile_kind(base, wlim);
+            const float mt = (kind == kTileNone ? -INFINITY
+                              : kind == kTileFull ? tile_max<false>(s, base, wlim)
+                                                  : tile_max<true>(s, base, wlim)) * sl2;  // sl2 > 0
+            const bool raise = mt > m_used + kRescaleG;
+            // O holds earlier P V products only once some P was nonzero
+            const bool resc = raise && m_used != -INFINITY;
+            const float fo = resc ? gex2(m_used - mt) : 1.f;
             // rescale O once the previous P V is complete (its commit is the
             // (n-1)-th completion of o_done; the n-th cannot come before this
             // tile's P, so the parity names it unambiguously)
-            if (n > 0 && __any_sync(0xffffffffu, corr != 1.f)) {
+            if (__any_sync(0xffffffffu, resc)) {
                 if (!(ok = gwait(o_done, (n - 1) & 1, abort, p))) break;
                 tc_fence_after();
 #pragma unroll
@@ -380,42 +489,32 @@ __global__ void __launch_bounds__(kGThreads, NB == 1 ? 2 : 1)
                     tmem_ld32(lanes + C::TM_O + c0, o);
                     tmem_wait_ld();
 #pragma unroll
-                    for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * corr);
+                    for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * fo);
                     tmem_st32(lanes + C::TM_O + c0, o);
                 }
             }
-            float sum = 0.f;
-            const float neg_m = m_new == -INFINITY ? 0.f : -m_new;
+            l_run *= fo;
+            if (raise) m_used = mt;
+            if (kind == kTileNone) {
+                uint32_t z[16];
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                uint32_t sr[32];
-                tmem_ld32(sbuf + 32 * h, sr);
-                tmem_wait_ld();
-                uint32_t pk[16];
-#pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    const int c = 32 * h + 2 * e;
-                    const float a = (uint32_t)(base - c) < wlim ? gex2(fmaf(__uint_as_float(sr[2 * e]), sl2, neg_m)) : 0.f;
-                    const float b = (uint32_t)(base - c - 1) < wlim ? gex2(fmaf(__uint_as_float(sr[2 * e + 1]), sl2, neg_m)) : 0.f;
-                    sum += a + b;
-                    pk[e] = pack_bf16(a, b);
-                }
-                tmem_st16(sbuf + 32 * h, pk);
-                if (tr) {
-                    // P' = eta lam^(tau-W-j) s for e_lo <= j <= tau - W
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        const int j = j0 + 32 * h + 2 * e;
-                        const int d0 = rd_hi - j, d1 = d0 - 1;
-                        const float a = (d0 >= 0 && j >= e_lo) ? eta * pw[min(d0, CG)] * __uint_as_float(sr[2 * e]) : 0.f;
-                        const float b = (d1 >= 0 && j + 1 >= e_lo) ? eta * pw[min(d1, CG)] * __uint_as_float(sr[2 * e + 1]) : 0.f;
-                        pk[e] = pack_bf16(a, b);
-                    }
-                    tmem_st16(sbuf + 32 * h + 16, pk);
-                }
+                for (int e = 0; e < 16; ++e) z[e] = 0u;
+                tmem_st16(sbuf, z);
+                tmem_st16(sbuf + 32, z);
+            } else {
+                const float m = m_used == -INFINITY ? 0.f : m_used;
+                l_run += kind == kTileFull ? tile_p<false>(s, base, wlim, sl2, m, sbuf)
+                                           : tile_p<true>(s, base, wlim, sl2, m, sbuf);
             }
-            l_run = fmaf(l_run, corr, sum);
-            m_run = m_new;
+            if (tile_reads(n)) {
+                // P' = eta lam^(tau-W-j) s for e_lo <= j <= tau - W: d = rd_hi - j0 - c,
+                // clamped so that every table index stays in [1, kEpw)
+                const int off = max(rd_hi - j0, -GX);
+                const int cmin = e_lo - j0;  // > 0 only in the first tile
+                const float *w = epw + 128 + off;
+                if (cmin > 0) tile_plin<true>(s, w, cmin, sbuf);
+                else tile_plin<false>(s, w, cmin, sbuf);
+            }
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
@@ -479,8 +578,7 @@ __global__ void __launch_bounds__(kGThreads, NB == 1 ? 2 : 1)
 // (D = 64) or all of it (D = 128) are the increments.
 constexpr uint32_t SUM_OFF_A = 0;                  // 2 blocks (TMA)
 constexpr uint32_t SUM_OFF_B = 2 * BLK128;         // hi: 2 blocks, lo: 2 blocks
-constexpr uint32_t SUM_OFF_PW = SUM_OFF_B + 4 * BLK128;
-constexpr uint32_t SUM_OFF_BAR = SUM_OFF_PW + 136 * 4;
+constexpr uint32_t SUM_OFF_BAR = SUM_OFF_B + 4 * BLK128;
 constexpr uint32_t SUM_SMEM = SUM_OFF_BAR + 64 + 1024;
 
 template <int NB>
@@ -494,12 +592,31 @@ __global__ void __launch_bounds__(kGThreads, 2)
     uint64_t *in_full = bars, *b_ready = bars + 1, *acc_full = bars + 2, *mma_done = bars + 3;
     uint32_t *tmem_base = reinterpret_cast<uint32_t *>(bars + 4);
     volatile int *abort = reinterpret_cast<volatile int *>(tmem_base + 1);
-    float *pw = reinterpret_cast<float *>(sm + SUM_OFF_PW);
     const int tid = threadIdx.x, warp = tid >> 5;
     const GSeq sq = gseq(p, blockIdx.y);
     const int bh = sq.bh, c_first = blockIdx.x * CPB;
     const int h = sq.h;
     if (c_first >= sq.nC) return;  // past this sequence's chunks (variable-length calls)
+    // element-wise warps: row x of B is, for each N block b, w * V row of the
+    // block's chunk (D = 64) or columns 64 b .. of the chunk's row (D = 128),
+    // w = lam^(L-1-x); the V rows are loaded before the setup below
+    const int x = 32 * (warp & 3) + (tid & 31);
+    uint4 vrow[2][8];
+    float wrow[2] = {0.f, 0.f};
+    if (warp >= 2) {
+#pragma unroll
+        for (int b = 0; b < 2; ++b) {
+            const int c = NB == 1 ? c_first + b : c_first;
+            int e0, e1;
+            chunk_range(p, sq, c, e0, e1);
+            const int L = c < sq.nC ? e1 - e0 : 0;
+            wrow[b] = x < L ? gpow(p.lam[h], L - 1 - x) : 0.f;
+            const int col0 = NB == 1 ? 0 : 64 * b;
+            const uint4 *src = reinterpret_cast<const uint4 *>(p.v + grow(sq, x < L ? e0 + x : 0, p.Tc, p.H, D) + col0);
+#pragma unroll
+            for (int u = 0; u < 8; ++u) vrow[b][u] = wrow[b] != 0.f ? src[u] : make_uint4(0u, 0u, 0u, 0u);
+        }
+    }
 
     if (tid == 0) {
         mbar_init(in_full, 1);
@@ -554,25 +671,13 @@ __global__ void __launch_bounds__(kGThreads, 2)
         mma_commit_w(mma_done);
         mbar_wait_drain(mma_done, 0);
     } else {
-        const int q4 = warp & 3;
-        const int x = 32 * q4 + (tid & 31);
-        const uint32_t lanes = tb + ((uint32_t)(32 * q4) << 16);
-        gpowers(pw, CG, p.lam[h], x);
-        gbar128();
-        // B row x: for each N block b, w * V row of the block's chunk (D = 64) or
-        // columns 64 b .. of the chunk's row (D = 128)
+        const uint32_t lanes = tb + ((uint32_t)(32 * (warp & 3)) << 16);
 #pragma unroll
         for (int b = 0; b < 2; ++b) {
-            const int c = NB == 1 ? c_first + b : c_first;
-            int e0, e1;
-            chunk_range(p, sq, c, e0, e1);
-            const int L = c < sq.nC ? e1 - e0 : 0;
-            const float w = x < L ? pw[L - 1 - x] : 0.f;
-            const int col0 = NB == 1 ? 0 : 64 * b;
-            const uint4 *src = reinterpret_cast<const uint4 *>(p.v + grow(sq, x < L ? e0 + x : 0, p.Tc, p.H, D) + col0);
+            const float w = wrow[b];
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
-                const uint4 a = w != 0.f ? src[u] : make_uint4(0u, 0u, 0u, 0u);
+                const uint4 a = vrow[b][u];
                 const uint32_t ws[4] = {a.x, a.y, a.z, a.w};
                 uint32_t hi[4], lo[4];
 #pragma unroll
@@ -628,49 +733,73 @@ __global__ void __launch_bounds__(kGThreads, 2)
 // Chunk start states, one thread per state element: A_c (in place over the
 // increments) and A_final.
 constexpr int kMaxScanChunks = 4096;  // chunk decays kept in shared memory (longer rows compute theirs)
-__global__ void __launch_bounds__(256) gen_scan_kernel(GenParams p, int D) {
-    __shared__ float decay[kMaxScanChunks];  // lam^(length of chunk c)
+constexpr int kScanThreads = 256;
+constexpr int kScanVec = 4;            // consecutive state elements per thread
+
+// bf16 hi + lo of four floats, as two 8-byte words
+__device__ __forceinline__ void split4(const float4 a, uint2 &hi, uint2 &lo) {
+    uint32_t h0, h1, l0, l1;
+    gsplit(a.x, a.y, h0, l0);
+    gsplit(a.z, a.w, h1, l1);
+    hi = make_uint2(h0, h1);
+    lo = make_uint2(l0, l1);
+}
+
+// Chunk start states A_c (c = 0 .. nC-1) of one row from A_init and the
+// increments, A_{c+1} = lam^(L_c) A_c + dA_c, written as bf16 hi + lo for the
+// window kernel's copies, and A_final.  Each thread carries kScanVec
+// consecutive elements of the D x D state through every chunk.
+__global__ void __launch_bounds__(kScanThreads) gen_scan_kernel(GenParams p, int D) {
+    extern __shared__ float decay[];  // lam^(length of chunk c), c < min(p.nC, kMaxScanChunks)
+    // the window kernel may start now: it reads these states only after
+    // waiting for this grid to complete
+    griddep_launch_dependents();
     const GSeq sq = gseq(p, blockIdx.y);
     const int bh = sq.bh, nC = sq.nC;
-    const double l2l = log2((double)p.lam[sq.h]);
+    const float lam = p.lam[sq.h];
     for (int c = threadIdx.x; c < nC && c < kMaxScanChunks; c += blockDim.x) {
         int e0, e1;
         chunk_range(p, sq, c, e0, e1);
-        decay[c] = (float)exp2((double)(e1 - e0) * l2l);
+        decay[c] = gpow(lam, e1 - e0);
     }
     __syncthreads();
-    const int x = blockIdx.x * blockDim.x + threadIdx.x;
     const int nel = D * D;
+    const int x = kScanVec * (blockIdx.x * blockDim.x + threadIdx.x);
     if (x >= nel) return;
-    float A = p.A_init ? p.A_init[(size_t)bh * nel + x] : 0.f;
-    float *dA = p.dA + (size_t)bh * p.nC * nel + x;  // p.nC: chunk slots per row
+    float4 A = p.A_init ? *reinterpret_cast<const float4 *>(p.A_init + (size_t)bh * nel + x)
+                        : make_float4(0.f, 0.f, 0.f, 0.f);
+    const float *dA = p.dA + (size_t)bh * p.nC * nel + x;  // p.nC: chunk slots per row
     constexpr int kB = 8;
     for (int c0 = 0; c0 < nC; c0 += kB) {
-        float d[kB];
+        float4 d[kB];
 #pragma unroll
-        for (int u = 0; u < kB; ++u) d[u] = (c0 + u < nC && sq.E > 0) ? dA[(size_t)(c0 + u) * nel] : 0.f;
+        for (int u = 0; u < kB; ++u)
+            d[u] = (c0 + u < nC && sq.E > 0) ? *reinterpret_cast<const float4 *>(dA + (size_t)(c0 + u) * nel)
+                                              : make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
         for (int u = 0; u < kB; ++u) {
             const int c = c0 + u;
             if (c < nC) {
                 // the start state as bf16 hi + lo, row-major, for the window kernel's copy
-                const __nv_bfloat16 hi = __float2bfloat16_rn(A);
+                uint2 hi, lo;
+                split4(A, hi, lo);
                 __nv_bfloat16 *o = p.ab + (((size_t)bh * p.nC + c) * 2) * nel + x;
-                o[0] = hi;
-                o[nel] = __float2bfloat16_rn(A - __bfloat162float(hi));
+                *reinterpret_cast<uint2 *>(o) = hi;
+                *reinterpret_cast<uint2 *>(o + nel) = lo;
                 float dc;
                 if (c < kMaxScanChunks) {
                     dc = decay[c];
                 } else {
                     int e0, e1;
                     chunk_range(p, sq, c, e0, e1);
-                    dc = (float)exp2((double)(e1 - e0) * l2l);
+                    dc = gpow(lam, e1 - e0);
                 }
-                A = fmaf(dc, A, d[u]);
+                A = make_float4(fmaf(dc, A.x, d[u].x), fmaf(dc, A.y, d[u].y), fmaf(dc, A.z, d[u].z),
+                                fmaf(dc, A.w, d[u].w));
             }
         }
     }
-    if (p.A_final) p.A_final[(size_t)bh * nel + x] = A;
+    if (p.A_final) *reinterpret_cast<float4 *>(p.A_final + (size_t)bh * nel + x) = A;
 }
 
 // ===========================================================================
@@ -831,16 +960,32 @@ cudaError_t launch_general_t(const PrefillParams &pp, const float *mrow_in, cuda
                 mk128, p);
             if ((e = cudaGetLastError()) != cudaSuccess) return e;
         }
-        gen_scan_kernel<<<dim3((unsigned)((D * D + 255) / 256), (unsigned)BH), 256, 0, s>>>(p, D);
+        const int per_cta = kScanThreads * kScanVec;
+        const size_t decay_bytes = (size_t)(p.nC < kMaxScanChunks ? p.nC : kMaxScanChunks) * sizeof(float);
+        gen_scan_kernel<<<dim3((unsigned)((D * D + per_cta - 1) / per_cta), (unsigned)BH), kScanThreads,
+                          decay_bytes, s>>>(p, D);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     if (queries) {
         using WC = WinCfg<NB>;
         e = cudaFuncSetAttribute(gen_window_kernel<NB>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)WC::SMEM);
         if (e != cudaSuccess) return e;
-        gen_window_kernel<NB><<<dim3((unsigned)((p.T + CG - 1) / CG), (unsigned)BH), kGThreads, WC::SMEM, s>>>(
-            mq128, mk64, mv64, mab, p);
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        // After the scan, the window kernel may start early (programmatic stream
+        // serialization): it reads the scan's states only after griddep_wait,
+        // and everything else it reads was complete before the sums kernel
+        // (launched in plain stream order) started.
+        cudaLaunchAttribute early[1];
+        early[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        early[0].val.programmaticStreamSerializationAllowed = 1;
+        cudaLaunchConfig_t wc = {};
+        wc.gridDim = dim3((unsigned)((p.T + CG - 1) / CG), (unsigned)BH);
+        wc.blockDim = dim3(kGThreads);
+        wc.dynamicSmemBytes = WC::SMEM;
+        wc.stream = s;
+        wc.attrs = early;
+        wc.numAttrs = l2 ? 1 : 0;
+        e = cudaLaunchKernelEx(&wc, gen_window_kernel<NB>, mq128, mk64, mv64, mab, p);
+        if (e != cudaSuccess) return e;
     }
     return cudaSuccess;
 }

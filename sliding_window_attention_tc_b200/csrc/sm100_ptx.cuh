@@ -400,6 +400,31 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     return r;
 }
 
+// Three-input maximum (one instruction on sm_100a).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
+// Two-wide float32 arithmetic (fma / add on register pairs).
+__device__ __forceinline__ uint64_t f2pack(float a, float b) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+    return r;
+}
+__device__ __forceinline__ void ffma2(float &d0, float &d1, float a0, float a1, uint64_t b, uint64_t c) {
+    asm("{\n\t.reg .b64 a, d;\n\tmov.b64 a, {%2, %3};\n\tfma.rn.f32x2 d, a, %4, %5;\n\t"
+        "mov.b64 {%0, %1}, d;\n\t}"
+        : "=f"(d0), "=f"(d1)
+        : "f"(a0), "f"(a1), "l"(b), "l"(c));
+}
+__device__ __forceinline__ void fadd2_acc(uint64_t &acc, float a0, float a1) {
+    asm("{\n\t.reg .b64 a;\n\tmov.b64 a, {%1, %2};\n\tadd.rn.f32x2 %0, %0, a;\n\t}"
+        : "+l"(acc)
+        : "f"(a0), "f"(a1));
+}
+
 // Byte offset of element (row, col) in a SWIZZLE_128B tile of 64-element
 // bf16 rows (col in [0, 64)).
 __host__ __device__ __forceinline__ uint32_t sw128_offset(uint32_t row, uint32_t col) {

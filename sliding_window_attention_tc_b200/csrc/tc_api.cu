@@ -98,7 +98,32 @@ int *status_ptr() {
 // Halo length of a call that continues at global position t0.
 int64_t halo_len(const tc_prefill_desc &d, int64_t t0) { return t0 < d.W ? t0 : d.W; }
 
-bool use_sm100(const tc_prefill_desc &d, int64_t n_halo) { return tc::sm100_supported(d, n_halo); }
+// tc_set_prefill_path: which tensor-core prefill takes a call both can run
+// (and a per-thread override, for tc_prefill_no_alloc).
+int g_prefill_path = TC_PATH_AUTO;
+thread_local int t_path_override = -1;
+
+// The automatic choice between the two tensor-core paths for a call both
+// take (bf16, d = 64, W a multiple of 128), from B200 measurements: the
+// general path for fixed-length calls (faster at the LM and long-context
+// shapes with and without the memory, for continuations and for the delta
+// rule's window part: by 15 % on the LM prefill, 25 % L1-only), the fused
+// kernel for variable-length calls (3 % faster on a 15-sequence batch of
+// 55..8192 tokens, whose spans it balances across the SMs).
+bool general_preferred(bool varlen) {
+    switch (t_path_override >= 0 ? t_path_override : g_prefill_path) {
+        case TC_PATH_FUSED: return false;
+        case TC_PATH_GENERAL: return true;
+        default: return !varlen;
+    }
+}
+
+// The fused kernel takes the call: it supports the shape, and the general
+// path does not or is not the one chosen.
+bool use_sm100(const tc_prefill_desc &d, int64_t n_halo, bool varlen = false) {
+    if (!tc::sm100_supported(d, n_halo)) return false;
+    return !(general_preferred(varlen) && tc::general_supported(d, n_halo));
+}
 
 // A delta-rule call with queries and no halo whose window part the
 // tensor-core kernel takes (its L1-only form): window part there, memory in
@@ -132,7 +157,7 @@ size_t prefill_ws(const tc_prefill_desc &d, int64_t n_halo, int num_sms) {
 bool varlen_supported(const tc_prefill_desc &d) {
     tc_prefill_desc c = d;
     if (c.T < 1) c.T = 1;
-    return use_sm100(c, 0) && !(d.flags & ~TC_PREFILL_L1_ONLY);
+    return use_sm100(c, 0, true) && !(d.flags & ~TC_PREFILL_L1_ONLY);
 }
 
 // Workspace of a variable-length call on the general path (at least 256
@@ -167,11 +192,32 @@ tc_status check_decode_state(const tc_decode_state *s) {
 
 }  // namespace
 
+namespace tc {
+ScopedPrefillPath::ScopedPrefillPath(int path) : prev(t_path_override) { t_path_override = path; }
+ScopedPrefillPath::~ScopedPrefillPath() { t_path_override = prev; }
+}  // namespace tc
+
 extern "C" {
 
 const char *tc_version(void) { return "0.1.0"; }
 
 void tc_set_wait_limit_ns(uint64_t ns) { g_wait_limit_ns = ns; }
+
+tc_status tc_set_prefill_path(int path) {
+    if (path != TC_PATH_AUTO && path != TC_PATH_FUSED && path != TC_PATH_GENERAL) return TC_ERR_INVALID_ARG;
+    g_prefill_path = path;
+    return TC_OK;
+}
+
+int tc_get_prefill_path(void) { return g_prefill_path; }
+
+int tc_prefill_path_for(const tc_prefill_desc *d, int64_t t0) {
+    if (check_desc(d) != TC_OK || t0 < 0) return -1;
+    const int64_t n_halo = halo_len(*d, t0);
+    if (use_sm100(*d, n_halo) || delta_window_on_sm100(*d, n_halo)) return TC_PATH_FUSED;
+    if (use_general(*d, n_halo)) return TC_PATH_GENERAL;
+    return -1;
+}
 
 const char *tc_status_string(tc_status s) {
     switch (s) {

@@ -213,4 +213,12 @@ size_t sm100_workspace_bytes(const tc_prefill_desc &d, int num_sms, bool varlen 
 cudaError_t launch_prefill_sm100(const PrefillParams &p, int num_sms, cudaStream_t s);
 int sm100_launch_count(const tc_prefill_desc &d);
 
+// tc_api.cu: a per-thread override of tc_set_prefill_path (TC_PATH_*, or -1
+// for none) for the calls this thread makes while the object lives.
+struct ScopedPrefillPath {
+    int prev;
+    explicit ScopedPrefillPath(int path);
+    ~ScopedPrefillPath();
+};
+
 }  // namespace tc

@@ -29,6 +29,7 @@
 #include <mutex>
 
 #include "tc.h"
+#include "tc_internal.cuh"
 
 namespace {
 
@@ -59,9 +60,21 @@ extern "C" tc_status tc_prefill_no_alloc(const tc_prefill_desc *desc, const void
                                          const void *k, const void *v, const float *lambda,
                                          const float *eta, const float *g, void *y,
                                          float *A_final, tc_stream_t stream) {
-    const size_t need = tc_prefill_workspace_size(desc);
+    size_t need = tc_prefill_workspace_size(desc);
     if (need == (size_t)-1) return TC_ERR_INVALID_ARG;
+    // Under TC_PATH_AUTO a call whose general-path scratch (per-chunk states)
+    // does not fit runs on the fused kernel when that one's does.
+    int path = -1;
+    if (need > (size_t)TC_NO_ALLOC_SCRATCH_BYTES && tc_get_prefill_path() == TC_PATH_AUTO) {
+        tc::ScopedPrefillPath fused(TC_PATH_FUSED);
+        const size_t f = tc_prefill_workspace_size(desc);
+        if (f <= (size_t)TC_NO_ALLOC_SCRATCH_BYTES) {
+            need = f;
+            path = TC_PATH_FUSED;
+        }
+    }
     if (need > (size_t)TC_NO_ALLOC_SCRATCH_BYTES) return TC_ERR_WORKSPACE;
+    tc::ScopedPrefillPath chosen(path);
     int count = 0, dev = 0;
     if (cudaGetDeviceCount(&count) != cudaSuccess || count == 0 || cudaGetDevice(&dev) != cudaSuccess) {
         cudaGetLastError();

@@ -20,3 +20,13 @@ def cuda_device():
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
     return torch.device("cuda:0")
+
+
+@pytest.fixture(params=["fused", "general"])
+def both_paths(request):
+    """Runs the test once on each tensor-core prefill path (tc_set_prefill_path),
+    for the calls both take (bf16, d = 64, W a multiple of 128); other calls
+    run where they always do."""
+    import sliding_window_attention_tc_b200 as tc
+    with tc.prefill_path(request.param):
+        yield request.param

@@ -202,11 +202,49 @@ def test_no_alloc_rejects_invalid_and_oversized():
     assert _no_alloc(big) == WORKSPACE
 
 
-def test_tensor_core_workspace_fits_the_no_alloc_scratch():
-    # span summaries are bounded by about 4 matrices per SM whatever the length
+def test_fused_workspace_fits_the_no_alloc_scratch():
+    # the fused kernel's span summaries are bounded by about 4 matrices per SM
+    # whatever the length; the general path keeps two states per chunk of 128 rows
     for B, H, T, W in [(8, 12, 4096, 512), (1, 16, 32768, 1024), (64, 64, 65536, 128)]:
         d = _desc(B=B, H=H, T=T, W=W, C=64, dtype=tc.TC_BF16)
-        assert 0 <= tc.prefill_workspace_size(d) <= 4 * 148 * 64 * 64 * 4
+        with tc.prefill_path("fused"):
+            assert 0 <= tc.prefill_workspace_size(d) <= 4 * 148 * 64 * 64 * 4
+        with tc.prefill_path("general"):
+            chunks = B * H * ((T + 127) // 128)
+            assert tc.prefill_workspace_size(d) >= 2 * chunks * 64 * 64 * 4
+
+
+def test_prefill_path_setting():
+    """tc_set_prefill_path / tc_get_prefill_path / tc_prefill_path_for: the
+    choice between the two tensor-core paths for the calls both take, and
+    which path a call takes (no device needed)."""
+    assert tc.get_prefill_path() == "auto"
+    lm = _desc(B=8, H=12, T=4096, W=512, C=64, dtype=tc.TC_BF16)
+    odd = _desc(B=8, H=12, T=4096, W=500, C=64, dtype=tc.TC_BF16)  # W not a multiple of 128
+    d128 = _desc(B=2, H=2, T=1000, dk=128, dv=128, W=256, C=64, dtype=tc.TC_BF16)
+    f32 = _desc(dtype=tc.TC_F32)
+    assert tc.prefill_path_for(lm) == "general"  # auto: fixed-length calls on the general path
+    assert tc.prefill_path_for(odd) == "general" and tc.prefill_path_for(d128) == "general"
+    assert tc.prefill_path_for(f32) is None      # float32: the SIMT path
+    with tc.prefill_path("fused"):
+        assert tc.get_prefill_path() == "fused"
+        assert tc.prefill_path_for(lm) == "fused"
+        assert tc.prefill_path_for(lm, 1024) == "fused"  # continuation at t0 >= W
+        assert tc.prefill_path_for(lm, 100) == "general"  # partial halo: only the general path
+        assert tc.prefill_path_for(odd) == "general"     # only the general path takes it
+        l1 = _desc(B=8, H=12, T=4096, W=512, C=64, dtype=tc.TC_BF16, l1_only=True)
+        assert tc.prefill_path_for(l1) == "fused"
+        # the delta rule's window part runs on the fused kernel, its memory in chunks
+        assert tc.prefill_path_for(_desc(B=8, H=12, T=4096, W=512, C=64, dtype=tc.TC_BF16,
+                                         flags=tc.TC_PREFILL_DELTA_RULE)) == "fused"
+    assert tc.get_prefill_path() == "auto"
+    with tc.prefill_path(tc.TC_PATH_GENERAL):
+        assert tc.prefill_path_for(lm) == "general"
+    assert tc.prefill_path_for(_desc(B=0)) is None
+    for bad in (3, -1, 100):
+        with pytest.raises(tc.TCError):
+            tc.set_prefill_path(bad)
+    assert tc.get_prefill_path() == "auto"  # a refused value keeps the setting
 
 
 @no_device_only

@@ -31,20 +31,22 @@ def _run(tc, x, dev):
 
 def test_wait_limit_runs_out_and_the_context_stays_usable(cuda_device):
     import sliding_window_attention_tc_b200 as tc
-    # bf16, d = 64, W = 128: the tensor-core path, several spans (pre-pass too)
+    # bf16, d = 64, W = 128 on the fused kernel: several spans (pre-pass too)
     B, H, T = 2, 4, 2048
     x = wl.random_prefill(B, H, T, 64, 64, 128, 64, dtype="bf16", seed=31)
     desc = tc.make_prefill_desc(B, H, T, 64, 64, 128, 64, tc.TC_BF16)
-    assert tc.prefill_launch_count(desc) == 3  # summaries, prefix, main kernel
-    assert tc.device_status() == 0
-    try:
-        tc.set_wait_limit_ns(1)
-        _run(tc, x, cuda_device)
-        assert tc.device_status() == TC_ERR_DEVICE_TIMEOUT
-    finally:
-        tc.set_wait_limit_ns(0)
-    assert tc.device_status() == 0  # read and cleared
-    y, A = _run(tc, x, cuda_device)
+    with tc.prefill_path("fused"):
+        assert tc.prefill_path_for(desc) == "fused"
+        assert tc.prefill_launch_count(desc) == 3  # summaries, prefix, main kernel
+        assert tc.device_status() == 0
+        try:
+            tc.set_wait_limit_ns(1)
+            _run(tc, x, cuda_device)
+            assert tc.device_status() == TC_ERR_DEVICE_TIMEOUT
+        finally:
+            tc.set_wait_limit_ns(0)
+        assert tc.device_status() == 0  # read and cleared
+        y, A = _run(tc, x, cuda_device)
     assert tc.device_status() == 0
     yo, Ao = oracle.prefill(x.q, x.k, x.v, x.lam, x.eta, x.g, x.W)
     y = y.float().cpu().numpy()

@@ -90,7 +90,7 @@ CASES = [
 
 
 @pytest.mark.parametrize("case", CASES, ids=[f"{c[7]}_W{c[5]}_t0{c[8]}" for c in CASES])
-def test_prefill_from_state_matches_whole_sequence(cuda_device, case):
+def test_prefill_from_state_matches_whole_sequence(cuda_device, case, both_paths):
     B, H, T, dk, dv, W, C, dtype, t0 = case
     x = wl.random_prefill(B, H, T, dk, dv, W, C, dtype=dtype, seed=600 + t0)
     y_ref, A_ref = oracle.prefill(x.q, x.k, x.v, x.lam, x.eta, x.g, W)
@@ -99,7 +99,7 @@ def test_prefill_from_state_matches_whole_sequence(cuda_device, case):
 
 
 @pytest.mark.parametrize("case", [CASES[1], CASES[3], CASES[7]], ids=["bf16", "bf16_W256", "f32"])
-def test_state_only_gives_the_final_state(cuda_device, case):
+def test_state_only_gives_the_final_state(cuda_device, case, both_paths):
     B, H, T, dk, dv, W, C, dtype, t0 = case
     x = wl.random_prefill(B, H, T, dk, dv, W, C, dtype=dtype, seed=700 + t0)
     _, A_ref = oracle.prefill(x.q, x.k, x.v, x.lam, x.eta, x.g, W)

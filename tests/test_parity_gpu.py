@@ -121,8 +121,17 @@ def test_prefill_recall_fp32(cuda_device):
     print("recall_fp32", out)
 
 
-def test_prefill_lm_bf16_full_size_sampled_heads(cuda_device):
+def _takes(x, path):
+    """The call of workload x runs on the tensor-core path named path."""
+    tc = _tc()
+    B, H, T, d = x.q.shape
+    desc = tc.make_prefill_desc(B, H, T, d, x.v.shape[-1], x.W, x.C, tc.TC_BF16)
+    assert tc.prefill_path_for(desc) == path
+
+
+def test_prefill_lm_bf16_full_size_sampled_heads(cuda_device, both_paths):
     x = wl.prefill_config("lm_prefill_bf16")
+    _takes(x, both_paths)
     y, A = run_prefill(x, cuda_device)
     yl1, _ = run_prefill(x, cuda_device, l1_only=True)
     heads = [(0, 0), (1, 5), (3, 11), (5, 2), (7, 7), (7, 11)]
@@ -131,8 +140,9 @@ def test_prefill_lm_bf16_full_size_sampled_heads(cuda_device):
     print("lm_prefill_bf16", out)
 
 
-def test_prefill_long_bf16_full_size_sampled_heads(cuda_device):
+def test_prefill_long_bf16_full_size_sampled_heads(cuda_device, both_paths):
     x = wl.prefill_config("long_prefill_bf16")
+    _takes(x, both_paths)
     y, A = run_prefill(x, cuda_device)
     yl1, _ = run_prefill(x, cuda_device, l1_only=True)
     out = check_prefill(x, y, A, [(0, 0), (0, 13)], l1_only_y=yl1)
@@ -140,10 +150,11 @@ def test_prefill_long_bf16_full_size_sampled_heads(cuda_device):
     print("long_prefill_bf16", out)
 
 
-def test_prefill_lm_bf16_every_head(cuda_device):
+def test_prefill_lm_bf16_every_head(cuda_device, both_paths):
     """All 96 (b, h) rows of the LM workload (8 x 12 x 4096, W = 512), y and
-    A_final, against one oracle call over every row."""
+    A_final, against one oracle call over every row, on each path."""
     x = wl.prefill_config("lm_prefill_bf16")
+    _takes(x, both_paths)
     y, A = run_prefill(x, cuda_device)
     yo, Ao = oracle.prefill(x.q, x.k, x.v, x.lam, x.eta, x.g, x.W)
     B, H = x.q.shape[:2]
@@ -156,10 +167,12 @@ def test_prefill_lm_bf16_every_head(cuda_device):
     print("lm_prefill_bf16, every head", worst)
 
 
-def test_prefill_long_bf16_every_head(cuda_device):
+def test_prefill_long_bf16_every_head(cuda_device, both_paths):
     """All 16 heads of the long-context workload (1 x 16 x 32768, W = 1024),
-    y and A_final, against one oracle call that runs the heads in parallel."""
+    y and A_final, against one oracle call that runs the heads in parallel,
+    on each path."""
     x = wl.prefill_config("long_prefill_bf16")
+    _takes(x, both_paths)
     y, A = run_prefill(x, cuda_device)
     yo, Ao = oracle.prefill(x.q, x.k, x.v, x.lam, x.eta, x.g, x.W)
     H = x.q.shape[1]
@@ -193,7 +206,7 @@ EDGE = [
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 @pytest.mark.parametrize("shape", EDGE, ids=[str(s) for s in EDGE])
-def test_prefill_edge_shapes(cuda_device, shape, dtype):
+def test_prefill_edge_shapes(cuda_device, shape, dtype, both_paths):
     B, H, T, dk, dv, W, C = shape
     x = wl.random_prefill(B, H, T, dk, dv, W, C, dtype=dtype, seed=hash(shape) % 1000)
     y, A = run_prefill(x, cuda_device)
@@ -204,7 +217,7 @@ def test_prefill_edge_shapes(cuda_device, shape, dtype):
     check_prefill(x, y, A, l1_only_y=yl1)
 
 
-def test_prefill_is_deterministic_and_keeps_inputs(cuda_device):
+def test_prefill_is_deterministic_and_keeps_inputs(cuda_device, both_paths):
     tc = _tc()
     x = wl.random_prefill(2, 3, 700, 64, 64, 128, 64, dtype="bf16", seed=3)
     q, k, v = (_dev(t, cuda_device) for t in (x.q, x.k, x.v))
@@ -217,7 +230,7 @@ def test_prefill_is_deterministic_and_keeps_inputs(cuda_device):
     assert torch.equal(q, q0) and torch.equal(k, k0) and torch.equal(v, v0)
 
 
-def test_prefill_host_variant_matches_device(cuda_device):
+def test_prefill_host_variant_matches_device(cuda_device, both_paths):
     tc = _tc()
     x = wl.random_prefill(2, 2, 500, 64, 64, 128, 64, dtype="bf16", seed=4)
     yd, Ad = tc.prefill(*(_dev(t, cuda_device) for t in (x.q, x.k, x.v, x.lam, x.eta, x.g)),

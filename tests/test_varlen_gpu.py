@@ -84,11 +84,13 @@ def test_varlen_matches_the_oracle_per_sequence(cuda_device, case):
         print(b, _check_sequence(x, b, y, A, yl1))
 
 
-def test_varlen_of_equal_lengths_equals_the_batched_call(cuda_device):
-    """Equal lengths give the batched call's schedule (same rows, same spans),
-    so the packed call must reproduce tc_prefill bit for bit."""
+def test_varlen_of_equal_lengths_equals_the_batched_call(cuda_device, both_paths):
+    """Equal lengths give the batched call's schedule (same rows, same spans
+    or chunks), so on either tensor-core path the packed call must reproduce
+    tc_prefill on that path bit for bit."""
     import sliding_window_attention_tc_b200 as tc
     B, H, T, W = 3, 4, 1500, 256
+    assert tc.prefill_path_for(tc.make_prefill_desc(B, H, T, 64, 64, W, 64, tc.TC_BF16)) == both_paths
     x = wl.random_varlen([T] * B, H, 64, 64, W, 64, dtype="bf16", seed=7)
     y, A = _run(tc, x, cuda_device)
     dev = cuda_device

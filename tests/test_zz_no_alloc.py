@@ -74,3 +74,30 @@ def test_no_alloc_rejects_more_scratch_than_it_has(cuda_device):
     assert tc.prefill_workspace_size(desc) > tc.NO_ALLOC_SCRATCH_BYTES
     st = tc.lib_handle().tc_prefill_no_alloc(ctypes.byref(desc), *([None] * 8), None)
     assert st == 7  # TC_ERR_WORKSPACE, nothing enqueued
+
+
+def test_no_alloc_runs_the_fused_kernel_when_only_its_scratch_fits(cuda_device):
+    """The LM workload (8 x 12 x 4096, d = 64, W = 512): the general path
+    would need 100 MiB of per-chunk states, the fused kernel fits the
+    built-in array.  Under the automatic choice the call runs on the fused
+    kernel and equals tc_prefill on that kernel bit for bit; with the general
+    path chosen explicitly it is refused."""
+    tc = _tc()
+    x = wl.prefill_config("lm_prefill_bf16")
+    B, H, T, d = x.q.shape
+    desc = tc.make_prefill_desc(B, H, T, d, d, x.W, x.C, tc.TC_BF16)
+    assert tc.get_prefill_path() == "auto"
+    assert tc.prefill_workspace_size(desc) > tc.NO_ALLOC_SCRATCH_BYTES
+    with tc.prefill_path("fused"):
+        assert tc.prefill_workspace_size(desc) <= tc.NO_ALLOC_SCRATCH_BYTES
+    y_na, A_na, args = _no_alloc(tc, x, cuda_device)
+    with tc.prefill_path("fused"):
+        y_ref, A_ref = tc.prefill(*args, x.W, x.C)
+    torch.cuda.synchronize()
+    assert tc.device_status() == 0
+    assert torch.equal(y_na, y_ref) and torch.equal(A_na, A_ref)
+    with tc.prefill_path("general"):
+        p = lambda t: ctypes.c_void_p(t.data_ptr())
+        st = tc.lib_handle().tc_prefill_no_alloc(ctypes.byref(desc), *[p(a) for a in args], p(y_na), p(A_na),
+                                                  ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+        assert st == 7  # TC_ERR_WORKSPACE, nothing enqueued
