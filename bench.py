@@ -47,10 +47,11 @@ HEADLINE = "lm_prefill_bf16"
 # kernels; they must be re-measured (or set to None) whenever a kernel changes.
 #   prefill_main_kernel: one LM launch, 159.2 MB read + 31.9 MB written
 #     (profiles/prefill_main_kernel_lm_prefill_bf16.md)
-#   gen_window_kernel: None until captured at the LM shape
+#   gen_window_kernel: one LM launch (W = 512), 195.1 MB read + 35.3 MB written
+#     (profiles/gen_window_kernel_lm_prefill_bf16.md)
 #   decode_kernel: the B = 32 capture scaled by heads to the 256 x 32 launch,
 #     (1.1417 + 0.0172) GB x 8 (profiles/decode_kernel_b32_w2048_d128.md)
-NCU_TRAFFIC_BYTES = {"prefill_main_kernel": 1.911e8, "gen_window_kernel": None, "decode_kernel": 9.27e9}
+NCU_TRAFFIC_BYTES = {"prefill_main_kernel": 1.911e8, "gen_window_kernel": 2.304e8, "decode_kernel": 9.27e9}
 # the kernel that dominates one prefill call on each tensor-core path
 PATH_KERNEL = {"fused": "prefill_main_kernel", "general": "gen_window_kernel"}
 METRIC = "prefill tokens/s & decode tok/s per B200; % of TC/HBM roofline"
