@@ -70,3 +70,45 @@ def test_cpu_baseline_reports_threads_used():
     assert 1 <= out["cores"] <= cores
     assert out["kind"] == "oracle" and out["value"] > 0
     assert "heads x 4096 tokens" in out["sample"]
+
+
+def _general_brute(T, W, d):
+    """Tensor-core FLOPs of the general path by enumerating keys: block b of
+    128 query rows scores every 64-key tile that holds a key it reads (the
+    window keys of its rows, and its chunk of evictions when it has one),
+    P V on the same tiles, P'V on the tiles holding its chunk, Q A_b (hi +
+    lo); one 128 x 128 x 128 sums product pair per CTA of chunks."""
+    E = max(0, T - W)
+    nC = -(-T // 128)
+    tiles = reads = qa = 0
+    for b in range(nC):
+        rows = range(128 * b, min(T, 128 * b + 128))
+        keys = {j for t in rows for j in range(max(0, t - W + 1), t + 1)}
+        chunk = set(range(max(0, 128 * b - W), max(0, min(E, 128 * b + 128 - W))))
+        keys |= chunk
+        # the kernel's tiles run from the first key read to the block's last row
+        lo, hi = min(keys), min(T - 1, 128 * b + 127)
+        tiles += hi // 64 - lo // 64 + 1
+        if chunk:
+            reads += len({j // 64 for j in chunk})
+            qa += 1
+    mma = 2 * 128 * 64 * d
+    sums = (((nC + 1) // 2) if d == 64 else nC) * 2 * (2 * 128 ** 3) if E > 0 else 0
+    return tiles * 2 * mma, reads * mma + qa * 2 * (2 * 128 * d * d) + sums
+
+
+def test_general_path_executed_flops_match_enumeration():
+    for T, W, d in [(128, 128, 64), (700, 200, 64), (1000, 256, 128), (333, 5, 64), (100, 300, 64),
+                    (4096, 500, 64), (2000, 512, 128)]:
+        assert bench.general_executed_flops(1, 1, T, W, d) == _general_brute(T, W, d), (T, W, d)
+
+
+def test_general_path_lm_counts():
+    # per head: 300 key tiles (blocks 0-3: 2, 4, 6, 8; blocks 4-31: 10 each),
+    # 56 tiles of P'V and 28 Q A_b products (blocks 4-31), 16 sums CTAs
+    e1, e2 = bench.general_executed_flops(8, 12, 4096, 512)
+    mma = 2 * 128 * 64 * 64
+    assert e1 == 96 * 300 * 2 * mma
+    assert e2 == 96 * (56 * mma + 28 * 2 * mma + 16 * 2 * (2 * 128 ** 3))
+    l1, l2 = bench.prefill_flops(8, 12, 4096, 64, 64, 512)
+    assert abs((e1 + e2) / (l1 + l2) - 1.567) < 1e-3
