@@ -583,7 +583,7 @@ constexpr uint32_t SUM_SMEM = SUM_OFF_BAR + 64 + 1024;
 
 template <int NB>
 __global__ void __launch_bounds__(kGThreads, 2)
-    gen_sums_kernel(const __grid_constant__ CUtensorMap tk, GenParams p) {
+    gen_sums_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv, GenParams p) {
     constexpr int D = 64 * NB;
     constexpr int CPB = NB == 1 ? 2 : 1;  // chunks per CTA
     extern __shared__ uint8_t smem_raw[];
@@ -597,27 +597,6 @@ __global__ void __launch_bounds__(kGThreads, 2)
     const int bh = sq.bh, c_first = blockIdx.x * CPB;
     const int h = sq.h;
     if (c_first >= sq.nC) return;  // past this sequence's chunks (variable-length calls)
-    // element-wise warps: row x of B is, for each N block b, w * V row of the
-    // block's chunk (D = 64) or columns 64 b .. of the chunk's row (D = 128),
-    // w = lam^(L-1-x); the V rows are loaded before the setup below
-    const int x = 32 * (warp & 3) + (tid & 31);
-    uint4 vrow[2][8];
-    float wrow[2] = {0.f, 0.f};
-    if (warp >= 2) {
-#pragma unroll
-        for (int b = 0; b < 2; ++b) {
-            const int c = NB == 1 ? c_first + b : c_first;
-            int e0, e1;
-            chunk_range(p, sq, c, e0, e1);
-            const int L = c < sq.nC ? e1 - e0 : 0;
-            wrow[b] = x < L ? gpow(p.lam[h], L - 1 - x) : 0.f;
-            const int col0 = NB == 1 ? 0 : 64 * b;
-            const uint4 *src = reinterpret_cast<const uint4 *>(p.v + grow(sq, x < L ? e0 + x : 0, p.Tc, p.H, D) + col0);
-#pragma unroll
-            for (int u = 0; u < 8; ++u) vrow[b][u] = wrow[b] != 0.f ? src[u] : make_uint4(0u, 0u, 0u, 0u);
-        }
-    }
-
     if (tid == 0) {
         mbar_init(in_full, 1);
         mbar_init(b_ready, 128);
@@ -637,20 +616,27 @@ __global__ void __launch_bounds__(kGThreads, 2)
 
     if (warp == 0) {
         if (tid == 0) {
-            mbar_expect_tx(in_full, 2 * BLK128);
-            // K of chunks c_first, c_first + 1 (D = 64) or the two column halves of
-            // chunk c_first (D = 128), from each chunk's first eviction; rows past
-            // the data read zero, rows past a chunk meet zero weights
+            mbar_expect_tx(in_full, 4 * BLK128);
+            // K and V of chunks c_first, c_first + 1 (D = 64) or the two column
+            // halves of chunk c_first (D = 128), from each chunk's first eviction;
+            // rows past the data read zero, rows past a chunk meet zero weights.
+            // V lands where B's hi blocks go: each element-wise thread turns its
+            // own row into the weighted hi part in place.
             int lo0, hi0, lo1, hi1;
             chunk_range(p, sq, c_first, lo0, hi0);
             chunk_range(p, sq, c_first + 1, lo1, hi1);
-            tma_rows_nb<1>(sm + SUM_OFF_A, &tk, in_full, lo0, sq, BLK128);
-            if (NB == 1)
-                tma_rows_nb<1>(sm + SUM_OFF_A + BLK128, &tk, in_full, lo1, sq, BLK128);
-            else if (sq.packed)
-                tma_load_3d(sm + SUM_OFF_A + BLK128, &tk, in_full, 64, sq.h, sq.row0 + lo0);
-            else
-                tma_load_3d(sm + SUM_OFF_A + BLK128, &tk, in_full, 64, lo0, bh);
+#pragma unroll
+            for (int t = 0; t < 2; ++t) {
+                const CUtensorMap *m = t == 0 ? &tk : &tv;
+                uint8_t *dst = sm + (t == 0 ? SUM_OFF_A : SUM_OFF_B);
+                tma_rows_nb<1>(dst, m, in_full, lo0, sq, BLK128);
+                if (NB == 1)
+                    tma_rows_nb<1>(dst + BLK128, m, in_full, lo1, sq, BLK128);
+                else if (sq.packed)
+                    tma_load_3d(dst + BLK128, m, in_full, 64, sq.h, sq.row0 + lo0);
+                else
+                    tma_load_3d(dst + BLK128, m, in_full, 64, lo0, bh);
+            }
             mbar_wait_drain(in_full, 0);
         }
     } else if (warp == 1) {
@@ -671,55 +657,82 @@ __global__ void __launch_bounds__(kGThreads, 2)
         mma_commit_w(mma_done);
         mbar_wait_drain(mma_done, 0);
     } else {
+        // row x of B is, for each N block b, w * V row of the block's chunk
+        // (D = 64) or columns 64 b .. of the chunk's row (D = 128), w = lam^(L-1-x)
+        const int x = 32 * (warp & 3) + (tid & 31);
         const uint32_t lanes = tb + ((uint32_t)(32 * (warp & 3)) << 16);
+        float wrow[2];
 #pragma unroll
         for (int b = 0; b < 2; ++b) {
-            const float w = wrow[b];
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                const uint4 a = vrow[b][u];
-                const uint32_t ws[4] = {a.x, a.y, a.z, a.w};
-                uint32_t hi[4], lo[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e)
-                    gsplit(w * __uint_as_float(ws[e] << 16), w * __uint_as_float(ws[e] & 0xffff0000u), hi[e], lo[e]);
-                *reinterpret_cast<uint4 *>(sm + SUM_OFF_B + b * BLK128 + sw128_offset(x, 8 * u)) =
-                    make_uint4(hi[0], hi[1], hi[2], hi[3]);
-                *reinterpret_cast<uint4 *>(sm + SUM_OFF_B + (2 + b) * BLK128 + sw128_offset(x, 8 * u)) =
-                    make_uint4(lo[0], lo[1], lo[2], lo[3]);
-            }
+            const int c = NB == 1 ? c_first + b : c_first;
+            int e0, e1;
+            chunk_range(p, sq, c, e0, e1);
+            const int L = c < sq.nC ? e1 - e0 : 0;
+            wrow[b] = x < L ? gpow(p.lam[h], L - 1 - x) : 0.f;
         }
-        fence_async_smem();
-        mbar_arrive(b_ready);
-        if (gwait(acc_full, 0, abort, p)) {
+        if (gwait(in_full, 0, abort, p)) {
+#pragma unroll
+            for (int b = 0; b < 2; ++b) {
+                const float w = wrow[b];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    uint8_t *hp = sm + SUM_OFF_B + b * BLK128 + sw128_offset(x, 8 * u);
+                    const uint4 a = w != 0.f ? *reinterpret_cast<const uint4 *>(hp) : make_uint4(0u, 0u, 0u, 0u);
+                    const uint32_t ws[4] = {a.x, a.y, a.z, a.w};
+                    uint32_t hi[4], lo[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        gsplit(w * __uint_as_float(ws[e] << 16), w * __uint_as_float(ws[e] & 0xffff0000u), hi[e],
+                               lo[e]);
+                    *reinterpret_cast<uint4 *>(hp) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+                    *reinterpret_cast<uint4 *>(sm + SUM_OFF_B + (2 + b) * BLK128 + sw128_offset(x, 8 * u)) =
+                        make_uint4(lo[0], lo[1], lo[2], lo[3]);
+                }
+            }
+            fence_async_smem();
+            mbar_arrive(b_ready);
+        }
+        // The result goes out through shared memory (the B region, free once the
+        // product is done) so that whole warps write contiguous rows: row x of
+        // the staged tile is lane x's TMEM row, eta-scaled, 16-byte chunk u at
+        // chunk u ^ (x & 15) of its row.
+        constexpr int RW = NB == 1 ? 64 : 128;  // floats per staged row
+        constexpr int NCH = RW / 4;             // 16-byte chunks per row
+        float *stage = reinterpret_cast<float *>(sm + SUM_OFF_B);
+        const bool have = gwait(acc_full, 0, abort, p);
+        if (have) {
             tc_fence_after();
             const float eta = p.eta[h];
             // D = 64: lanes 0..63 rows of chunk c_first (columns 0..63), 64..127 of
             // c_first + 1 (columns 64..127); D = 128: every lane a row, all columns
-            const int c = NB == 1 ? c_first + (x >> 6) : c_first;
-            const int r = NB == 1 ? (x & 63) : x;
             const uint32_t col0 = NB == 1 ? (uint32_t)(x & 64) : 0u;
-            if (c < sq.nC) {
-                float *dst = p.dA + (((size_t)bh * p.nC + c) * D + r) * D;
 #pragma unroll
-                for (int c0 = 0; c0 < (NB == 1 ? 64 : 128); c0 += 32) {
-                    uint32_t v[32];
-                    tmem_ld32(lanes + col0 + c0, v);
-                    tmem_wait_ld();
-                    float4 *d4 = reinterpret_cast<float4 *>(dst + c0);
-#pragma unroll
-                    for (int u = 0; u < 8; ++u)
-                        d4[u] = make_float4(eta * __uint_as_float(v[4 * u]), eta * __uint_as_float(v[4 * u + 1]),
-                                            eta * __uint_as_float(v[4 * u + 2]), eta * __uint_as_float(v[4 * u + 3]));
-                }
-            } else {
-                // the chunk past the end (odd chunk count, D = 64): its lanes still
-                // take part in the collective loads
+            for (int c0 = 0; c0 < RW; c0 += 32) {
                 uint32_t v[32];
-                tmem_ld32(lanes + col0, v);
+                tmem_ld32(lanes + col0 + c0, v);
                 tmem_wait_ld();
-                tmem_ld32(lanes + col0 + 32, v);
-                tmem_wait_ld();
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    const int u = c0 / 4 + q;
+                    *reinterpret_cast<float4 *>(stage + x * RW + 4 * (u ^ (x & 15))) =
+                        make_float4(eta * __uint_as_float(v[4 * q]), eta * __uint_as_float(v[4 * q + 1]),
+                                    eta * __uint_as_float(v[4 * q + 2]), eta * __uint_as_float(v[4 * q + 3]));
+                }
+            }
+        }
+        gbar128();  // every element-wise thread, whether or not its wait succeeded
+        if (!*abort) {
+            // rows 0..127 of the tile are consecutive rows of dA: chunk c_first's
+            // 64 (or 128) rows, then (D = 64) chunk c_first + 1's
+            float *dst = p.dA + ((size_t)bh * p.nC + c_first) * D * D;
+            const int et = tid - 64;  // 0 .. 127
+#pragma unroll 4
+            for (int i = et; i < 128 * NCH; i += 128) {
+                const int row = i / NCH, u = i % NCH;
+                const int c = NB == 1 ? c_first + (row >> 6) : c_first;
+                if (c < sq.nC)
+                    *reinterpret_cast<float4 *>(dst + (size_t)row * RW + 4 * u) =
+                        *reinterpret_cast<const float4 *>(stage + row * RW + 4 * (u ^ (row & 15)));
             }
         }
     }
@@ -940,12 +953,13 @@ cudaError_t launch_general_t(const PrefillParams &pp, const float *mrow_in, cuda
     p.ab = l2 ? reinterpret_cast<__nv_bfloat16 *>(ws + Lo.ab) : nullptr;
     p.mrow = pp.delta_rule ? const_cast<float *>(mrow_in) : nullptr;
     const bool queries = !pp.state_only && p.T > 0;
-    CUtensorMap mk128, mq128, mk64, mv64;
+    CUtensorMap mk128, mv128, mq128, mk64, mv64;
     auto map = [&](CUtensorMap *m, const void *base, int rows, int box) {
         return packed ? gen_map_packed(m, base, p.total, p.H, D, box) : gen_map(m, base, rows, BH, D, box);
     };
     if ((queries || (l2 && p.E > 0)) &&
-        (!map(&mk128, p.k, p.Tc, 128) || !map(&mk64, p.k, p.Tc, 64) || !map(&mv64, p.v, p.Tc, 64)))
+        (!map(&mk128, p.k, p.Tc, 128) || !map(&mv128, p.v, p.Tc, 128) || !map(&mk64, p.k, p.Tc, 64) ||
+         !map(&mv64, p.v, p.Tc, 64)))
         return cudaErrorInvalidValue;
     if (queries && !map(&mq128, p.q, p.T, 128)) return cudaErrorInvalidValue;
     CUtensorMap mab = mq128;  // any valid map when the memory is off (not read then)
@@ -957,7 +971,7 @@ cudaError_t launch_general_t(const PrefillParams &pp, const float *mrow_in, cuda
             if (e != cudaSuccess) return e;
             const int cpb = NB == 1 ? 2 : 1;
             gen_sums_kernel<NB><<<dim3((unsigned)((p.nC + cpb - 1) / cpb), (unsigned)BH), kGThreads, SUM_SMEM, s>>>(
-                mk128, p);
+                mk128, mv128, p);
             if ((e = cudaGetLastError()) != cudaSuccess) return e;
         }
         const int per_cta = kScanThreads * kScanVec;
