@@ -1,6 +1,8 @@
-// Tensor-core prefill for the shapes the fused prefill_main_kernel does not
-// take: bf16 with d_k = d_v = D in {64, 128}, any window W >= 1, any T, and
-// continuations with any halo (0 < t0 < W included).
+// The general tensor-core prefill: bf16 with d_k = d_v = D in {64, 128}, any
+// window W >= 1, any T, and continuations with any halo (0 < t0 < W
+// included).  It takes every fixed-length call by default (it measured faster
+// than the fused prefill_main_kernel at that kernel's shapes too); the fused
+// kernel keeps the variable-length calls at its shapes.
 //
 // "Tensor Cache: Eviction-conditioned Associative Memory for Transformers":
 // the window read of §3.1 eq. (1) and the memory of §3.2 / Fig. 2 (write on
@@ -743,8 +745,8 @@ __global__ void __launch_bounds__(kGThreads, 2)
 }
 
 // ===========================================================================
-// Chunk start states, one thread per state element: A_c (in place over the
-// increments) and A_final.
+// Chunk start states A_c (as bf16 hi + lo, for the window kernel's copies)
+// and A_final, from the increments of the sums kernel.
 constexpr int kMaxScanChunks = 4096;  // chunk decays kept in shared memory (longer rows compute theirs)
 constexpr int kScanThreads = 256;
 constexpr int kScanVec = 4;            // consecutive state elements per thread
