@@ -128,6 +128,13 @@ TC_API size_t tc_prefill_workspace_size(const tc_prefill_desc *desc);
  * contents on entry are ignored and on exit are undefined.
  * Inputs must not overlap outputs.
  *
+ * Paths: bf16 with d_k = d_v in {64, 128} runs on the tensor cores, by
+ * default on the general path (per-chunk sums, a chunk scan, and a window
+ * kernel that also computes the memory's reads); d = 64 with W a multiple of
+ * 128 can run on the fused kernel instead (tc_set_prefill_path).  Other
+ * calls run on the portable float32 kernels.  Both tensor-core paths keep A
+ * in float32 and meet the same tolerances; they are not bit-identical.
+ *
  * Errors: TC_ERR_INVALID_ARG, TC_ERR_UNSUPPORTED, TC_ERR_WORKSPACE,
  * TC_ERR_NO_DEVICE, TC_ERR_CUDA.  On error nothing is enqueued except for
  * TC_ERR_CUDA, after which the outputs are undefined. */
@@ -152,8 +159,10 @@ TC_API tc_status tc_prefill(const tc_prefill_desc *desc, const void *q, const vo
  *
  * q, k, v, y are the new tokens' rows [B,H,T,d].  A_final is A after the
  * last eviction of the call.  With TC_PREFILL_STATE_ONLY only A_final is
- * computed.  The tensor-core path takes bf16, d_k = d_v = 64, W a multiple of
- * 128 and t0 = 0 or t0 >= W; other calls run on the portable float32 path.
+ * computed.  bf16 with d_k = d_v in {64, 128} runs on the general
+ * tensor-core path (any W, any t0; the fused kernel when selected, for d =
+ * 64, W a multiple of 128 and t0 = 0 or t0 >= W); other calls run on the
+ * portable float32 path.
  * Workspace: tc_prefill_from_state_workspace_size(desc, t0) bytes.  Errors
  * as tc_prefill, plus TC_ERR_INVALID_ARG for t0 < 0 or a missing halo. */
 TC_API size_t tc_prefill_from_state_workspace_size(const tc_prefill_desc *desc, int64_t t0);
@@ -184,7 +193,8 @@ TC_API tc_status tc_prefill_from_state(const tc_prefill_desc *desc, int64_t t0,
  *
  * Supported: the tensor-core paths only (bf16, d_k = d_v in {64, 128}, any
  * W, flags 0 or TC_PREFILL_L1_ONLY; d = 64 with W a multiple of 128 runs the
- * fused kernel, the rest the general tensor-core path); other descriptions
+ * fused kernel unless tc_set_prefill_path selects the general path, the rest
+ * the general tensor-core path); other descriptions
  * return TC_ERR_UNSUPPORTED (and (size_t)-1 from the size query).  The offsets are
  * device data, so the host cannot check them: the kernels do.  A sequence
  * whose offsets are negative, decreasing, past total or longer than desc->T
