@@ -250,3 +250,21 @@ def test_prefill_path_setting():
 @no_device_only
 def test_no_alloc_valid_without_device():
     assert _no_alloc(_desc()) == NO_DEVICE
+
+
+def test_prefill_path_binding_edge_cases():
+    """The binding refuses unknown names, and the context manager restores
+    the previous setting even when its body raises."""
+    assert tc.get_prefill_path() == "auto"
+    with pytest.raises(tc.TCError):
+        tc.set_prefill_path("fastest")
+    with pytest.raises(RuntimeError):
+        with tc.prefill_path("general"):
+            assert tc.get_prefill_path() == "general"
+            raise RuntimeError("inside")
+    assert tc.get_prefill_path() == "auto"
+    with tc.prefill_path("fused"):
+        with tc.prefill_path("general"):
+            assert tc.get_prefill_path() == "general"
+        assert tc.get_prefill_path() == "fused"
+    assert tc.get_prefill_path() == "auto"
