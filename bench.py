@@ -702,6 +702,9 @@ def main():
                     help="batch of the decode workload (default 256)")
     ap.add_argument("--decode-steps", type=int, default=None,
                     help="decode steps (default 512)")
+    ap.add_argument("--path", choices=["auto", "fused", "general"], default="auto",
+                    help="tensor-core prefill for the calls both paths take (tc_set_prefill_path; "
+                         "profiling runs of one path)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -718,6 +721,7 @@ def main():
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     import sliding_window_attention_tc_b200 as tc
+    tc.set_prefill_path(args.path)
 
     peaks, peak_src = load_peaks()
     if args.only:
